@@ -1,0 +1,272 @@
+"""ORACLE — test infrastructure only.
+
+numpy front end of ``oracle.c``: the plain fp64 CPU statement of the routed
+mixture-of-experts layer that the CUDA path is checked against.  Only the
+tests, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline leg may
+import this package; the product path never does.  It shares no code with
+the CUDA path; the two meet only in the seeded input generators of
+``synth``.
+
+bf16 tensors travel as their uint16 bit patterns; everything the oracle
+computes is float64 unless the function says otherwise.
+"""
+from __future__ import annotations
+
+import ctypes
+import subprocess
+from pathlib import Path
+
+import numpy as np
+
+HERE = Path(__file__).resolve().parent
+_SRC = HERE / "oracle.c"
+_LIB = HERE / "liboracle.so"
+
+FX_SHIFT = 40
+
+_i64 = ctypes.c_int64
+_p = ctypes.c_void_p
+_f = ctypes.c_float
+
+
+def build(force: bool = False) -> Path:
+    if force or (not _LIB.exists()) or _LIB.stat().st_mtime < _SRC.stat().st_mtime:
+        subprocess.check_call([
+            "gcc", "-O3", "-fopenmp", "-ffp-contract=off", "-fno-fast-math", "-std=c11",
+            "-fPIC", "-shared", str(_SRC), "-o", str(_LIB), "-lm"])
+    return _LIB
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        L = ctypes.CDLL(str(build()))
+        sig = {
+            "oracle_router_logits_fx": (None, [_i64, _i64, _i64, _p, _p, _p, _p]),
+            "oracle_topk": (None, [_i64, _i64, _i64, _p, _p, _p]),
+            "oracle_permute": (None, [_i64, _i64, _i64, _p, _p, _p, _p, _p]),
+            "oracle_expert_bf16": (None, [_i64, _i64, _p, _p, _p, _p]),
+            "oracle_expert_rows_bf16": (ctypes.c_int, [_i64, _i64, _i64, _p, _p, _p, _p, _p, _p]),
+            "oracle_combine": (None, [_i64, _i64, _i64, _p, _p, _p, _p]),
+            "oracle_e4m3_encode": (ctypes.c_uint8, [_f]),
+            "oracle_e4m3_decode": (_f, [ctypes.c_uint8]),
+            "oracle_e4m3_encode_n": (None, [_i64, _p, _p]),
+            "oracle_e4m3_decode_n": (None, [_i64, _p, _p]),
+            "oracle_quantize_tensor_fp8": (_f, [_i64, _p, _p]),
+            "oracle_quantize_act_fp8": (None, [_i64, _p, _f, _p]),
+            "oracle_expert_fp8": (None, [_i64, _i64, _p, _f, _p, _f, _p, _f, _f, _p]),
+            "oracle_expert_rows_fp8": (ctypes.c_int, [_i64, _i64, _i64, _p, _p, _p, _p, _p, _p,
+                                                      _p, _f, _f, _p]),
+            "oracle_rmsnorm_bf16": (None, [_i64, _i64, _p, _f, _p]),
+            "oracle_round_bf16": (None, [_i64, _p, _p]),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _c(a, dtype):
+    a = np.ascontiguousarray(a, dtype=dtype)
+    return a, a.ctypes.data
+
+
+def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
+    return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+# --------------------------------------------------------------------------- routing
+
+def router_logits_fx(x, wr, bias=None) -> np.ndarray:
+    """Fixed-point router logits, int64 in units of 2^-40, shape [T, E]."""
+    x, px = _c(x, np.uint16)
+    wr, pw = _c(wr, np.uint16)
+    T, H = x.shape
+    E = wr.shape[0]
+    pb = None
+    if bias is not None:
+        bias, pb = _c(bias, np.float32)
+    L = np.empty((T, E), dtype=np.int64)
+    lib().oracle_router_logits_fx(T, H, E, px, pw, pb, L.ctypes.data)
+    return L
+
+
+def topk(L: np.ndarray, K: int):
+    L, pl = _c(L, np.int64)
+    T, E = L.shape
+    idx = np.empty((T, K), dtype=np.int32)
+    w = np.empty((T, K), dtype=np.float64)
+    lib().oracle_topk(T, E, K, pl, idx.ctypes.data, w.ctypes.data)
+    return idx, w
+
+
+def route(x, wr, bias, K):
+    L = router_logits_fx(x, wr, bias)
+    idx, w = topk(L, K)
+    return L, idx, w
+
+
+def permute(idx: np.ndarray, E: int):
+    idx, pi = _c(idx, np.int32)
+    T, K = idx.shape
+    counts = np.empty(E, dtype=np.int32)
+    offsets = np.empty(E + 1, dtype=np.int32)
+    perm_src = np.empty(T * K, dtype=np.int32)
+    inv_row = np.empty(T * K, dtype=np.int32)
+    lib().oracle_permute(T, K, E, pi, counts.ctypes.data, offsets.ctypes.data,
+                         perm_src.ctypes.data, inv_row.ctypes.data)
+    return counts, offsets, perm_src, inv_row
+
+
+# --------------------------------------------------------------------------- experts
+
+def expert_rows_bf16(xrows, ex, wup, wdown, slot) -> np.ndarray:
+    """y[r] = expert_{ex[r]}(xrows[r]) for float64 rows; banks given for a set of experts."""
+    xrows, px = _c(xrows, np.float64)
+    ex, pe = _c(ex, np.int32)
+    wup, pu = _c(wup, np.uint16)
+    wdown, pd = _c(wdown, np.uint16)
+    slot, ps = _c(slot, np.int32)
+    R, H = xrows.shape
+    F = wup.shape[1]
+    y = np.empty((R, H), dtype=np.float64)
+    if lib().oracle_expert_rows_bf16(R, H, F, px, pe, pu, pd, ps, y.ctypes.data) != 0:
+        raise ValueError("a routed expert's bank was not supplied")
+    return y
+
+
+def combine(y_tk, w, residual=None) -> np.ndarray:
+    y_tk, py = _c(y_tk, np.float64)
+    w, pw = _c(w, np.float64)
+    T, K, H = y_tk.shape
+    pr = None
+    if residual is not None:
+        residual, pr = _c(residual, np.uint16)
+    out = np.empty((T, H), dtype=np.float64)
+    lib().oracle_combine(T, K, H, py, pw, pr, out.ctypes.data)
+    return out
+
+
+def identity_slot(E: int) -> np.ndarray:
+    return np.arange(E, dtype=np.int32)
+
+
+def moe_layer_bf16(x, wr, bias, wup, wdown, K, tokens=None, slot=None, residual=None):
+    """The whole layer for the rows ``tokens`` of x (all rows if None).
+
+    Tokens do not interact (no capacity limit), so any subset is exact.
+    Returns a dict with logits, idx, w, the per-assignment expert outputs
+    y [n, K, H] and out [n, H] (float64, before bf16 rounding).
+    """
+    x = np.asarray(x, dtype=np.uint16)
+    if tokens is not None:
+        x = x[np.asarray(tokens)]
+        if residual is not None:
+            residual = np.asarray(residual)[np.asarray(tokens)]
+    E = wr.shape[0]
+    if slot is None:
+        slot = identity_slot(E)
+    L, idx, w = route(x, wr, bias, K)
+    n, H = x.shape
+    xr = np.repeat(bf16_to_f64(x), K, axis=0)
+    y = expert_rows_bf16(xr, idx.reshape(-1), wup, wdown, slot).reshape(n, K, H)
+    out = combine(y, w, residual)
+    return dict(logits=L, idx=idx, w=w, y=y, out=out)
+
+
+# --------------------------------------------------------------------------- FP8
+
+def e4m3_encode(v) -> np.ndarray:
+    v, pv = _c(v, np.float32)
+    q = np.empty(v.shape, dtype=np.uint8)
+    lib().oracle_e4m3_encode_n(v.size, pv, q.ctypes.data)
+    return q
+
+
+def e4m3_decode(q) -> np.ndarray:
+    q, pq = _c(q, np.uint8)
+    v = np.empty(q.shape, dtype=np.float32)
+    lib().oracle_e4m3_decode_n(q.size, pq, v.ctypes.data)
+    return v
+
+
+def quantize_tensor_fp8(w):
+    """Per-tensor E4M3 quantisation of a bf16 tensor: returns (codes, scale)."""
+    w, pw = _c(w, np.uint16)
+    q = np.empty(w.shape, dtype=np.uint8)
+    s = lib().oracle_quantize_tensor_fp8(w.size, pw, q.ctypes.data)
+    return q, np.float32(s)
+
+
+def quantize_bank_fp8(bank):
+    """Quantise each expert tensor of a bank [S, rows, cols] with its own scale."""
+    q = np.empty(bank.shape, dtype=np.uint8)
+    s = np.empty(bank.shape[0], dtype=np.float32)
+    for i in range(bank.shape[0]):
+        q[i], s[i] = quantize_tensor_fp8(bank[i])
+    return q, s
+
+
+def quantize_act_fp8(x, s: float) -> np.ndarray:
+    x, px = _c(x, np.uint16)
+    q = np.empty(x.shape, dtype=np.uint8)
+    lib().oracle_quantize_act_fp8(x.size, px, np.float32(s), q.ctypes.data)
+    return q
+
+
+def expert_rows_fp8(qx, ex, qup, sup, qdown, sdown, slot, sx, sh) -> np.ndarray:
+    qx, px = _c(qx, np.uint8)
+    ex, pe = _c(ex, np.int32)
+    qup, pu = _c(qup, np.uint8)
+    sup, psu = _c(sup, np.float32)
+    qdown, pd = _c(qdown, np.uint8)
+    sdown, psd = _c(sdown, np.float32)
+    slot, ps = _c(slot, np.int32)
+    R, H = qx.shape
+    F = qup.shape[1]
+    y = np.empty((R, H), dtype=np.float64)
+    rc = lib().oracle_expert_rows_fp8(R, H, F, px, pe, pu, psu, pd, psd, ps,
+                                      np.float32(sx), np.float32(sh), y.ctypes.data)
+    if rc != 0:
+        raise ValueError("a routed expert's bank was not supplied")
+    return y
+
+
+def moe_layer_fp8(x, wr, bias, qup, sup, qdown, sdown, sx, sh, K, tokens=None, slot=None,
+                  residual=None):
+    """W8A8 layer: bf16 router on x; experts on e4m3 codes with scalar scales."""
+    x = np.asarray(x, dtype=np.uint16)
+    if tokens is not None:
+        x = x[np.asarray(tokens)]
+        if residual is not None:
+            residual = np.asarray(residual)[np.asarray(tokens)]
+    E = wr.shape[0]
+    if slot is None:
+        slot = identity_slot(E)
+    L, idx, w = route(x, wr, bias, K)
+    n, H = x.shape
+    qx = quantize_act_fp8(x, sx)
+    qxr = np.repeat(qx, K, axis=0)
+    y = expert_rows_fp8(qxr, idx.reshape(-1), qup, sup, qdown, sdown, slot, sx, sh).reshape(n, K, H)
+    out = combine(y, w, residual)
+    return dict(logits=L, idx=idx, w=w, y=y, out=out, qx=qx)
+
+
+def rmsnorm_bf16(x, eps: float = 1e-5) -> np.ndarray:
+    x, px = _c(x, np.uint16)
+    T, H = x.shape
+    u = np.empty_like(x)
+    lib().oracle_rmsnorm_bf16(T, H, px, np.float32(eps), u.ctypes.data)
+    return u
+
+
+def round_bf16(v) -> np.ndarray:
+    v, pv = _c(v, np.float64)
+    out = np.empty(v.shape, dtype=np.uint16)
+    lib().oracle_round_bf16(v.size, pv, out.ctypes.data)
+    return out

@@ -1,0 +1,101 @@
+"""The five seeded workloads of the routed mixture-of-experts layer.
+
+Shapes follow the Nemotron 3.5 Transcribe decoder as the bloomery issue page
+states them ("2. Checkpoint facts": hidden width 2688, top-6 routing over 128
+experts, ungated ReLU^2 experts of width 1856, 23 MoE layers); the serving
+shapes follow the SGLang-Omni cookbook page (64 running requests, 4096-token
+chunked prefill).  Activations are ~N(0,1), router and expert weights
+~N(0,0.02), all rounded to bf16; the router bias of the skewed workload gives
+softmax(b) = Zipf(1.1) over a seeded expert ranking.
+
+Nothing here computes any part of the layer: these are inputs only.
+"""
+from __future__ import annotations
+
+import dataclasses
+
+import numpy as np
+
+from . import (T_BIAS, T_WDOWN, T_WR, T_WUP, T_X, key, normal_bf16, u64)
+
+SIGMA_X = 1.0
+SIGMA_W = 0.02
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    T: int
+    H: int
+    E: int
+    K: int
+    F: int
+    seed: int
+    zipf_bias: bool = False
+    layers: int = 1
+    fp8: bool = False
+
+    @property
+    def assignments(self) -> int:
+        return self.T * self.K
+
+
+WORKLOADS = {
+    0: Workload("tiny_T16_H256_E8_K2_F128", 16, 256, 8, 2, 128, seed=0),
+    1: Workload("decode_T64", 64, 2688, 128, 6, 1856, seed=1),
+    2: Workload("prefill_T4096", 4096, 2688, 128, 6, 1856, seed=2),
+    3: Workload("skewed_zipf_T576", 576, 2688, 128, 6, 1856, seed=3, zipf_bias=True),
+    4: Workload("chain23_fp8_T4096", 4096, 2688, 128, 6, 1856, seed=4, layers=23, fp8=True),
+}
+
+
+def zipf_bias(seed: int, E: int, s: float = 1.1) -> np.ndarray:
+    """Router bias b_e = ln(r_e^-s / sum_j j^-s), r_e = pi(e)+1 for a seeded permutation pi.
+
+    softmax(b) is then exactly the Zipf(s) law over the ranking; the bias is an
+    input of the layer, computed once on the host in float64 and stored fp32.
+    """
+    k = key(seed, T_BIAS, 0)
+    perm = list(range(E))
+    for i in range(E - 1, 0, -1):          # Fisher-Yates, draws from the counter stream
+        j = u64(k, i) % (i + 1)
+        perm[i], perm[j] = perm[j], perm[i]
+    ranks = np.array(perm, dtype=np.float64) + 1.0
+    z = np.sum(np.arange(1, E + 1, dtype=np.float64) ** (-s))
+    return (np.log(ranks ** (-s) / z)).astype(np.float32)
+
+
+def host_x(w: Workload, layer: int = 0, tensor: int = T_X) -> np.ndarray:
+    return normal_bf16(key(w.seed, tensor, layer), w.T * w.H, SIGMA_X).reshape(w.T, w.H)
+
+
+def host_router(w: Workload, layer: int = 0) -> np.ndarray:
+    return normal_bf16(key(w.seed, T_WR, layer), w.E * w.H, SIGMA_W).reshape(w.E, w.H)
+
+
+def host_w_up(w: Workload, layer: int = 0, experts=None) -> np.ndarray:
+    """W_up bits, [E, F, H] (or [len(experts), F, H] for a subset)."""
+    k = key(w.seed, T_WUP, layer)
+    n = w.F * w.H
+    if experts is None:
+        return normal_bf16(k, w.E * n, SIGMA_W).reshape(w.E, w.F, w.H)
+    out = np.empty((len(experts), w.F, w.H), dtype=np.uint16)
+    for i, e in enumerate(experts):
+        out[i] = normal_bf16(k, n, SIGMA_W, offset=int(e) * n).reshape(w.F, w.H)
+    return out
+
+
+def host_w_down(w: Workload, layer: int = 0, experts=None) -> np.ndarray:
+    """W_down bits, [E, H, F] (or a subset)."""
+    k = key(w.seed, T_WDOWN, layer)
+    n = w.H * w.F
+    if experts is None:
+        return normal_bf16(k, w.E * n, SIGMA_W).reshape(w.E, w.H, w.F)
+    out = np.empty((len(experts), w.H, w.F), dtype=np.uint16)
+    for i, e in enumerate(experts):
+        out[i] = normal_bf16(k, n, SIGMA_W, offset=int(e) * n).reshape(w.H, w.F)
+    return out
+
+
+def host_bias(w: Workload):
+    return zipf_bias(w.seed, w.E) if w.zipf_bias else None
