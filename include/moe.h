@@ -1,0 +1,172 @@
+/*
+ * routed_expert_moe_b200 — C ABI of a routed mixture-of-experts layer for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The layer is the routed MoE block of the Nemotron 3.5 Transcribe hybrid
+ * decoder as the bloomery issue page describes it (section 2 "Checkpoint
+ * facts": hidden width 2688, top-6 routing over 128 experts, ungated ReLU^2
+ * experts of width 1856; "FP8 uses scalar-scale E4M3 W8A8"; section 3:
+ * ungated up/down expert parts).  For one batch of T tokens x[T][H]:
+ *
+ *   l[t][e]  = sum_h x[t][h] * Wr[e][h] (+ b[e])                 router
+ *   S_t      = the K experts with the largest l[t][.], ties to the lower index
+ *   w[t][k]  = softmax over l[t][S_t] (= the full softmax renormalised on S_t)
+ *   y[t][k]  = W_down[S_tk] * relu(W_up[S_tk] * x[t])^2            expert
+ *   out[t]   = (residual[t] +) sum_k w[t][k] * y[t][k], k in order  combine
+ *
+ * Conventions for every call:
+ *  - Tensors are dense row-major device arrays owned by the caller; the
+ *    library allocates nothing.  Device pointers must be 16-byte aligned,
+ *    the workspace 256-byte aligned.
+ *  - bf16 is the IEEE-like bfloat16 bit pattern (uint16); fp8 is OCP E4M3
+ *    ("fn") stored as uint8.  Weight banks are [out][in]: W_up is [E][F][H],
+ *    W_down is [E][H][F], the router weight is [E][H].
+ *  - Every call is asynchronous on the given CUDA stream (a cudaStream_t
+ *    passed as void*; NULL is the legacy default stream).  Argument errors
+ *    are detected on the host and returned before anything is launched.
+ *    Errors found inside kernels (an out-of-range expert index, a bounded
+ *    wait that expired, a router magnitude outside the exact range) are
+ *    recorded in a per-device error word that moe_check_device_error reads.
+ *  - Results are deterministic: the same inputs give the same bits, on any
+ *    stream, at any batch size split (no floating-point atomics).
+ *  - Expert indices and the permutation are exact: the router ranks experts
+ *    on logits summed in fixed point (each bf16 product rounded to 2^-40,
+ *    summed exactly), computed fast in fp32 with a rigorous error bound and
+ *    recomputed exactly for the few experts whose rank the bound leaves open.
+ */
+#ifndef ROUTED_EXPERT_MOE_H
+#define ROUTED_EXPERT_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_ABI_VERSION 1
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_EINVAL = 1,        /* invalid argument: null pointer, bad size, misalignment */
+    MOE_EUNSUPPORTED = 2,  /* valid request this build does not support (e.g. not sm_100) */
+    MOE_ECUDA = 3,         /* a CUDA runtime call or a launch failed */
+    MOE_ETIMEOUT = 4,      /* a bounded wait inside a kernel expired (device error word) */
+    MOE_EWORKSPACE = 5,    /* workspace smaller than moe_workspace_size() */
+    MOE_ERANGE = 6,        /* router inputs beyond the exact fixed-point range (device) */
+    MOE_EINDEX = 7         /* an expert index outside [0, E) reached moe_permute (device) */
+} moe_status;
+
+typedef enum {
+    MOE_BF16 = 0,          /* expert banks and expert activations in bf16 */
+    MOE_FP8_E4M3 = 1       /* W8A8: expert banks and expert activations in E4M3 codes */
+} moe_dtype;
+
+/* Problem size.  Limits: 0 <= T, T*K < 2^31; 1 <= E <= 256; 1 <= K <= min(E, 16);
+ * 16 <= H <= 65536 and 16 <= F <= 65536, both multiples of 16. */
+typedef struct {
+    int64_t T;             /* tokens */
+    int32_t H;             /* hidden width (router and up-projection input, down output) */
+    int32_t E;             /* routed experts */
+    int32_t K;             /* experts per token */
+    int32_t F;             /* expert width (up output, down input) */
+    int32_t expert_dtype;  /* moe_dtype */
+} moe_dims;
+
+/* Scalar scales of the W8A8 experts (bloomery page, section 2: "scalar-scale
+ * E4M3 W8A8").  Real value = code * scale.  Ignored for MOE_BF16. */
+typedef struct {
+    const float* w_up_scale;    /* [E] device: one scale per expert up tensor */
+    const float* w_down_scale;  /* [E] device: one scale per expert down tensor */
+    float x_scale;              /* static scale of the expert input activations */
+    float h_scale;              /* static scale of the ReLU^2 activations */
+} moe_fp8_scales;
+
+/* Human-readable name of a status.  Never NULL. */
+const char* moe_status_string(moe_status s);
+
+/* MOE_ABI_VERSION of the loaded library. */
+int moe_abi_version(void);
+
+/* Bytes of workspace that moe_forward needs for these dims (moe_route,
+ * moe_permute and moe_expert_ffn need no more).  Host only; no device call. */
+moe_status moe_workspace_size(const moe_dims* d, size_t* bytes);
+
+/* Router: logits, top-K, renormalised softmax weights.
+ *   x         [T][H] bf16     w_router [E][H] bf16     bias [E] fp32 or NULL
+ *   topk_idx  [T][K] int32    out: experts by descending logit, ties to the lower index
+ *   topk_w    [T][K] fp32     out: weights, summing to 1 per token
+ * Cited: bloomery page s.2 (top-6 over 128 experts); audio.cpp model page,
+ * "CPU weight offload" (router and routing-weight formulas). */
+moe_status moe_route(const moe_dims* d, const void* x, const void* w_router, const float* bias,
+                     int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes, void* stream);
+
+/* Permutation into expert-contiguous rows: a stable counting sort of the
+ * assignments i = t*K + k by expert.
+ *   topk_idx [T][K] int32 in; counts [E], offsets [E+1] (exclusive scan),
+ *   perm_src [T*K] (row r of the grouped layout holds assignment perm_src[r]),
+ *   inv_row  [T*K] (assignment i sits in row inv_row[i]) out.
+ * An index outside [0, E) sets MOE_EINDEX in the device error word; the
+ * outputs are then unspecified.  Cited: audio.cpp model page, "CPU weight
+ * offload" (grouped expert matrix multiplication). */
+moe_status moe_permute(const moe_dims* d, const int32_t* topk_idx, int32_t* counts,
+                       int32_t* offsets, int32_t* perm_src, int32_t* inv_row, void* ws,
+                       size_t ws_bytes, void* stream);
+
+/* Grouped expert FFN over the permuted rows:
+ *   y_perm[r] = W_down[e] * relu(W_up[e] * x[perm_src[r] / K])^2,  e = expert of row r
+ *   x [T][H] bf16; offsets [E+1] and perm_src [T*K] as from moe_permute;
+ *   w_up [E][F][H], w_down [E][H][F] (bf16, or E4M3 codes with `scales`);
+ *   y_perm [T*K][H] bf16 out.
+ * scales must be non-NULL for MOE_FP8_E4M3.  Cited: bloomery page s.2 and
+ * s.3 (ungated ReLU^2 experts, up/down parts). */
+moe_status moe_expert_ffn(const moe_dims* d, const void* x, const int32_t* offsets,
+                          const int32_t* perm_src, const void* w_up, const void* w_down,
+                          const moe_fp8_scales* scales, void* y_perm, void* ws, size_t ws_bytes,
+                          void* stream);
+
+/* Weighted combine: out[t] = (residual[t] +) sum_{k=0..K-1} topk_w[t][k] * y_perm[inv_row[t*K+k]],
+ * summed in fp32 in the order k = 0..K-1 and rounded once to bf16.
+ *   y_perm [T*K][H] bf16, inv_row [T*K], topk_w [T][K] fp32, residual [T][H] bf16 or NULL,
+ *   out [T][H] bf16 (may alias residual). */
+moe_status moe_combine(const moe_dims* d, const void* y_perm, const int32_t* inv_row,
+                       const float* topk_w, const void* residual, void* out, void* stream);
+
+/* The whole layer in one call (route, permute, expert FFN, combine), all
+ * intermediates in the workspace.  topk_idx / topk_w ([T][K]) may be NULL;
+ * when given they receive the routing.  out may alias residual. */
+moe_status moe_forward(const moe_dims* d, const void* x, const void* w_router, const float* bias,
+                       const void* w_up, const void* w_down, const moe_fp8_scales* scales,
+                       const void* residual, void* out, int32_t* topk_idx, float* topk_w,
+                       void* ws, size_t ws_bytes, void* stream);
+
+/* Per-tensor E4M3 quantisation of n_tensors bf16 tensors of tensor_elems
+ * elements each (an expert bank): scale[i] = amax|W_i| / 448 (1 for an
+ * all-zero tensor), codes = e4m3_rne_satfinite(W / scale[i]).
+ *   src [n_tensors][tensor_elems] bf16, codes same shape uint8, scales [n_tensors] fp32.
+ * Cited: bloomery page s.2 ("scalar-scale E4M3 W8A8"). */
+moe_status moe_quantize_fp8(int64_t n_tensors, int64_t tensor_elems, const void* src,
+                            uint8_t* codes, float* scales, void* stream);
+
+/* RMS normalisation with unit gain of the residual stream between chained
+ * layers: u = bf16(x / sqrt(mean(x^2) + eps)), the mean of squares taken
+ * exactly (fixed point, 2^-16 per term) and the rest in correctly rounded fp32.
+ *   x, u [T][H] bf16 (u may not alias x).  Cited: audio.cpp model page,
+ * "Q4_K, Q3_K and Q2_K expert profiles" (the model's normalisation). */
+moe_status moe_rmsnorm(int64_t T, int32_t H, float eps, const void* x, void* u, void* stream);
+
+/* Synchronises `stream`, then reads and clears the device error word of the
+ * current device.  Returns MOE_OK, or the first error a kernel recorded. */
+moe_status moe_check_device_error(void* stream);
+
+/* Test hooks of the failure-detection tests.  what = 1: limit of every
+ * bounded wait in nanoseconds (value <= 0 restores the default of 4 s);
+ * what = 2: the grouped-GEMM producer of block 0 withholds its first load
+ * (value 1) so the consumer's wait must expire; 0 turns it off. */
+moe_status moe_debug_set(int32_t what, int64_t value);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ROUTED_EXPERT_MOE_H */

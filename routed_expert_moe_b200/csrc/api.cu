@@ -1,0 +1,424 @@
+// C ABI (include/moe.h): argument validation, workspace layout, per-device
+// setup and the launch sequence of each entry point.  All computation is in
+// the kernels of route.cu, permute.cu, grouped_gemm.cu and combine.cu.
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+// launchers (defined with their kernels)
+struct RouterPlan {
+    int S;
+    int nchunks;
+    size_t p_bytes, xn_bytes, wn_bytes;
+};
+RouterPlan router_plan(int64_t T, int H, int E, int num_sms);
+cudaError_t launch_route(const uint16_t* x, const uint16_t* wr, const float* bias, int64_t T, int H, int E,
+                         int K, int32_t* idx, float* w, double* P, double* xn2, double* wn2,
+                         const RouterPlan& plan, const DevCtx& ctx, cudaStream_t stream);
+cudaError_t launch_permute(const int32_t* idx, int64_t n, int E, int32_t* counts, int32_t* offsets,
+                           int32_t* perm_src, int32_t* inv_row, int4* sched, int* n_sched, int bn,
+                           const DevCtx& ctx, cudaStream_t stream);
+size_t permute_smem_bytes(int E);
+cudaError_t launch_schedule(const int32_t* offsets, int E, int bn, int4* sched, int* n_sched,
+                            cudaStream_t stream);
+cudaError_t launch_gather(const uint16_t* x, const int32_t* perm_src, int64_t rows, int K, int64_t T, int H,
+                          void* xp, bool fp8, float x_scale, int num_sms, const DevCtx& ctx,
+                          cudaStream_t stream);
+struct GemmPlan {
+    int bn;
+    int n_stages;
+    size_t smem_bytes;
+    int max_sched;
+};
+GemmPlan gemm_plan(int64_t T, int K, int E);
+cudaError_t launch_grouped_gemm(bool fp8, bool up, const void* W, int E, int Nout, int Kdim, const void* act,
+                                int64_t rows, const int4* sched, const int* n_sched, const GemmPlan& plan,
+                                void* out, const float* w_scale, float in_scale, float out_scale, int num_sms,
+                                int debug_withhold, const DevCtx& ctx, cudaStream_t stream);
+cudaError_t launch_combine(const uint16_t* yp, const int32_t* inv_row, const float* w, const uint16_t* residual,
+                           uint16_t* out, int64_t T, int K, int H, int num_sms, const DevCtx& ctx,
+                           cudaStream_t stream);
+cudaError_t launch_rmsnorm(const uint16_t* x, uint16_t* u, int64_t T, int H, float eps, int num_sms,
+                           cudaStream_t stream);
+cudaError_t launch_quantize(int64_t n_tensors, int64_t elems, const uint16_t* src, uint8_t* codes,
+                            float* scales, int num_sms, cudaStream_t stream);
+
+}  // namespace moe
+
+using namespace moe;
+
+// The per-device error word: the only device state of the library.
+__device__ int g_moe_error = 0;
+
+namespace {
+
+constexpr uint64_t kDefaultTimeoutNs = 4000000000ull;
+std::atomic<uint64_t> g_timeout_ns{kDefaultTimeoutNs};
+std::atomic<int> g_debug_withhold{0};
+
+struct DeviceInfo {
+    bool ready = false;
+    moe_status status = MOE_OK;
+    int num_sms = 0;
+    int* err = nullptr;
+};
+
+constexpr int kMaxDevices = 64;
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+moe_status device_setup(DeviceInfo** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ECUDA;
+    std::lock_guard<std::mutex> lock(g_dev_mu);
+    DeviceInfo& d = g_dev[dev];
+    if (!d.ready) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return MOE_ECUDA;
+        if (major != 10 || minor != 0) {
+            d.status = MOE_EUNSUPPORTED;
+        } else if (cudaGetSymbolAddress(reinterpret_cast<void**>(&d.err), g_moe_error) != cudaSuccess) {
+            return MOE_ECUDA;
+        }
+        d.ready = true;
+    }
+    if (d.status != MOE_OK) return d.status;
+    *out = &d;
+    return MOE_OK;
+}
+
+DevCtx make_ctx(const DeviceInfo* d) { return DevCtx{d->err, g_timeout_ns.load()}; }
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+moe_status check_dims(const moe_dims* d) {
+    if (!d) return MOE_EINVAL;
+    if (d->T < 0 || d->E < 1 || d->E > 256 || d->K < 1 || d->K > 16 || d->K > d->E) return MOE_EINVAL;
+    if (d->H < 16 || d->H > 65536 || d->H % 16 != 0) return MOE_EINVAL;
+    if (d->F < 16 || d->F > 65536 || d->F % 16 != 0) return MOE_EINVAL;
+    if (d->T * (int64_t)d->K >= (int64_t)1 << 31) return MOE_EINVAL;
+    if (d->expert_dtype != MOE_BF16 && d->expert_dtype != MOE_FP8_E4M3) return MOE_EINVAL;
+    return MOE_OK;
+}
+
+moe_status cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return MOE_OK;
+    if (e == cudaErrorInvalidValue) return MOE_EINVAL;
+    return MOE_ECUDA;
+}
+
+// Workspace layout: a bump allocator over the caller's buffer, 256-byte aligned.
+struct Carve {
+    size_t off = 0;
+    template <typename T>
+    T* take(void* base, size_t count) {
+        off = (off + 255) & ~size_t(255);
+        T* p = base ? reinterpret_cast<T*>(static_cast<uint8_t*>(base) + off) : nullptr;
+        off += count * sizeof(T);
+        return p;
+    }
+};
+
+struct RouteWs {
+    double* P;
+    double* xn2;
+    double* wn2;
+};
+struct FfnWs {
+    int4* sched;
+    int* n_sched;
+    void* xp;
+    void* hb;
+};
+struct ForwardWs {
+    int32_t* idx;
+    float* w;
+    int32_t* counts;
+    int32_t* offsets;
+    int32_t* perm_src;
+    int32_t* inv_row;
+    void* y_perm;
+};
+
+RouteWs carve_route(Carve& c, void* base, const moe_dims* d, const RouterPlan& rp) {
+    RouteWs r;
+    r.P = c.take<double>(base, rp.p_bytes / sizeof(double));
+    r.xn2 = c.take<double>(base, rp.xn_bytes / sizeof(double));
+    r.wn2 = c.take<double>(base, rp.wn_bytes / sizeof(double));
+    return r;
+}
+
+FfnWs carve_ffn(Carve& c, void* base, const moe_dims* d, const GemmPlan& gp) {
+    FfnWs f;
+    const size_t rows = (size_t)d->T * d->K;
+    const size_t es = d->expert_dtype == MOE_FP8_E4M3 ? 1 : 2;
+    f.sched = c.take<int4>(base, (size_t)gp.max_sched);
+    f.n_sched = c.take<int>(base, 1);
+    f.xp = c.take<uint8_t>(base, rows * d->H * es);
+    f.hb = c.take<uint8_t>(base, rows * d->F * es);
+    return f;
+}
+
+ForwardWs carve_forward(Carve& c, void* base, const moe_dims* d) {
+    ForwardWs f;
+    const size_t rows = (size_t)d->T * d->K;
+    f.idx = c.take<int32_t>(base, rows);
+    f.w = c.take<float>(base, rows);
+    f.counts = c.take<int32_t>(base, d->E);
+    f.offsets = c.take<int32_t>(base, d->E + 1);
+    f.perm_src = c.take<int32_t>(base, rows);
+    f.inv_row = c.take<int32_t>(base, rows);
+    f.y_perm = c.take<uint16_t>(base, rows * d->H);
+    return f;
+}
+
+size_t route_ws_bytes(const moe_dims* d, int sms) {
+    Carve c;
+    carve_route(c, nullptr, d, router_plan(d->T, d->H, d->E, sms));
+    return c.off;
+}
+
+size_t ffn_ws_bytes(const moe_dims* d) {
+    Carve c;
+    carve_ffn(c, nullptr, d, gemm_plan(d->T, d->K, d->E));
+    return c.off;
+}
+
+size_t forward_ws_bytes(const moe_dims* d, int sms) {
+    Carve c;
+    carve_forward(c, nullptr, d);
+    const size_t a = c.off;
+    // route and ffn scratch are carved after the forward buffers, reusing one region
+    const size_t r = route_ws_bytes(d, sms), f = ffn_ws_bytes(d);
+    return ((a + 255) & ~size_t(255)) + (r > f ? r : f) + 256;
+}
+
+// Run the expert FFN given a schedule already in `fw`.
+moe_status run_ffn(const moe_dims* d, const DeviceInfo* dev, const DevCtx& ctx, const GemmPlan& gp,
+                   const void* x, const int32_t* perm_src, const void* w_up, const void* w_down,
+                   const moe_fp8_scales* sc, FfnWs& fw, void* y_perm, cudaStream_t st) {
+    const bool fp8 = d->expert_dtype == MOE_FP8_E4M3;
+    const int64_t rows = d->T * d->K;
+    cudaError_t e = launch_gather(static_cast<const uint16_t*>(x), perm_src, rows, d->K, d->T, d->H, fw.xp, fp8,
+                                  fp8 ? sc->x_scale : 1.0f, dev->num_sms, ctx, st);
+    if (e != cudaSuccess) return cuda_status(e);
+    const int withhold = g_debug_withhold.load();
+    e = launch_grouped_gemm(fp8, true, w_up, d->E, d->F, d->H, fw.xp, rows, fw.sched, fw.n_sched, gp, fw.hb,
+                            fp8 ? sc->w_up_scale : nullptr, fp8 ? sc->x_scale : 1.0f,
+                            fp8 ? sc->h_scale : 1.0f, dev->num_sms, withhold, ctx, st);
+    if (e != cudaSuccess) return cuda_status(e);
+    e = launch_grouped_gemm(fp8, false, w_down, d->E, d->H, d->F, fw.hb, rows, fw.sched, fw.n_sched, gp, y_perm,
+                            fp8 ? sc->w_down_scale : nullptr, fp8 ? sc->h_scale : 1.0f, 1.0f, dev->num_sms, 0,
+                            ctx, st);
+    return cuda_status(e);
+}
+
+moe_status check_fp8_scales(const moe_dims* d, const moe_fp8_scales* sc) {
+    if (d->expert_dtype != MOE_FP8_E4M3) return MOE_OK;
+    if (!sc || !sc->w_up_scale || !sc->w_down_scale) return MOE_EINVAL;
+    if (!(sc->x_scale > 0.0f) || !(sc->h_scale > 0.0f)) return MOE_EINVAL;
+    return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_string(moe_status s) {
+    switch (s) {
+        case MOE_OK: return "MOE_OK";
+        case MOE_EINVAL: return "MOE_EINVAL: invalid argument";
+        case MOE_EUNSUPPORTED: return "MOE_EUNSUPPORTED: not supported on this device or build";
+        case MOE_ECUDA: return "MOE_ECUDA: CUDA runtime error";
+        case MOE_ETIMEOUT: return "MOE_ETIMEOUT: a bounded wait inside a kernel expired";
+        case MOE_EWORKSPACE: return "MOE_EWORKSPACE: workspace too small";
+        case MOE_ERANGE: return "MOE_ERANGE: router inputs beyond the exact fixed-point range";
+        case MOE_EINDEX: return "MOE_EINDEX: expert or row index out of range";
+    }
+    return "unknown moe_status";
+}
+
+int moe_abi_version(void) { return MOE_ABI_VERSION; }
+
+moe_status moe_workspace_size(const moe_dims* d, size_t* bytes) {
+    moe_status s = check_dims(d);
+    if (s != MOE_OK) return s;
+    if (!bytes) return MOE_EINVAL;
+    // plans depend on the SM count only through the router split; size for
+    // the largest split any device can choose
+    *bytes = forward_ws_bytes(d, 1024);
+    return MOE_OK;
+}
+
+moe_status moe_route(const moe_dims* d, const void* x, const void* w_router, const float* bias,
+                     int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes, void* stream) {
+    moe_status s = check_dims(d);
+    if (s != MOE_OK) return s;
+    if (d->T > 0 && (!x || !w_router || !topk_idx || !topk_w || !ws)) return MOE_EINVAL;
+    if (!aligned(x, 16) || !aligned(w_router, 16) || !aligned(ws, 256)) return MOE_EINVAL;
+    if (d->T == 0) return MOE_OK;
+    DeviceInfo* dev = nullptr;
+    if ((s = device_setup(&dev)) != MOE_OK) return s;
+    const RouterPlan rp = router_plan(d->T, d->H, d->E, dev->num_sms);
+    Carve c;
+    RouteWs rw = carve_route(c, ws, d, rp);
+    if (c.off > ws_bytes) return MOE_EWORKSPACE;
+    return cuda_status(launch_route(static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(w_router), bias,
+                                    d->T, d->H, d->E, d->K, topk_idx, topk_w, rw.P, rw.xn2, rw.wn2, rp,
+                                    make_ctx(dev), static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_permute(const moe_dims* d, const int32_t* topk_idx, int32_t* counts, int32_t* offsets,
+                       int32_t* perm_src, int32_t* inv_row, void* ws, size_t ws_bytes, void* stream) {
+    (void)ws;
+    (void)ws_bytes;
+    moe_status s = check_dims(d);
+    if (s != MOE_OK) return s;
+    if (!counts || !offsets) return MOE_EINVAL;
+    if (d->T > 0 && (!topk_idx || !perm_src || !inv_row)) return MOE_EINVAL;
+    DeviceInfo* dev = nullptr;
+    if ((s = device_setup(&dev)) != MOE_OK) return s;
+    return cuda_status(launch_permute(topk_idx, d->T * d->K, d->E, counts, offsets, perm_src, inv_row, nullptr,
+                                      nullptr, 16, make_ctx(dev), static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_expert_ffn(const moe_dims* d, const void* x, const int32_t* offsets, const int32_t* perm_src,
+                          const void* w_up, const void* w_down, const moe_fp8_scales* scales, void* y_perm,
+                          void* ws, size_t ws_bytes, void* stream) {
+    moe_status s = check_dims(d);
+    if (s != MOE_OK) return s;
+    if ((s = check_fp8_scales(d, scales)) != MOE_OK) return s;
+    if (d->T > 0 && (!x || !offsets || !perm_src || !w_up || !w_down || !y_perm || !ws)) return MOE_EINVAL;
+    if (!aligned(x, 16) || !aligned(w_up, 16) || !aligned(w_down, 16) || !aligned(y_perm, 16) || !aligned(ws, 256))
+        return MOE_EINVAL;
+    if (d->T == 0) return MOE_OK;
+    DeviceInfo* dev = nullptr;
+    if ((s = device_setup(&dev)) != MOE_OK) return s;
+    const GemmPlan gp = gemm_plan(d->T, d->K, d->E);
+    Carve c;
+    FfnWs fw = carve_ffn(c, ws, d, gp);
+    if (c.off > ws_bytes) return MOE_EWORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = launch_schedule(offsets, d->E, gp.bn, fw.sched, fw.n_sched, st);
+    if (e != cudaSuccess) return cuda_status(e);
+    return run_ffn(d, dev, make_ctx(dev), gp, x, perm_src, w_up, w_down, scales, fw, y_perm, st);
+}
+
+moe_status moe_combine(const moe_dims* d, const void* y_perm, const int32_t* inv_row, const float* topk_w,
+                       const void* residual, void* out, void* stream) {
+    moe_status s = check_dims(d);
+    if (s != MOE_OK) return s;
+    if (d->T > 0 && (!y_perm || !inv_row || !topk_w || !out)) return MOE_EINVAL;
+    if (!aligned(y_perm, 16) || !aligned(residual, 16) || !aligned(out, 16)) return MOE_EINVAL;
+    if (d->T == 0) return MOE_OK;
+    DeviceInfo* dev = nullptr;
+    if ((s = device_setup(&dev)) != MOE_OK) return s;
+    return cuda_status(launch_combine(static_cast<const uint16_t*>(y_perm), inv_row, topk_w,
+                                      static_cast<const uint16_t*>(residual), static_cast<uint16_t*>(out), d->T,
+                                      d->K, d->H, dev->num_sms, make_ctx(dev), static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_forward(const moe_dims* d, const void* x, const void* w_router, const float* bias, const void* w_up,
+                       const void* w_down, const moe_fp8_scales* scales, const void* residual, void* out,
+                       int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes, void* stream) {
+    moe_status s = check_dims(d);
+    if (s != MOE_OK) return s;
+    if ((s = check_fp8_scales(d, scales)) != MOE_OK) return s;
+    if (d->T > 0 && (!x || !w_router || !w_up || !w_down || !out || !ws)) return MOE_EINVAL;
+    if (!aligned(x, 16) || !aligned(w_router, 16) || !aligned(w_up, 16) || !aligned(w_down, 16) ||
+        !aligned(residual, 16) || !aligned(out, 16) || !aligned(ws, 256))
+        return MOE_EINVAL;
+    if (d->T == 0) return MOE_OK;
+    DeviceInfo* dev = nullptr;
+    if ((s = device_setup(&dev)) != MOE_OK) return s;
+    if (ws_bytes < forward_ws_bytes(d, dev->num_sms)) return MOE_EWORKSPACE;
+    const DevCtx ctx = make_ctx(dev);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+    Carve c;
+    ForwardWs fw = carve_forward(c, ws, d);
+    const size_t scratch = (c.off + 255) & ~size_t(255);
+    void* sbase = static_cast<uint8_t*>(ws) + scratch;
+    int32_t* idx = topk_idx ? topk_idx : fw.idx;
+    float* w = topk_w ? topk_w : fw.w;
+
+    const RouterPlan rp = router_plan(d->T, d->H, d->E, dev->num_sms);
+    Carve cr;
+    RouteWs rw = carve_route(cr, sbase, d, rp);
+    cudaError_t e = launch_route(static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(w_router), bias, d->T,
+                                 d->H, d->E, d->K, idx, w, rw.P, rw.xn2, rw.wn2, rp, ctx, st);
+    if (e != cudaSuccess) return cuda_status(e);
+
+    const GemmPlan gp = gemm_plan(d->T, d->K, d->E);
+    Carve cf;
+    FfnWs ffw = carve_ffn(cf, sbase, d, gp);   // reuses the router scratch region
+    e = launch_permute(idx, d->T * d->K, d->E, fw.counts, fw.offsets, fw.perm_src, fw.inv_row, ffw.sched,
+                       ffw.n_sched, gp.bn, ctx, st);
+    if (e != cudaSuccess) return cuda_status(e);
+    s = run_ffn(d, dev, ctx, gp, x, fw.perm_src, w_up, w_down, scales, ffw, fw.y_perm, st);
+    if (s != MOE_OK) return s;
+    return cuda_status(launch_combine(static_cast<const uint16_t*>(fw.y_perm), fw.inv_row, w,
+                                      static_cast<const uint16_t*>(residual), static_cast<uint16_t*>(out), d->T,
+                                      d->K, d->H, dev->num_sms, ctx, st));
+}
+
+moe_status moe_quantize_fp8(int64_t n_tensors, int64_t tensor_elems, const void* src, uint8_t* codes,
+                            float* scales, void* stream) {
+    if (n_tensors < 0 || tensor_elems < 0 || n_tensors > ((int64_t)1 << 31)) return MOE_EINVAL;
+    if (n_tensors == 0 || tensor_elems == 0) return MOE_OK;
+    if (!src || !codes || !scales || !aligned(src, 16) || !aligned(scales, 4)) return MOE_EINVAL;
+    DeviceInfo* dev = nullptr;
+    moe_status s = device_setup(&dev);
+    if (s != MOE_OK) return s;
+    return cuda_status(launch_quantize(n_tensors, tensor_elems, static_cast<const uint16_t*>(src), codes, scales,
+                                       dev->num_sms, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_rmsnorm(int64_t T, int32_t H, float eps, const void* x, void* u, void* stream) {
+    if (T < 0 || H < 16 || H > 65536 || H % 16 != 0 || !(eps >= 0.0f)) return MOE_EINVAL;
+    if (T == 0) return MOE_OK;
+    if (!x || !u || x == u || !aligned(x, 16) || !aligned(u, 16)) return MOE_EINVAL;
+    DeviceInfo* dev = nullptr;
+    moe_status s = device_setup(&dev);
+    if (s != MOE_OK) return s;
+    return cuda_status(launch_rmsnorm(static_cast<const uint16_t*>(x), static_cast<uint16_t*>(u), T, H, eps,
+                                      dev->num_sms, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_check_device_error(void* stream) {
+    DeviceInfo* dev = nullptr;
+    moe_status s = device_setup(&dev);
+    if (s != MOE_OK) return s;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ECUDA;
+    int v = 0;
+    if (cudaMemcpy(&v, dev->err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ECUDA;
+    if (v != 0) {
+        const int zero = 0;
+        if (cudaMemcpy(dev->err, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return MOE_ECUDA;
+        return static_cast<moe_status>(v);
+    }
+    return MOE_OK;
+}
+
+moe_status moe_debug_set(int32_t what, int64_t value) {
+    if (what == 1) {
+        g_timeout_ns.store(value > 0 ? (uint64_t)value : kDefaultTimeoutNs);
+        return MOE_OK;
+    }
+    if (what == 2) {
+        g_debug_withhold.store(value ? 1 : 0);
+        return MOE_OK;
+    }
+    return MOE_EINVAL;
+}
+
+}  // extern "C"

@@ -1,0 +1,203 @@
+// Memory-bound kernels around the expert products: the weighted combine, the
+// RMS normalisation of the chained stack, and the per-tensor E4M3 weight
+// quantiser.  All are HBM-bound streams: one warp per row, 16-byte accesses.
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+// out[t] = (residual[t] +) sum_{k=0..K-1} w[t][k] * y_perm[inv_row[t*K+k]]
+// in fp32, k ascending (descending routing logit), one rounding to bf16.
+__global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict__ yp,
+                                                      const int32_t* __restrict__ inv_row,
+                                                      const float* __restrict__ w,
+                                                      const uint16_t* residual, uint16_t* out,
+                                                      int64_t T, int K, int H, int64_t rows,
+                                                      DevCtx ctx) {
+    const int lane = threadIdx.x % 32;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x / 32);
+    const int nv = H / 8;
+    for (int64_t t = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32; t < T; t += warps) {
+        int my_row = 0;
+        float my_w = 0.0f;
+        if (lane < K) {
+            my_row = inv_row[t * K + lane];
+            my_w = w[t * K + lane];
+            if (my_row < 0 || my_row >= rows) {
+                record_error(ctx.err, MOE_EINDEX);
+                my_row = 0;
+                my_w = 0.0f;
+            }
+        }
+        for (int v = lane; v < nv; v += 32) {
+            float acc[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
+            for (int k = 0; k < K; ++k) {
+                const int r = __shfl_sync(0xffffffffu, my_row, k);
+                const float wk = __shfl_sync(0xffffffffu, my_w, k);
+                const uint4 q = reinterpret_cast<const uint4*>(yp + (int64_t)r * H)[v];
+                const uint32_t qq[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    acc[2 * j] = __fmaf_rn(wk, __uint_as_float(qq[j] << 16), acc[2 * j]);
+                    acc[2 * j + 1] = __fmaf_rn(wk, __uint_as_float(qq[j] & 0xFFFF0000u), acc[2 * j + 1]);
+                }
+            }
+            if (residual) {
+                const uint4 q = reinterpret_cast<const uint4*>(residual + t * H)[v];
+                const uint32_t qq[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    acc[2 * j] = __fadd_rn(__uint_as_float(qq[j] << 16), acc[2 * j]);
+                    acc[2 * j + 1] = __fadd_rn(__uint_as_float(qq[j] & 0xFFFF0000u), acc[2 * j + 1]);
+                }
+            }
+            uint32_t o[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(acc[2 * j]));
+                const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(acc[2 * j + 1]));
+                o[j] = lo | (hi << 16);
+            }
+            reinterpret_cast<uint4*>(out + t * H)[v] = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+    }
+}
+
+// u = bf16(x / sqrt(mean(x^2) + eps)): sum of squares in fixed point (each
+// x^2, exact in fp32, rounded to 2^-16 and summed exactly in int64), the rest
+// in correctly rounded fp32, so the result is bit-reproducible anywhere.
+__global__ void __launch_bounds__(256) rmsnorm_kernel(const uint16_t* __restrict__ x,
+                                                      uint16_t* __restrict__ u, int64_t T, int H,
+                                                      float eps) {
+    const int lane = threadIdx.x % 32;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x / 32);
+    const int nv = H / 8;
+    for (int64_t t = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32; t < T; t += warps) {
+        const uint4* xr = reinterpret_cast<const uint4*>(x + t * H);
+        long long acc = 0;
+        for (int v = lane; v < nv; v += 32) {
+            const uint4 q = xr[v];
+            const uint32_t qq[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const float f = __uint_as_float((j & 1) ? (qq[j / 2] & 0xFFFF0000u) : (qq[j / 2] << 16));
+                acc += __float2ll_rn(__fmul_rn(__fmul_rn(f, f), 65536.0f));
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        float ms = __ll2float_rn(acc);
+        ms = __fmul_rn(ms, 1.0f / 65536.0f);
+        ms = __fdiv_rn(ms, (float)H);
+        ms = __fadd_rn(ms, eps);
+        const float rstd = __fdiv_rn(1.0f, __fsqrt_rn(ms));
+        uint4* ur = reinterpret_cast<uint4*>(u + t * H);
+        for (int v = lane; v < nv; v += 32) {
+            const uint4 q = xr[v];
+            const uint32_t qq[4] = {q.x, q.y, q.z, q.w};
+            uint32_t o[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float a = __fmul_rn(__uint_as_float(qq[j] << 16), rstd);
+                const float b = __fmul_rn(__uint_as_float(qq[j] & 0xFFFF0000u), rstd);
+                o[j] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(a)) |
+                       ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(b)) << 16);
+            }
+            ur[v] = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+    }
+}
+
+// amax over each tensor (as the bits of |v|, which order like the values).
+__global__ void __launch_bounds__(256) amax_kernel(const uint16_t* __restrict__ src, int64_t elems,
+                                                   unsigned int* __restrict__ amax_bits) {
+    const int64_t tensor = blockIdx.y;
+    const uint16_t* p = src + tensor * elems;
+    uint32_t m = 0;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < elems; i += stride) {
+        const uint32_t b = ((uint32_t)p[i] << 16) & 0x7FFFFFFFu;
+        m = max(m, b);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
+    if ((threadIdx.x & 31) == 0) atomicMax(&amax_bits[tensor], m);
+}
+
+// scale = amax / 448 (1 for an all-zero tensor), in place over the amax bits.
+__global__ void finalize_scale_kernel(float* scales, int64_t n) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n) {
+        const float amax = __uint_as_float(reinterpret_cast<unsigned int*>(scales)[i]);
+        scales[i] = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+    }
+}
+
+__global__ void __launch_bounds__(256) quantize_kernel(const uint16_t* __restrict__ src, int64_t elems,
+                                                       const float* __restrict__ scales,
+                                                       uint8_t* __restrict__ codes) {
+    const int64_t tensor = blockIdx.y;
+    const float s = scales[tensor];
+    const uint16_t* p = src + tensor * elems;
+    uint8_t* q = codes + tensor * elems;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < elems; i += stride) {
+        const float v = __uint_as_float((uint32_t)p[i] << 16);
+        q[i] = (uint8_t)__nv_cvt_float_to_fp8(__fdiv_rn(v, s), __NV_SATFINITE, __NV_E4M3);
+    }
+}
+
+// ----------------------------------------------------------------------------- host
+
+static unsigned grid_rows(int64_t rows, int num_sms) {
+    int64_t b = (rows + 7) / 8;
+    const int64_t cap = (int64_t)num_sms * 8;
+    if (b > cap) b = cap;
+    return (unsigned)(b > 0 ? b : 1);
+}
+
+cudaError_t launch_combine(const uint16_t* yp, const int32_t* inv_row, const float* w,
+                           const uint16_t* residual, uint16_t* out, int64_t T, int K, int H,
+                           int num_sms, const DevCtx& ctx, cudaStream_t stream) {
+    if (T == 0) return cudaSuccess;
+    combine_kernel<<<grid_rows(T, num_sms), 256, 0, stream>>>(yp, inv_row, w, residual, out, T, K, H,
+                                                              T * K, ctx);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_rmsnorm(const uint16_t* x, uint16_t* u, int64_t T, int H, float eps, int num_sms,
+                           cudaStream_t stream) {
+    if (T == 0) return cudaSuccess;
+    rmsnorm_kernel<<<grid_rows(T, num_sms), 256, 0, stream>>>(x, u, T, H, eps);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quantize(int64_t n_tensors, int64_t elems, const uint16_t* src, uint8_t* codes,
+                            float* scales, int num_sms, cudaStream_t stream) {
+    if (n_tensors == 0 || elems == 0) return cudaSuccess;
+    cudaError_t err = cudaMemsetAsync(scales, 0, (size_t)n_tensors * sizeof(float), stream);
+    if (err != cudaSuccess) return err;
+    int64_t bx = (elems + 255) / 256;
+    const int64_t cap = (n_tensors >= num_sms) ? 4 : (int64_t)num_sms * 8 / n_tensors + 1;
+    if (bx > cap) bx = cap;
+    for (int64_t t0 = 0; t0 < n_tensors; t0 += 65535) {
+        const int64_t nt = n_tensors - t0 < 65535 ? n_tensors - t0 : 65535;
+        amax_kernel<<<dim3((unsigned)bx, (unsigned)nt), 256, 0, stream>>>(
+            src + t0 * elems, elems, reinterpret_cast<unsigned int*>(scales) + t0);
+    }
+    finalize_scale_kernel<<<(unsigned)((n_tensors + 255) / 256), 256, 0, stream>>>(scales, n_tensors);
+    for (int64_t t0 = 0; t0 < n_tensors; t0 += 65535) {
+        const int64_t nt = n_tensors - t0 < 65535 ? n_tensors - t0 : 65535;
+        quantize_kernel<<<dim3((unsigned)bx, (unsigned)nt), 256, 0, stream>>>(src + t0 * elems, elems,
+                                                                              scales + t0, codes + t0 * elems);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,365 @@
+// Grouped expert GEMMs on the 5th-generation tensor cores (tcgen05).
+//
+// The two expert projections (bloomery issue page, s.2 "Checkpoint facts":
+// ungated ReLU^2 experts, width 1856; s.3: ungated up/down parts) are, for
+// every expert e and the rows r of its segment in the permuted layout,
+//   up:    Hb[r, f] = relu( sum_h W_up[e][f][h] * X_perm[r][h] )^2
+//   down:  Y [r, j] =       sum_f W_down[e][j][f] * Hb[r][f]
+// Both are computed "swap-AB": the weight rows of one 128-row block of W[e]
+// are the MMA's M side (TMEM lanes), the expert's tokens are its N side
+// (16..256 TMEM columns).  A decode batch has a handful of tokens per expert,
+// so the kernel is a weight stream that the tensor cores consume at N = 16;
+// a prefill chunk has ~192 tokens per expert, so every weight tile is read
+// from HBM once and used for all of them.
+//
+// Work unit = (schedule entry s = {e, row0, nrows}, weight row block mb).
+// Persistent CTAs (one per SM) walk units u = blockIdx.x + i * gridDim.x.
+// Roles (192 threads):
+//   warp 0      TMA producer: per K stage one 128x128-byte weight tile (as
+//               64-row boxes) and ceil(nrows/16) 16x128-byte activation boxes,
+//               both in the 128-byte swizzle, into an NS-deep smem ring;
+//   warp 1      TMEM allocator; lane 0 issues tcgen05.mma (4 per stage, K=16
+//               bf16 or K=32 e4m3) into one of two TMEM accumulators;
+//   warps 2..5  epilogue: tcgen05.ld, scale, ReLU^2 (up) and stores; warp w
+//               reads TMEM lanes 32*(w%4) .. +31.
+// Every wait is bounded; on expiry the block records MOE_ETIMEOUT, drains what
+// it issued and returns.
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int GG_THREADS = 192;
+constexpr int GG_BM = 128;                 // weight rows per unit (MMA M)
+constexpr int GG_ROW_BYTES = 128;          // bytes of one operand row per stage (K extent)
+constexpr int GG_A_BYTES = GG_BM * GG_ROW_BYTES;   // 16 KB
+constexpr int GG_TMEM_COLS = 512;          // two accumulators of up to 256 columns
+
+struct GemmArgs {
+    const int4* sched;       // {e, row0, nrows, 0}
+    const int* n_sched;      // device count of schedule entries
+    int m_blocks;            // ceil(Nout / 128)
+    int Nout;                // rows of one expert's weight (F for up, H for down)
+    int k_stages;            // ceil(Kdim * elem / 128)
+    int n_stages;            // smem ring depth
+    int b_stage_bytes;       // bn_max * 128
+    void* out;               // [rows][Nout], bf16 (or e4m3 codes for the fp8 up output)
+    int64_t out_ld;          // elements
+    const float* w_scale;    // [E] (fp8) or null
+    float in_scale;          // x_scale (up) or h_scale (down), fp8 only
+    float out_scale;         // h_scale for the fp8 up output
+    int debug_withhold;      // 1: block 0 withholds its first load
+};
+
+template <bool FP8, bool UP>
+__global__ void __launch_bounds__(GG_THREADS, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                        GemmArgs g, DevCtx ctx) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    const int NS = g.n_stages;
+    uint8_t* smA = smem;
+    uint8_t* smB = smA + (size_t)NS * GG_A_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smB + (size_t)NS * g.b_stage_bytes);
+    uint64_t* full = bars;
+    uint64_t* empty = bars + NS;
+    uint64_t* tfull = bars + 2 * NS;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* drain = tempty + 2;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(drain + 1);
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1) + 1;
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(smem_u32(&full[s]), 1);
+            mbar_init(smem_u32(&empty[s]), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(smem_u32(&tfull[a]), 1);
+            mbar_init(smem_u32(&tempty[a]), 128);
+        }
+        mbar_init(smem_u32(drain), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) tmem_alloc(smem_u32(tmem_holder), GG_TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+
+    const int n_units = (*g.n_sched) * g.m_blocks;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            const uint64_t pol_w = l2_policy_evict_first();
+            const uint64_t pol_x = l2_policy_evict_last();
+            int stage = 0;
+            uint32_t phase = 0;
+            bool withhold = g.debug_withhold && blockIdx.x == 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+                const int4 sc = g.sched[u / g.m_blocks];
+                const int mb = u % g.m_blocks;
+                const int a_valid = min(GG_BM, g.Nout - mb * GG_BM);
+                const int a_boxes = (a_valid + 63) / 64;
+                const int b_boxes = (sc.z + 15) / 16;
+                const uint32_t bytes = (uint32_t)(a_boxes * 64 * GG_ROW_BYTES + b_boxes * 16 * GG_ROW_BYTES);
+                const int a_y = sc.x * g.Nout + mb * GG_BM;
+                for (int ks = 0; ks < g.k_stages; ++ks) {
+                    if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, ctx, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t fb = smem_u32(&full[stage]);
+                    mbar_arrive_expect_tx(fb, bytes);
+                    if (withhold) {
+                        withhold = false;   // this stage never completes: the consumer's wait expires
+                    } else {
+                        const int kx = ks * (FP8 ? 128 : 64);
+                        const uint32_t a_dst = smem_u32(smA + (size_t)stage * GG_A_BYTES);
+                        const uint32_t b_dst = smem_u32(smB + (size_t)stage * g.b_stage_bytes);
+                        for (int i = 0; i < a_boxes; ++i)
+                            tma_load_2d(a_dst + i * 64 * GG_ROW_BYTES, &tmA, fb, kx, a_y + i * 64, pol_w);
+                        for (int j = 0; j < b_boxes; ++j)
+                            tma_load_2d(b_dst + j * 16 * GG_ROW_BYTES, &tmB, fb, kx, sc.y + j * 16, pol_x);
+                    }
+                    if (++stage == NS) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                // let loads already in flight land before the block exits
+                const uint64_t t0 = globaltimer();
+                while (globaltimer() - t0 < 200000ull) __nanosleep(1000);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            bool issued = false;
+            for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+                const int4 sc = g.sched[u / g.m_blocks];
+                const int n_mma = max(16, (sc.z + 15) & ~15);
+                const uint32_t idesc = make_idesc(FP8 ? 0u : 1u, GG_BM, n_mma);
+                if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1u, ctx, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * 256);
+                for (int ks = 0; ks < g.k_stages; ++ks) {
+                    if (!mbar_wait(smem_u32(&full[stage]), phase, ctx, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_base = smem_u32(smA + (size_t)stage * GG_A_BYTES);
+                    const uint32_t b_base = smem_u32(smB + (size_t)stage * g.b_stage_bytes);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        mma_ss<FP8>(d_tmem, sw128_desc(a_base + kk * 32), sw128_desc(b_base + kk * 32),
+                                    idesc, (ks | kk) != 0 ? 1u : 0u);
+                    }
+                    issued = true;
+                    mma_commit(smem_u32(&empty[stage]));
+                    if (++stage == NS) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                mma_commit(smem_u32(&tfull[acc]));
+                if (++acc == 2) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
+            }
+            if (!ok && issued) {
+                // wait for every MMA issued so far before TMEM is released
+                mma_commit(smem_u32(drain));
+                mbar_wait_drain(smem_u32(drain), 0, ctx.timeout_ns);
+            }
+        }
+    } else {
+        const int q = warp & 3;                 // TMEM lane quadrant of this warp
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+            const int4 sc = g.sched[u / g.m_blocks];
+            const int mb = u % g.m_blocks;
+            if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, ctx, abort_flag)) break;
+            tc_fence_after();
+            const int f = mb * GG_BM + q * 32 + lane;
+            const bool fvalid = f < g.Nout;
+            float scale = 1.0f;
+            if constexpr (FP8) scale = __fmul_rn(g.w_scale[sc.x], g.in_scale);
+            const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * 256);
+            const int nchunks = (sc.z + 15) / 16;
+            for (int c = 0; c < nchunks; ++c) {
+                uint32_t v[16];
+                tmem_ld16(t_row + (uint32_t)(c * 16), v);
+                if (fvalid) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int r = c * 16 + j;
+                        if (r < sc.z) {
+                            float z = __uint_as_float(v[j]);
+                            if constexpr (FP8) z = __fmul_rn(z, scale);
+                            const int64_t o = (int64_t)(sc.y + r) * g.out_ld + f;
+                            if constexpr (UP) {
+                                const float a = z > 0.0f ? __fmul_rn(z, z) : 0.0f;
+                                if constexpr (FP8) {
+                                    static_cast<uint8_t*>(g.out)[o] = (uint8_t)__nv_cvt_float_to_fp8(
+                                        __fdiv_rn(a, g.out_scale), __NV_SATFINITE, __NV_E4M3);
+                                } else {
+                                    static_cast<__nv_bfloat16*>(g.out)[o] = __float2bfloat16_rn(a);
+                                }
+                            } else {
+                                static_cast<__nv_bfloat16*>(g.out)[o] = __float2bfloat16_rn(z);
+                            }
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(smem_u32(&tempty[acc]));
+            if (++acc == 2) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, GG_TMEM_COLS);
+    }
+}
+
+// ----------------------------------------------------------------------------- host
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// 2-D map over a row-major [rows][cols] matrix, box = 128 bytes x box_rows,
+// 128-byte swizzle, out-of-range elements read as zero.
+static bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, bool fp8, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const int es = fp8 ? 1 : 2;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(cols * es)};
+    cuuint32_t box[2] = {(cuuint32_t)(GG_ROW_BYTES / es), (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                    const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+struct GemmPlan {
+    int bn;              // max rows per schedule entry
+    int n_stages;
+    size_t smem_bytes;
+    int max_sched;       // schedule entries bound
+};
+
+GemmPlan gemm_plan(int64_t T, int K, int E) {
+    GemmPlan p;
+    const int64_t rows = T * K;
+    int64_t per_expert_max = T < rows ? T : rows;   // an expert gets each token at most once
+    int bn = (int)((per_expert_max + 15) / 16 * 16);
+    if (bn > 256) bn = 256;
+    if (bn < 16) bn = 16;
+    p.bn = bn;
+    const int stage = GG_A_BYTES + bn * GG_ROW_BYTES;
+    int ns = (200 * 1024) / stage;
+    if (ns > 8) ns = 8;
+    if (ns < 2) ns = 2;
+    p.n_stages = ns;
+    p.smem_bytes = 1024 + (size_t)ns * stage + (size_t)(2 * ns + 5) * 8 + 16;
+    const int64_t nonempty = E < rows ? E : rows;
+    p.max_sched = (int)(nonempty + (rows + bn - 1) / bn);
+    return p;
+}
+
+template <bool FP8, bool UP>
+static cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& g, int grid,
+                              size_t smem, const DevCtx& ctx, cudaStream_t stream) {
+    auto kfn = grouped_gemm_kernel<FP8, UP>;
+    cudaError_t err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    kfn<<<grid, GG_THREADS, smem, stream>>>(a, b, g, ctx);
+    return cudaGetLastError();
+}
+
+// One grouped projection.  W: [E * Nout][Kdim] (bf16 or e4m3), Act: [rows][Kdim],
+// out: [rows][Nout].  sched / n_sched: device schedule over the rows.
+cudaError_t launch_grouped_gemm(bool fp8, bool up, const void* W, int E, int Nout, int Kdim, const void* act,
+                                int64_t rows, const int4* sched, const int* n_sched, const GemmPlan& plan,
+                                void* out, const float* w_scale, float in_scale, float out_scale,
+                                int num_sms, int debug_withhold, const DevCtx& ctx, cudaStream_t stream) {
+    if (rows == 0) return cudaSuccess;
+    CUtensorMap ta, tb;
+    if (!make_map(&ta, W, (int64_t)E * Nout, Kdim, fp8, 64)) return cudaErrorInvalidValue;
+    if (!make_map(&tb, act, rows, Kdim, fp8, 16)) return cudaErrorInvalidValue;
+    GemmArgs g;
+    g.sched = sched;
+    g.n_sched = n_sched;
+    g.m_blocks = (Nout + GG_BM - 1) / GG_BM;
+    g.Nout = Nout;
+    const int es = fp8 ? 1 : 2;
+    g.k_stages = (int)(((int64_t)Kdim * es + GG_ROW_BYTES - 1) / GG_ROW_BYTES);
+    g.n_stages = plan.n_stages;
+    g.b_stage_bytes = plan.bn * GG_ROW_BYTES;
+    g.out = out;
+    g.out_ld = Nout;
+    g.w_scale = w_scale;
+    g.in_scale = in_scale;
+    g.out_scale = out_scale;
+    g.debug_withhold = debug_withhold;
+    const int64_t max_units = (int64_t)plan.max_sched * g.m_blocks;
+    const int grid = (int)(max_units < num_sms ? max_units : num_sms);
+    if (fp8) {
+        return up ? launch_one<true, true>(ta, tb, g, grid, plan.smem_bytes, ctx, stream)
+                  : launch_one<true, false>(ta, tb, g, grid, plan.smem_bytes, ctx, stream);
+    }
+    return up ? launch_one<false, true>(ta, tb, g, grid, plan.smem_bytes, ctx, stream)
+              : launch_one<false, false>(ta, tb, g, grid, plan.smem_bytes, ctx, stream);
+}
+
+}  // namespace moe

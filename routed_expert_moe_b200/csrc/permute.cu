@@ -1,0 +1,217 @@
+// Token permutation into expert-contiguous rows, the GEMM tile schedule, and
+// the row gather that feeds the up-projection.
+//
+// The grouped expert products (audio.cpp model page, "CPU weight offload")
+// run on rows grouped by expert.  The grouping is a stable counting sort of
+// the assignments i = t*K + k by expert: a histogram, an exclusive scan, and
+// a scatter that keeps ascending i inside each expert's segment.  The sort
+// is one block: at 24,576 assignments it is a few microseconds, and one
+// block keeps the stable ranks free of any cross-block protocol.
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_fp8.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int PM_THREADS = 1024;
+
+// Tile schedule: expert e's segment [offsets[e], offsets[e+1]) is cut into
+// near-equal blocks of at most bn rows, each a multiple of 16 rows except the
+// last: per = round16(ceil(cnt / ceil(cnt / bn))), nblk = ceil(cnt / per).
+// Entry {e, row0, nrows, 0}.  Called by the whole block; nb_s is shared
+// scratch of E ints.
+__device__ __forceinline__ int sched_per(int c, int bn) {
+    const int nb = (c + bn - 1) / bn;
+    const int per = (c + nb - 1) / nb;
+    return (per + 15) & ~15;
+}
+
+__device__ void build_schedule(const int* seg_off, int E, int bn, int* nb_s, int4* sched,
+                               int* n_sched) {
+    const int tid = threadIdx.x;
+    for (int e = tid; e < E; e += blockDim.x) {
+        const int c = seg_off[e + 1] - seg_off[e];
+        nb_s[e] = c > 0 ? (c + sched_per(c, bn) - 1) / sched_per(c, bn) : 0;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        int run = 0;
+        for (int e = 0; e < E; ++e) {
+            const int v = nb_s[e];
+            nb_s[e] = run;
+            run += v;
+        }
+        *n_sched = run;
+    }
+    __syncthreads();
+    for (int e = tid; e < E; e += blockDim.x) {
+        const int off = seg_off[e], c = seg_off[e + 1] - off;
+        if (c <= 0) continue;
+        const int per = sched_per(c, bn);
+        for (int r0 = 0, b = 0; r0 < c; r0 += per, ++b)
+            sched[nb_s[e] + b] = make_int4(e, off + r0, min(per, c - r0), 0);
+    }
+}
+
+struct PermuteArgs {
+    const int32_t* idx;
+    int64_t n;       // T*K
+    int E;
+    int32_t* counts;
+    int32_t* offsets;
+    int32_t* perm_src;
+    int32_t* inv_row;
+    int4* sched;     // may be null
+    int* n_sched;
+    int bn;
+};
+
+__global__ void __launch_bounds__(PM_THREADS) permute_kernel(PermuteArgs a, DevCtx ctx) {
+    extern __shared__ int sm[];
+    const int E = a.E;
+    int* hist = sm;               // [E]
+    int* base = hist + E;         // [E] next free row of each expert
+    int* tot = base + E;          // [E] chunk totals
+    int* offs = tot + E;          // [E+1]
+    int* wtab = offs + E + 1;     // [32][E] per-warp counts of the chunk
+    const int tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
+    const uint32_t lt_mask = (1u << lane) - 1u;
+
+    for (int e = tid; e < E; e += PM_THREADS) hist[e] = 0;
+    __syncthreads();
+    int bad = 0;
+    for (int64_t i = tid; i < a.n; i += PM_THREADS) {
+        const int e = a.idx[i];
+        if (e < 0 || e >= E) {
+            bad = 1;
+            continue;
+        }
+        atomicAdd(&hist[e], 1);
+    }
+    if (__syncthreads_or(bad)) {
+        if (tid == 0) record_error(ctx.err, MOE_EINDEX);
+    }
+    if (tid == 0) {
+        int run = 0;
+        for (int e = 0; e < E; ++e) {
+            offs[e] = run;
+            base[e] = run;
+            a.offsets[e] = run;
+            a.counts[e] = hist[e];
+            run += hist[e];
+        }
+        offs[E] = run;
+        a.offsets[E] = run;
+    }
+    __syncthreads();
+
+    for (int64_t c0 = 0; c0 < a.n; c0 += PM_THREADS) {
+        const int64_t i = c0 + tid;
+        int e = i < a.n ? a.idx[i] : -1;
+        if (e >= E) e = -1;
+        for (int q = tid; q < 32 * E; q += PM_THREADS) wtab[q] = 0;
+        __syncthreads();
+        const uint32_t peers = __match_any_sync(0xffffffffu, e);
+        const int rank_w = __popc(peers & lt_mask);
+        if (e >= 0 && rank_w == 0) wtab[warp * E + e] = __popc(peers);
+        __syncthreads();
+        for (int ex = tid; ex < E; ex += PM_THREADS) {
+            int run = 0;
+            for (int w = 0; w < 32; ++w) {
+                const int v = wtab[w * E + ex];
+                wtab[w * E + ex] = run;
+                run += v;
+            }
+            tot[ex] = run;
+        }
+        __syncthreads();
+        if (e >= 0) {
+            const int r = base[e] + wtab[warp * E + e] + rank_w;
+            a.perm_src[r] = (int32_t)i;
+            a.inv_row[i] = r;
+        }
+        __syncthreads();
+        for (int ex = tid; ex < E; ex += PM_THREADS) base[ex] += tot[ex];
+        __syncthreads();
+    }
+    if (a.sched) build_schedule(offs, E, a.bn, hist, a.sched, a.n_sched);
+}
+
+__global__ void schedule_kernel(const int32_t* offsets, int E, int bn, int4* sched, int* n_sched) {
+    __shared__ int offs[257];
+    __shared__ int nb[256];
+    for (int e = threadIdx.x; e <= E; e += blockDim.x) offs[e] = offsets[e];
+    __syncthreads();
+    build_schedule(offs, E, bn, nb, sched, n_sched);
+}
+
+// X_perm[r] = x[perm_src[r] / K], or its E4M3 codes e4m3(x / x_scale) (fp8).
+__global__ void gather_rows_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm_src,
+                                   int64_t rows, int K, int64_t T, int H, void* __restrict__ xp,
+                                   int fp8, float x_scale, DevCtx ctx) {
+    const int lane = threadIdx.x % 32;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x / 32);
+    const int nv = H / 8;
+    for (int64_t r = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32; r < rows; r += warps) {
+        const int32_t src = perm_src[r];
+        const int64_t t = src / K;
+        if (src < 0 || t >= T) {
+            if (lane == 0) record_error(ctx.err, MOE_EINDEX);
+            continue;
+        }
+        const uint4* xr = reinterpret_cast<const uint4*>(x + t * H);
+        if (!fp8) {
+            uint4* out = reinterpret_cast<uint4*>(static_cast<uint16_t*>(xp) + r * H);
+            for (int v = lane; v < nv; v += 32) out[v] = xr[v];
+        } else {
+            uint2* out = reinterpret_cast<uint2*>(static_cast<uint8_t*>(xp) + r * H);
+            for (int v = lane; v < nv; v += 32) {
+                const uint4 q = xr[v];
+                const uint32_t wv[4] = {q.x, q.y, q.z, q.w};
+                uint32_t packed[2] = {0, 0};
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const uint32_t bits = (j & 1) ? (wv[j / 2] & 0xFFFF0000u) : (wv[j / 2] << 16);
+                    const float f = __fdiv_rn(__uint_as_float(bits), x_scale);
+                    const uint32_t c = __nv_cvt_float_to_fp8(f, __NV_SATFINITE, __NV_E4M3);
+                    packed[j / 4] |= c << (8 * (j % 4));
+                }
+                out[v] = make_uint2(packed[0], packed[1]);
+            }
+        }
+    }
+}
+
+// ----------------------------------------------------------------------------- host
+
+size_t permute_smem_bytes(int E) { return (size_t)(4 * E + 1 + 32 * E) * sizeof(int); }
+
+cudaError_t launch_permute(const int32_t* idx, int64_t n, int E, int32_t* counts, int32_t* offsets,
+                           int32_t* perm_src, int32_t* inv_row, int4* sched, int* n_sched, int bn,
+                           const DevCtx& ctx, cudaStream_t stream) {
+    PermuteArgs a{idx, n, E, counts, offsets, perm_src, inv_row, sched, n_sched, bn};
+    permute_kernel<<<1, PM_THREADS, permute_smem_bytes(E), stream>>>(a, ctx);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_schedule(const int32_t* offsets, int E, int bn, int4* sched, int* n_sched,
+                            cudaStream_t stream) {
+    schedule_kernel<<<1, 256, 0, stream>>>(offsets, E, bn, sched, n_sched);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gather(const uint16_t* x, const int32_t* perm_src, int64_t rows, int K, int64_t T,
+                          int H, void* xp, bool fp8, float x_scale, int num_sms, const DevCtx& ctx,
+                          cudaStream_t stream) {
+    if (rows == 0) return cudaSuccess;
+    int64_t blocks = (rows + 7) / 8;
+    const int64_t cap = (int64_t)num_sms * 8;
+    if (blocks > cap) blocks = cap;
+    gather_rows_kernel<<<(unsigned)blocks, 256, 0, stream>>>(x, perm_src, rows, K, T, H, xp,
+                                                              fp8 ? 1 : 0, x_scale, ctx);
+    return cudaGetLastError();
+}
+
+}  // namespace moe
