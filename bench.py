@@ -1,0 +1,454 @@
+"""Benchmark of the routed mixture-of-experts layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode|prefill|skewed]
+                    [--impl native|reference]
+
+One step = one pass of the whole layer (router, top-K, permute, row gather,
+up GEMM + ReLU^2, down GEMM, combine) over one batch of seeded synthetic
+tokens, through the C ABI's moe_forward.  The default workload is the
+decode-sized layer (64 tokens, hidden 2688, 128 experts, top-6, expert width
+1856, bf16); a prefill-chunk (4096-token) measurement is reported beside it.
+
+Under torchrun (N > 1) every rank runs its own batch on its own GPU with
+replicated weights (the layer is independent per token): weak scaling, no
+data-path collective; the time is the max over ranks.
+
+Prints ONE JSON line on rank 0.  ``--impl reference`` times the CPU oracle
+(the plain fp64 statement of the layer) on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+from pathlib import Path
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+METRIC = "MoE-layer tokens/s on 1 B200; % of HBM roofline (decode), % TC peak (prefill)"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+WORKLOADS = {"tiny": 0, "decode": 1, "prefill": 2, "skewed": 3}
+
+
+def load_peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def reduce_max(value: float, dist=None, device=None) -> float:
+    """Max over ranks (identity on one rank): every multi-GPU time is the slowest rank's."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(world: int, tokens_per_rank: int, steps: int, ms: float) -> float:
+    """Whole-job throughput: tokens processed by all ranks / the max-over-ranks time."""
+    return world * tokens_per_rank * steps / (ms * 1e-3)
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+# --------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_uuid: str | None):
+        self.uuid = gpu_uuid
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
+        if self.uuid:
+            cmd[1:1] = ["-i", self.uuid]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        return self.summary()
+
+    def summary(self):
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = max(mx, float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- native arm
+
+class Layer:
+    """Device-resident weights and buffers of one workload."""
+
+    def __init__(self, wl, device, n_batches=4):
+        import torch
+        import synth
+        import routed_expert_moe_b200 as moe
+        from synth import workloads as W
+
+        self.wl = wl
+        self.moe = moe
+        self.device = device
+        bf = torch.bfloat16
+        stream = torch.cuda.current_stream().cuda_stream
+        self.wu = torch.empty(wl.E, wl.F, wl.H, dtype=bf, device=device)
+        self.wd = torch.empty(wl.E, wl.H, wl.F, dtype=bf, device=device)
+        self.wr = torch.empty(wl.E, wl.H, dtype=bf, device=device)
+        synth.normal_bf16_device(synth.key(wl.seed, synth.T_WUP, 0), self.wu.numel(), W.SIGMA_W,
+                                 self.wu.data_ptr(), stream)
+        synth.normal_bf16_device(synth.key(wl.seed, synth.T_WDOWN, 0), self.wd.numel(), W.SIGMA_W,
+                                 self.wd.data_ptr(), stream)
+        synth.normal_bf16_device(synth.key(wl.seed, synth.T_WR, 0), self.wr.numel(), W.SIGMA_W,
+                                 self.wr.data_ptr(), stream)
+        self.bias = None
+        b = W.host_bias(wl)
+        if b is not None:
+            self.bias = torch.from_numpy(b).to(device)
+        # several token batches (batch 0 is the workload's own x; others use layer ids 1..)
+        self.xs = []
+        for i in range(n_batches):
+            x = torch.empty(wl.T, wl.H, dtype=bf, device=device)
+            synth.normal_bf16_device(synth.key(wl.seed, synth.T_X, i), x.numel(), W.SIGMA_X, x.data_ptr(), stream)
+            self.xs.append(x)
+        self.dims = moe.dims(wl.T, wl.H, wl.E, wl.K, wl.F)
+        self.ws = moe.alloc_workspace(self.dims, device)
+        self.out = torch.empty(wl.T, wl.H, dtype=bf, device=device)
+        self.idx = torch.empty(wl.T, wl.K, dtype=torch.int32, device=device)
+        self.w = torch.empty(wl.T, wl.K, dtype=torch.float32, device=device)
+        torch.cuda.synchronize(device)
+
+    def step(self, i, x=None, out=None):
+        self.moe.forward(self.dims, self.xs[i % len(self.xs)] if x is None else x, self.wr, self.bias, self.wu,
+                         self.wd, self.out if out is None else out, self.ws, topk_idx=self.idx, topk_w=self.w)
+
+    def touched_experts(self, i):
+        import torch
+        self.step(i)
+        torch.cuda.synchronize()
+        return int(torch.unique(self.idx).numel()), int(self.idx.numel())
+
+
+def stage_profile(layer, steps, warmup):
+    """Per-stage device time (ms, mean over steps) from the library's stage events."""
+    import torch
+    moe = layer.moe
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(moe.STAGE_EVENTS)] for _ in range(steps)]
+    for i in range(warmup):
+        layer.step(i)
+    times = [[0.0] * (moe.STAGE_EVENTS - 1) for _ in range(steps)]
+    for i in range(steps):
+        moe.set_stage_events(ev[i])
+        layer.step(i)
+    moe.set_stage_events(None)
+    torch.cuda.synchronize()
+    for i in range(steps):
+        for s in range(moe.STAGE_EVENTS - 1):
+            times[i][s] = ev[i][s].elapsed_time(ev[i][s + 1])
+    return {name: statistics.mean(t[s] for t in times) for s, name in enumerate(moe.STAGES)}
+
+
+def timed_loop(layer, steps, warmup, barrier):
+    import torch
+    for i in range(warmup):
+        layer.step(i)
+    barrier()
+    torch.cuda.synchronize()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for i in range(steps):
+        layer.step(i)
+    stop.record()
+    torch.cuda.synchronize()
+    barrier()
+    return start.elapsed_time(stop)
+
+
+def e2e_loop(layer, steps, warmup):
+    """Same metric through the public API with host buffers: H2D of x, forward, D2H of out."""
+    import torch
+    wl = layer.wl
+    hx = [torch.empty(wl.T, wl.H, dtype=torch.bfloat16, pin_memory=True) for _ in range(len(layer.xs))]
+    for i, x in enumerate(layer.xs):
+        hx[i].copy_(x.cpu())
+    hout = torch.empty(wl.T, wl.H, dtype=torch.bfloat16, pin_memory=True)
+    dx = torch.empty(wl.T, wl.H, dtype=torch.bfloat16, device=layer.device)
+
+    def one(i):
+        dx.copy_(hx[i % len(hx)], non_blocking=True)
+        layer.step(i, x=dx)
+        hout.copy_(layer.out, non_blocking=True)
+
+    for i in range(warmup):
+        one(i)
+    torch.cuda.synchronize()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for i in range(steps):
+        one(i)
+    stop.record()
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(stop)
+    nb = wl.T * wl.H * 2
+    return ms, nb, nb
+
+
+def traffic_from_profile(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it matches this build."""
+    p = ROOT / "profiles" / "traffic.json"
+    if not p.exists():
+        return None
+    try:
+        d = json.loads(p.read_text())
+    except ValueError:
+        return None
+    ent = d.get(f"{kernel}@{workload}")
+    if not ent:
+        return None
+    import hashlib
+    h = hashlib.sha256()
+    for f in sorted((ROOT / "routed_expert_moe_b200" / "csrc").glob("*.cu*")):
+        h.update(f.read_bytes())
+    if ent.get("source_sha256") != h.hexdigest():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+def roofline_entry(wl, stages, touched, peaks, peak_kind, workload):
+    """Roofline of the dominant kernel of the step (an expert GEMM)."""
+    H, F, T, K = wl.H, wl.F, wl.T, wl.K
+    rows = T * K
+    up_ms, down_ms = stages["up_gemm"], stages["down_gemm"]
+    kernel = "up_gemm" if up_ms >= down_ms else "down_gemm"
+    ms = max(up_ms, down_ms)
+    flops = 2.0 * rows * F * H
+    if workload == "prefill":
+        peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+        achieved = flops / (ms * 1e-3) / 1e12
+        return {"kernel": kernel, "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "peak_source": f"{peak_kind} bf16 sustained",
+                "algorithmic_flops_per_launch": flops, "ms_per_launch": ms,
+                "traffic": traffic_from_profile(kernel, workload)}
+    wbytes = touched * F * H * 2
+    act = rows * H * 2 + rows * F * 2            # X_perm read + Hb write (up); Hb read + Y write (down)
+    if kernel == "down_gemm":
+        act = rows * F * 2 + rows * H * 2
+    algo = wbytes + act
+    peak = peaks["hbm_gbs"]
+    achieved = algo / (ms * 1e-3) / 1e9
+    return {"kernel": kernel, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+            "frac": achieved / peak, "peak_source": f"{peak_kind} hbm copy",
+            "algorithmic_bytes_per_launch": algo, "ms_per_launch": ms,
+            "traffic": traffic_from_profile(kernel, workload)}
+
+
+def cpu_baseline(wl, n_tokens, seed_batch=0):
+    """The oracle as it stands, on the host cores, over a bounded sample of the workload."""
+    import oracle
+    from synth import workloads as W
+    x = W.host_x(wl, seed_batch)[:n_tokens]
+    wr = W.host_router(wl)
+    t0 = time.perf_counter()
+    _, idx, _ = oracle.route(x, wr, W.host_bias(wl), wl.K)
+    used = sorted(set(idx.reshape(-1).tolist()))
+    slot = -__import__("numpy").ones(wl.E, dtype="int32")
+    slot[used] = range(len(used))
+    t_route = time.perf_counter() - t0
+    wu = W.host_w_up(wl, experts=used)       # generating inputs is not timed
+    wd = W.host_w_down(wl, experts=used)
+    t0 = time.perf_counter()
+    oracle.moe_layer_bf16(x, wr, W.host_bias(wl), wu, wd, wl.K, slot=slot)
+    dt = time.perf_counter() - t0 + t_route
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return {"value": n_tokens / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{n_tokens} of the {wl.T} tokens of batch {seed_batch} ({wl.name}), full layer "
+                      f"(router, top-{wl.K}, {len(used)} experts' up/ReLU^2/down in fp64, combine); "
+                      f"{dt:.2f} s"}
+
+
+def run_native(args):
+    import torch
+    import torch.distributed as dist
+    from synth import workloads as W
+
+    ws, rank, local = dist_env()
+    if ws > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+        barrier = lambda: dist.barrier()
+    else:
+        barrier = lambda: None
+    device = torch.device("cuda", torch.cuda.current_device())
+    peaks, peak_kind = load_peaks()
+
+    wl = W.WORKLOADS[WORKLOADS[args.workload]]
+    layer = Layer(wl, device)
+    touched, rows = layer.touched_experts(0)
+    stages = stage_profile(layer, max(3, min(args.steps, 20)), args.warmup)
+
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+    except Exception:
+        uuid = None
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    time.sleep(0.3)
+    ms = timed_loop(layer, args.steps, args.warmup, barrier)
+    clocks = sampler.stop()
+
+    ms = reduce_max(ms, dist if ws > 1 else None, device)
+    e2e_ms, bi, bo = e2e_loop(layer, args.steps, args.warmup)
+    e2e_ms = reduce_max(e2e_ms, dist if ws > 1 else None, device)
+
+    secondary = None
+    if not args.no_secondary and args.workload == "decode" and ws == 1:
+        del layer
+        torch.cuda.empty_cache()
+        wl2 = W.WORKLOADS[2]
+        layer2 = Layer(wl2, device, n_batches=2)
+        t2, _ = layer2.touched_experts(0)
+        st2 = stage_profile(layer2, 10, 3)
+        ms2 = timed_loop(layer2, 10, 3, barrier)
+        secondary = {"workload": wl2.name, "T": wl2.T, "tokens_per_s": wl2.T * 10 / (ms2 * 1e-3),
+                     "ms_per_step": ms2 / 10, "stages_ms": st2,
+                     "roofline": roofline_entry(wl2, st2, t2, peaks, peak_kind, "prefill")}
+        del layer2
+        torch.cuda.empty_cache()
+
+    if rank == 0:
+        value = job_value(ws, wl.T, args.steps, ms)
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic: seeded N(0,1) activations, N(0,0.02) router/expert weights (bf16)",
+            "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "E": wl.E, "K": wl.K, "F": wl.F,
+                       "touched_experts": touched,
+                       "l2": "inputs larger than L2: the touched experts' weights "
+                             f"({touched * wl.F * wl.H * 4 / 1e9:.2f} GB) stream from HBM every step; "
+                             "4 token batches rotate; no flush",
+                       "parallelism": f"dp{ws} (independent token batches per GPU, weights replicated)"},
+            "roofline": roofline_entry(wl, stages, touched, peaks, peak_kind, args.workload),
+            "stages_ms": stages,
+            "e2e": {"value": job_value(ws, wl.T, args.steps, e2e_ms), "unit": UNIT,
+                    "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo},
+            "gpu_launches": 7 * args.steps,
+            "clocks": clocks,
+        }
+        if secondary:
+            line["secondary"] = secondary
+        if ws == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(wl, min(wl.T, 64))
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        dist.destroy_process_group()
+
+
+# --------------------------------------------------------------------------- reference arm
+
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return
+    from synth import workloads as W
+    wl = W.WORKLOADS[WORKLOADS[args.workload]]
+    n = min(wl.T, 16)
+    for _ in range(args.warmup):
+        cpu_baseline(wl, min(n, 4))
+    vals = []
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        vals.append(cpu_baseline(wl, n))
+    wall = time.perf_counter() - t0
+    value = statistics.mean(v["value"] for v in vals)
+    cb = dict(vals[-1])
+    cb["value"] = value
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * n / value,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic: seeded N(0,1) activations, N(0,0.02) router/expert weights (bf16)",
+            "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "E": wl.E, "K": wl.K, "F": wl.F,
+                       "sample_tokens_per_step": n},
+            "cpu_baseline": cb,
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "wall_s": wall}
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode")
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_native(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -159,6 +159,15 @@ moe_status moe_rmsnorm(int64_t T, int32_t H, float eps, const void* x, void* u, 
  * current device.  Returns MOE_OK, or the first error a kernel recorded. */
 moe_status moe_check_device_error(void* stream);
 
+/* Measurement hook.  With n == MOE_STAGE_EVENTS and `events` an array of n
+ * cudaEvent_t (as void*), every later moe_forward on this process records
+ * events[i] on its stream before stage i and events[n-1] after the last
+ * stage (stages: 0 router logits, 1 router top-K, 2 permute, 3 row gather,
+ * 4 up GEMM, 5 down GEMM, 6 combine), so a caller can time each kernel in
+ * place.  n == 0 turns it off.  Host state shared by all threads. */
+#define MOE_STAGE_EVENTS 8
+moe_status moe_set_stage_events(void* const* events, int32_t n);
+
 /* Test hooks of the failure-detection tests.  what = 1: limit of every
  * bounded wait in nanoseconds (value <= 0 restores the default of 4 s);
  * what = 2: the grouped-GEMM producer of block 0 withholds its first load

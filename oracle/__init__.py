@@ -62,6 +62,7 @@ def lib():
                                                       _p, _f, _f, _p]),
             "oracle_rmsnorm_bf16": (None, [_i64, _i64, _p, _f, _p]),
             "oracle_round_bf16": (None, [_i64, _p, _p]),
+            "oracle_hidden_amax_bf16": (ctypes.c_double, [_i64, _i64, _i64, _p, _p, _p, _p]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -270,3 +271,31 @@ def round_bf16(v) -> np.ndarray:
     out = np.empty(v.shape, dtype=np.uint16)
     lib().oracle_round_bf16(v.size, pv, out.ctypes.data)
     return out
+
+
+def hidden_amax_bf16(xrows, ex, wup, slot) -> float:
+    """Largest ReLU^2 activation of the bf16 model over the given rows (calibration)."""
+    xrows, px = _c(xrows, np.float64)
+    ex, pe = _c(ex, np.int32)
+    wup, pu = _c(wup, np.uint16)
+    slot, ps = _c(slot, np.int32)
+    R, H = xrows.shape
+    F = wup.shape[1]
+    a = lib().oracle_hidden_amax_bf16(R, H, F, px, pe, pu, ps)
+    if a < 0:
+        raise ValueError("a routed expert's bank was not supplied")
+    return float(a)
+
+
+def calibrate_fp8(x_cal, wr, bias, wup, K, slot=None):
+    """Static W8A8 activation scales from a calibration batch of the bf16 model:
+    x_scale = amax|x| / 448 and h_scale = amax(relu(z)^2) / 448, both fp32."""
+    x_cal = np.asarray(x_cal, dtype=np.uint16)
+    E = wr.shape[0]
+    if slot is None:
+        slot = identity_slot(E)
+    _, idx, _ = route(x_cal, wr, bias, K)
+    xf = bf16_to_f64(x_cal)
+    ax = np.float32(np.max(np.abs(xf)))
+    ah = hidden_amax_bf16(np.repeat(xf, K, axis=0), idx.reshape(-1), wup, slot)
+    return np.float32(ax / np.float32(448.0)), np.float32(np.float32(ah) / np.float32(448.0))

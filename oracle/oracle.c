@@ -361,3 +361,25 @@ void oracle_e4m3_encode_n(int64_t n, const float* v, uint8_t* q) {
 void oracle_e4m3_decode_n(int64_t n, const uint8_t* q, float* v) {
     for (int64_t i = 0; i < n; ++i) v[i] = oracle_e4m3_decode(q[i]);
 }
+
+/*
+ * Calibration of the static activation scale of the ReLU^2 tensor (the
+ * "scalar scale per activation tensor" of [B] s.2): the largest
+ * a_f = max(z_f, 0)^2 of the bf16 model over the given rows, in fp64.
+ */
+double oracle_hidden_amax_bf16(int64_t R, int64_t H, int64_t F, const double* xrow, const int32_t* ex,
+                               const uint16_t* wup, const int32_t* slot) {
+    double amax = 0.0;
+    for (int64_t r = 0; r < R; ++r) {
+        const int64_t s = slot[ex[r]];
+        if (s < 0) return -1.0;
+        const uint16_t* wu = wup + s * F * H;
+        for (int64_t f = 0; f < F; ++f) {
+            double z = 0.0;
+            for (int64_t h = 0; h < H; ++h) z += bf16_to_double(wu[f * H + h]) * xrow[r * H + h];
+            const double a = z > 0.0 ? z * z : 0.0;
+            if (a > amax) amax = a;
+        }
+    }
+    return amax;
+}

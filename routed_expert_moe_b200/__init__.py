@@ -52,6 +52,7 @@ _SIG = {
     "moe_quantize_fp8": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int64, _P, _P, _P, _P]),
     "moe_rmsnorm": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int32, ctypes.c_float, _P, _P, _P]),
     "moe_check_device_error": (ctypes.c_int, [_P]),
+    "moe_set_stage_events": (ctypes.c_int, [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32]),
     "moe_debug_set": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int64]),
 }
 for _name, (_res, _args) in _SIG.items():
@@ -164,6 +165,22 @@ def check_device_error(stream=None):
 
 def check_device_error_status(stream=None) -> int:
     return _lib.moe_check_device_error(_stream(stream))
+
+
+STAGE_EVENTS = 8
+STAGES = ("router_logits", "router_topk", "permute", "gather", "up_gemm", "down_gemm", "combine")
+
+
+def set_stage_events(events):
+    """events: a list of STAGE_EVENTS torch.cuda.Event(enable_timing=True), or None to stop."""
+    if not events:
+        _check(_lib.moe_set_stage_events(None, 0), "moe_set_stage_events")
+        return
+    for e in events:
+        if not e.cuda_event:      # torch creates the CUDA event on its first record
+            e.record()
+    arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    _check(_lib.moe_set_stage_events(arr, len(events)), "moe_set_stage_events")
 
 
 def debug_set(what: int, value: int):

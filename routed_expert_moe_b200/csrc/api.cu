@@ -20,7 +20,8 @@ struct RouterPlan {
 RouterPlan router_plan(int64_t T, int H, int E, int num_sms);
 cudaError_t launch_route(const uint16_t* x, const uint16_t* wr, const float* bias, int64_t T, int H, int E,
                          int K, int32_t* idx, float* w, double* P, double* xn2, double* wn2,
-                         const RouterPlan& plan, const DevCtx& ctx, cudaStream_t stream);
+                         const RouterPlan& plan, const DevCtx& ctx, cudaStream_t stream,
+                         void (*between)(cudaStream_t) = nullptr);
 cudaError_t launch_permute(const int32_t* idx, int64_t n, int E, int32_t* counts, int32_t* offsets,
                            int32_t* perm_src, int32_t* inv_row, int4* sched, int* n_sched, int bn,
                            const DevCtx& ctx, cudaStream_t stream);
@@ -61,6 +62,13 @@ namespace {
 constexpr uint64_t kDefaultTimeoutNs = 4000000000ull;
 std::atomic<uint64_t> g_timeout_ns{kDefaultTimeoutNs};
 std::atomic<int> g_debug_withhold{0};
+void* g_stage_events[MOE_STAGE_EVENTS] = {};
+std::atomic<int> g_stage_events_on{0};
+
+void stage_mark(int i, cudaStream_t st) {
+    if (g_stage_events_on.load()) cudaEventRecord(static_cast<cudaEvent_t>(g_stage_events[i]), st);
+}
+void mark_stage1(cudaStream_t st) { stage_mark(1, st); }
 
 struct DeviceInfo {
     bool ready = false;
@@ -205,17 +213,20 @@ size_t forward_ws_bytes(const moe_dims* d, int sms) {
 // Run the expert FFN given a schedule already in `fw`.
 moe_status run_ffn(const moe_dims* d, const DeviceInfo* dev, const DevCtx& ctx, const GemmPlan& gp,
                    const void* x, const int32_t* perm_src, const void* w_up, const void* w_down,
-                   const moe_fp8_scales* sc, FfnWs& fw, void* y_perm, cudaStream_t st) {
+                   const moe_fp8_scales* sc, FfnWs& fw, void* y_perm, cudaStream_t st, bool marks = false) {
     const bool fp8 = d->expert_dtype == MOE_FP8_E4M3;
     const int64_t rows = d->T * d->K;
+    if (marks) stage_mark(3, st);
     cudaError_t e = launch_gather(static_cast<const uint16_t*>(x), perm_src, rows, d->K, d->T, d->H, fw.xp, fp8,
                                   fp8 ? sc->x_scale : 1.0f, dev->num_sms, ctx, st);
     if (e != cudaSuccess) return cuda_status(e);
     const int withhold = g_debug_withhold.load();
+    if (marks) stage_mark(4, st);
     e = launch_grouped_gemm(fp8, true, w_up, d->E, d->F, d->H, fw.xp, rows, fw.sched, fw.n_sched, gp, fw.hb,
                             fp8 ? sc->w_up_scale : nullptr, fp8 ? sc->x_scale : 1.0f,
                             fp8 ? sc->h_scale : 1.0f, dev->num_sms, withhold, ctx, st);
     if (e != cudaSuccess) return cuda_status(e);
+    if (marks) stage_mark(5, st);
     e = launch_grouped_gemm(fp8, false, w_down, d->E, d->H, d->F, fw.hb, rows, fw.sched, fw.n_sched, gp, y_perm,
                             fp8 ? sc->w_down_scale : nullptr, fp8 ? sc->h_scale : 1.0f, 1.0f, dev->num_sms, 0,
                             ctx, st);
@@ -354,21 +365,27 @@ moe_status moe_forward(const moe_dims* d, const void* x, const void* w_router, c
     const RouterPlan rp = router_plan(d->T, d->H, d->E, dev->num_sms);
     Carve cr;
     RouteWs rw = carve_route(cr, sbase, d, rp);
+    stage_mark(0, st);
     cudaError_t e = launch_route(static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(w_router), bias, d->T,
-                                 d->H, d->E, d->K, idx, w, rw.P, rw.xn2, rw.wn2, rp, ctx, st);
+                                 d->H, d->E, d->K, idx, w, rw.P, rw.xn2, rw.wn2, rp, ctx, st,
+                                 g_stage_events_on.load() ? mark_stage1 : nullptr);
     if (e != cudaSuccess) return cuda_status(e);
 
     const GemmPlan gp = gemm_plan(d->T, d->K, d->E);
     Carve cf;
     FfnWs ffw = carve_ffn(cf, sbase, d, gp);   // reuses the router scratch region
+    stage_mark(2, st);
     e = launch_permute(idx, d->T * d->K, d->E, fw.counts, fw.offsets, fw.perm_src, fw.inv_row, ffw.sched,
                        ffw.n_sched, gp.bn, ctx, st);
     if (e != cudaSuccess) return cuda_status(e);
-    s = run_ffn(d, dev, ctx, gp, x, fw.perm_src, w_up, w_down, scales, ffw, fw.y_perm, st);
+    s = run_ffn(d, dev, ctx, gp, x, fw.perm_src, w_up, w_down, scales, ffw, fw.y_perm, st, true);
     if (s != MOE_OK) return s;
-    return cuda_status(launch_combine(static_cast<const uint16_t*>(fw.y_perm), fw.inv_row, w,
-                                      static_cast<const uint16_t*>(residual), static_cast<uint16_t*>(out), d->T,
-                                      d->K, d->H, dev->num_sms, ctx, st));
+    stage_mark(6, st);
+    e = launch_combine(static_cast<const uint16_t*>(fw.y_perm), fw.inv_row, w,
+                       static_cast<const uint16_t*>(residual), static_cast<uint16_t*>(out), d->T, d->K, d->H,
+                       dev->num_sms, ctx, st);
+    stage_mark(7, st);
+    return cuda_status(e);
 }
 
 moe_status moe_quantize_fp8(int64_t n_tensors, int64_t tensor_elems, const void* src, uint8_t* codes,
@@ -406,6 +423,20 @@ moe_status moe_check_device_error(void* stream) {
         if (cudaMemcpy(dev->err, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return MOE_ECUDA;
         return static_cast<moe_status>(v);
     }
+    return MOE_OK;
+}
+
+moe_status moe_set_stage_events(void* const* events, int32_t n) {
+    if (n == 0) {
+        g_stage_events_on.store(0);
+        return MOE_OK;
+    }
+    if (n != MOE_STAGE_EVENTS || !events) return MOE_EINVAL;
+    for (int i = 0; i < n; ++i) {
+        if (!events[i]) return MOE_EINVAL;
+        g_stage_events[i] = events[i];
+    }
+    g_stage_events_on.store(1);
     return MOE_OK;
 }
 

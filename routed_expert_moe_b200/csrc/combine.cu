@@ -33,13 +33,23 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
                 my_w = 0.0f;
             }
         }
+        // broadcast the K rows and weights before the (lane-divergent) vector loop
+        int row_k[16];
+        float w_k[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            row_k[k] = __shfl_sync(0xffffffffu, my_row, k);
+            w_k[k] = __shfl_sync(0xffffffffu, my_w, k);
+        }
         for (int v = lane; v < nv; v += 32) {
             float acc[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
-            for (int k = 0; k < K; ++k) {
-                const int r = __shfl_sync(0xffffffffu, my_row, k);
-                const float wk = __shfl_sync(0xffffffffu, my_w, k);
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                if (k >= K) break;
+                const int r = row_k[k];
+                const float wk = w_k[k];
                 const uint4 q = reinterpret_cast<const uint4*>(yp + (int64_t)r * H)[v];
                 const uint32_t qq[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll

@@ -392,7 +392,8 @@ RouterPlan router_plan(int64_t T, int H, int E, int num_sms) {
 
 cudaError_t launch_route(const uint16_t* x, const uint16_t* wr, const float* bias, int64_t T, int H,
                          int E, int K, int32_t* idx, float* w, double* P, double* xn2, double* wn2,
-                         const RouterPlan& plan, const DevCtx& ctx, cudaStream_t stream) {
+                         const RouterPlan& plan, const DevCtx& ctx, cudaStream_t stream,
+                         void (*between)(cudaStream_t)) {
     if (T == 0) return cudaSuccess;
     RouterLogitsArgs la{x, wr, T, H, E, plan.S, plan.nchunks, P, xn2, wn2};
     dim3 grid((unsigned)((T + RT_TT - 1) / RT_TT), (unsigned)((E + RT_TE - 1) / RT_TE),
@@ -400,6 +401,7 @@ cudaError_t launch_route(const uint16_t* x, const uint16_t* wr, const float* bia
     router_logits_kernel<<<grid, RT_THREADS, 0, stream>>>(la);
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return err;
+    if (between) between(stream);
     RouterTopkArgs ta{P, xn2, wn2, x, wr, bias, T, H, E, K, plan.S, idx, w};
     const unsigned blocks = (unsigned)((T + 7) / 8);
     router_topk_kernel<<<blocks, 256, 0, stream>>>(ta, ctx);

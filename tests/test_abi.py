@@ -1,0 +1,105 @@
+"""The C ABI without a GPU: the library loads, exports every function the
+header declares, and its host-side validation answers before any device
+call (no compute is attempted here)."""
+import ctypes
+import re
+import subprocess
+from pathlib import Path
+
+import pytest
+
+ROOT = Path(__file__).resolve().parents[1]
+HEADER = ROOT / "include" / "moe.h"
+
+
+def declared_functions():
+    text = re.sub(r"/\*.*?\*/", "", HEADER.read_text(), flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\**\s+\**(moe_\w+)\s*\(", text, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def moe():
+    import routed_expert_moe_b200 as m
+    return m
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward",
+                     "moe_workspace_size", "moe_check_device_error"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(moe):
+    lib = moe.raw_library()
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", str(moe._LIB_PATH)], capture_output=True,
+                         text=True).stdout
+    exported = set(re.findall(r"\s[TW]\s+(moe_\w+)$", out, flags=re.M))
+    assert set(declared_functions()) <= exported
+    assert set(moe.EXPORTS) == set(declared_functions())
+
+
+def test_status_strings_and_version(moe):
+    assert moe.abi_version() == 1
+    for s in range(8):
+        assert moe.status_string(s).startswith("MOE_")
+    assert "unknown" in moe.status_string(99)
+
+
+def bad(moe, **kw):
+    base = dict(T=64, H=2688, E=128, K=6, F=1856)
+    base.update(kw)
+    return moe.dims(**base)
+
+
+@pytest.mark.parametrize("kw", [dict(K=0), dict(K=17), dict(E=0), dict(E=257), dict(K=9, E=8),
+                                dict(H=2690), dict(F=8), dict(H=0), dict(T=-1),
+                                dict(T=2 ** 29, K=6)])
+def test_invalid_dims_are_rejected_on_the_host(moe, kw):
+    d = bad(moe, **kw)
+    n = ctypes.c_size_t()
+    assert moe.raw_library().moe_workspace_size(ctypes.byref(d), ctypes.byref(n)) == moe.MOE_EINVAL
+    assert moe.raw_library().moe_forward(ctypes.byref(d), *([None] * 11), 0, None) == moe.MOE_EINVAL
+
+
+def test_workspace_size_scales_with_tokens(moe):
+    small = moe.workspace_size(moe.dims(64, 2688, 128, 6, 1856))
+    big = moe.workspace_size(moe.dims(4096, 2688, 128, 6, 1856))
+    assert 0 < small < big
+    # X_perm, H and Y_perm of 24576 rows in bf16 dominate
+    assert big >= 24576 * (2688 * 2 * 2 + 1856 * 2)
+    fp8 = moe.workspace_size(moe.dims(4096, 2688, 128, 6, 1856, fp8=True))
+    assert fp8 < big
+
+
+def test_null_and_missing_arguments(moe):
+    lib = moe.raw_library()
+    d = bad(moe)
+    assert lib.moe_workspace_size(ctypes.byref(d), None) == moe.MOE_EINVAL
+    assert lib.moe_workspace_size(None, None) == moe.MOE_EINVAL
+    assert lib.moe_route(ctypes.byref(d), None, None, None, None, None, None, 0, None) == moe.MOE_EINVAL
+    assert lib.moe_permute(ctypes.byref(d), None, None, None, None, None, None, 0, None) == moe.MOE_EINVAL
+    fp8 = moe.dims(64, 2688, 128, 6, 1856, fp8=True)
+    assert lib.moe_expert_ffn(ctypes.byref(fp8), *([None] * 5), None, None, None, 0, None) == moe.MOE_EINVAL
+    assert lib.moe_rmsnorm(4, 2690, 1e-5, None, None, None) == moe.MOE_EINVAL
+    assert lib.moe_quantize_fp8(-1, 4, None, None, None, None) == moe.MOE_EINVAL
+    assert lib.moe_debug_set(99, 0) == moe.MOE_EINVAL
+    assert lib.moe_set_stage_events(None, 3) == moe.MOE_EINVAL
+
+
+def test_empty_batch_is_ok_without_a_device(moe):
+    lib = moe.raw_library()
+    d = bad(moe, T=0)
+    assert lib.moe_forward(ctypes.byref(d), *([None] * 11), 0, None) == moe.MOE_OK
+    assert lib.moe_rmsnorm(0, 2688, 1e-5, None, None, None) == moe.MOE_OK
+    assert lib.moe_quantize_fp8(0, 10, None, None, None, None) == moe.MOE_OK
+
+
+def test_package_has_no_cpu_path():
+    src = (ROOT / "routed_expert_moe_b200" / "__init__.py").read_text()
+    assert "oracle" not in src and "numpy" not in src
+    for f in (ROOT / "routed_expert_moe_b200").rglob("*"):
+        if f.suffix in (".py", ".cu", ".cuh", ".h"):
+            assert "import oracle" not in f.read_text()

@@ -153,7 +153,7 @@ def test_forward_hot_experts_split_into_token_blocks(moe):
     w = W.Workload("hot", 600, 512, 16, 3, 256, seed=15)
     h = inputs(w)
     bias = np.zeros(w.E, np.float32)
-    bias[[2, 9, 14]] = [40.0, 39.0, 38.0]
+    bias[[2, 9, 14]] = [60.0, 50.0, 40.0]   # gaps far above the logit spread
     d = device_inputs(h)
     dims = moe.dims(w.T, w.H, w.E, w.K, w.F)
     ws = moe.alloc_workspace(dims)
