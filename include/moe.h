@@ -155,6 +155,24 @@ moe_status moe_quantize_fp8(int64_t n_tensors, int64_t tensor_elems, const void*
  * "Q4_K, Q3_K and Q2_K expert profiles" (the model's normalisation). */
 moe_status moe_rmsnorm(int64_t T, int32_t H, float eps, const void* x, void* u, void* stream);
 
+/* The router (as moe_route) without a caller-provided workspace.  The paper
+ * has no counterpart: this entry point serves callers that cannot allocate
+ * device memory for a workspace, such as code inside a host framework whose
+ * pool allocator owns all device memory, or a decode loop that must not call
+ * cudaMalloc because it can synchronise the device.  Its scratch is one
+ * fixed 8 MiB array of device memory held by the library on every GPU that
+ * loads it, until the process exits.  It allocates nothing.
+ *   Limit: the partial logits of one split, T*E*8 bytes plus T*8 + E*8
+ *   (each rounded up to 256 bytes), must fit in 8 MiB; at E = 128 that is
+ *   T <= 8127.  Larger batches return MOE_EWORKSPACE before any launch.
+ *   The first call on a device looks up the array's device address (with
+ *   that device current) and should come before any stream capture.
+ *   All calls share the array; calls whose kernels overlap on the GPU race.
+ *   Nothing in it needs clearing between calls: each call writes all the
+ *   scratch it reads.  Same arguments and results as moe_route. */
+moe_status moe_route_static(const moe_dims* d, const void* x, const void* w_router, const float* bias,
+                            int32_t* topk_idx, float* topk_w, void* stream);
+
 /* Synchronises `stream`, then reads and clears the device error word of the
  * current device.  Returns MOE_OK, or the first error a kernel recorded. */
 moe_status moe_check_device_error(void* stream);

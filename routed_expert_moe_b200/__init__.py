@@ -43,6 +43,7 @@ _SIG = {
     "moe_abi_version": (ctypes.c_int, []),
     "moe_workspace_size": (ctypes.c_int, [_DIMS, ctypes.POINTER(ctypes.c_size_t)]),
     "moe_route": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P, _S, _P]),
+    "moe_route_static": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P]),
     "moe_permute": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P, _S, _P]),
     "moe_expert_ffn": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, ctypes.POINTER(MoeFp8Scales), _P, _P,
                                       _S, _P]),
@@ -118,6 +119,12 @@ def fp8_scales(w_up_scale, w_down_scale, x_scale: float, h_scale: float) -> MoeF
 def route(d, x, w_router, bias, topk_idx, topk_w, ws, stream=None):
     _check(_lib.moe_route(ctypes.byref(d), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(topk_idx), _ptr(topk_w),
                           _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)), "moe_route")
+
+
+def route_static(d, x, w_router, bias, topk_idx, topk_w, stream=None):
+    """The router with its scratch in the library's fixed device array (no workspace)."""
+    _check(_lib.moe_route_static(ctypes.byref(d), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(topk_idx),
+                                 _ptr(topk_w), _stream(stream)), "moe_route_static")
 
 
 def permute(d, topk_idx, counts, offsets, perm_src, inv_row, ws=None, stream=None):

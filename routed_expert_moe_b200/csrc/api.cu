@@ -242,6 +242,19 @@ moe_status check_fp8_scales(const moe_dims* d, const moe_fp8_scales* sc) {
 
 }  // namespace
 
+namespace moe {
+// Device context and argument checks for entry points defined in other files.
+moe_status internal_check_dims(const moe_dims* d) { return check_dims(d); }
+moe_status internal_device(DevCtx* ctx, int* num_sms) {
+    DeviceInfo* dev = nullptr;
+    const moe_status s = device_setup(&dev);
+    if (s != MOE_OK) return s;
+    *ctx = make_ctx(dev);
+    *num_sms = dev->num_sms;
+    return MOE_OK;
+}
+}  // namespace moe
+
 extern "C" {
 
 const char* moe_status_string(moe_status s) {
