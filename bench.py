@@ -35,7 +35,7 @@ METRIC = "MoE-layer tokens/s on 1 B200; % of HBM roofline (decode), % TC peak (p
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-WORKLOADS = {"tiny": 0, "decode": 1, "prefill": 2, "skewed": 3}
+WORKLOADS = {"tiny": 0, "decode": 1, "prefill": 2, "skewed": 3, "chain": 4}
 
 
 def load_peaks():
@@ -185,17 +185,67 @@ class Layer:
         return int(torch.unique(self.idx).numel()), int(self.idx.numel())
 
 
+class Chain:
+    """The 23-layer W8A8 stack of the chain workload, weights made and quantised on the device."""
+
+    def __init__(self, wl, device):
+        import torch
+        import synth
+        import routed_expert_moe_b200 as moe
+        from routed_expert_moe_b200.stack import MoeStack
+        from synth import workloads as W
+
+        self.wl = wl
+        self.moe = moe
+        self.device = device
+        stream = torch.cuda.current_stream().cuda_stream
+        self.stack = MoeStack(wl.T, wl.H, wl.E, wl.K, wl.F, fp8=True, device=device)
+        wu = torch.empty(wl.E, wl.F, wl.H, dtype=torch.bfloat16, device=device)
+        wd = torch.empty(wl.E, wl.H, wl.F, dtype=torch.bfloat16, device=device)
+        for l, (sx, sh) in enumerate(W.chain_scales()[:wl.layers]):
+            wr = torch.empty(wl.E, wl.H, dtype=torch.bfloat16, device=device)
+            synth.normal_bf16_device(synth.key(wl.seed, synth.T_WR, l), wr.numel(), W.SIGMA_W, wr.data_ptr(), stream)
+            synth.normal_bf16_device(synth.key(wl.seed, synth.T_WUP, l), wu.numel(), W.SIGMA_W, wu.data_ptr(), stream)
+            synth.normal_bf16_device(synth.key(wl.seed, synth.T_WDOWN, l), wd.numel(), W.SIGMA_W, wd.data_ptr(),
+                                     stream)
+            self.stack.add_layer(wr, wu, wd, float(sx), float(sh))
+        del wu, wd
+        self.xs = []
+        for i in range(2):
+            x = torch.empty(wl.T, wl.H, dtype=torch.bfloat16, device=device)
+            synth.normal_bf16_device(synth.key(wl.seed, synth.T_X, i), x.numel(), W.SIGMA_X, x.data_ptr(), stream)
+            self.xs.append(x)
+        self.out = self.xs[0]
+        self.idx = torch.empty(wl.T, wl.K, dtype=torch.int32, device=device)
+        torch.cuda.synchronize(device)
+
+    def step(self, i, x=None, out=None):
+        y = self.stack.forward(self.xs[i % len(self.xs)] if x is None else x)
+        self.out = y if out is None else out.copy_(y)
+
+    def profile_layer(self, i):
+        """one pass of layer 0, for the stage events"""
+        self.stack.run_layer(0, self.xs[0], self.stack.x[1], topk_idx=self.idx)
+
+    def touched_experts(self, i):
+        import torch
+        self.profile_layer(0)
+        torch.cuda.synchronize()
+        return int(torch.unique(self.idx).numel()), int(self.idx.numel())
+
+
 def stage_profile(layer, steps, warmup):
     """Per-stage device time (ms, mean over steps) from the library's stage events."""
     import torch
     moe = layer.moe
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(moe.STAGE_EVENTS)] for _ in range(steps)]
+    one = layer.profile_layer if hasattr(layer, "profile_layer") else layer.step
     for i in range(warmup):
-        layer.step(i)
+        one(i)
     times = [[0.0] * (moe.STAGE_EVENTS - 1) for _ in range(steps)]
     for i in range(steps):
         moe.set_stage_events(ev[i])
-        layer.step(i)
+        one(i)
     moe.set_stage_events(None)
     torch.cuda.synchronize()
     for i in range(steps):
@@ -271,35 +321,60 @@ def traffic_from_profile(kernel: str, workload: str):
 
 
 def roofline_entry(wl, stages, touched, peaks, peak_kind, workload):
-    """Roofline of the dominant kernel of the step (an expert GEMM)."""
+    """Roofline of the dominant kernel of the step (an expert GEMM).
+
+    Decode is declared HBM-bound (a weight stream); prefill and the FP8 chain
+    are reported against the dense tensor peak of their dtype, as the metric
+    asks, with the HBM fraction of the same launch beside it.
+    """
     H, F, T, K = wl.H, wl.F, wl.T, wl.K
     rows = T * K
+    es = 1 if wl.fp8 else 2
     up_ms, down_ms = stages["up_gemm"], stages["down_gemm"]
     kernel = "up_gemm" if up_ms >= down_ms else "down_gemm"
     ms = max(up_ms, down_ms)
     flops = 2.0 * rows * F * H
-    if workload == "prefill":
-        peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-        achieved = flops / (ms * 1e-3) / 1e12
-        return {"kernel": kernel, "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "peak_source": f"{peak_kind} bf16 sustained",
-                "algorithmic_flops_per_launch": flops, "ms_per_launch": ms,
-                "traffic": traffic_from_profile(kernel, workload)}
-    wbytes = touched * F * H * 2
-    act = rows * H * 2 + rows * F * 2            # X_perm read + Hb write (up); Hb read + Y write (down)
-    if kernel == "down_gemm":
-        act = rows * F * 2 + rows * H * 2
-    algo = wbytes + act
-    peak = peaks["hbm_gbs"]
-    achieved = algo / (ms * 1e-3) / 1e9
-    return {"kernel": kernel, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-            "frac": achieved / peak, "peak_source": f"{peak_kind} hbm copy",
-            "algorithmic_bytes_per_launch": algo, "ms_per_launch": ms,
-            "traffic": traffic_from_profile(kernel, workload)}
+    # weights of the touched experts + activations in (es bytes) + activations out
+    if kernel == "up_gemm":
+        algo = touched * F * H * es + rows * H * es + rows * F * es
+    else:
+        algo = touched * F * H * es + rows * F * es + rows * H * 2
+    hbm_peak = peaks["hbm_gbs"]
+    gbs = algo / (ms * 1e-3) / 1e9
+    bf16_sust = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    tc_peak = bf16_sust * (2.0 if wl.fp8 else 1.0)   # fp8 dense = 2x bf16 dense (nominal ratio)
+    tflops = flops / (ms * 1e-3) / 1e12
+    common = {"kernel": kernel, "ms_per_launch": ms, "algorithmic_bytes_per_launch": algo,
+              "algorithmic_flops_per_launch": flops, "traffic": traffic_from_profile(kernel, workload),
+              "hbm_gbs": gbs, "hbm_frac": gbs / hbm_peak, "tensor_tflops": tflops, "tensor_frac": tflops / tc_peak}
+    if workload in ("prefill", "chain"):
+        src = f"{peak_kind} bf16 sustained" + (" x 2 (fp8/bf16 nominal ratio)" if wl.fp8 else "")
+        return dict(bound="tensor", achieved=tflops, peak=tc_peak, unit="TFLOP/s", frac=tflops / tc_peak,
+                    peak_source=src, **common)
+    return dict(bound="hbm", achieved=gbs, peak=hbm_peak, unit="GB/s", frac=gbs / hbm_peak,
+                peak_source=f"{peak_kind} hbm copy", **common)
+
+
+_BANKS = {}
+
+
+def _host_banks(wl, layer, used, fp8):
+    """Host weight banks of the used experts (input preparation, cached, never timed)."""
+    import oracle
+    from synth import workloads as W
+    key = (wl.name, layer, tuple(used), fp8)
+    if key not in _BANKS:
+        wu = W.host_w_up(wl, layer, experts=used)
+        wd = W.host_w_down(wl, layer, experts=used)
+        _BANKS.clear()
+        _BANKS[key] = (oracle.quantize_bank_fp8(wu), oracle.quantize_bank_fp8(wd)) if fp8 else (wu, wd)
+    return _BANKS[key]
 
 
 def cpu_baseline(wl, n_tokens, seed_batch=0):
     """The oracle as it stands, on the host cores, over a bounded sample of the workload."""
+    if wl.fp8:
+        return cpu_baseline_fp8(wl, n_tokens, seed_batch)
     import oracle
     from synth import workloads as W
     x = W.host_x(wl, seed_batch)[:n_tokens]
@@ -310,8 +385,7 @@ def cpu_baseline(wl, n_tokens, seed_batch=0):
     slot = -__import__("numpy").ones(wl.E, dtype="int32")
     slot[used] = range(len(used))
     t_route = time.perf_counter() - t0
-    wu = W.host_w_up(wl, experts=used)       # generating inputs is not timed
-    wd = W.host_w_down(wl, experts=used)
+    wu, wd = _host_banks(wl, 0, used, False)   # generating inputs is not timed
     t0 = time.perf_counter()
     oracle.moe_layer_bf16(x, wr, W.host_bias(wl), wu, wd, wl.K, slot=slot)
     dt = time.perf_counter() - t0 + t_route
@@ -320,6 +394,32 @@ def cpu_baseline(wl, n_tokens, seed_batch=0):
             "sample": f"{n_tokens} of the {wl.T} tokens of batch {seed_batch} ({wl.name}), full layer "
                       f"(router, top-{wl.K}, {len(used)} experts' up/ReLU^2/down in fp64, combine); "
                       f"{dt:.2f} s"}
+
+
+def cpu_baseline_fp8(wl, n_tokens, seed_batch=0, layer=0):
+    """The oracle's W8A8 layer (norm, router, quantised experts, combine + residual) on a token sample."""
+    import numpy as np
+    import oracle
+    import synth
+    from synth import workloads as W
+    x = synth.normal_bf16(synth.key(wl.seed, synth.T_X, seed_batch), n_tokens * wl.H, W.SIGMA_X).reshape(
+        n_tokens, wl.H)
+    wr = W.host_router(wl, layer)
+    sx, sh = W.chain_scales()[layer]
+    u = oracle.rmsnorm_bf16(x)
+    _, idx, _ = oracle.route(u, wr, None, wl.K)
+    used = sorted(set(idx.reshape(-1).tolist()))
+    slot = -np.ones(wl.E, dtype=np.int32)
+    slot[used] = np.arange(len(used))
+    (qu, su), (qd, sd) = _host_banks(wl, layer, used, True)   # weight preparation: untimed
+    t0 = time.perf_counter()
+    u = oracle.rmsnorm_bf16(x)
+    oracle.moe_layer_fp8(u, wr, None, qu, su, qd, sd, sx, sh, wl.K, slot=slot, residual=x)
+    dt = time.perf_counter() - t0
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return {"value": n_tokens / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{n_tokens} tokens through layer {layer} of {wl.name} (norm, router, {len(used)} W8A8 "
+                      f"experts in fp64 on dequantised codes, combine + residual); {dt:.2f} s"}
 
 
 def run_native(args):
@@ -338,7 +438,7 @@ def run_native(args):
     peaks, peak_kind = load_peaks()
 
     wl = W.WORKLOADS[WORKLOADS[args.workload]]
-    layer = Layer(wl, device)
+    layer = Chain(wl, device) if wl.layers > 1 else Layer(wl, device)
     touched, rows = layer.touched_experts(0)
     stages = stage_profile(layer, max(3, min(args.steps, 20)), args.warmup)
 
@@ -373,29 +473,31 @@ def run_native(args):
         torch.cuda.empty_cache()
 
     if rank == 0:
-        value = job_value(ws, wl.T, args.steps, ms)
+        # MoE-layer tokens: a step of the chain passes T tokens through every layer
+        value = job_value(ws, wl.T * wl.layers, args.steps, ms)
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "fp8_e4m3 (W8A8) experts, bf16 router" if wl.fp8 else "bf16",
             "data": "synthetic: seeded N(0,1) activations, N(0,0.02) router/expert weights (bf16)",
             "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "E": wl.E, "K": wl.K, "F": wl.F,
-                       "touched_experts": touched,
+                       "layers": wl.layers, "touched_experts": touched,
                        "l2": "inputs larger than L2: the touched experts' weights "
-                             f"({touched * wl.F * wl.H * 4 / 1e9:.2f} GB) stream from HBM every step; "
-                             "4 token batches rotate; no flush",
+                             f"({touched * wl.F * wl.H * (2 if wl.fp8 else 4) * wl.layers / 1e9:.2f} GB) "
+                             "stream from HBM every step; token batches rotate; no flush",
                        "parallelism": f"dp{ws} (independent token batches per GPU, weights replicated)"},
             "roofline": roofline_entry(wl, stages, touched, peaks, peak_kind, args.workload),
             "stages_ms": stages,
-            "e2e": {"value": job_value(ws, wl.T, args.steps, e2e_ms), "unit": UNIT,
+            "e2e": {"value": job_value(ws, wl.T * wl.layers, args.steps, e2e_ms), "unit": UNIT,
                     "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo},
-            "gpu_launches": 7 * args.steps,
+            "gpu_launches": (8 * wl.layers if wl.layers > 1 else 7) * args.steps,
             "clocks": clocks,
         }
         if secondary:
             line["secondary"] = secondary
         if ws == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(wl, min(wl.T, 64))
+            line["cpu_baseline"] = cpu_baseline(wl, 4 if wl.fp8 else min(wl.T, 64))
         print(json.dumps(line), flush=True)
     if ws > 1:
         dist.destroy_process_group()
@@ -409,7 +511,7 @@ def run_reference(args):
         return
     from synth import workloads as W
     wl = W.WORKLOADS[WORKLOADS[args.workload]]
-    n = min(wl.T, 16)
+    n = 4 if wl.fp8 else min(wl.T, 16)
     for _ in range(args.warmup):
         cpu_baseline(wl, min(n, 4))
     vals = []

@@ -106,6 +106,8 @@ moe_status moe_route(const moe_dims* d, const void* x, const void* w_router, con
  *   topk_idx [T][K] int32 in; counts [E], offsets [E+1] (exclusive scan),
  *   perm_src [T*K] (row r of the grouped layout holds assignment perm_src[r]),
  *   inv_row  [T*K] (assignment i sits in row inv_row[i]) out.
+ * ws: scratch of at least moe_workspace_size() bytes; it may be NULL (with
+ * ws_bytes 0) when T*K <= 4096.
  * An index outside [0, E) sets MOE_EINDEX in the device error word; the
  * outputs are then unspecified.  Cited: audio.cpp model page, "CPU weight
  * offload" (grouped expert matrix multiplication). */

@@ -248,11 +248,13 @@ float oracle_e4m3_decode(uint8_t q) {
  */
 float oracle_quantize_tensor_fp8(int64_t n, const uint16_t* w, uint8_t* q) {
     float amax = 0.0f;
+#pragma omp parallel for reduction(max : amax) schedule(static)
     for (int64_t i = 0; i < n; ++i) {
         float a = fabsf(bf16_to_float(w[i]));
         if (a > amax) amax = a;
     }
     float s = amax > 0.0f ? amax / 448.0f : 1.0f;
+#pragma omp parallel for schedule(static)
     for (int64_t i = 0; i < n; ++i) {
         float t = bf16_to_float(w[i]) / s;
         q[i] = oracle_e4m3_encode(t);
@@ -262,6 +264,7 @@ float oracle_quantize_tensor_fp8(int64_t n, const uint16_t* w, uint8_t* q) {
 
 /* Activation quantisation with a given static scale: q = e4m3(fl32(x / s)). */
 void oracle_quantize_act_fp8(int64_t n, const uint16_t* x, float s, uint8_t* q) {
+#pragma omp parallel for schedule(static)
     for (int64_t i = 0; i < n; ++i) q[i] = oracle_e4m3_encode(bf16_to_float(x[i]) / s);
 }
 
@@ -315,6 +318,7 @@ int oracle_expert_rows_fp8(int64_t R, int64_t H, int64_t F, const uint8_t* qxrow
  * fp32, rounded to the grid 2^-16, summed exactly), and u rounded to bf16.
  */
 void oracle_rmsnorm_bf16(int64_t T, int64_t H, const uint16_t* x, float eps, uint16_t* u) {
+#pragma omp parallel for schedule(static)
     for (int64_t t = 0; t < T; ++t) {
         int64_t acc = 0;
         for (int64_t h = 0; h < H; ++h) {

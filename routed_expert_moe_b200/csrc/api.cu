@@ -24,7 +24,8 @@ cudaError_t launch_route(const uint16_t* x, const uint16_t* wr, const float* bia
                          void (*between)(cudaStream_t) = nullptr);
 cudaError_t launch_permute(const int32_t* idx, int64_t n, int E, int32_t* counts, int32_t* offsets,
                            int32_t* perm_src, int32_t* inv_row, int4* sched, int* n_sched, int bn,
-                           const DevCtx& ctx, cudaStream_t stream);
+                           int* scratch, const DevCtx& ctx, cudaStream_t stream);
+size_t permute_scratch_ints(int64_t n, int E);
 size_t permute_smem_bytes(int E);
 cudaError_t launch_schedule(const int32_t* offsets, int E, int bn, int4* sched, int* n_sched,
                             cudaStream_t stream);
@@ -144,6 +145,7 @@ struct RouteWs {
 struct FfnWs {
     int4* sched;
     int* n_sched;
+    int* perm_scratch;
     void* xp;
     void* hb;
 };
@@ -171,6 +173,7 @@ FfnWs carve_ffn(Carve& c, void* base, const moe_dims* d, const GemmPlan& gp) {
     const size_t es = d->expert_dtype == MOE_FP8_E4M3 ? 1 : 2;
     f.sched = c.take<int4>(base, (size_t)gp.max_sched);
     f.n_sched = c.take<int>(base, 1);
+    f.perm_scratch = c.take<int>(base, permute_scratch_ints(d->T * d->K, d->E));
     f.xp = c.take<uint8_t>(base, rows * d->H * es);
     f.hb = c.take<uint8_t>(base, rows * d->F * es);
     return f;
@@ -217,14 +220,15 @@ moe_status run_ffn(const moe_dims* d, const DeviceInfo* dev, const DevCtx& ctx, 
     const bool fp8 = d->expert_dtype == MOE_FP8_E4M3;
     const int64_t rows = d->T * d->K;
     if (marks) stage_mark(3, st);
+    // permuted copy of x (or of its E4M3 codes), read by the up projection in contiguous row blocks
     cudaError_t e = launch_gather(static_cast<const uint16_t*>(x), perm_src, rows, d->K, d->T, d->H, fw.xp, fp8,
                                   fp8 ? sc->x_scale : 1.0f, dev->num_sms, ctx, st);
     if (e != cudaSuccess) return cuda_status(e);
     const int withhold = g_debug_withhold.load();
     if (marks) stage_mark(4, st);
     e = launch_grouped_gemm(fp8, true, w_up, d->E, d->F, d->H, fw.xp, rows, fw.sched, fw.n_sched, gp, fw.hb,
-                            fp8 ? sc->w_up_scale : nullptr, fp8 ? sc->x_scale : 1.0f,
-                            fp8 ? sc->h_scale : 1.0f, dev->num_sms, withhold, ctx, st);
+                            fp8 ? sc->w_up_scale : nullptr, fp8 ? sc->x_scale : 1.0f, fp8 ? sc->h_scale : 1.0f,
+                            dev->num_sms, withhold, ctx, st);
     if (e != cudaSuccess) return cuda_status(e);
     if (marks) stage_mark(5, st);
     e = launch_grouped_gemm(fp8, false, w_down, d->E, d->H, d->F, fw.hb, rows, fw.sched, fw.n_sched, gp, y_perm,
@@ -303,16 +307,18 @@ moe_status moe_route(const moe_dims* d, const void* x, const void* w_router, con
 
 moe_status moe_permute(const moe_dims* d, const int32_t* topk_idx, int32_t* counts, int32_t* offsets,
                        int32_t* perm_src, int32_t* inv_row, void* ws, size_t ws_bytes, void* stream) {
-    (void)ws;
-    (void)ws_bytes;
     moe_status s = check_dims(d);
     if (s != MOE_OK) return s;
     if (!counts || !offsets) return MOE_EINVAL;
     if (d->T > 0 && (!topk_idx || !perm_src || !inv_row)) return MOE_EINVAL;
+    const size_t need = permute_scratch_ints(d->T * d->K, d->E) * sizeof(int);
+    if (need > 0 && (!ws || ws_bytes < need)) return MOE_EWORKSPACE;
+    if (!aligned(ws, 256)) return MOE_EINVAL;
     DeviceInfo* dev = nullptr;
     if ((s = device_setup(&dev)) != MOE_OK) return s;
     return cuda_status(launch_permute(topk_idx, d->T * d->K, d->E, counts, offsets, perm_src, inv_row, nullptr,
-                                      nullptr, 16, make_ctx(dev), static_cast<cudaStream_t>(stream)));
+                                      nullptr, 16, static_cast<int*>(ws), make_ctx(dev),
+                                      static_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_expert_ffn(const moe_dims* d, const void* x, const int32_t* offsets, const int32_t* perm_src,
@@ -389,7 +395,7 @@ moe_status moe_forward(const moe_dims* d, const void* x, const void* w_router, c
     FfnWs ffw = carve_ffn(cf, sbase, d, gp);   // reuses the router scratch region
     stage_mark(2, st);
     e = launch_permute(idx, d->T * d->K, d->E, fw.counts, fw.offsets, fw.perm_src, fw.inv_row, ffw.sched,
-                       ffw.n_sched, gp.bn, ctx, st);
+                       ffw.n_sched, gp.bn, ffw.perm_scratch, ctx, st);
     if (e != cudaSuccess) return cuda_status(e);
     s = run_ffn(d, dev, ctx, gp, x, fw.perm_src, w_up, w_down, scales, ffw, fw.y_perm, st, true);
     if (s != MOE_OK) return s;

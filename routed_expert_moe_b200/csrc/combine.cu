@@ -12,46 +12,46 @@ namespace moe {
 
 // out[t] = (residual[t] +) sum_{k=0..K-1} w[t][k] * y_perm[inv_row[t*K+k]]
 // in fp32, k ascending (descending routing logit), one rounding to bf16.
-__global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict__ yp,
-                                                      const int32_t* __restrict__ inv_row,
-                                                      const float* __restrict__ w,
-                                                      const uint16_t* residual, uint16_t* out,
-                                                      int64_t T, int K, int H, int64_t rows,
-                                                      DevCtx ctx) {
-    const int lane = threadIdx.x % 32;
-    const int64_t warps = (int64_t)gridDim.x * (blockDim.x / 32);
+// One block per token (grid-stride over tokens): the K row indices and
+// weights are staged in shared memory, then every thread streams 16-byte
+// vectors of the K rows; a token's H/8 vectors are all in flight at once.
+constexpr int CB_THREADS = 128;
+
+__global__ void __launch_bounds__(CB_THREADS) combine_kernel(const uint16_t* __restrict__ yp,
+                                                             const int32_t* __restrict__ inv_row,
+                                                             const float* __restrict__ w,
+                                                             const uint16_t* residual, uint16_t* out,
+                                                             int64_t T, int K, int H, int64_t rows,
+                                                             DevCtx ctx) {
+    __shared__ int row_k[16];
+    __shared__ float w_k[16];
     const int nv = H / 8;
-    for (int64_t t = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32; t < T; t += warps) {
-        int my_row = 0;
-        float my_w = 0.0f;
-        if (lane < K) {
-            my_row = inv_row[t * K + lane];
-            my_w = w[t * K + lane];
-            if (my_row < 0 || my_row >= rows) {
+    for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+        if (threadIdx.x < K) {
+            int r = inv_row[t * K + threadIdx.x];
+            float wk = w[t * K + threadIdx.x];
+            if (r < 0 || r >= rows) {
                 record_error(ctx.err, MOE_EINDEX);
-                my_row = 0;
-                my_w = 0.0f;
+                r = 0;
+                wk = 0.0f;
             }
+            row_k[threadIdx.x] = r;
+            w_k[threadIdx.x] = wk;
         }
-        // broadcast the K rows and weights before the (lane-divergent) vector loop
-        int row_k[16];
-        float w_k[16];
+        __syncthreads();
+        for (int v = threadIdx.x; v < nv; v += CB_THREADS) {
+            uint4 q[16];
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            row_k[k] = __shfl_sync(0xffffffffu, my_row, k);
-            w_k[k] = __shfl_sync(0xffffffffu, my_w, k);
-        }
-        for (int v = lane; v < nv; v += 32) {
+            for (int k = 0; k < 16; ++k)
+                if (k < K) q[k] = reinterpret_cast<const uint4*>(yp + (int64_t)row_k[k] * H)[v];
             float acc[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
                 if (k >= K) break;
-                const int r = row_k[k];
                 const float wk = w_k[k];
-                const uint4 q = reinterpret_cast<const uint4*>(yp + (int64_t)r * H)[v];
-                const uint32_t qq[4] = {q.x, q.y, q.z, q.w};
+                const uint32_t qq[4] = {q[k].x, q[k].y, q[k].z, q[k].w};
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     acc[2 * j] = __fmaf_rn(wk, __uint_as_float(qq[j] << 16), acc[2 * j]);
@@ -59,8 +59,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
                 }
             }
             if (residual) {
-                const uint4 q = reinterpret_cast<const uint4*>(residual + t * H)[v];
-                const uint32_t qq[4] = {q.x, q.y, q.z, q.w};
+                const uint4 r4 = reinterpret_cast<const uint4*>(residual + t * H)[v];
+                const uint32_t qq[4] = {r4.x, r4.y, r4.z, r4.w};
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     acc[2 * j] = __fadd_rn(__uint_as_float(qq[j] << 16), acc[2 * j]);
@@ -76,6 +76,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
             }
             reinterpret_cast<uint4*>(out + t * H)[v] = make_uint4(o[0], o[1], o[2], o[3]);
         }
+        __syncthreads();
     }
 }
 
@@ -176,8 +177,9 @@ cudaError_t launch_combine(const uint16_t* yp, const int32_t* inv_row, const flo
                            const uint16_t* residual, uint16_t* out, int64_t T, int K, int H,
                            int num_sms, const DevCtx& ctx, cudaStream_t stream) {
     if (T == 0) return cudaSuccess;
-    combine_kernel<<<grid_rows(T, num_sms), 256, 0, stream>>>(yp, inv_row, w, residual, out, T, K, H,
-                                                              T * K, ctx);
+    const int64_t cap = (int64_t)num_sms * 16;
+    const unsigned grid = (unsigned)(T < cap ? T : cap);
+    combine_kernel<<<grid, CB_THREADS, 0, stream>>>(yp, inv_row, w, residual, out, T, K, H, T * K, ctx);
     return cudaGetLastError();
 }
 

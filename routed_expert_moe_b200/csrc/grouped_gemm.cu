@@ -3,23 +3,27 @@
 // The two expert projections (bloomery issue page, s.2 "Checkpoint facts":
 // ungated ReLU^2 experts, width 1856; s.3: ungated up/down parts) are, for
 // every expert e and the rows r of its segment in the permuted layout,
-//   up:    Hb[r, f] = relu( sum_h W_up[e][f][h] * X_perm[r][h] )^2
-//   down:  Y [r, j] =       sum_f W_down[e][j][f] * Hb[r][f]
-// Both are computed "swap-AB": the weight rows of one 128-row block of W[e]
-// are the MMA's M side (TMEM lanes), the expert's tokens are its N side
-// (16..256 TMEM columns).  A decode batch has a handful of tokens per expert,
-// so the kernel is a weight stream that the tensor cores consume at N = 16;
-// a prefill chunk has ~192 tokens per expert, so every weight tile is read
-// from HBM once and used for all of them.
+//   up:    H[r, f] = relu( sum_h W_up[e][f][h] * X_perm[r][h] )^2
+//   down:  Y[r, j] =       sum_f W_down[e][j][f] * H[r][f]
+// with X_perm[r] = x[perm_src[r] / K].  Both are computed "swap-AB": a block of
+// 128 weight rows of W[e] is the MMA's M side (TMEM lanes) and the expert's
+// tokens are its N side (16..256 TMEM columns).  A decode batch has a few
+// tokens per expert, so the kernel is a weight stream that the tensor cores
+// consume at N = 16; a prefill chunk has ~192 tokens per expert, so every
+// weight tile is read from HBM once and used for all of them.
 //
-// Work unit = (schedule entry s = {e, row0, nrows}, weight row block mb).
+// Work unit = (schedule entry {e, row0, nrows}, one 128-row weight block).
 // Persistent CTAs (one per SM) walk units u = blockIdx.x + i * gridDim.x.
 // Roles (192 threads):
-//   warp 0      TMA producer: per K stage one 128x128-byte weight tile (as
-//               64-row boxes) and ceil(nrows/16) 16x128-byte activation boxes,
-//               both in the 128-byte swizzle, into an NS-deep smem ring;
-//   warp 1      TMEM allocator; lane 0 issues tcgen05.mma (4 per stage, K=16
-//               bf16 or K=32 e4m3) into one of two TMEM accumulators;
+//   warp 0      TMA producer (one thread): per 128-byte K slice the weight
+//               tile (one 128-row box, or a 64-row box for the last block of
+//               a 1856-row expert) and the expert's rows (64-row boxes, then
+//               16-row boxes for the remainder), both in the 128-byte swizzle,
+//               into an NS-deep smem ring.  Few, large copies per stage: the
+//               copy engine's per-request cost, not bytes, is what limits a
+//               ring of many small boxes;
+//   warp 1      TMEM allocator; lane 0 issues tcgen05.mma (K = 16 bf16 or
+//               32 e4m3 per instruction) into one of two TMEM accumulators;
 //   warps 2..5  epilogue: tcgen05.ld, scale, ReLU^2 (up) and stores; warp w
 //               reads TMEM lanes 32*(w%4) .. +31.
 // Every wait is bounded; on expiry the block records MOE_ETIMEOUT, drains what
@@ -56,10 +60,17 @@ struct GemmArgs {
     int debug_withhold;      // 1: block 0 withholds its first load
 };
 
+struct GemmMaps {
+    CUtensorMap a128;        // weights, 128-row box
+    CUtensorMap a64;         // weights, 64-row box
+    CUtensorMap b64;         // activations, 64-row box
+    CUtensorMap b16;         // activations, 16-row box
+};
+
 template <bool FP8, bool UP>
 __global__ void __launch_bounds__(GG_THREADS, 1)
-    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                        GemmArgs g, DevCtx ctx) {
+    grouped_gemm_kernel(const __grid_constant__ GemmMaps maps, GemmArgs g, DevCtx ctx) {
+    constexpr int KEL = GG_ROW_BYTES / (FP8 ? 1 : 2);   // elements of K per stage
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
@@ -89,8 +100,10 @@ __global__ void __launch_bounds__(GG_THREADS, 1)
         mbar_init(smem_u32(drain), 1);
         *abort_flag = 0;
         fence_mbar_init();
-        tma_prefetch_desc(&tmA);
-        tma_prefetch_desc(&tmB);
+        tma_prefetch_desc(&maps.a128);
+        tma_prefetch_desc(&maps.a64);
+        tma_prefetch_desc(&maps.b64);
+        tma_prefetch_desc(&maps.b16);
     }
     if (warp == 1) tmem_alloc(smem_u32(tmem_holder), GG_TMEM_COLS);
     tc_fence_before();
@@ -111,10 +124,10 @@ __global__ void __launch_bounds__(GG_THREADS, 1)
             for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
                 const int4 sc = g.sched[u / g.m_blocks];
                 const int mb = u % g.m_blocks;
-                const int a_valid = min(GG_BM, g.Nout - mb * GG_BM);
-                const int a_boxes = (a_valid + 63) / 64;
-                const int b_boxes = (sc.z + 15) / 16;
-                const uint32_t bytes = (uint32_t)(a_boxes * 64 * GG_ROW_BYTES + b_boxes * 16 * GG_ROW_BYTES);
+                const bool a_full = g.Nout - mb * GG_BM > 64;
+                const int n16 = (sc.z + 15) / 16;         // 16-row groups of activations
+                const int n64 = n16 / 4, r16 = n16 % 4;
+                const uint32_t bytes = (uint32_t)((a_full ? 128 : 64) * GG_ROW_BYTES + n16 * 16 * GG_ROW_BYTES);
                 const int a_y = sc.x * g.Nout + mb * GG_BM;
                 for (int ks = 0; ks < g.k_stages; ++ks) {
                     if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, ctx, abort_flag)) {
@@ -126,13 +139,15 @@ __global__ void __launch_bounds__(GG_THREADS, 1)
                     if (withhold) {
                         withhold = false;   // this stage never completes: the consumer's wait expires
                     } else {
-                        const int kx = ks * (FP8 ? 128 : 64);
+                        const int kx = ks * KEL;
                         const uint32_t a_dst = smem_u32(smA + (size_t)stage * GG_A_BYTES);
                         const uint32_t b_dst = smem_u32(smB + (size_t)stage * g.b_stage_bytes);
-                        for (int i = 0; i < a_boxes; ++i)
-                            tma_load_2d(a_dst + i * 64 * GG_ROW_BYTES, &tmA, fb, kx, a_y + i * 64, pol_w);
-                        for (int j = 0; j < b_boxes; ++j)
-                            tma_load_2d(b_dst + j * 16 * GG_ROW_BYTES, &tmB, fb, kx, sc.y + j * 16, pol_x);
+                        tma_load_2d(a_dst, a_full ? &maps.a128 : &maps.a64, fb, kx, a_y, pol_w);
+                        for (int j = 0; j < n64; ++j)
+                            tma_load_2d(b_dst + j * 64 * GG_ROW_BYTES, &maps.b64, fb, kx, sc.y + j * 64, pol_x);
+                        for (int j = 0; j < r16; ++j)
+                            tma_load_2d(b_dst + (n64 * 4 + j) * 16 * GG_ROW_BYTES, &maps.b16, fb, kx,
+                                        sc.y + (n64 * 4 + j) * 16, pol_x);
                     }
                     if (++stage == NS) {
                         stage = 0;
@@ -174,8 +189,8 @@ __global__ void __launch_bounds__(GG_THREADS, 1)
                     const uint32_t b_base = smem_u32(smB + (size_t)stage * g.b_stage_bytes);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
-                        mma_ss<FP8>(d_tmem, sw128_desc(a_base + kk * 32), sw128_desc(b_base + kk * 32),
-                                    idesc, (ks | kk) != 0 ? 1u : 0u);
+                        mma_ss<FP8>(d_tmem, sw128_desc(a_base + kk * 32), sw128_desc(b_base + kk * 32), idesc,
+                                    (ks | kk) != 0 ? 1u : 0u);
                     }
                     issued = true;
                     mma_commit(smem_u32(&empty[stage]));
@@ -318,25 +333,27 @@ GemmPlan gemm_plan(int64_t T, int K, int E) {
 }
 
 template <bool FP8, bool UP>
-static cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& g, int grid,
-                              size_t smem, const DevCtx& ctx, cudaStream_t stream) {
+static cudaError_t launch_one(const GemmMaps& maps, const GemmArgs& g, int grid, size_t smem, const DevCtx& ctx,
+                              cudaStream_t stream) {
     auto kfn = grouped_gemm_kernel<FP8, UP>;
     cudaError_t err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
-    kfn<<<grid, GG_THREADS, smem, stream>>>(a, b, g, ctx);
+    kfn<<<grid, GG_THREADS, smem, stream>>>(maps, g, ctx);
     return cudaGetLastError();
 }
 
-// One grouped projection.  W: [E * Nout][Kdim] (bf16 or e4m3), Act: [rows][Kdim],
-// out: [rows][Nout].  sched / n_sched: device schedule over the rows.
+// One grouped projection.  W: [E * Nout][Kdim] (bf16 or e4m3), act: [rows][Kdim]
+// in the expert layout, out: [rows][Nout].  sched / n_sched: device schedule.
 cudaError_t launch_grouped_gemm(bool fp8, bool up, const void* W, int E, int Nout, int Kdim, const void* act,
                                 int64_t rows, const int4* sched, const int* n_sched, const GemmPlan& plan,
-                                void* out, const float* w_scale, float in_scale, float out_scale,
-                                int num_sms, int debug_withhold, const DevCtx& ctx, cudaStream_t stream) {
+                                void* out, const float* w_scale, float in_scale, float out_scale, int num_sms,
+                                int debug_withhold, const DevCtx& ctx, cudaStream_t stream) {
     if (rows == 0) return cudaSuccess;
-    CUtensorMap ta, tb;
-    if (!make_map(&ta, W, (int64_t)E * Nout, Kdim, fp8, 64)) return cudaErrorInvalidValue;
-    if (!make_map(&tb, act, rows, Kdim, fp8, 16)) return cudaErrorInvalidValue;
+    GemmMaps maps;
+    if (!make_map(&maps.a128, W, (int64_t)E * Nout, Kdim, fp8, 128) ||
+        !make_map(&maps.a64, W, (int64_t)E * Nout, Kdim, fp8, 64) ||
+        !make_map(&maps.b64, act, rows, Kdim, fp8, 64) || !make_map(&maps.b16, act, rows, Kdim, fp8, 16))
+        return cudaErrorInvalidValue;
     GemmArgs g;
     g.sched = sched;
     g.n_sched = n_sched;
@@ -355,11 +372,11 @@ cudaError_t launch_grouped_gemm(bool fp8, bool up, const void* W, int E, int Nou
     const int64_t max_units = (int64_t)plan.max_sched * g.m_blocks;
     const int grid = (int)(max_units < num_sms ? max_units : num_sms);
     if (fp8) {
-        return up ? launch_one<true, true>(ta, tb, g, grid, plan.smem_bytes, ctx, stream)
-                  : launch_one<true, false>(ta, tb, g, grid, plan.smem_bytes, ctx, stream);
+        return up ? launch_one<true, true>(maps, g, grid, plan.smem_bytes, ctx, stream)
+                  : launch_one<true, false>(maps, g, grid, plan.smem_bytes, ctx, stream);
     }
-    return up ? launch_one<false, true>(ta, tb, g, grid, plan.smem_bytes, ctx, stream)
-              : launch_one<false, false>(ta, tb, g, grid, plan.smem_bytes, ctx, stream);
+    return up ? launch_one<false, true>(maps, g, grid, plan.smem_bytes, ctx, stream)
+              : launch_one<false, false>(maps, g, grid, plan.smem_bytes, ctx, stream);
 }
 
 }  // namespace moe

@@ -16,6 +16,7 @@
 namespace moe {
 
 constexpr int PM_THREADS = 1024;
+constexpr int64_t kPermuteOneBlockMax = 4096;   // assignments sorted by the single-block kernel
 
 // Tile schedule: expert e's segment [offsets[e], offsets[e+1]) is cut into
 // near-equal blocks of at most bn rows, each a multiple of 16 rows except the
@@ -28,6 +29,39 @@ __device__ __forceinline__ int sched_per(int c, int bn) {
     return (per + 15) & ~15;
 }
 
+// In-place exclusive scan of v[0..n) (n <= 256) by the first 256 threads of
+// the block (blockDim.x >= 256); returns the total to every thread.
+__device__ int block_exclusive_scan256(int* v, int n) {
+    __shared__ int warp_tot[8];
+    __shared__ int total;
+    const int tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
+    int x = 0, incl = 0;
+    if (tid < 256) {
+        x = tid < n ? v[tid] : 0;
+        incl = x;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += y;
+        }
+        if (lane == 31) warp_tot[warp] = incl;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        int run = 0;
+        for (int w = 0; w < 8; ++w) {
+            const int y = warp_tot[w];
+            warp_tot[w] = run;
+            run += y;
+        }
+        total = run;
+    }
+    __syncthreads();
+    if (tid < n) v[tid] = warp_tot[warp] + incl - x;
+    __syncthreads();
+    return total;
+}
+
 __device__ void build_schedule(const int* seg_off, int E, int bn, int* nb_s, int4* sched,
                                int* n_sched) {
     const int tid = threadIdx.x;
@@ -36,16 +70,8 @@ __device__ void build_schedule(const int* seg_off, int E, int bn, int* nb_s, int
         nb_s[e] = c > 0 ? (c + sched_per(c, bn) - 1) / sched_per(c, bn) : 0;
     }
     __syncthreads();
-    if (tid == 0) {
-        int run = 0;
-        for (int e = 0; e < E; ++e) {
-            const int v = nb_s[e];
-            nb_s[e] = run;
-            run += v;
-        }
-        *n_sched = run;
-    }
-    __syncthreads();
+    const int total = block_exclusive_scan256(nb_s, E);
+    if (tid == 0) *n_sched = total;
     for (int e = tid; e < E; e += blockDim.x) {
         const int off = seg_off[e], c = seg_off[e + 1] - off;
         if (c <= 0) continue;
@@ -93,17 +119,17 @@ __global__ void __launch_bounds__(PM_THREADS) permute_kernel(PermuteArgs a, DevC
     if (__syncthreads_or(bad)) {
         if (tid == 0) record_error(ctx.err, MOE_EINDEX);
     }
+    for (int e = tid; e < E; e += PM_THREADS) offs[e] = hist[e];
+    __syncthreads();
+    const int total = block_exclusive_scan256(offs, E);
+    for (int e = tid; e < E; e += PM_THREADS) {
+        base[e] = offs[e];
+        a.offsets[e] = offs[e];
+        a.counts[e] = hist[e];
+    }
     if (tid == 0) {
-        int run = 0;
-        for (int e = 0; e < E; ++e) {
-            offs[e] = run;
-            base[e] = run;
-            a.offsets[e] = run;
-            a.counts[e] = hist[e];
-            run += hist[e];
-        }
-        offs[E] = run;
-        a.offsets[E] = run;
+        offs[E] = total;
+        a.offsets[E] = total;
     }
     __syncthreads();
 
@@ -139,6 +165,90 @@ __global__ void __launch_bounds__(PM_THREADS) permute_kernel(PermuteArgs a, DevC
     if (a.sched) build_schedule(offs, E, a.bn, hist, a.sched, a.n_sched);
 }
 
+// ---- multi-block permutation for large batches: one chunk of PM_THREADS
+// assignments per block; the stable rank inside a chunk is computed exactly
+// as in the single-block kernel, and chunks are ordered by their index.
+
+__global__ void __launch_bounds__(PM_THREADS) perm_hist_kernel(const int32_t* __restrict__ idx, int64_t n, int E,
+                                                               int* __restrict__ bcount, DevCtx ctx) {
+    __shared__ int hist[256];
+    const int tid = threadIdx.x;
+    for (int e = tid; e < E; e += PM_THREADS) hist[e] = 0;
+    __syncthreads();
+    const int64_t i = (int64_t)blockIdx.x * PM_THREADS + tid;
+    int bad = 0;
+    if (i < n) {
+        const int e = idx[i];
+        if (e < 0 || e >= E)
+            bad = 1;
+        else
+            atomicAdd(&hist[e], 1);
+    }
+    if (__syncthreads_or(bad) && tid == 0) record_error(ctx.err, MOE_EINDEX);
+    for (int e = tid; e < E; e += PM_THREADS) bcount[(int64_t)blockIdx.x * E + e] = hist[e];
+}
+
+// counts, offsets, per-(chunk, expert) bases, and the GEMM schedule
+__global__ void __launch_bounds__(256) perm_scan_kernel(const int* __restrict__ bcount, int G, int E,
+                                                        int* __restrict__ bbase, int32_t* counts,
+                                                        int32_t* offsets, int4* sched, int* n_sched, int bn) {
+    __shared__ int offs[257];
+    __shared__ int nb[256];
+    const int tid = threadIdx.x;
+    int tot = 0;
+    if (tid < E)
+        for (int b = 0; b < G; ++b) tot += bcount[(int64_t)b * E + tid];
+    if (tid < E) offs[tid] = tot;
+    __syncthreads();
+    const int total = block_exclusive_scan256(offs, E);
+    if (tid == 0) {
+        offs[E] = total;
+        offsets[E] = total;
+    }
+    if (tid < E) {
+        counts[tid] = tot;
+        offsets[tid] = offs[tid];
+        int run = offs[tid];
+        for (int b = 0; b < G; ++b) {
+            bbase[(int64_t)b * E + tid] = run;
+            run += bcount[(int64_t)b * E + tid];
+        }
+    }
+    __syncthreads();
+    if (sched) build_schedule(offs, E, bn, nb, sched, n_sched);
+}
+
+__global__ void __launch_bounds__(PM_THREADS) perm_scatter_kernel(const int32_t* __restrict__ idx, int64_t n,
+                                                                  int E, const int* __restrict__ bbase,
+                                                                  int32_t* __restrict__ perm_src,
+                                                                  int32_t* __restrict__ inv_row) {
+    extern __shared__ int wtab[];   // [32][E]
+    const int tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
+    const int64_t i = (int64_t)blockIdx.x * PM_THREADS + tid;
+    int e = i < n ? idx[i] : -1;
+    if (e >= E) e = -1;
+    for (int q = tid; q < 32 * E; q += PM_THREADS) wtab[q] = 0;
+    __syncthreads();
+    const uint32_t peers = __match_any_sync(0xffffffffu, e);
+    const int rank_w = __popc(peers & ((1u << lane) - 1u));
+    if (e >= 0 && rank_w == 0) wtab[warp * E + e] = __popc(peers);
+    __syncthreads();
+    for (int ex = tid; ex < E; ex += PM_THREADS) {
+        int run = bbase[(int64_t)blockIdx.x * E + ex];
+        for (int w = 0; w < 32; ++w) {
+            const int v = wtab[w * E + ex];
+            wtab[w * E + ex] = run;
+            run += v;
+        }
+    }
+    __syncthreads();
+    if (e >= 0) {
+        const int r = wtab[warp * E + e] + rank_w;
+        perm_src[r] = (int32_t)i;
+        inv_row[i] = r;
+    }
+}
+
 __global__ void schedule_kernel(const int32_t* offsets, int E, int bn, int4* sched, int* n_sched) {
     __shared__ int offs[257];
     __shared__ int nb[256];
@@ -147,7 +257,8 @@ __global__ void schedule_kernel(const int32_t* offsets, int E, int bn, int4* sch
     build_schedule(offs, E, bn, nb, sched, n_sched);
 }
 
-// X_perm[r] = x[perm_src[r] / K], or its E4M3 codes e4m3(x / x_scale) (fp8).
+// xp[r] = x[perm_src[r] / K], or its E4M3 codes e4m3(x / x_scale) (fp8);
+// with perm_src == null the rows are taken in order (xp[r] = x[r]).
 __global__ void gather_rows_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm_src,
                                    int64_t rows, int K, int64_t T, int H, void* __restrict__ xp,
                                    int fp8, float x_scale, DevCtx ctx) {
@@ -155,11 +266,14 @@ __global__ void gather_rows_kernel(const uint16_t* __restrict__ x, const int32_t
     const int64_t warps = (int64_t)gridDim.x * (blockDim.x / 32);
     const int nv = H / 8;
     for (int64_t r = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32; r < rows; r += warps) {
-        const int32_t src = perm_src[r];
-        const int64_t t = src / K;
-        if (src < 0 || t >= T) {
-            if (lane == 0) record_error(ctx.err, MOE_EINDEX);
-            continue;
+        int64_t t = r;
+        if (perm_src) {
+            const int32_t src = perm_src[r];
+            t = src / K;
+            if (src < 0 || t >= T) {
+                if (lane == 0) record_error(ctx.err, MOE_EINDEX);
+                continue;
+            }
         }
         const uint4* xr = reinterpret_cast<const uint4*>(x + t * H);
         if (!fp8) {
@@ -188,11 +302,29 @@ __global__ void gather_rows_kernel(const uint16_t* __restrict__ x, const int32_t
 
 size_t permute_smem_bytes(int E) { return (size_t)(4 * E + 1 + 32 * E) * sizeof(int); }
 
+// Scratch ints the multi-block path needs (0 when the single-block kernel runs).
+size_t permute_scratch_ints(int64_t n, int E) {
+    if (n <= kPermuteOneBlockMax) return 0;
+    const int64_t G = (n + PM_THREADS - 1) / PM_THREADS;
+    return (size_t)(2 * G * E);
+}
+
 cudaError_t launch_permute(const int32_t* idx, int64_t n, int E, int32_t* counts, int32_t* offsets,
                            int32_t* perm_src, int32_t* inv_row, int4* sched, int* n_sched, int bn,
-                           const DevCtx& ctx, cudaStream_t stream) {
-    PermuteArgs a{idx, n, E, counts, offsets, perm_src, inv_row, sched, n_sched, bn};
-    permute_kernel<<<1, PM_THREADS, permute_smem_bytes(E), stream>>>(a, ctx);
+                           int* scratch, const DevCtx& ctx, cudaStream_t stream) {
+    if (n <= kPermuteOneBlockMax) {
+        PermuteArgs a{idx, n, E, counts, offsets, perm_src, inv_row, sched, n_sched, bn};
+        permute_kernel<<<1, PM_THREADS, permute_smem_bytes(E), stream>>>(a, ctx);
+        return cudaGetLastError();
+    }
+    if (!scratch) return cudaErrorInvalidValue;
+    const int G = (int)((n + PM_THREADS - 1) / PM_THREADS);
+    int* bcount = scratch;
+    int* bbase = scratch + (size_t)G * E;
+    perm_hist_kernel<<<G, PM_THREADS, 0, stream>>>(idx, n, E, bcount, ctx);
+    perm_scan_kernel<<<1, 256, 0, stream>>>(bcount, G, E, bbase, counts, offsets, sched, n_sched, bn);
+    perm_scatter_kernel<<<G, PM_THREADS, (size_t)32 * E * sizeof(int), stream>>>(idx, n, E, bbase, perm_src,
+                                                                                  inv_row);
     return cudaGetLastError();
 }
 

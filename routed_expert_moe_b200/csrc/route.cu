@@ -9,15 +9,16 @@
 // product, exact in fp32, rounded to the grid 2^-40 and summed exactly in
 // int64), which makes the order independent of summation order.  The kernels
 // never need that sum for most tokens:
-//   1. router_logits_kernel computes l~ in fp32 over chunks of RT_HC terms,
-//      chunk sums accumulated in fp64, plus the squared norms of x and Wr.
+//   1. router_logits_kernel computes l~ in fp32 over chunks of RT_HC = 16
+//      terms, chunk sums accumulated in fp64, plus the squared norms of x and Wr.
 //      |l~ - l_fx| <= eps_e = (g_RT_HC + 2^-45) ||x|| ||w_e|| + (H+1) 2^-41
 //      (Cauchy-Schwarz bounds sum|x_h w_eh|; g_n = n u / (1 - n u), u = 2^-24).
 //   2. router_topk_kernel (one warp per token) ranks l~; if every gap among
 //      the K+1 best exceeds 2 eps* (eps* = max_e eps_e) the order is certified.
 //      Otherwise it recomputes l_fx exactly for the candidates
 //      {e : l~_e >= l~_(K) - 2 eps*} (no other expert can reach the top K)
-//      and ranks those.
+//      and ranks those; the candidates of a block's 8 tokens are computed by
+//      all its warps together.
 // Both kernels use only CUDA cores: the contraction is 2.8 GFLOP at 4096
 // tokens, and a tensor-core accumulation has no error bound to certify.
 #include <cstdint>
@@ -29,9 +30,8 @@
 
 namespace moe {
 
-constexpr int RT_TT = 32;       // tokens per block tile
-constexpr int RT_TE = 64;       // experts per block tile
-constexpr int RT_HC = 32;       // terms per fp32 partial sum
+constexpr int RT_TE = 128;      // experts per block tile
+constexpr int RT_HC = 16;       // terms per fp32 partial sum
 constexpr int RT_THREADS = 256;
 
 struct RouterLogitsArgs {
@@ -44,9 +44,17 @@ struct RouterLogitsArgs {
     double* wn2;          // [S][E]  partial ||w_e||^2
 };
 
+// One block: 16*TPT tokens x 128 experts over one split of the hidden
+// dimension.  Thread (tg, eg) owns tokens TPT*tg .. +TPT-1 x experts
+// 8eg..8eg+7.  Each 16-term chunk is a chain of fp32 FMAs from zero (the
+// products are exact), added into an fp64 total; smem tiles are
+// double-buffered.  TPT = 4 for large batches (64-token tiles), 1 for small
+// ones so that a decode batch still spreads over the whole GPU.
+template <int TPT>
 __global__ void __launch_bounds__(RT_THREADS) router_logits_kernel(RouterLogitsArgs a) {
-    __shared__ __align__(16) float xs[RT_HC][RT_TT];
-    __shared__ __align__(16) float ws[RT_HC][RT_TE];
+    constexpr int RT_TT = 16 * TPT;
+    __shared__ __align__(16) float xs[2][RT_HC][RT_TT];
+    __shared__ __align__(16) float ws[2][RT_HC][RT_TE];
 
     const int tid = threadIdx.x;
     const int64_t t0 = (int64_t)blockIdx.x * RT_TT;
@@ -55,120 +63,102 @@ __global__ void __launch_bounds__(RT_THREADS) router_logits_kernel(RouterLogitsA
     const int c_begin = (int)((int64_t)s * a.nchunks / a.S);
     const int c_end = (int)((int64_t)(s + 1) * a.nchunks / a.S);
 
-    const int tg = tid / 16;    // tokens 2*tg, 2*tg+1
-    const int eg = tid % 16;    // experts 4*eg .. 4*eg+3
+    const int tg = tid / 16;    // tokens TPT*tg .. TPT*tg+TPT-1
+    const int eg = tid % 16;    // experts 8*eg .. 8*eg+7
+    const int l_row = tid / 2, l_half = tid % 2;   // staging: row tid/2, 8 terms at 8*(tid%2)
 
-    // staging assignment: threads 0..127 load x (token tid/4, vector tid%4),
-    // all 256 load w (expert tid/4, vector tid%4); a vector is 8 bf16.
-    const int xl_t = tid / 4, xl_v = tid % 4;
-    const int wl_e = tid / 4, wl_v = tid % 4;
-
-    double acc[8];
+    double acc[TPT * 8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = 0.0;
+    for (int i = 0; i < TPT * 8; ++i) acc[i] = 0.0;
+    double xsq = 0.0, wsq = 0.0;   // squared norms of this thread's staged row halves
 
-    auto load_chunk = [&](int c, uint4& xv, uint4& wv) {
-        const int h = c * RT_HC;
+    auto load = [&](int c, uint4& xv, uint4& wv) {
+        const int h = c * RT_HC + l_half * 8;
         xv = make_uint4(0, 0, 0, 0);
         wv = make_uint4(0, 0, 0, 0);
-        if (tid < 128) {
-            const int64_t t = t0 + xl_t;
-            const int hh = h + xl_v * 8;
-            if (t < a.T && hh < a.H) xv = *reinterpret_cast<const uint4*>(a.x + t * a.H + hh);
-        }
-        {
-            const int e = e0 + wl_e;
-            const int hh = h + wl_v * 8;
-            if (e < a.E && hh < a.H)
-                wv = *reinterpret_cast<const uint4*>(a.wr + (int64_t)e * a.H + hh);
-        }
+        const int64_t t = t0 + l_row;
+        if (tid < 2 * RT_TT && t < a.T && h < a.H) xv = *reinterpret_cast<const uint4*>(a.x + t * a.H + h);
+        const int e = e0 + l_row;
+        if (e < a.E && h < a.H) wv = *reinterpret_cast<const uint4*>(a.wr + (int64_t)e * a.H + h);
     };
-    auto store_chunk = [&](const uint4& xv, const uint4& wv) {
+    auto store = [&](int buf, const uint4& xv, const uint4& wv) {
         const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
         const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
-        if (tid < 128) {
+        if (tid < 2 * RT_TT) {
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                xs[xl_v * 8 + 2 * q][xl_t] = __uint_as_float(xw[q] << 16);
-                xs[xl_v * 8 + 2 * q + 1][xl_t] = __uint_as_float(xw[q] & 0xFFFF0000u);
+                const float lo = __uint_as_float(xw[q] << 16), hi = __uint_as_float(xw[q] & 0xFFFF0000u);
+                xs[buf][l_half * 8 + 2 * q][l_row] = lo;
+                xs[buf][l_half * 8 + 2 * q + 1][l_row] = hi;
+                xsq += (double)lo * (double)lo + (double)hi * (double)hi;
             }
         }
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            ws[wl_v * 8 + 2 * q][wl_e] = __uint_as_float(ww[q] << 16);
-            ws[wl_v * 8 + 2 * q + 1][wl_e] = __uint_as_float(ww[q] & 0xFFFF0000u);
+            const float lo = __uint_as_float(ww[q] << 16), hi = __uint_as_float(ww[q] & 0xFFFF0000u);
+            ws[buf][l_half * 8 + 2 * q][l_row] = lo;
+            ws[buf][l_half * 8 + 2 * q + 1][l_row] = hi;
+            wsq += (double)lo * (double)lo + (double)hi * (double)hi;
         }
     };
 
     uint4 xv, wv;
-    if (c_begin < c_end) load_chunk(c_begin, xv, wv);
+    if (c_begin < c_end) {
+        load(c_begin, xv, wv);
+        store(0, xv, wv);
+    }
+    __syncthreads();
     for (int c = c_begin; c < c_end; ++c) {
-        __syncthreads();
-        store_chunk(xv, wv);
-        __syncthreads();
-        if (c + 1 < c_end) load_chunk(c + 1, xv, wv);
-        float p[8];
+        const int buf = (c - c_begin) & 1;
+        if (c + 1 < c_end) load(c + 1, xv, wv);
+        float p[TPT * 8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) p[i] = 0.0f;
-#pragma unroll 8
+        for (int i = 0; i < TPT * 8; ++i) p[i] = 0.0f;
+#pragma unroll
         for (int h = 0; h < RT_HC; ++h) {
-            const float2 xx = *reinterpret_cast<const float2*>(&xs[h][2 * tg]);
-            const float4 w4 = *reinterpret_cast<const float4*>(&ws[h][4 * eg]);
-            p[0] = __fmaf_rn(xx.x, w4.x, p[0]);
-            p[1] = __fmaf_rn(xx.x, w4.y, p[1]);
-            p[2] = __fmaf_rn(xx.x, w4.z, p[2]);
-            p[3] = __fmaf_rn(xx.x, w4.w, p[3]);
-            p[4] = __fmaf_rn(xx.y, w4.x, p[4]);
-            p[5] = __fmaf_rn(xx.y, w4.y, p[5]);
-            p[6] = __fmaf_rn(xx.y, w4.z, p[6]);
-            p[7] = __fmaf_rn(xx.y, w4.w, p[7]);
+            float xr[TPT];
+            if constexpr (TPT == 4) {
+                const float4 xx = *reinterpret_cast<const float4*>(&xs[buf][h][4 * tg]);
+                xr[0] = xx.x;
+                xr[1] = xx.y;
+                xr[2] = xx.z;
+                xr[3] = xx.w;
+            } else {
+                xr[0] = xs[buf][h][tg];
+            }
+            const float4 wa = *reinterpret_cast<const float4*>(&ws[buf][h][8 * eg]);
+            const float4 wb = *reinterpret_cast<const float4*>(&ws[buf][h][8 * eg + 4]);
+            const float wr8[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+#pragma unroll
+            for (int i = 0; i < TPT; ++i)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) p[i * 8 + j] = __fmaf_rn(xr[i], wr8[j], p[i * 8 + j]);
         }
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] += (double)p[i];
+        for (int i = 0; i < TPT * 8; ++i) acc[i] += (double)p[i];
+        if (c + 1 < c_end) store(buf ^ 1, xv, wv);
+        __syncthreads();
     }
 
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        const int64_t t = t0 + 2 * tg + i;
+    for (int i = 0; i < TPT; ++i) {
+        const int64_t t = t0 + TPT * tg + i;
         if (t >= a.T) continue;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int e = e0 + 4 * eg + j;
-            if (e < a.E) a.P[((int64_t)s * a.T + t) * a.E + e] = acc[i * 4 + j];
+        for (int j = 0; j < 8; ++j) {
+            const int e = e0 + 8 * eg + j;
+            if (e < a.E) a.P[((int64_t)s * a.T + t) * a.E + e] = acc[i * 8 + j];
         }
     }
 
-    // squared norms of this split's range (fp64 sums of exact squares)
-    const int warp = tid / 32, lane = tid % 32;
-    const int h_lo = c_begin * RT_HC;
-    const int h_hi = min(c_end * RT_HC, a.H);
-    if (blockIdx.y == 0) {
-        for (int i = warp; i < RT_TT; i += RT_THREADS / 32) {
-            const int64_t t = t0 + i;
-            if (t >= a.T) break;
-            double q = 0.0;
-            for (int h = h_lo + lane; h < h_hi; h += 32) {
-                const double v = (double)bf16_bits_to_float(a.x[t * a.H + h]);
-                q += v * v;
-            }
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) q += __shfl_xor_sync(0xffffffffu, q, off);
-            if (lane == 0) a.xn2[(int64_t)s * a.T + t] = q;
-        }
-    }
-    if (blockIdx.x == 0) {
-        for (int i = warp; i < RT_TE; i += RT_THREADS / 32) {
-            const int e = e0 + i;
-            if (e >= a.E) break;
-            double q = 0.0;
-            for (int h = h_lo + lane; h < h_hi; h += 32) {
-                const double v = (double)bf16_bits_to_float(a.wr[(int64_t)e * a.H + h]);
-                q += v * v;
-            }
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) q += __shfl_xor_sync(0xffffffffu, q, off);
-            if (lane == 0) a.wn2[(int64_t)s * a.E + e] = q;
-        }
+    // squared norms of this split's range: the two halves of a row sit in adjacent lanes
+    xsq += __shfl_xor_sync(0xffffffffu, xsq, 1);
+    wsq += __shfl_xor_sync(0xffffffffu, wsq, 1);
+    if (l_half == 0) {
+        const int64_t t = t0 + l_row;
+        if (blockIdx.y == 0 && tid < 2 * RT_TT && t < a.T) a.xn2[(int64_t)s * a.T + t] = xsq;
+        const int e = e0 + l_row;
+        if (blockIdx.x == 0 && e < a.E) a.wn2[(int64_t)s * a.E + e] = wsq;
     }
 }
 
@@ -185,7 +175,9 @@ struct RouterTopkArgs {
     float* w;             // [T][K]
 };
 
-constexpr int TK_MAXJ = 8;   // experts per lane (E <= 256)
+constexpr int TK_MAXJ = 8;        // experts per lane (E <= 256)
+constexpr int TK_WARPS = 8;       // tokens per block
+constexpr int TK_CAP = TK_WARPS * 256;
 
 // warp arg-max of (value, -index)
 __device__ __forceinline__ void warp_argmax(double& v, int& e) {
@@ -212,135 +204,182 @@ __device__ __forceinline__ void warp_argmax_i64(long long& v, int& e) {
     }
 }
 
-__global__ void __launch_bounds__(256) router_topk_kernel(RouterTopkArgs a, DevCtx ctx) {
-    const int lane = threadIdx.x % 32;
-    const int64_t t = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
-    if (t >= a.T) return;
+// Exact fixed-point logit (units of 2^-40) of expert e for token row xr:
+// every bf16 product (exact in fp32) scaled by 2^40 and rounded to the
+// nearest integer, summed exactly; 16-byte loads, one warp.
+__device__ long long exact_logit(const uint16_t* xr, const uint16_t* wrow, int H, const float* bias, int e,
+                                 int lane) {
+    const uint4* xv = reinterpret_cast<const uint4*>(xr);
+    const uint4* wv = reinterpret_cast<const uint4*>(wrow);
+    long long acc = 0;
+    for (int v = lane; v < H / 8; v += 32) {
+        const uint4 a = xv[v], b = wv[v];
+        const uint32_t aa[4] = {a.x, a.y, a.z, a.w};
+        const uint32_t bb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float p0 = __fmul_rn(__uint_as_float(aa[j] << 16), __uint_as_float(bb[j] << 16));
+            const float p1 = __fmul_rn(__uint_as_float(aa[j] & 0xFFFF0000u), __uint_as_float(bb[j] & 0xFFFF0000u));
+            acc += __float2ll_rn(__fmul_rn(p0, 0x1p40f));
+            acc += __float2ll_rn(__fmul_rn(p1, 0x1p40f));
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (bias) acc += __float2ll_rn(__fmul_rn(bias[e], 0x1p40f));
+    return acc;
+}
+
+// One warp per token ranks l~; tokens whose order the bound leaves open put
+// their candidates in a block-wide list whose exact logits all 8 warps
+// compute together, then finish their selection from it.
+__global__ void __launch_bounds__(TK_WARPS * 32, 2) router_topk_kernel(RouterTopkArgs a, DevCtx ctx) {
+    __shared__ int c_tok[TK_CAP];
+    __shared__ int c_e[TK_CAP];
+    __shared__ long long c_val[TK_CAP];
+    __shared__ int n_cand;
+
+    const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
+    const int64_t t = (int64_t)blockIdx.x * TK_WARPS + warp;
+    const bool active = t < a.T;
+    if (threadIdx.x == 0) n_cand = 0;
+    __syncthreads();
 
     const int nj = (a.E + 31) / 32;
-    // g_32 + 2^-45, with a little slack for the fp64 norm sums and sqrt
-    const double kRel = (32.0 * 0x1p-24) / (1.0 - 32.0 * 0x1p-24) + 0x1p-45 + 0x1p-40;
+    // g_16 + 2^-45 (fp64 sums of the chunk and split partials), with slack for the norm sums
+    const double kRel = (16.0 * 0x1p-24) / (1.0 - 16.0 * 0x1p-24) + 0x1p-45 + 0x1p-40;
     const double kFx = (double)(a.H + 1) * 0x1p-41;
 
-    double xn2 = 0.0;
-    for (int s = 0; s < a.S; ++s) xn2 += a.xn2[(int64_t)s * a.T + t];
-    const double xnorm = sqrt(xn2);
-
     double L[TK_MAXJ];
-    double wnorm[TK_MAXJ];
-    double eps_star = 0.0;
-    bool range_bad = false;
-#pragma unroll
-    for (int j = 0; j < TK_MAXJ; ++j) {
-        L[j] = -DBL_MAX;
-        wnorm[j] = 0.0;
-        const int e = lane + 32 * j;
-        if (j < nj && e < a.E) {
-            double l = 0.0, q = 0.0;
-            for (int s = 0; s < a.S; ++s) {
-                l += a.P[((int64_t)s * a.T + t) * a.E + e];
-                q += a.wn2[(int64_t)s * a.E + e];
-            }
-            double b = 0.0;
-            if (a.bias) {
-                b = (double)a.bias[e];
-                if (fabs(b) >= 0x1p21) range_bad = true;
-            }
-            l += b;
-            wnorm[j] = sqrt(q);
-            if (xnorm * wnorm[j] >= 0x1p22) range_bad = true;
-            const double eps = kRel * xnorm * wnorm[j] + kFx + fabs(l) * 0x1p-50;
-            eps_star = fmax(eps_star, eps);
-            L[j] = l;
-        }
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1)
-        eps_star = fmax(eps_star, __shfl_xor_sync(0xffffffffu, eps_star, off));
-
-    // the K+1 best by l~ (ties to the lower index)
-    const int nsel = min(a.K + 1, a.E);
-    uint32_t taken = 0;
-    int sel_e[17];
-    double sel_l[17];
-    for (int k = 0; k < nsel; ++k) {
-        double bv = -DBL_MAX;
-        int be = 0x7fffffff;
-#pragma unroll
-        for (int j = 0; j < TK_MAXJ; ++j) {
-            const int e = lane + 32 * j;
-            if (j < nj && e < a.E && !((taken >> j) & 1u)) {
-                if (L[j] > bv || (L[j] == bv && e < be)) {
-                    bv = L[j];
-                    be = e;
-                }
-            }
-        }
-        warp_argmax(bv, be);
-        sel_e[k] = be;
-        sel_l[k] = bv;
-        if ((be & 31) == lane) taken |= 1u << (be >> 5);
-    }
-
     bool certified = true;
-    for (int i = 0; i + 1 < nsel; ++i)
-        if (!(sel_l[i] - sel_l[i + 1] > 2.0 * eps_star)) certified = false;
-
+    bool range_bad = false;
     int out_e[16];
     double out_l[16];
-    if (certified) {
-        for (int k = 0; k < a.K; ++k) {
-            out_e[k] = sel_e[k];
-            out_l[k] = sel_l[k];
-        }
-    } else {
-        // exact fixed-point logits of every candidate
-        const double thr = sel_l[a.K - 1] - 2.0 * eps_star;
-        long long lfx[TK_MAXJ];
-        uint32_t cand = 0;
+    if (active) {
+        // partial logits and weight norms of every split: coalesced rows of E,
+        // loaded in groups of 8 splits with no dependence between the loads
+        double lsum[TK_MAXJ], qsum[TK_MAXJ];
+        double xn2 = 0.0;
 #pragma unroll
-        for (int j = 0; j < TK_MAXJ; ++j) {
-            lfx[j] = LLONG_MIN;
-            const int e = lane + 32 * j;
-            if (j < nj && e < a.E && L[j] >= thr) cand |= 1u << j;
-        }
-        const uint16_t* xr = a.x + t * a.H;
-        for (int j = 0; j < nj; ++j) {
-            uint32_t m = __ballot_sync(0xffffffffu, (cand >> j) & 1u);
-            while (m) {
-                const int src = __ffs(m) - 1;
-                m &= m - 1;
-                const int e = src + 32 * j;
-                const uint16_t* wrow = a.wr + (int64_t)e * a.H;
-                long long acc = 0;
-                for (int h = lane; h < a.H; h += 32) {
-                    const float p = __fmul_rn(bf16_bits_to_float(xr[h]), bf16_bits_to_float(wrow[h]));
-                    acc += __float2ll_rn(__fmul_rn(p, 0x1p40f));
+        for (int j = 0; j < TK_MAXJ; ++j) lsum[j] = qsum[j] = 0.0;
+        for (int s0 = 0; s0 < a.S; s0 += 8) {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int s = s0 + u;
+                if (s < a.S) {
+                    xn2 += a.xn2[(int64_t)s * a.T + t];
+                    const double* prow = a.P + ((int64_t)s * a.T + t) * a.E;
+                    const double* wrow = a.wn2 + (int64_t)s * a.E;
+#pragma unroll
+                    for (int j = 0; j < TK_MAXJ; ++j) {
+                        const int e = lane + 32 * j;
+                        if (j < nj && e < a.E) {
+                            lsum[j] += prow[e];
+                            qsum[j] += wrow[e];
+                        }
+                    }
                 }
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-                if (a.bias) acc += __float2ll_rn(__fmul_rn(a.bias[e], 0x1p40f));
-                if (lane == src) lfx[j] = acc;
             }
         }
-        uint32_t used = 0;
-        for (int k = 0; k < a.K; ++k) {
-            long long bv = LLONG_MIN;
+        const double xnorm = sqrt(xn2);
+        double eps_star = 0.0;
+#pragma unroll
+        for (int j = 0; j < TK_MAXJ; ++j) {
+            L[j] = -DBL_MAX;
+            const int e = lane + 32 * j;
+            if (j < nj && e < a.E) {
+                double l = lsum[j];
+                if (a.bias) {
+                    const double b = (double)a.bias[e];
+                    if (fabs(b) >= 0x1p21) range_bad = true;
+                    l += b;
+                }
+                const double wnorm = sqrt(qsum[j]);
+                if (xnorm * wnorm >= 0x1p22) range_bad = true;
+                eps_star = fmax(eps_star, kRel * xnorm * wnorm + kFx + fabs(l) * 0x1p-50);
+                L[j] = l;
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+            eps_star = fmax(eps_star, __shfl_xor_sync(0xffffffffu, eps_star, off));
+
+        // the K+1 best by l~ (ties to the lower index)
+        const int nsel = min(a.K + 1, a.E);
+        uint32_t taken = 0;
+        double prev = 0.0;
+        for (int k = 0; k < nsel; ++k) {
+            double bv = -DBL_MAX;
             int be = 0x7fffffff;
 #pragma unroll
             for (int j = 0; j < TK_MAXJ; ++j) {
                 const int e = lane + 32 * j;
-                if (((cand >> j) & 1u) && !((used >> j) & 1u)) {
-                    if (lfx[j] > bv || (lfx[j] == bv && e < be)) {
-                        bv = lfx[j];
+                if (j < nj && e < a.E && !((taken >> j) & 1u)) {
+                    if (L[j] > bv || (L[j] == bv && e < be)) {
+                        bv = L[j];
                         be = e;
                     }
                 }
             }
-            warp_argmax_i64(bv, be);
-            out_e[k] = be;
+            warp_argmax(bv, be);
+            if (k < a.K) {
+                out_e[k] = be;
+                out_l[k] = bv;
+            }
+            if (k > 0 && !(prev - bv > 2.0 * eps_star)) certified = false;
+            prev = bv;
+            if ((be & 31) == lane) taken |= 1u << (be >> 5);
+        }
+        if (!certified) {
+            // candidates: every expert that could still be in the exact top K
+            const double thr = out_l[a.K - 1] - 2.0 * eps_star;
+#pragma unroll
+            for (int j = 0; j < TK_MAXJ; ++j) {
+                const int e = lane + 32 * j;
+                const bool c = j < nj && e < a.E && L[j] >= thr;
+                const uint32_t m = __ballot_sync(0xffffffffu, c);
+                int base = 0;
+                if (lane == 0 && m) base = atomicAdd(&n_cand, __popc(m));
+                base = __shfl_sync(0xffffffffu, base, 0);
+                if (c) {
+                    const int i = base + __popc(m & ((1u << lane) - 1u));
+                    c_tok[i] = warp;
+                    c_e[i] = e;
+                }
+            }
+        }
+    }
+    __syncthreads();
+    const int nc = n_cand;
+    for (int i = warp; i < nc; i += TK_WARPS) {
+        const int64_t tt = (int64_t)blockIdx.x * TK_WARPS + c_tok[i];
+        const int e = c_e[i];
+        const long long v = exact_logit(a.x + tt * a.H, a.wr + (int64_t)e * a.H, a.H, a.bias, e, lane);
+        if (lane == 0) c_val[i] = v;
+    }
+    __syncthreads();
+
+    if (!active) return;
+    if (!certified) {
+        for (int k = 0; k < a.K; ++k) {
+            long long bv = LLONG_MIN;
+            int be = 0x7fffffff, bi = -1;
+            for (int i = lane; i < nc; i += 32) {
+                if (c_tok[i] != warp) continue;
+                const long long v = c_val[i];
+                const int e = c_e[i];
+                if (bi < 0 || v > bv || (v == bv && e < be)) {
+                    bv = v;
+                    be = e;
+                    bi = i;
+                }
+            }
+            int src_e = be;
+            warp_argmax_i64(bv, src_e);
+            if (bi >= 0 && be == src_e) c_tok[bi] = -1;   // taken (this lane held it)
+            __syncwarp();
+            out_e[k] = src_e;
             out_l[k] = (double)bv * 0x1p-40;
-            if ((be & 31) == lane) used |= 1u << (be >> 5);
         }
     }
     if (__any_sync(0xffffffffu, range_bad) && lane == 0) record_error(ctx.err, MOE_ERANGE);
@@ -353,7 +392,6 @@ __global__ void __launch_bounds__(256) router_topk_kernel(RouterTopkArgs a, DevC
         z += ex[k];
     }
     for (int k = lane; k < a.K; k += 32) {
-        // registers indexed by a lane-dependent k: select through a small loop
         int ek = 0;
         float wk = 0.0f;
         for (int q = 0; q < a.K; ++q)
@@ -374,13 +412,18 @@ struct RouterPlan {
     size_t p_bytes, xn_bytes, wn_bytes;
 };
 
+static int router_tt(int64_t T) { return T > 256 ? 64 : 16; }
+
 RouterPlan router_plan(int64_t T, int H, int E, int num_sms) {
     RouterPlan p;
     p.nchunks = (H + RT_HC - 1) / RT_HC;
-    const int64_t tiles = ((T + RT_TT - 1) / RT_TT) * ((E + RT_TE - 1) / RT_TE);
-    int64_t want = tiles > 0 ? (2 * (int64_t)num_sms + tiles - 1) / tiles : 1;
-    // keep at least 4 chunks per split so the fp64 partial traffic stays small
-    const int64_t cap = (p.nchunks + 3) / 4;
+    const int tt = router_tt(T);
+    const int64_t tiles = ((T + tt - 1) / tt) * ((E + RT_TE - 1) / RT_TE);
+    // about one wave of blocks; at least 4 chunks per split, at most 32 splits
+    int64_t want = tiles > 0 ? ((int64_t)num_sms + tiles - 1) / tiles : 1;
+    if (tiles * want > (int64_t)num_sms && want > 1) want -= 1;
+    int64_t cap = p.nchunks / 4 > 0 ? p.nchunks / 4 : 1;
+    if (cap > 32) cap = 32;
     if (want > cap) want = cap;
     if (want < 1) want = 1;
     p.S = (int)want;
@@ -396,15 +439,18 @@ cudaError_t launch_route(const uint16_t* x, const uint16_t* wr, const float* bia
                          void (*between)(cudaStream_t)) {
     if (T == 0) return cudaSuccess;
     RouterLogitsArgs la{x, wr, T, H, E, plan.S, plan.nchunks, P, xn2, wn2};
-    dim3 grid((unsigned)((T + RT_TT - 1) / RT_TT), (unsigned)((E + RT_TE - 1) / RT_TE),
-              (unsigned)plan.S);
-    router_logits_kernel<<<grid, RT_THREADS, 0, stream>>>(la);
+    const int tt = router_tt(T);
+    dim3 grid((unsigned)((T + tt - 1) / tt), (unsigned)((E + RT_TE - 1) / RT_TE), (unsigned)plan.S);
+    if (tt == 64)
+        router_logits_kernel<4><<<grid, RT_THREADS, 0, stream>>>(la);
+    else
+        router_logits_kernel<1><<<grid, RT_THREADS, 0, stream>>>(la);
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     if (between) between(stream);
     RouterTopkArgs ta{P, xn2, wn2, x, wr, bias, T, H, E, K, plan.S, idx, w};
-    const unsigned blocks = (unsigned)((T + 7) / 8);
-    router_topk_kernel<<<blocks, 256, 0, stream>>>(ta, ctx);
+    const unsigned blocks = (unsigned)((T + TK_WARPS - 1) / TK_WARPS);
+    router_topk_kernel<<<blocks, TK_WARPS * 32, 0, stream>>>(ta, ctx);
     return cudaGetLastError();
 }
 

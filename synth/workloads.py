@@ -99,3 +99,17 @@ def host_w_down(w: Workload, layer: int = 0, experts=None) -> np.ndarray:
 
 def host_bias(w: Workload):
     return zipf_bias(w.seed, w.E) if w.zipf_bias else None
+
+
+def chain_scales():
+    """Static W8A8 activation scales of the chain workload, per layer (x_scale, h_scale) as fp32.
+
+    Written by tests/golden/make_fp8_chain_scales.py from a calibration pass of the oracle.
+    """
+    import json
+    import struct
+    from pathlib import Path
+    p = Path(__file__).resolve().parents[1] / "tests" / "golden" / "fp8_chain_scales.json"
+    d = json.loads(p.read_text())
+    f32 = lambda h: np.float32(struct.unpack(">f", bytes.fromhex(h))[0])
+    return [(f32(l["x_scale_f32"]), f32(l["h_scale_f32"])) for l in d["layers"]]

@@ -64,7 +64,7 @@ def test_full_size_routing_permutation_and_sampled_outputs(moe, cfg):
     assert np.max(np.abs(wt.cpu().numpy() - rw)) <= 1e-5
     counts, offsets, perm_src, inv_row = oracle.permute(ridx, w.E)
     g = [torch.empty(n, dtype=torch.int32, device="cuda") for n in (w.E, w.E + 1, w.T * w.K, w.T * w.K)]
-    moe.permute(dims, idx, *g)
+    moe.permute(dims, idx, *g, ws=ws)
     moe.check_device_error()
     for got, ref in zip(g, (counts, offsets, perm_src, inv_row)):
         assert np.array_equal(got.cpu().numpy(), ref)

@@ -232,3 +232,24 @@ def test_host_rejects_bad_arguments(moe):
     with pytest.raises(moe.MoeError) as e:
         moe.forward(dims, d["x"][:, 1:], d["wr"], None, d["wu"], d["wd"], out, ws)   # misaligned
     assert e.value.status == moe.MOE_EINVAL
+
+
+@pytest.mark.parametrize("T,E,K,zipf", [(1000, 16, 5, True), (4096, 128, 6, False), (683, 256, 6, True)])
+def test_permute_multi_block_bit_exact(moe, T, E, K, zipf):
+    """More than 4096 assignments: the chunked multi-block sort (ragged last chunk, empty experts)."""
+    w = W.Workload(f"perm_T{T}_E{E}", T, 256, E, K, 128, seed=19)
+    x = W.host_x(w)
+    wr = W.host_router(w)
+    bias = W.zipf_bias(19, E) if zipf else None
+    _, ridx, _ = oracle.route(x, wr, bias, K)
+    ref = oracle.permute(ridx, E)
+    dims = moe.dims(T, 256, E, K, 128)
+    ws = moe.alloc_workspace(dims)
+    g = [torch.empty(n, dtype=torch.int32, device="cuda") for n in (E, E + 1, T * K, T * K)]
+    with pytest.raises(moe.MoeError) as err:
+        moe.permute(dims, dev(ridx), *g)        # needs scratch above 4096 assignments
+    assert err.value.status == moe.MOE_EWORKSPACE
+    moe.permute(dims, dev(ridx), *g, ws=ws)
+    moe.check_device_error()
+    for got, r in zip(g, ref):
+        assert np.array_equal(got.cpu().numpy(), r)
