@@ -12,6 +12,8 @@
 //   1. router_logits_kernel computes l~ in fp32 over chunks of RT_HC = 16
 //      terms, chunk sums accumulated in fp64, plus the squared norms of x and Wr.
 //      |l~ - l_fx| <= eps_e = (g_RT_HC + 2^-45) ||x|| ||w_e|| + (H+1) 2^-41
+//      (the squared norms are fp32 sums of exact squares, at most H terms per
+//      value, so they are inflated by 1 + (H+64) 2^-23 to stay upper bounds)
 //      (Cauchy-Schwarz bounds sum|x_h w_eh|; g_n = n u / (1 - n u), u = 2^-24).
 //   2. router_topk_kernel (one warp per token) ranks l~; if every gap among
 //      the K+1 best exceeds 2 eps* (eps* = max_e eps_e) the order is certified.
@@ -64,13 +66,13 @@ __global__ void __launch_bounds__(RT_THREADS) router_logits_kernel(RouterLogitsA
     const int c_end = (int)((int64_t)(s + 1) * a.nchunks / a.S);
 
     const int tg = tid / 16;    // tokens TPT*tg .. TPT*tg+TPT-1
-    const int eg = tid % 16;    // experts 8*eg .. 8*eg+7
+    const int eg = tid % 16;    // experts 4eg..4eg+3 and 64+4eg..64+4eg+3 (16-byte smem reads, no stride)
     const int l_row = tid / 2, l_half = tid % 2;   // staging: row tid/2, 8 terms at 8*(tid%2)
 
     double acc[TPT * 8];
 #pragma unroll
     for (int i = 0; i < TPT * 8; ++i) acc[i] = 0.0;
-    double xsq = 0.0, wsq = 0.0;   // squared norms of this thread's staged row halves
+    float xsq = 0.0f, wsq = 0.0f;  // squared norms of this thread's staged row halves (fp32; see below)
 
     auto load = [&](int c, uint4& xv, uint4& wv) {
         const int h = c * RT_HC + l_half * 8;
@@ -90,7 +92,7 @@ __global__ void __launch_bounds__(RT_THREADS) router_logits_kernel(RouterLogitsA
                 const float lo = __uint_as_float(xw[q] << 16), hi = __uint_as_float(xw[q] & 0xFFFF0000u);
                 xs[buf][l_half * 8 + 2 * q][l_row] = lo;
                 xs[buf][l_half * 8 + 2 * q + 1][l_row] = hi;
-                xsq += (double)lo * (double)lo + (double)hi * (double)hi;
+                xsq = __fmaf_rn(hi, hi, __fmaf_rn(lo, lo, xsq));
             }
         }
 #pragma unroll
@@ -98,7 +100,7 @@ __global__ void __launch_bounds__(RT_THREADS) router_logits_kernel(RouterLogitsA
             const float lo = __uint_as_float(ww[q] << 16), hi = __uint_as_float(ww[q] & 0xFFFF0000u);
             ws[buf][l_half * 8 + 2 * q][l_row] = lo;
             ws[buf][l_half * 8 + 2 * q + 1][l_row] = hi;
-            wsq += (double)lo * (double)lo + (double)hi * (double)hi;
+            wsq = __fmaf_rn(hi, hi, __fmaf_rn(lo, lo, wsq));
         }
     };
 
@@ -126,8 +128,8 @@ __global__ void __launch_bounds__(RT_THREADS) router_logits_kernel(RouterLogitsA
             } else {
                 xr[0] = xs[buf][h][tg];
             }
-            const float4 wa = *reinterpret_cast<const float4*>(&ws[buf][h][8 * eg]);
-            const float4 wb = *reinterpret_cast<const float4*>(&ws[buf][h][8 * eg + 4]);
+            const float4 wa = *reinterpret_cast<const float4*>(&ws[buf][h][4 * eg]);
+            const float4 wb = *reinterpret_cast<const float4*>(&ws[buf][h][64 + 4 * eg]);
             const float wr8[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
             for (int i = 0; i < TPT; ++i)
@@ -146,19 +148,19 @@ __global__ void __launch_bounds__(RT_THREADS) router_logits_kernel(RouterLogitsA
         if (t >= a.T) continue;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            const int e = e0 + 8 * eg + j;
+            const int e = e0 + (j < 4 ? 4 * eg + j : 64 + 4 * eg + j - 4);
             if (e < a.E) a.P[((int64_t)s * a.T + t) * a.E + e] = acc[i * 8 + j];
         }
     }
 
     // squared norms of this split's range: the two halves of a row sit in adjacent lanes
-    xsq += __shfl_xor_sync(0xffffffffu, xsq, 1);
-    wsq += __shfl_xor_sync(0xffffffffu, wsq, 1);
+    xsq = __fadd_rn(xsq, __shfl_xor_sync(0xffffffffu, xsq, 1));
+    wsq = __fadd_rn(wsq, __shfl_xor_sync(0xffffffffu, wsq, 1));
     if (l_half == 0) {
         const int64_t t = t0 + l_row;
-        if (blockIdx.y == 0 && tid < 2 * RT_TT && t < a.T) a.xn2[(int64_t)s * a.T + t] = xsq;
+        if (blockIdx.y == 0 && tid < 2 * RT_TT && t < a.T) a.xn2[(int64_t)s * a.T + t] = (double)xsq;
         const int e = e0 + l_row;
-        if (blockIdx.x == 0 && e < a.E) a.wn2[(int64_t)s * a.E + e] = wsq;
+        if (blockIdx.x == 0 && e < a.E) a.wn2[(int64_t)s * a.E + e] = (double)wsq;
     }
 }
 
@@ -234,15 +236,61 @@ __device__ long long exact_logit(const uint16_t* xr, const uint16_t* wrow, int H
 // their candidates in a block-wide list whose exact logits all 8 warps
 // compute together, then finish their selection from it.
 __global__ void __launch_bounds__(TK_WARPS * 32, 2) router_topk_kernel(RouterTopkArgs a, DevCtx ctx) {
-    __shared__ int c_tok[TK_CAP];
-    __shared__ int c_e[TK_CAP];
+    __shared__ uint8_t c_tok[TK_CAP];
+    __shared__ uint16_t c_e[TK_CAP];
     __shared__ long long c_val[TK_CAP];
+    __shared__ double Ls[TK_WARPS][256];   // sum over splits of the partial logits
+    __shared__ double Qs[256];             // sum over splits of ||w_e||^2
+    __shared__ double Xs[TK_WARPS];        // sum over splits of ||x||^2
     __shared__ int n_cand;
 
     const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
-    const int64_t t = (int64_t)blockIdx.x * TK_WARPS + warp;
+    const int64_t t_base = (int64_t)blockIdx.x * TK_WARPS;
+    const int64_t t = t_base + warp;
     const bool active = t < a.T;
     if (threadIdx.x == 0) n_cand = 0;
+    // the block's (token, expert) partial sums: consecutive threads take
+    // consecutive experts, and every load is independent of the others
+    {
+        const int n_tok = (int)min((int64_t)TK_WARPS, a.T - t_base);
+        const int pairs = n_tok * a.E;
+        const int64_t stride = a.T * a.E;
+        for (int i0 = threadIdx.x; i0 < pairs; i0 += 4 * TK_WARPS * 32) {
+            // four pairs per thread, their loads for every split issued together
+            int64_t off[4];
+            bool ok[4];
+            double acc[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int i = i0 + k * TK_WARPS * 32;
+                ok[k] = i < pairs;
+                const int w = ok[k] ? i / a.E : 0, e = ok[k] ? i % a.E : 0;
+                off[k] = (t_base + w) * a.E + e;
+                acc[k] = 0.0;
+            }
+#pragma unroll 8
+            for (int s = 0; s < a.S; ++s) {
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    if (ok[k]) acc[k] += a.P[(int64_t)s * stride + off[k]];
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int i = i0 + k * TK_WARPS * 32;
+                if (ok[k]) Ls[i / a.E][i % a.E] = acc[k];
+            }
+        }
+        for (int e = threadIdx.x; e < a.E; e += TK_WARPS * 32) {
+            double q = 0.0;
+            for (int s = 0; s < a.S; ++s) q += a.wn2[(int64_t)s * a.E + e];
+            Qs[e] = q;
+        }
+        if (threadIdx.x < n_tok) {
+            double q = 0.0;
+            for (int s = 0; s < a.S; ++s) q += a.xn2[(int64_t)s * a.T + t_base + threadIdx.x];
+            Xs[threadIdx.x] = q;
+        }
+    }
     __syncthreads();
 
     const int nj = (a.E + 31) / 32;
@@ -256,45 +304,21 @@ __global__ void __launch_bounds__(TK_WARPS * 32, 2) router_topk_kernel(RouterTop
     int out_e[16];
     double out_l[16];
     if (active) {
-        // partial logits and weight norms of every split: coalesced rows of E,
-        // loaded in groups of 8 splits with no dependence between the loads
-        double lsum[TK_MAXJ], qsum[TK_MAXJ];
-        double xn2 = 0.0;
-#pragma unroll
-        for (int j = 0; j < TK_MAXJ; ++j) lsum[j] = qsum[j] = 0.0;
-        for (int s0 = 0; s0 < a.S; s0 += 8) {
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int s = s0 + u;
-                if (s < a.S) {
-                    xn2 += a.xn2[(int64_t)s * a.T + t];
-                    const double* prow = a.P + ((int64_t)s * a.T + t) * a.E;
-                    const double* wrow = a.wn2 + (int64_t)s * a.E;
-#pragma unroll
-                    for (int j = 0; j < TK_MAXJ; ++j) {
-                        const int e = lane + 32 * j;
-                        if (j < nj && e < a.E) {
-                            lsum[j] += prow[e];
-                            qsum[j] += wrow[e];
-                        }
-                    }
-                }
-            }
-        }
-        const double xnorm = sqrt(xn2);
+        const double kNorm = 1.0 + (double)(a.H + 64) * 0x1p-23;   // fp32 norm sums -> upper bounds
+        const double xnorm = sqrt(Xs[warp] * kNorm);
         double eps_star = 0.0;
 #pragma unroll
         for (int j = 0; j < TK_MAXJ; ++j) {
             L[j] = -DBL_MAX;
             const int e = lane + 32 * j;
             if (j < nj && e < a.E) {
-                double l = lsum[j];
+                double l = Ls[warp][e];
                 if (a.bias) {
                     const double b = (double)a.bias[e];
                     if (fabs(b) >= 0x1p21) range_bad = true;
                     l += b;
                 }
-                const double wnorm = sqrt(qsum[j]);
+                const double wnorm = sqrt(Qs[e] * kNorm);
                 if (xnorm * wnorm >= 0x1p22) range_bad = true;
                 eps_star = fmax(eps_star, kRel * xnorm * wnorm + kFx + fabs(l) * 0x1p-50);
                 L[j] = l;
@@ -343,8 +367,8 @@ __global__ void __launch_bounds__(TK_WARPS * 32, 2) router_topk_kernel(RouterTop
                 base = __shfl_sync(0xffffffffu, base, 0);
                 if (c) {
                     const int i = base + __popc(m & ((1u << lane) - 1u));
-                    c_tok[i] = warp;
-                    c_e[i] = e;
+                    c_tok[i] = (uint8_t)warp;
+                    c_e[i] = (uint16_t)e;
                 }
             }
         }
@@ -365,7 +389,7 @@ __global__ void __launch_bounds__(TK_WARPS * 32, 2) router_topk_kernel(RouterTop
             long long bv = LLONG_MIN;
             int be = 0x7fffffff, bi = -1;
             for (int i = lane; i < nc; i += 32) {
-                if (c_tok[i] != warp) continue;
+                if (c_tok[i] != warp) continue;   // other tokens, or already taken (0xFF)
                 const long long v = c_val[i];
                 const int e = c_e[i];
                 if (bi < 0 || v > bv || (v == bv && e < be)) {
@@ -376,7 +400,7 @@ __global__ void __launch_bounds__(TK_WARPS * 32, 2) router_topk_kernel(RouterTop
             }
             int src_e = be;
             warp_argmax_i64(bv, src_e);
-            if (bi >= 0 && be == src_e) c_tok[bi] = -1;   // taken (this lane held it)
+            if (bi >= 0 && be == src_e) c_tok[bi] = 0xFF;   // taken (this lane held it)
             __syncwarp();
             out_e[k] = src_e;
             out_l[k] = (double)bv * 0x1p-40;
