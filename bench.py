@@ -436,6 +436,9 @@ def run_native(args):
         barrier = lambda: None
     device = torch.device("cuda", torch.cuda.current_device())
     peaks, peak_kind = load_peaks()
+    if args.gemm == "pair":
+        import routed_expert_moe_b200 as moe
+        moe.debug_set(3, 1)
 
     wl = W.WORKLOADS[WORKLOADS[args.workload]]
     layer = Chain(wl, device) if wl.layers > 1 else Layer(wl, device)
@@ -486,7 +489,8 @@ def run_native(args):
                        "l2": "inputs larger than L2: the touched experts' weights "
                              f"({touched * wl.F * wl.H * (2 if wl.fp8 else 4) * wl.layers / 1e9:.2f} GB) "
                              "stream from HBM every step; token batches rotate; no flush",
-                       "parallelism": f"dp{ws} (independent token batches per GPU, weights replicated)"},
+                       "parallelism": f"dp{ws} (independent token batches per GPU, weights replicated)",
+                       "grouped_gemm": "cta_pair" if args.gemm == "pair" else "single_cta"},
             "roofline": roofline_entry(wl, stages, touched, peaks, peak_kind, args.workload),
             "stages_ms": stages,
             "e2e": {"value": job_value(ws, wl.T * wl.layers, args.steps, e2e_ms), "unit": UNIT,
@@ -543,6 +547,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--gemm", choices=["single", "pair"], default="single",
+                    help="grouped GEMM on single CTAs, or on CTA pairs for tiles of more than 64 tokens")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

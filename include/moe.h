@@ -188,10 +188,20 @@ moe_status moe_check_device_error(void* stream);
 #define MOE_STAGE_EVENTS 8
 moe_status moe_set_stage_events(void* const* events, int32_t n);
 
-/* Test hooks of the failure-detection tests.  what = 1: limit of every
- * bounded wait in nanoseconds (value <= 0 restores the default of 4 s);
- * what = 2: the grouped-GEMM producer of block 0 withholds its first load
- * (value 1) so the consumer's wait must expire; 0 turns it off. */
+/* Test and measurement hooks (host state shared by all threads).
+ * what = 1: limit of every bounded wait in nanoseconds (value <= 0 restores
+ * the default of 4 s); what = 2: the grouped-GEMM producer of block 0
+ * withholds its first load (value 1) so the consumer's wait must expire;
+ * 0 turns it off; what = 3: value 1 runs the grouped GEMMs of batches with
+ * tiles of more than 64 tokens on CTA pairs (cta_group::2, M = 256), value 0
+ * (the default) on single CTAs; what = 4: largest batch (tokens) that the
+ * router computes in one launch of 8-CTA clusters split over the experts (0:
+ * never; value < 0 restores the default of 256); what = 5: router of the
+ * larger batches: 0 (the default) by batch size (one launch of clusters split
+ * over the hidden dimension from 3072 tokens when E <= 128, else the tiled
+ * logits kernel and the top-K kernel), 1 always the two kernels, 2 always the
+ * hidden-split clusters when E <= 128; other values MOE_EINVAL.  Other `what`:
+ * MOE_EINVAL. */
 moe_status moe_debug_set(int32_t what, int64_t value);
 
 #ifdef __cplusplus

@@ -15,6 +15,7 @@ namespace moe {
 struct RouterPlan {
     int S;
     int nchunks;
+    int num_sms;
     size_t p_bytes, xn_bytes, wn_bytes;
 };
 RouterPlan router_plan(int64_t T, int H, int E, int num_sms);
@@ -25,6 +26,8 @@ cudaError_t launch_route(const uint16_t* x, const uint16_t* wr, const float* bia
 cudaError_t launch_permute(const int32_t* idx, int64_t n, int E, int32_t* counts, int32_t* offsets,
                            int32_t* perm_src, int32_t* inv_row, int4* sched, int* n_sched, int bn,
                            int* scratch, const DevCtx& ctx, cudaStream_t stream);
+void set_router_small_max(int64_t v);
+void set_router_split(int v);
 size_t permute_scratch_ints(int64_t n, int E);
 size_t permute_smem_bytes(int E);
 cudaError_t launch_schedule(const int32_t* offsets, int E, int bn, int4* sched, int* n_sched,
@@ -43,6 +46,10 @@ cudaError_t launch_grouped_gemm(bool fp8, bool up, const void* W, int E, int Nou
                                 int64_t rows, const int4* sched, const int* n_sched, const GemmPlan& plan,
                                 void* out, const float* w_scale, float in_scale, float out_scale, int num_sms,
                                 int debug_withhold, const DevCtx& ctx, cudaStream_t stream);
+cudaError_t launch_grouped_gemm_pair(bool fp8, bool up, const void* W, int E, int Nout, int Kdim, const void* act,
+                                     int64_t rows, const int4* sched, const int* n_sched, int bn, int max_sched,
+                                     void* out, const float* w_scale, float in_scale, float out_scale,
+                                     int num_sms, const DevCtx& ctx, cudaStream_t stream);
 cudaError_t launch_combine(const uint16_t* yp, const int32_t* inv_row, const float* w, const uint16_t* residual,
                            uint16_t* out, int64_t T, int K, int H, int num_sms, const DevCtx& ctx,
                            cudaStream_t stream);
@@ -63,6 +70,7 @@ namespace {
 constexpr uint64_t kDefaultTimeoutNs = 4000000000ull;
 std::atomic<uint64_t> g_timeout_ns{kDefaultTimeoutNs};
 std::atomic<int> g_debug_withhold{0};
+std::atomic<int> g_gemm_pair{0};
 void* g_stage_events[MOE_STAGE_EVENTS] = {};
 std::atomic<int> g_stage_events_on{0};
 
@@ -225,15 +233,27 @@ moe_status run_ffn(const moe_dims* d, const DeviceInfo* dev, const DevCtx& ctx, 
                                   fp8 ? sc->x_scale : 1.0f, dev->num_sms, ctx, st);
     if (e != cudaSuccess) return cuda_status(e);
     const int withhold = g_debug_withhold.load();
+    // optional: tiles of more than 64 tokens on CTA pairs (one activation read per 256 weight rows)
+    const bool pair = g_gemm_pair.load() && gp.bn > 64 && !withhold;
     if (marks) stage_mark(4, st);
-    e = launch_grouped_gemm(fp8, true, w_up, d->E, d->F, d->H, fw.xp, rows, fw.sched, fw.n_sched, gp, fw.hb,
-                            fp8 ? sc->w_up_scale : nullptr, fp8 ? sc->x_scale : 1.0f, fp8 ? sc->h_scale : 1.0f,
-                            dev->num_sms, withhold, ctx, st);
+    if (pair)
+        e = launch_grouped_gemm_pair(fp8, true, w_up, d->E, d->F, d->H, fw.xp, rows, fw.sched, fw.n_sched, gp.bn,
+                                     gp.max_sched, fw.hb, fp8 ? sc->w_up_scale : nullptr, fp8 ? sc->x_scale : 1.0f,
+                                     fp8 ? sc->h_scale : 1.0f, dev->num_sms, ctx, st);
+    else
+        e = launch_grouped_gemm(fp8, true, w_up, d->E, d->F, d->H, fw.xp, rows, fw.sched, fw.n_sched, gp, fw.hb,
+                                fp8 ? sc->w_up_scale : nullptr, fp8 ? sc->x_scale : 1.0f, fp8 ? sc->h_scale : 1.0f,
+                                dev->num_sms, withhold, ctx, st);
     if (e != cudaSuccess) return cuda_status(e);
     if (marks) stage_mark(5, st);
-    e = launch_grouped_gemm(fp8, false, w_down, d->E, d->H, d->F, fw.hb, rows, fw.sched, fw.n_sched, gp, y_perm,
-                            fp8 ? sc->w_down_scale : nullptr, fp8 ? sc->h_scale : 1.0f, 1.0f, dev->num_sms, 0,
-                            ctx, st);
+    if (pair)
+        e = launch_grouped_gemm_pair(fp8, false, w_down, d->E, d->H, d->F, fw.hb, rows, fw.sched, fw.n_sched, gp.bn,
+                                     gp.max_sched, y_perm, fp8 ? sc->w_down_scale : nullptr,
+                                     fp8 ? sc->h_scale : 1.0f, 1.0f, dev->num_sms, ctx, st);
+    else
+        e = launch_grouped_gemm(fp8, false, w_down, d->E, d->H, d->F, fw.hb, rows, fw.sched, fw.n_sched, gp, y_perm,
+                                fp8 ? sc->w_down_scale : nullptr, fp8 ? sc->h_scale : 1.0f, 1.0f, dev->num_sms, 0,
+                                ctx, st);
     return cuda_status(e);
 }
 
@@ -466,6 +486,19 @@ moe_status moe_debug_set(int32_t what, int64_t value) {
     }
     if (what == 2) {
         g_debug_withhold.store(value ? 1 : 0);
+        return MOE_OK;
+    }
+    if (what == 3) {
+        g_gemm_pair.store(value ? 1 : 0);
+        return MOE_OK;
+    }
+    if (what == 4) {
+        set_router_small_max(value);
+        return MOE_OK;
+    }
+    if (what == 5) {
+        if (value < 0 || value > 2) return MOE_EINVAL;
+        set_router_split((int)value);
         return MOE_OK;
     }
     return MOE_EINVAL;

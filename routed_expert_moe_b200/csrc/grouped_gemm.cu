@@ -17,8 +17,8 @@
 // Roles (192 threads):
 //   warp 0      TMA producer (one thread): per 128-byte K slice the weight
 //               tile (one 128-row box, or a 64-row box for the last block of
-//               a 1856-row expert) and the expert's rows (64-row boxes, then
-//               16-row boxes for the remainder), both in the 128-byte swizzle,
+//               a 1856-row expert) and the expert's rows (128-, 64- and 16-row
+//               boxes, largest first), both in the 128-byte swizzle,
 //               into an NS-deep smem ring.  Few, large copies per stage: the
 //               copy engine's per-request cost, not bytes, is what limits a
 //               ring of many small boxes;
@@ -63,6 +63,7 @@ struct GemmArgs {
 struct GemmMaps {
     CUtensorMap a128;        // weights, 128-row box
     CUtensorMap a64;         // weights, 64-row box
+    CUtensorMap b128;        // activations, 128-row box
     CUtensorMap b64;         // activations, 64-row box
     CUtensorMap b16;         // activations, 16-row box
 };
@@ -102,6 +103,7 @@ __global__ void __launch_bounds__(GG_THREADS, 1)
         fence_mbar_init();
         tma_prefetch_desc(&maps.a128);
         tma_prefetch_desc(&maps.a64);
+        tma_prefetch_desc(&maps.b128);
         tma_prefetch_desc(&maps.b64);
         tma_prefetch_desc(&maps.b16);
     }
@@ -126,7 +128,7 @@ __global__ void __launch_bounds__(GG_THREADS, 1)
                 const int mb = u % g.m_blocks;
                 const bool a_full = g.Nout - mb * GG_BM > 64;
                 const int n16 = (sc.z + 15) / 16;         // 16-row groups of activations
-                const int n64 = n16 / 4, r16 = n16 % 4;
+                const int n128 = n16 / 8, n64 = (n16 % 8) / 4, r16 = n16 % 4;
                 const uint32_t bytes = (uint32_t)((a_full ? 128 : 64) * GG_ROW_BYTES + n16 * 16 * GG_ROW_BYTES);
                 const int a_y = sc.x * g.Nout + mb * GG_BM;
                 for (int ks = 0; ks < g.k_stages; ++ks) {
@@ -143,11 +145,13 @@ __global__ void __launch_bounds__(GG_THREADS, 1)
                         const uint32_t a_dst = smem_u32(smA + (size_t)stage * GG_A_BYTES);
                         const uint32_t b_dst = smem_u32(smB + (size_t)stage * g.b_stage_bytes);
                         tma_load_2d(a_dst, a_full ? &maps.a128 : &maps.a64, fb, kx, a_y, pol_w);
-                        for (int j = 0; j < n64; ++j)
-                            tma_load_2d(b_dst + j * 64 * GG_ROW_BYTES, &maps.b64, fb, kx, sc.y + j * 64, pol_x);
-                        for (int j = 0; j < r16; ++j)
-                            tma_load_2d(b_dst + (n64 * 4 + j) * 16 * GG_ROW_BYTES, &maps.b16, fb, kx,
-                                        sc.y + (n64 * 4 + j) * 16, pol_x);
+                        int row = 0;
+                        for (int j = 0; j < n128; ++j, row += 128)
+                            tma_load_2d(b_dst + row * GG_ROW_BYTES, &maps.b128, fb, kx, sc.y + row, pol_x);
+                        for (int j = 0; j < n64; ++j, row += 64)
+                            tma_load_2d(b_dst + row * GG_ROW_BYTES, &maps.b64, fb, kx, sc.y + row, pol_x);
+                        for (int j = 0; j < r16; ++j, row += 16)
+                            tma_load_2d(b_dst + row * GG_ROW_BYTES, &maps.b16, fb, kx, sc.y + row, pol_x);
                     }
                     if (++stage == NS) {
                         stage = 0;
@@ -225,6 +229,8 @@ __global__ void __launch_bounds__(GG_THREADS, 1)
             const bool fvalid = f < g.Nout;
             float scale = 1.0f;
             if constexpr (FP8) scale = __fmul_rn(g.w_scale[sc.x], g.in_scale);
+            // E4M3 codes of the ReLU^2 tensor: a * (1 / h_scale), the reciprocal correctly rounded
+            const float inv_out = (FP8 && UP) ? __frcp_rn(g.out_scale) : 1.0f;
             const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * 256);
             const int nchunks = (sc.z + 15) / 16;
             for (int c = 0; c < nchunks; ++c) {
@@ -242,7 +248,7 @@ __global__ void __launch_bounds__(GG_THREADS, 1)
                                 const float a = z > 0.0f ? __fmul_rn(z, z) : 0.0f;
                                 if constexpr (FP8) {
                                     static_cast<uint8_t*>(g.out)[o] = (uint8_t)__nv_cvt_float_to_fp8(
-                                        __fdiv_rn(a, g.out_scale), __NV_SATFINITE, __NV_E4M3);
+                                        __fmul_rn(a, inv_out), __NV_SATFINITE, __NV_E4M3);
                                 } else {
                                     static_cast<__nv_bfloat16*>(g.out)[o] = __float2bfloat16_rn(a);
                                 }
@@ -352,7 +358,8 @@ cudaError_t launch_grouped_gemm(bool fp8, bool up, const void* W, int E, int Nou
     GemmMaps maps;
     if (!make_map(&maps.a128, W, (int64_t)E * Nout, Kdim, fp8, 128) ||
         !make_map(&maps.a64, W, (int64_t)E * Nout, Kdim, fp8, 64) ||
-        !make_map(&maps.b64, act, rows, Kdim, fp8, 64) || !make_map(&maps.b16, act, rows, Kdim, fp8, 16))
+        !make_map(&maps.b128, act, rows, Kdim, fp8, 128) || !make_map(&maps.b64, act, rows, Kdim, fp8, 64) ||
+        !make_map(&maps.b16, act, rows, Kdim, fp8, 16))
         return cudaErrorInvalidValue;
     GemmArgs g;
     g.sched = sched;

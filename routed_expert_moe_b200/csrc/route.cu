@@ -26,6 +26,8 @@
 #include <cstdint>
 #include <cfloat>
 #include <climits>
+#include <atomic>
+#include <cooperative_groups.h>
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -172,7 +174,7 @@ struct RouterTopkArgs {
     const uint16_t* wr;
     const float* bias;    // [E] or null
     int64_t T;
-    int H, E, K, S;
+    int H, E, K, S, nchunks;
     int32_t* idx;         // [T][K]
     float* w;             // [T][K]
 };
@@ -208,28 +210,258 @@ __device__ __forceinline__ void warp_argmax_i64(long long& v, int& e) {
 
 // Exact fixed-point logit (units of 2^-40) of expert e for token row xr:
 // every bf16 product (exact in fp32) scaled by 2^40 and rounded to the
-// nearest integer, summed exactly; 16-byte loads, one warp.
+// nearest integer, summed exactly; one warp, 16-byte loads issued eight
+// fragments per lane at a time so that their latencies overlap.
 __device__ long long exact_logit(const uint16_t* xr, const uint16_t* wrow, int H, const float* bias, int e,
                                  int lane) {
+    constexpr int B = 8;
     const uint4* xv = reinterpret_cast<const uint4*>(xr);
     const uint4* wv = reinterpret_cast<const uint4*>(wrow);
+    const int nv = H / 8;
     long long acc = 0;
-    for (int v = lane; v < H / 8; v += 32) {
-        const uint4 a = xv[v], b = wv[v];
-        const uint32_t aa[4] = {a.x, a.y, a.z, a.w};
-        const uint32_t bb[4] = {b.x, b.y, b.z, b.w};
+    for (int v0 = lane; v0 < nv; v0 += 32 * B) {
+        uint4 a[B], b[B];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const float p0 = __fmul_rn(__uint_as_float(aa[j] << 16), __uint_as_float(bb[j] << 16));
-            const float p1 = __fmul_rn(__uint_as_float(aa[j] & 0xFFFF0000u), __uint_as_float(bb[j] & 0xFFFF0000u));
-            acc += __float2ll_rn(__fmul_rn(p0, 0x1p40f));
-            acc += __float2ll_rn(__fmul_rn(p1, 0x1p40f));
+        for (int i = 0; i < B; ++i) {
+            const int v = v0 + 32 * i;
+            a[i] = b[i] = make_uint4(0, 0, 0, 0);
+            if (v < nv) {
+                a[i] = xv[v];
+                b[i] = wv[v];
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < B; ++i) {
+            const uint32_t aa[4] = {a[i].x, a[i].y, a[i].z, a[i].w};
+            const uint32_t bb[4] = {b[i].x, b[i].y, b[i].z, b[i].w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float p0 = __fmul_rn(__uint_as_float(aa[j] << 16), __uint_as_float(bb[j] << 16));
+                const float p1 =
+                    __fmul_rn(__uint_as_float(aa[j] & 0xFFFF0000u), __uint_as_float(bb[j] & 0xFFFF0000u));
+                acc += __float2ll_rn(__fmul_rn(p0, 0x1p40f));
+                acc += __float2ll_rn(__fmul_rn(p1, 0x1p40f));
+            }
         }
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
     if (bias) acc += __float2ll_rn(__fmul_rn(bias[e], 0x1p40f));
     return acc;
+}
+
+constexpr int TK_MAXK = 16;       // K <= 16
+
+// Relative bound of an approximate logit l~ (in units of ||x|| ||w_e||, which
+// bounds sum_h |x_h w_eh| by Cauchy-Schwarz) for a summation whose fp32 part
+// rounds at most n32 times along any product's path (g_n32, u = 2^-24) and
+// whose fp64 part adds at most d64 times (d64 2^-52 >= g_d64 at u = 2^-53);
+// 2^-40 is slack for the roundings of the bound's own arithmetic.
+__host__ __device__ inline double router_k_rel(int n32, int d64) {
+    const double g = (double)n32 * 0x1p-24;
+    return g / (1.0 - g) + (double)d64 * 0x1p-52 + 0x1p-40;
+}
+
+// Order-preserving integer key of a double (unsigned order = numeric order;
+// -0 is mapped with +0 by adding 0.0 first).
+__device__ __forceinline__ unsigned long long order_key(double v) {
+    const unsigned long long u = (unsigned long long)__double_as_longlong(v + 0.0);
+    return (u >> 63) ? ~u : (u | 0x8000000000000000ull);
+}
+__device__ __forceinline__ double key_value(unsigned long long k) {
+    return __longlong_as_double((long long)((k >> 63) ? (k & 0x7fffffffffffffffull) : ~k));
+}
+
+// warp arg-max of (key, -index)
+__device__ __forceinline__ void warp_argmax_key(unsigned long long& k, int& e) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        const unsigned long long ok = __shfl_xor_sync(0xffffffffu, k, off);
+        const int oe = __shfl_xor_sync(0xffffffffu, e, off);
+        if (ok > k || (ok == k && oe < e)) {
+            k = ok;
+            e = oe;
+        }
+    }
+}
+
+// Per-block constants of the bound: the largest ||w_e|| (from the fp32 squared
+// norms Q, inflated by 1 + (H+64) 2^-23 to an upper bound) and the largest
+// |b_e|.  One warp; every lane returns both.
+__device__ __forceinline__ void bound_constants(const double* Q, const float* bias, int H, int E, int lane,
+                                                double& wnmax, double& bmax) {
+    double q = 0.0, b = 0.0;
+    for (int e = lane; e < E; e += 32) {
+        q = fmax(q, Q[e]);
+        if (bias) b = fmax(b, fabs((double)bias[e]));
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        q = fmax(q, __shfl_xor_sync(0xffffffffu, q, off));
+        b = fmax(b, __shfl_xor_sync(0xffffffffu, b, off));
+    }
+    wnmax = sqrt(q * (1.0 + (double)(H + 64) * 0x1p-23));
+    bmax = b;
+}
+
+// Ranks one token's approximate logits l~ (one warp, E <= 256): the K best
+// (ties to the lower index) into out_e/out_l (shared memory of this token,
+// written by lane 0), and whether every gap among the K+1 best exceeds
+// 2 eps*.  When it does not, the token's candidates (every expert whose exact
+// logit could still be in the top K) are appended to the block's list under
+// `slot`.  With k_rel bounding |l~ - l| / (||x|| ||w_e||) for the caller's
+// summation (see router_k_rel),
+//   eps* = k_rel ||x|| max_e ||w_e|| + (H+1) 2^-41 + (2 ||x|| max_e ||w_e|| + max_e |b_e| + 1) 2^-50
+// bounds every |l~_e - l_e| (the last term covers the fp64 roundings of l~ + b).
+// The ranking compares order-preserving integer keys of l~.
+__device__ __forceinline__ bool rank_certified(const double* Lrow, double xsq, const float* bias, int H, int E,
+                                               int K, double k_rel, double wnmax, double bmax, int lane, int slot,
+                                               int* out_e, double* out_l, bool& range_bad, uint8_t* c_tok,
+                                               uint16_t* c_e, int* n_cand) {
+    const int nj = (E + 31) / 32;
+    const double xnorm = sqrt(xsq * (1.0 + (double)(H + 64) * 0x1p-23));   // fp32 norm sum -> upper bound
+    const double xw = xnorm * wnmax;
+    if (xw >= 0x1p22 || bmax >= 0x1p21) range_bad = true;
+    const double eps_star = k_rel * xw + (double)(H + 1) * 0x1p-41 + (2.0 * xw + bmax + 1.0) * 0x1p-50;
+
+    // the lane's keys, sorted once by (key, -e) descending (empty slots: key 0, below every real key)
+    unsigned long long sk[TK_MAXJ];
+    int se[TK_MAXJ];
+#pragma unroll
+    for (int j = 0; j < TK_MAXJ; ++j) {
+        const int e = lane + 32 * j;
+        sk[j] = 0ull;
+        se[j] = e;
+        if (j < nj && e < E) {
+            double l = Lrow[e];
+            if (bias) l += (double)bias[e];
+            sk[j] = order_key(l);
+        }
+    }
+    auto cx = [&](int i, int j) {   // (i, j) in descending order after the exchange
+        const bool sw = sk[i] < sk[j] || (sk[i] == sk[j] && se[i] > se[j]);
+        const unsigned long long tk = sw ? sk[j] : sk[i];
+        const int te = sw ? se[j] : se[i];
+        sk[j] = sw ? sk[i] : sk[j];
+        se[j] = sw ? se[i] : se[j];
+        sk[i] = tk;
+        se[i] = te;
+    };
+    // Batcher's odd-even merge sort of 8
+    cx(0, 1); cx(2, 3); cx(4, 5); cx(6, 7);
+    cx(0, 2); cx(1, 3); cx(4, 6); cx(5, 7);
+    cx(1, 2); cx(5, 6);
+    cx(0, 4); cx(1, 5); cx(2, 6); cx(3, 7);
+    cx(2, 4); cx(3, 5);
+    cx(1, 2); cx(3, 4); cx(5, 6);
+
+    // the K+1 best by l~ (ties to the lower index): the best of the lanes' heads, popped
+    const int nsel = min(K + 1, E);
+    double prev = 0.0, lk = 0.0;
+    bool certified = true;
+    for (int k = 0; k < nsel; ++k) {
+        unsigned long long bk = sk[0];
+        int be = se[0];
+        warp_argmax_key(bk, be);
+        const double bv = key_value(bk);
+        if (k < K) {
+            if (lane == 0) {
+                out_e[k] = be;
+                out_l[k] = bv;
+            }
+            lk = bv;
+        }
+        if (k > 0 && !(prev - bv > 2.0 * eps_star)) certified = false;
+        prev = bv;
+        if ((be & 31) == lane) {
+#pragma unroll
+            for (int j = 0; j + 1 < TK_MAXJ; ++j) {
+                sk[j] = sk[j + 1];
+                se[j] = se[j + 1];
+            }
+            sk[TK_MAXJ - 1] = 0ull;
+        }
+    }
+    if (!certified) {
+        // candidates: every expert that could still be in the exact top K
+        const unsigned long long thr = order_key(lk - 2.0 * eps_star);
+#pragma unroll
+        for (int j = 0; j < TK_MAXJ; ++j) {
+            const int e = lane + 32 * j;
+            bool c = false;
+            if (j < nj && e < E) {
+                double l = Lrow[e];
+                if (bias) l += (double)bias[e];
+                c = order_key(l) >= thr;
+            }
+            const uint32_t m = __ballot_sync(0xffffffffu, c);
+            int base = 0;
+            if (lane == 0 && m) base = atomicAdd(n_cand, __popc(m));
+            base = __shfl_sync(0xffffffffu, base, 0);
+            if (c) {
+                const int i = base + __popc(m & ((1u << lane) - 1u));
+                c_tok[i] = (uint8_t)slot;
+                c_e[i] = (uint16_t)e;
+            }
+        }
+    }
+    __syncwarp();
+    return certified;
+}
+
+// Exact fixed-point logits of the block's listed candidates, one warp each;
+// token slot s of the list is token t_base + s.
+__device__ __forceinline__ void exact_candidates(int nc, const uint8_t* c_tok, const uint16_t* c_e,
+                                                 long long* c_val, int64_t t_base, const uint16_t* x,
+                                                 const uint16_t* wr, int H, const float* bias, int warp,
+                                                 int n_warps, int lane) {
+    for (int i = warp; i < nc; i += n_warps) {
+        const int e = c_e[i];
+        const long long v = exact_logit(x + (t_base + c_tok[i]) * H, wr + (int64_t)e * H, H, bias, e, lane);
+        if (lane == 0) c_val[i] = v;
+    }
+}
+
+// Finishes one token (one warp): if its order was not certified, ranks its
+// candidates by exact logit (ties to the lower index) into out_e/out_l; then
+// the renormalised softmax over the K kept logits (w_k = exp(l_k - l_0) / z,
+// z summed in order k = 0..K-1), and the K (index, weight) pairs of row t.
+__device__ __forceinline__ void finish_token(bool certified, int slot, int64_t t, int nc, uint8_t* c_tok,
+                                             const uint16_t* c_e, const long long* c_val, int K, int* out_e,
+                                             double* out_l, int lane, int32_t* idx, float* w) {
+    if (!certified) {
+        for (int k = 0; k < K; ++k) {
+            long long bv = LLONG_MIN;
+            int be = 0x7fffffff, bi = -1;
+            for (int i = lane; i < nc; i += 32) {
+                if (c_tok[i] != slot) continue;   // other tokens, or already taken (0xFF)
+                const long long v = c_val[i];
+                const int e = c_e[i];
+                if (bi < 0 || v > bv || (v == bv && e < be)) {
+                    bv = v;
+                    be = e;
+                    bi = i;
+                }
+            }
+            int src_e = be;
+            warp_argmax_i64(bv, src_e);
+            if (bi >= 0 && be == src_e) c_tok[bi] = 0xFF;   // taken (this lane held it)
+            if (lane == 0) {
+                out_e[k] = src_e;
+                out_l[k] = (double)bv * 0x1p-40;
+            }
+            __syncwarp();
+        }
+    }
+    // lane k < K holds term k
+    const double l0 = out_l[0];
+    const float ex = lane < K ? expf((float)(out_l[lane < K ? lane : 0] - l0)) : 0.0f;
+    float z = 0.0f;
+    for (int k = 0; k < K; ++k) z += __shfl_sync(0xffffffffu, ex, k);
+    if (lane < K) {
+        idx[t * K + lane] = out_e[lane];
+        w[t * K + lane] = ex / z;
+    }
 }
 
 // One warp per token ranks l~; tokens whose order the bound leaves open put
@@ -242,6 +474,9 @@ __global__ void __launch_bounds__(TK_WARPS * 32, 2) router_topk_kernel(RouterTop
     __shared__ double Ls[TK_WARPS][256];   // sum over splits of the partial logits
     __shared__ double Qs[256];             // sum over splits of ||w_e||^2
     __shared__ double Xs[TK_WARPS];        // sum over splits of ||x||^2
+    __shared__ int s_oe[TK_WARPS][TK_MAXK];
+    __shared__ double s_ol[TK_WARPS][TK_MAXK];
+    __shared__ double s_bound[2];
     __shared__ int n_cand;
 
     const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
@@ -293,138 +528,571 @@ __global__ void __launch_bounds__(TK_WARPS * 32, 2) router_topk_kernel(RouterTop
     }
     __syncthreads();
 
-    const int nj = (a.E + 31) / 32;
-    // g_16 + 2^-45 (fp64 sums of the chunk and split partials), with slack for the norm sums
-    const double kRel = (16.0 * 0x1p-24) / (1.0 - 16.0 * 0x1p-24) + 0x1p-45 + 0x1p-40;
-    const double kFx = (double)(a.H + 1) * 0x1p-41;
-
-    double L[TK_MAXJ];
-    bool certified = true;
-    bool range_bad = false;
-    int out_e[16];
-    double out_l[16];
-    if (active) {
-        const double kNorm = 1.0 + (double)(a.H + 64) * 0x1p-23;   // fp32 norm sums -> upper bounds
-        const double xnorm = sqrt(Xs[warp] * kNorm);
-        double eps_star = 0.0;
-#pragma unroll
-        for (int j = 0; j < TK_MAXJ; ++j) {
-            L[j] = -DBL_MAX;
-            const int e = lane + 32 * j;
-            if (j < nj && e < a.E) {
-                double l = Ls[warp][e];
-                if (a.bias) {
-                    const double b = (double)a.bias[e];
-                    if (fabs(b) >= 0x1p21) range_bad = true;
-                    l += b;
-                }
-                const double wnorm = sqrt(Qs[e] * kNorm);
-                if (xnorm * wnorm >= 0x1p22) range_bad = true;
-                eps_star = fmax(eps_star, kRel * xnorm * wnorm + kFx + fabs(l) * 0x1p-50);
-                L[j] = l;
-            }
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1)
-            eps_star = fmax(eps_star, __shfl_xor_sync(0xffffffffu, eps_star, off));
-
-        // the K+1 best by l~ (ties to the lower index)
-        const int nsel = min(a.K + 1, a.E);
-        uint32_t taken = 0;
-        double prev = 0.0;
-        for (int k = 0; k < nsel; ++k) {
-            double bv = -DBL_MAX;
-            int be = 0x7fffffff;
-#pragma unroll
-            for (int j = 0; j < TK_MAXJ; ++j) {
-                const int e = lane + 32 * j;
-                if (j < nj && e < a.E && !((taken >> j) & 1u)) {
-                    if (L[j] > bv || (L[j] == bv && e < be)) {
-                        bv = L[j];
-                        be = e;
-                    }
-                }
-            }
-            warp_argmax(bv, be);
-            if (k < a.K) {
-                out_e[k] = be;
-                out_l[k] = bv;
-            }
-            if (k > 0 && !(prev - bv > 2.0 * eps_star)) certified = false;
-            prev = bv;
-            if ((be & 31) == lane) taken |= 1u << (be >> 5);
-        }
-        if (!certified) {
-            // candidates: every expert that could still be in the exact top K
-            const double thr = out_l[a.K - 1] - 2.0 * eps_star;
-#pragma unroll
-            for (int j = 0; j < TK_MAXJ; ++j) {
-                const int e = lane + 32 * j;
-                const bool c = j < nj && e < a.E && L[j] >= thr;
-                const uint32_t m = __ballot_sync(0xffffffffu, c);
-                int base = 0;
-                if (lane == 0 && m) base = atomicAdd(&n_cand, __popc(m));
-                base = __shfl_sync(0xffffffffu, base, 0);
-                if (c) {
-                    const int i = base + __popc(m & ((1u << lane) - 1u));
-                    c_tok[i] = (uint8_t)warp;
-                    c_e[i] = (uint16_t)e;
-                }
-            }
+    if (warp == 0) {
+        double wn, bm;
+        bound_constants(Qs, a.bias, a.H, a.E, lane, wn, bm);
+        if (lane == 0) {
+            s_bound[0] = wn;
+            s_bound[1] = bm;
         }
     }
     __syncthreads();
+    // fp32 chains of RT_HC terms; fp64: the chunk sums of one split, then the S split partials
+    const int per_split = (a.nchunks + a.S - 1) / a.S;
+    const double k_rel = router_k_rel(RT_HC, per_split + a.S + 1);
+    bool certified = true;
+    bool range_bad = false;
+    if (active)
+        certified = rank_certified(Ls[warp], Xs[warp], a.bias, a.H, a.E, a.K, k_rel, s_bound[0], s_bound[1], lane,
+                                   warp, s_oe[warp], s_ol[warp], range_bad, c_tok, c_e, &n_cand);
+    __syncthreads();
     const int nc = n_cand;
-    for (int i = warp; i < nc; i += TK_WARPS) {
-        const int64_t tt = (int64_t)blockIdx.x * TK_WARPS + c_tok[i];
-        const int e = c_e[i];
-        const long long v = exact_logit(a.x + tt * a.H, a.wr + (int64_t)e * a.H, a.H, a.bias, e, lane);
-        if (lane == 0) c_val[i] = v;
-    }
+    exact_candidates(nc, c_tok, c_e, c_val, t_base, a.x, a.wr, a.H, a.bias, warp, TK_WARPS, lane);
     __syncthreads();
 
     if (!active) return;
-    if (!certified) {
-        for (int k = 0; k < a.K; ++k) {
-            long long bv = LLONG_MIN;
-            int be = 0x7fffffff, bi = -1;
-            for (int i = lane; i < nc; i += 32) {
-                if (c_tok[i] != warp) continue;   // other tokens, or already taken (0xFF)
-                const long long v = c_val[i];
-                const int e = c_e[i];
-                if (bi < 0 || v > bv || (v == bv && e < be)) {
-                    bv = v;
-                    be = e;
-                    bi = i;
-                }
+    if (__any_sync(0xffffffffu, range_bad) && lane == 0) record_error(ctx.err, MOE_ERANGE);
+    finish_token(certified, warp, t, nc, c_tok, c_e, c_val, a.K, s_oe[warp], s_ol[warp], lane, a.idx, a.w);
+}
+
+// ----------------------------------------------------------------------------- small batches
+//
+// One cluster of 8 CTAs per group of TB tokens computes the whole router in
+// one launch.  CTA r of the cluster owns experts [r*ceil(E/8), ...), whose
+// router rows are one contiguous block of W_r: two bulk copies bring that
+// block and the group's x rows into shared memory.  A warp handles experts
+// e and e+8 of the slice; each lane takes pairs of 16-byte fragments, which
+// give, per token, a chain of 16 fp32 FMAs from zero, added into an fp64
+// total; the warp then sums its lanes' totals in fp64.  The logits and the
+// squared weight norms go to the leader CTA's shared memory (distributed
+// shared memory); after the cluster barrier the leader's warps run the same
+// certified selection as router_topk_kernel, one token each.
+
+constexpr int RS_CLUSTER = 8;
+constexpr int RS_THREADS = 256;
+constexpr int RS_WARPS = RS_THREADS / 32;
+
+struct RouterSmallArgs {
+    const uint16_t* x;
+    const uint16_t* wr;
+    const float* bias;
+    int64_t T;
+    int H, E, K;
+    int32_t* idx;
+    float* w;
+};
+
+__host__ __device__ constexpr int rs_epc(int E) { return (E + RS_CLUSTER - 1) / RS_CLUSTER; }
+__host__ __device__ constexpr size_t rs_align(size_t v) { return (v + 15) & ~size_t(15); }
+
+// dynamic shared memory of one CTA: xs [TB][H] bf16 | ws [epc][H] bf16 | Ls [TB][E] f64 |
+// Qs [E] f64 | Xs [TB] f64 | xred [TB][8] f32 | c_val [TB*E] i64 | c_e [TB*E] u16 |
+// c_tok [TB*E] u8 | n_cand, abort flag | mbarrier
+__host__ __device__ inline size_t rs_smem_bytes(int TB, int H, int E) {
+    size_t o = rs_align((size_t)TB * H * 2) + rs_align((size_t)rs_epc(E) * H * 2);
+    o += rs_align((size_t)TB * E * 8) + rs_align((size_t)E * 8) + rs_align((size_t)TB * 8);
+    o += rs_align((size_t)TB * RS_WARPS * 4);
+    o += rs_align((size_t)TB * E * 8) + rs_align((size_t)TB * E * 2) + rs_align((size_t)TB * E) + 16 + 16;
+    return o;
+}
+
+__device__ __forceinline__ void bf16x8(const uint4& v, float (&f)[8]) {
+    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        f[2 * q] = __uint_as_float(u[q] << 16);
+        f[2 * q + 1] = __uint_as_float(u[q] & 0xFFFF0000u);
+    }
+}
+
+template <int TB>
+__global__ void __cluster_dims__(RS_CLUSTER, 1, 1) __launch_bounds__(RS_THREADS)
+    router_small_kernel(RouterSmallArgs a, DevCtx ctx) {
+    namespace cg = cooperative_groups;
+    extern __shared__ __align__(16) unsigned char rs_smem[];
+    const int H = a.H, E = a.E;
+    const int epc = rs_epc(E);
+    unsigned char* p = rs_smem;
+    uint16_t* xs = reinterpret_cast<uint16_t*>(p);
+    p += rs_align((size_t)TB * H * 2);
+    uint16_t* ws = reinterpret_cast<uint16_t*>(p);
+    p += rs_align((size_t)epc * H * 2);
+    double* Ls = reinterpret_cast<double*>(p);
+    p += rs_align((size_t)TB * E * 8);
+    double* Qs = reinterpret_cast<double*>(p);
+    p += rs_align((size_t)E * 8);
+    double* Xs = reinterpret_cast<double*>(p);
+    p += rs_align((size_t)TB * 8);
+    float* xred = reinterpret_cast<float*>(p);
+    p += rs_align((size_t)TB * RS_WARPS * 4);
+    long long* c_val = reinterpret_cast<long long*>(p);
+    p += rs_align((size_t)TB * E * 8);
+    uint16_t* c_e = reinterpret_cast<uint16_t*>(p);
+    p += rs_align((size_t)TB * E * 2);
+    uint8_t* c_tok = p;
+    p += rs_align((size_t)TB * E);
+    int* n_cand = reinterpret_cast<int*>(p);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(p + 4);
+    p += 16;
+    uint64_t* bar = reinterpret_cast<uint64_t*>(p);
+
+    cg::cluster_group cluster = cg::this_cluster();
+    const unsigned rank = cluster.block_rank();
+    const bool leader = rank == 0;
+    const int tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
+    const int64_t t_base = (int64_t)(blockIdx.x / RS_CLUSTER) * TB;
+    const int n_tok = (int)min((int64_t)TB, a.T - t_base);
+    const int HV = H / 8;   // 16-byte fragments per row
+    const int e_lo = (int)rank * epc, e_hi = min(E, e_lo + epc);
+    const int n_e = max(0, e_hi - e_lo);
+
+    // 1. the group's x rows and this CTA's router rows, one bulk copy each
+    if (tid == 0) {
+        *n_cand = 0;
+        *abort_flag = 0;
+        mbar_init(smem_u32(bar), 1);
+        fence_mbar_init();
+        const uint32_t xb = (uint32_t)n_tok * H * 2, wb = (uint32_t)n_e * H * 2;
+        mbar_arrive_expect_tx(smem_u32(bar), xb + wb);
+        bulk_load_1d(smem_u32(xs), a.x + t_base * H, xb, smem_u32(bar));
+        if (wb) bulk_load_1d(smem_u32(ws), a.wr + (int64_t)e_lo * H, wb, smem_u32(bar));
+    }
+    __syncthreads();
+    if (!mbar_wait(smem_u32(bar), 0, ctx, abort_flag)) mbar_wait_drain(smem_u32(bar), 0, ctx.timeout_ns);
+
+    // the leader's ||x||^2 (fp32 sums of exact squares)
+    if (leader) {
+        for (int t = 0; t < n_tok; ++t) {
+            float q = 0.0f;
+            for (int v = tid; v < HV; v += RS_THREADS) {
+                float f[8];
+                bf16x8(*reinterpret_cast<const uint4*>(xs + (size_t)t * H + 8 * v), f);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) q = __fmaf_rn(f[j], f[j], q);
             }
-            int src_e = be;
-            warp_argmax_i64(bv, src_e);
-            if (bi >= 0 && be == src_e) c_tok[bi] = 0xFF;   // taken (this lane held it)
-            __syncwarp();
-            out_e[k] = src_e;
-            out_l[k] = (double)bv * 0x1p-40;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) q = __fadd_rn(q, __shfl_xor_sync(0xffffffffu, q, off));
+            if (lane == 0) xred[t * RS_WARPS + warp] = q;
+        }
+        __syncthreads();
+        if (tid < n_tok) {
+            float q = 0.0f;
+            for (int i = 0; i < RS_WARPS; ++i) q = __fadd_rn(q, xred[tid * RS_WARPS + i]);
+            Xs[tid] = (double)q;
         }
     }
-    if (__any_sync(0xffffffffu, range_bad) && lane == 0) record_error(ctx.err, MOE_ERANGE);
 
-    // renormalised softmax over the selected logits
-    float z = 0.0f;
-    float ex[16];
-    for (int k = 0; k < a.K; ++k) {
-        ex[k] = expf((float)(out_l[k] - out_l[0]));
-        z += ex[k];
-    }
-    for (int k = lane; k < a.K; k += 32) {
-        int ek = 0;
-        float wk = 0.0f;
-        for (int q = 0; q < a.K; ++q)
-            if (q == k) {
-                ek = out_e[q];
-                wk = ex[q] / z;
+    // 2. this CTA's experts: warp w takes local experts w + 16m and w + 16m + 8
+    double* Ls_lead = cluster.map_shared_rank(Ls, 0);
+    double* Qs_lead = cluster.map_shared_rank(Qs, 0);
+    for (int l0 = warp; l0 < n_e; l0 += 2 * RS_WARPS) {
+        const int l1 = l0 + RS_WARPS;
+        const bool has1 = l1 < n_e;
+        const uint16_t* w0 = ws + (size_t)l0 * H;
+        const uint16_t* w1 = ws + (size_t)(has1 ? l1 : l0) * H;
+        double acc0[TB], acc1[TB];
+#pragma unroll
+        for (int t = 0; t < TB; ++t) acc0[t] = acc1[t] = 0.0;
+        float q0 = 0.0f, q1 = 0.0f;
+        for (int v0 = lane; v0 < HV; v0 += 64) {
+            const int v1 = v0 + 32;
+            const bool ok1 = v1 < HV;
+            const uint4 z4 = make_uint4(0, 0, 0, 0);
+            float a0[16], a1[16];
+            {
+                float f[8];
+                bf16x8(*reinterpret_cast<const uint4*>(w0 + 8 * v0), f);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) a0[j] = f[j];
+                bf16x8(ok1 ? *reinterpret_cast<const uint4*>(w0 + 8 * v1) : z4, f);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) a0[8 + j] = f[j];
+                bf16x8(*reinterpret_cast<const uint4*>(w1 + 8 * v0), f);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) a1[j] = f[j];
+                bf16x8(ok1 ? *reinterpret_cast<const uint4*>(w1 + 8 * v1) : z4, f);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) a1[8 + j] = f[j];
             }
-        a.idx[t * a.K + k] = ek;
-        a.w[t * a.K + k] = wk;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                q0 = __fmaf_rn(a0[j], a0[j], q0);
+                q1 = __fmaf_rn(a1[j], a1[j], q1);
+            }
+#pragma unroll
+            for (int t = 0; t < TB; ++t) {
+                float xv[16];
+                {
+                    float f[8];
+                    bf16x8(*reinterpret_cast<const uint4*>(xs + (size_t)t * H + 8 * v0), f);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) xv[j] = f[j];
+                    bf16x8(ok1 ? *reinterpret_cast<const uint4*>(xs + (size_t)t * H + 8 * v1) : z4, f);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) xv[8 + j] = f[j];
+                }
+                float c0 = 0.0f, c1 = 0.0f;
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    c0 = __fmaf_rn(xv[j], a0[j], c0);
+                    c1 = __fmaf_rn(xv[j], a1[j], c1);
+                }
+                acc0[t] += (double)c0;
+                acc1[t] += (double)c1;
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+#pragma unroll
+            for (int t = 0; t < TB; ++t) {
+                acc0[t] += __shfl_xor_sync(0xffffffffu, acc0[t], off);
+                acc1[t] += __shfl_xor_sync(0xffffffffu, acc1[t], off);
+            }
+            q0 = __fadd_rn(q0, __shfl_xor_sync(0xffffffffu, q0, off));
+            q1 = __fadd_rn(q1, __shfl_xor_sync(0xffffffffu, q1, off));
+        }
+        if (lane < TB) {
+            // lane t writes token t's two logits (registers indexed at compile time)
+#pragma unroll
+            for (int t = 0; t < TB; ++t)
+                if (t == lane) {
+                    Ls_lead[t * E + e_lo + l0] = acc0[t];
+                    if (has1) Ls_lead[t * E + e_lo + l1] = acc1[t];
+                }
+        }
+        if (lane == 0) {
+            Qs_lead[e_lo + l0] = (double)q0;
+            if (has1) Qs_lead[e_lo + l1] = (double)q1;
+        }
+    }
+    // every CTA's stores to the leader become visible to it here
+    cluster.sync();
+    if (!leader) return;
+
+    // 3. selection, one warp per token (the leader's shared memory only)
+    __shared__ int s_oe[RS_WARPS][TK_MAXK];
+    __shared__ double s_ol[RS_WARPS][TK_MAXK];
+    __shared__ double s_bound[2];
+    if (warp == 0) {
+        double wn, bm;
+        bound_constants(Qs, a.bias, H, E, lane, wn, bm);
+        if (lane == 0) {
+            s_bound[0] = wn;
+            s_bound[1] = bm;
+        }
+    }
+    __syncthreads();
+    // fp32 chains of 16 terms; fp64: the lane's chain sums, then 5 warp levels
+    const double k_rel = router_k_rel(16, (HV + 63) / 64 + 6);
+    const bool active = warp < n_tok;
+    bool certified = true;
+    bool range_bad = false;
+    if (active)
+        certified = rank_certified(Ls + (size_t)warp * E, Xs[warp], a.bias, H, E, a.K, k_rel, s_bound[0],
+                                   s_bound[1], lane, warp, s_oe[warp], s_ol[warp], range_bad, c_tok, c_e, n_cand);
+    __syncthreads();
+    const int nc = *n_cand;
+    exact_candidates(nc, c_tok, c_e, c_val, t_base, a.x, a.wr, H, a.bias, warp, RS_WARPS, lane);
+    __syncthreads();
+    if (!active) return;
+    if (__any_sync(0xffffffffu, range_bad) && lane == 0) record_error(ctx.err, MOE_ERANGE);
+    finish_token(certified, warp, t_base + warp, nc, c_tok, c_e, c_val, a.K, s_oe[warp], s_ol[warp], lane, a.idx,
+                 a.w);
+}
+
+// ----------------------------------------------------------------------------- large batches
+//
+// One cluster of CS CTAs per tile of BT = NTH/4 tokens (all E <= 128
+// experts): CTA r of the cluster takes stages [r n/CS, (r+1) n/CS) of the
+// hidden dimension, 32 values each, staged in shared memory as fp32 (double
+// buffered).  Thread (ty, tx) owns 4 tokens x 8 experts; per stage each
+// (token, expert) gets a chain of 32 fp32 FMAs from zero, added into an fp32
+// total (so a product passes through at most 31 + m roundings, m = stages per
+// CTA).  The CTA's fp32 partial logits and squared norms stay in its shared
+// memory; after the cluster barrier CTA r sums, in fp64, the CS partials of
+// its own BT/CS tokens over distributed shared memory, ranks them (one warp
+// per token), computes the exact logits of every open candidate with the
+// whole CTA, and finishes them.
+
+constexpr int RF_HS = 32;       // hidden values per stage and per fp32 chain
+constexpr int RF_E = 128;       // experts per tile (E <= 128)
+
+struct RouterFusedArgs {
+    const uint16_t* x;
+    const uint16_t* wr;
+    const float* bias;
+    int64_t T;
+    int H, E, K;
+    int n_stages;         // ceil(H / RF_HS)
+    int32_t* idx;
+    float* w;
+};
+
+template <int NTH, int CS>
+struct RfLayout {
+    static constexpr int WARPS = NTH / 32;
+    static constexpr int BT = NTH / 4;          // tokens per tile (16-byte x fragments per stage = NTH)
+    static constexpr int TPC = BT / CS;         // tokens each CTA selects
+    static constexpr int TPW = (TPC + WARPS - 1) / WARPS;
+    static constexpr int NWF = 4 * RF_E;        // 16-byte w fragments per stage
+    static constexpr size_t stage_floats = (size_t)RF_HS * (BT + RF_E);
+    static constexpr size_t ring_bytes = 2 * stage_floats * 4;
+    static constexpr size_t pl_bytes = (size_t)BT * RF_E * 4;
+    // the candidate lists of the selection reuse the ring after the partials are read
+    static constexpr size_t o_cv = 0;
+    static constexpr size_t o_ce = o_cv + (size_t)TPC * RF_E * 8;
+    static constexpr size_t o_ct = o_ce + (size_t)TPC * RF_E * 2;
+    static constexpr size_t cand_end = o_ct + (size_t)TPC * RF_E;
+    static constexpr size_t main_bytes =
+        ((ring_bytes > pl_bytes ? ring_bytes : pl_bytes) > cand_end ? (ring_bytes > pl_bytes ? ring_bytes : pl_bytes)
+                                                                    : (cand_end + 15) / 16 * 16);
+    static constexpr size_t o_xq = main_bytes;
+    static constexpr size_t o_wq = o_xq + NTH * 4;
+    static constexpr size_t o_xp = o_wq + NWF * 4;
+    static constexpr size_t o_wp = o_xp + BT * 4;
+    static constexpr size_t o_ls = o_wp + RF_E * 4;
+    static constexpr size_t o_qs = o_ls + (size_t)TPC * RF_E * 8;
+    static constexpr size_t o_xs = o_qs + RF_E * 8;
+    static constexpr size_t o_oe = o_xs + ((TPC * 8 + 15) / 16) * 16;   // [TPC][TK_MAXK] int
+    static constexpr size_t o_ol = o_oe + (size_t)TPC * TK_MAXK * 4;       // [TPC][TK_MAXK] double
+    static constexpr size_t o_nc = o_ol + (size_t)TPC * TK_MAXK * 8 + 16;   // + the two bound constants
+    static constexpr size_t bytes = o_nc + 16;
+};
+
+template <int NTH, int CS>
+__global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(NTH, 1)
+    router_fused_kernel(RouterFusedArgs a, DevCtx ctx) {
+    namespace cg = cooperative_groups;
+    using L = RfLayout<NTH, CS>;
+    constexpr int BT = L::BT, TPC = L::TPC, WARPS = L::WARPS, TPW = L::TPW, NWF = L::NWF;
+    constexpr int NW = (NWF + NTH - 1) / NTH;   // w fragments per thread and stage (the last may be empty)
+    extern __shared__ __align__(16) unsigned char rf_smem[];
+    float* ring = reinterpret_cast<float*>(rf_smem);
+    float* Pl = ring;                             // [BT][RF_E] after the main loop
+    long long* c_val = reinterpret_cast<long long*>(rf_smem + L::o_cv);   // after the partials are read
+    uint16_t* c_e = reinterpret_cast<uint16_t*>(rf_smem + L::o_ce);
+    uint8_t* c_tok = rf_smem + L::o_ct;
+    float* xq = reinterpret_cast<float*>(rf_smem + L::o_xq);
+    float* wq = reinterpret_cast<float*>(rf_smem + L::o_wq);
+    float* xpart = reinterpret_cast<float*>(rf_smem + L::o_xp);
+    float* wpart = reinterpret_cast<float*>(rf_smem + L::o_wp);
+    double* Ls = reinterpret_cast<double*>(rf_smem + L::o_ls);
+    double* Qs = reinterpret_cast<double*>(rf_smem + L::o_qs);
+    double* Xs = reinterpret_cast<double*>(rf_smem + L::o_xs);
+    int* s_oe = reinterpret_cast<int*>(rf_smem + L::o_oe);
+    double* s_ol = reinterpret_cast<double*>(rf_smem + L::o_ol);
+    int* n_cand = reinterpret_cast<int*>(rf_smem + L::o_nc);
+
+    cg::cluster_group cluster = cg::this_cluster();
+    const int rank = (int)cluster.block_rank();
+    const int tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
+    const int ty = tid / 16, tx = tid % 16;     // tokens 4ty..4ty+3; experts 4tx.. and 64+4tx..
+    const int64_t t0 = (int64_t)(blockIdx.x / CS) * BT;
+    const int H = a.H, E = a.E;
+    const int s_begin = rank * a.n_stages / CS, s_end = (rank + 1) * a.n_stages / CS;
+
+    // staging: x fragment tid is row tid % BT, 8 values at 8 (tid / BT); w fragment
+    // i = tid + NTH k is row i % 128, 8 values at 8 (i / 128).  Consecutive lanes take
+    // consecutive rows, so the transposed fp32 stores are conflict-free.  Each fragment
+    // slot keeps the fp32 sum of its squares.
+    uint4 xv, wv[NW];
+    float xsq = 0.0f, wsq[NW];
+#pragma unroll
+    for (int k = 0; k < NW; ++k) wsq[k] = 0.0f;
+    auto load = [&](int st) {
+        const int h0 = st * RF_HS;
+        {
+            const int row = tid % BT, h = h0 + 8 * (tid / BT);
+            const int64_t t = t0 + row;
+            xv = make_uint4(0, 0, 0, 0);
+            if (t < a.T && h < H) xv = *reinterpret_cast<const uint4*>(a.x + t * H + h);
+        }
+#pragma unroll
+        for (int k = 0; k < NW; ++k) {
+            const int i = tid + NTH * k, row = i % RF_E, h = h0 + 8 * (i / RF_E);
+            wv[k] = make_uint4(0, 0, 0, 0);
+            if (i < NWF && row < E && h < H) wv[k] = *reinterpret_cast<const uint4*>(a.wr + (int64_t)row * H + h);
+        }
+    };
+    auto store = [&](int buf) {
+        float* xs = ring + (size_t)buf * L::stage_floats;   // [RF_HS][BT]
+        float* ws = xs + RF_HS * BT;                        // [RF_HS][RF_E]
+        {
+            const int row = tid % BT, f8 = 8 * (tid / BT);
+            float f[8];
+            bf16x8(xv, f);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                xs[(f8 + j) * BT + row] = f[j];
+                xsq = __fmaf_rn(f[j], f[j], xsq);
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < NW; ++k) {
+            const int i = tid + NTH * k, row = i % RF_E, f8 = 8 * (i / RF_E);
+            if (i < NWF) {
+                float f[8];
+                bf16x8(wv[k], f);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    ws[(f8 + j) * RF_E + row] = f[j];
+                    wsq[k] = __fmaf_rn(f[j], f[j], wsq[k]);
+                }
+            }
+        }
+    };
+
+    float acc[4][8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
+
+    if (s_begin < s_end) {
+        load(s_begin);
+        store(0);
+    }
+    __syncthreads();
+    for (int st = s_begin; st < s_end; ++st) {
+        const int buf = (st - s_begin) & 1;
+        if (st + 1 < s_end) load(st + 1);
+        const float* xs = ring + (size_t)buf * L::stage_floats;
+        const float* ws = xs + RF_HS * BT;
+        float c[4][8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 8; ++j) c[i][j] = 0.0f;
+#pragma unroll
+        for (int h = 0; h < RF_HS; ++h) {
+            const float4 xx = *reinterpret_cast<const float4*>(xs + h * BT + 4 * ty);
+            const float4 wa = *reinterpret_cast<const float4*>(ws + h * RF_E + 4 * tx);
+            const float4 wb = *reinterpret_cast<const float4*>(ws + h * RF_E + 64 + 4 * tx);
+            const float xr[4] = {xx.x, xx.y, xx.z, xx.w};
+            const float w8[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) c[i][j] = __fmaf_rn(xr[i], w8[j], c[i][j]);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[i][j] = __fadd_rn(acc[i][j], c[i][j]);
+        if (st + 1 < s_end) store(buf ^ 1);
+        __syncthreads();
+    }
+
+    // this CTA's partials: logits [BT][RF_E] (over the ring, which is no longer read) and norms
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float* row = Pl + (4 * ty + i) * RF_E;
+        *reinterpret_cast<float4*>(row + 4 * tx) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+        *reinterpret_cast<float4*>(row + 64 + 4 * tx) = make_float4(acc[i][4], acc[i][5], acc[i][6], acc[i][7]);
+    }
+    xq[tid] = xsq;
+#pragma unroll
+    for (int k = 0; k < NW; ++k)
+        if (tid + NTH * k < NWF) wq[tid + NTH * k] = wsq[k];
+    if (tid == 0) *n_cand = 0;
+    __syncthreads();
+    if (tid < BT) {
+        float q = 0.0f;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) q = __fadd_rn(q, xq[g * BT + tid]);
+        xpart[tid] = q;
+    }
+    if (tid < RF_E) {
+        float q = 0.0f;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) q = __fadd_rn(q, wq[g * RF_E + tid]);
+        wpart[tid] = q;
+    }
+    cluster.sync();
+
+    // CTA `rank` selects tokens rank*TPC .. +TPC-1 of the tile: fp64 sums of the CS partials
+    {
+        const float* Pr[CS];
+        const float* Wr[CS];
+        const float* Xr[CS];
+#pragma unroll
+        for (int r = 0; r < CS; ++r) {
+            Pr[r] = cluster.map_shared_rank(Pl, r);
+            Wr[r] = cluster.map_shared_rank(wpart, r);
+            Xr[r] = cluster.map_shared_rank(xpart, r);
+        }
+        for (int i = tid; i < TPC * RF_E / 4; i += NTH) {
+            const int tl = (4 * i) / RF_E, e = (4 * i) % RF_E;
+            const int t = rank * TPC + tl;
+            float4 v[CS];
+#pragma unroll
+            for (int r = 0; r < CS; ++r) v[r] = *reinterpret_cast<const float4*>(Pr[r] + t * RF_E + e);
+            double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
+#pragma unroll
+            for (int r = 0; r < CS; ++r) {
+                s0 += (double)v[r].x;
+                s1 += (double)v[r].y;
+                s2 += (double)v[r].z;
+                s3 += (double)v[r].w;
+            }
+            double* dst = Ls + tl * RF_E + e;
+            dst[0] = s0;
+            dst[1] = s1;
+            dst[2] = s2;
+            dst[3] = s3;
+        }
+        if (tid < RF_E) {
+            double q = 0.0;
+#pragma unroll
+            for (int r = 0; r < CS; ++r) q += (double)Wr[r][tid];
+            Qs[tid] = q;
+        }
+        if (tid < TPC) {
+            double q = 0.0;
+#pragma unroll
+            for (int r = 0; r < CS; ++r) q += (double)Xr[r][rank * TPC + tid];
+            Xs[tid] = q;
+        }
+    }
+    // no CTA reuses or releases its shared memory while another still reads it
+    cluster.sync();
+    if (warp == 0) {
+        double wn, bm;
+        bound_constants(Qs, a.bias, H, E, lane, wn, bm);
+        if (lane == 0) {
+            s_ol[TPC * TK_MAXK] = wn;
+            s_ol[TPC * TK_MAXK + 1] = bm;
+        }
+    }
+    __syncthreads();
+    const double wnmax = s_ol[TPC * TK_MAXK], bmax = s_ol[TPC * TK_MAXK + 1];
+
+    // rank every token of this CTA, then one exact pass over all open candidates, then finish
+    const int m = (a.n_stages + CS - 1) / CS;
+    const double k_rel = router_k_rel(RF_HS + m, CS + 1);
+    const int64_t ts0 = t0 + (int64_t)rank * TPC;
+    bool cert[TPW];
+    bool range_bad = false;
+#pragma unroll
+    for (int k = 0; k < TPW; ++k) {
+        const int slot = warp + WARPS * k;
+        cert[k] = true;
+        if (slot < TPC && ts0 + slot < a.T)
+            cert[k] = rank_certified(Ls + (size_t)slot * RF_E, Xs[slot], a.bias, H, E, a.K, k_rel, wnmax, bmax, lane,
+                                     slot, s_oe + slot * TK_MAXK, s_ol + slot * TK_MAXK, range_bad, c_tok, c_e,
+                                     n_cand);
+    }
+    __syncthreads();
+    const int nc = *n_cand;
+    exact_candidates(nc, c_tok, c_e, c_val, ts0, a.x, a.wr, H, a.bias, warp, WARPS, lane);
+    __syncthreads();
+    if (__any_sync(0xffffffffu, range_bad) && lane == 0) record_error(ctx.err, MOE_ERANGE);
+#pragma unroll
+    for (int k = 0; k < TPW; ++k) {
+        const int slot = warp + WARPS * k;
+        if (slot < TPC && ts0 + slot < a.T)
+            finish_token(cert[k], slot, ts0 + slot, nc, c_tok, c_e, c_val, a.K, s_oe + slot * TK_MAXK,
+                         s_ol + slot * TK_MAXK, lane, a.idx, a.w);
     }
 }
 
@@ -433,13 +1101,24 @@ __global__ void __launch_bounds__(TK_WARPS * 32, 2) router_topk_kernel(RouterTop
 struct RouterPlan {
     int S;
     int nchunks;
+    int num_sms;
     size_t p_bytes, xn_bytes, wn_bytes;
 };
+
+// Batch-size boundaries of the three router shapes, from CUDA-event timings
+// on B200 (H=2688, E=128, K=6): the expert-split clusters up to 256 tokens
+// (17 us at 64), the two-kernel router in between, the hidden-split clusters
+// from 3072 tokens (101 us at 4096 against 154).
+constexpr int64_t kRouterSmallMaxDefault = 256;
+constexpr int64_t kRouterSplitMin = 3072;
+constexpr int64_t kRouterSmallTb4Max = 128;
+constexpr size_t kRouterSmallSmemMax = 200 * 1024;
 
 static int router_tt(int64_t T) { return T > 256 ? 64 : 16; }
 
 RouterPlan router_plan(int64_t T, int H, int E, int num_sms) {
     RouterPlan p;
+    p.num_sms = num_sms;
     p.nchunks = (H + RT_HC - 1) / RT_HC;
     const int tt = router_tt(T);
     const int64_t tiles = ((T + tt - 1) / tt) * ((E + RT_TE - 1) / RT_TE);
@@ -457,11 +1136,109 @@ RouterPlan router_plan(int64_t T, int H, int E, int num_sms) {
     return p;
 }
 
+// Largest batch the one-launch cluster router takes (tokens); larger batches
+// use the tiled logits kernel and router_topk_kernel.
+std::atomic<int64_t> g_router_small_max{kRouterSmallMaxDefault};
+// 0: by batch size; 1: every larger batch takes the two-kernel router; 2: every larger
+// batch with E <= 128 takes the hidden-split clusters
+std::atomic<int> g_router_split{0};
+
+void set_router_small_max(int64_t v) { g_router_small_max.store(v < 0 ? kRouterSmallMaxDefault : v); }
+void set_router_split(int v) { g_router_split.store(v == 1 || v == 2 ? v : 0); }
+
+// How many clusters of the split-cluster router fit on the device at once (a
+// cluster sits inside one GPC, so this is not the SM count over CS); cached
+// per device.
+template <int NTH, int CS>
+static int64_t fused_max_clusters(int num_sms) {
+    static std::atomic<int> cache[64];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64) {
+        const int c = cache[dev].load();
+        if (c > 0) return c;
+    }
+    using L = RfLayout<NTH, CS>;
+    auto kfn = router_fused_kernel<NTH, CS>;
+    int n = 0;
+    if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::bytes) == cudaSuccess) {
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = CS;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.gridDim = dim3((unsigned)(CS * (num_sms / CS)));
+        cfg.blockDim = dim3(NTH);
+        cfg.dynamicSmemBytes = L::bytes;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaOccupancyMaxActiveClusters(&n, kfn, &cfg) != cudaSuccess) n = 0;
+    }
+    cudaGetLastError();
+    if (n < 1) n = num_sms / CS > 0 ? num_sms / CS : 1;
+    if (dev >= 0 && dev < 64) cache[dev].store(n);
+    return n;
+}
+
+// Time model of one tiling: waves of clusters x the work of one CTA (tokens x stages).
+template <int NTH, int CS>
+static int64_t fused_cost(int64_t T, int num_sms) {
+    using L = RfLayout<NTH, CS>;
+    const int64_t tiles = (T + L::BT - 1) / L::BT;
+    const int64_t act = fused_max_clusters<NTH, CS>(num_sms);
+    return (tiles + act - 1) / act * (int64_t)(L::BT * 8 / CS);
+}
+
+template <int NTH, int CS>
+static cudaError_t launch_router_fused(const RouterFusedArgs& ra, const DevCtx& ctx, cudaStream_t stream) {
+    using L = RfLayout<NTH, CS>;
+    auto kfn = router_fused_kernel<NTH, CS>;
+    cudaError_t err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::bytes);
+    if (err != cudaSuccess) return err;
+    const unsigned tiles = (unsigned)((ra.T + L::BT - 1) / L::BT);
+    kfn<<<tiles * CS, NTH, L::bytes, stream>>>(ra, ctx);
+    return cudaGetLastError();
+}
+
+template <int TB>
+static cudaError_t launch_router_small(const RouterSmallArgs& ra, const DevCtx& ctx, cudaStream_t stream) {
+    const size_t smem = rs_smem_bytes(TB, ra.H, ra.E);
+    auto kfn = router_small_kernel<TB>;
+    cudaError_t err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    const unsigned groups = (unsigned)((ra.T + TB - 1) / TB);
+    kfn<<<groups * RS_CLUSTER, RS_THREADS, smem, stream>>>(ra, ctx);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_route(const uint16_t* x, const uint16_t* wr, const float* bias, int64_t T, int H,
                          int E, int K, int32_t* idx, float* w, double* P, double* xn2, double* wn2,
                          const RouterPlan& plan, const DevCtx& ctx, cudaStream_t stream,
                          void (*between)(cudaStream_t)) {
     if (T == 0) return cudaSuccess;
+    if (T <= g_router_small_max.load()) {
+        const int tb = T <= kRouterSmallTb4Max ? 4 : 8;
+        if (rs_smem_bytes(tb, H, E) <= kRouterSmallSmemMax) {
+            RouterSmallArgs ra{x, wr, bias, T, H, E, K, idx, w};
+            const cudaError_t err = tb == 4 ? launch_router_small<4>(ra, ctx, stream)
+                                            : launch_router_small<8>(ra, ctx, stream);
+            if (err == cudaSuccess && between) between(stream);   // one launch: nothing between
+            return err;
+        }
+    }
+    const int split_mode = g_router_split.load();
+    if (E <= RF_E && split_mode != 1 && (split_mode == 2 || T >= kRouterSplitMin)) {
+        RouterFusedArgs fa{x, wr, bias, T, H, E, K, (H + RF_HS - 1) / RF_HS, idx, w};
+        // the tiling with the fewest waves x work per CTA (ties: larger tiles, fewer CTAs)
+        const int64_t k0 = fused_cost<512, 4>(T, plan.num_sms), k1 = fused_cost<512, 8>(T, plan.num_sms),
+                      k2 = fused_cost<256, 8>(T, plan.num_sms);
+        const cudaError_t err = (k0 <= k1 && k0 <= k2) ? launch_router_fused<512, 4>(fa, ctx, stream)
+                                : (k1 <= k2)           ? launch_router_fused<512, 8>(fa, ctx, stream)
+                                                       : launch_router_fused<256, 8>(fa, ctx, stream);
+        if (err == cudaSuccess && between) between(stream);
+        return err;
+    }
     RouterLogitsArgs la{x, wr, T, H, E, plan.S, plan.nchunks, P, xn2, wn2};
     const int tt = router_tt(T);
     dim3 grid((unsigned)((T + tt - 1) / tt), (unsigned)((E + RT_TE - 1) / RT_TE), (unsigned)plan.S);
@@ -472,7 +1249,7 @@ cudaError_t launch_route(const uint16_t* x, const uint16_t* wr, const float* bia
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     if (between) between(stream);
-    RouterTopkArgs ta{P, xn2, wn2, x, wr, bias, T, H, E, K, plan.S, idx, w};
+    RouterTopkArgs ta{P, xn2, wn2, x, wr, bias, T, H, E, K, plan.S, plan.nchunks, idx, w};
     const unsigned blocks = (unsigned)((T + TK_WARPS - 1) / TK_WARPS);
     router_topk_kernel<<<blocks, TK_WARPS * 32, 0, stream>>>(ta, ctx);
     return cudaGetLastError();

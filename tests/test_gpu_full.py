@@ -182,3 +182,28 @@ def test_expired_wait_is_reported_and_the_context_stays_usable(moe):
     ref = oracle.expert_rows_bf16(xf[perm_src // w.K], ridx.reshape(-1)[perm_src], h["wu"], h["wd"],
                                   oracle.identity_slot(w.E))
     assert rel_err(host_f64(y), ref) <= BF16_TOL
+
+
+# --------------------------------------------------------------------------- CTA-pair GEMM
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_cta_pair_gemm_matches_oracle(moe, fp8):
+    """The cta_group::2 grouped GEMM (switched on by debug hook 3) on a batch whose
+    tiles exceed 64 tokens, including a ragged expert tail: same parity bar."""
+    w = W.Workload("pair_T600_ragged", 600, 512, 16, 4, 320, seed=21)
+    h = inputs(w)
+    moe.debug_set(3, 1)
+    try:
+        if fp8:
+            assert fp8_case(moe, w, h["x"], h["wr"], h["bias"], h["wu"], h["wd"]) <= FP8_TOL
+        else:
+            d = device_inputs(h)
+            dims = moe.dims(w.T, w.H, w.E, w.K, w.F)
+            ws = moe.alloc_workspace(dims)
+            out = torch.empty(w.T, w.H, dtype=torch.bfloat16, device="cuda")
+            moe.forward(dims, d["x"], d["wr"], None, d["wu"], d["wd"], out, ws)
+            moe.check_device_error()
+            r = oracle.moe_layer_bf16(h["x"], h["wr"], None, h["wu"], h["wd"], w.K)
+            assert rel_err(host_f64(out), r["out"]) <= BF16_TOL
+    finally:
+        moe.debug_set(3, 0)
