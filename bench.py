@@ -439,6 +439,9 @@ def run_native(args):
     if args.gemm == "pair":
         import routed_expert_moe_b200 as moe
         moe.debug_set(3, 1)
+    if args.pdl == "off":
+        import routed_expert_moe_b200 as moe
+        moe.debug_set(6, 0)
 
     wl = W.WORKLOADS[WORKLOADS[args.workload]]
     layer = Chain(wl, device) if wl.layers > 1 else Layer(wl, device)
@@ -490,7 +493,8 @@ def run_native(args):
                              f"({touched * wl.F * wl.H * (2 if wl.fp8 else 4) * wl.layers / 1e9:.2f} GB) "
                              "stream from HBM every step; token batches rotate; no flush",
                        "parallelism": f"dp{ws} (independent token batches per GPU, weights replicated)",
-                       "grouped_gemm": "cta_pair" if args.gemm == "pair" else "single_cta"},
+                       "grouped_gemm": "cta_pair" if args.gemm == "pair" else "single_cta",
+                       "programmatic_dependent_launch": args.pdl == "on"},
             "roofline": roofline_entry(wl, stages, touched, peaks, peak_kind, args.workload),
             "stages_ms": stages,
             "e2e": {"value": job_value(ws, wl.T * wl.layers, args.steps, e2e_ms), "unit": UNIT,
@@ -549,6 +553,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--gemm", choices=["single", "pair"], default="single",
                     help="grouped GEMM on single CTAs, or on CTA pairs for tiles of more than 64 tokens")
+    ap.add_argument("--pdl", choices=["on", "off"], default="on",
+                    help="programmatic dependent launch between the layer's kernels")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -200,8 +200,11 @@ moe_status moe_set_stage_events(void* const* events, int32_t n);
  * larger batches: 0 (the default) by batch size (one launch of clusters split
  * over the hidden dimension from 3072 tokens when E <= 128, else the tiled
  * logits kernel and the top-K kernel), 1 always the two kernels, 2 always the
- * hidden-split clusters when E <= 128; other values MOE_EINVAL.  Other `what`:
- * MOE_EINVAL. */
+ * hidden-split clusters when E <= 128; other values MOE_EINVAL; what = 6:
+ * value 0 launches every kernel without programmatic stream serialization
+ * (each kernel then starts only after its predecessor has finished), 1 (the
+ * default) lets each kernel start while its predecessor finishes and wait
+ * on the device for it.  Other `what`: MOE_EINVAL. */
 moe_status moe_debug_set(int32_t what, int64_t value);
 
 #ifdef __cplusplus

@@ -23,6 +23,7 @@ __global__ void __launch_bounds__(CB_THREADS) combine_kernel(const uint16_t* __r
                                                              const uint16_t* residual, uint16_t* out,
                                                              int64_t T, int K, int H, int64_t rows,
                                                              DevCtx ctx) {
+    pdl_enter();
     __shared__ int row_k[16];
     __shared__ float w_k[16];
     const int nv = H / 8;
@@ -86,6 +87,7 @@ __global__ void __launch_bounds__(CB_THREADS) combine_kernel(const uint16_t* __r
 __global__ void __launch_bounds__(256) rmsnorm_kernel(const uint16_t* __restrict__ x,
                                                       uint16_t* __restrict__ u, int64_t T, int H,
                                                       float eps) {
+    pdl_enter();
     const int lane = threadIdx.x % 32;
     const int64_t warps = (int64_t)gridDim.x * (blockDim.x / 32);
     const int nv = H / 8;
@@ -128,6 +130,7 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const uint16_t* __restrict
 // amax over each tensor (as the bits of |v|, which order like the values).
 __global__ void __launch_bounds__(256) amax_kernel(const uint16_t* __restrict__ src, int64_t elems,
                                                    unsigned int* __restrict__ amax_bits) {
+    pdl_enter();
     const int64_t tensor = blockIdx.y;
     const uint16_t* p = src + tensor * elems;
     uint32_t m = 0;
@@ -143,6 +146,7 @@ __global__ void __launch_bounds__(256) amax_kernel(const uint16_t* __restrict__ 
 
 // scale = amax / 448 (1 for an all-zero tensor), in place over the amax bits.
 __global__ void finalize_scale_kernel(float* scales, int64_t n) {
+    pdl_enter();
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i < n) {
         const float amax = __uint_as_float(reinterpret_cast<unsigned int*>(scales)[i]);
@@ -153,6 +157,7 @@ __global__ void finalize_scale_kernel(float* scales, int64_t n) {
 __global__ void __launch_bounds__(256) quantize_kernel(const uint16_t* __restrict__ src, int64_t elems,
                                                        const float* __restrict__ scales,
                                                        uint8_t* __restrict__ codes) {
+    pdl_enter();
     const int64_t tensor = blockIdx.y;
     const float s = scales[tensor];
     const uint16_t* p = src + tensor * elems;
@@ -179,15 +184,14 @@ cudaError_t launch_combine(const uint16_t* yp, const int32_t* inv_row, const flo
     if (T == 0) return cudaSuccess;
     const int64_t cap = (int64_t)num_sms * 16;
     const unsigned grid = (unsigned)(T < cap ? T : cap);
-    combine_kernel<<<grid, CB_THREADS, 0, stream>>>(yp, inv_row, w, residual, out, T, K, H, T * K, ctx);
-    return cudaGetLastError();
+    return launch_k(combine_kernel, dim3(grid), dim3(CB_THREADS), 0, stream, yp, inv_row, w, residual, out, T, K, H,
+                    T * K, ctx);
 }
 
 cudaError_t launch_rmsnorm(const uint16_t* x, uint16_t* u, int64_t T, int H, float eps, int num_sms,
                            cudaStream_t stream) {
     if (T == 0) return cudaSuccess;
-    rmsnorm_kernel<<<grid_rows(T, num_sms), 256, 0, stream>>>(x, u, T, H, eps);
-    return cudaGetLastError();
+    return launch_k(rmsnorm_kernel, dim3(grid_rows(T, num_sms)), dim3(256), 0, stream, x, u, T, H, eps);
 }
 
 cudaError_t launch_quantize(int64_t n_tensors, int64_t elems, const uint16_t* src, uint8_t* codes,

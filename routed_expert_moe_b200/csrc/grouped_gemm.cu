@@ -112,6 +112,7 @@ __global__ void __launch_bounds__(GG_THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
+    pdl_enter();   // after the local setup: nothing above reads what an earlier kernel writes
 
     const int n_units = (*g.n_sched) * g.m_blocks;
 
@@ -344,8 +345,7 @@ static cudaError_t launch_one(const GemmMaps& maps, const GemmArgs& g, int grid,
     auto kfn = grouped_gemm_kernel<FP8, UP>;
     cudaError_t err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
-    kfn<<<grid, GG_THREADS, smem, stream>>>(maps, g, ctx);
-    return cudaGetLastError();
+    return launch_k(kfn, dim3(grid), dim3(GG_THREADS), smem, stream, maps, g, ctx);
 }
 
 // One grouped projection.  W: [E * Nout][Kdim] (bf16 or e4m3), act: [rows][Kdim]

@@ -181,6 +181,7 @@ __global__ void __launch_bounds__(P2_THREADS, 1)
     cluster_sync();   // both CTAs' barriers initialised and TMEM allocated
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
+    pdl_enter();   // after the local setup: nothing above reads what an earlier kernel writes
 
     const int n_units = (*g.n_sched) * g.m_pairs;
 
@@ -382,7 +383,7 @@ cudaError_t launch_pair(const Gemm2Maps& maps, const Gemm2Args& g, int64_t max_u
     cudaError_t err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
@@ -390,8 +391,10 @@ cudaError_t launch_pair(const Gemm2Maps& maps, const Gemm2Args& g, int64_t max_u
     cfg.blockDim = dim3(P2_THREADS);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = pdl_enabled() ? 2 : 1;
     // every pair must be resident at once (the kernel is persistent)
     int max_clusters = 0;
     cfg.gridDim = dim3(2 * (unsigned)(num_sms / 2));

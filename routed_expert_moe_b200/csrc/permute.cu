@@ -95,6 +95,7 @@ struct PermuteArgs {
 };
 
 __global__ void __launch_bounds__(PM_THREADS) permute_kernel(PermuteArgs a, DevCtx ctx) {
+    pdl_enter();
     extern __shared__ int sm[];
     const int E = a.E;
     int* hist = sm;               // [E]
@@ -171,6 +172,7 @@ __global__ void __launch_bounds__(PM_THREADS) permute_kernel(PermuteArgs a, DevC
 
 __global__ void __launch_bounds__(PM_THREADS) perm_hist_kernel(const int32_t* __restrict__ idx, int64_t n, int E,
                                                                int* __restrict__ bcount, DevCtx ctx) {
+    pdl_enter();
     __shared__ int hist[256];
     const int tid = threadIdx.x;
     for (int e = tid; e < E; e += PM_THREADS) hist[e] = 0;
@@ -192,6 +194,7 @@ __global__ void __launch_bounds__(PM_THREADS) perm_hist_kernel(const int32_t* __
 __global__ void __launch_bounds__(256) perm_scan_kernel(const int* __restrict__ bcount, int G, int E,
                                                         int* __restrict__ bbase, int32_t* counts,
                                                         int32_t* offsets, int4* sched, int* n_sched, int bn) {
+    pdl_enter();
     __shared__ int offs[257];
     __shared__ int nb[256];
     const int tid = threadIdx.x;
@@ -222,6 +225,7 @@ __global__ void __launch_bounds__(PM_THREADS) perm_scatter_kernel(const int32_t*
                                                                   int E, const int* __restrict__ bbase,
                                                                   int32_t* __restrict__ perm_src,
                                                                   int32_t* __restrict__ inv_row) {
+    pdl_enter();
     extern __shared__ int wtab[];   // [32][E]
     const int tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
     const int64_t i = (int64_t)blockIdx.x * PM_THREADS + tid;
@@ -250,6 +254,7 @@ __global__ void __launch_bounds__(PM_THREADS) perm_scatter_kernel(const int32_t*
 }
 
 __global__ void schedule_kernel(const int32_t* offsets, int E, int bn, int4* sched, int* n_sched) {
+    pdl_enter();
     __shared__ int offs[257];
     __shared__ int nb[256];
     for (int e = threadIdx.x; e <= E; e += blockDim.x) offs[e] = offsets[e];
@@ -262,6 +267,7 @@ __global__ void schedule_kernel(const int32_t* offsets, int E, int bn, int4* sch
 __global__ void gather_rows_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm_src,
                                    int64_t rows, int K, int64_t T, int H, void* __restrict__ xp,
                                    int fp8, float x_scale, DevCtx ctx) {
+    pdl_enter();
     const int lane = threadIdx.x % 32;
     const int64_t warps = (int64_t)gridDim.x * (blockDim.x / 32);
     const int nv = H / 8;
@@ -314,24 +320,24 @@ cudaError_t launch_permute(const int32_t* idx, int64_t n, int E, int32_t* counts
                            int* scratch, const DevCtx& ctx, cudaStream_t stream) {
     if (n <= kPermuteOneBlockMax) {
         PermuteArgs a{idx, n, E, counts, offsets, perm_src, inv_row, sched, n_sched, bn};
-        permute_kernel<<<1, PM_THREADS, permute_smem_bytes(E), stream>>>(a, ctx);
-        return cudaGetLastError();
+        return launch_k(permute_kernel, dim3(1), dim3(PM_THREADS), permute_smem_bytes(E), stream, a, ctx);
     }
     if (!scratch) return cudaErrorInvalidValue;
     const int G = (int)((n + PM_THREADS - 1) / PM_THREADS);
     int* bcount = scratch;
     int* bbase = scratch + (size_t)G * E;
-    perm_hist_kernel<<<G, PM_THREADS, 0, stream>>>(idx, n, E, bcount, ctx);
-    perm_scan_kernel<<<1, 256, 0, stream>>>(bcount, G, E, bbase, counts, offsets, sched, n_sched, bn);
-    perm_scatter_kernel<<<G, PM_THREADS, (size_t)32 * E * sizeof(int), stream>>>(idx, n, E, bbase, perm_src,
-                                                                                  inv_row);
-    return cudaGetLastError();
+    cudaError_t err = launch_k(perm_hist_kernel, dim3(G), dim3(PM_THREADS), 0, stream, idx, n, E, bcount, ctx);
+    if (err != cudaSuccess) return err;
+    err = launch_k(perm_scan_kernel, dim3(1), dim3(256), 0, stream, bcount, G, E, bbase, counts, offsets, sched,
+                   n_sched, bn);
+    if (err != cudaSuccess) return err;
+    return launch_k(perm_scatter_kernel, dim3(G), dim3(PM_THREADS), (size_t)32 * E * sizeof(int), stream, idx, n,
+                    E, bbase, perm_src, inv_row);
 }
 
 cudaError_t launch_schedule(const int32_t* offsets, int E, int bn, int4* sched, int* n_sched,
                             cudaStream_t stream) {
-    schedule_kernel<<<1, 256, 0, stream>>>(offsets, E, bn, sched, n_sched);
-    return cudaGetLastError();
+    return launch_k(schedule_kernel, dim3(1), dim3(256), 0, stream, offsets, E, bn, sched, n_sched);
 }
 
 cudaError_t launch_gather(const uint16_t* x, const int32_t* perm_src, int64_t rows, int K, int64_t T,
@@ -341,9 +347,8 @@ cudaError_t launch_gather(const uint16_t* x, const int32_t* perm_src, int64_t ro
     int64_t blocks = (rows + 7) / 8;
     const int64_t cap = (int64_t)num_sms * 8;
     if (blocks > cap) blocks = cap;
-    gather_rows_kernel<<<(unsigned)blocks, 256, 0, stream>>>(x, perm_src, rows, K, T, H, xp,
-                                                              fp8 ? 1 : 0, x_scale, ctx);
-    return cudaGetLastError();
+    return launch_k(gather_rows_kernel, dim3((unsigned)blocks), dim3(256), 0, stream, x, perm_src, rows, K, T, H, xp,
+                    fp8 ? 1 : 0, x_scale, ctx);
 }
 
 }  // namespace moe

@@ -56,6 +56,7 @@ struct RouterLogitsArgs {
 // ones so that a decode batch still spreads over the whole GPU.
 template <int TPT>
 __global__ void __launch_bounds__(RT_THREADS) router_logits_kernel(RouterLogitsArgs a) {
+    pdl_enter();
     constexpr int RT_TT = 16 * TPT;
     __shared__ __align__(16) float xs[2][RT_HC][RT_TT];
     __shared__ __align__(16) float ws[2][RT_HC][RT_TE];
@@ -468,6 +469,7 @@ __device__ __forceinline__ void finish_token(bool certified, int slot, int64_t t
 // their candidates in a block-wide list whose exact logits all 8 warps
 // compute together, then finish their selection from it.
 __global__ void __launch_bounds__(TK_WARPS * 32, 2) router_topk_kernel(RouterTopkArgs a, DevCtx ctx) {
+    pdl_enter();
     __shared__ uint8_t c_tok[TK_CAP];
     __shared__ uint16_t c_e[TK_CAP];
     __shared__ long long c_val[TK_CAP];
@@ -608,6 +610,7 @@ __device__ __forceinline__ void bf16x8(const uint4& v, float (&f)[8]) {
 template <int TB>
 __global__ void __cluster_dims__(RS_CLUSTER, 1, 1) __launch_bounds__(RS_THREADS)
     router_small_kernel(RouterSmallArgs a, DevCtx ctx) {
+    pdl_enter();
     namespace cg = cooperative_groups;
     extern __shared__ __align__(16) unsigned char rs_smem[];
     const int H = a.H, E = a.E;
@@ -862,6 +865,7 @@ struct RfLayout {
 template <int NTH, int CS>
 __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(NTH, 1)
     router_fused_kernel(RouterFusedArgs a, DevCtx ctx) {
+    pdl_enter();
     namespace cg = cooperative_groups;
     using L = RfLayout<NTH, CS>;
     constexpr int BT = L::BT, TPC = L::TPC, WARPS = L::WARPS, TPW = L::TPW, NWF = L::NWF;
@@ -1197,8 +1201,7 @@ static cudaError_t launch_router_fused(const RouterFusedArgs& ra, const DevCtx& 
     cudaError_t err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::bytes);
     if (err != cudaSuccess) return err;
     const unsigned tiles = (unsigned)((ra.T + L::BT - 1) / L::BT);
-    kfn<<<tiles * CS, NTH, L::bytes, stream>>>(ra, ctx);
-    return cudaGetLastError();
+    return launch_k(kfn, dim3(tiles * CS), dim3(NTH), L::bytes, stream, ra, ctx);
 }
 
 template <int TB>
@@ -1208,8 +1211,7 @@ static cudaError_t launch_router_small(const RouterSmallArgs& ra, const DevCtx& 
     cudaError_t err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     const unsigned groups = (unsigned)((ra.T + TB - 1) / TB);
-    kfn<<<groups * RS_CLUSTER, RS_THREADS, smem, stream>>>(ra, ctx);
-    return cudaGetLastError();
+    return launch_k(kfn, dim3(groups * RS_CLUSTER), dim3(RS_THREADS), smem, stream, ra, ctx);
 }
 
 cudaError_t launch_route(const uint16_t* x, const uint16_t* wr, const float* bias, int64_t T, int H,
@@ -1242,17 +1244,13 @@ cudaError_t launch_route(const uint16_t* x, const uint16_t* wr, const float* bia
     RouterLogitsArgs la{x, wr, T, H, E, plan.S, plan.nchunks, P, xn2, wn2};
     const int tt = router_tt(T);
     dim3 grid((unsigned)((T + tt - 1) / tt), (unsigned)((E + RT_TE - 1) / RT_TE), (unsigned)plan.S);
-    if (tt == 64)
-        router_logits_kernel<4><<<grid, RT_THREADS, 0, stream>>>(la);
-    else
-        router_logits_kernel<1><<<grid, RT_THREADS, 0, stream>>>(la);
-    cudaError_t err = cudaGetLastError();
+    cudaError_t err = tt == 64 ? launch_k(router_logits_kernel<4>, grid, dim3(RT_THREADS), 0, stream, la)
+                               : launch_k(router_logits_kernel<1>, grid, dim3(RT_THREADS), 0, stream, la);
     if (err != cudaSuccess) return err;
     if (between) between(stream);
     RouterTopkArgs ta{P, xn2, wn2, x, wr, bias, T, H, E, K, plan.S, plan.nchunks, idx, w};
     const unsigned blocks = (unsigned)((T + TK_WARPS - 1) / TK_WARPS);
-    router_topk_kernel<<<blocks, TK_WARPS * 32, 0, stream>>>(ta, ctx);
-    return cudaGetLastError();
+    return launch_k(router_topk_kernel, dim3(blocks), dim3(TK_WARPS * 32), 0, stream, ta, ctx);
 }
 
 }  // namespace moe
