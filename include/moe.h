@@ -150,6 +150,16 @@ moe_status moe_forward(const moe_dims* d, const void* x, const void* w_router, c
 moe_status moe_quantize_fp8(int64_t n_tensors, int64_t tensor_elems, const void* src,
                             uint8_t* codes, float* scales, void* stream);
 
+/* Activation quantisation with a static scale (the X side of W8A8):
+ * codes[r][h] = e4m3_rne_satfinite(fl32(x[r][h] / x_scale)), the quotient
+ * rounded to nearest in fp32.  This is the step moe_forward and
+ * moe_expert_ffn apply to the permuted rows, here on rows in order.
+ *   x [rows][H] bf16 (16-byte aligned), codes [rows][H] uint8; H a multiple
+ * of 16; x_scale > 0 and finite.  Cited: bloomery page s.2 ("scalar-scale
+ * E4M3 W8A8"). */
+moe_status moe_quantize_act_fp8(int64_t rows, int32_t H, float x_scale, const void* x, uint8_t* codes,
+                                void* stream);
+
 /* RMS normalisation with unit gain of the residual stream between chained
  * layers: u = bf16(x / sqrt(mean(x^2) + eps)), the mean of squares taken
  * exactly (fixed point, 2^-16 per term) and the rest in correctly rounded fp32.

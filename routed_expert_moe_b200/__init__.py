@@ -52,6 +52,7 @@ _SIG = {
                                    _P, _P, _S, _P]),
     "moe_quantize_fp8": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int64, _P, _P, _P, _P]),
     "moe_rmsnorm": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int32, ctypes.c_float, _P, _P, _P]),
+    "moe_quantize_act_fp8": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int32, ctypes.c_float, _P, _P, _P]),
     "moe_check_device_error": (ctypes.c_int, [_P]),
     "moe_set_stage_events": (ctypes.c_int, [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32]),
     "moe_debug_set": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int64]),
@@ -159,6 +160,13 @@ def quantize_fp8(src, codes, scales, stream=None):
     per = src.numel() // max(n, 1)
     _check(_lib.moe_quantize_fp8(n, per, _ptr(src), _ptr(codes), _ptr(scales), _stream(stream)),
            "moe_quantize_fp8")
+
+
+def quantize_act_fp8(x, codes, x_scale, stream=None):
+    """E4M3 codes of x [rows, H] (bf16) with the static scale x_scale: e4m3(fl32(x / x_scale))."""
+    rows, H = x.shape
+    _check(_lib.moe_quantize_act_fp8(rows, H, float(x_scale), _ptr(x), _ptr(codes), _stream(stream)),
+           "moe_quantize_act_fp8")
 
 
 def rmsnorm(x, u, eps=1e-5, stream=None):

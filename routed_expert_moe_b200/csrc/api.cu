@@ -441,6 +441,19 @@ moe_status moe_quantize_fp8(int64_t n_tensors, int64_t tensor_elems, const void*
                                        dev->num_sms, static_cast<cudaStream_t>(stream)));
 }
 
+moe_status moe_quantize_act_fp8(int64_t rows, int32_t H, float x_scale, const void* x, uint8_t* codes,
+                                void* stream) {
+    if (rows < 0 || H < 16 || H > 65536 || H % 16 != 0) return MOE_EINVAL;
+    if (!(x_scale > 0.0f) || !(x_scale < 3.4e38f)) return MOE_EINVAL;
+    if (rows == 0) return MOE_OK;
+    if (!x || !codes || !aligned(x, 16) || !aligned(codes, 16)) return MOE_EINVAL;
+    DeviceInfo* dev = nullptr;
+    moe_status s = device_setup(&dev);
+    if (s != MOE_OK) return s;
+    return cuda_status(launch_gather(static_cast<const uint16_t*>(x), nullptr, rows, 1, rows, H, codes, true,
+                                     x_scale, dev->num_sms, make_ctx(dev), static_cast<cudaStream_t>(stream)));
+}
+
 moe_status moe_rmsnorm(int64_t T, int32_t H, float eps, const void* x, void* u, void* stream) {
     if (T < 0 || H < 16 || H > 65536 || H % 16 != 0 || !(eps >= 0.0f)) return MOE_EINVAL;
     if (T == 0) return MOE_OK;

@@ -12,11 +12,15 @@ namespace moe {
 
 // out[t] = (residual[t] +) sum_{k=0..K-1} w[t][k] * y_perm[inv_row[t*K+k]]
 // in fp32, k ascending (descending routing logit), one rounding to bf16.
-// One block per token (grid-stride over tokens): the K row indices and
-// weights are staged in shared memory, then every thread streams 16-byte
-// vectors of the K rows; a token's H/8 vectors are all in flight at once.
-constexpr int CB_THREADS = 128;
+// One warp per (token, chunk of 64 16-byte vectors), grid-stride: lane
+// k < K loads the token's k-th row index and weight, the others get them by
+// shuffle; each lane then loads two vectors of all K rows at once (2K loads
+// in flight).  Small batches thus still spread over the whole GPU.
+// KMAX (8 or 16) bounds K at compile time so that the vectors stay in
+// registers.
+constexpr int CB_THREADS = 256;
 
+template <int KMAX>
 __global__ void __launch_bounds__(CB_THREADS) combine_kernel(const uint16_t* __restrict__ yp,
                                                              const int32_t* __restrict__ inv_row,
                                                              const float* __restrict__ w,
@@ -24,60 +28,87 @@ __global__ void __launch_bounds__(CB_THREADS) combine_kernel(const uint16_t* __r
                                                              int64_t T, int K, int H, int64_t rows,
                                                              DevCtx ctx) {
     pdl_enter();
-    __shared__ int row_k[16];
-    __shared__ float w_k[16];
+    const int lane = threadIdx.x % 32;
     const int nv = H / 8;
-    for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
-        if (threadIdx.x < K) {
-            int r = inv_row[t * K + threadIdx.x];
-            float wk = w[t * K + threadIdx.x];
-            if (r < 0 || r >= rows) {
+    const int wpb = blockDim.x / 32;
+    const int64_t warps = (int64_t)gridDim.x * wpb;
+    const int nchunk = (nv + 63) / 64;
+    for (int64_t item = (int64_t)blockIdx.x * wpb + threadIdx.x / 32; item < T * nchunk; item += warps) {
+        const int64_t t = item / nchunk;
+        const int v0 = (int)(item - t * nchunk) * 64 + lane;
+        int my_r = 0;
+        float my_w = 0.0f;
+        if (lane < K) {
+            my_r = inv_row[t * K + lane];
+            my_w = w[t * K + lane];
+            if (my_r < 0 || my_r >= rows) {
                 record_error(ctx.err, MOE_EINDEX);
-                r = 0;
-                wk = 0.0f;
+                my_r = 0;
+                my_w = 0.0f;
             }
-            row_k[threadIdx.x] = r;
-            w_k[threadIdx.x] = wk;
         }
-        __syncthreads();
-        for (int v = threadIdx.x; v < nv; v += CB_THREADS) {
-            uint4 q[16];
+        const uint4* src[KMAX];
+        float wk[KMAX];
 #pragma unroll
-            for (int k = 0; k < 16; ++k)
-                if (k < K) q[k] = reinterpret_cast<const uint4*>(yp + (int64_t)row_k[k] * H)[v];
-            float acc[8];
+        for (int k = 0; k < KMAX; ++k) {
+            const int r = __shfl_sync(0xffffffffu, my_r, k);
+            wk[k] = __shfl_sync(0xffffffffu, my_w, k);
+            src[k] = reinterpret_cast<const uint4*>(yp + (int64_t)r * H);
+        }
+        const uint4* res = residual ? reinterpret_cast<const uint4*>(residual + t * H) : nullptr;
+        uint4* dst = reinterpret_cast<uint4*>(out + t * H);
+        if (v0 < nv) {
+            const int v1 = v0 + 32;
+            const bool has1 = v1 < nv;
+            uint4 q0[KMAX], q1[KMAX];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
-#pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                if (k >= K) break;
-                const float wk = w_k[k];
-                const uint32_t qq[4] = {q[k].x, q[k].y, q[k].z, q[k].w};
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    acc[2 * j] = __fmaf_rn(wk, __uint_as_float(qq[j] << 16), acc[2 * j]);
-                    acc[2 * j + 1] = __fmaf_rn(wk, __uint_as_float(qq[j] & 0xFFFF0000u), acc[2 * j + 1]);
+            for (int k = 0; k < KMAX; ++k) {
+                if (k < K) {
+                    q0[k] = src[k][v0];
+                    if (has1) q1[k] = src[k][v1];
                 }
             }
-            if (residual) {
-                const uint4 r4 = reinterpret_cast<const uint4*>(residual + t * H)[v];
-                const uint32_t qq[4] = {r4.x, r4.y, r4.z, r4.w};
+            uint4 r0, r1;
+            if (res) {
+                r0 = res[v0];
+                if (has1) r1 = res[v1];
+            }
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                if (half == 1 && !has1) break;
+                float acc[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
+#pragma unroll
+                for (int k = 0; k < KMAX; ++k) {
+                    if (k >= K) break;
+                    const uint4 q = half ? q1[k] : q0[k];
+                    const uint32_t qq[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        acc[2 * j] = __fmaf_rn(wk[k], __uint_as_float(qq[j] << 16), acc[2 * j]);
+                        acc[2 * j + 1] = __fmaf_rn(wk[k], __uint_as_float(qq[j] & 0xFFFF0000u), acc[2 * j + 1]);
+                    }
+                }
+                if (res) {
+                    const uint4 r4 = half ? r1 : r0;
+                    const uint32_t qq[4] = {r4.x, r4.y, r4.z, r4.w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        acc[2 * j] = __fadd_rn(__uint_as_float(qq[j] << 16), acc[2 * j]);
+                        acc[2 * j + 1] = __fadd_rn(__uint_as_float(qq[j] & 0xFFFF0000u), acc[2 * j + 1]);
+                    }
+                }
+                uint32_t o[4];
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    acc[2 * j] = __fadd_rn(__uint_as_float(qq[j] << 16), acc[2 * j]);
-                    acc[2 * j + 1] = __fadd_rn(__uint_as_float(qq[j] & 0xFFFF0000u), acc[2 * j + 1]);
+                    const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(acc[2 * j]));
+                    const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(acc[2 * j + 1]));
+                    o[j] = lo | (hi << 16);
                 }
+                dst[half ? v1 : v0] = make_uint4(o[0], o[1], o[2], o[3]);
             }
-            uint32_t o[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(acc[2 * j]));
-                const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(acc[2 * j + 1]));
-                o[j] = lo | (hi << 16);
-            }
-            reinterpret_cast<uint4*>(out + t * H)[v] = make_uint4(o[0], o[1], o[2], o[3]);
         }
-        __syncthreads();
     }
 }
 
@@ -182,10 +213,18 @@ cudaError_t launch_combine(const uint16_t* yp, const int32_t* inv_row, const flo
                            const uint16_t* residual, uint16_t* out, int64_t T, int K, int H,
                            int num_sms, const DevCtx& ctx, cudaStream_t stream) {
     if (T == 0) return cudaSuccess;
+    // warps per block: small batches spread over the SMs, large ones 8 per block
+    const int64_t items = T * ((H / 8 + 63) / 64);
+    int64_t wpb = items / num_sms;
+    if (wpb < 1) wpb = 1;
+    if (wpb > CB_THREADS / 32) wpb = CB_THREADS / 32;
     const int64_t cap = (int64_t)num_sms * 16;
-    const unsigned grid = (unsigned)(T < cap ? T : cap);
-    return launch_k(combine_kernel, dim3(grid), dim3(CB_THREADS), 0, stream, yp, inv_row, w, residual, out, T, K, H,
-                    T * K, ctx);
+    int64_t blocks = (items + wpb - 1) / wpb;
+    if (blocks > cap) blocks = cap;
+    const dim3 grid((unsigned)blocks), block((unsigned)(32 * wpb));
+    if (K <= 8)
+        return launch_k(combine_kernel<8>, grid, block, 0, stream, yp, inv_row, w, residual, out, T, K, H, T * K, ctx);
+    return launch_k(combine_kernel<16>, grid, block, 0, stream, yp, inv_row, w, residual, out, T, K, H, T * K, ctx);
 }
 
 cudaError_t launch_rmsnorm(const uint16_t* x, uint16_t* u, int64_t T, int H, float eps, int num_sms,

@@ -262,15 +262,33 @@ __global__ void schedule_kernel(const int32_t* offsets, int E, int bn, int4* sch
     build_schedule(offs, E, bn, nb, sched, n_sched);
 }
 
+// x / s rounded to nearest from y = RN(1/s): q = RN(x y), r = x - s q (exact,
+// one FMA), q' = RN(q + r y) -- Markstein's correction of a reciprocal
+// quotient (P. Markstein, "Computation of elementary functions on the IBM
+// RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990).  Zeros and
+// non-finite q are returned as they are (the correction would lose the sign
+// of a zero or turn an overflow into NaN).  The library's tests compare the
+// E4M3 codes this produces with those of a correctly rounded division for
+// every bf16 input at the scales in use.
+__device__ __forceinline__ float div_by_scale(float x, float s, float y) {
+    const float q = __fmul_rn(x, y);
+    if (q == 0.0f || !isfinite(q)) return q;
+    const float r = __fmaf_rn(-q, s, x);
+    return __fmaf_rn(r, y, q);
+}
+
 // xp[r] = x[perm_src[r] / K], or its E4M3 codes e4m3(x / x_scale) (fp8);
-// with perm_src == null the rows are taken in order (xp[r] = x[r]).
+// with perm_src == null the rows are taken in order (xp[r] = x[r]).  One
+// warp per row, four 16-byte loads per lane in flight before their stores.
 __global__ void gather_rows_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm_src,
                                    int64_t rows, int K, int64_t T, int H, void* __restrict__ xp,
                                    int fp8, float x_scale, DevCtx ctx) {
     pdl_enter();
+    constexpr int B = 4;
     const int lane = threadIdx.x % 32;
     const int64_t warps = (int64_t)gridDim.x * (blockDim.x / 32);
     const int nv = H / 8;
+    const float y = fp8 ? __frcp_rn(x_scale) : 1.0f;
     for (int64_t r = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32; r < rows; r += warps) {
         int64_t t = r;
         if (perm_src) {
@@ -282,23 +300,32 @@ __global__ void gather_rows_kernel(const uint16_t* __restrict__ x, const int32_t
             }
         }
         const uint4* xr = reinterpret_cast<const uint4*>(x + t * H);
-        if (!fp8) {
-            uint4* out = reinterpret_cast<uint4*>(static_cast<uint16_t*>(xp) + r * H);
-            for (int v = lane; v < nv; v += 32) out[v] = xr[v];
-        } else {
-            uint2* out = reinterpret_cast<uint2*>(static_cast<uint8_t*>(xp) + r * H);
-            for (int v = lane; v < nv; v += 32) {
-                const uint4 q = xr[v];
-                const uint32_t wv[4] = {q.x, q.y, q.z, q.w};
-                uint32_t packed[2] = {0, 0};
+        for (int v0 = lane; v0 < nv; v0 += 32 * B) {
+            uint4 q[B];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const uint32_t bits = (j & 1) ? (wv[j / 2] & 0xFFFF0000u) : (wv[j / 2] << 16);
-                    const float f = __fdiv_rn(__uint_as_float(bits), x_scale);
-                    const uint32_t c = __nv_cvt_float_to_fp8(f, __NV_SATFINITE, __NV_E4M3);
-                    packed[j / 4] |= c << (8 * (j % 4));
+            for (int i = 0; i < B; ++i)
+                if (v0 + 32 * i < nv) q[i] = xr[v0 + 32 * i];
+            if (!fp8) {
+                uint4* out = reinterpret_cast<uint4*>(static_cast<uint16_t*>(xp) + r * H);
+#pragma unroll
+                for (int i = 0; i < B; ++i)
+                    if (v0 + 32 * i < nv) out[v0 + 32 * i] = q[i];
+            } else {
+                uint2* out = reinterpret_cast<uint2*>(static_cast<uint8_t*>(xp) + r * H);
+#pragma unroll
+                for (int i = 0; i < B; ++i) {
+                    if (v0 + 32 * i >= nv) continue;
+                    const uint32_t wv[4] = {q[i].x, q[i].y, q[i].z, q[i].w};
+                    uint32_t packed[2] = {0, 0};
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const uint32_t bits = (j & 1) ? (wv[j / 2] & 0xFFFF0000u) : (wv[j / 2] << 16);
+                        const float f = div_by_scale(__uint_as_float(bits), x_scale, y);
+                        const uint32_t c = __nv_cvt_float_to_fp8(f, __NV_SATFINITE, __NV_E4M3);
+                        packed[j / 4] |= c << (8 * (j % 4));
+                    }
+                    out[v0 + 32 * i] = make_uint2(packed[0], packed[1]);
                 }
-                out[v] = make_uint2(packed[0], packed[1]);
             }
         }
     }

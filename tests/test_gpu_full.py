@@ -106,6 +106,33 @@ def test_quantize_fp8_zero_tensor_and_saturation(moe):
     assert np.array_equal(codes.cpu().numpy(), q_ref)
 
 
+def _act_scales():
+    sc = [np.float32(v) for v in (1.0, 0.001, 37.0, 448.0, 1.0 / 3.0, 0.0371, 2.0 ** -20, 6.1e4)]
+    for sx, sh in W.chain_scales():
+        sc += [sx, sh]
+    rng = np.random.default_rng(31)
+    sc += [np.float32(v) for v in np.exp(rng.uniform(np.log(1e-4), np.log(1e3), 16))]
+    return sc
+
+
+def test_activation_codes_match_a_correctly_rounded_division_for_every_bf16(moe):
+    """Every bf16 bit pattern but NaN, at every static scale of the chain workload and
+    24 more: the kernel's E4M3 codes of x / s (a reciprocal quotient with one FMA
+    correction) equal the oracle's, which divides with one correctly rounded fp32
+    division."""
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    nan = ((bits & 0x7F80) == 0x7F80) & ((bits & 0x007F) != 0)
+    bits = np.where(nan, np.uint16(0), bits).reshape(256, 256)
+    x = dev_bf16(bits)
+    codes = torch.empty(256, 256, dtype=torch.uint8, device="cuda")
+    for s in _act_scales():
+        moe.quantize_act_fp8(x, codes, float(s))
+        torch.cuda.synchronize()
+        ref = oracle.quantize_act_fp8(bits, float(s)).reshape(256, 256)
+        got = codes.cpu().numpy()
+        assert np.array_equal(got, ref), (float(s), int(np.sum(got != ref)))
+
+
 @pytest.mark.parametrize("scale", [1.0, 0.001, 37.0])
 def test_rmsnorm_bit_exact(moe, scale):
     x = synth.normal_bf16(synth.key(4, 7, 1), 300 * 2688, scale).reshape(300, 2688)
