@@ -63,6 +63,16 @@ def lib():
             "oracle_rmsnorm_bf16": (None, [_i64, _i64, _p, _f, _p]),
             "oracle_round_bf16": (None, [_i64, _p, _p]),
             "oracle_hidden_amax_bf16": (ctypes.c_double, [_i64, _i64, _i64, _p, _p, _p, _p]),
+            "oracle_e2m1_encode": (ctypes.c_uint8, [_f]),
+            "oracle_e2m1_decode": (_f, [ctypes.c_uint8]),
+            "oracle_e2m1_encode_n": (None, [_i64, _p, _p]),
+            "oracle_e2m1_decode_n": (None, [_i64, _p, _p]),
+            "oracle_nvfp4_tensor_scale": (_f, [_i64, _p]),
+            "oracle_quantize_nvfp4": (None, [_i64, _i64, _p, _f, _p, _p]),
+            "oracle_dequantize_nvfp4": (None, [_i64, _i64, _p, _p, _f, _p]),
+            "oracle_expert_nvfp4": (None, [_i64, _i64, _p, _p, _f, _p, _p, _f, _p, _p, _f, _f, _p]),
+            "oracle_expert_rows_nvfp4": (ctypes.c_int, [_i64, _i64, _i64, _p, _p, _p, _p, _p, _p, _p, _p, _p,
+                                                        _p, _f, _f, _p]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -256,6 +266,117 @@ def moe_layer_fp8(x, wr, bias, qup, sup, qdown, sdown, sx, sh, K, tokens=None, s
     y = expert_rows_fp8(qxr, idx.reshape(-1), qup, sup, qdown, sdown, slot, sx, sh).reshape(n, K, H)
     out = combine(y, w, residual)
     return dict(logits=L, idx=idx, w=w, y=y, out=out, qx=qx)
+
+
+# --------------------------------------------------------------------------- NVFP4
+
+def e2m1_encode(v) -> np.ndarray:
+    v, pv = _c(v, np.float32)
+    q = np.empty(v.shape, dtype=np.uint8)
+    lib().oracle_e2m1_encode_n(v.size, pv, q.ctypes.data)
+    return q
+
+
+def e2m1_decode(q) -> np.ndarray:
+    q, pq = _c(q, np.uint8)
+    v = np.empty(q.shape, dtype=np.float32)
+    lib().oracle_e2m1_decode_n(q.size, pq, v.ctypes.data)
+    return v
+
+
+def nvfp4_tensor_scale(x) -> np.float32:
+    x, px = _c(x, np.uint16)
+    return np.float32(lib().oracle_nvfp4_tensor_scale(x.size, px))
+
+
+def quantize_nvfp4(x, s_t):
+    """NVFP4 codes of a bf16 tensor [rows, K] with tensor scale s_t:
+    (packed codes [rows, K/2] uint8, block scale codes [rows, K/16] uint8)."""
+    x, px = _c(x, np.uint16)
+    rows, K = x.shape
+    codes = np.empty((rows, K // 2), dtype=np.uint8)
+    scales = np.empty((rows, K // 16), dtype=np.uint8)
+    lib().oracle_quantize_nvfp4(rows, K, px, np.float32(s_t), codes.ctypes.data, scales.ctypes.data)
+    return codes, scales
+
+
+def dequantize_nvfp4(codes, scales, s_t) -> np.ndarray:
+    codes, pc = _c(codes, np.uint8)
+    scales, ps = _c(scales, np.uint8)
+    rows = codes.shape[0]
+    K = codes.shape[1] * 2
+    out = np.empty((rows, K), dtype=np.float64)
+    lib().oracle_dequantize_nvfp4(rows, K, pc, ps, np.float32(s_t), out.ctypes.data)
+    return out
+
+
+def quantize_bank_nvfp4(bank):
+    """Each expert tensor of a bank [S, rows, K] with its own tensor scale amax / 2688:
+    (codes [S, rows, K/2], block scales [S, rows, K/16], tensor scales [S] fp32)."""
+    S, rows, K = bank.shape
+    c = np.empty((S, rows, K // 2), dtype=np.uint8)
+    sc = np.empty((S, rows, K // 16), dtype=np.uint8)
+    t = np.empty(S, dtype=np.float32)
+    for i in range(S):
+        t[i] = nvfp4_tensor_scale(bank[i])
+        c[i], sc[i] = quantize_nvfp4(bank[i], t[i])
+    return c, sc, t
+
+
+def expert_rows_nvfp4(cx, sx, ex, bank_up, bank_down, slot, tx, th) -> np.ndarray:
+    """W4A4 experts on NVFP4 rows (cx [R, H/2], sx [R, H/16]); banks from quantize_bank_nvfp4."""
+    cx, pcx = _c(cx, np.uint8)
+    sx, psx = _c(sx, np.uint8)
+    ex, pe = _c(ex, np.int32)
+    cu, pcu = _c(bank_up[0], np.uint8)
+    su, psu = _c(bank_up[1], np.uint8)
+    tu, ptu = _c(bank_up[2], np.float32)
+    cd, pcd = _c(bank_down[0], np.uint8)
+    sd, psd = _c(bank_down[1], np.uint8)
+    td, ptd = _c(bank_down[2], np.float32)
+    slot, ps = _c(slot, np.int32)
+    R = cx.shape[0]
+    H = cx.shape[1] * 2
+    F = cu.shape[1]
+    y = np.empty((R, H), dtype=np.float64)
+    rc = lib().oracle_expert_rows_nvfp4(R, H, F, pcx, psx, pe, pcu, psu, ptu, pcd, psd, ptd, ps,
+                                        np.float32(tx), np.float32(th), y.ctypes.data)
+    if rc != 0:
+        raise ValueError("a routed expert's bank was not supplied")
+    return y
+
+
+def moe_layer_nvfp4(x, wr, bias, bank_up, bank_down, tx, th, K, tokens=None, slot=None, residual=None):
+    """W4A4 layer: bf16 router on x; x and H quantised to NVFP4 with static tensor scales."""
+    x = np.asarray(x, dtype=np.uint16)
+    if tokens is not None:
+        x = x[np.asarray(tokens)]
+        if residual is not None:
+            residual = np.asarray(residual)[np.asarray(tokens)]
+    E = wr.shape[0]
+    if slot is None:
+        slot = identity_slot(E)
+    L, idx, w = route(x, wr, bias, K)
+    n, H = x.shape
+    cx, sx = quantize_nvfp4(x, tx)
+    y = expert_rows_nvfp4(np.repeat(cx, K, axis=0), np.repeat(sx, K, axis=0), idx.reshape(-1), bank_up,
+                          bank_down, slot, tx, th).reshape(n, K, H)
+    out = combine(y, w, residual)
+    return dict(logits=L, idx=idx, w=w, y=y, out=out, cx=cx, sx=sx)
+
+
+def calibrate_nvfp4(x_cal, wr, bias, wup, K, slot=None):
+    """Static NVFP4 activation tensor scales from a calibration batch of the bf16 model:
+    amax|x| / 2688 and amax(relu(z)^2) / 2688, both fp32 (6 x 448 = 2688)."""
+    x_cal = np.asarray(x_cal, dtype=np.uint16)
+    E = wr.shape[0]
+    if slot is None:
+        slot = identity_slot(E)
+    _, idx, _ = route(x_cal, wr, bias, K)
+    xf = bf16_to_f64(x_cal)
+    ax = np.float32(np.max(np.abs(xf)))
+    ah = hidden_amax_bf16(np.repeat(xf, K, axis=0), idx.reshape(-1), wup, slot)
+    return np.float32(ax / np.float32(2688.0)), np.float32(np.float32(ah) / np.float32(2688.0))
 
 
 def rmsnorm_bf16(x, eps: float = 1e-5) -> np.ndarray:

@@ -309,6 +309,167 @@ int oracle_expert_rows_fp8(int64_t R, int64_t H, int64_t F, const uint8_t* qxrow
     return 0;
 }
 
+/* ----------------------------------------------------------------------- */
+/* NVFP4 W4A4.  [B] s.2: the NVFP4 release runs the experts "W4A4".  The    */
+/* pages name the format without defining it; reading: NVIDIA's published  */
+/* NVFP4 -- E2M1 elements (magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6), one      */
+/* E4M3 scale per block of 16 consecutive elements along the contraction    */
+/* dimension, and one fp32 scale per tensor.  Quantisation (reading, the    */
+/* plainest recipe for that format):                                        */
+/*   s_t = amax|X| / 2688 (6 x 448; 1 for an all-zero tensor), or a static  */
+/*         calibrated value for activations;                                 */
+/*   per block b: S_b = e4m3(fl32(fl32(amax_b / 6) / s_t));                  */
+/*   e_b = fl32(dec(S_b) * s_t);  q = e2m1(fl32(x / e_b)), or 0 if e_b == 0;  */
+/*   E2M1 rounding: to nearest, ties to the even code, saturating at +-6.    */
+/* Dequantised value: dec(q) * dec(S_b) * s_t (exact in fp64).               */
+/* Codes are packed two per byte, element 2i in the low nibble.              */
+/* ----------------------------------------------------------------------- */
+
+static const double kE2m1Mag[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+uint8_t oracle_e2m1_encode(float v) {
+    uint8_t sign = signbit(v) ? 0x8 : 0x0;
+    double a = fabs((double)v);
+    if (isnan(v)) return 0;
+    if (a >= 6.0) return sign | 7;
+    /* walk the grid: the first point whose upper midpoint lies above a, ties to the even code */
+    int c = 0;
+    while (c < 7) {
+        double mid = 0.5 * (kE2m1Mag[c] + kE2m1Mag[c + 1]);
+        if (a < mid) break;
+        if (a == mid) {
+            if (c % 2 == 1) c += 1;   /* the upper neighbour has the even code */
+            break;
+        }
+        c += 1;
+    }
+    return sign | (uint8_t)c;
+}
+
+float oracle_e2m1_decode(uint8_t q) {
+    double v = kE2m1Mag[q & 7];
+    return (float)((q & 8) ? -v : v);
+}
+
+/* One block: scale code and 16 element codes (unpacked), from fp32 values and the tensor scale. */
+static uint8_t nvfp4_block(const float* x, int n, float s_t, uint8_t* q) {
+    float amax = 0.0f;
+    for (int i = 0; i < n; ++i) {
+        float a = fabsf(x[i]);
+        if (a > amax) amax = a;
+    }
+    uint8_t sc = oracle_e4m3_encode((amax / 6.0f) / s_t);
+    float e = oracle_e4m3_decode(sc) * s_t;
+    for (int i = 0; i < n; ++i) q[i] = (e == 0.0f) ? 0 : oracle_e2m1_encode(x[i] / e);
+    return sc;
+}
+
+/* Tensor scale of a bf16 tensor: amax / 2688, 1 for an all-zero tensor. */
+float oracle_nvfp4_tensor_scale(int64_t n, const uint16_t* w) {
+    float amax = 0.0f;
+    for (int64_t i = 0; i < n; ++i) {
+        float a = fabsf(bf16_to_float(w[i]));
+        if (a > amax) amax = a;
+    }
+    return amax > 0.0f ? amax / 2688.0f : 1.0f;
+}
+
+/*
+ * NVFP4 quantisation of a [rows][K] bf16 tensor (K a multiple of 16) with
+ * tensor scale s_t: packed codes [rows][K/2], block scale codes [rows][K/16].
+ */
+void oracle_quantize_nvfp4(int64_t rows, int64_t K, const uint16_t* x, float s_t, uint8_t* codes,
+                           uint8_t* scales) {
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        float blk[16];
+        uint8_t q[16];
+        for (int64_t b = 0; b < K / 16; ++b) {
+            for (int i = 0; i < 16; ++i) blk[i] = bf16_to_float(x[r * K + b * 16 + i]);
+            scales[r * (K / 16) + b] = nvfp4_block(blk, 16, s_t, q);
+            for (int i = 0; i < 8; ++i)
+                codes[r * (K / 2) + b * 8 + i] = (uint8_t)(q[2 * i] | (q[2 * i + 1] << 4));
+        }
+    }
+}
+
+/* Dequantised value of element k of a row (codes [K/2], scales [K/16]). */
+static double nvfp4_value(const uint8_t* codes, const uint8_t* scales, int64_t k, float s_t) {
+    uint8_t byte = codes[k / 2];
+    uint8_t q = (k % 2) ? (byte >> 4) : (byte & 0xF);
+    return (double)oracle_e2m1_decode(q) * (double)oracle_e4m3_decode(scales[k / 16]) * (double)s_t;
+}
+
+void oracle_dequantize_nvfp4(int64_t rows, int64_t K, const uint8_t* codes, const uint8_t* scales,
+                             float s_t, double* out) {
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t k = 0; k < K; ++k)
+            out[r * K + k] = nvfp4_value(codes + r * (K / 2), scales + r * (K / 16), k, s_t);
+}
+
+/*
+ * One W4A4 expert on one quantised row (all NVFP4, rows of the weight banks
+ * are [out][in]):
+ *   z_f  = sum_h deq(W_up)[f,h] deq(x)[h]
+ *   a_f  = fl32(max(z_f, 0)^2)
+ *   H    = the row a quantised to NVFP4 in blocks of 16 features with the
+ *          static tensor scale s_h
+ *   y_j  = sum_f deq(W_down)[j,f] deq(H)[f]
+ */
+void oracle_expert_nvfp4(int64_t H, int64_t F, const uint8_t* cu, const uint8_t* su, float tu,
+                         const uint8_t* cd, const uint8_t* sd, float td, const uint8_t* cx,
+                         const uint8_t* sx, float tx, float th, double* y) {
+    float* a = (float*)malloc((size_t)F * sizeof(float));
+    double* ad = (double*)malloc((size_t)F * sizeof(double));
+    double* xd = (double*)malloc((size_t)H * sizeof(double));
+    for (int64_t h = 0; h < H; ++h) xd[h] = nvfp4_value(cx, sx, h, tx);
+    for (int64_t f = 0; f < F; ++f) {
+        double z = 0.0;
+        for (int64_t h = 0; h < H; ++h)
+            z += nvfp4_value(cu + f * (H / 2), su + f * (H / 16), h, tu) * xd[h];
+        a[f] = (float)(z > 0.0 ? z * z : 0.0);
+    }
+    for (int64_t b = 0; b < F / 16; ++b) {
+        uint8_t q[16];
+        uint8_t sc = nvfp4_block(a + b * 16, 16, th, q);
+        for (int i = 0; i < 16; ++i)
+            ad[b * 16 + i] = (double)oracle_e2m1_decode(q[i]) * (double)oracle_e4m3_decode(sc) * (double)th;
+    }
+    for (int64_t j = 0; j < H; ++j) {
+        double s = 0.0;
+        for (int64_t f = 0; f < F; ++f) s += nvfp4_value(cd + j * (F / 2), sd + j * (F / 16), f, td) * ad[f];
+        y[j] = s;
+    }
+    free(a);
+    free(ad);
+    free(xd);
+}
+
+/* Rows of the permuted layout: row r uses expert ex[r] at slot[ex[r]] of the given banks. */
+int oracle_expert_rows_nvfp4(int64_t R, int64_t H, int64_t F, const uint8_t* cxrow, const uint8_t* sxrow,
+                             const int32_t* ex, const uint8_t* cup, const uint8_t* sup, const float* tup,
+                             const uint8_t* cdown, const uint8_t* sdown, const float* tdown,
+                             const int32_t* slot, float tx, float th, double* y) {
+    for (int64_t r = 0; r < R; ++r)
+        if (slot[ex[r]] < 0) return -1;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < R; ++r) {
+        int64_t s = slot[ex[r]];
+        oracle_expert_nvfp4(H, F, cup + s * F * (H / 2), sup + s * F * (H / 16), tup[s], cdown + s * H * (F / 2),
+                            sdown + s * H * (F / 16), tdown[s], cxrow + r * (H / 2), sxrow + r * (H / 16), tx, th,
+                            y + r * H);
+    }
+    return 0;
+}
+
+void oracle_e2m1_encode_n(int64_t n, const float* v, uint8_t* q) {
+    for (int64_t i = 0; i < n; ++i) q[i] = oracle_e2m1_encode(v[i]);
+}
+
+void oracle_e2m1_decode_n(int64_t n, const uint8_t* q, float* v) {
+    for (int64_t i = 0; i < n; ++i) v[i] = oracle_e2m1_decode(q[i]);
+}
+
 /*
  * RMS normalisation of the residual stream before each layer of the chained
  * stack.  [A] "Q4_K, Q3_K and Q2_K expert profiles" names a normalisation
