@@ -44,7 +44,7 @@
 extern "C" {
 #endif
 
-#define MOE_ABI_VERSION 1
+#define MOE_ABI_VERSION 2
 
 typedef enum {
     MOE_OK = 0,
@@ -59,11 +59,12 @@ typedef enum {
 
 typedef enum {
     MOE_BF16 = 0,          /* expert banks and expert activations in bf16 */
-    MOE_FP8_E4M3 = 1       /* W8A8: expert banks and expert activations in E4M3 codes */
+    MOE_FP8_E4M3 = 1,      /* W8A8: expert banks and expert activations in E4M3 codes */
+    MOE_NVFP4 = 2          /* W4A4: expert banks and expert activations in NVFP4 (see below) */
 } moe_dtype;
 
 /* Problem size.  Limits: 0 <= T, T*K < 2^31; 1 <= E <= 256; 1 <= K <= min(E, 16);
- * 16 <= H <= 65536 and 16 <= F <= 65536, both multiples of 16. */
+ * 16 <= H <= 65536 and 16 <= F <= 65536, both multiples of 16 (of 32 for MOE_NVFP4). */
 typedef struct {
     int64_t T;             /* tokens */
     int32_t H;             /* hidden width (router and up-projection input, down output) */
@@ -73,14 +74,31 @@ typedef struct {
     int32_t expert_dtype;  /* moe_dtype */
 } moe_dims;
 
-/* Scalar scales of the W8A8 experts (bloomery page, section 2: "scalar-scale
- * E4M3 W8A8").  Real value = code * scale.  Ignored for MOE_BF16. */
+/* Scales of the quantised experts.  Ignored for MOE_BF16.
+ *
+ * MOE_FP8_E4M3 (bloomery page, section 2: "scalar-scale E4M3 W8A8"): real
+ * value = code * scale; the two block-scale pointers are unused.
+ *
+ * MOE_NVFP4 (bloomery page, section 2: the NVFP4 release runs the experts
+ * W4A4; the format is NVIDIA's NVFP4): E2M1 codes packed two per byte
+ * (element 2i in the low nibble), one E4M3 scale per 16 consecutive elements
+ * along the contraction dimension, one fp32 scale per tensor; real value =
+ * e2m1(code) * e4m3(block scale) * tensor scale.  Block scales are stored
+ * [rows][KSP] bytes with KSP = K/16 rounded up to a multiple of 16 (padding
+ * zero; moe_quantize_nvfp4 writes this layout).  Weight banks: w_up codes
+ * [E][F][H/2], w_up_block [E][F][KSP(H)]; w_down codes [E][H][F/2],
+ * w_down_block [E][H][KSP(F)].  x and the ReLU^2 tensor are quantised inside
+ * the layer with block scales taken at run time and the static tensor scales
+ * x_scale and h_scale. */
 typedef struct {
-    const float* w_up_scale;    /* [E] device: one scale per expert up tensor */
-    const float* w_down_scale;  /* [E] device: one scale per expert down tensor */
-    float x_scale;              /* static scale of the expert input activations */
-    float h_scale;              /* static scale of the ReLU^2 activations */
-} moe_fp8_scales;
+    const float* w_up_scale;    /* [E] device: one (tensor) scale per expert up tensor */
+    const float* w_down_scale;  /* [E] device: one (tensor) scale per expert down tensor */
+    float x_scale;              /* static (tensor) scale of the expert input activations */
+    float h_scale;              /* static (tensor) scale of the ReLU^2 activations */
+    const uint8_t* w_up_block;  /* MOE_NVFP4: [E][F][KSP(H)] E4M3 block scales */
+    const uint8_t* w_down_block;/* MOE_NVFP4: [E][H][KSP(F)] E4M3 block scales */
+} moe_quant_scales;
+typedef moe_quant_scales moe_fp8_scales;
 
 /* Human-readable name of a status.  Never NULL. */
 const char* moe_status_string(moe_status s);
@@ -118,9 +136,10 @@ moe_status moe_permute(const moe_dims* d, const int32_t* topk_idx, int32_t* coun
 /* Grouped expert FFN over the permuted rows:
  *   y_perm[r] = W_down[e] * relu(W_up[e] * x[perm_src[r] / K])^2,  e = expert of row r
  *   x [T][H] bf16; offsets [E+1] and perm_src [T*K] as from moe_permute;
- *   w_up [E][F][H], w_down [E][H][F] (bf16, or E4M3 codes with `scales`);
+ *   w_up [E][F][H], w_down [E][H][F] (bf16, or E4M3 codes with `scales`, or
+ *   NVFP4 codes [E][F][H/2], [E][H][F/2] with `scales`);
  *   y_perm [T*K][H] bf16 out.
- * scales must be non-NULL for MOE_FP8_E4M3.  Cited: bloomery page s.2 and
+ * scales must be non-NULL for MOE_FP8_E4M3 and MOE_NVFP4.  Cited: bloomery page s.2 and
  * s.3 (ungated ReLU^2 experts, up/down parts). */
 moe_status moe_expert_ffn(const moe_dims* d, const void* x, const int32_t* offsets,
                           const int32_t* perm_src, const void* w_up, const void* w_down,
@@ -159,6 +178,25 @@ moe_status moe_quantize_fp8(int64_t n_tensors, int64_t tensor_elems, const void*
  * E4M3 W8A8"). */
 moe_status moe_quantize_act_fp8(int64_t rows, int32_t H, float x_scale, const void* x, uint8_t* codes,
                                 void* stream);
+
+/* NVFP4 quantisation of n_tensors bf16 tensors [rows][K] (an expert bank):
+ * tensor scale t[i] = amax|W_i| / 2688 (1 for an all-zero tensor), per block
+ * of 16 along K: S = e4m3(fl32(fl32(amax_b / 6) / t[i])), codes
+ * e2m1(fl32(W / fl32(S * t[i]))) nearest-even, saturating at 6.
+ *   src [n_tensors][rows][K] bf16; codes [n_tensors][rows][K/2];
+ *   block [n_tensors][rows][KSP(K)] (padding written as zero); tscale [n_tensors] fp32.
+ * K a multiple of 32.  Cited: bloomery page s.2 (NVFP4, W4A4 experts). */
+moe_status moe_quantize_nvfp4(int64_t n_tensors, int64_t rows, int32_t K, const void* src, uint8_t* codes,
+                              uint8_t* block, float* tscale, void* stream);
+
+/* Activation quantisation to NVFP4 with a static tensor scale (the X side
+ * of W4A4): per block of 16 along H, S = e4m3(fl32(fl32(amax_b / 6) /
+ * x_scale)), codes e2m1(fl32(x / fl32(S * x_scale))).  This is the step
+ * moe_forward and moe_expert_ffn apply to the permuted rows, here on rows
+ * in order.  x [rows][H] bf16; codes [rows][H/2]; block [rows][KSP(H)].
+ * H a multiple of 32.  Cited: bloomery page s.2 (NVFP4, W4A4 experts). */
+moe_status moe_quantize_act_nvfp4(int64_t rows, int32_t H, float x_scale, const void* x, uint8_t* codes,
+                                  uint8_t* block, void* stream);
 
 /* RMS normalisation with unit gain of the residual stream between chained
  * layers: u = bf16(x / sqrt(mean(x^2) + eps)), the mean of squares taken

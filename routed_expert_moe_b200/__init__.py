@@ -15,7 +15,7 @@ from pathlib import Path
 _LIB_PATH = Path(__file__).resolve().parent / "_lib" / "libmoe_b200.so"
 
 MOE_OK, MOE_EINVAL, MOE_EUNSUPPORTED, MOE_ECUDA, MOE_ETIMEOUT, MOE_EWORKSPACE, MOE_ERANGE, MOE_EINDEX = range(8)
-MOE_BF16, MOE_FP8_E4M3 = 0, 1
+MOE_BF16, MOE_FP8_E4M3, MOE_NVFP4 = 0, 1, 2
 
 if not _LIB_PATH.exists():
     raise ImportError(
@@ -31,8 +31,10 @@ class MoeDims(ctypes.Structure):
 
 
 class MoeFp8Scales(ctypes.Structure):
+    """moe_quant_scales: tensor scales (both formats) and the NVFP4 block-scale banks."""
     _fields_ = [("w_up_scale", ctypes.c_void_p), ("w_down_scale", ctypes.c_void_p),
-                ("x_scale", ctypes.c_float), ("h_scale", ctypes.c_float)]
+                ("x_scale", ctypes.c_float), ("h_scale", ctypes.c_float),
+                ("w_up_block", ctypes.c_void_p), ("w_down_block", ctypes.c_void_p)]
 
 
 _P = ctypes.c_void_p
@@ -51,8 +53,10 @@ _SIG = {
     "moe_forward": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, ctypes.POINTER(MoeFp8Scales), _P, _P, _P,
                                    _P, _P, _S, _P]),
     "moe_quantize_fp8": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int64, _P, _P, _P, _P]),
+    "moe_quantize_nvfp4": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, _P, _P, _P, _P, _P]),
     "moe_rmsnorm": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int32, ctypes.c_float, _P, _P, _P]),
     "moe_quantize_act_fp8": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int32, ctypes.c_float, _P, _P, _P]),
+    "moe_quantize_act_nvfp4": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int32, ctypes.c_float, _P, _P, _P, _P]),
     "moe_check_device_error": (ctypes.c_int, [_P]),
     "moe_set_stage_events": (ctypes.c_int, [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32]),
     "moe_debug_set": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int64]),
@@ -61,6 +65,10 @@ for _name, (_res, _args) in _SIG.items():
     _f = getattr(_lib, _name)
     _f.restype = _res
     _f.argtypes = _args
+
+_ABI = 2   # the struct layouts above
+if _lib.moe_abi_version() != _ABI:
+    raise ImportError(f"libmoe_b200 ABI {_lib.moe_abi_version()} does not match this binding ({_ABI}); rebuild")
 
 # every symbol include/moe.h declares (checked by the ABI test)
 EXPORTS = tuple(_SIG)
@@ -98,8 +106,9 @@ def _stream(stream):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-def dims(T, H, E, K, F, fp8=False) -> MoeDims:
-    return MoeDims(int(T), int(H), int(E), int(K), int(F), MOE_FP8_E4M3 if fp8 else MOE_BF16)
+def dims(T, H, E, K, F, fp8=False, nvfp4=False) -> MoeDims:
+    dt = MOE_NVFP4 if nvfp4 else (MOE_FP8_E4M3 if fp8 else MOE_BF16)
+    return MoeDims(int(T), int(H), int(E), int(K), int(F), dt)
 
 
 def workspace_size(d: MoeDims) -> int:
@@ -114,7 +123,26 @@ def alloc_workspace(d: MoeDims, device=None):
 
 
 def fp8_scales(w_up_scale, w_down_scale, x_scale: float, h_scale: float) -> MoeFp8Scales:
-    return MoeFp8Scales(w_up_scale.data_ptr(), w_down_scale.data_ptr(), float(x_scale), float(h_scale))
+    return MoeFp8Scales(w_up_scale.data_ptr(), w_down_scale.data_ptr(), float(x_scale), float(h_scale), None, None)
+
+
+def nvfp4_scales(w_up_tscale, w_down_tscale, x_scale: float, h_scale: float, w_up_block, w_down_block) -> MoeFp8Scales:
+    """Tensor scales [E] (fp32), static activation tensor scales, block-scale banks (uint8)."""
+    return MoeFp8Scales(w_up_tscale.data_ptr(), w_down_tscale.data_ptr(), float(x_scale), float(h_scale),
+                        w_up_block.data_ptr(), w_down_block.data_ptr())
+
+
+def nvfp4_scale_row(K: int) -> int:
+    """Bytes of one block-scale row: K/16 rounded up to a multiple of 16."""
+    return (K // 16 + 15) // 16 * 16
+
+
+def quantize_nvfp4(src, codes, block, tscale, stream=None):
+    """NVFP4 quantisation of a bank src [n, rows, K] (bf16): codes [n, rows, K/2], block scales
+    [n, rows, nvfp4_scale_row(K)], tensor scales [n]."""
+    n, rows, K = src.shape
+    _check(_lib.moe_quantize_nvfp4(n, rows, K, _ptr(src), _ptr(codes), _ptr(block), _ptr(tscale), _stream(stream)),
+           "moe_quantize_nvfp4")
 
 
 def route(d, x, w_router, bias, topk_idx, topk_w, ws, stream=None):
@@ -167,6 +195,13 @@ def quantize_act_fp8(x, codes, x_scale, stream=None):
     rows, H = x.shape
     _check(_lib.moe_quantize_act_fp8(rows, H, float(x_scale), _ptr(x), _ptr(codes), _stream(stream)),
            "moe_quantize_act_fp8")
+
+
+def quantize_act_nvfp4(x, codes, block, x_scale, stream=None):
+    """NVFP4 codes [rows, H/2] and block scales [rows, nvfp4_scale_row(H)] of x [rows, H] (bf16)."""
+    rows, H = x.shape
+    _check(_lib.moe_quantize_act_nvfp4(rows, H, float(x_scale), _ptr(x), _ptr(codes), _ptr(block), _stream(stream)),
+           "moe_quantize_act_nvfp4")
 
 
 def rmsnorm(x, u, eps=1e-5, stream=None):

@@ -50,6 +50,17 @@ cudaError_t launch_grouped_gemm_pair(bool fp8, bool up, const void* W, int E, in
                                      int64_t rows, const int4* sched, const int* n_sched, int bn, int max_sched,
                                      void* out, const float* w_scale, float in_scale, float out_scale,
                                      int num_sms, const DevCtx& ctx, cudaStream_t stream);
+cudaError_t launch_grouped_gemm_fp4(bool up, const uint8_t* w_codes, const uint8_t* w_scales, const float* w_tscale,
+                                    int E, int Nout, int Kdim, const uint8_t* a_codes, const uint8_t* a_scales,
+                                    float in_tscale, float out_tscale, int64_t rows, const int4* sched,
+                                    const int* n_sched, int bn, int max_sched, void* out, uint8_t* out_scale,
+                                    int num_sms, int debug_withhold, const DevCtx& ctx, cudaStream_t stream);
+cudaError_t launch_quantize_nvfp4(int64_t n_tensors, int64_t rows, int K, const uint16_t* src, uint8_t* codes,
+                                  uint8_t* bscale, float* tscale, int num_sms, cudaStream_t stream);
+cudaError_t launch_gather_nvfp4(const uint16_t* x, const int32_t* perm_src, int64_t rows, int K, int64_t T, int H,
+                                float s_t, uint8_t* codes, uint8_t* bscale, int num_sms, const DevCtx& ctx,
+                                cudaStream_t stream);
+size_t nvfp4_scale_row_bytes(int K);
 cudaError_t launch_combine(const uint16_t* yp, const int32_t* inv_row, const float* w, const uint16_t* residual,
                            uint16_t* out, int64_t T, int K, int H, int num_sms, const DevCtx& ctx,
                            cudaStream_t stream);
@@ -124,7 +135,9 @@ moe_status check_dims(const moe_dims* d) {
     if (d->H < 16 || d->H > 65536 || d->H % 16 != 0) return MOE_EINVAL;
     if (d->F < 16 || d->F > 65536 || d->F % 16 != 0) return MOE_EINVAL;
     if (d->T * (int64_t)d->K >= (int64_t)1 << 31) return MOE_EINVAL;
-    if (d->expert_dtype != MOE_BF16 && d->expert_dtype != MOE_FP8_E4M3) return MOE_EINVAL;
+    if (d->expert_dtype != MOE_BF16 && d->expert_dtype != MOE_FP8_E4M3 && d->expert_dtype != MOE_NVFP4)
+        return MOE_EINVAL;
+    if (d->expert_dtype == MOE_NVFP4 && (d->H % 32 != 0 || d->F % 32 != 0)) return MOE_EINVAL;
     return MOE_OK;
 }
 
@@ -155,8 +168,10 @@ struct FfnWs {
     int4* sched;
     int* n_sched;
     int* perm_scratch;
-    void* xp;
-    void* hb;
+    void* xp;            // permuted rows: bf16, E4M3 codes, or NVFP4 codes [rows][H/2]
+    void* hb;            // ReLU^2 rows: bf16, E4M3 codes, or NVFP4 codes [rows][F/2]
+    uint8_t* xp_block;   // NVFP4: block scales [rows][KSP(H)]
+    uint8_t* hb_block;   // NVFP4: block scales [rows][KSP(F)]
 };
 struct ForwardWs {
     int32_t* idx;
@@ -179,10 +194,18 @@ RouteWs carve_route(Carve& c, void* base, const moe_dims* d, const RouterPlan& r
 FfnWs carve_ffn(Carve& c, void* base, const moe_dims* d, const GemmPlan& gp) {
     FfnWs f;
     const size_t rows = (size_t)d->T * d->K;
-    const size_t es = d->expert_dtype == MOE_FP8_E4M3 ? 1 : 2;
     f.sched = c.take<int4>(base, (size_t)gp.max_sched);
     f.n_sched = c.take<int>(base, 1);
     f.perm_scratch = c.take<int>(base, permute_scratch_ints(d->T * d->K, d->E));
+    f.xp_block = f.hb_block = nullptr;
+    if (d->expert_dtype == MOE_NVFP4) {
+        f.xp = c.take<uint8_t>(base, rows * d->H / 2);
+        f.hb = c.take<uint8_t>(base, rows * d->F / 2);
+        f.xp_block = c.take<uint8_t>(base, rows * nvfp4_scale_row_bytes(d->H));
+        f.hb_block = c.take<uint8_t>(base, rows * nvfp4_scale_row_bytes(d->F));
+        return f;
+    }
+    const size_t es = d->expert_dtype == MOE_FP8_E4M3 ? 1 : 2;
     f.xp = c.take<uint8_t>(base, rows * d->H * es);
     f.hb = c.take<uint8_t>(base, rows * d->F * es);
     return f;
@@ -228,6 +251,26 @@ moe_status run_ffn(const moe_dims* d, const DeviceInfo* dev, const DevCtx& ctx, 
                    const moe_fp8_scales* sc, FfnWs& fw, void* y_perm, cudaStream_t st, bool marks = false) {
     const bool fp8 = d->expert_dtype == MOE_FP8_E4M3;
     const int64_t rows = d->T * d->K;
+    if (d->expert_dtype == MOE_NVFP4) {
+        const int withhold4 = g_debug_withhold.load();
+        if (marks) stage_mark(3, st);
+        cudaError_t e4 = launch_gather_nvfp4(static_cast<const uint16_t*>(x), perm_src, rows, d->K, d->T, d->H,
+                                             sc->x_scale, static_cast<uint8_t*>(fw.xp), fw.xp_block, dev->num_sms,
+                                             ctx, st);
+        if (e4 != cudaSuccess) return cuda_status(e4);
+        if (marks) stage_mark(4, st);
+        e4 = launch_grouped_gemm_fp4(true, static_cast<const uint8_t*>(w_up), sc->w_up_block, sc->w_up_scale, d->E,
+                                     d->F, d->H, static_cast<const uint8_t*>(fw.xp), fw.xp_block, sc->x_scale,
+                                     sc->h_scale, rows, fw.sched, fw.n_sched, gp.bn, gp.max_sched, fw.hb,
+                                     fw.hb_block, dev->num_sms, withhold4, ctx, st);
+        if (e4 != cudaSuccess) return cuda_status(e4);
+        if (marks) stage_mark(5, st);
+        e4 = launch_grouped_gemm_fp4(false, static_cast<const uint8_t*>(w_down), sc->w_down_block, sc->w_down_scale,
+                                     d->E, d->H, d->F, static_cast<const uint8_t*>(fw.hb), fw.hb_block, sc->h_scale,
+                                     1.0f, rows, fw.sched, fw.n_sched, gp.bn, gp.max_sched, y_perm, nullptr,
+                                     dev->num_sms, 0, ctx, st);
+        return cuda_status(e4);
+    }
     if (marks) stage_mark(3, st);
     // permuted copy of x (or of its E4M3 codes), read by the up projection in contiguous row blocks
     cudaError_t e = launch_gather(static_cast<const uint16_t*>(x), perm_src, rows, d->K, d->T, d->H, fw.xp, fp8,
@@ -259,9 +302,13 @@ moe_status run_ffn(const moe_dims* d, const DeviceInfo* dev, const DevCtx& ctx, 
 }
 
 moe_status check_fp8_scales(const moe_dims* d, const moe_fp8_scales* sc) {
-    if (d->expert_dtype != MOE_FP8_E4M3) return MOE_OK;
+    if (d->expert_dtype == MOE_BF16) return MOE_OK;
     if (!sc || !sc->w_up_scale || !sc->w_down_scale) return MOE_EINVAL;
     if (!(sc->x_scale > 0.0f) || !(sc->h_scale > 0.0f)) return MOE_EINVAL;
+    if (!(sc->x_scale < 3.4e38f) || !(sc->h_scale < 3.4e38f)) return MOE_EINVAL;
+    if (d->expert_dtype == MOE_NVFP4 && (!sc->w_up_block || !sc->w_down_block || !aligned(sc->w_up_block, 16) ||
+                                         !aligned(sc->w_down_block, 16)))
+        return MOE_EINVAL;
     return MOE_OK;
 }
 
@@ -439,6 +486,33 @@ moe_status moe_quantize_fp8(int64_t n_tensors, int64_t tensor_elems, const void*
     if (s != MOE_OK) return s;
     return cuda_status(launch_quantize(n_tensors, tensor_elems, static_cast<const uint16_t*>(src), codes, scales,
                                        dev->num_sms, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_quantize_nvfp4(int64_t n_tensors, int64_t rows, int32_t K, const void* src, uint8_t* codes,
+                              uint8_t* block, float* tscale, void* stream) {
+    if (n_tensors < 0 || rows < 0 || K < 32 || K > 65536 || K % 32 != 0) return MOE_EINVAL;
+    if (n_tensors == 0 || rows == 0) return MOE_OK;
+    if (!src || !codes || !block || !tscale || !aligned(src, 16) || !aligned(codes, 8) || !aligned(tscale, 4))
+        return MOE_EINVAL;
+    DeviceInfo* dev = nullptr;
+    moe_status s = device_setup(&dev);
+    if (s != MOE_OK) return s;
+    return cuda_status(launch_quantize_nvfp4(n_tensors, rows, K, static_cast<const uint16_t*>(src), codes, block,
+                                             tscale, dev->num_sms, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_quantize_act_nvfp4(int64_t rows, int32_t H, float x_scale, const void* x, uint8_t* codes,
+                                  uint8_t* block, void* stream) {
+    if (rows < 0 || H < 32 || H > 65536 || H % 32 != 0) return MOE_EINVAL;
+    if (!(x_scale > 0.0f) || !(x_scale < 3.4e38f)) return MOE_EINVAL;
+    if (rows == 0) return MOE_OK;
+    if (!x || !codes || !block || !aligned(x, 16) || !aligned(codes, 8)) return MOE_EINVAL;
+    DeviceInfo* dev = nullptr;
+    moe_status s = device_setup(&dev);
+    if (s != MOE_OK) return s;
+    return cuda_status(launch_gather_nvfp4(static_cast<const uint16_t*>(x), nullptr, rows, 1, rows, H, x_scale,
+                                           codes, block, dev->num_sms, make_ctx(dev),
+                                           static_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_quantize_act_fp8(int64_t rows, int32_t H, float x_scale, const void* x, uint8_t* codes,

@@ -42,7 +42,7 @@ def test_library_exports_every_declared_symbol(moe):
 
 
 def test_status_strings_and_version(moe):
-    assert moe.abi_version() == 1
+    assert moe.abi_version() == 2   # moe_quant_scales carries the NVFP4 block-scale banks
     for s in range(8):
         assert moe.status_string(s).startswith("MOE_")
     assert "unknown" in moe.status_string(99)
