@@ -35,7 +35,8 @@ METRIC = "MoE-layer tokens/s on 1 B200; % of HBM roofline (decode), % TC peak (p
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-WORKLOADS = {"tiny": 0, "decode": 1, "prefill": 2, "skewed": 3, "chain": 4}
+WORKLOADS = {"tiny": 0, "decode": 1, "prefill": 2, "skewed": 3, "chain": 4, "decode_nvfp4": 5,
+             "prefill_nvfp4": 6}
 
 
 def load_peaks():
@@ -167,7 +168,23 @@ class Layer:
             x = torch.empty(wl.T, wl.H, dtype=bf, device=device)
             synth.normal_bf16_device(synth.key(wl.seed, synth.T_X, i), x.numel(), W.SIGMA_X, x.data_ptr(), stream)
             self.xs.append(x)
-        self.dims = moe.dims(wl.T, wl.H, wl.E, wl.K, wl.F)
+        self.scales = None
+        if wl.nvfp4:
+            # NVFP4 banks quantised on the device from the bf16 masters; static activation scales
+            # from the oracle's calibration (tests/golden/nvfp4_scales.json)
+            banks = []
+            for src in (self.wu, self.wd):
+                n, rows, Kd = src.shape
+                codes = torch.empty(n, rows, Kd // 2, dtype=torch.uint8, device=device)
+                block = torch.empty(n, rows, moe.nvfp4_scale_row(Kd), dtype=torch.uint8, device=device)
+                tsc = torch.empty(n, dtype=torch.float32, device=device)
+                moe.quantize_nvfp4(src, codes, block, tsc)
+                banks.append((codes, block, tsc))
+            torch.cuda.synchronize(device)
+            (self.wu, self.bu, self.tu), (self.wd, self.bd, self.td) = banks
+            sx, sh = W.nvfp4_scales(wl)
+            self.scales = moe.nvfp4_scales(self.tu, self.td, float(sx), float(sh), self.bu, self.bd)
+        self.dims = moe.dims(wl.T, wl.H, wl.E, wl.K, wl.F, nvfp4=wl.nvfp4)
         self.ws = moe.alloc_workspace(self.dims, device)
         self.out = torch.empty(wl.T, wl.H, dtype=bf, device=device)
         self.idx = torch.empty(wl.T, wl.K, dtype=torch.int32, device=device)
@@ -176,7 +193,8 @@ class Layer:
 
     def step(self, i, x=None, out=None):
         self.moe.forward(self.dims, self.xs[i % len(self.xs)] if x is None else x, self.wr, self.bias, self.wu,
-                         self.wd, self.out if out is None else out, self.ws, topk_idx=self.idx, topk_w=self.w)
+                         self.wd, self.out if out is None else out, self.ws, scales=self.scales, topk_idx=self.idx,
+                         topk_w=self.w)
 
     def touched_experts(self, i):
         import torch
@@ -334,8 +352,14 @@ def roofline_entry(wl, stages, touched, peaks, peak_kind, workload):
     kernel = "up_gemm" if up_ms >= down_ms else "down_gemm"
     ms = max(up_ms, down_ms)
     flops = 2.0 * rows * F * H
+    if wl.nvfp4:
+        # packed codes (half a byte per value) + one E4M3 block scale per 16 values (rows padded to 16 bytes)
+        ksp = lambda k: (k // 16 + 15) // 16 * 16
+        w_b = touched * F * (H / 2 + ksp(H)) if kernel == "up_gemm" else touched * H * (F / 2 + ksp(F))
+        algo = (w_b + rows * (H / 2 + ksp(H)) + rows * (F / 2 + ksp(F)) if kernel == "up_gemm"
+                else w_b + rows * (F / 2 + ksp(F)) + rows * H * 2)
     # weights of the touched experts + activations in (es bytes) + activations out
-    if kernel == "up_gemm":
+    elif kernel == "up_gemm":
         algo = touched * F * H * es + rows * H * es + rows * F * es
     else:
         algo = touched * F * H * es + rows * F * es + rows * H * 2
@@ -347,7 +371,7 @@ def roofline_entry(wl, stages, touched, peaks, peak_kind, workload):
     common = {"kernel": kernel, "ms_per_launch": ms, "algorithmic_bytes_per_launch": algo,
               "algorithmic_flops_per_launch": flops, "traffic": traffic_from_profile(kernel, workload),
               "hbm_gbs": gbs, "hbm_frac": gbs / hbm_peak, "tensor_tflops": tflops, "tensor_frac": tflops / tc_peak}
-    if workload in ("prefill", "chain"):
+    if workload in ("prefill", "chain", "prefill_nvfp4"):
         src = f"{peak_kind} bf16 sustained" + (" x 2 (fp8/bf16 nominal ratio)" if wl.fp8 else "")
         return dict(bound="tensor", achieved=tflops, peak=tc_peak, unit="TFLOP/s", frac=tflops / tc_peak,
                     peak_source=src, **common)
@@ -379,6 +403,8 @@ def cpu_baseline(wl, n_tokens, seed_batch=0, target_s=CPU_SAMPLE_SECONDS):
     (the same token sample repeated until about CPU_SAMPLE_SECONDS of work)."""
     if wl.fp8:
         return cpu_baseline_fp8(wl, n_tokens, seed_batch, target_s=target_s)
+    if wl.nvfp4:
+        return cpu_baseline_nvfp4(wl, n_tokens, seed_batch, target_s=target_s)
     import oracle
     from synth import workloads as W
     x = W.host_x(wl, seed_batch)[:n_tokens]
@@ -401,6 +427,37 @@ def cpu_baseline(wl, n_tokens, seed_batch=0, target_s=CPU_SAMPLE_SECONDS):
     return {"value": reps * n_tokens / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"{n_tokens} of the {wl.T} tokens of batch {seed_batch} ({wl.name}), full layer "
                       f"(router, top-{wl.K}, {len(used)} experts' up/ReLU^2/down in fp64, combine), "
+                      f"{reps} times; {dt:.2f} s"}
+
+
+def cpu_baseline_nvfp4(wl, n_tokens, seed_batch=0, target_s=CPU_SAMPLE_SECONDS):
+    """The oracle's W4A4 layer (router, NVFP4 experts, combine) on a token sample."""
+    import numpy as np
+    import oracle
+    from synth import workloads as W
+    x = W.host_x(wl, seed_batch)[:n_tokens]
+    wr = W.host_router(wl)
+    _, idx, _ = oracle.route(x, wr, W.host_bias(wl), wl.K)
+    used = sorted(set(idx.reshape(-1).tolist()))
+    slot = -np.ones(wl.E, dtype=np.int32)
+    slot[used] = np.arange(len(used))
+    key = (wl.name, 0, tuple(used), "nvfp4")
+    if key not in _BANKS:   # weight preparation: untimed
+        _BANKS.clear()
+        _BANKS[key] = (oracle.quantize_bank_nvfp4(W.host_w_up(wl, experts=used)),
+                       oracle.quantize_bank_nvfp4(W.host_w_down(wl, experts=used)))
+    bank_up, bank_down = _BANKS[key]
+    sx, sh = W.nvfp4_scales(wl)
+    dt, reps = 0.0, 0
+    while (reps == 0 or dt < target_s) and reps < 1000:
+        t0 = time.perf_counter()
+        oracle.moe_layer_nvfp4(x, wr, W.host_bias(wl), bank_up, bank_down, sx, sh, wl.K, slot=slot)
+        dt += time.perf_counter() - t0
+        reps += 1
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return {"value": reps * n_tokens / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{n_tokens} of the {wl.T} tokens of batch {seed_batch} ({wl.name}), full layer "
+                      f"(router, top-{wl.K}, {len(used)} W4A4 experts in fp64 on dequantised codes, combine), "
                       f"{reps} times; {dt:.2f} s"}
 
 
@@ -496,12 +553,14 @@ def run_native(args):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,
-            "dtype": "fp8_e4m3 (W8A8) experts, bf16 router" if wl.fp8 else "bf16",
+            "dtype": ("fp8_e4m3 (W8A8) experts, bf16 router" if wl.fp8 else
+                      "nvfp4 (W4A4: e2m1 codes, e4m3 block scales; fp16 tensor-core products) experts, bf16 router"
+                      if wl.nvfp4 else "bf16"),
             "data": "synthetic: seeded N(0,1) activations, N(0,0.02) router/expert weights (bf16)",
             "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "E": wl.E, "K": wl.K, "F": wl.F,
                        "layers": wl.layers, "touched_experts": touched,
                        "l2": "inputs larger than L2: the touched experts' weights "
-                             f"({touched * wl.F * wl.H * (2 if wl.fp8 else 4) * wl.layers / 1e9:.2f} GB) "
+                             f"({touched * wl.F * wl.H * (1.125 if wl.nvfp4 else 2 if wl.fp8 else 4) * wl.layers / 1e9:.2f} GB) "
                              "stream from HBM every step; token batches rotate; no flush",
                        "parallelism": f"dp{ws} (independent token batches per GPU, weights replicated)",
                        "grouped_gemm": "cta_pair" if args.gemm == "pair" else "single_cta",
@@ -516,7 +575,7 @@ def run_native(args):
         if secondary:
             line["secondary"] = secondary
         if ws == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(wl, 4 if wl.fp8 else min(wl.T, 64))
+            line["cpu_baseline"] = cpu_baseline(wl, 4 if wl.fp8 else 8 if wl.nvfp4 else min(wl.T, 64))
         print(json.dumps(line), flush=True)
     if ws > 1:
         dist.destroy_process_group()

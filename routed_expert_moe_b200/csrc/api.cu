@@ -183,6 +183,21 @@ struct ForwardWs {
     void* y_perm;
 };
 
+// Plan of the expert FFN: the bf16/E4M3 kernel's plan; NVFP4 caps the rows of a
+// schedule entry (32 for batches up to 256 tokens, else 128) so that its fp16 stage
+// buffers (eight, or four) fit in shared memory.
+GemmPlan ffn_plan(const moe_dims* d) {
+    GemmPlan gp = gemm_plan(d->T, d->K, d->E);
+    const int cap = d->T <= 256 ? 32 : 128;
+    if (d->expert_dtype == MOE_NVFP4 && gp.bn > cap) {
+        const int64_t rows = d->T * d->K;
+        const int64_t nonempty = d->E < rows ? d->E : rows;
+        gp.bn = cap;
+        gp.max_sched = (int)(nonempty + (rows + cap - 1) / cap);
+    }
+    return gp;
+}
+
 RouteWs carve_route(Carve& c, void* base, const moe_dims* d, const RouterPlan& rp) {
     RouteWs r;
     r.P = c.take<double>(base, rp.p_bytes / sizeof(double));
@@ -232,7 +247,7 @@ size_t route_ws_bytes(const moe_dims* d, int sms) {
 
 size_t ffn_ws_bytes(const moe_dims* d) {
     Carve c;
-    carve_ffn(c, nullptr, d, gemm_plan(d->T, d->K, d->E));
+    carve_ffn(c, nullptr, d, ffn_plan(d));
     return c.off;
 }
 
@@ -402,7 +417,7 @@ moe_status moe_expert_ffn(const moe_dims* d, const void* x, const int32_t* offse
     if (d->T == 0) return MOE_OK;
     DeviceInfo* dev = nullptr;
     if ((s = device_setup(&dev)) != MOE_OK) return s;
-    const GemmPlan gp = gemm_plan(d->T, d->K, d->E);
+    const GemmPlan gp = ffn_plan(d);
     Carve c;
     FfnWs fw = carve_ffn(c, ws, d, gp);
     if (c.off > ws_bytes) return MOE_EWORKSPACE;
@@ -459,7 +474,7 @@ moe_status moe_forward(const moe_dims* d, const void* x, const void* w_router, c
                                  g_stage_events_on.load() ? mark_stage1 : nullptr);
     if (e != cudaSuccess) return cuda_status(e);
 
-    const GemmPlan gp = gemm_plan(d->T, d->K, d->E);
+    const GemmPlan gp = ffn_plan(d);
     Carve cf;
     FfnWs ffw = carve_ffn(cf, sbase, d, gp);   // reuses the router scratch region
     stage_mark(2, st);

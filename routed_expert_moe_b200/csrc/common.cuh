@@ -87,6 +87,19 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const D
     }
 }
 
+// Warp-wide bounded wait: lane 0 waits and the outcome is broadcast, so every
+// lane of the warp takes the same branch (warp-collective code follows: a
+// __syncwarp, tcgen05.ld).  The __syncwarp orders the other lanes' accesses
+// after lane 0's observation of the completed phase.
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, const DevCtx& ctx,
+                                               volatile int* abort) {
+    int ok = 1;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, ctx, abort) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    __syncwarp();
+    return ok != 0;
+}
+
 // Bounded wait that ignores the abort flag (used while draining after an abort).
 __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, uint64_t timeout_ns) {
     const uint64_t t0 = globaltimer();

@@ -224,7 +224,7 @@ __global__ void __launch_bounds__(GG_THREADS, 1)
         for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
             const int4 sc = g.sched[u / g.m_blocks];
             const int mb = u % g.m_blocks;
-            if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, ctx, abort_flag)) break;
+            if (!mbar_wait_warp(smem_u32(&tfull[acc]), acc_phase, ctx, abort_flag)) break;
             tc_fence_after();
             const int f = mb * GG_BM + q * 32 + lane;
             const bool fvalid = f < g.Nout;

@@ -293,7 +293,7 @@ __global__ void __launch_bounds__(P2_THREADS, 1)
         for (int u = pair; u < n_units; u += n_pairs) {
             const int4 sc = g.sched[u / g.m_pairs];
             const int mp = u % g.m_pairs;
-            if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, ctx, abort_flag)) break;
+            if (!mbar_wait_warp(smem_u32(&tfull[acc]), acc_phase, ctx, abort_flag)) break;
             tc_fence_after();
             const int f = (mp * 2 + (int)rank) * P2_BM + q * 32 + lane;
             const bool fvalid = f < g.Nout;

@@ -288,10 +288,10 @@ __global__ void __launch_bounds__(FG_THREADS, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < NR; ++s) {
             mbar_init(smem_u32(&raw_full[s]), 1);
-            mbar_init(smem_u32(&raw_empty[s]), 128);
+            mbar_init(smem_u32(&raw_empty[s]), 4);    // one arrival per converter warp
         }
         for (int s = 0; s < NF; ++s) {
-            mbar_init(smem_u32(&f16_full[s]), 128);
+            mbar_init(smem_u32(&f16_full[s]), 1);     // the converter warp of that stage
             mbar_init(smem_u32(&f16_empty[s]), 1);
         }
         for (int a = 0; a < 2; ++a) {
@@ -372,51 +372,61 @@ __global__ void __launch_bounds__(FG_THREADS, 1)
         }
     } else if (warp >= 6) {
         // ---------------------------------------------------------------- converters
-        const int i = threadIdx.x - 192;   // 0..127: weight row i, activation rows i and i + 128
-        int rs = 0, fs = 0;
-        uint32_t rph = 0, fph = 0;
+        // Converter warp w dequantises fp16 stage w of every raw stage (K values 64w .. 64w+63 of
+        // the 256): all 128 weight rows and the unit's token rows, four rows per lane at a time,
+        // into its own fp16 buffers w*NF/4 .. (w+1)*NF/4 - 1 in turn.  One producer per buffer,
+        // uses in order: a wait on a buffer's parity can never see a phase two ahead.  The MMA
+        // thread keeps the same count per warp (stage kf of a unit is warp kf % 4's).
+        const int w = warp - 6;
+        int rs = 0;
+        uint32_t rph = 0;
+        uint32_t uses = 0;
         bool ok = true;
         for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
             const int4 sc = g.sched[u / g.m_blocks];
             const int mb = u % g.m_blocks;
             const bool a_full = g.Nout - mb * FG_BM > 64;
             const int nrows = ((sc.z + 15) / 16) * 16;
-            for (int kr = 0; kr < g.k_raw && ok; ++kr) {
-                if (!mbar_wait(smem_u32(&raw_full[rs]), rph, ctx, abort_flag)) {
+            for (int kr = 0; kr < g.k_raw; ++kr) {
+                if (!mbar_wait_warp(smem_u32(&raw_full[rs]), rph, ctx, abort_flag)) {
                     ok = false;
                     break;
                 }
-                const uint8_t* st = raw + (size_t)rs * raw_bytes;
-                const uint8_t* a_c = st;
-                const uint8_t* b_c = st + FG_A_RAW;
-                const uint8_t* a_s = st + FG_A_RAW + b_raw;
-                const uint8_t* b_s = a_s + FG_A_SC;
-                for (int sub = 0; sub < 4; ++sub) {
-                    const int kf = kr * 4 + sub;
-                    if (kf >= g.k_f16) break;
-                    if (!mbar_wait(smem_u32(&f16_empty[fs]), fph ^ 1u, ctx, abort_flag)) {
+                const int kf = kr * 4 + w;
+                if (kf < g.k_f16) {
+                    const int m = NF / 4;   // buffers per converter warp
+                    const int fs = w * m + (int)(uses % (uint32_t)m);
+                    const uint32_t fph = (uses / (uint32_t)m) & 1u;
+                    ++uses;
+                    if (!mbar_wait_warp(smem_u32(&f16_empty[fs]), fph ^ 1u, ctx, abort_flag)) {
                         ok = false;
                         break;
                     }
+                    const uint8_t* st = raw + (size_t)rs * raw_bytes;
+                    const uint8_t* a_c = st;
+                    const uint8_t* b_c = st + FG_A_RAW;
+                    const uint8_t* a_s = st + FG_A_RAW + b_raw;
+                    const uint8_t* b_s = a_s + FG_A_SC;
                     uint8_t* fa = f16 + (size_t)fs * f16_bytes;
                     uint8_t* fbt = fa + FG_A_F16;
-                    const int kb0 = kr * 16 + sub * 4;
-                    if (a_full || i < 64)
-                        convert_row(a_c + i * 128, a_s + i * 16, fa + i * 128, i, sub, kb0, nbk);
-                    else
+                    const int kb0 = kr * 16 + w * 4;
+                    for (int r = lane; r < FG_BM; r += 32) {
+                        if (a_full || r < 64)
+                            convert_row(a_c + r * 128, a_s + r * 16, fa + r * 128, r, w, kb0, nbk);
+                        else
 #pragma unroll
-                        for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(fa + i * 128 + 16 * c) = make_uint4(0, 0, 0, 0);
-                    for (int j = i; j < nrows; j += 128)
-                        convert_row(b_c + j * 128, b_s + j * 16, fbt + j * 128, j, sub, kb0, nbk);
-                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                    mbar_arrive(smem_u32(&f16_full[fs]));
-                    if (++fs == NF) {
-                        fs = 0;
-                        fph ^= 1u;
+                            for (int c = 0; c < 8; ++c)
+                                *reinterpret_cast<uint4*>(fa + r * 128 + 16 * c) = make_uint4(0, 0, 0, 0);
                     }
+                    for (int j = lane; j < nrows; j += 32)
+                        convert_row(b_c + j * 128, b_s + j * 16, fbt + j * 128, j, w, kb0, nbk);
+                    // this lane's fp16 writes become visible to the tensor cores; one arrival per warp
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_u32(&f16_full[fs]));
                 }
-                if (!ok) break;
-                mbar_arrive(smem_u32(&raw_empty[rs]));
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&raw_empty[rs]));
                 if (++rs == NR) {
                     rs = 0;
                     rph ^= 1u;
@@ -426,8 +436,7 @@ __global__ void __launch_bounds__(FG_THREADS, 1)
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA
         if (lane == 0) {
-            int fs = 0;
-            uint32_t fph = 0;
+            uint32_t uses[4] = {0u, 0u, 0u, 0u};   // stages converter warp w has filled so far
             int acc = 0;
             uint32_t acc_phase = 0;
             bool ok = true, issued = false;
@@ -442,6 +451,11 @@ __global__ void __launch_bounds__(FG_THREADS, 1)
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * 256);
                 for (int kf = 0; kf < g.k_f16; ++kf) {
+                    const int m = NF / 4;
+                    const int wq = kf & 3;   // the converter warp of this stage
+                    const int fs = wq * m + (int)(uses[wq] % (uint32_t)m);
+                    const uint32_t fph = (uses[wq] / (uint32_t)m) & 1u;
+                    ++uses[wq];
                     if (!mbar_wait(smem_u32(&f16_full[fs]), fph, ctx, abort_flag)) {
                         ok = false;
                         break;
@@ -455,10 +469,6 @@ __global__ void __launch_bounds__(FG_THREADS, 1)
                                       (kf | kk) != 0 ? 1u : 0u);
                     issued = true;
                     mma_commit(smem_u32(&f16_empty[fs]));
-                    if (++fs == NF) {
-                        fs = 0;
-                        fph ^= 1u;
-                    }
                 }
                 if (!ok) break;
                 mma_commit(smem_u32(&tfull[acc]));
@@ -481,11 +491,12 @@ __global__ void __launch_bounds__(FG_THREADS, 1)
         for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
             const int4 sc = g.sched[u / g.m_blocks];
             const int mb = u % g.m_blocks;
-            if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, ctx, abort_flag)) break;
+            if (!mbar_wait_warp(smem_u32(&tfull[acc]), acc_phase, ctx, abort_flag)) break;
             tc_fence_after();
             const int f = mb * FG_BM + q * 32 + lane;
             const bool fvalid = f < g.Nout;
             const float scale = __fmul_rn(g.w_tscale[sc.x], g.in_tscale);
+            const float r6 = __frcp_rn(6.0f), rts = __frcp_rn(g.out_tscale);   // quotients via nv_div
             const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * 256);
             const int nchunks = (sc.z + 15) / 16;
             for (int c = 0; c < nchunks; ++c) {
@@ -502,7 +513,7 @@ __global__ void __launch_bounds__(FG_THREADS, 1)
 #pragma unroll
                         for (int off = 8; off > 0; off >>= 1)
                             amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-                        const uint32_t scode = e4m3_code(__fdiv_rn(__fdiv_rn(amax, 6.0f), g.out_tscale));
+                        const uint32_t scode = e4m3_code(nv_div(nv_div(amax, 6.0f, r6), g.out_tscale, rts));
                         const float e = __fmul_rn(e4m3_value(scode), g.out_tscale);
                         const float qv = e != 0.0f ? nv_div(a, e, __frcp_rn(e)) : 0.0f;
                         const float qn = __shfl_down_sync(0xffffffffu, qv, 1);   // the odd neighbour
@@ -581,7 +592,8 @@ Fp4Plan fp4_plan(int bn) {
     p.bn = bn;
     const int raw = (FG_A_RAW + bn * 128 + FG_A_SC + bn * 16 + 1023) & ~1023;
     const int f16 = FG_A_F16 + bn * 128;
-    int nf = bn > 64 ? 2 : 3;
+    // fp16 buffers: a multiple of 4 (each converter warp owns NF/4); eight when the tiles are small
+    const int nf = bn <= 32 ? 8 : 4;
     int nr = (220 * 1024 - nf * f16) / raw;
     if (nr > 8) nr = 8;
     if (nr < 2) nr = 2;

@@ -34,6 +34,7 @@ class Workload:
     zipf_bias: bool = False
     layers: int = 1
     fp8: bool = False
+    nvfp4: bool = False
 
     @property
     def assignments(self) -> int:
@@ -46,6 +47,9 @@ WORKLOADS = {
     2: Workload("prefill_T4096", 4096, 2688, 128, 6, 1856, seed=2),
     3: Workload("skewed_zipf_T576", 576, 2688, 128, 6, 1856, seed=3, zipf_bias=True),
     4: Workload("chain23_fp8_T4096", 4096, 2688, 128, 6, 1856, seed=4, layers=23, fp8=True),
+    # the NVFP4 (W4A4) release's experts on the decode and prefill shapes (same seeds and bf16 masters)
+    5: Workload("decode_nvfp4_T64", 64, 2688, 128, 6, 1856, seed=1, nvfp4=True),
+    6: Workload("prefill_nvfp4_T4096", 4096, 2688, 128, 6, 1856, seed=2, nvfp4=True),
 }
 
 
@@ -113,3 +117,17 @@ def chain_scales():
     d = json.loads(p.read_text())
     f32 = lambda h: np.float32(struct.unpack(">f", bytes.fromhex(h))[0])
     return [(f32(l["x_scale_f32"]), f32(l["h_scale_f32"])) for l in d["layers"]]
+
+
+def nvfp4_scales(w: Workload):
+    """Static NVFP4 activation tensor scales (x, H) of an NVFP4 workload, as fp32.
+
+    Written by tests/golden/make_nvfp4_scales.py from a calibration pass of the oracle.
+    """
+    import json
+    import struct
+    from pathlib import Path
+    p = Path(__file__).resolve().parents[1] / "tests" / "golden" / "nvfp4_scales.json"
+    d = json.loads(p.read_text())[w.name]
+    f32 = lambda h: np.float32(struct.unpack(">f", bytes.fromhex(h))[0])
+    return f32(d["x_scale_f32"]), f32(d["h_scale_f32"])
