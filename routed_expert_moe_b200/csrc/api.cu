@@ -183,20 +183,8 @@ struct ForwardWs {
     void* y_perm;
 };
 
-// Plan of the expert FFN: the bf16/E4M3 kernel's plan; NVFP4 caps the rows of a
-// schedule entry (32 for batches up to 256 tokens, else 128) so that its fp16 stage
-// buffers (eight, or four) fit in shared memory.
-GemmPlan ffn_plan(const moe_dims* d) {
-    GemmPlan gp = gemm_plan(d->T, d->K, d->E);
-    const int cap = d->T <= 256 ? 32 : 128;
-    if (d->expert_dtype == MOE_NVFP4 && gp.bn > cap) {
-        const int64_t rows = d->T * d->K;
-        const int64_t nonempty = d->E < rows ? d->E : rows;
-        gp.bn = cap;
-        gp.max_sched = (int)(nonempty + (rows + cap - 1) / cap);
-    }
-    return gp;
-}
+// Plan of the expert FFN: one tile schedule for every expert dtype.
+GemmPlan ffn_plan(const moe_dims* d) { return gemm_plan(d->T, d->K, d->E); }
 
 RouteWs carve_route(Carve& c, void* base, const moe_dims* d, const RouterPlan& rp) {
     RouteWs r;

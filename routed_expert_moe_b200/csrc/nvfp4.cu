@@ -288,10 +288,10 @@ __global__ void __launch_bounds__(FG_THREADS, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < NR; ++s) {
             mbar_init(smem_u32(&raw_full[s]), 1);
-            mbar_init(smem_u32(&raw_empty[s]), 4);    // one arrival per converter warp
+            mbar_init(smem_u32(&raw_empty[s]), 128);   // every converter thread
         }
         for (int s = 0; s < NF; ++s) {
-            mbar_init(smem_u32(&f16_full[s]), 1);     // the converter warp of that stage
+            mbar_init(smem_u32(&f16_full[s]), 128);
             mbar_init(smem_u32(&f16_empty[s]), 1);
         }
         for (int a = 0; a < 2; ++a) {
@@ -372,61 +372,56 @@ __global__ void __launch_bounds__(FG_THREADS, 1)
         }
     } else if (warp >= 6) {
         // ---------------------------------------------------------------- converters
-        // Converter warp w dequantises fp16 stage w of every raw stage (K values 64w .. 64w+63 of
-        // the 256): all 128 weight rows and the unit's token rows, four rows per lane at a time,
-        // into its own fp16 buffers w*NF/4 .. (w+1)*NF/4 - 1 in turn.  One producer per buffer,
-        // uses in order: a wait on a buffer's parity can never see a phase two ahead.  The MMA
-        // thread keeps the same count per warp (stage kf of a unit is warp kf % 4's).
-        const int w = warp - 6;
-        int rs = 0;
-        uint32_t rph = 0;
-        uint32_t uses = 0;
+        // The 128 converter threads dequantise the four fp16 stages of every raw stage in order:
+        // thread i converts weight row i and the unit's token rows i, i + 128, ...  All of them
+        // take the fp16 buffers in the same order and each arrives once per use, so a buffer's
+        // full / empty phases advance one use at a time.
+        const int i = threadIdx.x - 192;
+        int rs = 0, fs = 0;
+        uint32_t rph = 0, fph = 0;
         bool ok = true;
         for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
             const int4 sc = g.sched[u / g.m_blocks];
             const int mb = u % g.m_blocks;
             const bool a_full = g.Nout - mb * FG_BM > 64;
             const int nrows = ((sc.z + 15) / 16) * 16;
-            for (int kr = 0; kr < g.k_raw; ++kr) {
-                if (!mbar_wait_warp(smem_u32(&raw_full[rs]), rph, ctx, abort_flag)) {
+            for (int kr = 0; kr < g.k_raw && ok; ++kr) {
+                if (!mbar_wait(smem_u32(&raw_full[rs]), rph, ctx, abort_flag)) {
                     ok = false;
                     break;
                 }
-                const int kf = kr * 4 + w;
-                if (kf < g.k_f16) {
-                    const int m = NF / 4;   // buffers per converter warp
-                    const int fs = w * m + (int)(uses % (uint32_t)m);
-                    const uint32_t fph = (uses / (uint32_t)m) & 1u;
-                    ++uses;
-                    if (!mbar_wait_warp(smem_u32(&f16_empty[fs]), fph ^ 1u, ctx, abort_flag)) {
+                const uint8_t* st = raw + (size_t)rs * raw_bytes;
+                const uint8_t* a_c = st;
+                const uint8_t* b_c = st + FG_A_RAW;
+                const uint8_t* a_s = st + FG_A_RAW + b_raw;
+                const uint8_t* b_s = a_s + FG_A_SC;
+                for (int sub = 0; sub < 4; ++sub) {
+                    const int kf = kr * 4 + sub;
+                    if (kf >= g.k_f16) break;
+                    if (!mbar_wait(smem_u32(&f16_empty[fs]), fph ^ 1u, ctx, abort_flag)) {
                         ok = false;
                         break;
                     }
-                    const uint8_t* st = raw + (size_t)rs * raw_bytes;
-                    const uint8_t* a_c = st;
-                    const uint8_t* b_c = st + FG_A_RAW;
-                    const uint8_t* a_s = st + FG_A_RAW + b_raw;
-                    const uint8_t* b_s = a_s + FG_A_SC;
                     uint8_t* fa = f16 + (size_t)fs * f16_bytes;
                     uint8_t* fbt = fa + FG_A_F16;
-                    const int kb0 = kr * 16 + w * 4;
-                    for (int r = lane; r < FG_BM; r += 32) {
-                        if (a_full || r < 64)
-                            convert_row(a_c + r * 128, a_s + r * 16, fa + r * 128, r, w, kb0, nbk);
-                        else
+                    const int kb0 = kr * 16 + sub * 4;
+                    if (a_full || i < 64)
+                        convert_row(a_c + i * 128, a_s + i * 16, fa + i * 128, i, sub, kb0, nbk);
+                    else
 #pragma unroll
-                            for (int c = 0; c < 8; ++c)
-                                *reinterpret_cast<uint4*>(fa + r * 128 + 16 * c) = make_uint4(0, 0, 0, 0);
-                    }
-                    for (int j = lane; j < nrows; j += 32)
-                        convert_row(b_c + j * 128, b_s + j * 16, fbt + j * 128, j, w, kb0, nbk);
-                    // this lane's fp16 writes become visible to the tensor cores; one arrival per warp
+                        for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(fa + i * 128 + 16 * c) = make_uint4(0, 0, 0, 0);
+                    for (int j = i; j < nrows; j += 128)
+                        convert_row(b_c + j * 128, b_s + j * 16, fbt + j * 128, j, sub, kb0, nbk);
+                    // this thread's fp16 writes become visible to the tensor cores
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(smem_u32(&f16_full[fs]));
+                    mbar_arrive(smem_u32(&f16_full[fs]));
+                    if (++fs == NF) {
+                        fs = 0;
+                        fph ^= 1u;
+                    }
                 }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&raw_empty[rs]));
+                if (!ok) break;
+                mbar_arrive(smem_u32(&raw_empty[rs]));
                 if (++rs == NR) {
                     rs = 0;
                     rph ^= 1u;
@@ -436,7 +431,8 @@ __global__ void __launch_bounds__(FG_THREADS, 1)
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA
         if (lane == 0) {
-            uint32_t uses[4] = {0u, 0u, 0u, 0u};   // stages converter warp w has filled so far
+            int fs = 0;
+            uint32_t fph = 0;
             int acc = 0;
             uint32_t acc_phase = 0;
             bool ok = true, issued = false;
@@ -451,11 +447,6 @@ __global__ void __launch_bounds__(FG_THREADS, 1)
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * 256);
                 for (int kf = 0; kf < g.k_f16; ++kf) {
-                    const int m = NF / 4;
-                    const int wq = kf & 3;   // the converter warp of this stage
-                    const int fs = wq * m + (int)(uses[wq] % (uint32_t)m);
-                    const uint32_t fph = (uses[wq] / (uint32_t)m) & 1u;
-                    ++uses[wq];
                     if (!mbar_wait(smem_u32(&f16_full[fs]), fph, ctx, abort_flag)) {
                         ok = false;
                         break;
@@ -469,6 +460,10 @@ __global__ void __launch_bounds__(FG_THREADS, 1)
                                       (kf | kk) != 0 ? 1u : 0u);
                     issued = true;
                     mma_commit(smem_u32(&f16_empty[fs]));
+                    if (++fs == NF) {
+                        fs = 0;
+                        fph ^= 1u;
+                    }
                 }
                 if (!ok) break;
                 mma_commit(smem_u32(&tfull[acc]));
@@ -592,8 +587,8 @@ Fp4Plan fp4_plan(int bn) {
     p.bn = bn;
     const int raw = (FG_A_RAW + bn * 128 + FG_A_SC + bn * 16 + 1023) & ~1023;
     const int f16 = FG_A_F16 + bn * 128;
-    // fp16 buffers: a multiple of 4 (each converter warp owns NF/4); eight when the tiles are small
-    const int nf = bn <= 32 ? 8 : 4;
+    // fp16 buffers: two for the wide tiles of large batches, five when the tiles are small
+    const int nf = bn > 64 ? 2 : 5;
     int nr = (220 * 1024 - nf * f16) / raw;
     if (nr > 8) nr = 8;
     if (nr < 2) nr = 2;

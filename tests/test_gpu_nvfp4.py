@@ -110,6 +110,12 @@ def test_nvfp4_forward_parity_decode_shape(moe):
     assert nvfp4_case(moe, w, inputs(w), tokens=np.arange(0, 64, 9)) <= NVFP4_TOL
 
 
+def test_nvfp4_forward_parity_prefill_shape(moe):
+    """4096 tokens: tiles of up to 256 token rows (two fp16 stage buffers), sampled tokens."""
+    w = W.Workload("nvfp4_prefill_T4096", 4096, 2688, 128, 6, 1856, seed=29)
+    assert nvfp4_case(moe, w, inputs(w), tokens=np.arange(3, 4096, 611)) <= NVFP4_TOL
+
+
 def test_nvfp4_expired_wait_is_reported(moe):
     w = W.WORKLOADS[0]
     h = inputs(w)
