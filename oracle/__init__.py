@@ -51,6 +51,7 @@ def lib():
             "oracle_expert_bf16": (None, [_i64, _i64, _p, _p, _p, _p]),
             "oracle_expert_rows_bf16": (ctypes.c_int, [_i64, _i64, _i64, _p, _p, _p, _p, _p, _p]),
             "oracle_combine": (None, [_i64, _i64, _i64, _p, _p, _p, _p]),
+            "oracle_shared_expert_bf16": (None, [_i64, _i64, _i64, _p, _p, _p, _p]),
             "oracle_e4m3_encode": (ctypes.c_uint8, [_f]),
             "oracle_e4m3_decode": (_f, [ctypes.c_uint8]),
             "oracle_e4m3_encode_n": (None, [_i64, _p, _p]),
@@ -163,16 +164,32 @@ def combine(y_tk, w, residual=None) -> np.ndarray:
     return out
 
 
+def shared_expert_bf16(xrows, wup_s, wdown_s) -> np.ndarray:
+    """y_s[t] = W_down_s relu(W_up_s x_t)^2 for float64 rows x_t; W_up_s [Fs][H], W_down_s [H][Fs] bf16."""
+    xrows, px = _c(xrows, np.float64)
+    wup_s, pu = _c(wup_s, np.uint16)
+    wdown_s, pd = _c(wdown_s, np.uint16)
+    T, H = xrows.shape
+    Fs = wup_s.shape[0]
+    if wup_s.shape != (Fs, H) or wdown_s.shape != (H, Fs):
+        raise ValueError("shared expert weights must be [Fs][H] and [H][Fs]")
+    y = np.empty((T, H), dtype=np.float64)
+    lib().oracle_shared_expert_bf16(T, H, Fs, px, pu, pd, y.ctypes.data)
+    return y
+
+
 def identity_slot(E: int) -> np.ndarray:
     return np.arange(E, dtype=np.int32)
 
 
-def moe_layer_bf16(x, wr, bias, wup, wdown, K, tokens=None, slot=None, residual=None):
+def moe_layer_bf16(x, wr, bias, wup, wdown, K, tokens=None, slot=None, residual=None, shared=None):
     """The whole layer for the rows ``tokens`` of x (all rows if None).
 
     Tokens do not interact (no capacity limit), so any subset is exact.
     Returns a dict with logits, idx, w, the per-assignment expert outputs
-    y [n, K, H] and out [n, H] (float64, before bf16 rounding).
+    y [n, K, H] and out [n, H] (float64, before bf16 rounding).  With
+    ``shared = (W_up_s, W_down_s)`` the shared expert's output y_s [n, H]
+    is added to out with weight 1 (and returned as y_shared).
     """
     x = np.asarray(x, dtype=np.uint16)
     if tokens is not None:
@@ -187,7 +204,12 @@ def moe_layer_bf16(x, wr, bias, wup, wdown, K, tokens=None, slot=None, residual=
     xr = np.repeat(bf16_to_f64(x), K, axis=0)
     y = expert_rows_bf16(xr, idx.reshape(-1), wup, wdown, slot).reshape(n, K, H)
     out = combine(y, w, residual)
-    return dict(logits=L, idx=idx, w=w, y=y, out=out)
+    res = dict(logits=L, idx=idx, w=w, y=y, out=out)
+    if shared is not None:
+        ys = shared_expert_bf16(bf16_to_f64(x), *shared)
+        res["y_shared"] = ys
+        res["out"] = out + ys
+    return res
 
 
 # --------------------------------------------------------------------------- FP8

@@ -208,6 +208,23 @@ void oracle_combine(int64_t T, int64_t K, int64_t H, const double* y, const doub
         }
 }
 
+/*
+ * Shared expert.  [B] section 4 "Placement on card, host RAM and NVMe" lists
+ * the model's shared experts among what stays on the card: besides the
+ * routed experts, the MoE block has an expert that every token passes
+ * through.  The pages give neither its width nor how its output joins the
+ * routed sum.  Reading: the same ungated ReLU^2 FFN as a routed expert, of
+ * width Fs, added with weight 1 (no gate):
+ *   y_s[t] = W_down_s relu(W_up_s x_t)^2,  W_up_s [Fs][H], W_down_s [H][Fs],
+ *   out[t] = (residual[t] +) sum_k w[t,k] y[t,k] + y_s[t].
+ * This function gives y_s for T rows of x (fp64 values of bf16 inputs).
+ */
+void oracle_shared_expert_bf16(int64_t T, int64_t H, int64_t Fs, const double* x, const uint16_t* wu,
+                               const uint16_t* wd, double* y) {
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t t = 0; t < T; ++t) oracle_expert_bf16(H, Fs, wu, wd, x + t * H, y + t * H);
+}
+
 /* ----------------------------------------------------------------------- */
 /* FP8 E4M3 W8A8 with scalar scales.  [B] s.2: "FP8 uses scalar-scale E4M3  */
 /* W8A8".  Reading: OCP FP8 E4M3 ("fn": no infinities, one NaN code per     */

@@ -33,6 +33,8 @@ T_WDOWN = 4      # expert down banks [E, H, F]
 T_BIAS = 5       # router-bias expert ranking (Zipf)
 T_CALIB = 6      # calibration batch of the FP8 chain
 T_XLAYER = 7     # per-layer seeded input of the FP8 chain parity cases
+T_WUP_S = 8      # shared expert up weight [Fs, H]
+T_WDOWN_S = 9    # shared expert down weight [H, Fs]
 
 
 def _stale(lib: Path, src: Path) -> bool:

@@ -1,4 +1,4 @@
-"""The five seeded workloads of the routed mixture-of-experts layer.
+"""The seeded workloads of the routed mixture-of-experts layer.
 
 Shapes follow the Nemotron 3.5 Transcribe decoder as the bloomery issue page
 states them ("2. Checkpoint facts": hidden width 2688, top-6 routing over 128
@@ -16,7 +16,7 @@ import dataclasses
 
 import numpy as np
 
-from . import (T_BIAS, T_WDOWN, T_WR, T_WUP, T_X, key, normal_bf16, u64)
+from . import (T_BIAS, T_WDOWN, T_WDOWN_S, T_WR, T_WUP, T_WUP_S, T_X, key, normal_bf16, u64)
 
 SIGMA_X = 1.0
 SIGMA_W = 0.02
@@ -35,6 +35,7 @@ class Workload:
     layers: int = 1
     fp8: bool = False
     nvfp4: bool = False
+    shared: int = 0          # shared expert width Fs (0: none)
 
     @property
     def assignments(self) -> int:
@@ -50,6 +51,9 @@ WORKLOADS = {
     # the NVFP4 (W4A4) release's experts on the decode and prefill shapes (same seeds and bf16 masters)
     5: Workload("decode_nvfp4_T64", 64, 2688, 128, 6, 1856, seed=1, nvfp4=True),
     6: Workload("prefill_nvfp4_T4096", 4096, 2688, 128, 6, 1856, seed=2, nvfp4=True),
+    # the MoE block with its shared expert (the pages give no width: one expert of the routed shape)
+    7: Workload("decode_shared_T64", 64, 2688, 128, 6, 1856, seed=1, shared=1856),
+    8: Workload("prefill_shared_T4096", 4096, 2688, 128, 6, 1856, seed=2, shared=1856),
 }
 
 
@@ -99,6 +103,16 @@ def host_w_down(w: Workload, layer: int = 0, experts=None) -> np.ndarray:
     for i, e in enumerate(experts):
         out[i] = normal_bf16(k, n, SIGMA_W, offset=int(e) * n).reshape(w.H, w.F)
     return out
+
+
+def host_w_up_shared(w: Workload, layer: int = 0) -> np.ndarray:
+    """Shared expert W_up bits, [Fs, H]."""
+    return normal_bf16(key(w.seed, T_WUP_S, layer), w.shared * w.H, SIGMA_W).reshape(w.shared, w.H)
+
+
+def host_w_down_shared(w: Workload, layer: int = 0) -> np.ndarray:
+    """Shared expert W_down bits, [H, Fs]."""
+    return normal_bf16(key(w.seed, T_WDOWN_S, layer), w.H * w.shared, SIGMA_W).reshape(w.H, w.shared)
 
 
 def host_bias(w: Workload):
