@@ -36,7 +36,8 @@ UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 WORKLOADS = {"tiny": 0, "decode": 1, "prefill": 2, "skewed": 3, "chain": 4, "decode_nvfp4": 5,
-             "prefill_nvfp4": 6}
+             "prefill_nvfp4": 6, "decode_shared": 7, "prefill_shared": 8}
+TENSOR_BOUND = ("prefill", "chain", "prefill_nvfp4", "prefill_shared")   # reported against the tensor peak
 
 
 def load_peaks():
@@ -184,7 +185,17 @@ class Layer:
             (self.wu, self.bu, self.tu), (self.wd, self.bd, self.td) = banks
             sx, sh = W.nvfp4_scales(wl)
             self.scales = moe.nvfp4_scales(self.tu, self.td, float(sx), float(sh), self.bu, self.bd)
-        self.dims = moe.dims(wl.T, wl.H, wl.E, wl.K, wl.F, nvfp4=wl.nvfp4)
+        self.shared = None
+        if wl.shared:
+            # the shared expert: W_up_s [Fs][H], W_down_s [H][Fs], bf16
+            su = torch.empty(wl.shared, wl.H, dtype=bf, device=device)
+            sd = torch.empty(wl.H, wl.shared, dtype=bf, device=device)
+            synth.normal_bf16_device(synth.key(wl.seed, synth.T_WUP_S, 0), su.numel(), W.SIGMA_W, su.data_ptr(),
+                                     stream)
+            synth.normal_bf16_device(synth.key(wl.seed, synth.T_WDOWN_S, 0), sd.numel(), W.SIGMA_W, sd.data_ptr(),
+                                     stream)
+            self.shared = (su, sd)
+        self.dims = moe.dims(wl.T, wl.H, wl.E, wl.K, wl.F, nvfp4=wl.nvfp4, Fs=wl.shared)
         self.ws = moe.alloc_workspace(self.dims, device)
         self.out = torch.empty(wl.T, wl.H, dtype=bf, device=device)
         self.idx = torch.empty(wl.T, wl.K, dtype=torch.int32, device=device)
@@ -194,7 +205,7 @@ class Layer:
     def step(self, i, x=None, out=None):
         self.moe.forward(self.dims, self.xs[i % len(self.xs)] if x is None else x, self.wr, self.bias, self.wu,
                          self.wd, self.out if out is None else out, self.ws, scales=self.scales, topk_idx=self.idx,
-                         topk_w=self.w)
+                         topk_w=self.w, shared=self.shared)
 
     def touched_experts(self, i):
         import torch
@@ -346,7 +357,9 @@ def roofline_entry(wl, stages, touched, peaks, peak_kind, workload):
     asks, with the HBM fraction of the same launch beside it.
     """
     H, F, T, K = wl.H, wl.F, wl.T, wl.K
-    rows = T * K
+    ns = wl.shared // F        # shared-expert chunks: F-wide experts every token passes through
+    rows = T * (K + ns)
+    touched = touched + ns
     es = 1 if wl.fp8 else 2
     up_ms, down_ms = stages["up_gemm"], stages["down_gemm"]
     kernel = "up_gemm" if up_ms >= down_ms else "down_gemm"
@@ -371,7 +384,7 @@ def roofline_entry(wl, stages, touched, peaks, peak_kind, workload):
     common = {"kernel": kernel, "ms_per_launch": ms, "algorithmic_bytes_per_launch": algo,
               "algorithmic_flops_per_launch": flops, "traffic": traffic_from_profile(kernel, workload),
               "hbm_gbs": gbs, "hbm_frac": gbs / hbm_peak, "tensor_tflops": tflops, "tensor_frac": tflops / tc_peak}
-    if workload in ("prefill", "chain", "prefill_nvfp4"):
+    if workload in TENSOR_BOUND:
         src = f"{peak_kind} bf16 sustained" + (" x 2 (fp8/bf16 nominal ratio)" if wl.fp8 else "")
         return dict(bound="tensor", achieved=tflops, peak=tc_peak, unit="TFLOP/s", frac=tflops / tc_peak,
                     peak_source=src, **common)
@@ -416,17 +429,19 @@ def cpu_baseline(wl, n_tokens, seed_batch=0, target_s=CPU_SAMPLE_SECONDS):
     slot[used] = range(len(used))
     t_route = time.perf_counter() - t0
     wu, wd = _host_banks(wl, 0, used, False)   # generating inputs is not timed
+    shared = (W.host_w_up_shared(wl), W.host_w_down_shared(wl)) if wl.shared else None
     dt, reps = 0.0, 0
     while (reps == 0 or dt < target_s) and reps < 1000:
         t0 = time.perf_counter()
         _, idx, _ = oracle.route(x, wr, W.host_bias(wl), wl.K)
-        oracle.moe_layer_bf16(x, wr, W.host_bias(wl), wu, wd, wl.K, slot=slot)
+        oracle.moe_layer_bf16(x, wr, W.host_bias(wl), wu, wd, wl.K, slot=slot, shared=shared)
         dt += time.perf_counter() - t0
         reps += 1
     cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
     return {"value": reps * n_tokens / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"{n_tokens} of the {wl.T} tokens of batch {seed_batch} ({wl.name}), full layer "
-                      f"(router, top-{wl.K}, {len(used)} experts' up/ReLU^2/down in fp64, combine), "
+                      f"(router, top-{wl.K}, {len(used)} experts' up/ReLU^2/down in fp64, "
+                      f"{'a shared expert of width %d, ' % wl.shared if wl.shared else ''}combine), "
                       f"{reps} times; {dt:.2f} s"}
 
 
@@ -558,9 +573,9 @@ def run_native(args):
                       if wl.nvfp4 else "bf16"),
             "data": "synthetic: seeded N(0,1) activations, N(0,0.02) router/expert weights (bf16)",
             "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "E": wl.E, "K": wl.K, "F": wl.F,
-                       "layers": wl.layers, "touched_experts": touched,
+                       "layers": wl.layers, "touched_experts": touched, "shared_expert_width": wl.shared,
                        "l2": "inputs larger than L2: the touched experts' weights "
-                             f"({touched * wl.F * wl.H * (1.125 if wl.nvfp4 else 2 if wl.fp8 else 4) * wl.layers / 1e9:.2f} GB) "
+                             f"({(touched * wl.F + wl.shared) * wl.H * (1.125 if wl.nvfp4 else 2 if wl.fp8 else 4) * wl.layers / 1e9:.2f} GB) "
                              "stream from HBM every step; token batches rotate; no flush",
                        "parallelism": f"dp{ws} (independent token batches per GPU, weights replicated)",
                        "grouped_gemm": "cta_pair" if args.gemm == "pair" else "single_cta",

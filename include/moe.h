@@ -44,7 +44,7 @@
 extern "C" {
 #endif
 
-#define MOE_ABI_VERSION 2
+#define MOE_ABI_VERSION 3
 
 typedef enum {
     MOE_OK = 0,
@@ -64,7 +64,15 @@ typedef enum {
 } moe_dtype;
 
 /* Problem size.  Limits: 0 <= T, T*K < 2^31; 1 <= E <= 256; 1 <= K <= min(E, 16);
- * 16 <= H <= 65536 and 16 <= F <= 65536, both multiples of 16 (of 32 for MOE_NVFP4). */
+ * 16 <= H <= 65536 and 16 <= F <= 65536, both multiples of 16 (of 32 for MOE_NVFP4).
+ * Fs: width of the shared expert, 0 for none.  Cited: bloomery page s.4
+ * (the model's shared experts stay on the card beside the routed ones); the
+ * pages give neither its width nor how it joins the routed sum.  Reading:
+ * an ungated ReLU^2 FFN of width Fs that every token passes through, added
+ * with weight 1.  Fs must be a multiple of F (the kernels run it as Fs/F
+ * chunks of width F, an exact split since ReLU^2 is elementwise), with
+ * K + Fs/F <= 16, E + Fs/F <= 256, T*(K + Fs/F) < 2^31, and MOE_BF16 experts
+ * (MOE_EUNSUPPORTED otherwise). */
 typedef struct {
     int64_t T;             /* tokens */
     int32_t H;             /* hidden width (router and up-projection input, down output) */
@@ -72,6 +80,7 @@ typedef struct {
     int32_t K;             /* experts per token */
     int32_t F;             /* expert width (up output, down input) */
     int32_t expert_dtype;  /* moe_dtype */
+    int32_t Fs;            /* shared expert width (0: none) */
 } moe_dims;
 
 /* Scales of the quantised experts.  Ignored for MOE_BF16.
@@ -138,26 +147,37 @@ moe_status moe_permute(const moe_dims* d, const int32_t* topk_idx, int32_t* coun
  *   x [T][H] bf16; offsets [E+1] and perm_src [T*K] as from moe_permute;
  *   w_up [E][F][H], w_down [E][H][F] (bf16, or E4M3 codes with `scales`, or
  *   NVFP4 codes [E][F][H/2], [E][H][F/2] with `scales`);
- *   y_perm [T*K][H] bf16 out.
+ *   y_perm [T*K + T*Fs/F][H] bf16 out.
+ * With a shared expert (d->Fs > 0): w_up_shared [Fs][H] and w_down_shared
+ * [H][Fs] bf16 (both NULL when Fs = 0), and rows T*K + j*T + t of y_perm
+ * receive chunk j of it for token t:
+ *   W_down_s[:, jF:(j+1)F] * relu(W_up_s[jF:(j+1)F, :] * x[t])^2.
  * scales must be non-NULL for MOE_FP8_E4M3 and MOE_NVFP4.  Cited: bloomery page s.2 and
  * s.3 (ungated ReLU^2 experts, up/down parts). */
 moe_status moe_expert_ffn(const moe_dims* d, const void* x, const int32_t* offsets,
                           const int32_t* perm_src, const void* w_up, const void* w_down,
+                          const void* w_up_shared, const void* w_down_shared,
                           const moe_fp8_scales* scales, void* y_perm, void* ws, size_t ws_bytes,
                           void* stream);
 
-/* Weighted combine: out[t] = (residual[t] +) sum_{k=0..K-1} topk_w[t][k] * y_perm[inv_row[t*K+k]],
- * summed in fp32 in the order k = 0..K-1 and rounded once to bf16.
- *   y_perm [T*K][H] bf16, inv_row [T*K], topk_w [T][K] fp32, residual [T][H] bf16 or NULL,
- *   out [T][H] bf16 (may alias residual). */
+/* Weighted combine: out[t] = (residual[t] +) sum_{k=0..K-1} topk_w[t][k] * y_perm[inv_row[t*K+k]]
+ *                              (+ sum_j y_perm[T*K + j*T + t] with a shared expert of Fs/F chunks),
+ * summed in fp32 in the order k = 0..K-1, then j = 0.., then the residual, and rounded
+ * once to bf16.
+ *   y_perm [T*K + T*Fs/F][H] bf16, inv_row [T*K], topk_w [T][K] fp32, residual [T][H] bf16
+ *   or NULL, out [T][H] bf16 (may alias residual). */
 moe_status moe_combine(const moe_dims* d, const void* y_perm, const int32_t* inv_row,
                        const float* topk_w, const void* residual, void* out, void* stream);
 
 /* The whole layer in one call (route, permute, expert FFN, combine), all
  * intermediates in the workspace.  topk_idx / topk_w ([T][K]) may be NULL;
- * when given they receive the routing.  out may alias residual. */
+ * when given they receive the routing.  out may alias residual.  With
+ * d->Fs > 0 the shared expert (w_up_shared [Fs][H], w_down_shared [H][Fs],
+ * bf16) runs in the same grouped GEMM launches as the routed experts and its
+ * output joins the combine with weight 1; both pointers NULL when Fs = 0. */
 moe_status moe_forward(const moe_dims* d, const void* x, const void* w_router, const float* bias,
-                       const void* w_up, const void* w_down, const moe_fp8_scales* scales,
+                       const void* w_up, const void* w_down, const void* w_up_shared,
+                       const void* w_down_shared, const moe_fp8_scales* scales,
                        const void* residual, void* out, int32_t* topk_idx, float* topk_w,
                        void* ws, size_t ws_bytes, void* stream);
 

@@ -27,7 +27,8 @@ _lib = ctypes.CDLL(str(_LIB_PATH))
 
 class MoeDims(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int64), ("H", ctypes.c_int32), ("E", ctypes.c_int32),
-                ("K", ctypes.c_int32), ("F", ctypes.c_int32), ("expert_dtype", ctypes.c_int32)]
+                ("K", ctypes.c_int32), ("F", ctypes.c_int32), ("expert_dtype", ctypes.c_int32),
+                ("Fs", ctypes.c_int32)]
 
 
 class MoeFp8Scales(ctypes.Structure):
@@ -47,11 +48,11 @@ _SIG = {
     "moe_route": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P, _S, _P]),
     "moe_route_static": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P]),
     "moe_permute": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P, _S, _P]),
-    "moe_expert_ffn": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, ctypes.POINTER(MoeFp8Scales), _P, _P,
-                                      _S, _P]),
+    "moe_expert_ffn": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P, _P, ctypes.POINTER(MoeFp8Scales), _P,
+                                      _P, _S, _P]),
     "moe_combine": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P]),
-    "moe_forward": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, ctypes.POINTER(MoeFp8Scales), _P, _P, _P,
-                                   _P, _P, _S, _P]),
+    "moe_forward": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P, _P, ctypes.POINTER(MoeFp8Scales), _P, _P,
+                                   _P, _P, _P, _S, _P]),
     "moe_quantize_fp8": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int64, _P, _P, _P, _P]),
     "moe_quantize_nvfp4": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, _P, _P, _P, _P, _P]),
     "moe_rmsnorm": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int32, ctypes.c_float, _P, _P, _P]),
@@ -66,7 +67,7 @@ for _name, (_res, _args) in _SIG.items():
     _f.restype = _res
     _f.argtypes = _args
 
-_ABI = 2   # the struct layouts above
+_ABI = 3   # the struct layouts and signatures above
 if _lib.moe_abi_version() != _ABI:
     raise ImportError(f"libmoe_b200 ABI {_lib.moe_abi_version()} does not match this binding ({_ABI}); rebuild")
 
@@ -106,9 +107,10 @@ def _stream(stream):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-def dims(T, H, E, K, F, fp8=False, nvfp4=False) -> MoeDims:
+def dims(T, H, E, K, F, fp8=False, nvfp4=False, Fs=0) -> MoeDims:
+    """Problem size; Fs is the width of the shared expert (0: none, else a multiple of F)."""
     dt = MOE_NVFP4 if nvfp4 else (MOE_FP8_E4M3 if fp8 else MOE_BF16)
-    return MoeDims(int(T), int(H), int(E), int(K), int(F), dt)
+    return MoeDims(int(T), int(H), int(E), int(K), int(F), dt, int(Fs))
 
 
 def workspace_size(d: MoeDims) -> int:
@@ -162,11 +164,14 @@ def permute(d, topk_idx, counts, offsets, perm_src, inv_row, ws=None, stream=Non
                             _ptr(inv_row), _ptr(ws), nbytes, _stream(stream)), "moe_permute")
 
 
-def expert_ffn(d, x, offsets, perm_src, w_up, w_down, scales, y_perm, ws, stream=None):
+def expert_ffn(d, x, offsets, perm_src, w_up, w_down, scales, y_perm, ws, stream=None, shared=None):
+    """shared = (w_up_shared [Fs, H], w_down_shared [H, Fs]) when d.Fs > 0; y_perm then has
+    T*K + T*Fs/F rows."""
     sp = ctypes.byref(scales) if scales is not None else None
+    su, sd = shared if shared is not None else (None, None)
     _check(_lib.moe_expert_ffn(ctypes.byref(d), _ptr(x), _ptr(offsets), _ptr(perm_src), _ptr(w_up),
-                               _ptr(w_down), sp, _ptr(y_perm), _ptr(ws), ws.numel() * ws.element_size(),
-                               _stream(stream)), "moe_expert_ffn")
+                               _ptr(w_down), _ptr(su), _ptr(sd), sp, _ptr(y_perm), _ptr(ws),
+                               ws.numel() * ws.element_size(), _stream(stream)), "moe_expert_ffn")
 
 
 def combine(d, y_perm, inv_row, topk_w, residual, out, stream=None):
@@ -175,11 +180,13 @@ def combine(d, y_perm, inv_row, topk_w, residual, out, stream=None):
 
 
 def forward(d, x, w_router, bias, w_up, w_down, out, ws, scales=None, residual=None, topk_idx=None,
-            topk_w=None, stream=None):
+            topk_w=None, stream=None, shared=None):
+    """The whole layer; shared = (w_up_shared [Fs, H], w_down_shared [H, Fs]) when d.Fs > 0."""
     sp = ctypes.byref(scales) if scales is not None else None
+    su, sd = shared if shared is not None else (None, None)
     _check(_lib.moe_forward(ctypes.byref(d), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(w_up), _ptr(w_down),
-                            sp, _ptr(residual), _ptr(out), _ptr(topk_idx), _ptr(topk_w), _ptr(ws),
-                            ws.numel() * ws.element_size(), _stream(stream)), "moe_forward")
+                            _ptr(su), _ptr(sd), sp, _ptr(residual), _ptr(out), _ptr(topk_idx), _ptr(topk_w),
+                            _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)), "moe_forward")
 
 
 def quantize_fp8(src, codes, scales, stream=None):

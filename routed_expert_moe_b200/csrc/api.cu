@@ -23,17 +23,17 @@ cudaError_t launch_route(const uint16_t* x, const uint16_t* wr, const float* bia
                          int K, int32_t* idx, float* w, double* P, double* xn2, double* wn2,
                          const RouterPlan& plan, const DevCtx& ctx, cudaStream_t stream,
                          void (*between)(cudaStream_t) = nullptr);
-cudaError_t launch_permute(const int32_t* idx, int64_t n, int E, int32_t* counts, int32_t* offsets,
-                           int32_t* perm_src, int32_t* inv_row, int4* sched, int* n_sched, int bn,
+cudaError_t launch_permute(const int32_t* idx, int64_t n, int K, int E, int32_t* counts, int32_t* offsets,
+                           int32_t* perm_src, int32_t* inv_row, int4* sched, int* n_sched, int bn, int ns,
                            int* scratch, const DevCtx& ctx, cudaStream_t stream);
 void set_router_small_max(int64_t v);
 void set_router_split(int v);
 size_t permute_scratch_ints(int64_t n, int E);
 size_t permute_smem_bytes(int E);
-cudaError_t launch_schedule(const int32_t* offsets, int E, int bn, int4* sched, int* n_sched,
-                            cudaStream_t stream);
-cudaError_t launch_gather(const uint16_t* x, const int32_t* perm_src, int64_t rows, int K, int64_t T, int H,
-                          void* xp, bool fp8, float x_scale, int num_sms, const DevCtx& ctx,
+cudaError_t launch_schedule(const int32_t* offsets, int E, int bn, int4* sched, int* n_sched, int ns, int64_t T,
+                            int K, cudaStream_t stream);
+cudaError_t launch_gather(const uint16_t* x, const int32_t* perm_src, int64_t rows, int64_t routed_rows, int K,
+                          int64_t T, int H, void* xp, bool fp8, float x_scale, int num_sms, const DevCtx& ctx,
                           cudaStream_t stream);
 struct GemmPlan {
     int bn;
@@ -45,7 +45,8 @@ GemmPlan gemm_plan(int64_t T, int K, int E);
 cudaError_t launch_grouped_gemm(bool fp8, bool up, const void* W, int E, int Nout, int Kdim, const void* act,
                                 int64_t rows, const int4* sched, const int* n_sched, const GemmPlan& plan,
                                 void* out, const float* w_scale, float in_scale, float out_scale, int num_sms,
-                                int debug_withhold, const DevCtx& ctx, cudaStream_t stream);
+                                int debug_withhold, const DevCtx& ctx, cudaStream_t stream, const void* Ws,
+                                int n_shared);
 cudaError_t launch_grouped_gemm_pair(bool fp8, bool up, const void* W, int E, int Nout, int Kdim, const void* act,
                                      int64_t rows, const int4* sched, const int* n_sched, int bn, int max_sched,
                                      void* out, const float* w_scale, float in_scale, float out_scale,
@@ -62,7 +63,7 @@ cudaError_t launch_gather_nvfp4(const uint16_t* x, const int32_t* perm_src, int6
                                 cudaStream_t stream);
 size_t nvfp4_scale_row_bytes(int K);
 cudaError_t launch_combine(const uint16_t* yp, const int32_t* inv_row, const float* w, const uint16_t* residual,
-                           uint16_t* out, int64_t T, int K, int H, int num_sms, const DevCtx& ctx,
+                           uint16_t* out, int64_t T, int K, int ns, int H, int num_sms, const DevCtx& ctx,
                            cudaStream_t stream);
 cudaError_t launch_rmsnorm(const uint16_t* x, uint16_t* u, int64_t T, int H, float eps, int num_sms,
                            cudaStream_t stream);
@@ -138,8 +139,20 @@ moe_status check_dims(const moe_dims* d) {
     if (d->expert_dtype != MOE_BF16 && d->expert_dtype != MOE_FP8_E4M3 && d->expert_dtype != MOE_NVFP4)
         return MOE_EINVAL;
     if (d->expert_dtype == MOE_NVFP4 && (d->H % 32 != 0 || d->F % 32 != 0)) return MOE_EINVAL;
+    // shared expert: chunks of the routed width, each an extra term of the combine
+    if (d->Fs < 0 || d->Fs % d->F != 0) return MOE_EINVAL;
+    const int ns = d->Fs / d->F;
+    if (ns > 0) {
+        if (d->K + ns > 16 || d->E + ns > 256) return MOE_EINVAL;
+        if (d->T * (int64_t)(d->K + ns) >= (int64_t)1 << 31) return MOE_EINVAL;
+        if (d->expert_dtype != MOE_BF16) return MOE_EUNSUPPORTED;
+    }
     return MOE_OK;
 }
+
+int n_shared(const moe_dims* d) { return d->Fs / d->F; }
+// rows of the expert layout: T*K routed rows, then T per shared-expert chunk
+int64_t ffn_rows(const moe_dims* d) { return d->T * (int64_t)(d->K + n_shared(d)); }
 
 moe_status cuda_status(cudaError_t e) {
     if (e == cudaSuccess) return MOE_OK;
@@ -183,8 +196,13 @@ struct ForwardWs {
     void* y_perm;
 };
 
-// Plan of the expert FFN: one tile schedule for every expert dtype.
-GemmPlan ffn_plan(const moe_dims* d) { return gemm_plan(d->T, d->K, d->E); }
+// Plan of the expert FFN: one tile schedule for every expert dtype, plus the
+// shared expert's entries (ns chunks of T rows, cut into tiles of at most bn).
+GemmPlan ffn_plan(const moe_dims* d) {
+    GemmPlan gp = gemm_plan(d->T, d->K, d->E);
+    gp.max_sched += n_shared(d) * (int)((d->T + gp.bn - 1) / gp.bn);
+    return gp;
+}
 
 RouteWs carve_route(Carve& c, void* base, const moe_dims* d, const RouterPlan& rp) {
     RouteWs r;
@@ -196,7 +214,7 @@ RouteWs carve_route(Carve& c, void* base, const moe_dims* d, const RouterPlan& r
 
 FfnWs carve_ffn(Carve& c, void* base, const moe_dims* d, const GemmPlan& gp) {
     FfnWs f;
-    const size_t rows = (size_t)d->T * d->K;
+    const size_t rows = (size_t)ffn_rows(d);
     f.sched = c.take<int4>(base, (size_t)gp.max_sched);
     f.n_sched = c.take<int>(base, 1);
     f.perm_scratch = c.take<int>(base, permute_scratch_ints(d->T * d->K, d->E));
@@ -223,7 +241,7 @@ ForwardWs carve_forward(Carve& c, void* base, const moe_dims* d) {
     f.offsets = c.take<int32_t>(base, d->E + 1);
     f.perm_src = c.take<int32_t>(base, rows);
     f.inv_row = c.take<int32_t>(base, rows);
-    f.y_perm = c.take<uint16_t>(base, rows * d->H);
+    f.y_perm = c.take<uint16_t>(base, (size_t)ffn_rows(d) * d->H);
     return f;
 }
 
@@ -251,9 +269,11 @@ size_t forward_ws_bytes(const moe_dims* d, int sms) {
 // Run the expert FFN given a schedule already in `fw`.
 moe_status run_ffn(const moe_dims* d, const DeviceInfo* dev, const DevCtx& ctx, const GemmPlan& gp,
                    const void* x, const int32_t* perm_src, const void* w_up, const void* w_down,
-                   const moe_fp8_scales* sc, FfnWs& fw, void* y_perm, cudaStream_t st, bool marks = false) {
+                   const void* w_up_s, const void* w_down_s, const moe_fp8_scales* sc, FfnWs& fw, void* y_perm,
+                   cudaStream_t st, bool marks = false) {
     const bool fp8 = d->expert_dtype == MOE_FP8_E4M3;
-    const int64_t rows = d->T * d->K;
+    const int64_t rows = ffn_rows(d);
+    const int ns = n_shared(d);
     if (d->expert_dtype == MOE_NVFP4) {
         const int withhold4 = g_debug_withhold.load();
         if (marks) stage_mark(3, st);
@@ -276,12 +296,12 @@ moe_status run_ffn(const moe_dims* d, const DeviceInfo* dev, const DevCtx& ctx, 
     }
     if (marks) stage_mark(3, st);
     // permuted copy of x (or of its E4M3 codes), read by the up projection in contiguous row blocks
-    cudaError_t e = launch_gather(static_cast<const uint16_t*>(x), perm_src, rows, d->K, d->T, d->H, fw.xp, fp8,
-                                  fp8 ? sc->x_scale : 1.0f, dev->num_sms, ctx, st);
+    cudaError_t e = launch_gather(static_cast<const uint16_t*>(x), perm_src, rows, d->T * d->K, d->K, d->T, d->H,
+                                  fw.xp, fp8, fp8 ? sc->x_scale : 1.0f, dev->num_sms, ctx, st);
     if (e != cudaSuccess) return cuda_status(e);
     const int withhold = g_debug_withhold.load();
     // optional: tiles of more than 64 tokens on CTA pairs (one activation read per 256 weight rows)
-    const bool pair = g_gemm_pair.load() && gp.bn > 64 && !withhold;
+    const bool pair = g_gemm_pair.load() && gp.bn > 64 && !withhold && ns == 0;
     if (marks) stage_mark(4, st);
     if (pair)
         e = launch_grouped_gemm_pair(fp8, true, w_up, d->E, d->F, d->H, fw.xp, rows, fw.sched, fw.n_sched, gp.bn,
@@ -290,7 +310,7 @@ moe_status run_ffn(const moe_dims* d, const DeviceInfo* dev, const DevCtx& ctx, 
     else
         e = launch_grouped_gemm(fp8, true, w_up, d->E, d->F, d->H, fw.xp, rows, fw.sched, fw.n_sched, gp, fw.hb,
                                 fp8 ? sc->w_up_scale : nullptr, fp8 ? sc->x_scale : 1.0f, fp8 ? sc->h_scale : 1.0f,
-                                dev->num_sms, withhold, ctx, st);
+                                dev->num_sms, withhold, ctx, st, w_up_s, ns);
     if (e != cudaSuccess) return cuda_status(e);
     if (marks) stage_mark(5, st);
     if (pair)
@@ -300,8 +320,15 @@ moe_status run_ffn(const moe_dims* d, const DeviceInfo* dev, const DevCtx& ctx, 
     else
         e = launch_grouped_gemm(fp8, false, w_down, d->E, d->H, d->F, fw.hb, rows, fw.sched, fw.n_sched, gp, y_perm,
                                 fp8 ? sc->w_down_scale : nullptr, fp8 ? sc->h_scale : 1.0f, 1.0f, dev->num_sms, 0,
-                                ctx, st);
+                                ctx, st, w_down_s, ns);
     return cuda_status(e);
+}
+
+// The shared expert's weights: both given (16-byte aligned) exactly when Fs > 0.
+moe_status check_shared(const moe_dims* d, const void* w_up_s, const void* w_down_s) {
+    if (d->Fs == 0) return (w_up_s || w_down_s) ? MOE_EINVAL : MOE_OK;
+    if (d->T > 0 && (!w_up_s || !w_down_s)) return MOE_EINVAL;
+    return aligned(w_up_s, 16) && aligned(w_down_s, 16) ? MOE_OK : MOE_EINVAL;
 }
 
 moe_status check_fp8_scales(const moe_dims* d, const moe_fp8_scales* sc) {
@@ -388,17 +415,18 @@ moe_status moe_permute(const moe_dims* d, const int32_t* topk_idx, int32_t* coun
     if (!aligned(ws, 256)) return MOE_EINVAL;
     DeviceInfo* dev = nullptr;
     if ((s = device_setup(&dev)) != MOE_OK) return s;
-    return cuda_status(launch_permute(topk_idx, d->T * d->K, d->E, counts, offsets, perm_src, inv_row, nullptr,
-                                      nullptr, 16, static_cast<int*>(ws), make_ctx(dev),
+    return cuda_status(launch_permute(topk_idx, d->T * d->K, d->K, d->E, counts, offsets, perm_src, inv_row, nullptr,
+                                      nullptr, 16, 0, static_cast<int*>(ws), make_ctx(dev),
                                       static_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_expert_ffn(const moe_dims* d, const void* x, const int32_t* offsets, const int32_t* perm_src,
-                          const void* w_up, const void* w_down, const moe_fp8_scales* scales, void* y_perm,
-                          void* ws, size_t ws_bytes, void* stream) {
+                          const void* w_up, const void* w_down, const void* w_up_shared, const void* w_down_shared,
+                          const moe_fp8_scales* scales, void* y_perm, void* ws, size_t ws_bytes, void* stream) {
     moe_status s = check_dims(d);
     if (s != MOE_OK) return s;
     if ((s = check_fp8_scales(d, scales)) != MOE_OK) return s;
+    if ((s = check_shared(d, w_up_shared, w_down_shared)) != MOE_OK) return s;
     if (d->T > 0 && (!x || !offsets || !perm_src || !w_up || !w_down || !y_perm || !ws)) return MOE_EINVAL;
     if (!aligned(x, 16) || !aligned(w_up, 16) || !aligned(w_down, 16) || !aligned(y_perm, 16) || !aligned(ws, 256))
         return MOE_EINVAL;
@@ -410,9 +438,10 @@ moe_status moe_expert_ffn(const moe_dims* d, const void* x, const int32_t* offse
     FfnWs fw = carve_ffn(c, ws, d, gp);
     if (c.off > ws_bytes) return MOE_EWORKSPACE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    cudaError_t e = launch_schedule(offsets, d->E, gp.bn, fw.sched, fw.n_sched, st);
+    cudaError_t e = launch_schedule(offsets, d->E, gp.bn, fw.sched, fw.n_sched, n_shared(d), d->T, d->K, st);
     if (e != cudaSuccess) return cuda_status(e);
-    return run_ffn(d, dev, make_ctx(dev), gp, x, perm_src, w_up, w_down, scales, fw, y_perm, st);
+    return run_ffn(d, dev, make_ctx(dev), gp, x, perm_src, w_up, w_down, w_up_shared, w_down_shared, scales, fw,
+                   y_perm, st);
 }
 
 moe_status moe_combine(const moe_dims* d, const void* y_perm, const int32_t* inv_row, const float* topk_w,
@@ -426,15 +455,18 @@ moe_status moe_combine(const moe_dims* d, const void* y_perm, const int32_t* inv
     if ((s = device_setup(&dev)) != MOE_OK) return s;
     return cuda_status(launch_combine(static_cast<const uint16_t*>(y_perm), inv_row, topk_w,
                                       static_cast<const uint16_t*>(residual), static_cast<uint16_t*>(out), d->T,
-                                      d->K, d->H, dev->num_sms, make_ctx(dev), static_cast<cudaStream_t>(stream)));
+                                      d->K, n_shared(d), d->H, dev->num_sms, make_ctx(dev),
+                                      static_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_forward(const moe_dims* d, const void* x, const void* w_router, const float* bias, const void* w_up,
-                       const void* w_down, const moe_fp8_scales* scales, const void* residual, void* out,
-                       int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes, void* stream) {
+                       const void* w_down, const void* w_up_shared, const void* w_down_shared,
+                       const moe_fp8_scales* scales, const void* residual, void* out, int32_t* topk_idx,
+                       float* topk_w, void* ws, size_t ws_bytes, void* stream) {
     moe_status s = check_dims(d);
     if (s != MOE_OK) return s;
     if ((s = check_fp8_scales(d, scales)) != MOE_OK) return s;
+    if ((s = check_shared(d, w_up_shared, w_down_shared)) != MOE_OK) return s;
     if (d->T > 0 && (!x || !w_router || !w_up || !w_down || !out || !ws)) return MOE_EINVAL;
     if (!aligned(x, 16) || !aligned(w_router, 16) || !aligned(w_up, 16) || !aligned(w_down, 16) ||
         !aligned(residual, 16) || !aligned(out, 16) || !aligned(ws, 256))
@@ -466,15 +498,16 @@ moe_status moe_forward(const moe_dims* d, const void* x, const void* w_router, c
     Carve cf;
     FfnWs ffw = carve_ffn(cf, sbase, d, gp);   // reuses the router scratch region
     stage_mark(2, st);
-    e = launch_permute(idx, d->T * d->K, d->E, fw.counts, fw.offsets, fw.perm_src, fw.inv_row, ffw.sched,
-                       ffw.n_sched, gp.bn, ffw.perm_scratch, ctx, st);
+    e = launch_permute(idx, d->T * d->K, d->K, d->E, fw.counts, fw.offsets, fw.perm_src, fw.inv_row, ffw.sched,
+                       ffw.n_sched, gp.bn, n_shared(d), ffw.perm_scratch, ctx, st);
     if (e != cudaSuccess) return cuda_status(e);
-    s = run_ffn(d, dev, ctx, gp, x, fw.perm_src, w_up, w_down, scales, ffw, fw.y_perm, st, true);
+    s = run_ffn(d, dev, ctx, gp, x, fw.perm_src, w_up, w_down, w_up_shared, w_down_shared, scales, ffw, fw.y_perm,
+                st, true);
     if (s != MOE_OK) return s;
     stage_mark(6, st);
     e = launch_combine(static_cast<const uint16_t*>(fw.y_perm), fw.inv_row, w,
-                       static_cast<const uint16_t*>(residual), static_cast<uint16_t*>(out), d->T, d->K, d->H,
-                       dev->num_sms, ctx, st);
+                       static_cast<const uint16_t*>(residual), static_cast<uint16_t*>(out), d->T, d->K,
+                       n_shared(d), d->H, dev->num_sms, ctx, st);
     stage_mark(7, st);
     return cuda_status(e);
 }
@@ -527,7 +560,7 @@ moe_status moe_quantize_act_fp8(int64_t rows, int32_t H, float x_scale, const vo
     DeviceInfo* dev = nullptr;
     moe_status s = device_setup(&dev);
     if (s != MOE_OK) return s;
-    return cuda_status(launch_gather(static_cast<const uint16_t*>(x), nullptr, rows, 1, rows, H, codes, true,
+    return cuda_status(launch_gather(static_cast<const uint16_t*>(x), nullptr, rows, rows, 1, rows, H, codes, true,
                                      x_scale, dev->num_sms, make_ctx(dev), static_cast<cudaStream_t>(stream)));
 }
 

@@ -16,8 +16,10 @@ namespace moe {
 // k < K loads the token's k-th row index and weight, the others get them by
 // shuffle; each lane then loads two vectors of all K rows at once (2K loads
 // in flight).  Small batches thus still spread over the whole GPU.
-// KMAX (8 or 16) bounds K at compile time so that the vectors stay in
-// registers.
+// KMAX (8 or 16) bounds K + ns at compile time so that the vectors stay in
+// registers.  With a shared expert of ns chunks, slots k = K + j add row
+// T*K + j*T + t with weight 1 after the routed terms (the shared expert joins
+// the routed sum with weight 1).
 constexpr int CB_THREADS = 256;
 
 template <int KMAX>
@@ -25,8 +27,8 @@ __global__ void __launch_bounds__(CB_THREADS) combine_kernel(const uint16_t* __r
                                                              const int32_t* __restrict__ inv_row,
                                                              const float* __restrict__ w,
                                                              const uint16_t* residual, uint16_t* out,
-                                                             int64_t T, int K, int H, int64_t rows,
-                                                             DevCtx ctx) {
+                                                             int64_t T, int K, int ns, int H,
+                                                             int64_t rows, DevCtx ctx) {
     pdl_enter();
     const int lane = threadIdx.x % 32;
     const int nv = H / 8;
@@ -46,7 +48,11 @@ __global__ void __launch_bounds__(CB_THREADS) combine_kernel(const uint16_t* __r
                 my_r = 0;
                 my_w = 0.0f;
             }
+        } else if (lane < K + ns) {
+            my_r = (int)(T * K + (lane - K) * T + t);
+            my_w = 1.0f;
         }
+        const int KT = K + ns;   // terms of the sum
         const uint4* src[KMAX];
         float wk[KMAX];
 #pragma unroll
@@ -63,7 +69,7 @@ __global__ void __launch_bounds__(CB_THREADS) combine_kernel(const uint16_t* __r
             uint4 q0[KMAX], q1[KMAX];
 #pragma unroll
             for (int k = 0; k < KMAX; ++k) {
-                if (k < K) {
+                if (k < KT) {
                     q0[k] = src[k][v0];
                     if (has1) q1[k] = src[k][v1];
                 }
@@ -81,7 +87,7 @@ __global__ void __launch_bounds__(CB_THREADS) combine_kernel(const uint16_t* __r
                 for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
 #pragma unroll
                 for (int k = 0; k < KMAX; ++k) {
-                    if (k >= K) break;
+                    if (k >= KT) break;
                     const uint4 q = half ? q1[k] : q0[k];
                     const uint32_t qq[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
@@ -210,7 +216,7 @@ static unsigned grid_rows(int64_t rows, int num_sms) {
 }
 
 cudaError_t launch_combine(const uint16_t* yp, const int32_t* inv_row, const float* w,
-                           const uint16_t* residual, uint16_t* out, int64_t T, int K, int H,
+                           const uint16_t* residual, uint16_t* out, int64_t T, int K, int ns, int H,
                            int num_sms, const DevCtx& ctx, cudaStream_t stream) {
     if (T == 0) return cudaSuccess;
     // warps per block: small batches spread over the SMs, large ones 8 per block
@@ -222,9 +228,12 @@ cudaError_t launch_combine(const uint16_t* yp, const int32_t* inv_row, const flo
     int64_t blocks = (items + wpb - 1) / wpb;
     if (blocks > cap) blocks = cap;
     const dim3 grid((unsigned)blocks), block((unsigned)(32 * wpb));
-    if (K <= 8)
-        return launch_k(combine_kernel<8>, grid, block, 0, stream, yp, inv_row, w, residual, out, T, K, H, T * K, ctx);
-    return launch_k(combine_kernel<16>, grid, block, 0, stream, yp, inv_row, w, residual, out, T, K, H, T * K, ctx);
+    const int64_t rows = T * K;   // routed rows: the range inv_row may name
+    if (K + ns <= 8)
+        return launch_k(combine_kernel<8>, grid, block, 0, stream, yp, inv_row, w, residual, out, T, K, ns, H, rows,
+                        ctx);
+    return launch_k(combine_kernel<16>, grid, block, 0, stream, yp, inv_row, w, residual, out, T, K, ns, H, rows,
+                    ctx);
 }
 
 cudaError_t launch_rmsnorm(const uint16_t* x, uint16_t* u, int64_t T, int H, float eps, int num_sms,

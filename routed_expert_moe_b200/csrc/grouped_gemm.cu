@@ -58,6 +58,9 @@ struct GemmArgs {
     float in_scale;          // x_scale (up) or h_scale (down), fp8 only
     float out_scale;         // h_scale for the fp8 up output
     int debug_withhold;      // 1: block 0 withholds its first load
+    int e_shared;            // schedule entries with e >= e_shared are chunk e - e_shared of the shared expert
+    int shared_cols;         // down: chunk j starts at column j * shared_cols of a {n * F, H, 1} map
+                             // (0: chunk j is z = j of a {F, H, n} map)
 };
 
 struct GemmMaps {
@@ -66,9 +69,15 @@ struct GemmMaps {
     CUtensorMap b128;        // activations, 128-row box
     CUtensorMap b64;         // activations, 64-row box
     CUtensorMap b16;         // activations, 16-row box
+    CUtensorMap s128;        // shared-expert weights, 128-row box: [n * F][H] (up) or 3-D (down, below)
+    CUtensorMap s64;         // shared-expert weights, 64-row box
+    CUtensorMap r128;        // down projection with a shared expert: the routed bank as 3-D {F, H, E}
+    CUtensorMap r64;
 };
 
-template <bool FP8, bool UP>
+// SHD: the schedule may name chunks of the shared expert (a separate
+// instantiation, so the routed-only kernel carries none of that code).
+template <bool FP8, bool UP, bool SHD>
 __global__ void __launch_bounds__(GG_THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ GemmMaps maps, GemmArgs g, DevCtx ctx) {
     constexpr int KEL = GG_ROW_BYTES / (FP8 ? 1 : 2);   // elements of K per stage
@@ -131,7 +140,22 @@ __global__ void __launch_bounds__(GG_THREADS, 1)
                 const int n16 = (sc.z + 15) / 16;         // 16-row groups of activations
                 const int n128 = n16 / 8, n64 = (n16 % 8) / 4, r16 = n16 % 4;
                 const uint32_t bytes = (uint32_t)((a_full ? 128 : 64) * GG_ROW_BYTES + n16 * 16 * GG_ROW_BYTES);
-                const int a_y = sc.x * g.Nout + mb * GG_BM;
+                // the weight box of this unit: one map and one origin for all its K stages
+                const CUtensorMap* amap = a_full ? &maps.a128 : &maps.a64;
+                int ax0 = 0, ay = sc.x * g.Nout + mb * GG_BM, az = 0;
+                if constexpr (SHD) {
+                    const bool shd = sc.x >= g.e_shared;   // a chunk of the shared expert
+                    const int a_e = shd ? sc.x - g.e_shared : sc.x;
+                    if (shd) amap = a_full ? &maps.s128 : &maps.s64;
+                    if constexpr (UP) {
+                        ay = a_e * g.Nout + mb * GG_BM;   // rows a_e * F + mb * 128 of [n * F][H] or [E * F][H]
+                    } else {
+                        if (!shd) amap = a_full ? &maps.r128 : &maps.r64;
+                        ay = mb * GG_BM;                  // routed: (kx, row, e); shared: (kx, row, j) or
+                        az = shd && g.shared_cols ? 0 : a_e;   // (j * F + kx, row, 0)
+                        ax0 = shd ? a_e * g.shared_cols : 0;
+                    }
+                }
                 for (int ks = 0; ks < g.k_stages; ++ks) {
                     if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, ctx, abort_flag)) {
                         ok = false;
@@ -145,7 +169,10 @@ __global__ void __launch_bounds__(GG_THREADS, 1)
                         const int kx = ks * KEL;
                         const uint32_t a_dst = smem_u32(smA + (size_t)stage * GG_A_BYTES);
                         const uint32_t b_dst = smem_u32(smB + (size_t)stage * g.b_stage_bytes);
-                        tma_load_2d(a_dst, a_full ? &maps.a128 : &maps.a64, fb, kx, a_y, pol_w);
+                        if constexpr (SHD && !UP)
+                            tma_load_3d(a_dst, amap, fb, ax0 + kx, ay, az, pol_w);
+                        else
+                            tma_load_2d(a_dst, amap, fb, kx, ay, pol_w);
                         int row = 0;
                         for (int j = 0; j < n128; ++j, row += 128)
                             tma_load_2d(b_dst + row * GG_ROW_BYTES, &maps.b128, fb, kx, sc.y + row, pol_x);
@@ -313,6 +340,30 @@ static bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t col
     return r == CUDA_SUCCESS;
 }
 
+// 3-D bf16 map with dims {d0, d1, d2} (d0 contiguous) and byte strides s1,
+// s2 of dims 1 and 2; box = 128 bytes x box_rows x 1, 128-byte swizzle,
+// out-of-range elements read as zero.
+static bool make_map3(CUtensorMap* m, const void* base, int64_t d0, int64_t d1, int64_t d2, int64_t s1,
+                      int64_t s2, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)d0, (cuuint64_t)d1, (cuuint64_t)d2};
+    cuuint64_t strides[2] = {(cuuint64_t)s1, (cuuint64_t)s2};
+    cuuint32_t box[3] = {(cuuint32_t)(GG_ROW_BYTES / 2), (cuuint32_t)box_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// The column chunks of a row-major bf16 [rows][n * chunk] matrix as {chunk,
+// rows, n}: a box never reads into the next chunk.
+static bool make_map_chunks(CUtensorMap* m, const void* base, int64_t rows, int64_t chunk, int64_t n,
+                            int box_rows) {
+    return make_map3(m, base, chunk, rows, n, n * chunk * 2, chunk * 2, box_rows);
+}
+
 struct GemmPlan {
     int bn;              // max rows per schedule entry
     int n_stages;
@@ -339,10 +390,10 @@ GemmPlan gemm_plan(int64_t T, int K, int E) {
     return p;
 }
 
-template <bool FP8, bool UP>
+template <bool FP8, bool UP, bool SHD = false>
 static cudaError_t launch_one(const GemmMaps& maps, const GemmArgs& g, int grid, size_t smem, const DevCtx& ctx,
                               cudaStream_t stream) {
-    auto kfn = grouped_gemm_kernel<FP8, UP>;
+    auto kfn = grouped_gemm_kernel<FP8, UP, SHD>;
     cudaError_t err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     return launch_k(kfn, dim3(grid), dim3(GG_THREADS), smem, stream, maps, g, ctx);
@@ -350,10 +401,15 @@ static cudaError_t launch_one(const GemmMaps& maps, const GemmArgs& g, int grid,
 
 // One grouped projection.  W: [E * Nout][Kdim] (bf16 or e4m3), act: [rows][Kdim]
 // in the expert layout, out: [rows][Nout].  sched / n_sched: device schedule.
+// Ws (n_shared > 0, bf16): the shared expert as n_shared chunks of width F,
+// schedule entries E .. E + n_shared - 1 -- the up weight [n_shared * Nout][Kdim]
+// (chunk j = rows j * Nout ..), the down weight [Nout][n_shared * Kdim] (chunk j =
+// columns j * Kdim ..).
 cudaError_t launch_grouped_gemm(bool fp8, bool up, const void* W, int E, int Nout, int Kdim, const void* act,
                                 int64_t rows, const int4* sched, const int* n_sched, const GemmPlan& plan,
                                 void* out, const float* w_scale, float in_scale, float out_scale, int num_sms,
-                                int debug_withhold, const DevCtx& ctx, cudaStream_t stream) {
+                                int debug_withhold, const DevCtx& ctx, cudaStream_t stream, const void* Ws,
+                                int n_shared) {
     if (rows == 0) return cudaSuccess;
     GemmMaps maps;
     if (!make_map(&maps.a128, W, (int64_t)E * Nout, Kdim, fp8, 128) ||
@@ -361,6 +417,28 @@ cudaError_t launch_grouped_gemm(bool fp8, bool up, const void* W, int E, int Nou
         !make_map(&maps.b128, act, rows, Kdim, fp8, 128) || !make_map(&maps.b64, act, rows, Kdim, fp8, 64) ||
         !make_map(&maps.b16, act, rows, Kdim, fp8, 16))
         return cudaErrorInvalidValue;
+    int shared_cols = 0;
+    maps.s128 = maps.r128 = maps.a128;   // read only by the instantiation for a shared expert
+    maps.s64 = maps.r64 = maps.a64;
+    if (n_shared > 0) {
+        if (fp8 || !Ws) return cudaErrorInvalidValue;
+        bool ok = up ? make_map(&maps.s128, Ws, (int64_t)n_shared * Nout, Kdim, false, 128) &&
+                           make_map(&maps.s64, Ws, (int64_t)n_shared * Nout, Kdim, false, 64)
+                     : make_map_chunks(&maps.s128, Ws, Nout, Kdim, n_shared, 128) &&
+                           make_map_chunks(&maps.s64, Ws, Nout, Kdim, n_shared, 64);
+        if (!ok && !up) {
+            // a driver that refuses the chunked view: the plain [H][n * F] matrix as {n * F, H, 1},
+            // chunk j from column j * F (a K tail meets activation columns that read as zero)
+            shared_cols = Kdim;
+            ok = make_map_chunks(&maps.s128, Ws, Nout, (int64_t)n_shared * Kdim, 1, 128) &&
+                 make_map_chunks(&maps.s64, Ws, Nout, (int64_t)n_shared * Kdim, 1, 64);
+        }
+        // the routed bank [E][H][F] as {F, H, E}: the down kernel then issues one load form
+        if (ok && !up)
+            ok = make_map3(&maps.r128, W, Kdim, Nout, E, (int64_t)Kdim * 2, (int64_t)Nout * Kdim * 2, 128) &&
+                 make_map3(&maps.r64, W, Kdim, Nout, E, (int64_t)Kdim * 2, (int64_t)Nout * Kdim * 2, 64);
+        if (!ok) return cudaErrorInvalidValue;
+    }
     GemmArgs g;
     g.sched = sched;
     g.n_sched = n_sched;
@@ -376,12 +454,17 @@ cudaError_t launch_grouped_gemm(bool fp8, bool up, const void* W, int E, int Nou
     g.in_scale = in_scale;
     g.out_scale = out_scale;
     g.debug_withhold = debug_withhold;
+    g.e_shared = n_shared > 0 ? E : 0x7fffffff;
+    g.shared_cols = shared_cols;
     const int64_t max_units = (int64_t)plan.max_sched * g.m_blocks;
     const int grid = (int)(max_units < num_sms ? max_units : num_sms);
     if (fp8) {
         return up ? launch_one<true, true>(maps, g, grid, plan.smem_bytes, ctx, stream)
                   : launch_one<true, false>(maps, g, grid, plan.smem_bytes, ctx, stream);
     }
+    if (n_shared > 0)   // bf16 only
+        return up ? launch_one<false, true, true>(maps, g, grid, plan.smem_bytes, ctx, stream)
+                  : launch_one<false, false, true>(maps, g, grid, plan.smem_bytes, ctx, stream);
     return up ? launch_one<false, true>(maps, g, grid, plan.smem_bytes, ctx, stream)
               : launch_one<false, false>(maps, g, grid, plan.smem_bytes, ctx, stream);
 }

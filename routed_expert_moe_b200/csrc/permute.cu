@@ -22,7 +22,9 @@ constexpr int64_t kPermuteOneBlockMax = 4096;   // assignments sorted by the sin
 // near-equal blocks of at most bn rows, each a multiple of 16 rows except the
 // last: per = round16(ceil(cnt / ceil(cnt / bn))), nblk = ceil(cnt / per).
 // Entry {e, row0, nrows, 0}.  Called by the whole block; nb_s is shared
-// scratch of E ints.
+// scratch of E ints.  With ns > 0 the ns chunks of the shared expert follow
+// as entries e = E + j over rows row0 + j * Tsh .. row0 + (j + 1) * Tsh, cut
+// the same way.
 __device__ __forceinline__ int sched_per(int c, int bn) {
     const int nb = (c + bn - 1) / bn;
     const int per = (c + nb - 1) / nb;
@@ -63,7 +65,7 @@ __device__ int block_exclusive_scan256(int* v, int n) {
 }
 
 __device__ void build_schedule(const int* seg_off, int E, int bn, int* nb_s, int4* sched,
-                               int* n_sched) {
+                               int* n_sched, int ns, int Tsh, int row0) {
     const int tid = threadIdx.x;
     for (int e = tid; e < E; e += blockDim.x) {
         const int c = seg_off[e + 1] - seg_off[e];
@@ -71,7 +73,13 @@ __device__ void build_schedule(const int* seg_off, int E, int bn, int* nb_s, int
     }
     __syncthreads();
     const int total = block_exclusive_scan256(nb_s, E);
-    if (tid == 0) *n_sched = total;
+    const int pers = ns > 0 && Tsh > 0 ? sched_per(Tsh, bn) : 16;
+    const int nbs = ns > 0 && Tsh > 0 ? (Tsh + pers - 1) / pers : 0;
+    if (tid == 0) *n_sched = total + ns * nbs;
+    for (int q = tid; q < ns * nbs; q += blockDim.x) {
+        const int j = q / nbs, r0 = (q % nbs) * pers;
+        sched[total + q] = make_int4(E + j, row0 + j * Tsh + r0, min(pers, Tsh - r0), 0);
+    }
     for (int e = tid; e < E; e += blockDim.x) {
         const int off = seg_off[e], c = seg_off[e + 1] - off;
         if (c <= 0) continue;
@@ -92,6 +100,8 @@ struct PermuteArgs {
     int4* sched;     // may be null
     int* n_sched;
     int bn;
+    int ns;          // shared-expert chunks in the schedule (rows n + j * (n / K) ..)
+    int K;
 };
 
 __global__ void __launch_bounds__(PM_THREADS) permute_kernel(PermuteArgs a, DevCtx ctx) {
@@ -163,7 +173,7 @@ __global__ void __launch_bounds__(PM_THREADS) permute_kernel(PermuteArgs a, DevC
         for (int ex = tid; ex < E; ex += PM_THREADS) base[ex] += tot[ex];
         __syncthreads();
     }
-    if (a.sched) build_schedule(offs, E, a.bn, hist, a.sched, a.n_sched);
+    if (a.sched) build_schedule(offs, E, a.bn, hist, a.sched, a.n_sched, a.ns, (int)(a.n / a.K), (int)a.n);
 }
 
 // ---- multi-block permutation for large batches: one chunk of PM_THREADS
@@ -193,7 +203,8 @@ __global__ void __launch_bounds__(PM_THREADS) perm_hist_kernel(const int32_t* __
 // counts, offsets, per-(chunk, expert) bases, and the GEMM schedule
 __global__ void __launch_bounds__(256) perm_scan_kernel(const int* __restrict__ bcount, int G, int E,
                                                         int* __restrict__ bbase, int32_t* counts,
-                                                        int32_t* offsets, int4* sched, int* n_sched, int bn) {
+                                                        int32_t* offsets, int4* sched, int* n_sched, int bn,
+                                                        int ns, int Tsh, int row0) {
     pdl_enter();
     __shared__ int offs[257];
     __shared__ int nb[256];
@@ -218,7 +229,7 @@ __global__ void __launch_bounds__(256) perm_scan_kernel(const int* __restrict__ 
         }
     }
     __syncthreads();
-    if (sched) build_schedule(offs, E, bn, nb, sched, n_sched);
+    if (sched) build_schedule(offs, E, bn, nb, sched, n_sched, ns, Tsh, row0);
 }
 
 __global__ void __launch_bounds__(PM_THREADS) perm_scatter_kernel(const int32_t* __restrict__ idx, int64_t n,
@@ -253,13 +264,14 @@ __global__ void __launch_bounds__(PM_THREADS) perm_scatter_kernel(const int32_t*
     }
 }
 
-__global__ void schedule_kernel(const int32_t* offsets, int E, int bn, int4* sched, int* n_sched) {
+__global__ void schedule_kernel(const int32_t* offsets, int E, int bn, int4* sched, int* n_sched, int ns,
+                                int Tsh, int row0) {
     pdl_enter();
     __shared__ int offs[257];
     __shared__ int nb[256];
     for (int e = threadIdx.x; e <= E; e += blockDim.x) offs[e] = offsets[e];
     __syncthreads();
-    build_schedule(offs, E, bn, nb, sched, n_sched);
+    build_schedule(offs, E, bn, nb, sched, n_sched, ns, Tsh, row0);
 }
 
 // x / s rounded to nearest from y = RN(1/s): q = RN(x y), r = x - s q (exact,
@@ -278,11 +290,12 @@ __device__ __forceinline__ float div_by_scale(float x, float s, float y) {
 }
 
 // xp[r] = x[perm_src[r] / K], or its E4M3 codes e4m3(x / x_scale) (fp8);
-// with perm_src == null the rows are taken in order (xp[r] = x[r]).  One
+// with perm_src == null the rows are taken in order (xp[r] = x[r]).  Rows
+// r >= routed_rows are the shared expert's: xp[r] = x[(r - routed_rows) % T].  One
 // warp per row, four 16-byte loads per lane in flight before their stores.
 __global__ void gather_rows_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm_src,
-                                   int64_t rows, int K, int64_t T, int H, void* __restrict__ xp,
-                                   int fp8, float x_scale, DevCtx ctx) {
+                                   int64_t rows, int64_t routed_rows, int K, int64_t T, int H,
+                                   void* __restrict__ xp, int fp8, float x_scale, DevCtx ctx) {
     pdl_enter();
     constexpr int B = 4;
     const int lane = threadIdx.x % 32;
@@ -291,7 +304,9 @@ __global__ void gather_rows_kernel(const uint16_t* __restrict__ x, const int32_t
     const float y = fp8 ? __frcp_rn(x_scale) : 1.0f;
     for (int64_t r = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32; r < rows; r += warps) {
         int64_t t = r;
-        if (perm_src) {
+        if (r >= routed_rows) {
+            t = (r - routed_rows) % T;
+        } else if (perm_src) {
             const int32_t src = perm_src[r];
             t = src / K;
             if (src < 0 || t >= T) {
@@ -342,11 +357,11 @@ size_t permute_scratch_ints(int64_t n, int E) {
     return (size_t)(2 * G * E);
 }
 
-cudaError_t launch_permute(const int32_t* idx, int64_t n, int E, int32_t* counts, int32_t* offsets,
-                           int32_t* perm_src, int32_t* inv_row, int4* sched, int* n_sched, int bn,
+cudaError_t launch_permute(const int32_t* idx, int64_t n, int K, int E, int32_t* counts, int32_t* offsets,
+                           int32_t* perm_src, int32_t* inv_row, int4* sched, int* n_sched, int bn, int ns,
                            int* scratch, const DevCtx& ctx, cudaStream_t stream) {
     if (n <= kPermuteOneBlockMax) {
-        PermuteArgs a{idx, n, E, counts, offsets, perm_src, inv_row, sched, n_sched, bn};
+        PermuteArgs a{idx, n, E, counts, offsets, perm_src, inv_row, sched, n_sched, bn, ns, K};
         return launch_k(permute_kernel, dim3(1), dim3(PM_THREADS), permute_smem_bytes(E), stream, a, ctx);
     }
     if (!scratch) return cudaErrorInvalidValue;
@@ -356,26 +371,27 @@ cudaError_t launch_permute(const int32_t* idx, int64_t n, int E, int32_t* counts
     cudaError_t err = launch_k(perm_hist_kernel, dim3(G), dim3(PM_THREADS), 0, stream, idx, n, E, bcount, ctx);
     if (err != cudaSuccess) return err;
     err = launch_k(perm_scan_kernel, dim3(1), dim3(256), 0, stream, bcount, G, E, bbase, counts, offsets, sched,
-                   n_sched, bn);
+                   n_sched, bn, ns, (int)(n / K), (int)n);
     if (err != cudaSuccess) return err;
     return launch_k(perm_scatter_kernel, dim3(G), dim3(PM_THREADS), (size_t)32 * E * sizeof(int), stream, idx, n,
                     E, bbase, perm_src, inv_row);
 }
 
-cudaError_t launch_schedule(const int32_t* offsets, int E, int bn, int4* sched, int* n_sched,
-                            cudaStream_t stream) {
-    return launch_k(schedule_kernel, dim3(1), dim3(256), 0, stream, offsets, E, bn, sched, n_sched);
+cudaError_t launch_schedule(const int32_t* offsets, int E, int bn, int4* sched, int* n_sched, int ns, int64_t T,
+                            int K, cudaStream_t stream) {
+    return launch_k(schedule_kernel, dim3(1), dim3(256), 0, stream, offsets, E, bn, sched, n_sched, ns, (int)T,
+                    (int)(T * K));
 }
 
-cudaError_t launch_gather(const uint16_t* x, const int32_t* perm_src, int64_t rows, int K, int64_t T,
-                          int H, void* xp, bool fp8, float x_scale, int num_sms, const DevCtx& ctx,
+cudaError_t launch_gather(const uint16_t* x, const int32_t* perm_src, int64_t rows, int64_t routed_rows, int K,
+                          int64_t T, int H, void* xp, bool fp8, float x_scale, int num_sms, const DevCtx& ctx,
                           cudaStream_t stream) {
     if (rows == 0) return cudaSuccess;
     int64_t blocks = (rows + 7) / 8;
     const int64_t cap = (int64_t)num_sms * 8;
     if (blocks > cap) blocks = cap;
-    return launch_k(gather_rows_kernel, dim3((unsigned)blocks), dim3(256), 0, stream, x, perm_src, rows, K, T, H, xp,
-                    fp8 ? 1 : 0, x_scale, ctx);
+    return launch_k(gather_rows_kernel, dim3((unsigned)blocks), dim3(256), 0, stream, x, perm_src, rows, routed_rows,
+                    K, T, H, xp, fp8 ? 1 : 0, x_scale, ctx);
 }
 
 }  // namespace moe

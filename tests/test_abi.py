@@ -42,7 +42,7 @@ def test_library_exports_every_declared_symbol(moe):
 
 
 def test_status_strings_and_version(moe):
-    assert moe.abi_version() == 2   # moe_quant_scales carries the NVFP4 block-scale banks
+    assert moe.abi_version() == 3   # moe_dims.Fs and the shared-expert weights of moe_expert_ffn / moe_forward
     for s in range(8):
         assert moe.status_string(s).startswith("MOE_")
     assert "unknown" in moe.status_string(99)
@@ -61,7 +61,7 @@ def test_invalid_dims_are_rejected_on_the_host(moe, kw):
     d = bad(moe, **kw)
     n = ctypes.c_size_t()
     assert moe.raw_library().moe_workspace_size(ctypes.byref(d), ctypes.byref(n)) == moe.MOE_EINVAL
-    assert moe.raw_library().moe_forward(ctypes.byref(d), *([None] * 11), 0, None) == moe.MOE_EINVAL
+    assert moe.raw_library().moe_forward(ctypes.byref(d), *([None] * 13), 0, None) == moe.MOE_EINVAL
 
 
 def test_workspace_size_scales_with_tokens(moe):
@@ -82,7 +82,7 @@ def test_null_and_missing_arguments(moe):
     assert lib.moe_route(ctypes.byref(d), None, None, None, None, None, None, 0, None) == moe.MOE_EINVAL
     assert lib.moe_permute(ctypes.byref(d), None, None, None, None, None, None, 0, None) == moe.MOE_EINVAL
     fp8 = moe.dims(64, 2688, 128, 6, 1856, fp8=True)
-    assert lib.moe_expert_ffn(ctypes.byref(fp8), *([None] * 5), None, None, None, 0, None) == moe.MOE_EINVAL
+    assert lib.moe_expert_ffn(ctypes.byref(fp8), *([None] * 10), 0, None) == moe.MOE_EINVAL
     assert lib.moe_rmsnorm(4, 2690, 1e-5, None, None, None) == moe.MOE_EINVAL
     assert lib.moe_quantize_fp8(-1, 4, None, None, None, None) == moe.MOE_EINVAL
     assert lib.moe_debug_set(99, 0) == moe.MOE_EINVAL
@@ -92,9 +92,33 @@ def test_null_and_missing_arguments(moe):
 def test_empty_batch_is_ok_without_a_device(moe):
     lib = moe.raw_library()
     d = bad(moe, T=0)
-    assert lib.moe_forward(ctypes.byref(d), *([None] * 11), 0, None) == moe.MOE_OK
+    assert lib.moe_forward(ctypes.byref(d), *([None] * 13), 0, None) == moe.MOE_OK
     assert lib.moe_rmsnorm(0, 2688, 1e-5, None, None, None) == moe.MOE_OK
     assert lib.moe_quantize_fp8(0, 10, None, None, None, None) == moe.MOE_OK
+
+
+def test_shared_expert_dims_and_pointers_are_checked_on_the_host(moe):
+    lib = moe.raw_library()
+    n = ctypes.c_size_t()
+    ws = lambda d: lib.moe_workspace_size(ctypes.byref(d), ctypes.byref(n))
+    assert ws(bad(moe, Fs=1000)) == moe.MOE_EINVAL                 # not a multiple of F
+    assert ws(bad(moe, Fs=-1856)) == moe.MOE_EINVAL
+    assert ws(bad(moe, Fs=11 * 1856)) == moe.MOE_EINVAL            # K + Fs/F > 16
+    fp8 = moe.dims(64, 2688, 128, 6, 1856, fp8=True, Fs=1856)
+    assert ws(fp8) == moe.MOE_EUNSUPPORTED                           # bf16 experts only
+    plain = moe.workspace_size(bad(moe))
+    shared = moe.workspace_size(bad(moe, Fs=2 * 1856))
+    assert shared >= plain + 2 * 64 * (2688 * 2 * 2 + 1856 * 2)     # X, H and Y rows of two chunks
+    fake = ctypes.c_void_p(4096)
+    d0 = bad(moe, T=0)                                               # no device call before these checks
+    assert lib.moe_forward(ctypes.byref(d0), *([None] * 5), fake, None, *([None] * 6), 0, None) == moe.MOE_EINVAL
+    ds = bad(moe, T=0, Fs=1856)
+    assert lib.moe_forward(ctypes.byref(ds), *([None] * 13), 0, None) == moe.MOE_OK
+    ds = bad(moe, Fs=1856)
+    assert lib.moe_forward(ctypes.byref(ds), *([None] * 13), 0, None) == moe.MOE_EINVAL
+    odd = ctypes.c_void_p(4100)                                      # not 16-byte aligned
+    assert lib.moe_forward(ctypes.byref(bad(moe, T=0, Fs=1856)), *([None] * 5), odd, fake,
+                           *([None] * 6), 0, None) == moe.MOE_EINVAL
 
 
 def test_package_has_no_cpu_path():
