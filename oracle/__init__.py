@@ -64,6 +64,11 @@ def lib():
             "oracle_rmsnorm_bf16": (None, [_i64, _i64, _p, _f, _p]),
             "oracle_round_bf16": (None, [_i64, _p, _p]),
             "oracle_hidden_amax_bf16": (ctypes.c_double, [_i64, _i64, _i64, _p, _p, _p, _p]),
+            "oracle_b128_kp": (_i64, [_i64]),
+            "oracle_quantize_fp8_b128": (None, [_i64, _i64, _p, _p, _p]),
+            "oracle_expert_fp8_b128": (None, [_i64, _i64, _p, _p, _p, _p, _p, _f, _f, _p]),
+            "oracle_expert_rows_fp8_b128": (ctypes.c_int, [_i64, _i64, _i64, _p, _p, _p, _p, _p, _p, _p,
+                                                           _f, _f, _p]),
             "oracle_e2m1_encode": (ctypes.c_uint8, [_f]),
             "oracle_e2m1_decode": (_f, [ctypes.c_uint8]),
             "oracle_e2m1_encode_n": (None, [_i64, _p, _p]),
@@ -286,6 +291,86 @@ def moe_layer_fp8(x, wr, bias, qup, sup, qdown, sdown, sx, sh, K, tokens=None, s
     qx = quantize_act_fp8(x, sx)
     qxr = np.repeat(qx, K, axis=0)
     y = expert_rows_fp8(qxr, idx.reshape(-1), qup, sup, qdown, sdown, slot, sx, sh).reshape(n, K, H)
+    out = combine(y, w, residual)
+    return dict(logits=L, idx=idx, w=w, y=y, out=out, qx=qx)
+
+
+# --------------------------------------------------------------------------- FP8_B128
+
+def b128_kp(K: int) -> int:
+    """K padded to whole blocks of 128 (1856 -> 1920)."""
+    return int(lib().oracle_b128_kp(K))
+
+
+def quantize_fp8_b128(w):
+    """W [..., rows, K] bf16 bits -> (codes [..., rows, Kp], scales [..., rows, Kp/128] fp32)."""
+    w = np.ascontiguousarray(w, dtype=np.uint16)
+    *lead, rows, K = w.shape
+    n = int(np.prod(lead)) if lead else 1
+    Kp = b128_kp(K)
+    q = np.empty((n * rows, Kp), dtype=np.uint8)
+    s = np.empty((n * rows, Kp // 128), dtype=np.float32)
+    lib().oracle_quantize_fp8_b128(n * rows, K, w.ctypes.data, q.ctypes.data, s.ctypes.data)
+    return q.reshape(*lead, rows, Kp), s.reshape(*lead, rows, Kp // 128)
+
+
+def scalar_to_fp8_b128(q, s, K: int):
+    """Per-tensor E4M3 codes q [..., rows, K] with tensor scales s [...] as FP8_B128: codes padded
+    with zeros to Kp, every block scale = the tensor scale."""
+    q = np.asarray(q, dtype=np.uint8)
+    Kp = b128_kp(K)
+    qp = np.zeros(q.shape[:-1] + (Kp,), dtype=np.uint8)
+    qp[..., :K] = q
+    s = np.asarray(s, dtype=np.float32)
+    sb = np.broadcast_to(s.reshape(s.shape + (1, 1)), q.shape[:-1] + (Kp // 128,)).astype(np.float32)
+    return qp, np.ascontiguousarray(sb)
+
+
+def quantize_act_fp8_b128(x, s: float) -> np.ndarray:
+    """Static-scale activation codes of x [rows, K], zero-padded to Kp."""
+    q = quantize_act_fp8(x, s)
+    K = q.shape[-1]
+    qp = np.zeros(q.shape[:-1] + (b128_kp(K),), dtype=np.uint8)
+    qp[..., :K] = q
+    return qp
+
+
+def expert_rows_fp8_b128(qx, ex, bank_up, bank_down, slot, sx, sh, H: int, F: int) -> np.ndarray:
+    """y[r] = W8A8 expert ex[r] with FP8_B128 banks ((codes, scales) for up [n][F][Hp] and down
+    [n][H][Fp]) on the zero-padded activation codes qx [R][Hp]."""
+    qx, px = _c(qx, np.uint8)
+    ex, pe = _c(ex, np.int32)
+    qu, pqu = _c(bank_up[0], np.uint8)
+    su, psu = _c(bank_up[1], np.float32)
+    qd, pqd = _c(bank_down[0], np.uint8)
+    sd, psd = _c(bank_down[1], np.float32)
+    slot, ps = _c(slot, np.int32)
+    R = qx.shape[0]
+    if qu.shape[1:] != (F, b128_kp(H)) or qd.shape[1:] != (H, b128_kp(F)) or qx.shape[1] != b128_kp(H):
+        raise ValueError("FP8_B128 shapes do not match H and F")
+    y = np.empty((R, H), dtype=np.float64)
+    if lib().oracle_expert_rows_fp8_b128(R, H, F, px, pe, pqu, psu, pqd, psd, ps, np.float32(sx),
+                                         np.float32(sh), y.ctypes.data) != 0:
+        raise ValueError("a routed expert's bank was not supplied")
+    return y
+
+
+def moe_layer_fp8_b128(x, wr, bias, bank_up, bank_down, sx, sh, K, H, F, tokens=None, slot=None,
+                       residual=None):
+    """W8A8 layer with FP8_B128 expert banks: bf16 router on x; x and H quantised with static scales."""
+    x = np.asarray(x, dtype=np.uint16)
+    if tokens is not None:
+        x = x[np.asarray(tokens)]
+        if residual is not None:
+            residual = np.asarray(residual)[np.asarray(tokens)]
+    E = wr.shape[0]
+    if slot is None:
+        slot = identity_slot(E)
+    L, idx, w = route(x, wr, bias, K)
+    n = x.shape[0]
+    qx = quantize_act_fp8_b128(x, sx)
+    y = expert_rows_fp8_b128(np.repeat(qx, K, axis=0), idx.reshape(-1), bank_up, bank_down, slot, sx, sh,
+                             H, F).reshape(n, K, H)
     out = combine(y, w, residual)
     return dict(logits=L, idx=idx, w=w, y=y, out=out, qx=qx)
 

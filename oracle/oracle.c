@@ -327,6 +327,90 @@ int oracle_expert_rows_fp8(int64_t R, int64_t H, int64_t F, const uint8_t* qxrow
 }
 
 /* ----------------------------------------------------------------------- */
+/* FP8_B128.  [B] s.3 ("Kernel dispatch") and the FP8 release notes: the    */
+/* FP8 matrix normaliser maps scalar scales to FP8_B128, and the 64-value  */
+/* tail of K = 1856 remains (physical K 1920).  Reading: E4M3 codes with   */
+/* one fp32 scale per block of 128 consecutive values along K of each row; */
+/* K is padded with zero codes to Kp = 128 * ceil(K / 128), and a block's  */
+/* scale is amax / 448 over its real values (1 for an all-zero block).  A   */
+/* scalar scale s maps to FP8_B128 as every block scale = s, codes kept.   */
+/* Activations keep the release's W8A8 rule: static scalar scales for x    */
+/* and H, their codes zero-padded to Kp like the weights'.                  */
+/* ----------------------------------------------------------------------- */
+
+int64_t oracle_b128_kp(int64_t K) { return (K + 127) / 128 * 128; }
+
+/* W [rows][K] bf16 -> codes [rows][Kp] (zero past K), scales [rows][Kp / 128]. */
+void oracle_quantize_fp8_b128(int64_t rows, int64_t K, const uint16_t* w, uint8_t* q, float* s) {
+    const int64_t Kp = oracle_b128_kp(K), nb = Kp / 128;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t b = 0; b < nb; ++b) {
+            const int64_t k0 = b * 128, k1 = k0 + 128 < K ? k0 + 128 : K;
+            float amax = 0.0f;
+            for (int64_t k = k0; k < k1; ++k) {
+                float a = fabsf(bf16_to_float(w[r * K + k]));
+                if (a > amax) amax = a;
+            }
+            const float sc = amax > 0.0f ? amax / 448.0f : 1.0f;
+            s[r * nb + b] = sc;
+            for (int64_t k = k0; k < k0 + 128; ++k)
+                q[r * Kp + k] = k < K ? oracle_e4m3_encode(bf16_to_float(w[r * K + k]) / sc) : 0;
+        }
+    }
+}
+
+/* sum over the blocks of one row: sum_b s[b] * sum_{k in b} dec(qw[k]) * v[k], v of length Kp */
+static double b128_dot(int64_t Kp, const uint8_t* qw, const float* s, const double* v) {
+    double tot = 0.0;
+    for (int64_t b = 0; b < Kp / 128; ++b) {
+        double part = 0.0;
+        for (int64_t k = b * 128; k < b * 128 + 128; ++k) part += (double)oracle_e4m3_decode(qw[k]) * v[k];
+        tot += (double)s[b] * part;
+    }
+    return tot;
+}
+
+/*
+ * One W8A8 expert with FP8_B128 weights on one quantised row.
+ *   qx [Hp]: e4m3(fl32(x / s_x)), zero past H
+ *   z_f  = s_x * sum_b su[f,b] * sum_{h in b} dec(qu[f,h]) dec(qx[h])
+ *   a_f  = max(z_f, 0)^2,  qa_f = e4m3(fl32(fl32(a_f) / s_h)), zero past F
+ *   y_j  = s_h * sum_b sd[j,b] * sum_{f in b} dec(qd[j,f]) dec(qa_f)
+ * qu [F][Hp] with su [F][Hp/128]; qd [H][Fp] with sd [H][Fp/128].
+ */
+void oracle_expert_fp8_b128(int64_t H, int64_t F, const uint8_t* qu, const float* su, const uint8_t* qd,
+                            const float* sd, const uint8_t* qx, float sx, float sh, double* y) {
+    const int64_t Hp = oracle_b128_kp(H), Fp = oracle_b128_kp(F);
+    double* xd = (double*)malloc((size_t)Hp * sizeof(double));
+    double* a = (double*)calloc((size_t)Fp, sizeof(double));
+    for (int64_t h = 0; h < Hp; ++h) xd[h] = (double)oracle_e4m3_decode(qx[h]);
+    for (int64_t f = 0; f < F; ++f) {
+        double z = (double)sx * b128_dot(Hp, qu + f * Hp, su + f * (Hp / 128), xd);
+        double act = z > 0.0 ? z * z : 0.0;
+        a[f] = (double)oracle_e4m3_decode(oracle_e4m3_encode((float)act / sh));
+    }
+    for (int64_t j = 0; j < H; ++j) y[j] = (double)sh * b128_dot(Fp, qd + j * Fp, sd + j * (Fp / 128), a);
+    free(xd);
+    free(a);
+}
+
+int oracle_expert_rows_fp8_b128(int64_t R, int64_t H, int64_t F, const uint8_t* qxrow, const int32_t* ex,
+                                const uint8_t* qup, const float* sup, const uint8_t* qdown, const float* sdown,
+                                const int32_t* slot, float sx, float sh, double* y) {
+    const int64_t Hp = oracle_b128_kp(H), Fp = oracle_b128_kp(F);
+    for (int64_t r = 0; r < R; ++r)
+        if (slot[ex[r]] < 0) return -1;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < R; ++r) {
+        int64_t e = slot[ex[r]];
+        oracle_expert_fp8_b128(H, F, qup + e * F * Hp, sup + e * F * (Hp / 128), qdown + e * H * Fp,
+                               sdown + e * H * (Fp / 128), qxrow + r * Hp, sx, sh, y + r * H);
+    }
+    return 0;
+}
+
+/* ----------------------------------------------------------------------- */
 /* NVFP4 W4A4.  [B] s.2: the NVFP4 release runs the experts "W4A4".  The    */
 /* pages name the format without defining it; reading: NVIDIA's published  */
 /* NVFP4 -- E2M1 elements (magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6), one      */
