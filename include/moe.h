@@ -272,7 +272,10 @@ moe_status moe_set_stage_events(void* const* events, int32_t n);
  * value 0 launches every kernel without programmatic stream serialization
  * (each kernel then starts only after its predecessor has finished), 1 (the
  * default) lets each kernel start while its predecessor finishes and wait
- * on the device for it.  Other `what`: MOE_EINVAL. */
+ * on the device for it; what = 7: value 1 reads the shared expert's down
+ * weight through the fallback map (the plain [H][Fs] matrix, chunk j from
+ * column j*F) instead of the chunked 3-D view, 0 (the default) restores the
+ * view.  Other `what`: MOE_EINVAL. */
 moe_status moe_debug_set(int32_t what, int64_t value);
 
 #ifdef __cplusplus

@@ -84,6 +84,7 @@ std::atomic<uint64_t> g_timeout_ns{kDefaultTimeoutNs};
 std::atomic<int> g_debug_withhold{0};
 std::atomic<int> g_gemm_pair{0};
 std::atomic<int> g_pdl{1};
+std::atomic<int> g_shared_2d{0};   // 1: the shared down weight through its 2-D fallback map
 void* g_stage_events[MOE_STAGE_EVENTS] = {};
 std::atomic<int> g_stage_events_on{0};
 
@@ -346,6 +347,7 @@ moe_status check_fp8_scales(const moe_dims* d, const moe_fp8_scales* sc) {
 
 namespace moe {
 bool pdl_enabled() { return g_pdl.load() != 0; }
+bool shared_map_2d() { return g_shared_2d.load() != 0; }
 // Device context and argument checks for entry points defined in other files.
 moe_status internal_check_dims(const moe_dims* d) { return check_dims(d); }
 moe_status internal_device(DevCtx* ctx, int* num_sms) {
@@ -623,6 +625,10 @@ moe_status moe_debug_set(int32_t what, int64_t value) {
     }
     if (what == 6) {
         g_pdl.store(value ? 1 : 0);
+        return MOE_OK;
+    }
+    if (what == 7) {
+        g_shared_2d.store(value ? 1 : 0);
         return MOE_OK;
     }
     if (what == 5) {

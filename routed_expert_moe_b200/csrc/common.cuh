@@ -249,6 +249,7 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
 // Host: launch `kernel` on `stream`, marked for programmatic stream
 // serialization unless that is switched off (moe_debug_set what = 6).
 bool pdl_enabled();
+bool shared_map_2d();   // test hook: read the shared down weight through the 2-D fallback map
 template <typename... KArgs, typename... Args>
 cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
                      Args&&... args) {

@@ -424,7 +424,7 @@ cudaError_t launch_grouped_gemm(bool fp8, bool up, const void* W, int E, int Nou
         if (fp8 || !Ws) return cudaErrorInvalidValue;
         bool ok = up ? make_map(&maps.s128, Ws, (int64_t)n_shared * Nout, Kdim, false, 128) &&
                            make_map(&maps.s64, Ws, (int64_t)n_shared * Nout, Kdim, false, 64)
-                     : make_map_chunks(&maps.s128, Ws, Nout, Kdim, n_shared, 128) &&
+                     : !shared_map_2d() && make_map_chunks(&maps.s128, Ws, Nout, Kdim, n_shared, 128) &&
                            make_map_chunks(&maps.s64, Ws, Nout, Kdim, n_shared, 64);
         if (!ok && !up) {
             // a driver that refuses the chunked view: the plain [H][n * F] matrix as {n * F, H, 1},

@@ -1,0 +1,77 @@
+"""Host-side arithmetic of the benchmark: the dominant kernel's algorithmic
+bytes and flops per launch for each expert precision (the roofline's
+numerator), the bound it is reported against, and the rule that committed
+ncu traffic is used only while the kernel sources still hash to the capture's.
+No GPU: these are the formulas, checked against sums written out here.
+"""
+import json
+
+import pytest
+
+import bench
+from synth import workloads as W
+
+PEAKS = {"hbm_gbs": 6500.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}
+H, F = 2688, 1856
+
+
+def entry(cfg, touched, up_ms, down_ms, workload):
+    return bench.roofline_entry(W.WORKLOADS[cfg], {"up_gemm": up_ms, "down_gemm": down_ms}, touched, PEAKS,
+                                "measured", workload)
+
+
+def test_decode_bf16_bytes_and_hbm_bound():
+    r = entry(1, 121, 0.2, 0.1, "decode")
+    rows = 64 * 6
+    assert r["kernel"] == "up_gemm" and r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert r["algorithmic_bytes_per_launch"] == 121 * F * H * 2 + rows * H * 2 + rows * F * 2
+    assert r["algorithmic_flops_per_launch"] == 2.0 * rows * F * H
+    assert r["achieved"] == pytest.approx(r["algorithmic_bytes_per_launch"] / 0.2e-3 / 1e9)
+    assert r["frac"] == pytest.approx(r["achieved"] / PEAKS["hbm_gbs"])
+
+
+def test_down_projection_is_picked_when_slower():
+    r = entry(1, 121, 0.1, 0.2, "decode")
+    rows = 64 * 6
+    assert r["kernel"] == "down_gemm"
+    assert r["algorithmic_bytes_per_launch"] == 121 * F * H * 2 + rows * F * 2 + rows * H * 2
+
+
+def test_shared_expert_adds_one_expert_of_weights_and_T_rows():
+    base = entry(1, 121, 0.2, 0.1, "decode")
+    sh = entry(7, 121, 0.2, 0.1, "decode_shared")
+    assert sh["algorithmic_bytes_per_launch"] - base["algorithmic_bytes_per_launch"] == F * H * 2 + 64 * (H + F) * 2
+    assert sh["algorithmic_flops_per_launch"] == 2.0 * 64 * 7 * F * H
+
+
+def test_nvfp4_bytes_count_half_byte_codes_and_padded_block_scales():
+    r = entry(5, 121, 0.3, 0.2, "decode_nvfp4")
+    rows = 64 * 6
+    ksp_h, ksp_f = 176, 128          # 2688/16 = 168 -> 176;  1856/16 = 116 -> 128
+    assert r["algorithmic_bytes_per_launch"] == (121 * F * (H // 2 + ksp_h) + rows * (H // 2 + ksp_h)
+                                                 + rows * (F // 2 + ksp_f))
+
+
+def test_prefill_is_reported_against_the_sustained_tensor_peak():
+    r = entry(2, 128, 0.3, 0.31, "prefill")
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s" and r["kernel"] == "down_gemm"
+    assert r["achieved"] == pytest.approx(2.0 * 4096 * 6 * F * H / 0.31e-3 / 1e12)
+    assert r["peak"] == PEAKS["bf16_tflops_sustained"]
+    fp8 = entry(4, 128, 0.3, 0.31, "chain")
+    assert fp8["peak"] == 2 * PEAKS["bf16_tflops_sustained"]      # fp8 dense = 2x bf16 (nominal ratio)
+
+
+def test_traffic_is_used_only_while_the_sources_match(tmp_path, monkeypatch):
+    csrc = tmp_path / "routed_expert_moe_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "a.cu").write_text("kernel v1")
+    (tmp_path / "profiles").mkdir()
+    import hashlib
+    sha = hashlib.sha256(b"kernel v1").hexdigest()
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(
+        {"up_gemm@decode": {"dram_bytes_per_launch": 1234, "source_sha256": sha}}))
+    monkeypatch.setattr(bench, "ROOT", tmp_path)
+    assert bench.traffic_from_profile("up_gemm", "decode") == 1234
+    assert bench.traffic_from_profile("down_gemm", "decode") is None
+    (csrc / "a.cu").write_text("kernel v2")
+    assert bench.traffic_from_profile("up_gemm", "decode") is None

@@ -32,7 +32,8 @@ SMALL = [with_shared(W.WORKLOADS[0], 128), with_shared(W.WORKLOADS[0], 256),
          with_shared(W.Workload("ragged_T37_E16_K4", 37, 512, 16, 4, 192, seed=11), 576),
          with_shared(W.Workload("T1", 1, 2688, 128, 6, 1856, seed=12), 1856),
          with_shared(W.Workload("odd_F_tail_H272_F208", 21, 272, 8, 3, 208, seed=14), 416),
-         with_shared(W.Workload("K10_three_chunks", 40, 256, 16, 10, 64, seed=15), 192)]
+         with_shared(W.Workload("K10_three_chunks", 40, 256, 16, 10, 64, seed=15), 192),
+         with_shared(W.Workload("K12_four_chunks", 33, 256, 16, 12, 64, seed=16), 256)]   # K + Fs/F = 16
 
 
 def run_forward(moe, w, h, su, sd, residual=None):
@@ -59,6 +60,23 @@ def test_shared_forward_parity_small(moe, w):
     assert rel_err(host_f64(out), r["out"]) <= BF16_TOL
     if res is None:   # the shared expert is not negligible here: the check would fail without it
         assert rel_err(r["out"] - r["y_shared"], r["out"]) > 5 * BF16_TOL
+
+
+@pytest.mark.parametrize("w", [SMALL[1], SMALL[4], SMALL[5]], ids=lambda w: w.name)
+def test_shared_down_weight_through_the_fallback_map(moe, w):
+    """The plain [H][Fs] map, chunk j from column j*F: a K tail (F = 208) reads the next chunk's
+    weights against activation columns that read as zero."""
+    h = inputs(w)
+    h["wu_d"], h["wd_d"] = dev_bf16(h["wu"]), dev_bf16(h["wd"])
+    su, sd = W.host_w_up_shared(w), W.host_w_down_shared(w)
+    moe.debug_set(7, 1)
+    try:
+        out, idx = run_forward(moe, w, h, dev_bf16(su), dev_bf16(sd))
+    finally:
+        moe.debug_set(7, 0)
+    r = oracle.moe_layer_bf16(h["x"], h["wr"], h["bias"], h["wu"], h["wd"], w.K, shared=(su, sd))
+    assert np.array_equal(idx.cpu().numpy(), r["idx"])
+    assert rel_err(host_f64(out), r["out"]) <= BF16_TOL
 
 
 def test_expert_ffn_writes_each_shared_chunk_to_its_rows(moe):
