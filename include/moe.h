@@ -181,6 +181,19 @@ moe_status moe_forward(const moe_dims* d, const void* x, const void* w_router, c
                        const void* residual, void* out, int32_t* topk_idx, float* topk_w,
                        void* ws, size_t ws_bytes, void* stream);
 
+/* Row gather: out[r] = x[perm_src[r] / K] for r < rows, rows of H bf16 values
+ * (16-byte aligned).  This is the step moe_expert_ffn applies to the token
+ * rows before the up projection, exposed for callers that move rows between
+ * devices themselves (an expert-parallel exchange: the rows a rank sends to
+ * the experts' owners, and the owners' outputs back in the order received).
+ *   x [src_rows][H], perm_src [rows] int32 (K = 1: a plain row index),
+ *   out [rows][H].  An index outside [0, src_rows * K) sets MOE_EINDEX in
+ *   the device error word and leaves that row unwritten.  H a multiple of 8.
+ * Cited: audio.cpp model page, "CPU weight offload" (grouped expert matrix
+ * multiplication). */
+moe_status moe_gather_rows(int64_t rows, int64_t src_rows, int32_t H, int32_t K, const void* x,
+                           const int32_t* perm_src, void* out, void* stream);
+
 /* Per-tensor E4M3 quantisation of n_tensors bf16 tensors of tensor_elems
  * elements each (an expert bank): scale[i] = amax|W_i| / 448 (1 for an
  * all-zero tensor), codes = e4m3_rne_satfinite(W / scale[i]).

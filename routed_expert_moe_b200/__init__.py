@@ -53,6 +53,8 @@ _SIG = {
     "moe_combine": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P]),
     "moe_forward": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P, _P, ctypes.POINTER(MoeFp8Scales), _P, _P,
                                    _P, _P, _P, _S, _P]),
+    "moe_gather_rows": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, _P, _P,
+                                       _P, _P]),
     "moe_quantize_fp8": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int64, _P, _P, _P, _P]),
     "moe_quantize_nvfp4": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, _P, _P, _P, _P, _P]),
     "moe_rmsnorm": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int32, ctypes.c_float, _P, _P, _P]),
@@ -187,6 +189,13 @@ def forward(d, x, w_router, bias, w_up, w_down, out, ws, scales=None, residual=N
     _check(_lib.moe_forward(ctypes.byref(d), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(w_up), _ptr(w_down),
                             _ptr(su), _ptr(sd), sp, _ptr(residual), _ptr(out), _ptr(topk_idx), _ptr(topk_w),
                             _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)), "moe_forward")
+
+
+def gather_rows(x, perm_src, out, K=1, stream=None):
+    """out[r] = x[perm_src[r] // K] for the rows of out (bf16 rows of x [src_rows, H])."""
+    rows, H = out.shape[0], x.shape[1]
+    _check(_lib.moe_gather_rows(rows, x.shape[0], H, int(K), _ptr(x), _ptr(perm_src), _ptr(out), _stream(stream)),
+           "moe_gather_rows")
 
 
 def quantize_fp8(src, codes, scales, stream=None):

@@ -514,6 +514,18 @@ moe_status moe_forward(const moe_dims* d, const void* x, const void* w_router, c
     return cuda_status(e);
 }
 
+moe_status moe_gather_rows(int64_t rows, int64_t src_rows, int32_t H, int32_t K, const void* x,
+                           const int32_t* perm_src, void* out, void* stream) {
+    if (rows < 0 || src_rows < 0 || K < 1 || H < 8 || H % 8 != 0 || rows >= ((int64_t)1 << 31)) return MOE_EINVAL;
+    if (rows == 0) return MOE_OK;
+    if (!x || !perm_src || !out || !aligned(x, 16) || !aligned(out, 16)) return MOE_EINVAL;
+    DeviceInfo* dev = nullptr;
+    moe_status s = device_setup(&dev);
+    if (s != MOE_OK) return s;
+    return cuda_status(launch_gather(static_cast<const uint16_t*>(x), perm_src, rows, rows, K, src_rows, H, out,
+                                     false, 1.0f, dev->num_sms, make_ctx(dev), static_cast<cudaStream_t>(stream)));
+}
+
 moe_status moe_quantize_fp8(int64_t n_tensors, int64_t tensor_elems, const void* src, uint8_t* codes,
                             float* scales, void* stream) {
     if (n_tensors < 0 || tensor_elems < 0 || n_tensors > ((int64_t)1 << 31)) return MOE_EINVAL;

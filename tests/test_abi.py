@@ -86,6 +86,11 @@ def test_null_and_missing_arguments(moe):
     assert lib.moe_rmsnorm(4, 2690, 1e-5, None, None, None) == moe.MOE_EINVAL
     assert lib.moe_quantize_fp8(-1, 4, None, None, None, None) == moe.MOE_EINVAL
     assert lib.moe_debug_set(99, 0) == moe.MOE_EINVAL
+    assert lib.moe_gather_rows(-1, 4, 256, 1, None, None, None, None) == moe.MOE_EINVAL
+    assert lib.moe_gather_rows(4, 4, 260, 1, None, None, None, None) == moe.MOE_EINVAL   # H % 8
+    assert lib.moe_gather_rows(4, 4, 256, 0, None, None, None, None) == moe.MOE_EINVAL   # K < 1
+    assert lib.moe_gather_rows(4, 4, 256, 1, None, None, None, None) == moe.MOE_EINVAL   # null buffers
+    assert lib.moe_gather_rows(0, 0, 256, 1, None, None, None, None) == moe.MOE_OK
     assert lib.moe_set_stage_events(None, 3) == moe.MOE_EINVAL
 
 
