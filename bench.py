@@ -354,8 +354,23 @@ def e2e_loop(layer, steps, warmup):
     return ms, nb, nb
 
 
+# the sources that decide what the grouped GEMM kernel runs and reads: its own
+# file, the shared device helpers, and the permutation that writes its schedule
+TRAFFIC_SOURCES = ("routed_expert_moe_b200/csrc/grouped_gemm.cu", "routed_expert_moe_b200/csrc/common.cuh",
+                   "routed_expert_moe_b200/csrc/permute.cu")
+
+
+def sources_sha256(paths) -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for rel in paths:
+        h.update((ROOT / rel).read_bytes())
+    return h.hexdigest()
+
+
 def traffic_from_profile(kernel: str, workload: str):
-    """DRAM bytes per launch from the committed ncu summary, if it matches this build."""
+    """DRAM bytes per launch from the committed ncu summary, if the kernel's sources still hash
+    to those of the captured build."""
     p = ROOT / "profiles" / "traffic.json"
     if not p.exists():
         return None
@@ -366,11 +381,11 @@ def traffic_from_profile(kernel: str, workload: str):
     ent = d.get(f"{kernel}@{workload}")
     if not ent:
         return None
-    import hashlib
-    h = hashlib.sha256()
-    for f in sorted((ROOT / "routed_expert_moe_b200" / "csrc").glob("*.cu*")):
-        h.update(f.read_bytes())
-    if ent.get("source_sha256") != h.hexdigest():
+    srcs = ent.get("sources", TRAFFIC_SOURCES)
+    try:
+        if ent.get("source_sha256") != sources_sha256(srcs):
+            return None
+    except OSError:
         return None
     return ent.get("dram_bytes_per_launch")
 

@@ -68,10 +68,14 @@ def test_traffic_is_used_only_while_the_sources_match(tmp_path, monkeypatch):
     (tmp_path / "profiles").mkdir()
     import hashlib
     sha = hashlib.sha256(b"kernel v1").hexdigest()
+    (csrc / "b.cu").write_text("another kernel")
     (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(
-        {"up_gemm@decode": {"dram_bytes_per_launch": 1234, "source_sha256": sha}}))
+        {"up_gemm@decode": {"dram_bytes_per_launch": 1234, "source_sha256": sha,
+                            "sources": ["routed_expert_moe_b200/csrc/a.cu"]}}))
     monkeypatch.setattr(bench, "ROOT", tmp_path)
     assert bench.traffic_from_profile("up_gemm", "decode") == 1234
     assert bench.traffic_from_profile("down_gemm", "decode") is None
+    (csrc / "b.cu").write_text("a file the captured kernel does not use")
+    assert bench.traffic_from_profile("up_gemm", "decode") == 1234
     (csrc / "a.cu").write_text("kernel v2")
     assert bench.traffic_from_profile("up_gemm", "decode") is None
