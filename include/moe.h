@@ -60,7 +60,8 @@ typedef enum {
 typedef enum {
     MOE_BF16 = 0,          /* expert banks and expert activations in bf16 */
     MOE_FP8_E4M3 = 1,      /* W8A8: expert banks and expert activations in E4M3 codes */
-    MOE_NVFP4 = 2          /* W4A4: expert banks and expert activations in NVFP4 (see below) */
+    MOE_NVFP4 = 2,         /* W4A4: expert banks and expert activations in NVFP4 (see below) */
+    MOE_FP8_B128 = 3       /* W8A8: E4M3 banks with one fp32 scale per 128 values along K (see below) */
 } moe_dtype;
 
 /* Problem size.  Limits: 0 <= T, T*K < 2^31; 1 <= E <= 256; 1 <= K <= min(E, 16);
@@ -99,6 +100,11 @@ typedef struct {
  * w_down_block [E][H][KSP(F)].  x and the ReLU^2 tensor are quantised inside
  * the layer with block scales taken at run time and the static tensor scales
  * x_scale and h_scale. */
+/* Scales of the quantised expert formats.  MOE_FP8_E4M3 and MOE_NVFP4: one
+ * tensor scale per expert tensor.  MOE_FP8_B128: w_up_scale [E][F][Kp(H)/128]
+ * and w_down_scale [E][H][Kp(F)/128], one per block of 128 values along K,
+ * with the banks' codes [E][F][Kp(H)] and [E][H][Kp(F)], Kp(K) = 128*ceil(K/128)
+ * (zero codes past K).  Activation scales are static in every format. */
 typedef struct {
     const float* w_up_scale;    /* [E] device: one (tensor) scale per expert up tensor */
     const float* w_down_scale;  /* [E] device: one (tensor) scale per expert down tensor */
@@ -211,6 +217,17 @@ moe_status moe_quantize_fp8(int64_t n_tensors, int64_t tensor_elems, const void*
  * E4M3 W8A8"). */
 moe_status moe_quantize_act_fp8(int64_t rows, int32_t H, float x_scale, const void* x, uint8_t* codes,
                                 void* stream);
+
+/* FP8_B128 quantisation of n_tensors bf16 tensors [rows][K] (an expert bank):
+ * per row and block of 128 values along K, scale = amax|block| / 448 (an fp32
+ * division; 1 for an all-zero block), codes e4m3(fl32(W / scale)) nearest-even
+ * and saturating; K is padded to Kp = 128*ceil(K/128) with zero codes.
+ *   src [n_tensors][rows][K] bf16; codes [n_tensors][rows][Kp];
+ *   scales [n_tensors][rows][Kp/128] fp32.  K a multiple of 16.
+ * Cited: bloomery page s.3 ("Kernel dispatch": FP8_B128 with the 64-value
+ * tail of K = 1856). */
+moe_status moe_quantize_fp8_b128(int64_t n_tensors, int64_t rows, int32_t K, const void* src, uint8_t* codes,
+                                 float* scales, void* stream);
 
 /* NVFP4 quantisation of n_tensors bf16 tensors [rows][K] (an expert bank):
  * tensor scale t[i] = amax|W_i| / 2688 (1 for an all-zero tensor), per block

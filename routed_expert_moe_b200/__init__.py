@@ -15,7 +15,7 @@ from pathlib import Path
 _LIB_PATH = Path(__file__).resolve().parent / "_lib" / "libmoe_b200.so"
 
 MOE_OK, MOE_EINVAL, MOE_EUNSUPPORTED, MOE_ECUDA, MOE_ETIMEOUT, MOE_EWORKSPACE, MOE_ERANGE, MOE_EINDEX = range(8)
-MOE_BF16, MOE_FP8_E4M3, MOE_NVFP4 = 0, 1, 2
+MOE_BF16, MOE_FP8_E4M3, MOE_NVFP4, MOE_FP8_B128 = 0, 1, 2, 3
 
 if not _LIB_PATH.exists():
     raise ImportError(
@@ -57,6 +57,7 @@ _SIG = {
                                        _P, _P]),
     "moe_quantize_fp8": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int64, _P, _P, _P, _P]),
     "moe_quantize_nvfp4": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, _P, _P, _P, _P, _P]),
+    "moe_quantize_fp8_b128": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, _P, _P, _P, _P]),
     "moe_rmsnorm": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int32, ctypes.c_float, _P, _P, _P]),
     "moe_quantize_act_fp8": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int32, ctypes.c_float, _P, _P, _P]),
     "moe_quantize_act_nvfp4": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int32, ctypes.c_float, _P, _P, _P, _P]),
@@ -109,9 +110,9 @@ def _stream(stream):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-def dims(T, H, E, K, F, fp8=False, nvfp4=False, Fs=0) -> MoeDims:
+def dims(T, H, E, K, F, fp8=False, nvfp4=False, Fs=0, fp8_b128=False) -> MoeDims:
     """Problem size; Fs is the width of the shared expert (0: none, else a multiple of F)."""
-    dt = MOE_NVFP4 if nvfp4 else (MOE_FP8_E4M3 if fp8 else MOE_BF16)
+    dt = MOE_NVFP4 if nvfp4 else MOE_FP8_B128 if fp8_b128 else (MOE_FP8_E4M3 if fp8 else MOE_BF16)
     return MoeDims(int(T), int(H), int(E), int(K), int(F), dt, int(Fs))
 
 
@@ -139,6 +140,19 @@ def nvfp4_scales(w_up_tscale, w_down_tscale, x_scale: float, h_scale: float, w_u
 def nvfp4_scale_row(K: int) -> int:
     """Bytes of one block-scale row: K/16 rounded up to a multiple of 16."""
     return (K // 16 + 15) // 16 * 16
+
+
+def b128_kp(K: int) -> int:
+    """K padded to whole blocks of 128 (the FP8_B128 banks' row length)."""
+    return (K + 127) // 128 * 128
+
+
+def quantize_fp8_b128(src, codes, scales, stream=None):
+    """FP8_B128 quantisation of a bank src [n, rows, K] (bf16): codes [n, rows, b128_kp(K)] (uint8),
+    scales [n, rows, b128_kp(K) / 128] (fp32)."""
+    n, rows, K = src.shape
+    _check(_lib.moe_quantize_fp8_b128(n, rows, K, _ptr(src), _ptr(codes), _ptr(scales), _stream(stream)),
+           "moe_quantize_fp8_b128")
 
 
 def quantize_nvfp4(src, codes, block, tscale, stream=None):

@@ -62,6 +62,12 @@ cudaError_t launch_gather_nvfp4(const uint16_t* x, const int32_t* perm_src, int6
                                 float s_t, uint8_t* codes, uint8_t* bscale, int num_sms, const DevCtx& ctx,
                                 cudaStream_t stream);
 size_t nvfp4_scale_row_bytes(int K);
+cudaError_t launch_grouped_gemm_b128(bool up, const uint8_t* W, const float* w_scale, int E, int Nout, int Kdim,
+                                     const uint8_t* act, int64_t rows, const int4* sched, const int* n_sched, int bn,
+                                     int max_sched, void* out, float in_scale, float out_scale, int num_sms,
+                                     int debug_withhold, const DevCtx& ctx, cudaStream_t stream);
+cudaError_t launch_quantize_fp8_b128(int64_t rows, int K, const uint16_t* src, uint8_t* codes, float* scales,
+                                     int num_sms, cudaStream_t stream);
 cudaError_t launch_combine(const uint16_t* yp, const int32_t* inv_row, const float* w, const uint16_t* residual,
                            uint16_t* out, int64_t T, int K, int ns, int H, int num_sms, const DevCtx& ctx,
                            cudaStream_t stream);
@@ -137,7 +143,8 @@ moe_status check_dims(const moe_dims* d) {
     if (d->H < 16 || d->H > 65536 || d->H % 16 != 0) return MOE_EINVAL;
     if (d->F < 16 || d->F > 65536 || d->F % 16 != 0) return MOE_EINVAL;
     if (d->T * (int64_t)d->K >= (int64_t)1 << 31) return MOE_EINVAL;
-    if (d->expert_dtype != MOE_BF16 && d->expert_dtype != MOE_FP8_E4M3 && d->expert_dtype != MOE_NVFP4)
+    if (d->expert_dtype != MOE_BF16 && d->expert_dtype != MOE_FP8_E4M3 && d->expert_dtype != MOE_NVFP4 &&
+        d->expert_dtype != MOE_FP8_B128)
         return MOE_EINVAL;
     if (d->expert_dtype == MOE_NVFP4 && (d->H % 32 != 0 || d->F % 32 != 0)) return MOE_EINVAL;
     // shared expert: chunks of the routed width, each an extra term of the combine
@@ -197,10 +204,18 @@ struct ForwardWs {
     void* y_perm;
 };
 
-// Plan of the expert FFN: one tile schedule for every expert dtype, plus the
-// shared expert's entries (ns chunks of T rows, cut into tiles of at most bn).
+// Plan of the expert FFN: one tile schedule for every expert dtype (FP8_B128
+// caps a tile at 64 token rows: its epilogue keeps a tile's sums in registers),
+// plus the shared expert's entries (ns chunks of T rows, cut into tiles of at
+// most bn).
 GemmPlan ffn_plan(const moe_dims* d) {
     GemmPlan gp = gemm_plan(d->T, d->K, d->E);
+    if (d->expert_dtype == MOE_FP8_B128 && gp.bn > 64) {
+        const int64_t rows = d->T * d->K;
+        const int64_t nonempty = d->E < rows ? d->E : rows;
+        gp.bn = 64;
+        gp.max_sched = (int)(nonempty + (rows + 63) / 64);
+    }
     gp.max_sched += n_shared(d) * (int)((d->T + gp.bn - 1) / gp.bn);
     return gp;
 }
@@ -227,7 +242,7 @@ FfnWs carve_ffn(Carve& c, void* base, const moe_dims* d, const GemmPlan& gp) {
         f.hb_block = c.take<uint8_t>(base, rows * nvfp4_scale_row_bytes(d->F));
         return f;
     }
-    const size_t es = d->expert_dtype == MOE_FP8_E4M3 ? 1 : 2;
+    const size_t es = (d->expert_dtype == MOE_FP8_E4M3 || d->expert_dtype == MOE_FP8_B128) ? 1 : 2;
     f.xp = c.take<uint8_t>(base, rows * d->H * es);
     f.hb = c.take<uint8_t>(base, rows * d->F * es);
     return f;
@@ -272,9 +287,26 @@ moe_status run_ffn(const moe_dims* d, const DeviceInfo* dev, const DevCtx& ctx, 
                    const void* x, const int32_t* perm_src, const void* w_up, const void* w_down,
                    const void* w_up_s, const void* w_down_s, const moe_fp8_scales* sc, FfnWs& fw, void* y_perm,
                    cudaStream_t st, bool marks = false) {
-    const bool fp8 = d->expert_dtype == MOE_FP8_E4M3;
+    const bool fp8 = d->expert_dtype == MOE_FP8_E4M3 || d->expert_dtype == MOE_FP8_B128;
     const int64_t rows = ffn_rows(d);
     const int ns = n_shared(d);
+    if (d->expert_dtype == MOE_FP8_B128) {
+        const int withhold_b = g_debug_withhold.load();
+        if (marks) stage_mark(3, st);
+        cudaError_t eb = launch_gather(static_cast<const uint16_t*>(x), perm_src, rows, rows, d->K, d->T, d->H,
+                                       fw.xp, true, sc->x_scale, dev->num_sms, ctx, st);
+        if (eb != cudaSuccess) return cuda_status(eb);
+        if (marks) stage_mark(4, st);
+        eb = launch_grouped_gemm_b128(true, static_cast<const uint8_t*>(w_up), sc->w_up_scale, d->E, d->F, d->H,
+                                      static_cast<const uint8_t*>(fw.xp), rows, fw.sched, fw.n_sched, gp.bn,
+                                      gp.max_sched, fw.hb, sc->x_scale, sc->h_scale, dev->num_sms, withhold_b, ctx, st);
+        if (eb != cudaSuccess) return cuda_status(eb);
+        if (marks) stage_mark(5, st);
+        eb = launch_grouped_gemm_b128(false, static_cast<const uint8_t*>(w_down), sc->w_down_scale, d->E, d->H, d->F,
+                                      static_cast<const uint8_t*>(fw.hb), rows, fw.sched, fw.n_sched, gp.bn,
+                                      gp.max_sched, y_perm, sc->h_scale, 1.0f, dev->num_sms, 0, ctx, st);
+        return cuda_status(eb);
+    }
     if (d->expert_dtype == MOE_NVFP4) {
         const int withhold4 = g_debug_withhold.load();
         if (marks) stage_mark(3, st);
@@ -536,6 +568,18 @@ moe_status moe_quantize_fp8(int64_t n_tensors, int64_t tensor_elems, const void*
     if (s != MOE_OK) return s;
     return cuda_status(launch_quantize(n_tensors, tensor_elems, static_cast<const uint16_t*>(src), codes, scales,
                                        dev->num_sms, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_quantize_fp8_b128(int64_t n_tensors, int64_t rows, int32_t K, const void* src, uint8_t* codes,
+                                 float* scales, void* stream) {
+    if (n_tensors < 0 || rows < 0 || K < 16 || K > 65536 || K % 16 != 0) return MOE_EINVAL;
+    if (n_tensors == 0 || rows == 0) return MOE_OK;
+    if (!src || !codes || !scales || !aligned(codes, 4) || !aligned(scales, 4)) return MOE_EINVAL;
+    DeviceInfo* dev = nullptr;
+    moe_status s = device_setup(&dev);
+    if (s != MOE_OK) return s;
+    return cuda_status(launch_quantize_fp8_b128(n_tensors * rows, K, static_cast<const uint16_t*>(src), codes, scales,
+                                                dev->num_sms, static_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_quantize_nvfp4(int64_t n_tensors, int64_t rows, int32_t K, const void* src, uint8_t* codes,

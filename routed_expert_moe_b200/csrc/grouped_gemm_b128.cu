@@ -1,0 +1,390 @@
+// FP8_B128 W8A8 grouped expert GEMMs (bloomery issue page, s.3 "Kernel
+// dispatch" and the FP8 release: FP8_B128 scales, the 64-value tail of
+// K = 1856, physical K 1920).  The weights are E4M3 codes with one fp32
+// scale per block of 128 values along K of each row (K padded with zero codes
+// to Kp = 128 * ceil(K / 128)); the activations are E4M3 codes with one static
+// scale per tensor.  For a weight row f and a token row r,
+//   z[r, f] = s_act * sum_b s_w[f, b] * sum_{k in block b} q_w[f, k] q_act[r, k],
+// followed by ReLU^2 and the E4M3 requantisation of H (up) or the bf16 output
+// (down), as in the scalar-scale path.
+//
+// Same swap-AB orientation, schedule and TMA ring as the bf16 / E4M3 kernel:
+// a 128-row weight block is the MMA's M side, the expert's token rows (at most
+// 64 per schedule entry here) its N side.  A 128-byte K stage of E4M3 values
+// is exactly one scale block, so every stage's product goes to its own TMEM
+// partial (one of four slots of 64 columns): the MMA overwrites the slot with
+// the block's sum, and the epilogue warps, which hold the running fp32 sums
+// of their weight row in registers, add s_w[f, b] times the partial and free
+// the slot.  Roles (192 threads): warp 0 TMA producer, warp 1 MMA, warps 2..5
+// the partial sums and the epilogue.  Every wait is bounded.
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int GB_THREADS = 192;
+constexpr int GB_BM = 128;                  // weight rows per unit
+constexpr int GB_ROW = 128;                 // bytes = E4M3 values of one K stage = one scale block
+constexpr int GB_A_BYTES = GB_BM * GB_ROW;  // 16 KB
+constexpr int GB_BN = 64;                   // token rows per schedule entry at most
+constexpr int GB_NP = 4;                    // TMEM partial slots of GB_BN columns
+constexpr int GB_TMEM_COLS = GB_NP * GB_BN;
+
+struct B128Maps {
+    CUtensorMap a128;   // weight codes [E * Nout][Kp], 128-row box
+    CUtensorMap a64;    // 64-row box
+    CUtensorMap b64;    // activation codes [rows][K], 64-row box
+    CUtensorMap b16;    // 16-row box
+};
+
+struct B128Args {
+    const int4* sched;     // {e, row0, nrows, 0}, nrows <= GB_BN
+    const int* n_sched;
+    int m_blocks;          // ceil(Nout / 128)
+    int Nout;
+    int k_stages;          // Kp / 128 = scale blocks per weight row
+    int n_stages;          // smem ring depth
+    int b_stage_bytes;     // bn * 128
+    void* out;             // up: e4m3 codes [rows][Nout]; down: bf16 [rows][Nout]
+    int64_t out_ld;
+    const float* w_scale;  // [E][Nout][k_stages]
+    float in_scale;        // x_scale (up) or h_scale (down)
+    float out_scale;       // h_scale (up)
+    int debug_withhold;
+};
+
+template <bool UP>
+__global__ void __launch_bounds__(GB_THREADS, 1)
+    grouped_gemm_b128_kernel(const __grid_constant__ B128Maps maps, B128Args g, DevCtx ctx) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    const int NS = g.n_stages;
+    uint8_t* smA = smem;
+    uint8_t* smB = smA + (size_t)NS * GB_A_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smB + (size_t)NS * g.b_stage_bytes);
+    uint64_t* full = bars;
+    uint64_t* empty = bars + NS;
+    uint64_t* pfull = bars + 2 * NS;
+    uint64_t* pempty = pfull + GB_NP;
+    uint64_t* drain = pempty + GB_NP;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(drain + 1);
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1) + 1;
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(smem_u32(&full[s]), 1);
+            mbar_init(smem_u32(&empty[s]), 1);
+        }
+        for (int p = 0; p < GB_NP; ++p) {
+            mbar_init(smem_u32(&pfull[p]), 1);
+            mbar_init(smem_u32(&pempty[p]), 128);
+        }
+        mbar_init(smem_u32(drain), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&maps.a128);
+        tma_prefetch_desc(&maps.a64);
+        tma_prefetch_desc(&maps.b64);
+        tma_prefetch_desc(&maps.b16);
+    }
+    if (warp == 1) tmem_alloc(smem_u32(tmem_holder), GB_TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+    pdl_enter();
+
+    const int n_units = (*g.n_sched) * g.m_blocks;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            const uint64_t pol_w = l2_policy_evict_first();
+            const uint64_t pol_x = l2_policy_evict_last();
+            int stage = 0;
+            uint32_t phase = 0;
+            bool withhold = g.debug_withhold && blockIdx.x == 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+                const int4 sc = g.sched[u / g.m_blocks];
+                const int mb = u % g.m_blocks;
+                const bool a_full = g.Nout - mb * GB_BM > 64;
+                const int n16 = (sc.z + 15) / 16;   // <= 4
+                const int n64 = n16 / 4, r16 = n16 % 4;
+                const uint32_t bytes = (uint32_t)((a_full ? 128 : 64) * GB_ROW + n16 * 16 * GB_ROW);
+                const int a_y = sc.x * g.Nout + mb * GB_BM;
+                for (int ks = 0; ks < g.k_stages; ++ks) {
+                    if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, ctx, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t fb = smem_u32(&full[stage]);
+                    mbar_arrive_expect_tx(fb, bytes);
+                    if (withhold) {
+                        withhold = false;   // this stage never completes: the consumer's wait expires
+                    } else {
+                        const int kx = ks * GB_ROW;
+                        const uint32_t a_dst = smem_u32(smA + (size_t)stage * GB_A_BYTES);
+                        const uint32_t b_dst = smem_u32(smB + (size_t)stage * g.b_stage_bytes);
+                        tma_load_2d(a_dst, a_full ? &maps.a128 : &maps.a64, fb, kx, a_y, pol_w);
+                        int row = 0;
+                        for (int j = 0; j < n64; ++j, row += 64)
+                            tma_load_2d(b_dst + row * GB_ROW, &maps.b64, fb, kx, sc.y + row, pol_x);
+                        for (int j = 0; j < r16; ++j, row += 16)
+                            tma_load_2d(b_dst + row * GB_ROW, &maps.b16, fb, kx, sc.y + row, pol_x);
+                    }
+                    if (++stage == NS) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                const uint64_t t0 = globaltimer();
+                while (globaltimer() - t0 < 200000ull) __nanosleep(1000);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            int stage = 0, ps = 0;
+            uint32_t phase = 0, pph = 0;
+            bool ok = true, issued = false;
+            for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+                const int4 sc = g.sched[u / g.m_blocks];
+                const int n_mma = max(16, (sc.z + 15) & ~15);
+                const uint32_t idesc = make_idesc(0u, GB_BM, n_mma);
+                for (int ks = 0; ks < g.k_stages; ++ks) {
+                    if (!mbar_wait(smem_u32(&full[stage]), phase, ctx, abort_flag) ||
+                        !mbar_wait(smem_u32(&pempty[ps]), pph ^ 1u, ctx, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t d_tmem = tmem_base + (uint32_t)(ps * GB_BN);
+                    const uint32_t a_base = smem_u32(smA + (size_t)stage * GB_A_BYTES);
+                    const uint32_t b_base = smem_u32(smB + (size_t)stage * g.b_stage_bytes);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)   // 4 x K = 32: the block's sum, the slot overwritten first
+                        mma_ss<true>(d_tmem, sw128_desc(a_base + kk * 32), sw128_desc(b_base + kk * 32), idesc,
+                                     kk != 0 ? 1u : 0u);
+                    issued = true;
+                    mma_commit(smem_u32(&empty[stage]));
+                    mma_commit(smem_u32(&pfull[ps]));
+                    if (++stage == NS) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                    if (++ps == GB_NP) {
+                        ps = 0;
+                        pph ^= 1u;
+                    }
+                }
+            }
+            if (!ok && issued) {
+                mma_commit(smem_u32(drain));
+                mbar_wait_drain(smem_u32(drain), 0, ctx.timeout_ns);
+            }
+        }
+    } else {
+        const int q = warp & 3;   // TMEM lane quadrant of this warp
+        int ps = 0;
+        uint32_t pph = 0;
+        bool ok = true;
+        const float inv_out = UP ? __frcp_rn(g.out_scale) : 1.0f;
+        for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+            const int4 sc = g.sched[u / g.m_blocks];
+            const int mb = u % g.m_blocks;
+            const int f = mb * GB_BM + q * 32 + lane;
+            const bool fvalid = f < g.Nout;
+            const int nch = (sc.z + 15) / 16;   // warp-uniform, <= 4
+            const float* wrow = g.w_scale + ((int64_t)sc.x * g.Nout + (fvalid ? f : 0)) * g.k_stages;
+            float acc[GB_BN];
+#pragma unroll
+            for (int i = 0; i < GB_BN; ++i) acc[i] = 0.0f;
+            for (int ks = 0; ks < g.k_stages; ++ks) {
+                if (!mbar_wait_warp(smem_u32(&pfull[ps]), pph, ctx, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const float sw = wrow[ks];
+                const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(ps * GB_BN);
+#pragma unroll
+                for (int c = 0; c < GB_BN / 16; ++c) {
+                    if (c < nch) {
+                        uint32_t v[16];
+                        tmem_ld16(t_row + (uint32_t)(c * 16), v);
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) acc[c * 16 + j] = __fmaf_rn(sw, __uint_as_float(v[j]), acc[c * 16 + j]);
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(smem_u32(&pempty[ps]));
+                if (++ps == GB_NP) {
+                    ps = 0;
+                    pph ^= 1u;
+                }
+            }
+            if (!ok) break;
+            if (fvalid) {
+#pragma unroll
+                for (int c = 0; c < GB_BN / 16; ++c) {
+                    if (c >= nch) break;
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int r = c * 16 + j;
+                        if (r < sc.z) {
+                            const float z = __fmul_rn(acc[r], g.in_scale);
+                            const int64_t o = (int64_t)(sc.y + r) * g.out_ld + f;
+                            if constexpr (UP) {
+                                const float a = z > 0.0f ? __fmul_rn(z, z) : 0.0f;
+                                static_cast<uint8_t*>(g.out)[o] =
+                                    (uint8_t)__nv_cvt_float_to_fp8(__fmul_rn(a, inv_out), __NV_SATFINITE, __NV_E4M3);
+                            } else {
+                                static_cast<__nv_bfloat16*>(g.out)[o] = __float2bfloat16_rn(z);
+                            }
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, GB_TMEM_COLS);
+    }
+}
+
+// One warp per (row, block of 128): scale amax / 448 (1 for a zero block),
+// codes e4m3(fl32(w / scale)) nearest-even and saturating, zero past K.
+__global__ void quantize_fp8_b128_kernel(const uint16_t* __restrict__ src, int64_t rows, int K, int Kp,
+                                         uint8_t* __restrict__ codes, float* __restrict__ scales) {
+    const int nb = Kp / 128;
+    const int lane = threadIdx.x % 32;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x / 32);
+    for (int64_t item = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32; item < rows * nb;
+         item += warps) {
+        const int64_t r = item / nb;
+        const int k0 = (int)(item % nb) * 128 + lane * 4;
+        float v[4];
+        float amax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int k = k0 + i;
+            v[i] = k < K ? __uint_as_float((uint32_t)src[r * K + k] << 16) : 0.0f;
+            amax = fmaxf(amax, fabsf(v[i]));
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+        const float s = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+        uint32_t packed = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t c = k0 + i < K ? (uint32_t)__nv_cvt_float_to_fp8(__fdiv_rn(v[i], s), __NV_SATFINITE,
+                                                                             __NV_E4M3)
+                                          : 0u;
+            packed |= c << (8 * i);
+        }
+        *reinterpret_cast<uint32_t*>(codes + r * Kp + k0) = packed;
+        if (lane == 0) scales[item] = s;
+    }
+}
+
+// ----------------------------------------------------------------------------- host
+
+typedef CUresult (*EncodeTiledFnB)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFnB encode_fn_b128() {
+    static EncodeTiledFnB fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFnB>(p);
+    }
+    return fn;
+}
+
+// 2-D map over a row-major u8 [rows][cols] matrix, box 128 bytes x box_rows, 128-byte swizzle.
+static bool make_map_u8_b128(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows) {
+    EncodeTiledFnB fn = encode_fn_b128();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols};
+    cuuint32_t box[2] = {(cuuint32_t)GB_ROW, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int b128_kp(int K) { return (K + 127) / 128 * 128; }
+
+// One FP8_B128 projection.  W: codes [E * Nout][Kp], w_scale [E][Nout][Kp / 128];
+// act: E4M3 codes [rows][Kdim] in the expert layout; out [rows][Nout] (e4m3 codes
+// for the up projection, bf16 for the down).  bn <= 64 (the schedule's tile).
+cudaError_t launch_grouped_gemm_b128(bool up, const uint8_t* W, const float* w_scale, int E, int Nout, int Kdim,
+                                     const uint8_t* act, int64_t rows, const int4* sched, const int* n_sched, int bn,
+                                     int max_sched, void* out, float in_scale, float out_scale, int num_sms,
+                                     int debug_withhold, const DevCtx& ctx, cudaStream_t stream) {
+    if (rows == 0) return cudaSuccess;
+    if (bn < 16 || bn > GB_BN || bn % 16 != 0) return cudaErrorInvalidValue;
+    const int Kp = b128_kp(Kdim);
+    B128Maps maps;
+    if (!make_map_u8_b128(&maps.a128, W, (int64_t)E * Nout, Kp, 128) ||
+        !make_map_u8_b128(&maps.a64, W, (int64_t)E * Nout, Kp, 64) ||
+        !make_map_u8_b128(&maps.b64, act, rows, Kdim, 64) || !make_map_u8_b128(&maps.b16, act, rows, Kdim, 16))
+        return cudaErrorInvalidValue;
+    B128Args g;
+    g.sched = sched;
+    g.n_sched = n_sched;
+    g.m_blocks = (Nout + GB_BM - 1) / GB_BM;
+    g.Nout = Nout;
+    g.k_stages = Kp / GB_ROW;
+    g.b_stage_bytes = bn * GB_ROW;
+    const int stage = GB_A_BYTES + g.b_stage_bytes;
+    int ns = (200 * 1024) / stage;
+    if (ns > 8) ns = 8;
+    if (ns < 2) ns = 2;
+    g.n_stages = ns;
+    g.out = out;
+    g.out_ld = Nout;
+    g.w_scale = w_scale;
+    g.in_scale = in_scale;
+    g.out_scale = out_scale;
+    g.debug_withhold = debug_withhold;
+    const size_t smem = 1024 + (size_t)ns * stage + (size_t)(2 * ns + 2 * GB_NP + 1) * 8 + 16;
+    const int64_t max_units = (int64_t)max_sched * g.m_blocks;
+    const int grid = (int)(max_units < num_sms ? max_units : num_sms);
+    auto kfn = up ? grouped_gemm_b128_kernel<true> : grouped_gemm_b128_kernel<false>;
+    cudaError_t err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    return launch_k(kfn, dim3(grid), dim3(GB_THREADS), smem, stream, maps, g, ctx);
+}
+
+cudaError_t launch_quantize_fp8_b128(int64_t rows, int K, const uint16_t* src, uint8_t* codes, float* scales,
+                                     int num_sms, cudaStream_t stream) {
+    if (rows == 0) return cudaSuccess;
+    const int Kp = b128_kp(K);
+    const int64_t items = rows * (Kp / 128);
+    int64_t blocks = (items + 7) / 8;
+    const int64_t cap = (int64_t)num_sms * 16;
+    if (blocks > cap) blocks = cap;
+    quantize_fp8_b128_kernel<<<(unsigned)blocks, 256, 0, stream>>>(src, rows, K, Kp, codes, scales);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

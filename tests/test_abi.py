@@ -91,6 +91,15 @@ def test_null_and_missing_arguments(moe):
     assert lib.moe_gather_rows(4, 4, 256, 0, None, None, None, None) == moe.MOE_EINVAL   # K < 1
     assert lib.moe_gather_rows(4, 4, 256, 1, None, None, None, None) == moe.MOE_EINVAL   # null buffers
     assert lib.moe_gather_rows(0, 0, 256, 1, None, None, None, None) == moe.MOE_OK
+    assert lib.moe_quantize_fp8_b128(1, 4, 8, None, None, None, None) == moe.MOE_EINVAL      # K < 16
+    assert lib.moe_quantize_fp8_b128(1, 4, 200, None, None, None, None) == moe.MOE_EINVAL    # K % 16
+    assert lib.moe_quantize_fp8_b128(1, 4, 256, None, None, None, None) == moe.MOE_EINVAL    # null buffers
+    assert lib.moe_quantize_fp8_b128(0, 4, 256, None, None, None, None) == moe.MOE_OK
+    n = ctypes.c_size_t()
+    b128 = moe.dims(64, 2688, 128, 6, 1856, fp8_b128=True)
+    assert lib.moe_workspace_size(ctypes.byref(b128), ctypes.byref(n)) == moe.MOE_OK
+    b128s = moe.dims(64, 2688, 128, 6, 1856, fp8_b128=True, Fs=1856)
+    assert lib.moe_workspace_size(ctypes.byref(b128s), ctypes.byref(n)) == moe.MOE_EUNSUPPORTED
     assert lib.moe_set_stage_events(None, 3) == moe.MOE_EINVAL
 
 
