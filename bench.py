@@ -36,8 +36,10 @@ UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 WORKLOADS = {"tiny": 0, "decode": 1, "prefill": 2, "skewed": 3, "chain": 4, "decode_nvfp4": 5,
-             "prefill_nvfp4": 6, "decode_shared": 7, "prefill_shared": 8}
-TENSOR_BOUND = ("prefill", "chain", "prefill_nvfp4", "prefill_shared")   # reported against the tensor peak
+             "prefill_nvfp4": 6, "decode_shared": 7, "prefill_shared": 8, "decode_fp8_b128": 9,
+             "prefill_fp8_b128": 10}
+TENSOR_BOUND = ("prefill", "chain", "prefill_nvfp4", "prefill_shared",
+                "prefill_fp8_b128")   # reported against the tensor peak
 
 
 def load_peaks():
@@ -185,6 +187,21 @@ class Layer:
             (self.wu, self.bu, self.tu), (self.wd, self.bd, self.td) = banks
             sx, sh = W.nvfp4_scales(wl)
             self.scales = moe.nvfp4_scales(self.tu, self.td, float(sx), float(sh), self.bu, self.bd)
+        if wl.fp8_b128:
+            # FP8_B128 banks quantised on the device from the bf16 masters; static activation scales
+            # from the oracle's calibration (tests/golden/fp8_b128_scales.json)
+            banks = []
+            for src in (self.wu, self.wd):
+                n, rows, Kd = src.shape
+                kp = moe.b128_kp(Kd)
+                codes = torch.empty(n, rows, kp, dtype=torch.uint8, device=device)
+                sc = torch.empty(n, rows, kp // 128, dtype=torch.float32, device=device)
+                moe.quantize_fp8_b128(src, codes, sc)
+                banks.append((codes, sc))
+            torch.cuda.synchronize(device)
+            (self.wu, self.su), (self.wd, self.sd) = banks
+            sx, sh = W.fp8_b128_scales(wl)
+            self.scales = moe.fp8_scales(self.su, self.sd, float(sx), float(sh))
         self.shared = None
         if wl.shared:
             # the shared expert: W_up_s [Fs][H], W_down_s [H][Fs], bf16
@@ -195,7 +212,7 @@ class Layer:
             synth.normal_bf16_device(synth.key(wl.seed, synth.T_WDOWN_S, 0), sd.numel(), W.SIGMA_W, sd.data_ptr(),
                                      stream)
             self.shared = (su, sd)
-        self.dims = moe.dims(wl.T, wl.H, wl.E, wl.K, wl.F, nvfp4=wl.nvfp4, Fs=wl.shared)
+        self.dims = moe.dims(wl.T, wl.H, wl.E, wl.K, wl.F, nvfp4=wl.nvfp4, Fs=wl.shared, fp8_b128=wl.fp8_b128)
         self.ws = moe.alloc_workspace(self.dims, device)
         self.out = torch.empty(wl.T, wl.H, dtype=bf, device=device)
         self.idx = torch.empty(wl.T, wl.K, dtype=torch.int32, device=device)
@@ -401,7 +418,8 @@ def roofline_entry(wl, stages, touched, peaks, peak_kind, workload):
     ns = wl.shared // F        # shared-expert chunks: F-wide experts every token passes through
     rows = T * (K + ns)
     touched = touched + ns
-    es = 1 if wl.fp8 else 2
+    fp8 = wl.fp8 or wl.fp8_b128
+    es = 1 if fp8 else 2
     up_ms, down_ms = stages["up_gemm"], stages["down_gemm"]
     kernel = "up_gemm" if up_ms >= down_ms else "down_gemm"
     ms = max(up_ms, down_ms)
@@ -412,6 +430,11 @@ def roofline_entry(wl, stages, touched, peaks, peak_kind, workload):
         w_b = touched * F * (H / 2 + ksp(H)) if kernel == "up_gemm" else touched * H * (F / 2 + ksp(F))
         algo = (w_b + rows * (H / 2 + ksp(H)) + rows * (F / 2 + ksp(F)) if kernel == "up_gemm"
                 else w_b + rows * (F / 2 + ksp(F)) + rows * H * 2)
+    elif wl.fp8_b128:
+        # codes padded to whole blocks of 128 along K + one fp32 scale per block
+        kp = lambda k: (k + 127) // 128 * 128
+        w_b = touched * F * (kp(H) + kp(H) // 128 * 4) if kernel == "up_gemm" else touched * H * (kp(F) + kp(F) // 128 * 4)
+        algo = w_b + rows * H + rows * F if kernel == "up_gemm" else w_b + rows * F + rows * H * 2
     # weights of the touched experts + activations in (es bytes) + activations out
     elif kernel == "up_gemm":
         algo = touched * F * H * es + rows * H * es + rows * F * es
@@ -420,13 +443,13 @@ def roofline_entry(wl, stages, touched, peaks, peak_kind, workload):
     hbm_peak = peaks["hbm_gbs"]
     gbs = algo / (ms * 1e-3) / 1e9
     bf16_sust = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-    tc_peak = bf16_sust * (2.0 if wl.fp8 else 1.0)   # fp8 dense = 2x bf16 dense (nominal ratio)
+    tc_peak = bf16_sust * (2.0 if fp8 else 1.0)   # fp8 dense = 2x bf16 dense (nominal ratio)
     tflops = flops / (ms * 1e-3) / 1e12
     common = {"kernel": kernel, "ms_per_launch": ms, "algorithmic_bytes_per_launch": algo,
               "algorithmic_flops_per_launch": flops, "traffic": traffic_from_profile(kernel, workload),
               "hbm_gbs": gbs, "hbm_frac": gbs / hbm_peak, "tensor_tflops": tflops, "tensor_frac": tflops / tc_peak}
     if workload in TENSOR_BOUND:
-        src = f"{peak_kind} bf16 sustained" + (" x 2 (fp8/bf16 nominal ratio)" if wl.fp8 else "")
+        src = f"{peak_kind} bf16 sustained" + (" x 2 (fp8/bf16 nominal ratio)" if fp8 else "")
         return dict(bound="tensor", achieved=tflops, peak=tc_peak, unit="TFLOP/s", frac=tflops / tc_peak,
                     peak_source=src, **common)
     return dict(bound="hbm", achieved=gbs, peak=hbm_peak, unit="GB/s", frac=gbs / hbm_peak,
@@ -459,6 +482,8 @@ def cpu_baseline(wl, n_tokens, seed_batch=0, target_s=CPU_SAMPLE_SECONDS):
         return cpu_baseline_fp8(wl, n_tokens, seed_batch, target_s=target_s)
     if wl.nvfp4:
         return cpu_baseline_nvfp4(wl, n_tokens, seed_batch, target_s=target_s)
+    if wl.fp8_b128:
+        return cpu_baseline_fp8_b128(wl, n_tokens, seed_batch, target_s=target_s)
     import oracle
     from synth import workloads as W
     x = W.host_x(wl, seed_batch)[:n_tokens]
@@ -515,6 +540,36 @@ def cpu_baseline_nvfp4(wl, n_tokens, seed_batch=0, target_s=CPU_SAMPLE_SECONDS):
             "sample": f"{n_tokens} of the {wl.T} tokens of batch {seed_batch} ({wl.name}), full layer "
                       f"(router, top-{wl.K}, {len(used)} W4A4 experts in fp64 on dequantised codes, combine), "
                       f"{reps} times; {dt:.2f} s"}
+
+
+def cpu_baseline_fp8_b128(wl, n_tokens, seed_batch=0, target_s=CPU_SAMPLE_SECONDS):
+    """The oracle's W8A8 layer with FP8_B128 banks (router, experts, combine) on a token sample."""
+    import numpy as np
+    import oracle
+    from synth import workloads as W
+    x = W.host_x(wl, seed_batch)[:n_tokens]
+    wr = W.host_router(wl)
+    _, idx, _ = oracle.route(x, wr, W.host_bias(wl), wl.K)
+    used = sorted(set(idx.reshape(-1).tolist()))
+    slot = -np.ones(wl.E, dtype=np.int32)
+    slot[used] = np.arange(len(used))
+    key = (wl.name, 0, tuple(used), "fp8_b128")
+    if key not in _BANKS:   # weight preparation: untimed
+        _BANKS.clear()
+        _BANKS[key] = (oracle.quantize_fp8_b128(W.host_w_up(wl, experts=used)),
+                       oracle.quantize_fp8_b128(W.host_w_down(wl, experts=used)))
+    bank_up, bank_down = _BANKS[key]
+    sx, sh = W.fp8_b128_scales(wl)
+    dt, reps = 0.0, 0
+    while (reps == 0 or dt < target_s) and reps < 1000:
+        t0 = time.perf_counter()
+        oracle.moe_layer_fp8_b128(x, wr, W.host_bias(wl), bank_up, bank_down, sx, sh, wl.K, wl.H, wl.F, slot=slot)
+        dt += time.perf_counter() - t0
+        reps += 1
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return {"value": reps * n_tokens / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{n_tokens} of the {wl.T} tokens of batch {seed_batch} ({wl.name}), FP8_B128 W8A8 layer "
+                      f"(router, top-{wl.K}, {len(used)} experts in fp64, combine), {reps} times; {dt:.2f} s"}
 
 
 def cpu_baseline_fp8(wl, n_tokens, seed_batch=0, layer=0, target_s=CPU_SAMPLE_SECONDS):
@@ -610,13 +665,15 @@ def run_native(args):
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,
             "dtype": ("fp8_e4m3 (W8A8) experts, bf16 router" if wl.fp8 else
+                      "fp8_e4m3 FP8_B128 (W8A8, one fp32 weight scale per 128 along K) experts, bf16 router"
+                      if wl.fp8_b128 else
                       "nvfp4 (W4A4: e2m1 codes, e4m3 block scales; fp16 tensor-core products) experts, bf16 router"
                       if wl.nvfp4 else "bf16"),
             "data": "synthetic: seeded N(0,1) activations, N(0,0.02) router/expert weights (bf16)",
             "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "E": wl.E, "K": wl.K, "F": wl.F,
                        "layers": wl.layers, "touched_experts": touched, "shared_expert_width": wl.shared,
                        "l2": "inputs larger than L2: the touched experts' weights "
-                             f"({(touched * wl.F + wl.shared) * wl.H * (1.125 if wl.nvfp4 else 2 if wl.fp8 else 4) * wl.layers / 1e9:.2f} GB) "
+                             f"({(touched * wl.F + wl.shared) * wl.H * (1.125 if wl.nvfp4 else 2 if (wl.fp8 or wl.fp8_b128) else 4) * wl.layers / 1e9:.2f} GB) "
                              "stream from HBM every step; token batches rotate; no flush",
                        "parallelism": f"dp{ws} (independent token batches per GPU, weights replicated)",
                        "grouped_gemm": "cta_pair" if args.gemm == "pair" else "single_cta",
@@ -631,7 +688,7 @@ def run_native(args):
         if secondary:
             line["secondary"] = secondary
         if ws == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(wl, 4 if wl.fp8 else 8 if wl.nvfp4 else min(wl.T, 64))
+            line["cpu_baseline"] = cpu_baseline(wl, 4 if wl.fp8 else 8 if (wl.nvfp4 or wl.fp8_b128) else min(wl.T, 64))
         print(json.dumps(line), flush=True)
     if ws > 1:
         dist.destroy_process_group()

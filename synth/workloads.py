@@ -36,6 +36,7 @@ class Workload:
     fp8: bool = False
     nvfp4: bool = False
     shared: int = 0          # shared expert width Fs (0: none)
+    fp8_b128: bool = False   # E4M3 experts with one scale per 128 values along K
 
     @property
     def assignments(self) -> int:
@@ -54,6 +55,9 @@ WORKLOADS = {
     # the MoE block with its shared expert (the pages give no width: one expert of the routed shape)
     7: Workload("decode_shared_T64", 64, 2688, 128, 6, 1856, seed=1, shared=1856),
     8: Workload("prefill_shared_T4096", 4096, 2688, 128, 6, 1856, seed=2, shared=1856),
+    # the FP8 release's block-scaled experts (FP8_B128) on the decode and prefill shapes
+    9: Workload("decode_fp8_b128_T64", 64, 2688, 128, 6, 1856, seed=1, fp8_b128=True),
+    10: Workload("prefill_fp8_b128_T4096", 4096, 2688, 128, 6, 1856, seed=2, fp8_b128=True),
 }
 
 
@@ -142,6 +146,19 @@ def nvfp4_scales(w: Workload):
     import struct
     from pathlib import Path
     p = Path(__file__).resolve().parents[1] / "tests" / "golden" / "nvfp4_scales.json"
+    d = json.loads(p.read_text())[w.name]
+    f32 = lambda h: np.float32(struct.unpack(">f", bytes.fromhex(h))[0])
+    return f32(d["x_scale_f32"]), f32(d["h_scale_f32"])
+
+
+def fp8_b128_scales(w: Workload):
+    """Static W8A8 activation scales (x, H) of an FP8_B128 workload, as fp32.
+    Written by tests/golden/make_fp8_b128_scales.py from a calibration pass of the oracle.
+    """
+    import json
+    import struct
+    from pathlib import Path
+    p = Path(__file__).resolve().parents[1] / "tests" / "golden" / "fp8_b128_scales.json"
     d = json.loads(p.read_text())[w.name]
     f32 = lambda h: np.float32(struct.unpack(">f", bytes.fromhex(h))[0])
     return f32(d["x_scale_f32"]), f32(d["h_scale_f32"])

@@ -52,6 +52,17 @@ def test_nvfp4_bytes_count_half_byte_codes_and_padded_block_scales():
                                                  + rows * (F // 2 + ksp_f))
 
 
+def test_fp8_b128_bytes_count_padded_codes_and_block_scales():
+    up = entry(9, 121, 0.2, 0.1, "decode_fp8_b128")
+    rows = 64 * 6
+    assert up["bound"] == "hbm"
+    assert up["algorithmic_bytes_per_launch"] == 121 * F * (2688 + 21 * 4) + rows * H + rows * F
+    down = entry(10, 128, 0.2, 0.3, "prefill_fp8_b128")
+    rows = 4096 * 6
+    assert down["bound"] == "tensor" and down["peak"] == 2 * PEAKS["bf16_tflops_sustained"]
+    assert down["algorithmic_bytes_per_launch"] == 128 * H * (1920 + 15 * 4) + rows * F + rows * H * 2
+
+
 def test_prefill_is_reported_against_the_sustained_tensor_peak():
     r = entry(2, 128, 0.3, 0.31, "prefill")
     assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s" and r["kernel"] == "down_gemm"
