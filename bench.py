@@ -230,6 +230,10 @@ class Layer:
         torch.cuda.synchronize()
         return int(torch.unique(self.idx).numel()), int(self.idx.numel())
 
+    def launches_per_step(self):
+        """The library's kernel launches in one step (one moe_forward)."""
+        return self.moe.forward_launches(self.dims)
+
 
 class Chain:
     """The 23-layer W8A8 stack of the chain workload, weights made and quantised on the device."""
@@ -268,6 +272,10 @@ class Chain:
     def step(self, i, x=None, out=None):
         y = self.stack.forward(self.xs[i % len(self.xs)] if x is None else x)
         self.out = y if out is None else out.copy_(y)
+
+    def launches_per_step(self):
+        """Per layer: the RMS norm, then one moe_forward."""
+        return self.wl.layers * (1 + self.moe.forward_launches(self.stack.dims))
 
     def profile_layer(self, i):
         """one pass of layer 0, for the stage events"""
@@ -624,6 +632,7 @@ def run_native(args):
 
     wl = W.WORKLOADS[WORKLOADS[args.workload]]
     layer = Chain(wl, device) if wl.layers > 1 else Layer(wl, device)
+    launches = layer.launches_per_step()
     touched, rows = layer.touched_experts(0)
     stages = stage_profile(layer, max(3, min(args.steps, 20)), args.warmup)
 
@@ -682,7 +691,7 @@ def run_native(args):
             "stages_ms": stages,
             "e2e": {"value": job_value(ws, wl.T * wl.layers, args.steps, e2e_ms), "unit": UNIT,
                     "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo},
-            "gpu_launches": (8 * wl.layers if wl.layers > 1 else 7) * args.steps,
+            "gpu_launches": launches * args.steps,
             "clocks": clocks,
         }
         if secondary:

@@ -125,6 +125,11 @@ int moe_abi_version(void);
  * moe_permute and moe_expert_ffn need no more).  Host only; no device call. */
 moe_status moe_workspace_size(const moe_dims* d, size_t* bytes);
 
+/* Number of kernels one moe_forward call with these dims launches on its
+ * stream, under the current test hooks (the router's shape and the
+ * permutation's depend on the batch size).  Host only; no device call. */
+moe_status moe_forward_launches(const moe_dims* d, int32_t* launches);
+
 /* Router: logits, top-K, renormalised softmax weights.
  *   x         [T][H] bf16     w_router [E][H] bf16     bias [E] fp32 or NULL
  *   topk_idx  [T][K] int32    out: experts by descending logit, ties to the lower index

@@ -45,6 +45,7 @@ _SIG = {
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "moe_abi_version": (ctypes.c_int, []),
     "moe_workspace_size": (ctypes.c_int, [_DIMS, ctypes.POINTER(ctypes.c_size_t)]),
+    "moe_forward_launches": (ctypes.c_int, [_DIMS, ctypes.POINTER(ctypes.c_int32)]),
     "moe_route": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P, _S, _P]),
     "moe_route_static": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P]),
     "moe_permute": (ctypes.c_int, [_DIMS, _P, _P, _P, _P, _P, _P, _S, _P]),
@@ -119,6 +120,13 @@ def dims(T, H, E, K, F, fp8=False, nvfp4=False, Fs=0, fp8_b128=False) -> MoeDims
 def workspace_size(d: MoeDims) -> int:
     n = ctypes.c_size_t(0)
     _check(_lib.moe_workspace_size(ctypes.byref(d), ctypes.byref(n)), "moe_workspace_size")
+    return n.value
+
+
+def forward_launches(d: MoeDims) -> int:
+    """Kernels one forward() with these dims launches (host only)."""
+    n = ctypes.c_int32(0)
+    _check(_lib.moe_forward_launches(ctypes.byref(d), ctypes.byref(n)), "moe_forward_launches")
     return n.value
 
 

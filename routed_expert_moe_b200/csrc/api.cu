@@ -29,6 +29,7 @@ cudaError_t launch_permute(const int32_t* idx, int64_t n, int K, int E, int32_t*
 void set_router_small_max(int64_t v);
 void set_router_split(int v);
 size_t permute_scratch_ints(int64_t n, int E);
+int route_launches(int64_t T, int H, int E);
 size_t permute_smem_bytes(int E);
 cudaError_t launch_schedule(const int32_t* offsets, int E, int bn, int4* sched, int* n_sched, int ns, int64_t T,
                             int K, cudaStream_t stream);
@@ -417,6 +418,21 @@ moe_status moe_workspace_size(const moe_dims* d, size_t* bytes) {
     // plans depend on the SM count only through the router split; size for
     // the largest split any device can choose
     *bytes = forward_ws_bytes(d, 1024);
+    return MOE_OK;
+}
+
+moe_status moe_forward_launches(const moe_dims* d, int32_t* launches) {
+    moe_status s = check_dims(d);
+    if (s != MOE_OK) return s;
+    if (!launches) return MOE_EINVAL;
+    if (d->T == 0) {
+        *launches = 0;
+        return MOE_OK;
+    }
+    int n = route_launches(d->T, d->H, d->E);
+    n += permute_scratch_ints(d->T * d->K, d->E) == 0 ? 1 : 3;   // one block, or histogram + scan + scatter
+    n += 1 + 2 + 1;   // row gather, up and down projections, combine
+    *launches = n;
     return MOE_OK;
 }
 

@@ -1214,6 +1214,19 @@ static cudaError_t launch_router_small(const RouterSmallArgs& ra, const DevCtx& 
     return launch_k(kfn, dim3(groups * RS_CLUSTER), dim3(RS_THREADS), smem, stream, ra, ctx);
 }
 
+// Kernel launches launch_route makes for these sizes under the current hooks:
+// the same tests, in the same order, as launch_route below.
+int route_launches(int64_t T, int H, int E) {
+    if (T == 0) return 0;
+    if (T <= g_router_small_max.load()) {
+        const int tb = T <= kRouterSmallTb4Max ? 4 : 8;
+        if (rs_smem_bytes(tb, H, E) <= kRouterSmallSmemMax) return 1;   // expert-split clusters
+    }
+    const int split_mode = g_router_split.load();
+    if (E <= RF_E && split_mode != 1 && (split_mode == 2 || T >= kRouterSplitMin)) return 1;   // hidden-split
+    return 2;   // logits, then top-K
+}
+
 cudaError_t launch_route(const uint16_t* x, const uint16_t* wr, const float* bias, int64_t T, int H,
                          int E, int K, int32_t* idx, float* w, double* P, double* xn2, double* wn2,
                          const RouterPlan& plan, const DevCtx& ctx, cudaStream_t stream,

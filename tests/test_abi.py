@@ -135,6 +135,26 @@ def test_shared_expert_dims_and_pointers_are_checked_on_the_host(moe):
                            *([None] * 6), 0, None) == moe.MOE_EINVAL
 
 
+def test_forward_launch_count_follows_the_dispatch(moe):
+    """Router: one launch up to 256 tokens (expert-split clusters) and from 3072 (hidden-split
+    clusters), two in between; permutation: one block up to 4096 assignments, else three kernels;
+    then the row gather, two projections and the combine."""
+    count = lambda T, **kw: moe.forward_launches(moe.dims(T, 2688, 128, 6, 1856, **kw))
+    assert [count(T) for T in (0, 1, 64, 256, 257, 682, 683, 3071, 3072, 4096)] == [0, 6, 6, 6, 7, 7, 9, 9, 8, 8]
+    assert count(64, nvfp4=True) == count(64, fp8_b128=True) == count(64, Fs=1856) == 6
+    try:
+        moe.debug_set(4, 0)             # never the expert-split clusters
+        assert count(64) == 7
+        moe.debug_set(5, 2)             # always the hidden-split clusters
+        assert count(64) == 6 and count(576) == 6
+        moe.debug_set(5, 1)             # always the two kernels
+        assert count(4096) == 9
+    finally:
+        moe.debug_set(4, -1)
+        moe.debug_set(5, 0)
+    assert count(64) == 6
+
+
 def test_package_has_no_cpu_path():
     src = (ROOT / "routed_expert_moe_b200" / "__init__.py").read_text()
     assert "oracle" not in src and "numpy" not in src
