@@ -1,0 +1,374 @@
+"""Model check of the mbarrier protocols of the grouped-GEMM kernels (no GPU).
+
+Each kernel hands buffers between roles through mbarriers waited on by phase
+parity: a TMA ring of shared-memory stages (producer -> MMA), TMEM
+accumulators or partial slots (MMA -> epilogue warps) and, in the NVFP4
+kernel, a second ring of fp16 stages (converter threads -> MMA).  A parity
+wait cannot tell a phase from the one two ahead, so a protocol is only right
+if no waiter can ever be two phases behind.  Compute-sanitizer is not
+available, so this test runs the protocols, as the kernels write them (the
+same counters, parities and arrival counts), in a discrete-event model:
+
+- an mbarrier completes a phase when its arrival count is reached;
+  ``try_wait.parity(p)`` passes while the current phase's parity is not p;
+- TMA copies land at any later moment, in any order; tcgen05 work completes
+  in issue order (``tcgen05.commit`` arrives when all earlier MMAs are done);
+- every buffer carries the tag of the data last written into it.
+
+Under many random interleavings every consumer must read exactly the tag it
+expects, no producer may overwrite data that has not been consumed, and every
+role must finish.  Two planted protocol mistakes must be caught, so the check
+is not vacuous.
+"""
+import random
+from collections import deque
+
+import pytest
+
+
+class Bar:
+    def __init__(self, count):
+        self.count, self.pending, self.phase = count, count, 0
+
+    def arrive(self):
+        self.pending -= 1
+        assert self.pending >= 0, "more arrivals than the barrier's count"
+        if self.pending == 0:
+            self.phase += 1
+            self.pending = self.count
+
+    def passed(self, parity):
+        return (self.phase & 1) != parity
+
+
+class Violation(AssertionError):
+    pass
+
+
+def check(cond, msg):
+    if not cond:
+        raise Violation(msg)
+
+
+class Sim:
+    """Roles are generators that yield the predicate they wait on; async work is posted to
+    queues (one FIFO per in-order engine, a fresh queue per out-of-order copy)."""
+
+    def __init__(self, seed):
+        self.rng = random.Random(seed)
+        self.roles = {}
+        self.queues = {}
+        self.n = 0
+
+    def role(self, name, gen):
+        self.roles[name] = [gen, lambda: True]
+
+    def post(self, queue, fn):
+        if queue is None:                       # out of order: its own queue
+            self.n += 1
+            queue = ("copy", self.n)
+        self.queues.setdefault(queue, deque()).append(fn)
+
+    def run(self, max_steps=2_000_000):
+        for _ in range(max_steps):
+            ready = [("role", k) for k, (g, pred) in self.roles.items() if pred()]
+            ready += [("queue", k) for k, q in self.queues.items() if q]
+            if not ready:
+                if not self.roles:
+                    return "done"
+                return "deadlock: " + ", ".join(sorted(self.roles))
+            kind, key = self.rng.choice(ready)
+            if kind == "queue":
+                self.queues[key].popleft()()
+            else:
+                g = self.roles[key][0]
+                try:
+                    self.roles[key][1] = next(g)
+                except StopIteration:
+                    del self.roles[key]
+        return "no end"
+
+
+# ----------------------------------------------------------------------------- bf16 / E4M3 grouped GEMM
+
+def gemm(sim, units, k_stages, NS, n_epi=4, plant=None):
+    """grouped_gemm_kernel: NS-stage TMA ring, two TMEM accumulators (tempty: 128 epilogue
+    threads, modelled as 4 warps)."""
+    full, empty = [Bar(1) for _ in range(NS)], [Bar(1) for _ in range(NS)]
+    tfull, tempty = [Bar(1) for _ in range(2)], [Bar(n_epi) for _ in range(2)]
+    smem, fresh = [None] * NS, [False] * NS       # fresh: landed and not yet consumed by the MMA
+    tmem, readers = [None] * 2, [n_epi] * 2
+
+    def producer():
+        st, ph = 0, 0
+        for u in range(units):
+            for ks in range(k_stages):
+                yield (lambda s=st, p=ph: empty[s].passed(p ^ 1))
+
+                def land(s=st, tag=(u, ks)):
+                    check(not fresh[s], f"TMA overwrote stage {s} before the MMA consumed it")
+                    smem[s], fresh[s] = tag, True
+                    full[s].arrive()
+                sim.post(None, land)
+                st += 1
+                if st == NS:
+                    st, ph = 0, ph ^ 1
+
+    def mma():
+        st, ph, acc, aph = 0, 0, 0, 0
+        for u in range(units):
+            yield (lambda a=acc, p=aph: tempty[a].passed(p ^ 1))
+            check(readers[acc] == n_epi, f"MMA wrote accumulator {acc} while the epilogue was reading it")
+            for ks in range(k_stages):
+                yield (lambda s=st, p=ph: full[s].passed(p))
+                check(smem[st] == (u, ks), f"MMA read stage {st} holding {smem[st]}, expected {(u, ks)}")
+
+                def mma_done(s=st, a=acc, first=ks == 0, u=u):
+                    fresh[s] = False
+                    if first:
+                        tmem[a] = ("partial", u)
+                    empty[s].arrive()
+                sim.post("tc", mma_done)
+                st += 1
+                if st == NS:
+                    st, ph = 0, ph ^ 1
+
+            def acc_done(a=acc, u=u):
+                tmem[a], readers[a] = u, 0
+                tfull[a].arrive()
+            sim.post("tc", acc_done)
+            acc += 1
+            if acc == 2:
+                acc, aph = 0, aph ^ 1
+
+    def epilogue(w):
+        acc, aph = 0, 0
+        for u in range(units):
+            yield (lambda a=acc, p=aph: tfull[a].passed(p))
+            if plant == "release_before_read":
+                tempty[acc].arrive()
+                yield (lambda: True)
+                check(tmem[acc] == u, f"epilogue read accumulator {acc} holding {tmem[acc]}, expected {u}")
+                readers[acc] += 1
+            else:
+                check(tmem[acc] == u, f"epilogue read accumulator {acc} holding {tmem[acc]}, expected {u}")
+                readers[acc] += 1
+                tempty[acc].arrive()
+            acc += 1
+            if acc == 2:
+                acc, aph = 0, aph ^ 1
+
+    sim.role("producer", producer())
+    sim.role("mma", mma())
+    for w in range(n_epi):
+        sim.role(f"epilogue{w}", epilogue(w))
+
+
+# ----------------------------------------------------------------------------- FP8_B128 grouped GEMM
+
+def gemm_b128(sim, units, k_stages, NS, NP=4, n_epi=4, plant=None):
+    """grouped_gemm_b128_kernel: the TMA ring, and NP TMEM partial slots, one per K stage
+    (pfull: the MMA's commit; pempty: 128 epilogue threads, modelled as 4 warps)."""
+    full, empty = [Bar(1) for _ in range(NS)], [Bar(1) for _ in range(NS)]
+    pfull, pempty = [Bar(1) for _ in range(NP)], [Bar(n_epi) for _ in range(NP)]
+    smem, fresh = [None] * NS, [False] * NS
+    part, readers = [None] * NP, [n_epi] * NP
+
+    def producer():
+        st, ph = 0, 0
+        for u in range(units):
+            for ks in range(k_stages):
+                yield (lambda s=st, p=ph: empty[s].passed(p ^ 1))
+
+                def land(s=st, tag=(u, ks)):
+                    check(not fresh[s], f"TMA overwrote stage {s} before the MMA consumed it")
+                    smem[s], fresh[s] = tag, True
+                    full[s].arrive()
+                sim.post(None, land)
+                st += 1
+                if st == NS:
+                    st, ph = 0, ph ^ 1
+
+    def mma():
+        st, ph, ps, pph = 0, 0, 0, 0
+        wait_parity = (lambda p: p) if plant == "wrong_parity" else (lambda p: p ^ 1)
+        for u in range(units):
+            for ks in range(k_stages):
+                yield (lambda s=st, p=ph: full[s].passed(p))
+                yield (lambda q=ps, p=pph: pempty[q].passed(wait_parity(p)))
+                check(smem[st] == (u, ks), f"MMA read stage {st} holding {smem[st]}, expected {(u, ks)}")
+                check(readers[ps] == n_epi, f"MMA wrote partial slot {ps} while the epilogue was reading it")
+                readers[ps] = 0
+
+                def mma_done(s=st, q=ps, tag=(u, ks)):
+                    fresh[s] = False
+                    part[q] = tag
+                    empty[s].arrive()
+                    pfull[q].arrive()
+                sim.post("tc", mma_done)
+                st += 1
+                if st == NS:
+                    st, ph = 0, ph ^ 1
+                ps += 1
+                if ps == NP:
+                    ps, pph = 0, pph ^ 1
+
+    def epilogue(w):
+        ps, pph = 0, 0
+        for u in range(units):
+            for ks in range(k_stages):
+                yield (lambda q=ps, p=pph: pfull[q].passed(p))
+                check(part[ps] == (u, ks), f"epilogue read partial slot {ps} holding {part[ps]}, expected {(u, ks)}")
+                readers[ps] += 1
+                pempty[ps].arrive()
+                ps += 1
+                if ps == NP:
+                    ps, pph = 0, pph ^ 1
+
+    sim.role("producer", producer())
+    sim.role("mma", mma())
+    for w in range(n_epi):
+        sim.role(f"epilogue{w}", epilogue(w))
+
+
+# ----------------------------------------------------------------------------- NVFP4 grouped GEMM
+
+def gemm_fp4(sim, units, k_raw, k_f16, NR, NF, n_conv=8, n_epi=4):
+    """grouped_gemm_fp4_kernel: a raw TMA ring (raw_empty: every converter thread), the
+    converters' fp16 ring (f16_full: every converter thread; f16_empty: the MMA's commit),
+    two TMEM accumulators.  The 128 converter threads take the fp16 buffers in the same
+    order; they are modelled as n_conv independent agents (any of them may run ahead)."""
+    raw_full, raw_empty = [Bar(1) for _ in range(NR)], [Bar(n_conv) for _ in range(NR)]
+    f16_full, f16_empty = [Bar(n_conv) for _ in range(NF)], [Bar(1) for _ in range(NF)]
+    tfull, tempty = [Bar(1) for _ in range(2)], [Bar(n_epi) for _ in range(2)]
+    raw, raw_reads = [None] * NR, [n_conv] * NR
+    f16 = [[None] * n_conv for _ in range(NF)]
+    f16_fresh = [[False] * n_conv for _ in range(NF)]
+    tmem, readers = [None] * 2, [n_epi] * 2
+
+    def producer():
+        rs, rph = 0, 0
+        for u in range(units):
+            for kr in range(k_raw):
+                yield (lambda s=rs, p=rph: raw_empty[s].passed(p ^ 1))
+
+                def land(s=rs, tag=(u, kr)):
+                    check(raw_reads[s] == n_conv, f"TMA overwrote raw stage {s} before every converter read it")
+                    raw[s], raw_reads[s] = tag, 0
+                    raw_full[s].arrive()
+                sim.post(None, land)
+                rs += 1
+                if rs == NR:
+                    rs, rph = 0, rph ^ 1
+
+    def converter(i):
+        rs, rph, fs, fph = 0, 0, 0, 0
+        for u in range(units):
+            for kr in range(k_raw):
+                yield (lambda s=rs, p=rph: raw_full[s].passed(p))
+                check(raw[rs] == (u, kr), f"converter {i} read raw stage {rs} holding {raw[rs]}, expected {(u, kr)}")
+                for sub in range(4):
+                    kf = kr * 4 + sub
+                    if kf >= k_f16:
+                        break
+                    yield (lambda f=fs, p=fph: f16_empty[f].passed(p ^ 1))
+                    check(not f16_fresh[fs][i], f"converter {i} overwrote fp16 stage {fs} before the MMA read it")
+                    f16[fs][i], f16_fresh[fs][i] = (u, kf), True
+                    f16_full[fs].arrive()
+                    fs += 1
+                    if fs == NF:
+                        fs, fph = 0, fph ^ 1
+                raw_reads[rs] += 1
+                raw_empty[rs].arrive()
+                rs += 1
+                if rs == NR:
+                    rs, rph = 0, rph ^ 1
+
+    def mma():
+        fs, fph, acc, aph = 0, 0, 0, 0
+        for u in range(units):
+            yield (lambda a=acc, p=aph: tempty[a].passed(p ^ 1))
+            check(readers[acc] == n_epi, f"MMA wrote accumulator {acc} while the epilogue was reading it")
+            for kf in range(k_f16):
+                yield (lambda f=fs, p=fph: f16_full[f].passed(p))
+                check(all(t == (u, kf) for t in f16[fs]), f"MMA read fp16 stage {fs} holding {f16[fs]}")
+
+                def mma_done(f=fs):
+                    f16_fresh[f] = [False] * n_conv
+                    f16_empty[f].arrive()
+                sim.post("tc", mma_done)
+                fs += 1
+                if fs == NF:
+                    fs, fph = 0, fph ^ 1
+
+            def acc_done(a=acc, u=u):
+                tmem[a], readers[a] = u, 0
+                tfull[a].arrive()
+            sim.post("tc", acc_done)
+            acc += 1
+            if acc == 2:
+                acc, aph = 0, aph ^ 1
+
+    def epilogue(w):
+        acc, aph = 0, 0
+        for u in range(units):
+            yield (lambda a=acc, p=aph: tfull[a].passed(p))
+            check(tmem[acc] == u, f"epilogue read accumulator {acc} holding {tmem[acc]}, expected {u}")
+            readers[acc] += 1
+            tempty[acc].arrive()
+            acc += 1
+            if acc == 2:
+                acc, aph = 0, aph ^ 1
+
+    sim.role("producer", producer())
+    sim.role("mma", mma())
+    for i in range(n_conv):
+        sim.role(f"converter{i}", converter(i))
+    for w in range(n_epi):
+        sim.role(f"epilogue{w}", epilogue(w))
+
+
+SEEDS = range(40)
+
+
+@pytest.mark.parametrize("units,k_stages,NS", [(5, 21, 8), (7, 3, 2), (4, 1, 3), (6, 42, 4)])
+def test_grouped_gemm_protocol(units, k_stages, NS):
+    for seed in SEEDS:
+        sim = Sim(seed)
+        gemm(sim, units, k_stages, NS)
+        assert sim.run() == "done"
+
+
+@pytest.mark.parametrize("units,k_stages,NS", [(4, 21, 8), (6, 15, 8), (5, 3, 2), (3, 1, 4), (3, 9, 5)])
+def test_fp8_b128_protocol(units, k_stages, NS):
+    for seed in SEEDS:
+        sim = Sim(seed)
+        gemm_b128(sim, units, k_stages, NS)
+        assert sim.run() == "done"
+
+
+@pytest.mark.parametrize("units,k_raw,k_f16,NR,NF", [(3, 11, 42, 4, 5), (3, 8, 29, 2, 2), (4, 1, 4, 3, 5),
+                                                     (3, 2, 7, 5, 2), (2, 11, 42, 8, 3)])
+def test_nvfp4_protocol(units, k_raw, k_f16, NR, NF):
+    for seed in range(15):
+        sim = Sim(seed)
+        gemm_fp4(sim, units, k_raw, k_f16, NR, NF)
+        assert sim.run() == "done"
+
+
+def test_a_wait_on_the_wrong_parity_is_caught():
+    sim = Sim(0)
+    gemm_b128(sim, 3, 5, 4, plant="wrong_parity")
+    assert sim.run().startswith("deadlock")
+
+
+def test_releasing_an_accumulator_before_reading_it_is_caught():
+    caught = 0
+    for seed in SEEDS:
+        sim = Sim(seed)
+        gemm(sim, 6, 2, 2, plant="release_before_read")
+        try:
+            sim.run()
+        except Violation:
+            caught += 1
+    assert caught > 0
