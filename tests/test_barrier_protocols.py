@@ -27,15 +27,30 @@ import pytest
 
 
 class Bar:
+    """An mbarrier: a phase completes when its arrivals reach the count and its transaction
+    count (bytes announced by expect_tx, less bytes landed; it may go below zero while the
+    phase is open) is back to zero."""
+
     def __init__(self, count):
-        self.count, self.pending, self.phase = count, count, 0
+        self.count, self.pending, self.phase, self.tx = count, count, 0, 0
+
+    def _maybe_complete(self):
+        if self.pending == 0 and self.tx == 0:
+            self.phase += 1
+            self.pending = self.count
 
     def arrive(self):
         self.pending -= 1
         assert self.pending >= 0, "more arrivals than the barrier's count"
-        if self.pending == 0:
-            self.phase += 1
-            self.pending = self.count
+        self._maybe_complete()
+
+    def arrive_expect_tx(self, n):
+        self.tx += n
+        self.arrive()
+
+    def complete_tx(self, n):
+        self.tx -= n
+        self._maybe_complete()
 
     def passed(self, parity):
         return (self.phase & 1) != parity
@@ -328,6 +343,87 @@ def gemm_fp4(sim, units, k_raw, k_f16, NR, NF, n_conv=8, n_epi=4):
         sim.role(f"epilogue{w}", epilogue(w))
 
 
+# ----------------------------------------------------------------------------- CTA-pair grouped GEMM
+
+def gemm_pair(sim, units, k_stages, NS, n_epi=4):
+    """grouped_gemm_kernel_pair (cta_group::2): each CTA's producer waits its own `empty` and
+    loads its half of the stage; the leader arms its `full` with both halves' bytes, and both
+    halves complete transactions on the leader's `full` (the peer's may land before the
+    leader arms it).  The leader's MMA commits to `empty` and `tfull` of both CTAs (multicast
+    commit); the 4 epilogue warps of each CTA arrive on the leader's `tempty` (count 8)."""
+    full = [Bar(1) for _ in range(NS)]                                   # leader only
+    empty = [[Bar(1) for _ in range(NS)] for _ in range(2)]
+    tfull = [[Bar(1) for _ in range(2)] for _ in range(2)]
+    tempty = [Bar(2 * n_epi) for _ in range(2)]                          # leader only
+    smem = [[None] * NS for _ in range(2)]
+    fresh = [[False] * NS for _ in range(2)]
+    tmem = [[None] * 2 for _ in range(2)]
+    readers = [2 * n_epi] * 2
+
+    def producer(rank):
+        st, ph = 0, 0
+        for u in range(units):
+            for ks in range(k_stages):
+                yield (lambda s=st, p=ph: empty[rank][s].passed(p ^ 1))
+                if rank == 0:
+                    full[st].arrive_expect_tx(2)                         # both halves
+
+                def land(s=st, tag=(u, ks)):
+                    check(not fresh[rank][s], f"TMA overwrote stage {s} of CTA {rank} before the MMA consumed it")
+                    smem[rank][s], fresh[rank][s] = tag, True
+                    full[s].complete_tx(1)
+                sim.post(None, land)
+                st += 1
+                if st == NS:
+                    st, ph = 0, ph ^ 1
+
+    def mma():
+        st, ph, acc, aph = 0, 0, 0, 0
+        for u in range(units):
+            yield (lambda a=acc, p=aph: tempty[a].passed(p ^ 1))
+            check(readers[acc] == 2 * n_epi, f"MMA wrote accumulator {acc} while an epilogue was reading it")
+            for ks in range(k_stages):
+                yield (lambda s=st, p=ph: full[s].passed(p))
+                for r in range(2):
+                    check(smem[r][st] == (u, ks), f"MMA read stage {st} of CTA {r} holding {smem[r][st]}")
+
+                def mma_done(s=st):
+                    for r in range(2):
+                        fresh[r][s] = False
+                        empty[r][s].arrive()
+                sim.post("tc", mma_done)
+                st += 1
+                if st == NS:
+                    st, ph = 0, ph ^ 1
+
+            def acc_done(a=acc, u=u):
+                readers[a] = 0
+                for r in range(2):
+                    tmem[r][a] = u
+                    tfull[r][a].arrive()
+            sim.post("tc", acc_done)
+            acc += 1
+            if acc == 2:
+                acc, aph = 0, aph ^ 1
+
+    def epilogue(rank, w):
+        acc, aph = 0, 0
+        for u in range(units):
+            yield (lambda a=acc, p=aph: tfull[rank][a].passed(p))
+            check(tmem[rank][acc] == u, f"epilogue of CTA {rank} read accumulator {acc} holding {tmem[rank][acc]}")
+            readers[acc] += 1
+            tempty[acc].arrive()
+            acc += 1
+            if acc == 2:
+                acc, aph = 0, aph ^ 1
+
+    for r in range(2):
+        sim.role(f"producer{r}", producer(r))
+        for w in range(n_epi):
+            sim.role(f"epilogue{r}.{w}", epilogue(r, w))
+    sim.role("mma", mma())
+
+
 SEEDS = range(40)
 
 
@@ -336,6 +432,14 @@ def test_grouped_gemm_protocol(units, k_stages, NS):
     for seed in SEEDS:
         sim = Sim(seed)
         gemm(sim, units, k_stages, NS)
+        assert sim.run() == "done"
+
+
+@pytest.mark.parametrize("units,k_stages,NS", [(5, 21, 6), (6, 3, 2), (4, 1, 3), (3, 42, 6)])
+def test_cta_pair_gemm_protocol(units, k_stages, NS):
+    for seed in SEEDS:
+        sim = Sim(seed)
+        gemm_pair(sim, units, k_stages, NS)
         assert sim.run() == "done"
 
 
