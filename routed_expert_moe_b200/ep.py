@@ -20,7 +20,10 @@ row exchange moves raw bytes, so any row dtype travels unchanged.
 
 The kernels come from an ``ops`` object (``CudaOps``: the library's calls on
 the current CUDA device); the collectives from ``torch.distributed`` (NCCL on
-GPUs).  The expert banks a rank passes hold its own experts only.
+GPUs).  The expert banks a rank passes hold its own experts only, in any of
+the library's expert formats (bf16, FP8 E4M3, NVFP4, FP8_B128): the rows
+travel in bf16 and the owner's grouped FFN quantises them, with the scales of
+its own experts.
 """
 from __future__ import annotations
 
@@ -29,14 +32,20 @@ import torch
 import torch.distributed as dist
 
 
+FORMATS = ("bf16", "fp8", "nvfp4", "fp8_b128")
+
+
 class CudaOps:
     """The layer's steps on the current CUDA device, through the library's C ABI."""
 
-    def __init__(self, H: int, E: int, K: int, F: int):
+    def __init__(self, H: int, E: int, K: int, F: int, experts: str = "bf16"):
         from . import dims as _dims
         import routed_expert_moe_b200 as moe
+        if experts not in FORMATS:
+            raise ValueError(f"expert format {experts!r} is not one of {FORMATS}")
         self.moe, self._dims = moe, _dims
         self.H, self.E, self.K, self.F = H, E, K, F
+        self.fmt = {k: experts == k for k in ("fp8", "nvfp4", "fp8_b128")}
 
     def _ws(self, d):
         return self.moe.alloc_workspace(d)
@@ -66,11 +75,11 @@ class CudaOps:
             self.moe.gather_rows(x, perm_src, out, K=K)
         return out
 
-    def expert_ffn(self, rows, offsets, perm, w_up, w_down):
+    def expert_ffn(self, rows, offsets, perm, w_up, w_down, scales=None):
         R, E_loc = rows.shape[0], w_up.shape[0]
         y = torch.empty(R, self.H, dtype=torch.bfloat16, device=rows.device)
-        d = self._dims(R, self.H, E_loc, 1, self.F)
-        self.moe.expert_ffn(d, rows, offsets, perm, w_up, w_down, None, y, self._ws(d))
+        d = self._dims(R, self.H, E_loc, 1, self.F, **self.fmt)
+        self.moe.expert_ffn(d, rows, offsets, perm, w_up, w_down, scales, y, self._ws(d))
         return y
 
     def combine(self, y_perm, inv_row, w, residual, out):
@@ -104,7 +113,7 @@ def regroup(recv_counts: np.ndarray):
 class ExpertParallelLayer:
     """One MoE layer split over the ranks of ``group`` by expert."""
 
-    def __init__(self, H: int, E: int, K: int, F: int, group=None, ops=None):
+    def __init__(self, H: int, E: int, K: int, F: int, group=None, ops=None, experts: str = "bf16"):
         self.group = group
         self.W = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
@@ -112,15 +121,16 @@ class ExpertParallelLayer:
             raise ValueError(f"{E} experts do not split evenly over {self.W} ranks")
         self.H, self.E, self.K, self.F = H, E, K, F
         self.E_loc = E // self.W
-        self.ops = ops if ops is not None else CudaOps(H, E, K, F)
+        self.ops = ops if ops is not None else CudaOps(H, E, K, F, experts)
 
     def experts(self, rank=None):
         r = self.rank if rank is None else rank
         return range(r * self.E_loc, (r + 1) * self.E_loc)
 
-    def forward(self, x, w_router, bias, w_up_local, w_down_local, out, residual=None):
-        """x [T, H] (this rank's tokens); w_up_local [E/W, F, H], w_down_local [E/W, H, F] (this
-        rank's experts); out [T, H].  Returns (topk_idx, topk_w)."""
+    def forward(self, x, w_router, bias, w_up_local, w_down_local, out, residual=None, scales=None):
+        """x [T, H] (this rank's tokens); w_up_local, w_down_local: this rank's E/W experts in the
+        layer's expert format, with ``scales`` (moe_quant_scales of those experts; None for bf16);
+        out [T, H].  Returns (topk_idx, topk_w)."""
         ops, W, E_loc, K = self.ops, self.W, self.E_loc, self.K
         idx, w = ops.route(x, w_router, bias)
         counts, offsets, perm_src, inv_row = ops.permute(idx)
@@ -140,7 +150,7 @@ class ExpertParallelLayer:
         loc_off, perm, inv = regroup(rc_mat)
         dev = x.device
         y_loc = ops.expert_ffn(recv_rows, torch.from_numpy(loc_off).to(dev), torch.from_numpy(perm).to(dev),
-                               w_up_local, w_down_local)
+                               w_up_local, w_down_local, scales)
         y_back = ops.gather(y_loc, torch.from_numpy(inv).to(dev), 1)  # arrival order
 
         y_perm = torch.empty((sum(sc),) + tuple(y_back.shape[1:]), dtype=y_back.dtype, device=dev)

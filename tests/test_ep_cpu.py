@@ -49,13 +49,18 @@ class OracleOps:
     def gather(self, x, perm, K):
         return x[perm.long() // K]
 
-    def expert_ffn(self, rows, offsets, perm, w_up, w_down):
+    def expert_ffn(self, rows, offsets, perm, w_up, w_down, scales=None):
         R = rows.shape[0]
         if R == 0:
             return torch.zeros(0, self.H, dtype=torch.float64)
-        xr = self.o.bf16_to_f64(rows.numpy().view(np.uint16))[perm.numpy()]
+        bits = rows.numpy().view(np.uint16)[perm.numpy()]
         ex = (np.searchsorted(offsets.numpy(), np.arange(R), side="right") - 1).astype(np.int32)
-        y = self.o.expert_rows_bf16(xr, ex, w_up, w_down, self.o.identity_slot(w_up.shape[0]))
+        slot = self.o.identity_slot(w_up[0].shape[0] if scales is not None else w_up.shape[0])
+        if scales is None:
+            y = self.o.expert_rows_bf16(self.o.bf16_to_f64(bits), ex, w_up, w_down, slot)
+        else:                              # W8A8: banks (codes, tensor scales), scales (x, h)
+            (qu, su), (qd, sd), (sx, sh) = w_up, w_down, scales
+            y = self.o.expert_rows_fp8(self.o.quantize_act_fp8(bits, sx), ex, qu, su, qd, sd, slot, sx, sh)
         return torch.from_numpy(y)
 
     def combine(self, y_perm, inv_row, w, residual, out):
@@ -65,16 +70,16 @@ class OracleOps:
         return out
 
 
-def _worker(rank, world, port, T, q):
+def _worker(rank, world, port, T, q, fp8=False):
     try:
-        _run(rank, world, port, T, q)
+        _run(rank, world, port, T, q, fp8)
     except BaseException:                                 # report, so the parent fails at once
         import traceback
         q.put((rank, None, traceback.format_exc()))
         raise
 
 
-def _run(rank, world, port, T, q):
+def _run(rank, world, port, T, q, fp8):
     import torch.distributed as dist
     sys.path.insert(0, str(ROOT))
     from synth import workloads as W
@@ -88,19 +93,27 @@ def _run(rank, world, port, T, q):
         layer = ExpertParallelLayer(w.H, w.E, w.K, w.F, ops=OracleOps(w.E, w.K, w.H))
         mine = list(layer.experts())
         out = torch.empty(T, w.H, dtype=torch.float64)
-        idx, _ = layer.forward(torch.from_numpy(x.view(np.int16)), wr, None, np.ascontiguousarray(wu[mine]),
-                               np.ascontiguousarray(wd[mine]), out)
+        if fp8:
+            import oracle
+            qu, su = oracle.quantize_bank_fp8(wu)
+            qd, sd = oracle.quantize_bank_fp8(wd)
+            sc = oracle.calibrate_fp8(W.host_x(w)[:16], wr, None, wu, w.K)
+            idx, _ = layer.forward(torch.from_numpy(x.view(np.int16)), wr, None, (qu[mine], su[mine]),
+                                   (qd[mine], sd[mine]), out, scales=sc)
+        else:
+            idx, _ = layer.forward(torch.from_numpy(x.view(np.int16)), wr, None, np.ascontiguousarray(wu[mine]),
+                                   np.ascontiguousarray(wd[mine]), out)
         q.put((rank, out.numpy(), idx.numpy()))
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world,T", [(2, 16), (4, 9), (2, 1)])
-def test_expert_parallel_layer_equals_the_one_process_layer(world, T):
+@pytest.mark.parametrize("world,T,fp8", [(2, 16, False), (4, 9, False), (2, 1, False), (2, 12, True)])
+def test_expert_parallel_layer_equals_the_one_process_layer(world, T, fp8):
     port = _free_port()
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
-    procs = [ctx.Process(target=_worker, args=(r, world, port, T, q)) for r in range(world)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, T, q, fp8)) for r in range(world)]
     for p in procs:
         p.start()
     res = {}
@@ -118,8 +131,13 @@ def test_expert_parallel_layer_equals_the_one_process_layer(world, T):
     from synth import workloads as W
     w = W.Workload("ep", T, 256, 8, 2, 128, seed=31)
     wr, wu, wd = W.host_router(w), W.host_w_up(w), W.host_w_down(w)
+    if fp8:
+        qu, su = oracle.quantize_bank_fp8(wu)
+        qd, sd = oracle.quantize_bank_fp8(wd)
+        sx, sh = oracle.calibrate_fp8(W.host_x(w)[:16], wr, None, wu, w.K)
     for rank in range(world):
-        ref = oracle.moe_layer_bf16(W.host_x(w, layer=rank), wr, None, wu, wd, w.K)
+        ref = (oracle.moe_layer_fp8(W.host_x(w, layer=rank), wr, None, qu, su, qd, sd, sx, sh, w.K) if fp8 else
+               oracle.moe_layer_bf16(W.host_x(w, layer=rank), wr, None, wu, wd, w.K))
         out, idx = res[rank]
         assert np.array_equal(idx, ref["idx"])
         assert np.array_equal(out, ref["out"])
