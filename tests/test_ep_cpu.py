@@ -32,11 +32,11 @@ def _free_port():
 
 class OracleOps:
     """The layer's steps on CPU from the oracle (bf16 rows travel as int16 bit patterns, expert
-    outputs as float64)."""
+    outputs as float64).  fmt: the experts' format; the banks and scales are the oracle's."""
 
-    def __init__(self, E, K, H):
+    def __init__(self, E, K, H, F=None, fmt="bf16"):
         import oracle
-        self.o, self.E, self.K, self.H = oracle, E, K, H
+        self.o, self.E, self.K, self.H, self.F, self.fmt = oracle, E, K, H, F, fmt
 
     def route(self, x, w_router, bias):
         _, idx, w = self.o.route(x.numpy().view(np.uint16), w_router, bias, self.K)
@@ -53,14 +53,23 @@ class OracleOps:
         R = rows.shape[0]
         if R == 0:
             return torch.zeros(0, self.H, dtype=torch.float64)
+        o = self.o
         bits = rows.numpy().view(np.uint16)[perm.numpy()]
         ex = (np.searchsorted(offsets.numpy(), np.arange(R), side="right") - 1).astype(np.int32)
-        slot = self.o.identity_slot(w_up[0].shape[0] if scales is not None else w_up.shape[0])
-        if scales is None:
-            y = self.o.expert_rows_bf16(self.o.bf16_to_f64(bits), ex, w_up, w_down, slot)
-        else:                              # W8A8: banks (codes, tensor scales), scales (x, h)
+        slot = o.identity_slot(len(w_up[0]) if scales is not None else w_up.shape[0])
+        if self.fmt == "bf16":
+            y = o.expert_rows_bf16(o.bf16_to_f64(bits), ex, w_up, w_down, slot)
+        elif self.fmt == "fp8":            # banks (codes, tensor scales); scales (x, h)
             (qu, su), (qd, sd), (sx, sh) = w_up, w_down, scales
-            y = self.o.expert_rows_fp8(self.o.quantize_act_fp8(bits, sx), ex, qu, su, qd, sd, slot, sx, sh)
+            y = o.expert_rows_fp8(o.quantize_act_fp8(bits, sx), ex, qu, su, qd, sd, slot, sx, sh)
+        elif self.fmt == "nvfp4":          # banks (codes, block scales, tensor scales)
+            tx, th = scales
+            cx, sx_ = o.quantize_nvfp4(bits, tx)
+            y = o.expert_rows_nvfp4(cx, sx_, ex, w_up, w_down, slot, tx, th)
+        else:                              # fp8_b128: banks (codes, block scales)
+            sx, sh = scales
+            y = o.expert_rows_fp8_b128(o.quantize_act_fp8_b128(bits, sx), ex, w_up, w_down, slot, sx, sh,
+                                       self.H, self.F)
         return torch.from_numpy(y)
 
     def combine(self, y_perm, inv_row, w, residual, out):
@@ -70,16 +79,50 @@ class OracleOps:
         return out
 
 
-def _worker(rank, world, port, T, q, fp8=False):
+def _worker(rank, world, port, T, q, fmt="bf16"):
     try:
-        _run(rank, world, port, T, q, fp8)
+        _run(rank, world, port, T, q, fmt)
     except BaseException:                                 # report, so the parent fails at once
         import traceback
         q.put((rank, None, traceback.format_exc()))
         raise
 
 
-def _run(rank, world, port, T, q, fp8):
+def local_banks(o, fmt, wu, wd, mine):
+    """This rank's experts in the layer's format (the oracle quantises every bank)."""
+    if fmt == "bf16":
+        return np.ascontiguousarray(wu[mine]), np.ascontiguousarray(wd[mine])
+    q = {"fp8": o.quantize_bank_fp8, "nvfp4": o.quantize_bank_nvfp4, "fp8_b128": o.quantize_fp8_b128}[fmt]
+    bu, bd = q(wu), q(wd)
+    return tuple(np.ascontiguousarray(a[mine]) for a in bu), tuple(np.ascontiguousarray(a[mine]) for a in bd)
+
+
+def act_scales(o, fmt, w, wr, wu):
+    if fmt == "nvfp4":
+        return o.calibrate_nvfp4(_x(w, 0)[:16], wr, None, wu, w.K)
+    return o.calibrate_fp8(_x(w, 0)[:16], wr, None, wu, w.K)
+
+
+def _x(w, rank):
+    from synth import workloads as W
+    return W.host_x(w, layer=rank)
+
+
+def reference(o, fmt, w, x, wr, wu, wd):
+    if fmt == "bf16":
+        return o.moe_layer_bf16(x, wr, None, wu, wd, w.K)
+    s1, s2 = act_scales(o, fmt, w, wr, wu)
+    if fmt == "fp8":
+        qu, su = o.quantize_bank_fp8(wu)
+        qd, sd = o.quantize_bank_fp8(wd)
+        return o.moe_layer_fp8(x, wr, None, qu, su, qd, sd, s1, s2, w.K)
+    if fmt == "nvfp4":
+        return o.moe_layer_nvfp4(x, wr, None, o.quantize_bank_nvfp4(wu), o.quantize_bank_nvfp4(wd), s1, s2, w.K)
+    return o.moe_layer_fp8_b128(x, wr, None, o.quantize_fp8_b128(wu), o.quantize_fp8_b128(wd), s1, s2, w.K,
+                                w.H, w.F)
+
+
+def _run(rank, world, port, T, q, fmt):
     import torch.distributed as dist
     sys.path.insert(0, str(ROOT))
     from synth import workloads as W
@@ -90,30 +133,25 @@ def _run(rank, world, port, T, q, fp8):
         w = W.Workload("ep", T, 256, 8, 2, 128, seed=31)
         x = W.host_x(w, layer=rank)                       # each rank its own tokens
         wr, wu, wd = W.host_router(w), W.host_w_up(w), W.host_w_down(w)
-        layer = ExpertParallelLayer(w.H, w.E, w.K, w.F, ops=OracleOps(w.E, w.K, w.H))
+        import oracle
+        layer = ExpertParallelLayer(w.H, w.E, w.K, w.F, ops=OracleOps(w.E, w.K, w.H, w.F, fmt))
         mine = list(layer.experts())
         out = torch.empty(T, w.H, dtype=torch.float64)
-        if fp8:
-            import oracle
-            qu, su = oracle.quantize_bank_fp8(wu)
-            qd, sd = oracle.quantize_bank_fp8(wd)
-            sc = oracle.calibrate_fp8(W.host_x(w)[:16], wr, None, wu, w.K)
-            idx, _ = layer.forward(torch.from_numpy(x.view(np.int16)), wr, None, (qu[mine], su[mine]),
-                                   (qd[mine], sd[mine]), out, scales=sc)
-        else:
-            idx, _ = layer.forward(torch.from_numpy(x.view(np.int16)), wr, None, np.ascontiguousarray(wu[mine]),
-                                   np.ascontiguousarray(wd[mine]), out)
+        bu, bd = local_banks(oracle, fmt, wu, wd, mine)
+        sc = None if fmt == "bf16" else act_scales(oracle, fmt, w, wr, wu)
+        idx, _ = layer.forward(torch.from_numpy(x.view(np.int16)), wr, None, bu, bd, out, scales=sc)
         q.put((rank, out.numpy(), idx.numpy()))
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world,T,fp8", [(2, 16, False), (4, 9, False), (2, 1, False), (2, 12, True)])
-def test_expert_parallel_layer_equals_the_one_process_layer(world, T, fp8):
+@pytest.mark.parametrize("world,T,fmt", [(2, 16, "bf16"), (4, 9, "bf16"), (2, 1, "bf16"), (2, 12, "fp8"),
+                                         (2, 12, "nvfp4"), (2, 12, "fp8_b128")])
+def test_expert_parallel_layer_equals_the_one_process_layer(world, T, fmt):
     port = _free_port()
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
-    procs = [ctx.Process(target=_worker, args=(r, world, port, T, q, fp8)) for r in range(world)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, T, q, fmt)) for r in range(world)]
     for p in procs:
         p.start()
     res = {}
@@ -131,13 +169,8 @@ def test_expert_parallel_layer_equals_the_one_process_layer(world, T, fp8):
     from synth import workloads as W
     w = W.Workload("ep", T, 256, 8, 2, 128, seed=31)
     wr, wu, wd = W.host_router(w), W.host_w_up(w), W.host_w_down(w)
-    if fp8:
-        qu, su = oracle.quantize_bank_fp8(wu)
-        qd, sd = oracle.quantize_bank_fp8(wd)
-        sx, sh = oracle.calibrate_fp8(W.host_x(w)[:16], wr, None, wu, w.K)
     for rank in range(world):
-        ref = (oracle.moe_layer_fp8(W.host_x(w, layer=rank), wr, None, qu, su, qd, sd, sx, sh, w.K) if fp8 else
-               oracle.moe_layer_bf16(W.host_x(w, layer=rank), wr, None, wu, wd, w.K))
+        ref = reference(oracle, fmt, w, W.host_x(w, layer=rank), wr, wu, wd)
         out, idx = res[rank]
         assert np.array_equal(idx, ref["idx"])
         assert np.array_equal(out, ref["out"])
