@@ -189,3 +189,51 @@ def test_regroup_orders_rows_by_expert_then_source():
         assert perm.tolist() == want
         assert np.array_equal(inv[perm], np.arange(len(labels)))
         assert off.tolist() == [0] + np.cumsum(counts.sum(0)).tolist()
+
+
+def _failing_worker(rank, world, port, q):
+    """Rank 1 leaves before the layer's first exchange; rank 0 must get an error from its
+    collective (the group's short timeout, or the peer's closed connection), not hang."""
+    import datetime
+    import time
+    import torch.distributed as dist
+    sys.path.insert(0, str(ROOT))
+    from synth import workloads as W
+    from routed_expert_moe_b200.ep import ExpertParallelLayer
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=3))
+    if rank == 1:
+        q.put((rank, "left"))
+        q.close()
+        q.join_thread()                                 # the message is sent before the process goes
+        os._exit(0)                                     # gone, with no collective in flight
+    w = W.Workload("ep", 8, 256, 8, 2, 128, seed=31)
+    layer = ExpertParallelLayer(w.H, w.E, w.K, w.F, ops=OracleOps(w.E, w.K, w.H))
+    mine = list(layer.experts())
+    out = torch.empty(w.T, w.H, dtype=torch.float64)
+    t0 = time.monotonic()
+    try:
+        layer.forward(torch.from_numpy(W.host_x(w).view(np.int16)), W.host_router(w), None,
+                      np.ascontiguousarray(W.host_w_up(w)[mine]), np.ascontiguousarray(W.host_w_down(w)[mine]), out)
+        q.put((rank, "no error"))
+    except Exception as e:                              # the failure reaches this rank as an error
+        q.put((rank, f"error after {time.monotonic() - t0:.1f} s: {type(e).__name__}"))
+    q.close()
+    q.join_thread()
+    os._exit(0)
+
+
+def test_a_rank_that_leaves_ends_the_exchange_with_an_error():
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_failing_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = dict(q.get(timeout=120) for _ in range(2))
+    for p in procs:
+        p.join(timeout=60)
+    assert res[1] == "left"
+    assert res[0].startswith("error after"), res[0]
+    assert float(res[0].split()[2]) < 60
+
