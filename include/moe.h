@@ -84,10 +84,23 @@ typedef struct {
     int32_t Fs;            /* shared expert width (0: none) */
 } moe_dims;
 
-/* Scales of the quantised experts.  Ignored for MOE_BF16.
+/* Scales of the quantised expert formats.  Ignored for MOE_BF16; required
+ * (non-NULL, with every pointer named below for the format non-NULL) for the
+ * three others.  Activation scales are static in every format: x_scale and
+ * h_scale are finite and > 0.  Per format:
  *
  * MOE_FP8_E4M3 (bloomery page, section 2: "scalar-scale E4M3 W8A8"): real
- * value = code * scale; the two block-scale pointers are unused.
+ * value = code * scale.  Banks: w_up codes [E][F][H], w_down codes [E][H][F].
+ *   w_up_scale [E], w_down_scale [E]: one scale per expert tensor.
+ *   w_up_block, w_down_block: unused.
+ *
+ * MOE_FP8_B128 (bloomery page, section 3: the FP8 release's matrix
+ * normaliser maps scalar scales to FP8_B128; the 64-value tail of K = 1856):
+ * E4M3 codes with one fp32 scale per block of 128 values along K of each
+ * weight row; K zero-padded to Kp(K) = 128*ceil(K/128).  Banks: w_up codes
+ * [E][F][Kp(H)], w_down codes [E][H][Kp(F)] (zero codes past K).
+ *   w_up_scale [E][F][Kp(H)/128], w_down_scale [E][H][Kp(F)/128].
+ *   w_up_block, w_down_block: unused.
  *
  * MOE_NVFP4 (bloomery page, section 2: the NVFP4 release runs the experts
  * W4A4; the format is NVIDIA's NVFP4): E2M1 codes packed two per byte
@@ -95,23 +108,20 @@ typedef struct {
  * along the contraction dimension, one fp32 scale per tensor; real value =
  * e2m1(code) * e4m3(block scale) * tensor scale.  Block scales are stored
  * [rows][KSP] bytes with KSP = K/16 rounded up to a multiple of 16 (padding
- * zero; moe_quantize_nvfp4 writes this layout).  Weight banks: w_up codes
- * [E][F][H/2], w_up_block [E][F][KSP(H)]; w_down codes [E][H][F/2],
- * w_down_block [E][H][KSP(F)].  x and the ReLU^2 tensor are quantised inside
- * the layer with block scales taken at run time and the static tensor scales
- * x_scale and h_scale. */
-/* Scales of the quantised expert formats.  MOE_FP8_E4M3 and MOE_NVFP4: one
- * tensor scale per expert tensor.  MOE_FP8_B128: w_up_scale [E][F][Kp(H)/128]
- * and w_down_scale [E][H][Kp(F)/128], one per block of 128 values along K,
- * with the banks' codes [E][F][Kp(H)] and [E][H][Kp(F)], Kp(K) = 128*ceil(K/128)
- * (zero codes past K).  Activation scales are static in every format. */
+ * zero; moe_quantize_nvfp4 writes this layout).  Banks: w_up codes
+ * [E][F][H/2], w_down codes [E][H][F/2].
+ *   w_up_scale [E], w_down_scale [E]: the tensor scales.
+ *   w_up_block [E][F][KSP(H)], w_down_block [E][H][KSP(F)]: the block
+ *   scales, 16-byte aligned.
+ *   x and the ReLU^2 tensor are quantised inside the layer with block scales
+ *   taken at run time and the static tensor scales x_scale and h_scale. */
 typedef struct {
-    const float* w_up_scale;    /* [E] device: one (tensor) scale per expert up tensor */
-    const float* w_down_scale;  /* [E] device: one (tensor) scale per expert down tensor */
+    const float* w_up_scale;    /* device; shape per format (above) */
+    const float* w_down_scale;  /* device; shape per format (above) */
     float x_scale;              /* static (tensor) scale of the expert input activations */
     float h_scale;              /* static (tensor) scale of the ReLU^2 activations */
-    const uint8_t* w_up_block;  /* MOE_NVFP4: [E][F][KSP(H)] E4M3 block scales */
-    const uint8_t* w_down_block;/* MOE_NVFP4: [E][H][KSP(F)] E4M3 block scales */
+    const uint8_t* w_up_block;  /* MOE_NVFP4 only: [E][F][KSP(H)] E4M3 block scales */
+    const uint8_t* w_down_block;/* MOE_NVFP4 only: [E][H][KSP(F)] E4M3 block scales */
 } moe_quant_scales;
 typedef moe_quant_scales moe_fp8_scales;
 
@@ -156,14 +166,18 @@ moe_status moe_permute(const moe_dims* d, const int32_t* topk_idx, int32_t* coun
 /* Grouped expert FFN over the permuted rows:
  *   y_perm[r] = W_down[e] * relu(W_up[e] * x[perm_src[r] / K])^2,  e = expert of row r
  *   x [T][H] bf16; offsets [E+1] and perm_src [T*K] as from moe_permute;
- *   w_up [E][F][H], w_down [E][H][F] (bf16, or E4M3 codes with `scales`, or
- *   NVFP4 codes [E][F][H/2], [E][H][F/2] with `scales`);
+ *   w_up, w_down: the banks in the layout moe_quant_scales gives for the
+ *   format ([E][F][H] and [E][H][F] for bf16 and MOE_FP8_E4M3; [E][F][Kp(H)]
+ *   and [E][H][Kp(F)] for MOE_FP8_B128; [E][F][H/2] and [E][H][F/2] for
+ *   MOE_NVFP4);
  *   y_perm [T*K + T*Fs/F][H] bf16 out.
  * With a shared expert (d->Fs > 0): w_up_shared [Fs][H] and w_down_shared
  * [H][Fs] bf16 (both NULL when Fs = 0), and rows T*K + j*T + t of y_perm
  * receive chunk j of it for token t:
  *   W_down_s[:, jF:(j+1)F] * relu(W_up_s[jF:(j+1)F, :] * x[t])^2.
- * scales must be non-NULL for MOE_FP8_E4M3 and MOE_NVFP4.  Cited: bloomery page s.2 and
+ * scales must be non-NULL for MOE_FP8_E4M3, MOE_FP8_B128 and MOE_NVFP4, with the
+ * pointers moe_quant_scales names for the format; otherwise MOE_EINVAL (checked
+ * on the host before any launch, also for T = 0).  Cited: bloomery page s.2 and
  * s.3 (ungated ReLU^2 experts, up/down parts). */
 moe_status moe_expert_ffn(const moe_dims* d, const void* x, const int32_t* offsets,
                           const int32_t* perm_src, const void* w_up, const void* w_down,

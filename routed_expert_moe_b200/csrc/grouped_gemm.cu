@@ -35,6 +35,7 @@
 #include <cuda_fp8.h>
 
 #include "common.cuh"
+#include "internal.h"
 
 namespace moe {
 
@@ -363,13 +364,6 @@ static bool make_map_chunks(CUtensorMap* m, const void* base, int64_t rows, int6
                             int box_rows) {
     return make_map3(m, base, chunk, rows, n, n * chunk * 2, chunk * 2, box_rows);
 }
-
-struct GemmPlan {
-    int bn;              // max rows per schedule entry
-    int n_stages;
-    size_t smem_bytes;
-    int max_sched;       // schedule entries bound
-};
 
 GemmPlan gemm_plan(int64_t T, int K, int E) {
     GemmPlan p;

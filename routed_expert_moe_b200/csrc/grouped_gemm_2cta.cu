@@ -29,6 +29,7 @@
 #include <cuda_fp8.h>
 
 #include "common.cuh"
+#include "internal.h"
 
 namespace moe {
 
@@ -363,7 +364,7 @@ EncodeTiledFn encode2_fn() {
     return fn;
 }
 
-bool make_map2(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, bool fp8, int box_rows) {
+static bool make_map2(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, bool fp8, int box_rows) {
     EncodeTiledFn fn = encode2_fn();
     if (!fn) return false;
     const int es = fp8 ? 1 : 2;
@@ -377,7 +378,7 @@ bool make_map2(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, boo
 }
 
 template <bool FP8, bool UP>
-cudaError_t launch_pair(const Gemm2Maps& maps, const Gemm2Args& g, int64_t max_units, int num_sms, size_t smem,
+static cudaError_t launch_pair(const Gemm2Maps& maps, const Gemm2Args& g, int64_t max_units, int num_sms, size_t smem,
                         const DevCtx& ctx, cudaStream_t stream) {
     auto kfn = grouped_gemm_pair_kernel<FP8, UP>;
     cudaError_t err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -409,7 +410,7 @@ cudaError_t launch_pair(const Gemm2Maps& maps, const Gemm2Args& g, int64_t max_u
 }  // namespace
 
 // Stage bytes and ring depth of the pair kernel for token blocks of up to bn rows.
-size_t gemm_pair_smem(int bn, int* n_stages) {
+static size_t gemm_pair_smem(int bn, int* n_stages) {
     const int stage = P2_A_BYTES + (bn / 2) * P2_ROW_BYTES;
     int ns = (200 * 1024) / stage;
     if (ns > 8) ns = 8;

@@ -24,6 +24,7 @@
 #include <cuda_fp8.h>
 
 #include "common.cuh"
+#include "internal.h"
 
 namespace moe {
 

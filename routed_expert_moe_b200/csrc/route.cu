@@ -31,6 +31,7 @@
 #include <cuda_runtime.h>
 
 #include "common.cuh"
+#include "internal.h"
 
 namespace moe {
 
@@ -1101,13 +1102,6 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(NTH, 1)
 }
 
 // ----------------------------------------------------------------------------- host
-
-struct RouterPlan {
-    int S;
-    int nchunks;
-    int num_sms;
-    size_t p_bytes, xn_bytes, wn_bytes;
-};
 
 // Batch-size boundaries of the three router shapes, from CUDA-event timings
 // on B200 (H=2688, E=128, K=6): the expert-split clusters up to 256 tokens

@@ -23,22 +23,7 @@
 #include <cuda_runtime.h>
 
 #include "common.cuh"
-
-namespace moe {
-
-struct RouterPlan {
-    int S;
-    int nchunks;
-    size_t p_bytes, xn_bytes, wn_bytes;
-};
-RouterPlan router_plan(int64_t T, int H, int E, int num_sms);
-cudaError_t launch_route(const uint16_t* x, const uint16_t* wr, const float* bias, int64_t T, int H, int E, int K,
-                         int32_t* idx, float* w, double* P, double* xn2, double* wn2, const RouterPlan& plan,
-                         const DevCtx& ctx, cudaStream_t stream, void (*between)(cudaStream_t));
-moe_status internal_check_dims(const moe_dims* d);
-moe_status internal_device(DevCtx* ctx, int* num_sms);
-
-}  // namespace moe
+#include "internal.h"
 
 namespace {
 
@@ -80,30 +65,29 @@ extern "C" moe_status moe_route_static(const moe_dims* d, const void* x, const v
     if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(w_router)) % 16 != 0) return MOE_EINVAL;
     if (d->T == 0) return MOE_OK;
 
-    // the smallest plan (one split of the hidden dimension) must fit the array
-    moe::RouterPlan one;
-    one.S = 1;
-    one.nchunks = (d->H + 31) / 32;
-    one.p_bytes = (size_t)d->T * (size_t)d->E * sizeof(double);
-    one.xn_bytes = (size_t)d->T * sizeof(double);
-    one.wn_bytes = (size_t)d->E * sizeof(double);
-    if (scratch_bytes(one) > kRouteScratchBytes) return MOE_EWORKSPACE;
+    // the smallest plan (one split of the hidden dimension) must fit the array; this is
+    // checked before any device call
+    moe::RouterPlan plan{};
+    const auto resize = [&](int S) {
+        plan.S = S;
+        plan.p_bytes = (size_t)S * (size_t)d->T * (size_t)d->E * sizeof(double);
+        plan.xn_bytes = (size_t)S * (size_t)d->T * sizeof(double);
+        plan.wn_bytes = (size_t)S * (size_t)d->E * sizeof(double);
+    };
+    resize(1);
+    if (scratch_bytes(plan) > kRouteScratchBytes) return MOE_EWORKSPACE;
 
     moe::DevCtx ctx;
     int sms = 0;
     if ((s = moe::internal_device(&ctx, &sms)) != MOE_OK) return s;
-    void* base = nullptr;
-    if ((s = scratch_address(&base)) != MOE_OK) return s;
 
     // the library's usual split of the hidden dimension, reduced until it fits
-    moe::RouterPlan plan = moe::router_plan(d->T, d->H, d->E, sms);
-    while (plan.S > 1 && scratch_bytes(plan) > kRouteScratchBytes) {
-        plan.S -= 1;
-        plan.p_bytes = (size_t)plan.S * d->T * d->E * sizeof(double);
-        plan.xn_bytes = (size_t)plan.S * d->T * sizeof(double);
-        plan.wn_bytes = (size_t)plan.S * d->E * sizeof(double);
-    }
-    if (scratch_bytes(plan) > kRouteScratchBytes) plan = one;
+    plan = moe::router_plan(d->T, d->H, d->E, sms);
+    while (plan.S > 1 && scratch_bytes(plan) > kRouteScratchBytes) resize(plan.S - 1);
+    if (scratch_bytes(plan) > kRouteScratchBytes) return MOE_EWORKSPACE;
+
+    void* base = nullptr;
+    if ((s = scratch_address(&base)) != MOE_OK) return s;
 
     unsigned char* b = static_cast<unsigned char*>(base);
     double* P = reinterpret_cast<double*>(b);

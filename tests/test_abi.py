@@ -103,6 +103,29 @@ def test_null_and_missing_arguments(moe):
     assert lib.moe_set_stage_events(None, 3) == moe.MOE_EINVAL
 
 
+def test_quantised_formats_need_their_scales(moe):
+    """Every quantised format checks its scales on the host before any launch, even for an
+    empty batch, where no other pointer is needed."""
+    lib = moe.raw_library()
+    fake = ctypes.c_void_p(4096)
+    for kw in (dict(fp8=True), dict(fp8_b128=True), dict(nvfp4=True)):
+        d = moe.dims(0, 2688, 128, 6, 1856, **kw)
+        assert lib.moe_expert_ffn(ctypes.byref(d), *([None] * 7), None, None, None, 0, None) == moe.MOE_EINVAL
+        sc = moe.MoeFp8Scales(None, fake, 1.0, 1.0, fake, fake)          # no up-projection scales
+        assert lib.moe_expert_ffn(ctypes.byref(d), *([None] * 7), ctypes.byref(sc), None, None, 0,
+                                  None) == moe.MOE_EINVAL
+        sc = moe.MoeFp8Scales(fake, fake, 1.0, 0.0, fake, fake)          # h_scale must be > 0
+        assert lib.moe_expert_ffn(ctypes.byref(d), *([None] * 7), ctypes.byref(sc), None, None, 0,
+                                  None) == moe.MOE_EINVAL
+        sc = moe.MoeFp8Scales(fake, fake, 1.0, 1.0, fake, fake)
+        assert lib.moe_expert_ffn(ctypes.byref(d), *([None] * 7), ctypes.byref(sc), None, None, 0,
+                                  None) == moe.MOE_OK
+    d = moe.dims(0, 2688, 128, 6, 1856, nvfp4=True)                       # NVFP4 also needs its block scales
+    sc = moe.MoeFp8Scales(fake, fake, 1.0, 1.0, None, fake)
+    assert lib.moe_expert_ffn(ctypes.byref(d), *([None] * 7), ctypes.byref(sc), None, None, 0,
+                              None) == moe.MOE_EINVAL
+
+
 def test_empty_batch_is_ok_without_a_device(moe):
     lib = moe.raw_library()
     d = bad(moe, T=0)

@@ -77,3 +77,31 @@ def test_static_scratch_router_rejects_batches_beyond_its_array(moe):
                                             ctypes.c_void_p(x.data_ptr()), None, ctypes.c_void_p(out.data_ptr()),
                                             ctypes.c_void_p(out.data_ptr()), None)
     assert rc == moe.MOE_EWORKSPACE
+
+
+@pytest.mark.parametrize("T,split", [(1200, 0), (8000, 1)])
+def test_static_scratch_router_at_large_batches(moe, T, split):
+    """Batches whose usual split of the hidden dimension does not fit the array.
+
+    T = 1200 takes the two-kernel router, whose usual plan (7 splits, 8.6 MB of
+    partial logits) is cut down until it fits; T = 8000, near the 8127 limit,
+    is forced onto the two-kernel router so that one split's partials fill
+    most of the array.  Indices bit for bit against moe_route under the same
+    router shape, weights within 1e-5, two calls in a row."""
+    import synth
+    H, E, K, F = 2688, 128, 6, 1856
+    stream = torch.cuda.current_stream().cuda_stream
+    x = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
+    wr = torch.empty(E, H, dtype=torch.bfloat16, device="cuda")
+    synth.normal_bf16_device(synth.key(11, synth.T_X, 0), x.numel(), W.SIGMA_X, x.data_ptr(), stream)
+    synth.normal_bf16_device(synth.key(11, synth.T_WR, 0), wr.numel(), W.SIGMA_W, wr.data_ptr(), stream)
+    dims = moe.dims(T, H, E, K, F)
+    moe.debug_set(5, split)
+    try:
+        ref_idx, ref_w = _route_with_workspace(moe, dims, x, wr, None, T, K)
+        for _ in range(2):
+            idx, wt = _route_static_abi(moe, dims, x, wr, None, T, K)
+            assert np.array_equal(idx, ref_idx)
+            assert np.max(np.abs(wt - ref_w)) <= 1e-5
+    finally:
+        moe.debug_set(5, 0)
