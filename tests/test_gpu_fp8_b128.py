@@ -98,3 +98,48 @@ def test_b128_expired_wait_is_reported(moe):
         moe.debug_set(1, 0)
     moe.forward(dims, dev_bf16(h["x"]), dev_bf16(h["wr"]), None, cu, cd, out, ws, scales=sc)
     moe.check_device_error()
+
+
+def test_b128_forward_parity_prefill_shape(moe):
+    """The prefill workload with FP8_B128 experts (T = 4096, 128 experts, ~192 rows per
+    expert, so every expert's rows span several 64-row tiles): routing bit for bit on every
+    token, the output on sampled tokens within FP8_TOL.  The banks are made and quantised on
+    the device from the seeded bf16 masters; the oracle quantises the used experts' masters
+    itself (the quantiser is bit-exact, above)."""
+    import synth
+    w = W.WORKLOADS[10]
+    sx, sh = W.fp8_b128_scales(w)
+    stream = torch.cuda.current_stream().cuda_stream
+    banks = []
+    for tid, shape in ((synth.T_WUP, (w.E, w.F, w.H)), (synth.T_WDOWN, (w.E, w.H, w.F))):
+        t = torch.empty(*shape, dtype=torch.bfloat16, device="cuda")
+        synth.normal_bf16_device(synth.key(w.seed, tid, 0), t.numel(), W.SIGMA_W, t.data_ptr(), stream)
+        n, rows, K = shape
+        kp = moe.b128_kp(K)
+        codes = torch.empty(n, rows, kp, dtype=torch.uint8, device="cuda")
+        sc = torch.empty(n, rows, kp // 128, dtype=torch.float32, device="cuda")
+        moe.quantize_fp8_b128(t, codes, sc)
+        banks.append((codes, sc))
+        del t
+    (cu, su), (cd, sd) = banks
+    x, wr = W.host_x(w), W.host_router(w)
+    dims = moe.dims(w.T, w.H, w.E, w.K, w.F, fp8_b128=True)
+    ws = moe.alloc_workspace(dims)
+    out = torch.empty(w.T, w.H, dtype=torch.bfloat16, device="cuda")
+    idx = torch.empty(w.T, w.K, dtype=torch.int32, device="cuda")
+    moe.forward(dims, dev_bf16(x), dev_bf16(wr), None, cu, cd, out, ws,
+                scales=moe.fp8_scales(su, sd, float(sx), float(sh)), topk_idx=idx)
+    moe.check_device_error()
+
+    _, ridx, _ = oracle.route(x, wr, None, w.K)
+    assert np.array_equal(idx.cpu().numpy(), ridx)
+    rng = np.random.default_rng(10)
+    tok = np.unique(np.concatenate([[0, w.T - 1], rng.choice(w.T, size=6, replace=False)]))
+    used = sorted(set(ridx[tok].reshape(-1).tolist()))
+    slot = -np.ones(w.E, np.int32)
+    slot[used] = np.arange(len(used))
+    bu = oracle.quantize_fp8_b128(W.host_w_up(w, experts=used))
+    bd = oracle.quantize_fp8_b128(W.host_w_down(w, experts=used))
+    r = oracle.moe_layer_fp8_b128(x, wr, None, bu, bd, sx, sh, w.K, w.H, w.F, tokens=tok, slot=slot)
+    assert np.array_equal(r["idx"], ridx[tok])
+    assert rel_err(host_f64(out)[tok], r["out"]) <= FP8_TOL
