@@ -744,6 +744,123 @@ def run_native(args):
         dist.destroy_process_group()
 
 
+# --------------------------------------------------------------------------- expert parallelism
+
+class EpLayer:
+    """The layer split by expert over the ranks (routed_expert_moe_b200.ep): rank p owns experts
+    [p*E/N, (p+1)*E/N) and routes its own batch; rows cross ranks in two all-to-alls."""
+
+    def __init__(self, wl, device, n_batches=4):
+        import torch
+        import torch.distributed as dist
+        import synth
+        from routed_expert_moe_b200.ep import ExpertParallelLayer
+        from synth import workloads as W
+        self.wl, self.device = wl, device
+        rank = dist.get_rank() if dist.is_initialized() else 0
+        bf = torch.bfloat16
+        stream = torch.cuda.current_stream().cuda_stream
+        self.layer = ExpertParallelLayer(wl.H, wl.E, wl.K, wl.F) if dist.is_initialized() else None
+        E_loc = self.layer.E_loc if self.layer else wl.E
+        lo = rank * E_loc
+        banks = []
+        for tid, shape in ((synth.T_WUP, (wl.E, wl.F, wl.H)), (synth.T_WDOWN, (wl.E, wl.H, wl.F))):
+            full = torch.empty(*shape, dtype=bf, device=device)
+            synth.normal_bf16_device(synth.key(wl.seed, tid, 0), full.numel(), W.SIGMA_W, full.data_ptr(), stream)
+            banks.append(full[lo:lo + E_loc].clone())
+            del full
+        self.wu, self.wd = banks
+        self.wr = torch.empty(wl.E, wl.H, dtype=bf, device=device)
+        synth.normal_bf16_device(synth.key(wl.seed, synth.T_WR, 0), self.wr.numel(), W.SIGMA_W, self.wr.data_ptr(),
+                                 stream)
+        self.xs = []
+        for i in range(n_batches):   # each rank its own token batches
+            x = torch.empty(wl.T, wl.H, dtype=bf, device=device)
+            synth.normal_bf16_device(synth.key(wl.seed, synth.T_X, 16 * rank + i), x.numel(), W.SIGMA_X,
+                                     x.data_ptr(), stream)
+            self.xs.append(x)
+        self.out = torch.empty(wl.T, wl.H, dtype=bf, device=device)
+        torch.cuda.synchronize(device)
+
+    def step(self, i, x=None, out=None):
+        self.layer.forward(self.xs[i % len(self.xs)] if x is None else x, self.wr, None, self.wu, self.wd,
+                           self.out if out is None else out)
+
+
+# kernels of one expert-parallel pass beyond those of moe_forward: the regrouping, the owner's
+# tile schedule, and the gather that returns the outputs in arrival order
+EP_EXTRA_LAUNCHES = 3
+
+
+def ep_line(ws, wl, steps, warmup, ms, e2e_ms, clocks, launches_per_step):
+    """The JSON line of the expert-parallel mode: every rank processed wl.T tokens per step;
+    ms and e2e_ms are the max over ranks."""
+    nb = wl.T * wl.H * 2
+    return {"metric": METRIC, "value": job_value(ws, wl.T, steps, ms), "unit": UNIT, "n_gpus": ws, "steps": steps,
+            "warmup": warmup, "ms_per_step": ms / steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic: seeded N(0,1) activations, N(0,0.02) router/expert weights (bf16)",
+            "config": {"workload": wl.name, "T_per_rank": wl.T, "H": wl.H, "E": wl.E, "K": wl.K, "F": wl.F,
+                       "parallelism": f"ep{ws} ({wl.E // ws} experts per rank, two NCCL all-to-alls per pass)",
+                       "l2": "inputs larger than L2: each rank's experts stream from HBM every step"},
+            "e2e": {"value": job_value(ws, wl.T, steps, e2e_ms), "unit": UNIT,
+                    "h2d_bytes_per_step": nb, "d2h_bytes_per_step": nb},
+            "gpu_launches": launches_per_step * steps, "clocks": clocks}
+
+
+def run_ep(args):
+    """--ep: the expert-parallel split under torchrun (one rank per GPU, NCCL)."""
+    import datetime
+    import torch
+    import torch.distributed as dist
+    from synth import workloads as W
+
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    os.environ.setdefault("NCCL_NVLS_ENABLE", "0")
+    if "MASTER_ADDR" not in os.environ:      # a single process without torchrun
+        import socket
+        so = socket.socket()
+        so.bind(("127.0.0.1", 0))
+        os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(so.getsockname()[1]), RANK="0", WORLD_SIZE="1")
+        so.close()
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    device = torch.device("cuda", local)
+    barrier = lambda: dist.barrier()
+    wl = W.WORKLOADS[WORKLOADS[args.workload]]
+    layer = EpLayer(wl, device)
+    sampler = ClockSampler(None)
+    sampler.start()
+    time.sleep(0.3)
+    ms = timed_loop(layer, args.steps, args.warmup, barrier)
+    clocks = sampler.stop()
+    ms = reduce_max(ms, dist, device)
+    # end to end: this rank's batch from pinned host memory, its output back, every step
+    hx = layer.xs[0].cpu().pin_memory()
+    hout = torch.empty(wl.T, wl.H, dtype=torch.bfloat16, pin_memory=True)
+    dx = torch.empty_like(layer.xs[0])
+    for i in range(args.warmup):
+        dx.copy_(hx, non_blocking=True)
+        layer.step(i, x=dx)
+        hout.copy_(layer.out, non_blocking=True)
+    barrier()
+    torch.cuda.synchronize()
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0.record()
+    for i in range(args.steps):
+        dx.copy_(hx, non_blocking=True)
+        layer.step(i, x=dx)
+        hout.copy_(layer.out, non_blocking=True)
+    s1.record()
+    torch.cuda.synchronize()
+    e2e_ms = reduce_max(s0.elapsed_time(s1), dist, device)
+    if rank == 0:
+        import routed_expert_moe_b200 as moe
+        launches = moe.forward_launches(moe.dims(wl.T, wl.H, wl.E, wl.K, wl.F)) + EP_EXTRA_LAUNCHES
+        print(json.dumps(ep_line(ws, wl, args.steps, args.warmup, ms, e2e_ms, clocks, launches)), flush=True)
+    dist.destroy_process_group()
+
+
 # --------------------------------------------------------------------------- reference arm
 
 def run_reference(args):
@@ -786,6 +903,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--gemm", choices=["single", "pair"], default="single",
                     help="grouped GEMM on single CTAs, or on CTA pairs for tiles of more than 64 tokens")
+    ap.add_argument("--ep", action="store_true",
+                    help="time the expert-parallel split (experts divided over the ranks) instead of replicas")
     ap.add_argument("--pdl", choices=["on", "off"], default="on",
                     help="programmatic dependent launch between the layer's kernels")
     args = ap.parse_args(argv)
@@ -793,6 +912,8 @@ def main(argv=None):
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.ep:
+        run_ep(args)
     else:
         run_native(args)
 

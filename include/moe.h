@@ -219,6 +219,24 @@ moe_status moe_forward(const moe_dims* d, const void* x, const void* w_router, c
 moe_status moe_gather_rows(int64_t rows, int64_t src_rows, int32_t H, int32_t K, const void* x,
                            const int32_t* perm_src, void* out, void* stream);
 
+/* Regrouping of the rows an expert's owner receives in an expert-parallel
+ * exchange (the experts split over W ranks, E_loc = E / W each).  Received
+ * rows arrive source-major: from rank 0 its rows for local experts 0, 1, ...,
+ * then rank 1, ...  The grouped layout moe_expert_ffn reads (with K = 1) is
+ * expert-major, then source rank, then arrival order.
+ *   recv_counts [W][E_loc] int64 (device): rows from rank p for local expert e;
+ *   R = the sum of recv_counts (the received rows);
+ *   offsets [E_loc + 1] int32 out: the grouped layout's expert offsets;
+ *   perm [R] int32 out: grouped row g holds received row perm[g];
+ *   inv [R] int32 out: received row i sits in grouped row inv[i].
+ * W * E_loc <= 256.  Counts that are negative or do not sum to R set
+ * MOE_EINDEX in the device error word and leave the outputs unwritten.  The
+ * pages say nothing about several GPUs; this serves the split of the grouped
+ * expert products by owner (audio.cpp model page, "CPU weight offload":
+ * grouped expert matrix multiplication). */
+moe_status moe_ep_regroup(int32_t W, int32_t E_loc, int64_t R, const int64_t* recv_counts, int32_t* offsets,
+                          int32_t* perm, int32_t* inv, void* stream);
+
 /* Per-tensor E4M3 quantisation of n_tensors bf16 tensors of tensor_elems
  * elements each (an expert bank): scale[i] = amax|W_i| / 448 (1 for an
  * all-zero tensor), codes = e4m3_rne_satfinite(W / scale[i]).

@@ -56,6 +56,7 @@ _SIG = {
                                    _P, _P, _P, _S, _P]),
     "moe_gather_rows": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, _P, _P,
                                        _P, _P]),
+    "moe_ep_regroup": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int32, ctypes.c_int64, _P, _P, _P, _P, _P]),
     "moe_quantize_fp8": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int64, _P, _P, _P, _P]),
     "moe_quantize_nvfp4": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, _P, _P, _P, _P, _P]),
     "moe_quantize_fp8_b128": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, _P, _P, _P, _P]),
@@ -218,6 +219,14 @@ def gather_rows(x, perm_src, out, K=1, stream=None):
     rows, H = out.shape[0], x.shape[1]
     _check(_lib.moe_gather_rows(rows, x.shape[0], H, int(K), _ptr(x), _ptr(perm_src), _ptr(out), _stream(stream)),
            "moe_gather_rows")
+
+
+def ep_regroup(recv_counts, offsets, perm, inv, stream=None):
+    """Grouped layout of the rows an expert's owner received: recv_counts [W, E_loc] int64 (device),
+    offsets [E_loc + 1], perm [R], inv [R] int32 out (R = recv_counts.sum())."""
+    W, E_loc = recv_counts.shape
+    _check(_lib.moe_ep_regroup(int(W), int(E_loc), perm.numel(), _ptr(recv_counts), _ptr(offsets), _ptr(perm),
+                               _ptr(inv), _stream(stream)), "moe_ep_regroup")
 
 
 def quantize_fp8(src, codes, scales, stream=None):

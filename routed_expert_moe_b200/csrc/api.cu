@@ -137,16 +137,18 @@ struct ForwardWs {
 };
 
 // Plan of the expert FFN: one tile schedule for every expert dtype (FP8_B128
-// caps a tile at 64 token rows: its epilogue keeps a tile's sums in registers),
+// caps a tile at 64 token rows: its epilogue keeps a tile's sums in registers;
+// NVFP4 at 224: its accumulators share TMEM with the scale factors),
 // plus the shared expert's entries (ns chunks of T rows, cut into tiles of at
 // most bn).
 GemmPlan ffn_plan(const moe_dims* d) {
     GemmPlan gp = gemm_plan(d->T, d->K, d->E);
-    if (d->expert_dtype == MOE_FP8_B128 && gp.bn > 64) {
+    const int cap = d->expert_dtype == MOE_FP8_B128 ? 64 : d->expert_dtype == MOE_NVFP4 ? kFp4MaxTileRows : 0;
+    if (cap > 0 && gp.bn > cap) {
         const int64_t rows = d->T * d->K;
         const int64_t nonempty = d->E < rows ? d->E : rows;
-        gp.bn = 64;
-        gp.max_sched = (int)(nonempty + (rows + 63) / 64);
+        gp.bn = cap;
+        gp.max_sched = (int)(nonempty + (rows + cap - 1) / cap);
     }
     gp.max_sched += n_shared(d) * (int)((d->T + gp.bn - 1) / gp.bn);
     return gp;
@@ -503,6 +505,17 @@ moe_status moe_gather_rows(int64_t rows, int64_t src_rows, int32_t H, int32_t K,
     if (s != MOE_OK) return s;
     return cuda_status(launch_gather(static_cast<const uint16_t*>(x), perm_src, rows, rows, K, src_rows, H, out,
                                      false, 1.0f, dev->num_sms, make_ctx(dev), static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_ep_regroup(int32_t W, int32_t E_loc, int64_t R, const int64_t* recv_counts, int32_t* offsets,
+                          int32_t* perm, int32_t* inv, void* stream) {
+    if (W < 1 || E_loc < 1 || (int64_t)W * E_loc > 256 || R < 0 || R >= ((int64_t)1 << 31)) return MOE_EINVAL;
+    if (!recv_counts || !offsets || (R > 0 && (!perm || !inv))) return MOE_EINVAL;
+    DeviceInfo* dev = nullptr;
+    moe_status s = device_setup(&dev);
+    if (s != MOE_OK) return s;
+    return cuda_status(launch_ep_regroup(recv_counts, W, E_loc, R, offsets, perm, inv, make_ctx(dev),
+                                         static_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_quantize_fp8(int64_t n_tensors, int64_t tensor_elems, const void* src, uint8_t* codes,

@@ -79,6 +79,13 @@ cudaError_t launch_quantize(int64_t n_tensors, int64_t elems, const uint16_t* sr
                             float* scales, int num_sms, cudaStream_t stream);
 
 
+cudaError_t launch_ep_regroup(const int64_t* recv_counts, int W, int E_loc, int64_t R, int32_t* offsets,
+                              int32_t* perm, int32_t* inv, const DevCtx& ctx, cudaStream_t stream);
+
+// Token rows per schedule entry of the NVFP4 grouped GEMM: its two TMEM
+// accumulators of this many columns leave room for the scale factors.
+constexpr int kFp4MaxTileRows = 224;
+
 // Sizes the plans must keep: a plan is passed by value and by reference
 // between files, so a field added in one place shows up as a size change here.
 static_assert(sizeof(RouterPlan) == 40, "RouterPlan layout changed: update every user");

@@ -176,14 +176,41 @@ __global__ void __launch_bounds__(256) nvfp4_gather_kernel(const uint16_t* __res
 
 // ----------------------------------------------------------------------------- grouped GEMM
 
-constexpr int FG_THREADS = 320;            // 10 warps
-constexpr int FG_BM = 128;                 // weight rows per unit
-constexpr int FG_KR = 256;                 // K values per raw (packed) stage
-constexpr int FG_KF = 64;                  // K values per fp16 stage (128-byte rows)
-constexpr int FG_A_RAW = FG_BM * FG_KR / 2;   // 16 KB of codes
-constexpr int FG_A_SC = FG_BM * 16;           // 2 KB of block scales (16 blocks x 128 rows)
-constexpr int FG_A_F16 = FG_BM * 128;         // 16 KB
+// The tensor cores multiply NVFP4 operands directly: tcgen05.mma
+// kind::mxf4nvf4 with block scaling (scale_vec::4X: one E4M3 scale per 16
+// values along K, four per row per instruction of K = 64).  Each MMA reads its
+// scale factors from TMEM; tcgen05.cp copies them there from 512-byte atoms in
+// shared memory.  An atom holds the four scales of one K block of 64 for 128
+// rows, row r = r0 + 32 * r1 at byte 16 * r0 + 4 * r1 (+ the scale index
+// 0..3); the copy (32x128b.warpx4) replicates its 32 x 16 bytes into the four
+// TMEM lane quadrants, so that the MMA finds row r's scales in lane r,
+// column r / 32 of the atom's four columns (B: the same layout over its N
+// rows, one atom per 128 rows).  The TMA brings the scales in row-major, 16
+// bytes per row per stage, and four "scale" warps rearrange them into atoms.
+//
+// Roles (320 threads):
+//   warp 0      TMA producer: per stage of 256 K values the weight block's
+//               codes (128 rows x 128 bytes, 128-byte swizzle) and scales
+//               (128 x 16 bytes), the token rows' codes and scales;
+//   warp 1      TMEM allocator; one lane copies each stage's atoms to TMEM and
+//               issues the four block-scaled MMAs into one of two accumulators;
+//   warps 2..5  epilogue: tensor scales, ReLU^2 and the NVFP4 quantisation of
+//               H (up) or the bf16 store (down); warp w reads lanes 32*(w%4)..;
+//   warps 6..9  scale warps: thread i writes row i's (and row i + 128's)
+//               scales into the stage's atoms, zero for rows a tile lacks.
+constexpr int FG_THREADS = 320;
+constexpr int FG_BM = 128;                    // weight rows per unit (MMA M)
+constexpr int FG_KR = 256;                    // K values per stage (128 code bytes per row)
+constexpr int FG_A_CODES = FG_BM * 128;       // 16 KB
+constexpr int FG_A_SC = FG_BM * 16;           // 2 KB
+constexpr int FG_ATOM = 512;                  // scales of one K block of 64 for 128 rows
 constexpr int FG_TMEM_COLS = 512;
+constexpr int FG_ACC_COLS = 224;              // two accumulators of up to 224 token columns
+constexpr int FG_SFA_COL = 2 * FG_ACC_COLS;   // A scales: 4 K blocks x 4 columns
+constexpr int FG_SFB_COL = FG_SFA_COL + 16;   // B scales: 4 K blocks x 8 columns (two atoms)
+constexpr int FG_BN_MAX = FG_ACC_COLS;        // token rows per schedule entry
+static_assert(FG_BN_MAX == kFp4MaxTileRows, "NVFP4 tile rows");
+static_assert(FG_SFB_COL + 32 <= FG_TMEM_COLS, "TMEM columns");
 
 struct Fp4Args {
     const int4* sched;
@@ -191,10 +218,10 @@ struct Fp4Args {
     int m_blocks;
     int Nout;
     int Kdim;
-    int k_raw;               // ceil(K / 256)
-    int k_f16;               // ceil(K / 64)
-    int nr, nf;              // ring depths
-    int bn;                  // max rows per schedule entry
+    int k_stages;            // ceil(K / 256)
+    int ns;                  // ring depth
+    int bn;                  // max rows per schedule entry (<= FG_BN_MAX)
+    int stage_bytes;
     const float* w_tscale;   // [E]
     float in_tscale;         // x (up) or H (down) tensor scale
     float out_tscale;        // H tensor scale (up)
@@ -210,55 +237,47 @@ struct Fp4Maps {
     CUtensorMap bs128, bs64, bs16;   // activation block scales
 };
 
-__device__ __forceinline__ void e2m1x8_to_f16(uint32_t packed, uint32_t (&out)[4]) {
-    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-        "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
-        : "=r"(out[0]), "=r"(out[1]), "=r"(out[2]), "=r"(out[3]) : "r"(packed));
-}
-
-__device__ __forceinline__ uint32_t e4m3_pair_f16(uint32_t code) {
-    uint32_t r;
-    const uint16_t two = (uint16_t)(code * 0x0101u);
-    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(two));
-    return r;
-}
-
-__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
-    uint32_t r;
-    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-    return r;
-}
-
-// One row of one fp16 stage: 64 values (32 code bytes at chunks 2*sub, 2*sub+1 of a
-// 128-byte-swizzled raw row; 4 scale bytes) -> 128 bytes into a 128-byte-swizzled fp16 row.
-// Scales of blocks at or beyond nb read as zero.
-__device__ __forceinline__ void convert_row(const uint8_t* raw_row, const uint8_t* sc_row, uint8_t* f16_row, int row,
-                                            int sub, int kb0, int nb) {
-    const int sw = row & 7;
-    const uint4 c0 = *reinterpret_cast<const uint4*>(raw_row + 16 * ((2 * sub) ^ sw));
-    const uint4 c1 = *reinterpret_cast<const uint4*>(raw_row + 16 * ((2 * sub + 1) ^ sw));
-    const uint32_t scw = *reinterpret_cast<const uint32_t*>(sc_row + 4 * sub);
-    const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-#pragma unroll
-    for (int blk = 0; blk < 4; ++blk) {
-        uint32_t sc = (scw >> (8 * blk)) & 0xFFu;
-        if (kb0 + blk >= nb) sc = 0;
-        const uint32_t s2 = e4m3_pair_f16(sc);
-        uint32_t h[8];
-        uint32_t t[4];
-        e2m1x8_to_f16(words[2 * blk], t);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) h[i] = hmul2(t[i], s2);
-        e2m1x8_to_f16(words[2 * blk + 1], t);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) h[4 + i] = hmul2(t[i], s2);
-        *reinterpret_cast<uint4*>(f16_row + 16 * ((2 * blk) ^ sw)) = make_uint4(h[0], h[1], h[2], h[3]);
-        *reinterpret_cast<uint4*>(f16_row + 16 * ((2 * blk + 1) ^ sw)) = make_uint4(h[4], h[5], h[6], h[7]);
+// Byte offsets inside one ring stage (codes first: their regions start on 1024-byte boundaries).
+struct Fp4Stage {
+    int b_codes, a_sc, b_sc, a_atoms, b_atoms, nbat, bytes;
+    __host__ __device__ explicit Fp4Stage(int bn) {
+        nbat = bn > 128 ? 2 : 1;
+        b_codes = FG_A_CODES;
+        a_sc = b_codes + bn * 128;
+        b_sc = a_sc + FG_A_SC;
+        a_atoms = (b_sc + bn * 16 + 127) & ~127;
+        b_atoms = a_atoms + 4 * FG_ATOM;
+        bytes = (b_atoms + 4 * nbat * FG_ATOM + 1023) & ~1023;
     }
+};
+
+// No-swizzle K-major descriptor of one 512-byte scale atom (32 rows of 16 bytes:
+// core matrices of 8 rows, 128 bytes apart), the source of tcgen05.cp.
+__device__ __forceinline__ uint64_t atom_desc(uint32_t smem_addr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((smem_addr & 0x3FFFFu) >> 4);
+    d |= (uint64_t)(128u >> 4) << 16;
+    d |= (uint64_t)(128u >> 4) << 32;
+    d |= (uint64_t)1u << 46;
+    return d;
+}
+
+__device__ __forceinline__ void tmem_cp_atom(uint32_t taddr, uint64_t desc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
+}
+
+// Instruction descriptor of the block-scaled MMA: E2M1 A and B (K-major), UE4M3 scales,
+// fp32 accumulate, M x N.
+__host__ __device__ __forceinline__ uint32_t fp4_idesc(int M, int N) {
+    return (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_fp4(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t sfa,
+                                        uint32_t sfb, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n"
+        ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb));
 }
 
 template <bool UP>
@@ -267,19 +286,13 @@ __global__ void __launch_bounds__(FG_THREADS, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
-    const int NR = g.nr, NF = g.nf;
-    const int b_raw = g.bn * 128, b_sc = g.bn * 16, b_f16 = g.bn * 128;
-    // codes first, then scales; every stage starts on a 1024-byte boundary (128-byte swizzle atoms)
-    const int raw_bytes = (FG_A_RAW + b_raw + FG_A_SC + b_sc + 1023) & ~1023;
-    const int f16_bytes = FG_A_F16 + b_f16;
-    uint8_t* raw = smem;
-    uint8_t* f16 = raw + (size_t)NR * raw_bytes;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(f16 + (size_t)NF * f16_bytes);
-    uint64_t* raw_full = bars;
-    uint64_t* raw_empty = raw_full + NR;
-    uint64_t* f16_full = raw_empty + NR;
-    uint64_t* f16_empty = f16_full + NF;
-    uint64_t* tfull = f16_empty + NF;
+    const int NS = g.ns;
+    const Fp4Stage L(g.bn);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)NS * L.bytes);
+    uint64_t* full = bars;             // the stage's TMA bytes have landed
+    uint64_t* sfready = full + NS;     // its scale atoms are written (128 scale threads)
+    uint64_t* empty = sfready + NS;    // its MMAs are complete
+    uint64_t* tfull = empty + NS;
     uint64_t* tempty = tfull + 2;
     uint64_t* drain = tempty + 2;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(drain + 1);
@@ -287,13 +300,10 @@ __global__ void __launch_bounds__(FG_THREADS, 1)
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     if (threadIdx.x == 0) {
-        for (int s = 0; s < NR; ++s) {
-            mbar_init(smem_u32(&raw_full[s]), 1);
-            mbar_init(smem_u32(&raw_empty[s]), 128);   // every converter thread
-        }
-        for (int s = 0; s < NF; ++s) {
-            mbar_init(smem_u32(&f16_full[s]), 128);
-            mbar_init(smem_u32(&f16_empty[s]), 1);
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(smem_u32(&full[s]), 1);
+            mbar_init(smem_u32(&sfready[s]), 128);
+            mbar_init(smem_u32(&empty[s]), 1);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(smem_u32(&tfull[a]), 1);
@@ -311,7 +321,6 @@ __global__ void __launch_bounds__(FG_THREADS, 1)
     pdl_enter();
 
     const int n_units = (*g.n_sched) * g.m_blocks;
-    const int nbk = g.Kdim / 16;   // valid blocks along K
 
     if (warp == 0) {
         // ---------------------------------------------------------------- producer
@@ -329,38 +338,37 @@ __global__ void __launch_bounds__(FG_THREADS, 1)
                 const int n16 = (sc.z + 15) / 16;
                 const int n128 = n16 / 8, n64 = (n16 % 8) / 4, r16 = n16 % 4;
                 const int arows = a_full ? 128 : 64;
-                const uint32_t bytes = (uint32_t)(arows * 128 + arows * 16 + n16 * 16 * 128 + n16 * 16 * 16);
+                const uint32_t bytes = (uint32_t)(arows * (128 + 16) + n16 * 16 * (128 + 16));
                 const int a_y = sc.x * g.Nout + mb * FG_BM;
-                for (int kr = 0; kr < g.k_raw; ++kr) {
-                    if (!mbar_wait(smem_u32(&raw_empty[stage]), phase ^ 1u, ctx, abort_flag)) {
+                for (int ks = 0; ks < g.k_stages; ++ks) {
+                    if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, ctx, abort_flag)) {
                         ok = false;
                         break;
                     }
-                    const uint32_t fb = smem_u32(&raw_full[stage]);
+                    const uint32_t fb = smem_u32(&full[stage]);
                     mbar_arrive_expect_tx(fb, bytes);
                     if (withhold) {
                         withhold = false;   // this stage never completes: the consumers' waits expire
                     } else {
-                        uint8_t* st = raw + (size_t)stage * raw_bytes;
-                        const uint32_t a_c = smem_u32(st), b_c = smem_u32(st + FG_A_RAW);
-                        const uint32_t a_s = smem_u32(st + FG_A_RAW + b_raw), b_s = smem_u32(st + FG_A_RAW + b_raw + FG_A_SC);
-                        tma_load_2d(a_c, a_full ? &maps.a128 : &maps.a64, fb, kr * 128, a_y, pol_w);
-                        tma_load_2d(a_s, a_full ? &maps.as128 : &maps.as64, fb, kr * 16, a_y, pol_w);
+                        const uint32_t st = smem_u32(smem + (size_t)stage * L.bytes);
+                        const uint32_t b_c = st + L.b_codes, a_s = st + L.a_sc, b_s = st + L.b_sc;
+                        tma_load_2d(st, a_full ? &maps.a128 : &maps.a64, fb, ks * 128, a_y, pol_w);
+                        tma_load_2d(a_s, a_full ? &maps.as128 : &maps.as64, fb, ks * 16, a_y, pol_w);
                         int row = 0;
                         for (int j = 0; j < n128; ++j, row += 128) {
-                            tma_load_2d(b_c + row * 128, &maps.b128, fb, kr * 128, sc.y + row, pol_x);
-                            tma_load_2d(b_s + row * 16, &maps.bs128, fb, kr * 16, sc.y + row, pol_x);
+                            tma_load_2d(b_c + row * 128, &maps.b128, fb, ks * 128, sc.y + row, pol_x);
+                            tma_load_2d(b_s + row * 16, &maps.bs128, fb, ks * 16, sc.y + row, pol_x);
                         }
                         for (int j = 0; j < n64; ++j, row += 64) {
-                            tma_load_2d(b_c + row * 128, &maps.b64, fb, kr * 128, sc.y + row, pol_x);
-                            tma_load_2d(b_s + row * 16, &maps.bs64, fb, kr * 16, sc.y + row, pol_x);
+                            tma_load_2d(b_c + row * 128, &maps.b64, fb, ks * 128, sc.y + row, pol_x);
+                            tma_load_2d(b_s + row * 16, &maps.bs64, fb, ks * 16, sc.y + row, pol_x);
                         }
                         for (int j = 0; j < r16; ++j, row += 16) {
-                            tma_load_2d(b_c + row * 128, &maps.b16, fb, kr * 128, sc.y + row, pol_x);
-                            tma_load_2d(b_s + row * 16, &maps.bs16, fb, kr * 16, sc.y + row, pol_x);
+                            tma_load_2d(b_c + row * 128, &maps.b16, fb, ks * 128, sc.y + row, pol_x);
+                            tma_load_2d(b_s + row * 16, &maps.bs16, fb, ks * 16, sc.y + row, pol_x);
                         }
                     }
-                    if (++stage == NR) {
+                    if (++stage == NS) {
                         stage = 0;
                         phase ^= 1u;
                     }
@@ -372,98 +380,94 @@ __global__ void __launch_bounds__(FG_THREADS, 1)
             }
         }
     } else if (warp >= 6) {
-        // ---------------------------------------------------------------- converters
-        // The 128 converter threads dequantise the four fp16 stages of every raw stage in order:
-        // thread i converts weight row i and the unit's token rows i, i + 128, ...  All of them
-        // take the fp16 buffers in the same order and each arrives once per use, so a buffer's
-        // full / empty phases advance one use at a time.
+        // ---------------------------------------------------------------- scale warps
+        // Thread i moves weight row i's 16 scales (four per K block) and token rows i and
+        // i + 128 into the stage's atoms; rows past the tile's rows get zero scales, so
+        // their (unstored) products are zero rather than whatever the smem held.
         const int i = threadIdx.x - 192;
-        int rs = 0, fs = 0;
-        uint32_t rph = 0, fph = 0;
+        int stage = 0;
+        uint32_t phase = 0;
         bool ok = true;
         for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
             const int4 sc = g.sched[u / g.m_blocks];
             const int mb = u % g.m_blocks;
-            const bool a_full = g.Nout - mb * FG_BM > 64;
-            const int nrows = ((sc.z + 15) / 16) * 16;
-            for (int kr = 0; kr < g.k_raw && ok; ++kr) {
-                if (!mbar_wait(smem_u32(&raw_full[rs]), rph, ctx, abort_flag)) {
+            const int arows = g.Nout - mb * FG_BM > 64 ? 128 : 64;
+            const int nrows = (sc.z + 15) / 16 * 16;
+            for (int ks = 0; ks < g.k_stages; ++ks) {
+                if (!mbar_wait(smem_u32(&full[stage]), phase, ctx, abort_flag)) {
                     ok = false;
                     break;
                 }
-                const uint8_t* st = raw + (size_t)rs * raw_bytes;
-                const uint8_t* a_c = st;
-                const uint8_t* b_c = st + FG_A_RAW;
-                const uint8_t* a_s = st + FG_A_RAW + b_raw;
-                const uint8_t* b_s = a_s + FG_A_SC;
-                for (int sub = 0; sub < 4; ++sub) {
-                    const int kf = kr * 4 + sub;
-                    if (kf >= g.k_f16) break;
-                    if (!mbar_wait(smem_u32(&f16_empty[fs]), fph ^ 1u, ctx, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    uint8_t* fa = f16 + (size_t)fs * f16_bytes;
-                    uint8_t* fbt = fa + FG_A_F16;
-                    const int kb0 = kr * 16 + sub * 4;
-                    if (a_full || i < 64)
-                        convert_row(a_c + i * 128, a_s + i * 16, fa + i * 128, i, sub, kb0, nbk);
-                    else
-#pragma unroll
-                        for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(fa + i * 128 + 16 * c) = make_uint4(0, 0, 0, 0);
-                    for (int j = i; j < nrows; j += 128)
-                        convert_row(b_c + j * 128, b_s + j * 16, fbt + j * 128, j, sub, kb0, nbk);
-                    // this thread's fp16 writes become visible to the tensor cores
-                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                    mbar_arrive(smem_u32(&f16_full[fs]));
-                    if (++fs == NF) {
-                        fs = 0;
-                        fph ^= 1u;
-                    }
+                uint8_t* st = smem + (size_t)stage * L.bytes;
+                {
+                    const uint4 v = i < arows ? *reinterpret_cast<const uint4*>(st + L.a_sc + 16 * i)
+                                              : make_uint4(0u, 0u, 0u, 0u);
+                    uint8_t* at = st + L.a_atoms + 16 * (i % 32) + 4 * (i / 32);
+                    *reinterpret_cast<uint32_t*>(at) = v.x;
+                    *reinterpret_cast<uint32_t*>(at + FG_ATOM) = v.y;
+                    *reinterpret_cast<uint32_t*>(at + 2 * FG_ATOM) = v.z;
+                    *reinterpret_cast<uint32_t*>(at + 3 * FG_ATOM) = v.w;
                 }
-                if (!ok) break;
-                mbar_arrive(smem_u32(&raw_empty[rs]));
-                if (++rs == NR) {
-                    rs = 0;
-                    rph ^= 1u;
+                for (int n = i; n < L.nbat * 128; n += 128) {
+                    const uint4 v = n < nrows ? *reinterpret_cast<const uint4*>(st + L.b_sc + 16 * n)
+                                              : make_uint4(0u, 0u, 0u, 0u);
+                    uint8_t* at = st + L.b_atoms + (n / 128) * FG_ATOM + 16 * (n % 32) + 4 * ((n / 32) % 4);
+                    const int kstep = L.nbat * FG_ATOM;
+                    *reinterpret_cast<uint32_t*>(at) = v.x;
+                    *reinterpret_cast<uint32_t*>(at + kstep) = v.y;
+                    *reinterpret_cast<uint32_t*>(at + 2 * kstep) = v.z;
+                    *reinterpret_cast<uint32_t*>(at + 3 * kstep) = v.w;
+                }
+                // the atoms become visible to the tensor cores' copies
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                mbar_arrive(smem_u32(&sfready[stage]));
+                if (++stage == NS) {
+                    stage = 0;
+                    phase ^= 1u;
                 }
             }
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA
         if (lane == 0) {
-            int fs = 0;
-            uint32_t fph = 0;
+            int stage = 0;
+            uint32_t phase = 0;
             int acc = 0;
             uint32_t acc_phase = 0;
             bool ok = true, issued = false;
+            const uint32_t sfa = tmem_base + FG_SFA_COL, sfb = tmem_base + FG_SFB_COL;
             for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
                 const int4 sc = g.sched[u / g.m_blocks];
                 const int n_mma = max(16, (sc.z + 15) & ~15);
-                const uint32_t idesc = make_idesc(0u, FG_BM, n_mma);   // fp16 A and B, fp32 accumulate
+                const uint32_t idesc = fp4_idesc(FG_BM, n_mma);
                 if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1u, ctx, abort_flag)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * 256);
-                for (int kf = 0; kf < g.k_f16; ++kf) {
-                    if (!mbar_wait(smem_u32(&f16_full[fs]), fph, ctx, abort_flag)) {
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * FG_ACC_COLS);
+                for (int ks = 0; ks < g.k_stages; ++ks) {
+                    if (!mbar_wait(smem_u32(&sfready[stage]), phase, ctx, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t a_base = smem_u32(f16 + (size_t)fs * f16_bytes);
-                    const uint32_t b_base = a_base + FG_A_F16;
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_ss<false>(d_tmem, sw128_desc(a_base + kk * 32), sw128_desc(b_base + kk * 32), idesc,
-                                      (kf | kk) != 0 ? 1u : 0u);
+                    const uint32_t st = smem_u32(smem + (size_t)stage * L.bytes);
+                    const int left = g.Kdim - ks * FG_KR;                 // K values of this stage
+                    const int nk = left >= FG_KR ? 4 : (left + 63) / 64;   // MMAs of K = 64
+                    for (int kk = 0; kk < nk; ++kk) {
+                        tmem_cp_atom(sfa + 4 * kk, atom_desc(st + L.a_atoms + kk * FG_ATOM));
+                        for (int j = 0; j < L.nbat; ++j)
+                            tmem_cp_atom(sfb + 8 * kk + 4 * j, atom_desc(st + L.b_atoms + (kk * L.nbat + j) * FG_ATOM));
+                    }
+                    for (int kk = 0; kk < nk; ++kk)
+                        mma_fp4(d_tmem, sw128_desc(st + kk * 32), sw128_desc(st + L.b_codes + kk * 32), idesc,
+                                sfa + 4 * kk, sfb + 8 * kk, (ks | kk) != 0 ? 1u : 0u);
                     issued = true;
-                    mma_commit(smem_u32(&f16_empty[fs]));
-                    if (++fs == NF) {
-                        fs = 0;
-                        fph ^= 1u;
+                    mma_commit(smem_u32(&empty[stage]));
+                    if (++stage == NS) {
+                        stage = 0;
+                        phase ^= 1u;
                     }
                 }
                 if (!ok) break;
@@ -493,7 +497,7 @@ __global__ void __launch_bounds__(FG_THREADS, 1)
             const bool fvalid = f < g.Nout;
             const float scale = __fmul_rn(g.w_tscale[sc.x], g.in_tscale);
             const float r6 = __frcp_rn(6.0f), rts = __frcp_rn(g.out_tscale);   // quotients via nv_div
-            const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * 256);
+            const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * FG_ACC_COLS);
             const int nchunks = (sc.z + 15) / 16;
             for (int c = 0; c < nchunks; ++c) {
                 uint32_t v[16];
@@ -576,27 +580,17 @@ static bool make_map_u8(CUtensorMap* m, const void* base, int64_t rows, int64_t 
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-struct Fp4Plan {
-    int bn, nr, nf;
-    size_t smem_bytes;
-};
-
 static int ksp_of(int K) { return (K / 16 + 15) / 16 * 16; }
 
-Fp4Plan fp4_plan(int bn) {
-    Fp4Plan p;
-    p.bn = bn;
-    const int raw = (FG_A_RAW + bn * 128 + FG_A_SC + bn * 16 + 1023) & ~1023;
-    const int f16 = FG_A_F16 + bn * 128;
-    // fp16 buffers: two for the wide tiles of large batches, five when the tiles are small
-    const int nf = bn > 64 ? 2 : 5;
-    int nr = (220 * 1024 - nf * f16) / raw;
-    if (nr > 8) nr = 8;
-    if (nr < 2) nr = 2;
-    p.nr = nr;
-    p.nf = nf;
-    p.smem_bytes = 1024 + (size_t)nr * raw + (size_t)nf * f16 + (size_t)(2 * nr + 2 * nf + 5) * 8 + 16;
-    return p;
+// Ring depth of the NVFP4 kernel for entries of up to bn token rows: as many stages as fit in
+// 225 KB of shared memory, at most 8.
+static int fp4_stages(int bn, size_t* smem) {
+    const Fp4Stage L(bn);
+    int ns = (225 * 1024) / L.bytes;
+    if (ns > 8) ns = 8;
+    if (ns < 2) ns = 2;
+    *smem = 1024 + (size_t)ns * L.bytes + (size_t)(3 * ns + 5) * 8 + 16;
+    return ns;
 }
 
 size_t nvfp4_scale_row_bytes(int K) { return (size_t)ksp_of(K); }
@@ -634,17 +628,17 @@ cudaError_t launch_grouped_gemm_fp4(bool up, const uint8_t* w_codes, const uint8
         !make_map_u8(&maps.bs64, a_scales, rows, ksp, ksp, 16, 64, false) ||
         !make_map_u8(&maps.bs16, a_scales, rows, ksp, ksp, 16, 16, false))
         return cudaErrorInvalidValue;
-    const Fp4Plan plan = fp4_plan(bn);
+    if (bn > FG_BN_MAX) return cudaErrorInvalidValue;
+    size_t smem = 0;
     Fp4Args g;
+    g.ns = fp4_stages(bn, &smem);
+    g.stage_bytes = Fp4Stage(bn).bytes;
     g.sched = sched;
     g.n_sched = n_sched;
     g.m_blocks = (Nout + FG_BM - 1) / FG_BM;
     g.Nout = Nout;
     g.Kdim = Kdim;
-    g.k_raw = (Kdim + FG_KR - 1) / FG_KR;
-    g.k_f16 = (Kdim + FG_KF - 1) / FG_KF;
-    g.nr = plan.nr;
-    g.nf = plan.nf;
+    g.k_stages = (Kdim + FG_KR - 1) / FG_KR;
     g.bn = bn;
     g.w_tscale = w_tscale;
     g.in_tscale = in_tscale;
@@ -654,8 +648,8 @@ cudaError_t launch_grouped_gemm_fp4(bool up, const uint8_t* w_codes, const uint8
     g.debug_withhold = debug_withhold;
     const int64_t max_units = (int64_t)max_sched * g.m_blocks;
     const int grid = (int)(max_units < num_sms ? max_units : num_sms);
-    return up ? launch_fp4<true>(maps, g, grid, plan.smem_bytes, stream, ctx)
-              : launch_fp4<false>(maps, g, grid, plan.smem_bytes, stream, ctx);
+    return up ? launch_fp4<true>(maps, g, grid, smem, stream, ctx)
+              : launch_fp4<false>(maps, g, grid, smem, stream, ctx);
 }
 
 cudaError_t launch_quantize_nvfp4(int64_t n_tensors, int64_t rows, int K, const uint16_t* src, uint8_t* codes,

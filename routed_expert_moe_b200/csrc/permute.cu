@@ -395,4 +395,89 @@ cudaError_t launch_gather(const uint16_t* x, const int32_t* perm_src, int64_t ro
                     K, T, H, xp, fp8 ? 1 : 0, x_scale, ctx);
 }
 
+// ----------------------------------------------------------------------------- expert-parallel regrouping
+
+// Rows received by an expert's owner arrive source-major: for each source rank p,
+// its rows for local expert 0, then 1, ... (each block in the source's order).  The
+// grouped layout the expert FFN reads is expert-major, then source, then arrival
+// order.  One block: thread 0 builds the small prefix tables (W * E_loc <= 256
+// entries), then every thread places rows i, i + blockDim.x, ...:
+//   received row i = (source p, local expert e, j-th of that block)
+//   grouped row     = off[e] + before[p][e] + j
+// with off[e] = rows of experts < e (all sources) and before[p][e] = rows of
+// expert e from sources < p.  perm[grouped] = i and inv[i] = grouped.
+constexpr int RG_THREADS = 512;
+constexpr int RG_MAX_ENTRIES = 256;
+
+__global__ void __launch_bounds__(RG_THREADS) ep_regroup_kernel(const int64_t* __restrict__ rc, int W, int E_loc,
+                                                                int64_t R, int32_t* __restrict__ offsets,
+                                                                int32_t* __restrict__ perm, int32_t* __restrict__ inv,
+                                                                DevCtx ctx) {
+    pdl_enter();
+    __shared__ int64_t src_base[RG_MAX_ENTRIES + 1];               // [W + 1]
+    __shared__ int64_t within[RG_MAX_ENTRIES + RG_MAX_ENTRIES];    // [W][E_loc + 1]
+    __shared__ int64_t before[RG_MAX_ENTRIES];                     // [W][E_loc]
+    __shared__ int64_t off[RG_MAX_ENTRIES + 1];                    // [E_loc + 1]
+    __shared__ int bad;
+    if (threadIdx.x == 0) {
+        bad = 0;
+        int64_t total = 0;
+        for (int p = 0; p < W; ++p) {
+            src_base[p] = total;
+            int64_t w = 0;
+            within[p * (E_loc + 1)] = 0;
+            for (int e = 0; e < E_loc; ++e) {
+                const int64_t c = rc[(int64_t)p * E_loc + e];
+                if (c < 0) bad = 1;
+                w += c;
+                within[p * (E_loc + 1) + e + 1] = w;
+            }
+            total += w;
+        }
+        src_base[W] = total;
+        if (total != R) bad = 1;
+        int64_t o = 0;
+        for (int e = 0; e < E_loc; ++e) {
+            off[e] = o;
+            int64_t b = 0;
+            for (int p = 0; p < W; ++p) {
+                before[p * E_loc + e] = b;
+                b += rc[(int64_t)p * E_loc + e];
+            }
+            o += b;
+        }
+        off[E_loc] = o;
+        if (bad) record_error(ctx.err, MOE_EINDEX);
+        for (int e = 0; e <= E_loc && !bad; ++e) offsets[e] = (int32_t)off[e];
+    }
+    __syncthreads();
+    if (bad) return;
+    for (int64_t i = threadIdx.x; i < R; i += blockDim.x) {
+        int lo = 0, hi = W;                      // last p with src_base[p] <= i
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) / 2;
+            if (src_base[mid] <= i) lo = mid; else hi = mid;
+        }
+        const int p = lo;
+        const int64_t local = i - src_base[p];
+        const int64_t* wp = within + p * (E_loc + 1);
+        int a = 0, b = E_loc;                    // last e with wp[e] <= local (wp[E_loc] > local)
+        while (b - a > 1) {
+            const int mid = (a + b) / 2;
+            if (wp[mid] <= local) a = mid; else b = mid;
+        }
+        const int e = a;
+        const int64_t pos = off[e] + before[p * E_loc + e] + (local - wp[e]);
+        perm[pos] = (int32_t)i;
+        inv[i] = (int32_t)pos;
+    }
+}
+
+cudaError_t launch_ep_regroup(const int64_t* recv_counts, int W, int E_loc, int64_t R, int32_t* offsets,
+                              int32_t* perm, int32_t* inv, const DevCtx& ctx, cudaStream_t stream) {
+    if (W < 1 || E_loc < 1 || (int64_t)W * E_loc > RG_MAX_ENTRIES) return cudaErrorInvalidValue;
+    return launch_k(ep_regroup_kernel, dim3(1), dim3(RG_THREADS), 0, stream, recv_counts, W, E_loc, R, offsets, perm,
+                    inv, ctx);
+}
+
 }  // namespace moe

@@ -8,14 +8,15 @@ layer pass on every rank:
 2. gather the token rows in that order and send each owner its rows (one
    all-to-all for the per-expert counts, one for the rows);
 3. regroup the received rows by local expert (source rank, then the source's
-   order, inside each expert) and run the local grouped FFN;
+   order, inside each expert; a kernel, from the received counts on the
+   device) and run the local grouped FFN;
 4. put the outputs back in the order they arrived and return them (one
    all-to-all);
 5. combine the returned rows with the routing weights, as the one-device layer.
 
 Tokens never interact and each assignment's expert output depends only on its
-token row, so the result equals the one-device layer.  Per-expert counts cross
-to the host once per pass: the all-to-all needs the split sizes there.  The
+token row, so the result equals the one-device layer.  The split sizes cross
+to the host once per pass (one read): NCCL's all-to-all needs them there.  The
 row exchange moves raw bytes, so any row dtype travels unchanged.
 
 The kernels come from an ``ops`` object (``CudaOps``: the library's calls on
@@ -27,7 +28,6 @@ its own experts.
 """
 from __future__ import annotations
 
-import numpy as np
 import torch
 import torch.distributed as dist
 
@@ -36,7 +36,8 @@ FORMATS = ("bf16", "fp8", "nvfp4", "fp8_b128")
 
 
 class CudaOps:
-    """The layer's steps on the current CUDA device, through the library's C ABI."""
+    """The layer's steps on the current CUDA device, through the library's C ABI.  Workspaces
+    are kept per problem size and reused across passes (no allocation once warm)."""
 
     def __init__(self, H: int, E: int, K: int, F: int, experts: str = "bf16"):
         from . import dims as _dims
@@ -46,9 +47,15 @@ class CudaOps:
         self.moe, self._dims = moe, _dims
         self.H, self.E, self.K, self.F = H, E, K, F
         self.fmt = {k: experts == k for k in ("fp8", "nvfp4", "fp8_b128")}
+        self._wss = {}
 
     def _ws(self, d):
-        return self.moe.alloc_workspace(d)
+        need = self.moe.workspace_size(d)
+        ws = self._wss.get(d.expert_dtype)
+        if ws is None or ws.numel() < need:
+            ws = self.moe.alloc_workspace(d)
+            self._wss[d.expert_dtype] = ws
+        return ws
 
     def route(self, x, w_router, bias):
         T = x.shape[0]
@@ -75,6 +82,16 @@ class CudaOps:
             self.moe.gather_rows(x, perm_src, out, K=K)
         return out
 
+    def regroup(self, recv_counts, R):
+        """recv_counts [W, E_loc] int64 on the device -> (offsets, perm, inv) on the device (a kernel)."""
+        dev = recv_counts.device
+        E_loc = recv_counts.shape[1]
+        offsets = torch.empty(E_loc + 1, dtype=torch.int32, device=dev)
+        perm = torch.empty(R, dtype=torch.int32, device=dev)
+        inv = torch.empty(R, dtype=torch.int32, device=dev)
+        self.moe.ep_regroup(recv_counts, offsets, perm, inv)
+        return offsets, perm, inv
+
     def expert_ffn(self, rows, offsets, perm, w_up, w_down, scales=None):
         R, E_loc = rows.shape[0], w_up.shape[0]
         y = torch.empty(R, self.H, dtype=torch.bfloat16, device=rows.device)
@@ -92,22 +109,6 @@ class CudaOps:
 def _bytes(t: torch.Tensor) -> torch.Tensor:
     """Rows [rows, n] as raw bytes [rows, n * itemsize] (a view; empty tensors included)."""
     return t.contiguous().view(torch.uint8)
-
-
-def regroup(recv_counts: np.ndarray):
-    """Received rows arrive source-major ([source][local expert] blocks).  Returns the grouped
-    layout's per-expert offsets and, for grouped row r, the received row it holds (expert-major,
-    then source, then arrival order), plus the inverse."""
-    W, E_loc = recv_counts.shape
-    src_base = np.concatenate([[0], np.cumsum(recv_counts.sum(1))])[:-1]
-    within = np.concatenate([np.zeros((W, 1), np.int64), np.cumsum(recv_counts, axis=1)[:, :-1]], axis=1)
-    perm = [np.arange(src_base[p] + within[p, e], src_base[p] + within[p, e] + recv_counts[p, e])
-            for e in range(E_loc) for p in range(W)]
-    perm = np.concatenate(perm).astype(np.int32) if perm else np.zeros(0, np.int32)
-    offsets = np.concatenate([[0], np.cumsum(recv_counts.sum(0))]).astype(np.int32)
-    inv = np.empty_like(perm)
-    inv[perm] = np.arange(perm.size, dtype=np.int32)
-    return offsets, perm, inv
 
 
 class ExpertParallelLayer:
@@ -139,19 +140,18 @@ class ExpertParallelLayer:
         send_counts = counts.reshape(W, E_loc).to(torch.int64).contiguous()
         recv_counts = torch.empty_like(send_counts)
         dist.all_to_all_single(recv_counts, send_counts, group=self.group)
-        sc = send_counts.sum(1).cpu().tolist()
-        rc_mat = recv_counts.cpu().numpy()
-        rc = rc_mat.sum(1).tolist()
+        # the split sizes of the row exchange: one device-to-host read per pass
+        both = torch.stack([send_counts.sum(1), recv_counts.sum(1)]).cpu()
+        sc, rc = both[0].tolist(), both[1].tolist()
 
         recv_rows = torch.empty(sum(rc), x.shape[1], dtype=x.dtype, device=x.device)
         dist.all_to_all_single(_bytes(recv_rows), _bytes(send_rows), output_split_sizes=rc, input_split_sizes=sc,
                                group=self.group)
 
-        loc_off, perm, inv = regroup(rc_mat)
+        loc_off, perm, inv = ops.regroup(recv_counts, sum(rc))
+        y_loc = ops.expert_ffn(recv_rows, loc_off, perm, w_up_local, w_down_local, scales)
+        y_back = ops.gather(y_loc, inv, 1)                           # arrival order
         dev = x.device
-        y_loc = ops.expert_ffn(recv_rows, torch.from_numpy(loc_off).to(dev), torch.from_numpy(perm).to(dev),
-                               w_up_local, w_down_local, scales)
-        y_back = ops.gather(y_loc, torch.from_numpy(inv).to(dev), 1)  # arrival order
 
         y_perm = torch.empty((sum(sc),) + tuple(y_back.shape[1:]), dtype=y_back.dtype, device=dev)
         dist.all_to_all_single(_bytes(y_perm), _bytes(y_back), output_split_sizes=sc, input_split_sizes=rc,

@@ -3,7 +3,8 @@
 Each kernel hands buffers between roles through mbarriers waited on by phase
 parity: a TMA ring of shared-memory stages (producer -> MMA), TMEM
 accumulators or partial slots (MMA -> epilogue warps) and, in the NVFP4
-kernel, a second ring of fp16 stages (converter threads -> MMA).  A parity
+kernel, a second hand between the TMA and the MMA (the scale threads, which
+rearrange each stage's block scales before the MMA copies them to TMEM).  A parity
 wait cannot tell a phase from the one two ahead, so a protocol is only right
 if no waiter can ever be two phases behind.  Compute-sanitizer is not
 available, so this test runs the protocols, as the kernels write them (the
@@ -248,73 +249,61 @@ def gemm_b128(sim, units, k_stages, NS, NP=4, n_epi=4, plant=None):
 
 # ----------------------------------------------------------------------------- NVFP4 grouped GEMM
 
-def gemm_fp4(sim, units, k_raw, k_f16, NR, NF, n_conv=8, n_epi=4):
-    """grouped_gemm_fp4_kernel: a raw TMA ring (raw_empty: every converter thread), the
-    converters' fp16 ring (f16_full: every converter thread; f16_empty: the MMA's commit),
-    two TMEM accumulators.  The 128 converter threads take the fp16 buffers in the same
-    order; they are modelled as n_conv independent agents (any of them may run ahead)."""
-    raw_full, raw_empty = [Bar(1) for _ in range(NR)], [Bar(n_conv) for _ in range(NR)]
-    f16_full, f16_empty = [Bar(n_conv) for _ in range(NF)], [Bar(1) for _ in range(NF)]
+def gemm_fp4(sim, units, k_stages, NS, n_sc=8, n_epi=4):
+    """grouped_gemm_fp4_kernel: one TMA ring whose stages pass through two hands before the
+    MMA frees them -- full (the TMA bytes), then sfready (every scale thread has written the
+    stage's scale atoms), then empty (the MMA's commit) -- and two TMEM accumulators.  The
+    128 scale threads are modelled as n_sc independent agents (any of them may run ahead)."""
+    full, sfready, empty = [Bar(1) for _ in range(NS)], [Bar(n_sc) for _ in range(NS)], [Bar(1) for _ in range(NS)]
     tfull, tempty = [Bar(1) for _ in range(2)], [Bar(n_epi) for _ in range(2)]
-    raw, raw_reads = [None] * NR, [n_conv] * NR
-    f16 = [[None] * n_conv for _ in range(NF)]
-    f16_fresh = [[False] * n_conv for _ in range(NF)]
+    smem, fresh = [None] * NS, [False] * NS
+    atoms = [[None] * n_sc for _ in range(NS)]
     tmem, readers = [None] * 2, [n_epi] * 2
 
     def producer():
-        rs, rph = 0, 0
+        st, ph = 0, 0
         for u in range(units):
-            for kr in range(k_raw):
-                yield (lambda s=rs, p=rph: raw_empty[s].passed(p ^ 1))
+            for ks in range(k_stages):
+                yield (lambda s=st, p=ph: empty[s].passed(p ^ 1))
 
-                def land(s=rs, tag=(u, kr)):
-                    check(raw_reads[s] == n_conv, f"TMA overwrote raw stage {s} before every converter read it")
-                    raw[s], raw_reads[s] = tag, 0
-                    raw_full[s].arrive()
+                def land(s=st, tag=(u, ks)):
+                    check(not fresh[s], f"TMA overwrote stage {s} before the MMA consumed it")
+                    smem[s], fresh[s] = tag, True
+                    full[s].arrive()
                 sim.post(None, land)
-                rs += 1
-                if rs == NR:
-                    rs, rph = 0, rph ^ 1
+                st += 1
+                if st == NS:
+                    st, ph = 0, ph ^ 1
 
-    def converter(i):
-        rs, rph, fs, fph = 0, 0, 0, 0
+    def scale_thread(i):
+        st, ph = 0, 0
         for u in range(units):
-            for kr in range(k_raw):
-                yield (lambda s=rs, p=rph: raw_full[s].passed(p))
-                check(raw[rs] == (u, kr), f"converter {i} read raw stage {rs} holding {raw[rs]}, expected {(u, kr)}")
-                for sub in range(4):
-                    kf = kr * 4 + sub
-                    if kf >= k_f16:
-                        break
-                    yield (lambda f=fs, p=fph: f16_empty[f].passed(p ^ 1))
-                    check(not f16_fresh[fs][i], f"converter {i} overwrote fp16 stage {fs} before the MMA read it")
-                    f16[fs][i], f16_fresh[fs][i] = (u, kf), True
-                    f16_full[fs].arrive()
-                    fs += 1
-                    if fs == NF:
-                        fs, fph = 0, fph ^ 1
-                raw_reads[rs] += 1
-                raw_empty[rs].arrive()
-                rs += 1
-                if rs == NR:
-                    rs, rph = 0, rph ^ 1
+            for ks in range(k_stages):
+                yield (lambda s=st, p=ph: full[s].passed(p))
+                check(smem[st] == (u, ks), f"scale thread {i} read stage {st} holding {smem[st]}, expected {(u, ks)}")
+                atoms[st][i] = (u, ks)
+                sfready[st].arrive()
+                st += 1
+                if st == NS:
+                    st, ph = 0, ph ^ 1
 
     def mma():
-        fs, fph, acc, aph = 0, 0, 0, 0
+        st, ph, acc, aph = 0, 0, 0, 0
         for u in range(units):
             yield (lambda a=acc, p=aph: tempty[a].passed(p ^ 1))
             check(readers[acc] == n_epi, f"MMA wrote accumulator {acc} while the epilogue was reading it")
-            for kf in range(k_f16):
-                yield (lambda f=fs, p=fph: f16_full[f].passed(p))
-                check(all(t == (u, kf) for t in f16[fs]), f"MMA read fp16 stage {fs} holding {f16[fs]}")
+            for ks in range(k_stages):
+                yield (lambda s=st, p=ph: sfready[s].passed(p))
+                check(smem[st] == (u, ks), f"MMA read stage {st} holding {smem[st]}, expected {(u, ks)}")
+                check(all(t == (u, ks) for t in atoms[st]), f"MMA copied the atoms of stage {st}: {atoms[st]}")
 
-                def mma_done(f=fs):
-                    f16_fresh[f] = [False] * n_conv
-                    f16_empty[f].arrive()
+                def mma_done(s=st):
+                    fresh[s] = False
+                    empty[s].arrive()
                 sim.post("tc", mma_done)
-                fs += 1
-                if fs == NF:
-                    fs, fph = 0, fph ^ 1
+                st += 1
+                if st == NS:
+                    st, ph = 0, ph ^ 1
 
             def acc_done(a=acc, u=u):
                 tmem[a], readers[a] = u, 0
@@ -337,8 +326,8 @@ def gemm_fp4(sim, units, k_raw, k_f16, NR, NF, n_conv=8, n_epi=4):
 
     sim.role("producer", producer())
     sim.role("mma", mma())
-    for i in range(n_conv):
-        sim.role(f"converter{i}", converter(i))
+    for i in range(n_sc):
+        sim.role(f"scale{i}", scale_thread(i))
     for w in range(n_epi):
         sim.role(f"epilogue{w}", epilogue(w))
 
@@ -451,12 +440,11 @@ def test_fp8_b128_protocol(units, k_stages, NS):
         assert sim.run() == "done"
 
 
-@pytest.mark.parametrize("units,k_raw,k_f16,NR,NF", [(3, 11, 42, 4, 5), (3, 8, 29, 2, 2), (4, 1, 4, 3, 5),
-                                                     (3, 2, 7, 5, 2), (2, 11, 42, 8, 3)])
-def test_nvfp4_protocol(units, k_raw, k_f16, NR, NF):
+@pytest.mark.parametrize("units,k_stages,NS", [(3, 11, 4), (3, 8, 2), (4, 1, 3), (3, 2, 5), (2, 11, 8)])
+def test_nvfp4_protocol(units, k_stages, NS):
     for seed in range(15):
         sim = Sim(seed)
-        gemm_fp4(sim, units, k_raw, k_f16, NR, NF)
+        gemm_fp4(sim, units, k_stages, NS)
         assert sim.run() == "done"
 
 

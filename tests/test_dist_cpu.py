@@ -74,3 +74,41 @@ def test_reference_arm_prints_on_rank_zero_only():
     assert line["impl"] == "reference" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def _ep_worker(rank, world, port, q):
+    """The --ep mode's cross-rank steps on gloo: every rank times its own pass, the line takes
+    the slowest rank's time and counts every rank's tokens."""
+    import torch.distributed as dist
+    sys.path.insert(0, str(ROOT))
+    import bench
+    from synth import workloads as W
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    ms = bench.reduce_max(4.0 + rank, dist, "cpu")
+    e2e = bench.reduce_max(6.0 - rank, dist, "cpu")
+    dist.barrier()
+    line = bench.ep_line(world, W.WORKLOADS[1], 10, 3, ms, e2e, {}, 7)
+    q.put((rank, json.dumps(line)))
+    dist.destroy_process_group()
+
+
+def test_expert_parallel_line_takes_the_slowest_rank():
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_ep_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    lines = [json.loads(r[1]) for r in res]
+    assert lines[0] == lines[1]
+    line = lines[0]
+    assert line["ms_per_step"] == pytest.approx(0.5)                     # max(4, 5) / 10 steps
+    assert line["value"] == pytest.approx(2 * 64 * 10 / 5e-3)           # both ranks' tokens
+    assert line["e2e"]["value"] == pytest.approx(2 * 64 * 10 / 6e-3)
+    assert line["config"]["parallelism"].startswith("ep2 (64 experts per rank")
+    assert line["gpu_launches"] == 70 and line["scaling"] == "weak"

@@ -30,6 +30,22 @@ def _free_port():
     return p
 
 
+def host_regroup(recv_counts: np.ndarray):
+    """The grouped layout of received rows, stated on the host: rows arrive source-major
+    ([source][local expert] blocks); grouped row r holds the received row given by the
+    expert-major, then source, then arrival order.  Returns (offsets, perm, inv)."""
+    W, E_loc = recv_counts.shape
+    src_base = np.concatenate([[0], np.cumsum(recv_counts.sum(1))])[:-1]
+    within = np.concatenate([np.zeros((W, 1), np.int64), np.cumsum(recv_counts, axis=1)[:, :-1]], axis=1)
+    perm = [np.arange(src_base[p] + within[p, e], src_base[p] + within[p, e] + recv_counts[p, e])
+            for e in range(E_loc) for p in range(W)]
+    perm = np.concatenate(perm).astype(np.int32) if perm else np.zeros(0, np.int32)
+    offsets = np.concatenate([[0], np.cumsum(recv_counts.sum(0))]).astype(np.int32)
+    inv = np.empty_like(perm)
+    inv[perm] = np.arange(perm.size, dtype=np.int32)
+    return offsets, perm, inv
+
+
 class OracleOps:
     """The layer's steps on CPU from the oracle (bf16 rows travel as int16 bit patterns, expert
     outputs as float64).  fmt: the experts' format; the banks and scales are the oracle's."""
@@ -71,6 +87,11 @@ class OracleOps:
             y = o.expert_rows_fp8_b128(o.quantize_act_fp8_b128(bits, sx), ex, w_up, w_down, slot, sx, sh,
                                        self.H, self.F)
         return torch.from_numpy(y)
+
+    def regroup(self, recv_counts, R):
+        off, perm, inv = host_regroup(recv_counts.numpy())
+        assert perm.size == R
+        return tuple(torch.from_numpy(a) for a in (off, perm, inv))
 
     def combine(self, y_perm, inv_row, w, residual, out):
         T = out.shape[0]
@@ -177,12 +198,11 @@ def test_expert_parallel_layer_equals_the_one_process_layer(world, T, fmt):
 
 
 def test_regroup_orders_rows_by_expert_then_source():
-    from routed_expert_moe_b200.ep import regroup
     rng = np.random.default_rng(3)
     for W_, E_loc in ((1, 4), (3, 2), (4, 5)):
         counts = rng.integers(0, 4, size=(W_, E_loc))
         counts[0, 0] = 0
-        off, perm, inv = regroup(counts)
+        off, perm, inv = host_regroup(counts)
         # brute force: label every received row (source p, expert e, i) in arrival order
         labels = [(p, e, i) for p in range(W_) for e in range(E_loc) for i in range(counts[p, e])]
         want = sorted(range(len(labels)), key=lambda r: (labels[r][1], labels[r][0], labels[r][2]))

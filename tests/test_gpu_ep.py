@@ -63,3 +63,38 @@ def test_expert_parallel_world_one_matches_forward(w):
         assert rel_err(host_f64(out)[tok], r["out"]) <= BF16_TOL
     finally:
         dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("W_,E_loc", [(1, 128), (2, 64), (8, 16), (4, 5), (16, 16)])
+def test_device_regroup_orders_rows_by_expert_then_source(W_, E_loc):
+    """moe_ep_regroup against a brute-force labelling of the received rows: every received row
+    is (source p, local expert e, i-th of its block) in arrival order, and the grouped layout
+    sorts them by (e, p, i)."""
+    import routed_expert_moe_b200 as moe
+    rng = np.random.default_rng(W_ * 100 + E_loc)
+    counts = rng.integers(0, 7, size=(W_, E_loc))
+    counts[0, 0] = 0
+    counts[-1, :] = 0                         # a source that sends nothing
+    labels = [(p, e, i) for p in range(W_) for e in range(E_loc) for i in range(counts[p, e])]
+    want = sorted(range(len(labels)), key=lambda r: (labels[r][1], labels[r][0], labels[r][2]))
+    R = len(labels)
+    rc = torch.from_numpy(counts.astype(np.int64)).cuda()
+    off = torch.empty(E_loc + 1, dtype=torch.int32, device="cuda")
+    perm = torch.empty(R, dtype=torch.int32, device="cuda")
+    inv = torch.empty(R, dtype=torch.int32, device="cuda")
+    moe.ep_regroup(rc, off, perm, inv)
+    moe.check_device_error()
+    assert perm.cpu().tolist() == want
+    assert np.array_equal(inv.cpu().numpy()[np.array(want, dtype=np.int64)], np.arange(R))
+    assert off.cpu().tolist() == [0] + np.cumsum(counts.sum(0)).tolist()
+
+
+def test_device_regroup_rejects_counts_that_do_not_sum_to_the_rows():
+    import routed_expert_moe_b200 as moe
+    rc = torch.tensor([[3, 1], [2, 2]], dtype=torch.int64, device="cuda")
+    off = torch.full((3,), -1, dtype=torch.int32, device="cuda")
+    perm = torch.empty(7, dtype=torch.int32, device="cuda")    # 8 rows were announced
+    inv = torch.empty(7, dtype=torch.int32, device="cuda")
+    moe.ep_regroup(rc, off, perm, inv)
+    assert moe.check_device_error_status() == moe.MOE_EINDEX
+    assert off.cpu().tolist() == [-1, -1, -1]
