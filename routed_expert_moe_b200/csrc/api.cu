@@ -21,6 +21,7 @@ constexpr uint64_t kDefaultTimeoutNs = 4000000000ull;
 std::atomic<uint64_t> g_timeout_ns{kDefaultTimeoutNs};
 std::atomic<int> g_debug_withhold{0};
 std::atomic<int> g_gemm_pair{0};
+std::atomic<int> g_fused_ffn{1};   // 1: both bf16/E4M3 projections in one launch (grouped_ffn.cu)
 std::atomic<int> g_pdl{1};
 std::atomic<int> g_shared_2d{0};   // 1: the shared down weight through its 2-D fallback map
 void* g_stage_events[MOE_STAGE_EVENTS] = {};
@@ -125,6 +126,7 @@ struct FfnWs {
     void* hb;            // ReLU^2 rows: bf16, E4M3 codes, or NVFP4 codes [rows][F/2]
     uint8_t* xp_block;   // NVFP4: block scales [rows][KSP(H)]
     uint8_t* hb_block;   // NVFP4: block scales [rows][KSP(F)]
+    int* done;           // [max_sched] up units reported per schedule entry (one-launch FFN)
 };
 struct ForwardWs {
     int32_t* idx;
@@ -137,13 +139,21 @@ struct ForwardWs {
 };
 
 // Plan of the expert FFN: one tile schedule for every expert dtype (FP8_B128
-// caps a tile at 64 token rows: its epilogue keeps a tile's sums in registers;
+// caps a tile at 128 token rows: its epilogue keeps a tile's sums in registers;
 // NVFP4 at 224: its accumulators share TMEM with the scale factors),
 // plus the shared expert's entries (ns chunks of T rows, cut into tiles of at
 // most bn).
+// Whether the expert FFN runs as one launch (bf16 or E4M3 experts without a shared expert).
+bool fused_ffn(const moe_dims* d) {
+    return g_fused_ffn.load() && n_shared(d) == 0 &&
+           (d->expert_dtype == MOE_BF16 || d->expert_dtype == MOE_FP8_E4M3);
+}
+
 GemmPlan ffn_plan(const moe_dims* d) {
     GemmPlan gp = gemm_plan(d->T, d->K, d->E);
-    const int cap = d->expert_dtype == MOE_FP8_B128 ? 64 : d->expert_dtype == MOE_NVFP4 ? kFp4MaxTileRows : 0;
+    const int cap = d->expert_dtype == MOE_FP8_B128 ? kB128MaxTileRows
+                    : d->expert_dtype == MOE_NVFP4    ? kFp4MaxTileRows
+                                                      : 0;
     if (cap > 0 && gp.bn > cap) {
         const int64_t rows = d->T * d->K;
         const int64_t nonempty = d->E < rows ? d->E : rows;
@@ -168,6 +178,7 @@ FfnWs carve_ffn(Carve& c, void* base, const moe_dims* d, const GemmPlan& gp) {
     f.sched = c.take<int4>(base, (size_t)gp.max_sched);
     f.n_sched = c.take<int>(base, 1);
     f.perm_scratch = c.take<int>(base, permute_scratch_ints(d->T * d->K, d->E));
+    f.done = c.take<int>(base, (size_t)gp.max_sched);
     f.xp_block = f.hb_block = nullptr;
     if (d->expert_dtype == MOE_NVFP4) {
         f.xp = c.take<uint8_t>(base, rows * d->H / 2);
@@ -262,13 +273,24 @@ moe_status run_ffn(const moe_dims* d, const DeviceInfo* dev, const DevCtx& ctx, 
         return cuda_status(e4);
     }
     if (marks) stage_mark(3, st);
-    // permuted copy of x (or of its E4M3 codes), read by the up projection in contiguous row blocks
-    cudaError_t e = launch_gather(static_cast<const uint16_t*>(x), perm_src, rows, d->T * d->K, d->K, d->T, d->H,
-                                  fw.xp, fp8, fp8 ? sc->x_scale : 1.0f, dev->num_sms, ctx, st);
-    if (e != cudaSuccess) return cuda_status(e);
     const int withhold = g_debug_withhold.load();
     // optional: tiles of more than 64 tokens on CTA pairs (one activation read per 256 weight rows)
     const bool pair = g_gemm_pair.load() && gp.bn > 64 && !withhold && ns == 0;
+    const bool fused = fused_ffn(d) && !pair;
+    // permuted copy of x (or of its E4M3 codes), read by the up projection in contiguous row blocks;
+    // it also zeroes the one-launch FFN's per-entry counters
+    cudaError_t e = launch_gather(static_cast<const uint16_t*>(x), perm_src, rows, d->T * d->K, d->K, d->T, d->H,
+                                  fw.xp, fp8, fp8 ? sc->x_scale : 1.0f, dev->num_sms, ctx, st,
+                                  fused ? fw.done : nullptr, fused ? gp.max_sched : 0);
+    if (e != cudaSuccess) return cuda_status(e);
+    if (fused) {
+        if (marks) stage_mark(4, st);
+        e = launch_grouped_ffn(fp8, w_up, w_down, d->E, d->F, d->H, fw.xp, fw.hb, y_perm, rows, fw.sched, fw.n_sched,
+                               fw.done, gp, fp8 ? sc->w_up_scale : nullptr, fp8 ? sc->w_down_scale : nullptr,
+                               fp8 ? sc->x_scale : 1.0f, fp8 ? sc->h_scale : 1.0f, dev->num_sms, withhold, ctx, st);
+        if (marks) stage_mark(5, st);
+        return cuda_status(e);
+    }
     if (marks) stage_mark(4, st);
     if (pair)
         e = launch_grouped_gemm_pair(fp8, true, w_up, d->E, d->F, d->H, fw.xp, rows, fw.sched, fw.n_sched, gp.bn,
@@ -364,7 +386,8 @@ moe_status moe_forward_launches(const moe_dims* d, int32_t* launches) {
     }
     int n = route_launches(d->T, d->H, d->E);
     n += permute_scratch_ints(d->T * d->K, d->E) == 0 ? 1 : 3;   // one block, or histogram + scan + scatter
-    n += 1 + 2 + 1;   // row gather, up and down projections, combine
+    // row gather, up and down projections (one launch or two), combine
+    n += 1 + (fused_ffn(d) && !(g_gemm_pair.load() && gemm_plan(d->T, d->K, d->E).bn > 64) ? 1 : 2) + 1;
     *launches = n;
     return MOE_OK;
 }
@@ -645,6 +668,10 @@ moe_status moe_debug_set(int32_t what, int64_t value) {
     }
     if (what == 7) {
         g_shared_2d.store(value ? 1 : 0);
+        return MOE_OK;
+    }
+    if (what == 8) {
+        g_fused_ffn.store(value ? 1 : 0);
         return MOE_OK;
     }
     if (what == 5) {

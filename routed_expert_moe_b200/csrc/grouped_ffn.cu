@@ -1,0 +1,410 @@
+// Both expert projections in one persistent launch (bf16 or E4M3 experts, no
+// shared expert): the up projection's units, then the down projection's, in
+// one list that every CTA walks round-robin.
+//
+// The products are those of grouped_gemm.cu (bloomery issue page, s.2
+// "Checkpoint facts" and s.3: ungated ReLU^2 experts with up/down parts):
+//   up:    H[r, f] = relu( sum_h W_up[e][f][h] * X_perm[r][h] )^2
+//   down:  Y[r, j] =       sum_f W_down[e][j][f] * H[r][f]
+// with the same swap-AB units, TMA ring, TMEM accumulators and epilogue.
+// What changes is the boundary between the two: a down unit of schedule entry
+// s reads the rows of H that the up units of s write, so instead of a kernel
+// boundary (every down unit waits for every up unit, and the last up wave
+// leaves SMs idle), the producer of a down unit waits only for entry s:
+//   up epilogue   each of the four epilogue warps stores its rows of H, every
+//                 lane fences (generic -> async proxy, then device scope), and
+//                 lane 0 adds 1 to done[s] with release semantics;
+//   down producer spins (bounded) on an acquire load of done[s] until it
+//                 reaches 4 * m_up, fences the async proxy, then issues the
+//                 TMA loads of H.
+// Deadlock freedom: every CTA walks all of its up units before any of its down
+// units, so the up units a down unit waits for are all issued by CTAs that
+// never wait on anything but their own pipeline.  done[] is zeroed by the row
+// gather that precedes this kernel on the stream.
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int FF_THREADS = 192;
+constexpr int FF_BM = 128;
+constexpr int FF_ROW_BYTES = 128;
+constexpr int FF_A_BYTES = FF_BM * FF_ROW_BYTES;
+constexpr int FF_TMEM_COLS = 512;
+constexpr int FF_EPI_WARPS = 4;
+
+struct FfnArgs {
+    const int4* sched;      // {e, row0, nrows, 0}
+    const int* n_sched;
+    int* done;              // [max_sched] up epilogue warps finished per entry (zero at launch)
+    int m_up, m_down;       // 128-row blocks of F and of H
+    int F, H;
+    int k_up, k_down;       // 128-byte K stages of H and of F
+    int n_stages;
+    int b_stage_bytes;
+    void* hb;               // up output [rows][F] (bf16, or E4M3 codes)
+    void* y;                // down output [rows][H] bf16
+    const float* su;        // [E] E4M3 weight scales (null for bf16)
+    const float* sd;
+    float x_scale, h_scale;
+    int debug_hold;         // 1: block 0's first up unit never reports its rows (a wait must expire)
+};
+
+struct FfnMaps {
+    CUtensorMap ua128, ua64;          // W_up [E * F][H]
+    CUtensorMap ub128, ub64, ub16;    // X_perm [rows][H]
+    CUtensorMap da128, da64;          // W_down [E * H][F]
+    CUtensorMap db128, db64, db16;    // H [rows][F]
+};
+
+__device__ __forceinline__ int ld_acquire(const int* p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void red_release_add(int* p, int v) {
+    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Bounded wait until *p >= target (acquire).  Gives up on the time limit or the block's abort flag.
+__device__ __forceinline__ bool wait_count(const int* p, int target, const DevCtx& ctx, volatile int* abort) {
+    if (ld_acquire(p) >= target) return true;
+    const uint64_t t0 = globaltimer();
+    while (true) {
+        __nanosleep(64);
+        if (ld_acquire(p) >= target) return true;
+        if (*abort) return false;
+        if (globaltimer() - t0 > ctx.timeout_ns) {
+            record_error(ctx.err, MOE_ETIMEOUT);
+            *abort = 1;
+            return false;
+        }
+    }
+}
+
+template <bool FP8>
+__global__ void __launch_bounds__(FF_THREADS, 1)
+    grouped_ffn_kernel(const __grid_constant__ FfnMaps maps, FfnArgs g, DevCtx ctx) {
+    constexpr int KEL = FF_ROW_BYTES / (FP8 ? 1 : 2);   // elements of K per stage
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    const int NS = g.n_stages;
+    uint8_t* smA = smem;
+    uint8_t* smB = smA + (size_t)NS * FF_A_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smB + (size_t)NS * g.b_stage_bytes);
+    uint64_t* full = bars;
+    uint64_t* empty = bars + NS;
+    uint64_t* tfull = bars + 2 * NS;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* drain = tempty + 2;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(drain + 1);
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1) + 1;
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(smem_u32(&full[s]), 1);
+            mbar_init(smem_u32(&empty[s]), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(smem_u32(&tfull[a]), 1);
+            mbar_init(smem_u32(&tempty[a]), 128);
+        }
+        mbar_init(smem_u32(drain), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) tmem_alloc(smem_u32(tmem_holder), FF_TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+    pdl_enter();
+
+    const int n_sched = *g.n_sched;
+    const int n_up = n_sched * g.m_up;
+    const int n_units = n_up + n_sched * g.m_down;
+    const int up_target = FF_EPI_WARPS * g.m_up;   // reports of one entry's up units
+
+    if (warp == 0) {
+        if (lane == 0) {
+            const uint64_t pol_w = l2_policy_evict_first();
+            const uint64_t pol_x = l2_policy_evict_last();
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+                const bool up = u < n_up;
+                const int v = up ? u : u - n_up;
+                const int m_blocks = up ? g.m_up : g.m_down;
+                const int s_idx = v / m_blocks, mb = v % m_blocks;
+                const int4 sc = g.sched[s_idx];
+                const int Nout = up ? g.F : g.H;
+                const int k_stages = up ? g.k_up : g.k_down;
+                const bool a_full = Nout - mb * FF_BM > 64;
+                const int n16 = (sc.z + 15) / 16;
+                const int n128 = n16 / 8, n64 = (n16 % 8) / 4, r16 = n16 % 4;
+                const uint32_t bytes = (uint32_t)((a_full ? 128 : 64) * FF_ROW_BYTES + n16 * 16 * FF_ROW_BYTES);
+                const CUtensorMap* amap = up ? (a_full ? &maps.ua128 : &maps.ua64) : (a_full ? &maps.da128 : &maps.da64);
+                const CUtensorMap* b128 = up ? &maps.ub128 : &maps.db128;
+                const CUtensorMap* b64 = up ? &maps.ub64 : &maps.db64;
+                const CUtensorMap* b16 = up ? &maps.ub16 : &maps.db16;
+                const int ay = sc.x * Nout + mb * FF_BM;
+                if (!up) {
+                    // the rows of H this unit reads are written by the up units of its entry
+                    if (!wait_count(g.done + s_idx, up_target, ctx, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    fence_proxy_async_global();
+                }
+                for (int ks = 0; ks < k_stages; ++ks) {
+                    if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, ctx, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t fb = smem_u32(&full[stage]);
+                    mbar_arrive_expect_tx(fb, bytes);
+                    const int kx = ks * KEL;
+                    const uint32_t a_dst = smem_u32(smA + (size_t)stage * FF_A_BYTES);
+                    const uint32_t b_dst = smem_u32(smB + (size_t)stage * g.b_stage_bytes);
+                    tma_load_2d(a_dst, amap, fb, kx, ay, pol_w);
+                    int row = 0;
+                    for (int j = 0; j < n128; ++j, row += 128)
+                        tma_load_2d(b_dst + row * FF_ROW_BYTES, b128, fb, kx, sc.y + row, pol_x);
+                    for (int j = 0; j < n64; ++j, row += 64)
+                        tma_load_2d(b_dst + row * FF_ROW_BYTES, b64, fb, kx, sc.y + row, pol_x);
+                    for (int j = 0; j < r16; ++j, row += 16)
+                        tma_load_2d(b_dst + row * FF_ROW_BYTES, b16, fb, kx, sc.y + row, pol_x);
+                    if (++stage == NS) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                // let loads already in flight land before the block exits
+                const uint64_t t0 = globaltimer();
+                while (globaltimer() - t0 < 200000ull) __nanosleep(1000);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true, issued = false;
+            for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+                const bool up = u < n_up;
+                const int v = up ? u : u - n_up;
+                const int4 sc = g.sched[v / (up ? g.m_up : g.m_down)];
+                const int k_stages = up ? g.k_up : g.k_down;
+                const int n_mma = max(16, (sc.z + 15) & ~15);
+                const uint32_t idesc = make_idesc(FP8 ? 0u : 1u, FF_BM, n_mma);
+                if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1u, ctx, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * 256);
+                for (int ks = 0; ks < k_stages; ++ks) {
+                    if (!mbar_wait(smem_u32(&full[stage]), phase, ctx, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_base = smem_u32(smA + (size_t)stage * FF_A_BYTES);
+                    const uint32_t b_base = smem_u32(smB + (size_t)stage * g.b_stage_bytes);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_ss<FP8>(d_tmem, sw128_desc(a_base + kk * 32), sw128_desc(b_base + kk * 32), idesc,
+                                    (ks | kk) != 0 ? 1u : 0u);
+                    issued = true;
+                    mma_commit(smem_u32(&empty[stage]));
+                    if (++stage == NS) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                mma_commit(smem_u32(&tfull[acc]));
+                if (++acc == 2) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
+            }
+            if (!ok && issued) {
+                // wait for every MMA issued so far before TMEM is released
+                mma_commit(smem_u32(drain));
+                mbar_wait_drain(smem_u32(drain), 0, ctx.timeout_ns);
+            }
+        }
+    } else {
+        const int q = warp & 3;   // TMEM lane quadrant of this warp
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        const float inv_h = (FP8) ? __frcp_rn(g.h_scale) : 1.0f;
+        for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+            const bool up = u < n_up;
+            const int v = up ? u : u - n_up;
+            const int m_blocks = up ? g.m_up : g.m_down;
+            const int s_idx = v / m_blocks, mb = v % m_blocks;
+            const int4 sc = g.sched[s_idx];
+            const int Nout = up ? g.F : g.H;
+            if (!mbar_wait_warp(smem_u32(&tfull[acc]), acc_phase, ctx, abort_flag)) break;
+            tc_fence_after();
+            const int f = mb * FF_BM + q * 32 + lane;
+            const bool fvalid = f < Nout;
+            float scale = 1.0f;
+            if constexpr (FP8) scale = up ? __fmul_rn(g.su[sc.x], g.x_scale) : __fmul_rn(g.sd[sc.x], g.h_scale);
+            const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * 256);
+            const int nchunks = (sc.z + 15) / 16;
+            for (int c = 0; c < nchunks; ++c) {
+                uint32_t vv[16];
+                tmem_ld16(t_row + (uint32_t)(c * 16), vv);
+                if (fvalid) {
+                    if (up) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const int r = c * 16 + j;
+                            if (r < sc.z) {
+                                float z = __uint_as_float(vv[j]);
+                                if constexpr (FP8) z = __fmul_rn(z, scale);
+                                const float a = z > 0.0f ? __fmul_rn(z, z) : 0.0f;
+                                const int64_t o = (int64_t)(sc.y + r) * g.F + f;
+                                if constexpr (FP8)
+                                    static_cast<uint8_t*>(g.hb)[o] = (uint8_t)__nv_cvt_float_to_fp8(
+                                        __fmul_rn(a, inv_h), __NV_SATFINITE, __NV_E4M3);
+                                else
+                                    static_cast<__nv_bfloat16*>(g.hb)[o] = __float2bfloat16_rn(a);
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const int r = c * 16 + j;
+                            if (r < sc.z) {
+                                float z = __uint_as_float(vv[j]);
+                                if constexpr (FP8) z = __fmul_rn(z, scale);
+                                static_cast<__nv_bfloat16*>(g.y)[(int64_t)(sc.y + r) * g.H + f] = __float2bfloat16_rn(z);
+                            }
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(smem_u32(&tempty[acc]));
+            if (up) {
+                // this warp's rows of H are complete: make them visible to the TMA loads of
+                // other CTAs, then report them to the entry's down units
+                fence_proxy_async_global();
+                __threadfence();
+                __syncwarp();
+                const bool hold = g.debug_hold && blockIdx.x == 0 && u == (int)blockIdx.x;
+                if (lane == 0 && !hold) red_release_add(g.done + s_idx, 1);
+            }
+            if (++acc == 2) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, FF_TMEM_COLS);
+    }
+}
+
+typedef CUresult (*EncodeTiledFnF)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFnF encode_fn_ffn() {
+    static EncodeTiledFnF fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFnF>(p);
+    }
+    return fn;
+}
+
+// 2-D map over a row-major [rows][cols] matrix, box = 128 bytes x box_rows, 128-byte swizzle.
+bool map_ffn(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, bool fp8, int box_rows) {
+    EncodeTiledFnF fn = encode_fn_ffn();
+    if (!fn) return false;
+    const int es = fp8 ? 1 : 2;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(cols * es)};
+    cuuint32_t box[2] = {(cuuint32_t)(FF_ROW_BYTES / es), (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
+              dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+// Both projections of the grouped FFN in one launch.  xp [rows][H] and hb [rows][F]
+// (bf16, or E4M3 codes), y [rows][H] bf16; done: max_sched ints, zero before the launch.
+cudaError_t launch_grouped_ffn(bool fp8, const void* w_up, const void* w_down, int E, int F, int H, const void* xp,
+                               void* hb, void* y, int64_t rows, const int4* sched, const int* n_sched, int* done,
+                               const GemmPlan& plan, const float* su, const float* sd, float x_scale, float h_scale,
+                               int num_sms, int debug_hold, const DevCtx& ctx, cudaStream_t stream) {
+    if (rows == 0) return cudaSuccess;
+    FfnMaps maps;
+    if (!map_ffn(&maps.ua128, w_up, (int64_t)E * F, H, fp8, 128) || !map_ffn(&maps.ua64, w_up, (int64_t)E * F, H, fp8, 64) ||
+        !map_ffn(&maps.ub128, xp, rows, H, fp8, 128) || !map_ffn(&maps.ub64, xp, rows, H, fp8, 64) ||
+        !map_ffn(&maps.ub16, xp, rows, H, fp8, 16) || !map_ffn(&maps.da128, w_down, (int64_t)E * H, F, fp8, 128) ||
+        !map_ffn(&maps.da64, w_down, (int64_t)E * H, F, fp8, 64) || !map_ffn(&maps.db128, hb, rows, F, fp8, 128) ||
+        !map_ffn(&maps.db64, hb, rows, F, fp8, 64) || !map_ffn(&maps.db16, hb, rows, F, fp8, 16))
+        return cudaErrorInvalidValue;
+    FfnArgs g;
+    g.sched = sched;
+    g.n_sched = n_sched;
+    g.done = done;
+    g.m_up = (F + FF_BM - 1) / FF_BM;
+    g.m_down = (H + FF_BM - 1) / FF_BM;
+    g.F = F;
+    g.H = H;
+    const int es = fp8 ? 1 : 2;
+    g.k_up = (int)(((int64_t)H * es + FF_ROW_BYTES - 1) / FF_ROW_BYTES);
+    g.k_down = (int)(((int64_t)F * es + FF_ROW_BYTES - 1) / FF_ROW_BYTES);
+    g.n_stages = plan.n_stages;
+    g.b_stage_bytes = plan.bn * FF_ROW_BYTES;
+    g.hb = hb;
+    g.y = y;
+    g.su = su;
+    g.sd = sd;
+    g.x_scale = x_scale;
+    g.h_scale = h_scale;
+    g.debug_hold = debug_hold;
+    const int64_t max_units = (int64_t)plan.max_sched * (g.m_up + g.m_down);
+    const int grid = (int)(max_units < num_sms ? max_units : num_sms);
+    auto kfn = fp8 ? grouped_ffn_kernel<true> : grouped_ffn_kernel<false>;
+    cudaError_t err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan.smem_bytes);
+    if (err != cudaSuccess) return err;
+    return launch_k(kfn, dim3(grid), dim3(FF_THREADS), plan.smem_bytes, stream, maps, g, ctx);
+}
+
+}  // namespace moe

@@ -10,9 +10,9 @@
 //
 // Same swap-AB orientation, schedule and TMA ring as the bf16 / E4M3 kernel:
 // a 128-row weight block is the MMA's M side, the expert's token rows (at most
-// 64 per schedule entry here) its N side.  A 128-byte K stage of E4M3 values
+// 128 per schedule entry here) its N side.  A 128-byte K stage of E4M3 values
 // is exactly one scale block, so every stage's product goes to its own TMEM
-// partial (one of four slots of 64 columns): the MMA overwrites the slot with
+// partial (one of four slots of 64 or 128 columns): the MMA overwrites the slot with
 // the block's sum, and the epilogue warps, which hold the running fp32 sums
 // of their weight row in registers, add s_w[f, b] times the partial and free
 // the slot.  Roles (192 threads): warp 0 TMA producer, warp 1 MMA, warps 2..5
@@ -32,9 +32,9 @@ constexpr int GB_THREADS = 192;
 constexpr int GB_BM = 128;                  // weight rows per unit
 constexpr int GB_ROW = 128;                 // bytes = E4M3 values of one K stage = one scale block
 constexpr int GB_A_BYTES = GB_BM * GB_ROW;  // 16 KB
-constexpr int GB_BN = 64;                   // token rows per schedule entry at most
-constexpr int GB_NP = 4;                    // TMEM partial slots of GB_BN columns
-constexpr int GB_TMEM_COLS = GB_NP * GB_BN;
+constexpr int GB_NP = 4;                    // TMEM partial slots of BN columns
+// BN: token rows per schedule entry at most, 64 or 128 (a template parameter: the
+// running sums are BN registers per thread); TMEM holds GB_NP slots of BN columns.
 
 struct B128Maps {
     CUtensorMap a128;   // weight codes [E * Nout][Kp], 128-row box
@@ -44,7 +44,7 @@ struct B128Maps {
 };
 
 struct B128Args {
-    const int4* sched;     // {e, row0, nrows, 0}, nrows <= GB_BN
+    const int4* sched;     // {e, row0, nrows, 0}, nrows <= BN
     const int* n_sched;
     int m_blocks;          // ceil(Nout / 128)
     int Nout;
@@ -59,7 +59,7 @@ struct B128Args {
     int debug_withhold;
 };
 
-template <bool UP>
+template <bool UP, int BN>
 __global__ void __launch_bounds__(GB_THREADS, 1)
     grouped_gemm_b128_kernel(const __grid_constant__ B128Maps maps, B128Args g, DevCtx ctx) {
     extern __shared__ uint8_t smem_raw[];
@@ -96,7 +96,7 @@ __global__ void __launch_bounds__(GB_THREADS, 1)
         tma_prefetch_desc(&maps.b64);
         tma_prefetch_desc(&maps.b16);
     }
-    if (warp == 1) tmem_alloc(smem_u32(tmem_holder), GB_TMEM_COLS);
+    if (warp == 1) tmem_alloc(smem_u32(tmem_holder), GB_NP * BN);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -168,7 +168,7 @@ __global__ void __launch_bounds__(GB_THREADS, 1)
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t d_tmem = tmem_base + (uint32_t)(ps * GB_BN);
+                    const uint32_t d_tmem = tmem_base + (uint32_t)(ps * BN);
                     const uint32_t a_base = smem_u32(smA + (size_t)stage * GB_A_BYTES);
                     const uint32_t b_base = smem_u32(smB + (size_t)stage * g.b_stage_bytes);
 #pragma unroll
@@ -206,9 +206,9 @@ __global__ void __launch_bounds__(GB_THREADS, 1)
             const bool fvalid = f < g.Nout;
             const int nch = (sc.z + 15) / 16;   // warp-uniform, <= 4
             const float* wrow = g.w_scale + ((int64_t)sc.x * g.Nout + (fvalid ? f : 0)) * g.k_stages;
-            float acc[GB_BN];
+            float acc[BN];
 #pragma unroll
-            for (int i = 0; i < GB_BN; ++i) acc[i] = 0.0f;
+            for (int i = 0; i < BN; ++i) acc[i] = 0.0f;
             for (int ks = 0; ks < g.k_stages; ++ks) {
                 if (!mbar_wait_warp(smem_u32(&pfull[ps]), pph, ctx, abort_flag)) {
                     ok = false;
@@ -216,9 +216,9 @@ __global__ void __launch_bounds__(GB_THREADS, 1)
                 }
                 tc_fence_after();
                 const float sw = wrow[ks];
-                const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(ps * GB_BN);
+                const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(ps * BN);
 #pragma unroll
-                for (int c = 0; c < GB_BN / 16; ++c) {
+                for (int c = 0; c < BN / 16; ++c) {
                     if (c < nch) {
                         uint32_t v[16];
                         tmem_ld16(t_row + (uint32_t)(c * 16), v);
@@ -236,7 +236,7 @@ __global__ void __launch_bounds__(GB_THREADS, 1)
             if (!ok) break;
             if (fvalid) {
 #pragma unroll
-                for (int c = 0; c < GB_BN / 16; ++c) {
+                for (int c = 0; c < BN / 16; ++c) {
                     if (c >= nch) break;
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
@@ -262,7 +262,7 @@ __global__ void __launch_bounds__(GB_THREADS, 1)
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, GB_TMEM_COLS);
+        tmem_dealloc(tmem_base, GB_NP * BN);
     }
 }
 
@@ -336,13 +336,14 @@ int b128_kp(int K) { return (K + 127) / 128 * 128; }
 
 // One FP8_B128 projection.  W: codes [E * Nout][Kp], w_scale [E][Nout][Kp / 128];
 // act: E4M3 codes [rows][Kdim] in the expert layout; out [rows][Nout] (e4m3 codes
-// for the up projection, bf16 for the down).  bn <= 64 (the schedule's tile).
+// for the up projection, bf16 for the down).  bn <= 128 (the schedule's tile): the
+// kernel's running sums are 64 registers per thread up to 64 rows, 128 beyond.
 cudaError_t launch_grouped_gemm_b128(bool up, const uint8_t* W, const float* w_scale, int E, int Nout, int Kdim,
                                      const uint8_t* act, int64_t rows, const int4* sched, const int* n_sched, int bn,
                                      int max_sched, void* out, float in_scale, float out_scale, int num_sms,
                                      int debug_withhold, const DevCtx& ctx, cudaStream_t stream) {
     if (rows == 0) return cudaSuccess;
-    if (bn < 16 || bn > GB_BN || bn % 16 != 0) return cudaErrorInvalidValue;
+    if (bn < 16 || bn > kB128MaxTileRows || bn % 16 != 0) return cudaErrorInvalidValue;
     const int Kp = b128_kp(Kdim);
     B128Maps maps;
     if (!make_map_u8_b128(&maps.a128, W, (int64_t)E * Nout, Kp, 128) ||
@@ -370,7 +371,8 @@ cudaError_t launch_grouped_gemm_b128(bool up, const uint8_t* W, const float* w_s
     const size_t smem = 1024 + (size_t)ns * stage + (size_t)(2 * ns + 2 * GB_NP + 1) * 8 + 16;
     const int64_t max_units = (int64_t)max_sched * g.m_blocks;
     const int grid = (int)(max_units < num_sms ? max_units : num_sms);
-    auto kfn = up ? grouped_gemm_b128_kernel<true> : grouped_gemm_b128_kernel<false>;
+    auto kfn = bn > 64 ? (up ? grouped_gemm_b128_kernel<true, 128> : grouped_gemm_b128_kernel<false, 128>)
+                       : (up ? grouped_gemm_b128_kernel<true, 64> : grouped_gemm_b128_kernel<false, 64>);
     cudaError_t err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     return launch_k(kfn, dim3(grid), dim3(GB_THREADS), smem, stream, maps, g, ctx);

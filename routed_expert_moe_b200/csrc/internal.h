@@ -36,7 +36,7 @@ cudaError_t launch_schedule(const int32_t* offsets, int E, int bn, int4* sched, 
                             int K, cudaStream_t stream);
 cudaError_t launch_gather(const uint16_t* x, const int32_t* perm_src, int64_t rows, int64_t routed_rows, int K,
                           int64_t T, int H, void* xp, bool fp8, float x_scale, int num_sms, const DevCtx& ctx,
-                          cudaStream_t stream);
+                          cudaStream_t stream, int* zero = nullptr, int n_zero = 0);
 struct GemmPlan {
     int bn;
     int n_stages;
@@ -49,6 +49,10 @@ cudaError_t launch_grouped_gemm(bool fp8, bool up, const void* W, int E, int Nou
                                 void* out, const float* w_scale, float in_scale, float out_scale, int num_sms,
                                 int debug_withhold, const DevCtx& ctx, cudaStream_t stream, const void* Ws,
                                 int n_shared);
+cudaError_t launch_grouped_ffn(bool fp8, const void* w_up, const void* w_down, int E, int F, int H, const void* xp,
+                               void* hb, void* y, int64_t rows, const int4* sched, const int* n_sched, int* done,
+                               const GemmPlan& plan, const float* su, const float* sd, float x_scale, float h_scale,
+                               int num_sms, int debug_hold, const DevCtx& ctx, cudaStream_t stream);
 cudaError_t launch_grouped_gemm_pair(bool fp8, bool up, const void* W, int E, int Nout, int Kdim, const void* act,
                                      int64_t rows, const int4* sched, const int* n_sched, int bn, int max_sched,
                                      void* out, const float* w_scale, float in_scale, float out_scale,
@@ -81,6 +85,10 @@ cudaError_t launch_quantize(int64_t n_tensors, int64_t elems, const uint16_t* sr
 
 cudaError_t launch_ep_regroup(const int64_t* recv_counts, int W, int E_loc, int64_t R, int32_t* offsets,
                               int32_t* perm, int32_t* inv, const DevCtx& ctx, cudaStream_t stream);
+
+// Token rows per schedule entry of the FP8_B128 grouped GEMM: its epilogue
+// keeps one running fp32 sum per row in registers.
+constexpr int kB128MaxTileRows = 128;
 
 // Token rows per schedule entry of the NVFP4 grouped GEMM: its two TMEM
 // accumulators of this many columns leave room for the scale factors.

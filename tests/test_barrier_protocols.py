@@ -413,6 +413,117 @@ def gemm_pair(sim, units, k_stages, NS, n_epi=4):
     sim.role("mma", mma())
 
 
+# ----------------------------------------------------------------------------- one-launch FFN (grouped_ffn.cu)
+
+def ffn_fused(sim, n_ctas, entries, m_up, m_down, k_up, k_down, NS, n_epi=4, plant=None):
+    """grouped_ffn_kernel on n_ctas CTAs: each walks units u = cta, cta + n_ctas, ... of the list
+    [up units (entry, block)] + [down units], with the per-CTA TMA ring and two accumulators of
+    the grouped GEMM.  A down unit of entry s reads H[s]; its producer first waits until the
+    global counter done[s] reaches n_epi * m_up (every epilogue warp of every up unit of s has
+    stored its rows and reported).  Shared: done[] and, per entry, how many up epilogue warps
+    have stored their rows of H."""
+    n_up, n_down = entries * m_up, entries * m_down
+    units = [("up", u // m_up) for u in range(n_up)] + [("down", u // m_down) for u in range(n_down)]
+    done = [0] * entries
+    stored = [0] * entries
+    target = n_epi * m_up if plant != "early_read" else n_epi * (m_up - 1)   # planted: one up unit short
+
+    def cta(c):
+        mine = units[c::n_ctas]
+        full, empty = [Bar(1) for _ in range(NS)], [Bar(1) for _ in range(NS)]
+        tfull, tempty = [Bar(1) for _ in range(2)], [Bar(n_epi) for _ in range(2)]
+        smem, fresh = [None] * NS, [False] * NS
+        tmem = [None] * 2
+
+        def producer():
+            st, ph = 0, 0
+            for i, (kind, s) in enumerate(mine):
+                if kind == "down":
+                    yield (lambda s=s: done[s] >= target)
+                ks_n = k_up if kind == "up" else k_down
+                for ks in range(ks_n):
+                    yield (lambda s_=st, p=ph: empty[s_].passed(p ^ 1))
+
+                    def land(s_=st, tag=(c, i, ks), kind=kind, s=s):
+                        check(not fresh[s_], f"CTA {c}: TMA overwrote stage {s_} before the MMA consumed it")
+                        if kind == "down":
+                            check(stored[s] == n_epi * m_up, f"CTA {c}: read H of entry {s} with "
+                                                             f"{stored[s]} of {n_epi * m_up} up warps stored")
+                        smem[s_], fresh[s_] = tag, True
+                        full[s_].arrive()
+                    sim.post(None, land)
+                    st += 1
+                    if st == NS:
+                        st, ph = 0, ph ^ 1
+
+        def mma():
+            st, ph, acc, aph = 0, 0, 0, 0
+            for i, (kind, s) in enumerate(mine):
+                yield (lambda a=acc, p=aph: tempty[a].passed(p ^ 1))
+                for ks in range(k_up if kind == "up" else k_down):
+                    yield (lambda s_=st, p=ph: full[s_].passed(p))
+                    check(smem[st] == (c, i, ks), f"CTA {c}: MMA read stage {st} holding {smem[st]}")
+
+                    def mma_done(s_=st):
+                        fresh[s_] = False
+                        empty[s_].arrive()
+                    sim.post(("tc", c), mma_done)
+                    st += 1
+                    if st == NS:
+                        st, ph = 0, ph ^ 1
+
+                def acc_done(a=acc, i=i):
+                    tmem[a] = i
+                    tfull[a].arrive()
+                sim.post(("tc", c), acc_done)
+                acc += 1
+                if acc == 2:
+                    acc, aph = 0, aph ^ 1
+
+        def epilogue(w):
+            acc, aph = 0, 0
+            for i, (kind, s) in enumerate(mine):
+                yield (lambda a=acc, p=aph: tfull[a].passed(p))
+                check(tmem[acc] == i, f"CTA {c}: epilogue read accumulator {acc} holding {tmem[acc]}")
+                tempty[acc].arrive()
+                if kind == "up":
+                    stored[s] += 1           # this warp's rows of H are stored (and fenced)
+                    yield (lambda: True)
+                    done[s] += 1             # then reported with a release add
+                acc += 1
+                if acc == 2:
+                    acc, aph = 0, aph ^ 1
+
+        sim.role(f"producer{c}", producer())
+        sim.role(f"mma{c}", mma())
+        for w in range(n_epi):
+            sim.role(f"epilogue{c}.{w}", epilogue(w))
+
+    for c in range(n_ctas):
+        cta(c)
+
+
+@pytest.mark.parametrize("n_ctas,entries,m_up,m_down,k_up,k_down,NS",
+                         [(3, 4, 3, 4, 4, 3, 3), (2, 5, 2, 3, 3, 2, 2), (4, 3, 2, 2, 2, 2, 4), (5, 2, 3, 2, 2, 3, 2)])
+def test_one_launch_ffn_protocol(n_ctas, entries, m_up, m_down, k_up, k_down, NS):
+    for seed in range(25):
+        sim = Sim(seed)
+        ffn_fused(sim, n_ctas, entries, m_up, m_down, k_up, k_down, NS)
+        assert sim.run() == "done"
+
+
+def test_a_down_unit_waiting_for_too_few_reports_is_caught():
+    caught = 0
+    for seed in range(25):
+        sim = Sim(seed)
+        ffn_fused(sim, 3, 4, 3, 4, 4, 3, 3, plant="early_read")
+        try:
+            sim.run()
+        except Violation:
+            caught += 1
+    assert caught > 0
+
+
 SEEDS = range(40)
 
 

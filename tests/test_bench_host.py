@@ -96,3 +96,16 @@ def test_traffic_is_used_only_while_the_sources_match(tmp_path, monkeypatch):
     assert bench.traffic_from_profile("up_gemm", "decode") == 1234
     (csrc / "a.cu").write_text("kernel v2")
     assert bench.traffic_from_profile("up_gemm", "decode") is None
+
+
+def test_one_launch_ffn_counts_both_projections():
+    """With both projections in one launch, the dominant kernel is that launch: the weight bytes
+    of both banks of the touched experts, the activations in and out of both, twice the flops."""
+    st = bench.stage_view({"up_gemm": 0.4, "down_gemm": 0.001, "combine": 0.01}, True)
+    assert set(st) == {"expert_ffn", "combine"} and st["expert_ffn"] == pytest.approx(0.401)
+    r = bench.roofline_entry(W.WORKLOADS[1], st, 121, PEAKS, "measured", "decode")
+    rows = 64 * 6
+    assert r["bound"] == "hbm" and r["kernel"].startswith("expert_ffn")
+    assert r["algorithmic_bytes_per_launch"] == 2 * 121 * F * H * 2 + rows * (H + F) * 2 + rows * (F + H) * 2
+    assert r["algorithmic_flops_per_launch"] == 2 * 2.0 * rows * F * H
+    assert bench.stage_view({"up_gemm": 1.0, "down_gemm": 2.0}, False) == {"up_gemm": 1.0, "down_gemm": 2.0}
