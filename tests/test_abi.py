@@ -161,21 +161,27 @@ def test_shared_expert_dims_and_pointers_are_checked_on_the_host(moe):
 def test_forward_launch_count_follows_the_dispatch(moe):
     """Router: one launch up to 256 tokens (expert-split clusters) and from 3072 (hidden-split
     clusters), two in between; permutation: one block up to 4096 assignments, else three kernels;
-    then the row gather, two projections and the combine."""
+    then the row gather, the expert FFN (one launch for bf16 and E4M3 experts without a shared
+    expert, else the two projections) and the combine."""
     count = lambda T, **kw: moe.forward_launches(moe.dims(T, 2688, 128, 6, 1856, **kw))
-    assert [count(T) for T in (0, 1, 64, 256, 257, 682, 683, 3071, 3072, 4096)] == [0, 6, 6, 6, 7, 7, 9, 9, 8, 8]
+    assert [count(T) for T in (0, 1, 64, 256, 257, 682, 683, 3071, 3072, 4096)] == [0, 5, 5, 5, 6, 6, 8, 8, 7, 7]
+    assert count(64, fp8=True) == 5
     assert count(64, nvfp4=True) == count(64, fp8_b128=True) == count(64, Fs=1856) == 6
     try:
+        moe.debug_set(8, 0)             # the two projections as two launches
+        assert count(64) == 6 and count(4096) == 8
+        moe.debug_set(8, 1)
         moe.debug_set(4, 0)             # never the expert-split clusters
-        assert count(64) == 7
+        assert count(64) == 6
         moe.debug_set(5, 2)             # always the hidden-split clusters
-        assert count(64) == 6 and count(576) == 6
+        assert count(64) == 5 and count(576) == 5
         moe.debug_set(5, 1)             # always the two kernels
-        assert count(4096) == 9
+        assert count(4096) == 8
     finally:
+        moe.debug_set(8, 1)
         moe.debug_set(4, -1)
         moe.debug_set(5, 0)
-    assert count(64) == 6
+    assert count(64) == 5
 
 
 def test_package_has_no_cpu_path():
