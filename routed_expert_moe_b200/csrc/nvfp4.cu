@@ -385,6 +385,7 @@ __global__ void __launch_bounds__(FG_THREADS, 1)
         // i + 128 into the stage's atoms; rows past the tile's rows get zero scales, so
         // their (unstored) products are zero rather than whatever the smem held.
         const int i = threadIdx.x - 192;
+        const int nbk = g.Kdim / 16;   // scale blocks along K; the rest of a padded scale row is masked
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
@@ -399,9 +400,21 @@ __global__ void __launch_bounds__(FG_THREADS, 1)
                     break;
                 }
                 uint8_t* st = smem + (size_t)stage * L.bytes;
+                // scales of blocks past K read as zero whatever the padding bytes hold (the H
+                // tensor's padding is never written), so that 0 codes times them stay 0
+                const int valid = min(16, max(0, nbk - ks * 16));
+                uint4 km;
+                km.x = valid >= 4 ? 0xFFFFFFFFu : (valid <= 0 ? 0u : (0xFFFFFFFFu >> (8 * (4 - valid))));
+                km.y = valid >= 8 ? 0xFFFFFFFFu : (valid <= 4 ? 0u : (0xFFFFFFFFu >> (8 * (8 - valid))));
+                km.z = valid >= 12 ? 0xFFFFFFFFu : (valid <= 8 ? 0u : (0xFFFFFFFFu >> (8 * (12 - valid))));
+                km.w = valid >= 16 ? 0xFFFFFFFFu : (valid <= 12 ? 0u : (0xFFFFFFFFu >> (8 * (16 - valid))));
                 {
-                    const uint4 v = i < arows ? *reinterpret_cast<const uint4*>(st + L.a_sc + 16 * i)
-                                              : make_uint4(0u, 0u, 0u, 0u);
+                    uint4 v = i < arows ? *reinterpret_cast<const uint4*>(st + L.a_sc + 16 * i)
+                                        : make_uint4(0u, 0u, 0u, 0u);
+                    v.x &= km.x;
+                    v.y &= km.y;
+                    v.z &= km.z;
+                    v.w &= km.w;
                     uint8_t* at = st + L.a_atoms + 16 * (i % 32) + 4 * (i / 32);
                     *reinterpret_cast<uint32_t*>(at) = v.x;
                     *reinterpret_cast<uint32_t*>(at + FG_ATOM) = v.y;
@@ -409,8 +422,12 @@ __global__ void __launch_bounds__(FG_THREADS, 1)
                     *reinterpret_cast<uint32_t*>(at + 3 * FG_ATOM) = v.w;
                 }
                 for (int n = i; n < L.nbat * 128; n += 128) {
-                    const uint4 v = n < nrows ? *reinterpret_cast<const uint4*>(st + L.b_sc + 16 * n)
-                                              : make_uint4(0u, 0u, 0u, 0u);
+                    uint4 v = n < nrows ? *reinterpret_cast<const uint4*>(st + L.b_sc + 16 * n)
+                                        : make_uint4(0u, 0u, 0u, 0u);
+                    v.x &= km.x;
+                    v.y &= km.y;
+                    v.z &= km.z;
+                    v.w &= km.w;
                     uint8_t* at = st + L.b_atoms + (n / 128) * FG_ATOM + 16 * (n % 32) + 4 * ((n / 32) % 4);
                     const int kstep = L.nbat * FG_ATOM;
                     *reinterpret_cast<uint32_t*>(at) = v.x;

@@ -186,7 +186,20 @@ def test_fp8_forward_parity_decode_shape(moe):
 
 # --------------------------------------------------------------------------- bounded waits
 
-def test_expired_wait_is_reported_and_the_context_stays_usable(moe):
+@pytest.mark.parametrize("one_launch", [1, 0], ids=["one_launch_ffn", "two_launches"])
+def test_expired_wait_is_reported_and_the_context_stays_usable(moe, one_launch):
+    """Two launches: block 0's producer withholds its first load, so the MMA's wait expires.
+    One launch: block 0's first up unit withholds its report, so the down units of its entry
+    wait on the counter in vain.  Either way the status is MOE_ETIMEOUT and the next call is
+    right."""
+    moe.debug_set(8, one_launch)
+    try:
+        _expired_wait_case(moe)
+    finally:
+        moe.debug_set(8, 1)
+
+
+def _expired_wait_case(moe):
     w = W.WORKLOADS[0]
     h = inputs(w)
     d = device_inputs(h)
@@ -196,7 +209,7 @@ def test_expired_wait_is_reported_and_the_context_stays_usable(moe):
     ws = moe.alloc_workspace(dims)
     y = torch.empty(w.T * w.K, w.H, dtype=torch.bfloat16, device="cuda")
     moe.debug_set(1, 20_000_000)   # 20 ms limit on every bounded wait
-    moe.debug_set(2, 1)            # block 0's producer withholds its first load
+    moe.debug_set(2, 1)            # block 0 withholds its first load (or its first report)
     try:
         moe.expert_ffn(dims, d["x"], dev(offsets), dev(perm_src), d["wu"], d["wd"], None, y, ws)
         assert moe.check_device_error_status() == moe.MOE_ETIMEOUT
@@ -234,3 +247,41 @@ def test_cta_pair_gemm_matches_oracle(moe, fp8):
             assert rel_err(host_f64(out), r["out"]) <= BF16_TOL
     finally:
         moe.debug_set(3, 0)
+
+
+# --------------------------------------------------------------------------- one-launch expert FFN
+
+@pytest.mark.parametrize("fp8", [False, True])
+@pytest.mark.parametrize("w", [W.WORKLOADS[1], W.WORKLOADS[3],
+                               W.Workload("ffn_T700_E16_K4", 700, 512, 16, 4, 320, seed=23)],
+                         ids=lambda w: w.name if hasattr(w, "name") else str(w))
+def test_one_launch_ffn_equals_two_launches_bitwise(moe, w, fp8):
+    """Both projections in one launch compute exactly the products of the two launches (same
+    tiles, same accumulation order), so the layer output is the same bit for bit."""
+    h = inputs(w)
+    d = device_inputs(h)
+    dims = moe.dims(w.T, w.H, w.E, w.K, w.F, fp8=fp8)
+    ws = moe.alloc_workspace(dims)
+    scales = None
+    wu, wd = d["wu"], d["wd"]
+    if fp8:
+        cu = torch.empty(wu.shape, dtype=torch.uint8, device="cuda")
+        cd = torch.empty(wd.shape, dtype=torch.uint8, device="cuda")
+        su = torch.empty(w.E, dtype=torch.float32, device="cuda")
+        sd = torch.empty(w.E, dtype=torch.float32, device="cuda")
+        moe.quantize_fp8(wu, cu, su)
+        moe.quantize_fp8(wd, cd, sd)
+        sx, sh = oracle.calibrate_fp8(h["x"][:64], h["wr"], h["bias"], h["wu"], w.K)
+        scales = moe.fp8_scales(su, sd, float(sx), float(sh))
+        wu, wd = cu, cd
+    outs = []
+    for one in (1, 0):
+        moe.debug_set(8, one)
+        try:
+            out = torch.empty(w.T, w.H, dtype=torch.bfloat16, device="cuda")
+            moe.forward(dims, d["x"], d["wr"], d["bias"], wu, wd, out, ws, scales=scales)
+            moe.check_device_error()
+            outs.append(out)
+        finally:
+            moe.debug_set(8, 1)
+    assert torch.equal(outs[0], outs[1])

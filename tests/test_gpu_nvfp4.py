@@ -75,9 +75,11 @@ def test_activation_quantiser_bit_exact(moe, x_scale):
     assert np.array_equal(b[:, :H // 16], s_ref) and not b[:, H // 16:].any()
 
 
-def nvfp4_case(moe, w, h, tokens=None, slot_experts=None):
+def nvfp4_case(moe, w, h, tokens=None, slot_experts=None, ws_fill=None):
     """Quantise banks on the GPU (checked bit-exact against the oracle), calibrate static
-    tensor scales with the oracle, run the layer on both sides."""
+    tensor scales with the oracle, run the layer on both sides.  ws_fill: a byte written over
+    the whole workspace first (0x7F is an E4M3 NaN: stale workspace bytes must not reach the
+    tensor cores as scales)."""
     bank_up = oracle.quantize_bank_nvfp4(h["wu"])
     bank_down = oracle.quantize_bank_nvfp4(h["wd"])
     cu, bu, tu = gpu_bank(moe, h["wu"])
@@ -86,6 +88,8 @@ def nvfp4_case(moe, w, h, tokens=None, slot_experts=None):
     tx, th = oracle.calibrate_nvfp4(h["x"][:64], h["wr"], h["bias"], h["wu"], w.K)
     dims = moe.dims(w.T, w.H, w.E, w.K, w.F, nvfp4=True)
     ws = moe.alloc_workspace(dims)
+    if ws_fill is not None:
+        ws.fill_(ws_fill)
     out = torch.empty(w.T, w.H, dtype=torch.bfloat16, device="cuda")
     idx = torch.empty(w.T, w.K, dtype=torch.int32, device="cuda")
     sc = moe.nvfp4_scales(tu, td, float(tx), float(th), bu, bd)
@@ -103,6 +107,15 @@ def nvfp4_case(moe, w, h, tokens=None, slot_experts=None):
                          ids=lambda w: w.name)
 def test_nvfp4_forward_parity_small(moe, w):
     assert nvfp4_case(moe, w, inputs(w)) <= NVFP4_TOL
+
+
+@pytest.mark.parametrize("w", [W.Workload("nvfp4_tail_F224_T300", 300, 256, 8, 3, 224, seed=27),
+                               W.Workload("nvfp4_tail_H288_F96", 40, 288, 8, 2, 96, seed=29)],
+                         ids=lambda w: w.name)
+def test_nvfp4_forward_ignores_stale_workspace_bytes(moe, w):
+    """K = 224 (or 96, 288) is not a whole stage of 256: the last stage's padding blocks are
+    masked, so a workspace full of E4M3 NaN bytes gives the same, finite result."""
+    assert nvfp4_case(moe, w, inputs(w), ws_fill=0x7F) <= NVFP4_TOL
 
 
 def test_nvfp4_forward_parity_decode_shape(moe):
