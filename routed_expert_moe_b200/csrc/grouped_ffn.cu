@@ -12,8 +12,9 @@
 // boundary (every down unit waits for every up unit, and the last up wave
 // leaves SMs idle), the producer of a down unit waits only for entry s:
 //   up epilogue   each of the four epilogue warps stores its rows of H, every
-//                 lane fences (generic -> async proxy, then device scope), and
-//                 lane 0 adds 1 to done[s] with release semantics;
+//                 lane fences its stores for the async proxy, the warp
+//                 synchronises, and lane 0 adds 1 to done[s] with release
+//                 semantics (cumulative over the warp's stores);
 //   down producer spins (bounded) on an acquire load of done[s] until it
 //                 reaches 4 * m_up, fences the async proxy, then issues the
 //                 TMA loads of H.
@@ -113,6 +114,9 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
     uint64_t* drain = tempty + 2;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(drain + 1);
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1) + 1;
+    // the epilogue warps' turn-around tiles: 16 x 32 fp32 each, 16-byte aligned
+    float* tbuf = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(tmem_holder + 1) + 15) &
+                                           ~static_cast<uintptr_t>(15));
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     if (threadIdx.x == 0) {
@@ -255,7 +259,13 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
             }
         }
     } else {
+        // Epilogue: a warp reads 32 weight rows (features) x 16 token columns from TMEM, one
+        // feature per lane, and turns the tile around through shared memory so that each lane
+        // holds 16 consecutive features of one token: the conversions then go two values per
+        // instruction and every lane stores 32 (bf16) or 16 (E4M3) contiguous bytes.
         const int q = warp & 3;   // TMEM lane quadrant of this warp
+        float* tb = tbuf + (warp - 2) * (16 * 32);
+        const int tj = lane & 15, th = lane >> 4;   // after the turn: token column, feature half
         int acc = 0;
         uint32_t acc_phase = 0;
         const float inv_h = (FP8) ? __frcp_rn(g.h_scale) : 1.0f;
@@ -268,8 +278,7 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
             const int Nout = up ? g.F : g.H;
             if (!mbar_wait_warp(smem_u32(&tfull[acc]), acc_phase, ctx, abort_flag)) break;
             tc_fence_after();
-            const int f = mb * FF_BM + q * 32 + lane;
-            const bool fvalid = f < Nout;
+            const int f16 = mb * FF_BM + q * 32 + th * 16;   // first of this lane's 16 features
             float scale = 1.0f;
             if constexpr (FP8) scale = up ? __fmul_rn(g.su[sc.x], g.x_scale) : __fmul_rn(g.sd[sc.x], g.h_scale);
             const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * 256);
@@ -277,43 +286,63 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
             for (int c = 0; c < nchunks; ++c) {
                 uint32_t vv[16];
                 tmem_ld16(t_row + (uint32_t)(c * 16), vv);
-                if (fvalid) {
-                    if (up) {
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const int r = c * 16 + j;
-                            if (r < sc.z) {
-                                float z = __uint_as_float(vv[j]);
-                                if constexpr (FP8) z = __fmul_rn(z, scale);
-                                const float a = z > 0.0f ? __fmul_rn(z, z) : 0.0f;
-                                const int64_t o = (int64_t)(sc.y + r) * g.F + f;
-                                if constexpr (FP8)
-                                    static_cast<uint8_t*>(g.hb)[o] = (uint8_t)__nv_cvt_float_to_fp8(
-                                        __fmul_rn(a, inv_h), __NV_SATFINITE, __NV_E4M3);
-                                else
-                                    static_cast<__nv_bfloat16*>(g.hb)[o] = __float2bfloat16_rn(a);
-                            }
+                for (int j = 0; j < 16; ++j) {
+                    float z = __uint_as_float(vv[j]);
+                    if constexpr (FP8) z = __fmul_rn(z, scale);
+                    if (up) z = z > 0.0f ? __fmul_rn(z, z) : 0.0f;
+                    // row j, feature `lane`: 16-byte chunk (lane / 4) xor (j mod 8)
+                    tb[j * 32 + (((lane >> 2) ^ (j & 7)) << 2) + (lane & 3)] = z;
+                }
+                __syncwarp();
+                float a[16];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float4 t4 = *reinterpret_cast<const float4*>(tb + tj * 32 + (((4 * th + k) ^ (tj & 7)) << 2));
+                    a[4 * k] = t4.x;
+                    a[4 * k + 1] = t4.y;
+                    a[4 * k + 2] = t4.z;
+                    a[4 * k + 3] = t4.w;
+                }
+                __syncwarp();
+                const int r = c * 16 + tj;
+                if (r < sc.z && f16 < Nout) {
+                    const int64_t row = sc.y + r;
+                    if (up && FP8) {
+                        uint32_t w4[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const uint32_t lo = __nv_cvt_float2_to_fp8x2(
+                                make_float2(__fmul_rn(a[4 * i], inv_h), __fmul_rn(a[4 * i + 1], inv_h)),
+                                __NV_SATFINITE, __NV_E4M3);
+                            const uint32_t hi = __nv_cvt_float2_to_fp8x2(
+                                make_float2(__fmul_rn(a[4 * i + 2], inv_h), __fmul_rn(a[4 * i + 3], inv_h)),
+                                __NV_SATFINITE, __NV_E4M3);
+                            w4[i] = (lo & 0xFFFFu) | (hi << 16);
                         }
+                        *reinterpret_cast<uint4*>(static_cast<uint8_t*>(g.hb) + row * g.F + f16) =
+                            make_uint4(w4[0], w4[1], w4[2], w4[3]);
                     } else {
+                        uint32_t w8[8];
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const int r = c * 16 + j;
-                            if (r < sc.z) {
-                                float z = __uint_as_float(vv[j]);
-                                if constexpr (FP8) z = __fmul_rn(z, scale);
-                                static_cast<__nv_bfloat16*>(g.y)[(int64_t)(sc.y + r) * g.H + f] = __float2bfloat16_rn(z);
-                            }
+                        for (int i = 0; i < 8; ++i) {
+                            const __nv_bfloat162 p2 = __floats2bfloat162_rn(a[2 * i], a[2 * i + 1]);
+                            w8[i] = *reinterpret_cast<const uint32_t*>(&p2);
                         }
+                        __nv_bfloat16* dst = up ? static_cast<__nv_bfloat16*>(g.hb) + row * g.F + f16
+                                                : static_cast<__nv_bfloat16*>(g.y) + row * g.H + f16;
+                        uint4* d4 = reinterpret_cast<uint4*>(dst);
+                        d4[0] = make_uint4(w8[0], w8[1], w8[2], w8[3]);
+                        d4[1] = make_uint4(w8[4], w8[5], w8[6], w8[7]);
                     }
                 }
             }
             tc_fence_before();
             mbar_arrive(smem_u32(&tempty[acc]));
             if (up) {
-                // this warp's rows of H are complete: make them visible to the TMA loads of
-                // other CTAs, then report them to the entry's down units
+                // this warp's rows of H are complete: every lane orders its stores for the async
+                // proxy (the TMA loads of H), the warp barrier orders them before lane 0's release
                 fence_proxy_async_global();
-                __threadfence();
                 __syncwarp();
                 const bool hold = g.debug_hold && blockIdx.x == 0 && u == (int)blockIdx.x;
                 if (lane == 0 && !hold) red_release_add(g.done + s_idx, 1);
@@ -402,9 +431,10 @@ cudaError_t launch_grouped_ffn(bool fp8, const void* w_up, const void* w_down, i
     const int64_t max_units = (int64_t)plan.max_sched * (g.m_up + g.m_down);
     const int grid = (int)(max_units < num_sms ? max_units : num_sms);
     auto kfn = fp8 ? grouped_ffn_kernel<true> : grouped_ffn_kernel<false>;
-    cudaError_t err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan.smem_bytes);
+    const size_t smem = plan.smem_bytes + 16 + (size_t)FF_EPI_WARPS * 16 * 32 * sizeof(float);
+    cudaError_t err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
-    return launch_k(kfn, dim3(grid), dim3(FF_THREADS), plan.smem_bytes, stream, maps, g, ctx);
+    return launch_k(kfn, dim3(grid), dim3(FF_THREADS), smem, stream, maps, g, ctx);
 }
 
 }  // namespace moe

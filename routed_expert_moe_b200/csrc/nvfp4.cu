@@ -195,7 +195,9 @@ __global__ void __launch_bounds__(256) nvfp4_gather_kernel(const uint16_t* __res
 //   warp 1      TMEM allocator; one lane copies each stage's atoms to TMEM and
 //               issues the four block-scaled MMAs into one of two accumulators;
 //   warps 2..5  epilogue: tensor scales, ReLU^2 and the NVFP4 quantisation of
-//               H (up) or the bf16 store (down); warp w reads lanes 32*(w%4)..;
+//               H (up) or the bf16 store (down); warp w reads lanes 32*(w%4)..
+//               and turns each 32 x 16 tile around in shared memory so that a
+//               lane holds one 16-feature block of one token;
 //   warps 6..9  scale warps: thread i writes row i's (and row i + 128's)
 //               scales into the stage's atoms, zero for rows a tile lacks.
 constexpr int FG_THREADS = 320;
@@ -297,6 +299,8 @@ __global__ void __launch_bounds__(FG_THREADS, 1)
     uint64_t* drain = tempty + 2;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(drain + 1);
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1) + 1;
+    float* tbuf = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(tmem_holder + 1) + 15) &
+                                           ~static_cast<uintptr_t>(15));   // 4 x (16 x 32) fp32
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     if (threadIdx.x == 0) {
@@ -501,19 +505,25 @@ __global__ void __launch_bounds__(FG_THREADS, 1)
         }
     } else {
         // ---------------------------------------------------------------- epilogue (warps 2..5)
+        // A warp reads 32 weight rows (features) x 16 token columns from TMEM, one feature per
+        // lane, and turns the tile around through shared memory: each lane then holds 16
+        // consecutive features of one token -- exactly one NVFP4 block of H (up), or 32 bytes
+        // of bf16 Y (down) -- so the block amax needs no shuffles, the block's scale and its
+        // reciprocal are computed once, and the stores are 8- or 32-byte vectors.
         const int q = warp & 3;
+        float* tb = tbuf + (warp - 2) * (16 * 32);
+        const int tj = lane & 15, th = lane >> 4;
         int acc = 0;
         uint32_t acc_phase = 0;
         const int fsp = (g.Nout / 16 + 15) / 16 * 16;   // padded block-scale row of the H tensor (up)
+        const float r6 = __frcp_rn(6.0f), rts = __frcp_rn(g.out_tscale);   // quotients via nv_div
         for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
             const int4 sc = g.sched[u / g.m_blocks];
             const int mb = u % g.m_blocks;
             if (!mbar_wait_warp(smem_u32(&tfull[acc]), acc_phase, ctx, abort_flag)) break;
             tc_fence_after();
-            const int f = mb * FG_BM + q * 32 + lane;
-            const bool fvalid = f < g.Nout;
+            const int f16 = mb * FG_BM + q * 32 + th * 16;   // first feature of this lane's block
             const float scale = __fmul_rn(g.w_tscale[sc.x], g.in_tscale);
-            const float r6 = __frcp_rn(6.0f), rts = __frcp_rn(g.out_tscale);   // quotients via nv_div
             const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * FG_ACC_COLS);
             const int nchunks = (sc.z + 15) / 16;
             for (int c = 0; c < nchunks; ++c) {
@@ -521,30 +531,52 @@ __global__ void __launch_bounds__(FG_THREADS, 1)
                 tmem_ld16(t_row + (uint32_t)(c * 16), v);
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
-                    const int r = c * 16 + j;
-                    const float z = __fmul_rn(__uint_as_float(v[j]), scale);
-                    if constexpr (UP) {
-                        // H = relu(z)^2 in blocks of 16 features (this half warp), quantised with s_h
-                        const float a = z > 0.0f ? __fmul_rn(z, z) : 0.0f;
-                        float amax = a;
+                    float z = __fmul_rn(__uint_as_float(v[j]), scale);
+                    if constexpr (UP) z = z > 0.0f ? __fmul_rn(z, z) : 0.0f;   // H = relu(z)^2
+                    tb[j * 32 + (((lane >> 2) ^ (j & 7)) << 2) + (lane & 3)] = z;
+                }
+                __syncwarp();
+                float a[16];
 #pragma unroll
-                        for (int off = 8; off > 0; off >>= 1)
-                            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+                for (int k = 0; k < 4; ++k) {
+                    const float4 t4 = *reinterpret_cast<const float4*>(tb + tj * 32 + (((4 * th + k) ^ (tj & 7)) << 2));
+                    a[4 * k] = t4.x;
+                    a[4 * k + 1] = t4.y;
+                    a[4 * k + 2] = t4.z;
+                    a[4 * k + 3] = t4.w;
+                }
+                __syncwarp();
+                const int r = c * 16 + tj;
+                if (r < sc.z && f16 < g.Nout) {
+                    const int64_t row = sc.y + r;
+                    if constexpr (UP) {
+                        // one block of 16 features, quantised with the static tensor scale s_h
+                        float amax = 0.0f;
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) amax = fmaxf(amax, a[i]);
                         const uint32_t scode = e4m3_code(nv_div(nv_div(amax, 6.0f, r6), g.out_tscale, rts));
                         const float e = __fmul_rn(e4m3_value(scode), g.out_tscale);
-                        const float qv = e != 0.0f ? nv_div(a, e, __frcp_rn(e)) : 0.0f;
-                        const float qn = __shfl_down_sync(0xffffffffu, qv, 1);   // the odd neighbour
-                        if (r < sc.z && fvalid) {
-                            const int64_t row = sc.y + r;
-                            if ((lane & 1) == 0)
-                                static_cast<uint8_t*>(g.out)[row * (g.Nout / 2) + f / 2] =
-                                    e != 0.0f ? (uint8_t)e2m1_pack(qv, qn) : (uint8_t)0;
-                            if ((lane & 15) == 0) g.out_scale[row * fsp + f / 16] = (uint8_t)scode;
+                        uint32_t packed[2] = {0u, 0u};
+                        if (e != 0.0f) {
+                            const float y = __frcp_rn(e);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i)
+                                packed[i / 4] |= e2m1_pack(nv_div(a[2 * i], e, y), nv_div(a[2 * i + 1], e, y))
+                                                 << (8 * (i % 4));
                         }
+                        *reinterpret_cast<uint2*>(static_cast<uint8_t*>(g.out) + row * (g.Nout / 2) + f16 / 2) =
+                            make_uint2(packed[0], packed[1]);
+                        g.out_scale[row * fsp + f16 / 16] = (uint8_t)scode;
                     } else {
-                        if (r < sc.z && fvalid)
-                            static_cast<__nv_bfloat16*>(g.out)[(int64_t)(sc.y + r) * g.Nout + f] =
-                                __float2bfloat16_rn(z);
+                        uint32_t w8[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const __nv_bfloat162 p2 = __floats2bfloat162_rn(a[2 * i], a[2 * i + 1]);
+                            w8[i] = *reinterpret_cast<const uint32_t*>(&p2);
+                        }
+                        uint4* d4 = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) + row * g.Nout + f16);
+                        d4[0] = make_uint4(w8[0], w8[1], w8[2], w8[3]);
+                        d4[1] = make_uint4(w8[4], w8[5], w8[6], w8[7]);
                     }
                 }
             }
@@ -600,13 +632,13 @@ static bool make_map_u8(CUtensorMap* m, const void* base, int64_t rows, int64_t 
 static int ksp_of(int K) { return (K / 16 + 15) / 16 * 16; }
 
 // Ring depth of the NVFP4 kernel for entries of up to bn token rows: as many stages as fit in
-// 225 KB of shared memory, at most 8.
+// 216 KB of shared memory, at most 8; then the barriers and the epilogue's 8 KB turn-around tiles.
 static int fp4_stages(int bn, size_t* smem) {
     const Fp4Stage L(bn);
-    int ns = (225 * 1024) / L.bytes;
+    int ns = (216 * 1024) / L.bytes;
     if (ns > 8) ns = 8;
     if (ns < 2) ns = 2;
-    *smem = 1024 + (size_t)ns * L.bytes + (size_t)(3 * ns + 5) * 8 + 16;
+    *smem = 1024 + (size_t)ns * L.bytes + (size_t)(3 * ns + 5) * 8 + 32 + 4 * 16 * 32 * sizeof(float);
     return ns;
 }
 
