@@ -114,9 +114,9 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
     uint64_t* drain = tempty + 2;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(drain + 1);
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1) + 1;
-    // the epilogue warps' turn-around tiles: 16 x 32 fp32 each, 16-byte aligned
-    float* tbuf = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(tmem_holder + 1) + 15) &
-                                           ~static_cast<uintptr_t>(15));
+    // the epilogue warps' turn-around tiles: 16 x 32 16-bit values each, 16-byte aligned
+    uint16_t* tbuf = reinterpret_cast<uint16_t*>((reinterpret_cast<uintptr_t>(tmem_holder + 1) + 15) &
+                                                 ~static_cast<uintptr_t>(15));
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     if (threadIdx.x == 0) {
@@ -260,12 +260,12 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
         }
     } else {
         // Epilogue: a warp reads 32 weight rows (features) x 16 token columns from TMEM, one
-        // feature per lane, and turns the tile around through shared memory so that each lane
-        // holds 16 consecutive features of one token: the conversions then go two values per
-        // instruction and every lane stores 32 (bf16) or 16 (E4M3) contiguous bytes.
+        // feature per lane, rounds them to their stored type and turns the tile around
+        // through shared memory, so that each lane holds 16 consecutive features of one token
+        // and stores them as 32 (bf16) or 16 (E4M3) contiguous bytes.
         const int q = warp & 3;   // TMEM lane quadrant of this warp
-        float* tb = tbuf + (warp - 2) * (16 * 32);
-        const int tj = lane & 15, th = lane >> 4;   // after the turn: token column, feature half
+        uint16_t* tb = tbuf + (warp - 2) * (16 * 32);   // 16 rows x 32 bf16 (or E4M3 codes in the low byte)
+        const int tj = lane & 15, th = lane >> 4;       // after the turn: token column, feature half
         int acc = 0;
         uint32_t acc_phase = 0;
         const float inv_h = (FP8) ? __frcp_rn(g.h_scale) : 1.0f;
@@ -287,53 +287,51 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
                 uint32_t vv[16];
                 tmem_ld16(t_row + (uint32_t)(c * 16), vv);
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    float z = __uint_as_float(vv[j]);
-                    if constexpr (FP8) z = __fmul_rn(z, scale);
-                    if (up) z = z > 0.0f ? __fmul_rn(z, z) : 0.0f;
-                    // row j, feature `lane`: 16-byte chunk (lane / 4) xor (j mod 8)
-                    tb[j * 32 + (((lane >> 2) ^ (j & 7)) << 2) + (lane & 3)] = z;
+                for (int j = 0; j < 16; j += 2) {
+                    // token columns j and j + 1 of this lane's feature, converted as a pair
+                    float z0 = __uint_as_float(vv[j]), z1 = __uint_as_float(vv[j + 1]);
+                    if constexpr (FP8) {
+                        z0 = __fmul_rn(z0, scale);
+                        z1 = __fmul_rn(z1, scale);
+                    }
+                    if (up) {
+                        z0 = z0 > 0.0f ? __fmul_rn(z0, z0) : 0.0f;
+                        z1 = z1 > 0.0f ? __fmul_rn(z1, z1) : 0.0f;
+                    }
+                    uint32_t pair;
+                    if (up && FP8) {
+                        pair = __nv_cvt_float2_to_fp8x2(make_float2(__fmul_rn(z0, inv_h), __fmul_rn(z1, inv_h)),
+                                                        __NV_SATFINITE, __NV_E4M3);
+                        pair = (pair & 0xFFu) | ((pair & 0xFF00u) << 8);   // one code per 16-bit slot
+                    } else {
+                        const __nv_bfloat162 p2 = __floats2bfloat162_rn(z0, z1);
+                        pair = *reinterpret_cast<const uint32_t*>(&p2);
+                    }
+                    // row j, feature `lane`: 16-byte chunk (lane / 8) xor (j mod 4)
+                    tb[j * 32 + ((((lane >> 3) ^ (j & 3))) << 3) + (lane & 7)] = (uint16_t)(pair & 0xFFFFu);
+                    tb[(j + 1) * 32 + ((((lane >> 3) ^ ((j + 1) & 3))) << 3) + (lane & 7)] = (uint16_t)(pair >> 16);
                 }
                 __syncwarp();
-                float a[16];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const float4 t4 = *reinterpret_cast<const float4*>(tb + tj * 32 + (((4 * th + k) ^ (tj & 7)) << 2));
-                    a[4 * k] = t4.x;
-                    a[4 * k + 1] = t4.y;
-                    a[4 * k + 2] = t4.z;
-                    a[4 * k + 3] = t4.w;
-                }
+                const uint4 c0 = *reinterpret_cast<const uint4*>(tb + tj * 32 + (((2 * th) ^ (tj & 3)) << 3));
+                const uint4 c1 = *reinterpret_cast<const uint4*>(tb + tj * 32 + (((2 * th + 1) ^ (tj & 3)) << 3));
                 __syncwarp();
                 const int r = c * 16 + tj;
                 if (r < sc.z && f16 < Nout) {
                     const int64_t row = sc.y + r;
                     if (up && FP8) {
-                        uint32_t w4[4];
+                        // 16 codes, one per 16-bit slot: keep the low bytes
+                        const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+                        uint32_t p4[4];
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const uint32_t lo = __nv_cvt_float2_to_fp8x2(
-                                make_float2(__fmul_rn(a[4 * i], inv_h), __fmul_rn(a[4 * i + 1], inv_h)),
-                                __NV_SATFINITE, __NV_E4M3);
-                            const uint32_t hi = __nv_cvt_float2_to_fp8x2(
-                                make_float2(__fmul_rn(a[4 * i + 2], inv_h), __fmul_rn(a[4 * i + 3], inv_h)),
-                                __NV_SATFINITE, __NV_E4M3);
-                            w4[i] = (lo & 0xFFFFu) | (hi << 16);
-                        }
+                        for (int i = 0; i < 4; ++i)
+                            p4[i] = __byte_perm(w[2 * i], w[2 * i + 1], 0x6420);
                         *reinterpret_cast<uint4*>(static_cast<uint8_t*>(g.hb) + row * g.F + f16) =
-                            make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                            make_uint4(p4[0], p4[1], p4[2], p4[3]);
                     } else {
-                        uint32_t w8[8];
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const __nv_bfloat162 p2 = __floats2bfloat162_rn(a[2 * i], a[2 * i + 1]);
-                            w8[i] = *reinterpret_cast<const uint32_t*>(&p2);
-                        }
-                        __nv_bfloat16* dst = up ? static_cast<__nv_bfloat16*>(g.hb) + row * g.F + f16
-                                                : static_cast<__nv_bfloat16*>(g.y) + row * g.H + f16;
-                        uint4* d4 = reinterpret_cast<uint4*>(dst);
-                        d4[0] = make_uint4(w8[0], w8[1], w8[2], w8[3]);
-                        d4[1] = make_uint4(w8[4], w8[5], w8[6], w8[7]);
+                        uint4* d4 = reinterpret_cast<uint4*>(up ? static_cast<uint16_t*>(g.hb) + row * g.F + f16
+                                                                : static_cast<uint16_t*>(g.y) + row * g.H + f16);
+                        d4[0] = c0;
+                        d4[1] = c1;
                     }
                 }
             }
@@ -431,7 +429,7 @@ cudaError_t launch_grouped_ffn(bool fp8, const void* w_up, const void* w_down, i
     const int64_t max_units = (int64_t)plan.max_sched * (g.m_up + g.m_down);
     const int grid = (int)(max_units < num_sms ? max_units : num_sms);
     auto kfn = fp8 ? grouped_ffn_kernel<true> : grouped_ffn_kernel<false>;
-    const size_t smem = plan.smem_bytes + 16 + (size_t)FF_EPI_WARPS * 16 * 32 * sizeof(float);
+    const size_t smem = plan.smem_bytes + 16 + (size_t)FF_EPI_WARPS * 16 * 32 * sizeof(uint16_t);
     cudaError_t err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     return launch_k(kfn, dim3(grid), dim3(FF_THREADS), smem, stream, maps, g, ctx);

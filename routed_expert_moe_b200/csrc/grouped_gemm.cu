@@ -370,11 +370,13 @@ GemmPlan gemm_plan(int64_t T, int K, int E) {
     const int64_t rows = T * K;
     int64_t per_expert_max = T < rows ? T : rows;   // an expert gets each token at most once
     int bn = (int)((per_expert_max + 15) / 16 * 16);
-    if (bn > 256) bn = 256;
+    // 224 rows: a prefill chunk's experts (~192 rows each, rarely above 224) take one tile each,
+    // and five stages of 16 KB of weights + 28 KB of rows fit the ring's 220 KB
+    if (bn > 224) bn = 224;
     if (bn < 16) bn = 16;
     p.bn = bn;
     const int stage = GG_A_BYTES + bn * GG_ROW_BYTES;
-    int ns = (200 * 1024) / stage;
+    int ns = (220 * 1024) / stage;
     if (ns > 8) ns = 8;
     if (ns < 2) ns = 2;
     p.n_stages = ns;
