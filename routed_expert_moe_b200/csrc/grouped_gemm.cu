@@ -370,9 +370,13 @@ GemmPlan gemm_plan(int64_t T, int K, int E) {
     const int64_t rows = T * K;
     int64_t per_expert_max = T < rows ? T : rows;   // an expert gets each token at most once
     int bn = (int)((per_expert_max + 15) / 16 * 16);
-    // 224 rows: a prefill chunk's experts (~192 rows each, rarely above 224) take one tile each,
-    // and five stages of 16 KB of weights + 28 KB of rows fit the ring's 220 KB
-    if (bn > 224) bn = 224;
+    // Tile height: when experts average 128 rows or more (a prefill chunk: ~192 each) a
+    // 256-row tile holds nearly every expert whole, in four 48 KB stages; when they are sparse
+    // (most tiles small, a few hot experts) 224-row tiles give five 44 KB stages and split
+    // only the hot experts.  Measured on B200: prefill FFN 558 us at 256 against 580 at 224;
+    // the skewed batch 303 us at 224 against 318 at 256.
+    const int cap = rows / (E > 0 ? E : 1) >= 128 ? 256 : 224;
+    if (bn > cap) bn = cap;
     if (bn < 16) bn = 16;
     p.bn = bn;
     const int stage = GG_A_BYTES + bn * GG_ROW_BYTES;
