@@ -36,7 +36,7 @@ cudaError_t launch_schedule(const int32_t* offsets, int E, int bn, int4* sched, 
                             int K, cudaStream_t stream);
 cudaError_t launch_gather(const uint16_t* x, const int32_t* perm_src, int64_t rows, int64_t routed_rows, int K,
                           int64_t T, int H, void* xp, bool fp8, float x_scale, int num_sms, const DevCtx& ctx,
-                          cudaStream_t stream, int* zero = nullptr, int n_zero = 0);
+                          cudaStream_t stream, int* zero = nullptr, int64_t n_zero = 0);
 struct GemmPlan {
     int bn;
     int n_stages;
@@ -49,10 +49,22 @@ cudaError_t launch_grouped_gemm(bool fp8, bool up, const void* W, int E, int Nou
                                 void* out, const float* w_scale, float in_scale, float out_scale, int num_sms,
                                 int debug_withhold, const DevCtx& ctx, cudaStream_t stream, const void* Ws,
                                 int n_shared);
+// The weighted combine folded into the one-launch FFN (see grouped_ffn.cu).
+struct FfnCombine {
+    int* cnt;                   // [T][H / 16], zero before the launch
+    const int32_t* perm_src;
+    const int32_t* inv_row;
+    const float* topk_w;
+    const uint16_t* residual;   // or null
+    uint16_t* out;
+    int K;
+    int64_t routed_rows;        // T * K
+};
 cudaError_t launch_grouped_ffn(bool fp8, const void* w_up, const void* w_down, int E, int F, int H, const void* xp,
                                void* hb, void* y, int64_t rows, const int4* sched, const int* n_sched, int* done,
                                const GemmPlan& plan, const float* su, const float* sd, float x_scale, float h_scale,
-                               int num_sms, int debug_hold, const DevCtx& ctx, cudaStream_t stream);
+                               int num_sms, int debug_hold, const DevCtx& ctx, cudaStream_t stream,
+                               const FfnCombine* comb = nullptr);
 cudaError_t launch_grouped_gemm_pair(bool fp8, bool up, const void* W, int E, int Nout, int Kdim, const void* act,
                                      int64_t rows, const int4* sched, const int* n_sched, int bn, int max_sched,
                                      void* out, const float* w_scale, float in_scale, float out_scale,

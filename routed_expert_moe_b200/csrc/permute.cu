@@ -296,11 +296,16 @@ __device__ __forceinline__ float div_by_scale(float x, float s, float y) {
 // warp per row, four 16-byte loads per lane in flight before their stores.
 __global__ void gather_rows_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm_src,
                                    int64_t rows, int64_t routed_rows, int K, int64_t T, int H,
-                                   void* __restrict__ xp, int fp8, float x_scale, int* zero, int n_zero,
+                                   void* __restrict__ xp, int fp8, float x_scale, int* zero, int64_t n_zero,
                                    DevCtx ctx) {
     pdl_enter();
     // counters of the kernel that follows (the one-launch FFN), zero before it starts
-    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n_zero; i += gridDim.x * blockDim.x) zero[i] = 0;
+    // (zero is 16-byte aligned: whole int4s, then the tail)
+    {
+        const int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x, step = (int64_t)gridDim.x * blockDim.x;
+        for (int64_t i = i0; i < n_zero / 4; i += step) reinterpret_cast<int4*>(zero)[i] = make_int4(0, 0, 0, 0);
+        for (int64_t i = (n_zero & ~int64_t(3)) + i0; i < n_zero; i += step) zero[i] = 0;
+    }
     constexpr int B = 4;
     const int lane = threadIdx.x % 32;
     const int64_t warps = (int64_t)gridDim.x * (blockDim.x / 32);
@@ -389,7 +394,7 @@ cudaError_t launch_schedule(const int32_t* offsets, int E, int bn, int4* sched, 
 
 cudaError_t launch_gather(const uint16_t* x, const int32_t* perm_src, int64_t rows, int64_t routed_rows, int K,
                           int64_t T, int H, void* xp, bool fp8, float x_scale, int num_sms, const DevCtx& ctx,
-                          cudaStream_t stream, int* zero, int n_zero) {
+                          cudaStream_t stream, int* zero, int64_t n_zero) {
     if (rows == 0) return cudaSuccess;
     int64_t blocks = (rows + 7) / 8;
     const int64_t cap = (int64_t)num_sms * 8;

@@ -252,12 +252,16 @@ def test_cta_pair_gemm_matches_oracle(moe, fp8):
 # --------------------------------------------------------------------------- one-launch expert FFN
 
 @pytest.mark.parametrize("fp8", [False, True])
-@pytest.mark.parametrize("w", [W.WORKLOADS[1], W.WORKLOADS[3],
-                               W.Workload("ffn_T700_E16_K4", 700, 512, 16, 4, 320, seed=23)],
+@pytest.mark.parametrize("w", [W.WORKLOADS[1], W.WORKLOADS[3], W.WORKLOADS[2],
+                               W.Workload("ffn_T700_E16_K4", 700, 512, 16, 4, 320, seed=23),
+                               W.Workload("ffn_T37_H272_E8_K3_F208", 37, 272, 8, 3, 208, seed=24)],
                          ids=lambda w: w.name if hasattr(w, "name") else str(w))
-def test_one_launch_ffn_equals_two_launches_bitwise(moe, w, fp8):
+@pytest.mark.parametrize("with_residual", [False, True], ids=["no_residual", "residual_aliased_to_out"])
+def test_one_launch_ffn_equals_two_launches_bitwise(moe, w, fp8, with_residual):
     """Both projections in one launch compute exactly the products of the two launches (same
-    tiles, same accumulation order), so the layer output is the same bit for bit."""
+    tiles, same accumulation order), and the combine folded into its down epilogue takes the
+    combine kernel's arithmetic (k order, one rounding): the layer output of the three ways
+    (debug hook 8 = 1, 2, 0) is the same bit for bit, also with the residual in `out`."""
     h = inputs(w)
     d = device_inputs(h)
     dims = moe.dims(w.T, w.H, w.E, w.K, w.F, fp8=fp8)
@@ -274,14 +278,41 @@ def test_one_launch_ffn_equals_two_launches_bitwise(moe, w, fp8):
         sx, sh = oracle.calibrate_fp8(h["x"][:64], h["wr"], h["bias"], h["wu"], w.K)
         scales = moe.fp8_scales(su, sd, float(sx), float(sh))
         wu, wd = cu, cd
+    g = torch.Generator().manual_seed(w.seed + 1000)
+    res = torch.randn(w.T, w.H, generator=g).to(torch.bfloat16).cuda() if with_residual else None
     outs = []
-    for one in (1, 0):
-        moe.debug_set(8, one)
+    for mode in (1, 2, 0):
+        moe.debug_set(8, mode)
         try:
-            out = torch.empty(w.T, w.H, dtype=torch.bfloat16, device="cuda")
-            moe.forward(dims, d["x"], d["wr"], d["bias"], wu, wd, out, ws, scales=scales)
+            out = res.clone() if with_residual else torch.empty(w.T, w.H, dtype=torch.bfloat16, device="cuda")
+            moe.forward(dims, d["x"], d["wr"], d["bias"], wu, wd, out, ws, scales=scales,
+                        residual=out if with_residual else None)
             moe.check_device_error()
             outs.append(out)
         finally:
             moe.debug_set(8, 1)
-    assert torch.equal(outs[0], outs[1])
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[1], outs[2])
+
+
+@pytest.mark.parametrize("fill", [0x00, 0x7F, 0xFF], ids=["zeros", "0x7F", "0xFF"])
+def test_folded_combine_ignores_stale_workspace(moe, fill):
+    """The folded combine's counters live in the workspace and are zeroed by the row gather of
+    every call: a workspace full of stale bytes (or the previous call's counts) gives the same
+    output bit for bit, call after call."""
+    w = W.WORKLOADS[1]
+    h = inputs(w)
+    d = device_inputs(h)
+    dims = moe.dims(w.T, w.H, w.E, w.K, w.F)
+    ws = moe.alloc_workspace(dims)
+    ref = torch.empty(w.T, w.H, dtype=torch.bfloat16, device="cuda")
+    moe.debug_set(8, 2)
+    try:
+        moe.forward(dims, d["x"], d["wr"], d["bias"], d["wu"], d["wd"], ref, ws)
+    finally:
+        moe.debug_set(8, 1)
+    ws.fill_(fill)
+    for _ in range(3):
+        out = torch.full((w.T, w.H), 7.0, dtype=torch.bfloat16, device="cuda")
+        moe.forward(dims, d["x"], d["wr"], d["bias"], d["wu"], d["wd"], out, ws)
+        moe.check_device_error()
+        assert torch.equal(out, ref)
