@@ -199,11 +199,7 @@ moe_status moe_combine(const moe_dims* d, const void* y_perm, const int32_t* inv
  * when given they receive the routing.  out may alias residual.  With
  * d->Fs > 0 the shared expert (w_up_shared [Fs][H], w_down_shared [H][Fs],
  * bf16) runs in the same grouped GEMM launches as the routed experts and its
- * output joins the combine with weight 1; both pointers NULL when Fs = 0.
- * With bf16 or E4M3 experts and no shared expert the combine runs inside the
- * expert FFN's single launch: the down-projection lane that completes a
- * token's K rows for 16 features sums them (the arithmetic of moe_combine,
- * so the output is the same bit for bit). */
+ * output joins the combine with weight 1; both pointers NULL when Fs = 0. */
 moe_status moe_forward(const moe_dims* d, const void* x, const void* w_router, const float* bias,
                        const void* w_up, const void* w_down, const void* w_up_shared,
                        const void* w_down_shared, const moe_fp8_scales* scales,
@@ -323,8 +319,7 @@ moe_status moe_check_device_error(void* stream);
  * events[i] on its stream before stage i and events[n-1] after the last
  * stage (stages: 0 router logits, 1 router top-K, 2 permute, 3 row gather,
  * 4 up GEMM, 5 down GEMM, 6 combine; when both projections run in one
- * launch, stage 4 holds that launch and stage 5 is empty, and when the
- * combine runs inside it, stage 6 is empty too), so a caller can
+ * launch, stage 4 holds that launch and stage 5 is empty), so a caller can
  * time each kernel in place.  n == 0 turns it off.  Host state shared by all threads. */
 #define MOE_STAGE_EVENTS 8
 moe_status moe_set_stage_events(void* const* events, int32_t n);
@@ -351,10 +346,8 @@ moe_status moe_set_stage_events(void* const* events, int32_t n);
  * column j*F) instead of the chunked 3-D view, 0 (the default) restores the
  * view; what = 8: value 1 (the default) runs both expert projections of bf16
  * and E4M3 layers without a shared expert in one launch (the down units of a
- * schedule entry start once that entry's up units have reported) with
- * moe_forward's combine folded into it, 2 the same launch with the combine
- * as a launch of its own, 0 the projections as two launches (other values
- * MOE_EINVAL).  Other `what`: MOE_EINVAL. */
+ * schedule entry start once that entry's up units have reported), 0 as two
+ * launches.  Other `what`: MOE_EINVAL. */
 moe_status moe_debug_set(int32_t what, int64_t value);
 
 #ifdef __cplusplus

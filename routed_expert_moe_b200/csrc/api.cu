@@ -21,9 +21,7 @@ constexpr uint64_t kDefaultTimeoutNs = 4000000000ull;
 std::atomic<uint64_t> g_timeout_ns{kDefaultTimeoutNs};
 std::atomic<int> g_debug_withhold{0};
 std::atomic<int> g_gemm_pair{0};
-// bf16/E4M3 expert FFN: 0 two launches; 1 one launch (grouped_ffn.cu) with the layer's combine
-// folded into its down epilogue; 2 one launch, combine as its own launch
-std::atomic<int> g_fused_ffn{1};
+std::atomic<int> g_fused_ffn{1};   // 1: both bf16/E4M3 projections in one launch (grouped_ffn.cu)
 std::atomic<int> g_pdl{1};
 std::atomic<int> g_shared_2d{0};   // 1: the shared down weight through its 2-D fallback map
 void* g_stage_events[MOE_STAGE_EVENTS] = {};
@@ -129,8 +127,6 @@ struct FfnWs {
     uint8_t* xp_block;   // NVFP4: block scales [rows][KSP(H)]
     uint8_t* hb_block;   // NVFP4: block scales [rows][KSP(F)]
     int* done;           // [max_sched] up units reported per schedule entry (one-launch FFN)
-    int* cnt;            // [T][H/16] down parts per (token, 16 features), right after done (moe_forward)
-    int64_t cnt_ints;
 };
 struct ForwardWs {
     int32_t* idx;
@@ -151,12 +147,6 @@ struct ForwardWs {
 bool fused_ffn(const moe_dims* d) {
     return g_fused_ffn.load() && n_shared(d) == 0 &&
            (d->expert_dtype == MOE_BF16 || d->expert_dtype == MOE_FP8_E4M3);
-}
-
-// Counters of the combine folded into the one-launch FFN (moe_forward only).
-int64_t combine_counter_ints(const moe_dims* d) {
-    const bool can = n_shared(d) == 0 && (d->expert_dtype == MOE_BF16 || d->expert_dtype == MOE_FP8_E4M3);
-    return can ? d->T * (int64_t)(d->H / 16) : 0;
 }
 
 GemmPlan ffn_plan(const moe_dims* d) {
@@ -182,15 +172,13 @@ RouteWs carve_route(Carve& c, void* base, const moe_dims* d, const RouterPlan& r
     return r;
 }
 
-FfnWs carve_ffn(Carve& c, void* base, const moe_dims* d, const GemmPlan& gp, int64_t cnt_ints = 0) {
+FfnWs carve_ffn(Carve& c, void* base, const moe_dims* d, const GemmPlan& gp) {
     FfnWs f;
     const size_t rows = (size_t)ffn_rows(d);
     f.sched = c.take<int4>(base, (size_t)gp.max_sched);
     f.n_sched = c.take<int>(base, 1);
     f.perm_scratch = c.take<int>(base, permute_scratch_ints(d->T * d->K, d->E));
-    f.done = c.take<int>(base, (size_t)gp.max_sched + (size_t)cnt_ints);   // the gather zeroes both
-    f.cnt = base ? f.done + gp.max_sched : nullptr;
-    f.cnt_ints = cnt_ints;
+    f.done = c.take<int>(base, (size_t)gp.max_sched);
     f.xp_block = f.hb_block = nullptr;
     if (d->expert_dtype == MOE_NVFP4) {
         f.xp = c.take<uint8_t>(base, rows * d->H / 2);
@@ -224,9 +212,9 @@ size_t route_ws_bytes(const moe_dims* d, int sms) {
     return c.off;
 }
 
-size_t ffn_ws_bytes(const moe_dims* d, int64_t cnt_ints = 0) {
+size_t ffn_ws_bytes(const moe_dims* d) {
     Carve c;
-    carve_ffn(c, nullptr, d, ffn_plan(d), cnt_ints);
+    carve_ffn(c, nullptr, d, ffn_plan(d));
     return c.off;
 }
 
@@ -235,26 +223,15 @@ size_t forward_ws_bytes(const moe_dims* d, int sms) {
     carve_forward(c, nullptr, d);
     const size_t a = c.off;
     // route and ffn scratch are carved after the forward buffers, reusing one region
-    const size_t r = route_ws_bytes(d, sms), f = ffn_ws_bytes(d, combine_counter_ints(d));
+    const size_t r = route_ws_bytes(d, sms), f = ffn_ws_bytes(d);
     return ((a + 255) & ~size_t(255)) + (r > f ? r : f) + 256;
 }
 
-// Whether run_ffn takes the one-launch FFN (bf16 or E4M3 experts, no shared expert, the
-// CTA-pair variant off).
-bool one_launch_ffn(const moe_dims* d, int bn) {
-    const bool pair = g_gemm_pair.load() && bn > 64 && !g_debug_withhold.load() && n_shared(d) == 0;
-    return fused_ffn(d) && !pair;
-}
-
-// Whether moe_forward folds its combine into the one-launch FFN.
-bool combine_in_ffn(const moe_dims* d, int bn) { return g_fused_ffn.load() == 1 && one_launch_ffn(d, bn); }
-
-// Run the expert FFN given a schedule already in `fw`.  comb (one-launch FFN only): fold the
-// layer's combine into the down epilogue; its counters are fw.cnt.
+// Run the expert FFN given a schedule already in `fw`.
 moe_status run_ffn(const moe_dims* d, const DeviceInfo* dev, const DevCtx& ctx, const GemmPlan& gp,
                    const void* x, const int32_t* perm_src, const void* w_up, const void* w_down,
                    const void* w_up_s, const void* w_down_s, const moe_fp8_scales* sc, FfnWs& fw, void* y_perm,
-                   cudaStream_t st, bool marks = false, const FfnCombine* comb = nullptr) {
+                   cudaStream_t st, bool marks = false) {
     const bool fp8 = d->expert_dtype == MOE_FP8_E4M3 || d->expert_dtype == MOE_FP8_B128;
     const int64_t rows = ffn_rows(d);
     const int ns = n_shared(d);
@@ -299,20 +276,18 @@ moe_status run_ffn(const moe_dims* d, const DeviceInfo* dev, const DevCtx& ctx, 
     const int withhold = g_debug_withhold.load();
     // optional: tiles of more than 64 tokens on CTA pairs (one activation read per 256 weight rows)
     const bool pair = g_gemm_pair.load() && gp.bn > 64 && !withhold && ns == 0;
-    const bool fused = one_launch_ffn(d, gp.bn);
-    if (comb && (!fused || comb->cnt != fw.cnt || fw.cnt_ints != d->T * (int64_t)(d->H / 16))) return MOE_EINVAL;
+    const bool fused = fused_ffn(d) && !pair;
     // permuted copy of x (or of its E4M3 codes), read by the up projection in contiguous row blocks;
-    // it also zeroes the one-launch FFN's per-entry counters (and the combine's, carved right after)
+    // it also zeroes the one-launch FFN's per-entry counters
     cudaError_t e = launch_gather(static_cast<const uint16_t*>(x), perm_src, rows, d->T * d->K, d->K, d->T, d->H,
                                   fw.xp, fp8, fp8 ? sc->x_scale : 1.0f, dev->num_sms, ctx, st,
-                                  fused ? fw.done : nullptr, fused ? gp.max_sched + (comb ? fw.cnt_ints : 0) : 0);
+                                  fused ? fw.done : nullptr, fused ? gp.max_sched : 0);
     if (e != cudaSuccess) return cuda_status(e);
     if (fused) {
         if (marks) stage_mark(4, st);
         e = launch_grouped_ffn(fp8, w_up, w_down, d->E, d->F, d->H, fw.xp, fw.hb, y_perm, rows, fw.sched, fw.n_sched,
                                fw.done, gp, fp8 ? sc->w_up_scale : nullptr, fp8 ? sc->w_down_scale : nullptr,
-                               fp8 ? sc->x_scale : 1.0f, fp8 ? sc->h_scale : 1.0f, dev->num_sms, withhold, ctx, st,
-                               comb);
+                               fp8 ? sc->x_scale : 1.0f, fp8 ? sc->h_scale : 1.0f, dev->num_sms, withhold, ctx, st);
         if (marks) stage_mark(5, st);
         return cuda_status(e);
     }
@@ -411,9 +386,8 @@ moe_status moe_forward_launches(const moe_dims* d, int32_t* launches) {
     }
     int n = route_launches(d->T, d->H, d->E);
     n += permute_scratch_ints(d->T * d->K, d->E) == 0 ? 1 : 3;   // one block, or histogram + scan + scatter
-    // row gather, up and down projections (one launch or two), combine (folded into the one-launch FFN)
-    const int bn = ffn_plan(d).bn;
-    n += 1 + (one_launch_ffn(d, bn) ? 1 : 2) + (combine_in_ffn(d, bn) ? 0 : 1);
+    // row gather, up and down projections (one launch or two), combine
+    n += 1 + (fused_ffn(d) && !(g_gemm_pair.load() && gemm_plan(d->T, d->K, d->E).bn > 64) ? 1 : 2) + 1;
     *launches = n;
     return MOE_OK;
 }
@@ -528,22 +502,18 @@ moe_status moe_forward(const moe_dims* d, const void* x, const void* w_router, c
 
     const GemmPlan gp = ffn_plan(d);
     Carve cf;
-    FfnWs ffw = carve_ffn(cf, sbase, d, gp, combine_counter_ints(d));   // reuses the router scratch region
+    FfnWs ffw = carve_ffn(cf, sbase, d, gp);   // reuses the router scratch region
     stage_mark(2, st);
     e = launch_permute(idx, d->T * d->K, d->K, d->E, fw.counts, fw.offsets, fw.perm_src, fw.inv_row, ffw.sched,
                        ffw.n_sched, gp.bn, n_shared(d), ffw.perm_scratch, ctx, st);
     if (e != cudaSuccess) return cuda_status(e);
-    const bool folded = combine_in_ffn(d, gp.bn);
-    FfnCombine comb{ffw.cnt, fw.perm_src, fw.inv_row, w, static_cast<const uint16_t*>(residual),
-                    static_cast<uint16_t*>(out), d->K, d->T * d->K};
     s = run_ffn(d, dev, ctx, gp, x, fw.perm_src, w_up, w_down, w_up_shared, w_down_shared, scales, ffw, fw.y_perm,
-                st, true, folded ? &comb : nullptr);
+                st, true);
     if (s != MOE_OK) return s;
     stage_mark(6, st);
-    if (!folded)
-        e = launch_combine(static_cast<const uint16_t*>(fw.y_perm), fw.inv_row, w,
-                           static_cast<const uint16_t*>(residual), static_cast<uint16_t*>(out), d->T, d->K,
-                           n_shared(d), d->H, dev->num_sms, ctx, st);
+    e = launch_combine(static_cast<const uint16_t*>(fw.y_perm), fw.inv_row, w,
+                       static_cast<const uint16_t*>(residual), static_cast<uint16_t*>(out), d->T, d->K,
+                       n_shared(d), d->H, dev->num_sms, ctx, st);
     stage_mark(7, st);
     return cuda_status(e);
 }
@@ -701,8 +671,7 @@ moe_status moe_debug_set(int32_t what, int64_t value) {
         return MOE_OK;
     }
     if (what == 8) {
-        if (value < 0 || value > 2) return MOE_EINVAL;
-        g_fused_ffn.store((int)value);
+        g_fused_ffn.store(value ? 1 : 0);
         return MOE_OK;
     }
     if (what == 5) {

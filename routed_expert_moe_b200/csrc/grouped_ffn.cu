@@ -18,12 +18,6 @@
 //   down producer spins (bounded) on an acquire load of done[s] until it
 //                 reaches 4 * m_up, fences the async proxy, then issues the
 //                 TMA loads of H.
-// With the combine folded in (moe_forward), each down epilogue lane, once it has
-// stored 16 features of each of its tile's token rows, issues one release fence
-// and adds 1 to each (token, features) counter; the lane that brings one to K
-// issues an acquire fence, sums the token's K rows in the fixed k order (+ the
-// residual) and stores the output: the combine kernel's arithmetic, so the
-// output is the same bit for bit.
 // Deadlock freedom: every CTA walks all of its up units before any of its down
 // units, so the up units a down unit waits for are all issued by CTAs that
 // never wait on anything but their own pipeline.  done[] is zeroed by the row
@@ -47,7 +41,6 @@ constexpr int FF_ROW_BYTES = 128;
 constexpr int FF_A_BYTES = FF_BM * FF_ROW_BYTES;
 constexpr int FF_TMEM_COLS = 512;
 constexpr int FF_EPI_WARPS = 4;
-constexpr int FF_MAX_CHUNKS = FF_TMEM_COLS / 2 / 16;   // 16-token chunks of the widest tile (256)
 
 struct FfnArgs {
     const int4* sched;      // {e, row0, nrows, 0}
@@ -64,15 +57,6 @@ struct FfnArgs {
     const float* sd;
     float x_scale, h_scale;
     int debug_hold;         // 1: block 0's first up unit never reports its rows (a wait must expire)
-    // the weighted combine, done by the last down unit of each (token, 16-feature group):
-    int* cnt;                   // [T][H / 16] down arrivals (zero at launch); null: no combine
-    const int32_t* perm_src;    // [T * K] assignment t * K + k of each grouped row
-    const int32_t* inv_row;     // [T * K] grouped row of each assignment
-    const float* topk_w;        // [T * K]
-    const uint16_t* residual;   // [T][H] bf16 or null
-    uint16_t* out;              // [T][H] bf16 (may alias residual)
-    int K;
-    int64_t routed_rows;        // T * K
 };
 
 struct FfnMaps {
@@ -94,52 +78,6 @@ __device__ __forceinline__ void red_release_add(int* p, int v) {
 
 __device__ __forceinline__ void fence_proxy_async_global() {
     asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-
-__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
-
-// out[t][f0 .. f0 + 15] = (residual +) sum_k w[t][k] * Y[inv_row[t * K + k]][f0 ..], k ascending,
-// in fp32 with one rounding to bf16: the arithmetic of the combine kernel.  Called by the
-// lane whose count completed the group, after its acquire fence (the others' rows are visible).
-__device__ __forceinline__ void combine_group(const FfnArgs& g, const DevCtx& ctx, int64_t t, int f0) {
-    float acc[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) acc[i] = 0.0f;
-    for (int k = 0; k < g.K; ++k) {
-        const int32_t rk = g.inv_row[t * g.K + k];
-        const float wk = g.topk_w[t * g.K + k];
-        if (rk < 0 || rk >= g.routed_rows) {
-            record_error(ctx.err, MOE_EINDEX);
-            continue;
-        }
-        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(g.y) + (int64_t)rk * g.H + f0);
-        const uint4 a0 = __ldcg(src), a1 = __ldcg(src + 1);
-        const uint32_t wv[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            acc[2 * i] = __fmaf_rn(wk, __uint_as_float(wv[i] << 16), acc[2 * i]);
-            acc[2 * i + 1] = __fmaf_rn(wk, __uint_as_float(wv[i] & 0xFFFF0000u), acc[2 * i + 1]);
-        }
-    }
-    if (g.residual) {
-        const uint4* rs = reinterpret_cast<const uint4*>(g.residual + t * g.H + f0);
-        const uint4 r0 = __ldcg(rs), r1 = __ldcg(rs + 1);
-        const uint32_t rv[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            acc[2 * i] = __fadd_rn(__uint_as_float(rv[i] << 16), acc[2 * i]);
-            acc[2 * i + 1] = __fadd_rn(__uint_as_float(rv[i] & 0xFFFF0000u), acc[2 * i + 1]);
-        }
-    }
-    uint32_t o[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const __nv_bfloat162 p2 = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
-        o[i] = *reinterpret_cast<const uint32_t*>(&p2);
-    }
-    uint4* dst = reinterpret_cast<uint4*>(g.out + t * g.H + f0);
-    dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
-    dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
 // Bounded wait until *p >= target (acquire).  Gives up on the time limit or the block's abort flag.
@@ -399,33 +337,6 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
             }
             tc_fence_before();
             mbar_arrive(smem_u32(&tempty[acc]));
-            if (!up && g.cnt && f16 < Nout) {
-                // count this lane's (token, 16 features) parts in, after one release fence for all
-                // its stores; the lane whose count completes a token's K parts combines them,
-                // after an acquire fence
-                fence_acq_rel_gpu();
-                uint32_t last = 0;
-#pragma unroll
-                for (int c = 0; c < FF_MAX_CHUNKS; ++c) {
-                    const int r = c * 16 + tj;
-                    if (c < nchunks && r < sc.z) {
-                        const int32_t a = g.perm_src[sc.y + r];
-                        if (a < 0 || a >= g.routed_rows) {
-                            record_error(ctx.err, MOE_EINDEX);
-                        } else if (atomicAdd(g.cnt + (int64_t)(a / g.K) * (g.H / 16) + f16 / 16, 1) == g.K - 1) {
-                            last |= 1u << c;
-                        }
-                    }
-                }
-                if (last) {
-                    fence_acq_rel_gpu();
-                    while (last) {
-                        const int c = __ffs(last) - 1;
-                        last &= last - 1;
-                        combine_group(g, ctx, g.perm_src[sc.y + c * 16 + tj] / g.K, f16);
-                    }
-                }
-            }
             if (up) {
                 // this warp's rows of H are complete: every lane orders its stores for the async
                 // proxy (the TMA loads of H), the warp barrier orders them before lane 0's release
@@ -483,15 +394,11 @@ bool map_ffn(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, bool 
 
 // Both projections of the grouped FFN in one launch.  xp [rows][H] and hb [rows][F]
 // (bf16, or E4M3 codes), y [rows][H] bf16; done: max_sched ints, zero before the launch.
-// comb (optional): also the weighted combine into comb->out, each (token, 16 features) by the
-// last of its K down parts; comb->cnt ([T][H/16] ints) zero before the launch.
 cudaError_t launch_grouped_ffn(bool fp8, const void* w_up, const void* w_down, int E, int F, int H, const void* xp,
                                void* hb, void* y, int64_t rows, const int4* sched, const int* n_sched, int* done,
                                const GemmPlan& plan, const float* su, const float* sd, float x_scale, float h_scale,
-                               int num_sms, int debug_hold, const DevCtx& ctx, cudaStream_t stream,
-                               const FfnCombine* comb) {
+                               int num_sms, int debug_hold, const DevCtx& ctx, cudaStream_t stream) {
     if (rows == 0) return cudaSuccess;
-    if (plan.bn > FF_MAX_CHUNKS * 16 || (comb && (comb->K < 1 || H % 16 != 0))) return cudaErrorInvalidValue;
     FfnMaps maps;
     if (!map_ffn(&maps.ua128, w_up, (int64_t)E * F, H, fp8, 128) || !map_ffn(&maps.ua64, w_up, (int64_t)E * F, H, fp8, 64) ||
         !map_ffn(&maps.ub128, xp, rows, H, fp8, 128) || !map_ffn(&maps.ub64, xp, rows, H, fp8, 64) ||
@@ -519,14 +426,6 @@ cudaError_t launch_grouped_ffn(bool fp8, const void* w_up, const void* w_down, i
     g.x_scale = x_scale;
     g.h_scale = h_scale;
     g.debug_hold = debug_hold;
-    g.cnt = comb ? comb->cnt : nullptr;
-    g.perm_src = comb ? comb->perm_src : nullptr;
-    g.inv_row = comb ? comb->inv_row : nullptr;
-    g.topk_w = comb ? comb->topk_w : nullptr;
-    g.residual = comb ? comb->residual : nullptr;
-    g.out = comb ? comb->out : nullptr;
-    g.K = comb ? comb->K : 1;
-    g.routed_rows = comb ? comb->routed_rows : rows;
     const int64_t max_units = (int64_t)plan.max_sched * (g.m_up + g.m_down);
     const int grid = (int)(max_units < num_sms ? max_units : num_sms);
     auto kfn = fp8 ? grouped_ffn_kernel<true> : grouped_ffn_kernel<false>;

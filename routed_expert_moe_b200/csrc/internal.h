@@ -49,22 +49,10 @@ cudaError_t launch_grouped_gemm(bool fp8, bool up, const void* W, int E, int Nou
                                 void* out, const float* w_scale, float in_scale, float out_scale, int num_sms,
                                 int debug_withhold, const DevCtx& ctx, cudaStream_t stream, const void* Ws,
                                 int n_shared);
-// The weighted combine folded into the one-launch FFN (see grouped_ffn.cu).
-struct FfnCombine {
-    int* cnt;                   // [T][H / 16], zero before the launch
-    const int32_t* perm_src;
-    const int32_t* inv_row;
-    const float* topk_w;
-    const uint16_t* residual;   // or null
-    uint16_t* out;
-    int K;
-    int64_t routed_rows;        // T * K
-};
 cudaError_t launch_grouped_ffn(bool fp8, const void* w_up, const void* w_down, int E, int F, int H, const void* xp,
                                void* hb, void* y, int64_t rows, const int4* sched, const int* n_sched, int* done,
                                const GemmPlan& plan, const float* su, const float* sd, float x_scale, float h_scale,
-                               int num_sms, int debug_hold, const DevCtx& ctx, cudaStream_t stream,
-                               const FfnCombine* comb = nullptr);
+                               int num_sms, int debug_hold, const DevCtx& ctx, cudaStream_t stream);
 cudaError_t launch_grouped_gemm_pair(bool fp8, bool up, const void* W, int E, int Nout, int Kdim, const void* act,
                                      int64_t rows, const int4* sched, const int* n_sched, int bn, int max_sched,
                                      void* out, const float* w_scale, float in_scale, float out_scale,

@@ -143,9 +143,7 @@ def test_shared_expert_dims_and_pointers_are_checked_on_the_host(moe):
     assert ws(bad(moe, Fs=11 * 1856)) == moe.MOE_EINVAL            # K + Fs/F > 16
     fp8 = moe.dims(64, 2688, 128, 6, 1856, fp8=True, Fs=1856)
     assert ws(fp8) == moe.MOE_EUNSUPPORTED                           # bf16 experts only
-    # the plain layer's workspace less the counters of its folded combine (one int per token and
-    # 16 features), which a layer with a shared expert does not use
-    plain = moe.workspace_size(bad(moe)) - 64 * (2688 // 16) * 4
+    plain = moe.workspace_size(bad(moe))
     shared = moe.workspace_size(bad(moe, Fs=2 * 1856))
     assert shared >= plain + 2 * 64 * (2688 * 2 * 2 + 1856 * 2)     # X, H and Y rows of two chunks
     fake = ctypes.c_void_p(4096)
@@ -164,29 +162,26 @@ def test_forward_launch_count_follows_the_dispatch(moe):
     """Router: one launch up to 256 tokens (expert-split clusters) and from 3072 (hidden-split
     clusters), two in between; permutation: one block up to 4096 assignments, else three kernels;
     then the row gather, the expert FFN (one launch for bf16 and E4M3 experts without a shared
-    expert, with the combine folded in; else the two projections) and the combine."""
+    expert, else the two projections) and the combine."""
     count = lambda T, **kw: moe.forward_launches(moe.dims(T, 2688, 128, 6, 1856, **kw))
-    assert [count(T) for T in (0, 1, 64, 256, 257, 682, 683, 3071, 3072, 4096)] == [0, 4, 4, 4, 5, 5, 7, 7, 6, 6]
-    assert count(64, fp8=True) == 4
+    assert [count(T) for T in (0, 1, 64, 256, 257, 682, 683, 3071, 3072, 4096)] == [0, 5, 5, 5, 6, 6, 8, 8, 7, 7]
+    assert count(64, fp8=True) == 5
     assert count(64, nvfp4=True) == count(64, fp8_b128=True) == count(64, Fs=1856) == 6
     try:
         moe.debug_set(8, 0)             # the two projections as two launches
         assert count(64) == 6 and count(4096) == 8
-        moe.debug_set(8, 2)             # one FFN launch, the combine a launch of its own
-        assert count(64) == 5 and count(4096) == 7
-        assert moe.raw_library().moe_debug_set(8, 3) == moe.MOE_EINVAL
         moe.debug_set(8, 1)
         moe.debug_set(4, 0)             # never the expert-split clusters
-        assert count(64) == 5
+        assert count(64) == 6
         moe.debug_set(5, 2)             # always the hidden-split clusters
-        assert count(64) == 4 and count(576) == 4
+        assert count(64) == 5 and count(576) == 5
         moe.debug_set(5, 1)             # always the two kernels
-        assert count(4096) == 7
+        assert count(4096) == 8
     finally:
         moe.debug_set(8, 1)
         moe.debug_set(4, -1)
         moe.debug_set(5, 0)
-    assert count(64) == 4
+    assert count(64) == 5
 
 
 def test_package_has_no_cpu_path():
