@@ -1109,7 +1109,6 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(NTH, 1)
 // from 3072 tokens (101 us at 4096 against 154).
 constexpr int64_t kRouterSmallMaxDefault = 256;
 constexpr int64_t kRouterSplitMin = 3072;
-constexpr int64_t kRouterSmallTb4Max = 128;
 constexpr size_t kRouterSmallSmemMax = 200 * 1024;
 
 static int router_tt(int64_t T) { return T > 256 ? 64 : 16; }
@@ -1198,6 +1197,40 @@ static cudaError_t launch_router_fused(const RouterFusedArgs& ra, const DevCtx& 
     return launch_k(kfn, dim3(tiles * CS), dim3(NTH), L::bytes, stream, ra, ctx);
 }
 
+// Clusters of the expert-split router that fit on the current device at once (its clusters
+// of 8 CTAs of one SM each must fit inside GPCs: 15 on a 148-SM B200), queried once per device.
+static int router_small_max_clusters(int TB, int H, int E) {
+    static std::atomic<int> cache[2][64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 1;
+    const int slot = TB == 4 ? 0 : 1;
+    int n = cache[slot][dev].load();
+    if (n > 0) return n;
+    const size_t smem = rs_smem_bytes(TB, H, E);
+    auto kfn = TB == 4 ? router_small_kernel<4> : router_small_kernel<8>;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(RS_CLUSTER);
+    cfg.blockDim = dim3(RS_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess ||
+        cudaOccupancyMaxActiveClusters(&n, kfn, &cfg) != cudaSuccess || n < 1) {
+        (void)cudaGetLastError();
+        n = 1;
+    }
+    cache[slot][dev].store(n);
+    return n;
+}
+
+// Tokens per cluster of the expert-split router (0: the batch does not take it): 4 when the
+// batch's clusters of 4 tokens fit on the device at once, else 8 (a second wave of clusters
+// would double the time: at 64 tokens, 16 clusters of 4 against 15 that fit).
+static int router_small_tb(int64_t T, int H, int E, bool query) {
+    if (T > g_router_small_max.load() || rs_smem_bytes(4, H, E) > kRouterSmallSmemMax) return 0;
+    if (rs_smem_bytes(8, H, E) > kRouterSmallSmemMax) return 4;
+    if (!query) return 8;
+    return (T + 3) / 4 <= router_small_max_clusters(4, H, E) ? 4 : 8;
+}
+
 template <int TB>
 static cudaError_t launch_router_small(const RouterSmallArgs& ra, const DevCtx& ctx, cudaStream_t stream) {
     const size_t smem = rs_smem_bytes(TB, ra.H, ra.E);
@@ -1212,10 +1245,7 @@ static cudaError_t launch_router_small(const RouterSmallArgs& ra, const DevCtx& 
 // the same tests, in the same order, as launch_route below.
 int route_launches(int64_t T, int H, int E) {
     if (T == 0) return 0;
-    if (T <= g_router_small_max.load()) {
-        const int tb = T <= kRouterSmallTb4Max ? 4 : 8;
-        if (rs_smem_bytes(tb, H, E) <= kRouterSmallSmemMax) return 1;   // expert-split clusters
-    }
+    if (router_small_tb(T, H, E, false) > 0) return 1;   // expert-split clusters
     const int split_mode = g_router_split.load();
     if (E <= RF_E && split_mode != 1 && (split_mode == 2 || T >= kRouterSplitMin)) return 1;   // hidden-split
     return 2;   // logits, then top-K
@@ -1226,15 +1256,13 @@ cudaError_t launch_route(const uint16_t* x, const uint16_t* wr, const float* bia
                          const RouterPlan& plan, const DevCtx& ctx, cudaStream_t stream,
                          void (*between)(cudaStream_t)) {
     if (T == 0) return cudaSuccess;
-    if (T <= g_router_small_max.load()) {
-        const int tb = T <= kRouterSmallTb4Max ? 4 : 8;
-        if (rs_smem_bytes(tb, H, E) <= kRouterSmallSmemMax) {
-            RouterSmallArgs ra{x, wr, bias, T, H, E, K, idx, w};
-            const cudaError_t err = tb == 4 ? launch_router_small<4>(ra, ctx, stream)
-                                            : launch_router_small<8>(ra, ctx, stream);
-            if (err == cudaSuccess && between) between(stream);   // one launch: nothing between
-            return err;
-        }
+    const int tb = router_small_tb(T, H, E, true);
+    if (tb > 0) {
+        RouterSmallArgs ra{x, wr, bias, T, H, E, K, idx, w};
+        const cudaError_t err = tb == 4 ? launch_router_small<4>(ra, ctx, stream)
+                                        : launch_router_small<8>(ra, ctx, stream);
+        if (err == cudaSuccess && between) between(stream);   // one launch: nothing between
+        return err;
     }
     const int split_mode = g_router_split.load();
     if (E <= RF_E && split_mode != 1 && (split_mode == 2 || T >= kRouterSplitMin)) {
