@@ -328,7 +328,7 @@ moe_status moe_set_stage_events(void* const* events, int32_t n);
  * what = 1: limit of every bounded wait in nanoseconds (value <= 0 restores
  * the default of 4 s); what = 2: the grouped-GEMM producer of block 0
  * withholds its first load (value 1) so the consumer's wait must expire --
- * in the one-launch FFN, block 0's first up unit withholds its report so
+ * in the one-launch FFN, the list's first up unit withholds its report so
  * that the down units of its entry wait in vain; 0 turns it off; what = 3: value 1 runs the grouped GEMMs of batches with
  * tiles of more than 64 tokens on CTA pairs (cta_group::2, M = 256), value 0
  * (the default) on single CTAs; what = 4: largest batch (tokens) that the

@@ -126,7 +126,7 @@ struct FfnWs {
     void* hb;            // ReLU^2 rows: bf16, E4M3 codes, or NVFP4 codes [rows][F/2]
     uint8_t* xp_block;   // NVFP4: block scales [rows][KSP(H)]
     uint8_t* hb_block;   // NVFP4: block scales [rows][KSP(F)]
-    int* done;           // [max_sched] up units reported per schedule entry (one-launch FFN)
+    int* done;           // [max_sched] up units reported per schedule entry (one-launch FFN), then its claim counter
 };
 struct ForwardWs {
     int32_t* idx;
@@ -178,7 +178,7 @@ FfnWs carve_ffn(Carve& c, void* base, const moe_dims* d, const GemmPlan& gp) {
     f.sched = c.take<int4>(base, (size_t)gp.max_sched);
     f.n_sched = c.take<int>(base, 1);
     f.perm_scratch = c.take<int>(base, permute_scratch_ints(d->T * d->K, d->E));
-    f.done = c.take<int>(base, (size_t)gp.max_sched);
+    f.done = c.take<int>(base, (size_t)gp.max_sched + 1);   // + the FFN's unit claim counter
     f.xp_block = f.hb_block = nullptr;
     if (d->expert_dtype == MOE_NVFP4) {
         f.xp = c.take<uint8_t>(base, rows * d->H / 2);
@@ -281,7 +281,7 @@ moe_status run_ffn(const moe_dims* d, const DeviceInfo* dev, const DevCtx& ctx, 
     // it also zeroes the one-launch FFN's per-entry counters
     cudaError_t e = launch_gather(static_cast<const uint16_t*>(x), perm_src, rows, d->T * d->K, d->K, d->T, d->H,
                                   fw.xp, fp8, fp8 ? sc->x_scale : 1.0f, dev->num_sms, ctx, st,
-                                  fused ? fw.done : nullptr, fused ? gp.max_sched : 0);
+                                  fused ? fw.done : nullptr, fused ? gp.max_sched + 1 : 0);
     if (e != cudaSuccess) return cuda_status(e);
     if (fused) {
         if (marks) stage_mark(4, st);

@@ -1,6 +1,6 @@
 // Both expert projections in one persistent launch (bf16 or E4M3 experts, no
 // shared expert): the up projection's units, then the down projection's, in
-// one list that every CTA walks round-robin.
+// one list from which the CTAs claim units in order.
 //
 // The products are those of grouped_gemm.cu (bloomery issue page, s.2
 // "Checkpoint facts" and s.3: ungated ReLU^2 experts with up/down parts):
@@ -18,10 +18,20 @@
 //   down producer spins (bounded) on an acquire load of done[s] until it
 //                 reaches 4 * m_up, fences the async proxy, then issues the
 //                 TMA loads of H.
-// Deadlock freedom: every CTA walks all of its up units before any of its down
-// units, so the up units a down unit waits for are all issued by CTAs that
-// never wait on anything but their own pipeline.  done[] is zeroed by the row
-// gather that precedes this kernel on the stream.
+// Claiming: each CTA's producer takes the next unit of the list from a global
+// counter (one relaxed atomic add per unit, issued while the previous unit
+// loads) and passes it to the MMA thread and the epilogue warps through a
+// small queue in shared memory (FF_UQ slots, each with a full and an empty
+// mbarrier).  A CTA that runs ahead simply claims more units, so the CTAs end
+// within about one unit of each other (a fixed round-robin left the last CTA
+// 16 us behind the median at decode).
+// Deadlock freedom: units are claimed in list order, so every up unit is
+// claimed, by a running CTA, before any down unit is, and a CTA processes its
+// units in claim order; the up units a down unit waits for therefore belong to
+// running CTAs that finish them without waiting on anything but their own
+// pipeline (no CTA needs to be resident for another to progress).  done[] and
+// the claim counter are zeroed by the row gather that precedes this kernel on
+// the stream.
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -41,8 +51,10 @@ constexpr int FF_ROW_BYTES = 128;
 constexpr int FF_A_BYTES = FF_BM * FF_ROW_BYTES;
 constexpr int FF_TMEM_COLS = 512;
 constexpr int FF_EPI_WARPS = 4;
+constexpr int FF_UQ = 4;   // unit queue slots (producer -> MMA and epilogue warps)
 
 struct FfnArgs {
+    int* claim;             // unit counter (zero at launch; right after done[]): producers claim units
     const int4* sched;      // {e, row0, nrows, 0}
     const int* n_sched;
     int* done;              // [max_sched] up epilogue warps finished per entry (zero at launch)
@@ -56,7 +68,7 @@ struct FfnArgs {
     const float* su;        // [E] E4M3 weight scales (null for bf16)
     const float* sd;
     float x_scale, h_scale;
-    int debug_hold;         // 1: block 0's first up unit never reports its rows (a wait must expire)
+    int debug_hold;         // 1: the list's first up unit never reports its rows (a wait must expire)
 };
 
 struct FfnMaps {
@@ -117,6 +129,10 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
     // the epilogue warps' turn-around tiles: 16 x 32 16-bit values each, 16-byte aligned
     uint16_t* tbuf = reinterpret_cast<uint16_t*>((reinterpret_cast<uintptr_t>(tmem_holder + 1) + 15) &
                                                  ~static_cast<uintptr_t>(15));
+    // the unit queue: the units this block claimed, in claim order
+    uint64_t* uq_full = reinterpret_cast<uint64_t*>(tbuf + FF_EPI_WARPS * 16 * 32);
+    uint64_t* uq_empty = uq_full + FF_UQ;
+    volatile int* uq = reinterpret_cast<volatile int*>(uq_empty + FF_UQ);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     if (threadIdx.x == 0) {
@@ -129,6 +145,10 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
             mbar_init(smem_u32(&tempty[a]), 128);
         }
         mbar_init(smem_u32(drain), 1);
+        for (int q = 0; q < FF_UQ; ++q) {
+            mbar_init(smem_u32(&uq_full[q]), 1);
+            mbar_init(smem_u32(&uq_empty[q]), 1 + FF_EPI_WARPS);
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -151,7 +171,24 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
-            for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+            int qs = 0;
+            uint32_t qph = 0;
+            int claim = atomicAdd(g.claim, 1);
+            while (ok) {
+                // publish the claimed unit (or the end) to the MMA and epilogue warps
+                const int u = claim < n_units ? claim : -1;
+                if (!mbar_wait(smem_u32(&uq_empty[qs]), qph ^ 1u, ctx, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                uq[qs] = u;
+                mbar_arrive(smem_u32(&uq_full[qs]));
+                if (++qs == FF_UQ) {
+                    qs = 0;
+                    qph ^= 1u;
+                }
+                if (u < 0) break;
+                claim = atomicAdd(g.claim, 1);   // the next unit, claimed while this one loads
                 const bool up = u < n_up;
                 const int v = up ? u : u - n_up;
                 const int m_blocks = up ? g.m_up : g.m_down;
@@ -213,7 +250,20 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
             int acc = 0;
             uint32_t acc_phase = 0;
             bool ok = true, issued = false;
-            for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+            int qs = 0;
+            uint32_t qph = 0;
+            while (ok) {
+                if (!mbar_wait(smem_u32(&uq_full[qs]), qph, ctx, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                const int u = uq[qs];
+                mbar_arrive(smem_u32(&uq_empty[qs]));
+                if (++qs == FF_UQ) {
+                    qs = 0;
+                    qph ^= 1u;
+                }
+                if (u < 0) break;
                 const bool up = u < n_up;
                 const int v = up ? u : u - n_up;
                 const int4 sc = g.sched[v / (up ? g.m_up : g.m_down)];
@@ -269,7 +319,18 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
         int acc = 0;
         uint32_t acc_phase = 0;
         const float inv_h = (FP8) ? __frcp_rn(g.h_scale) : 1.0f;
-        for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+        int qs = 0;
+        uint32_t qph = 0;
+        while (true) {
+            if (!mbar_wait_warp(smem_u32(&uq_full[qs]), qph, ctx, abort_flag)) break;
+            const int u = uq[qs];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&uq_empty[qs]));
+            if (++qs == FF_UQ) {
+                qs = 0;
+                qph ^= 1u;
+            }
+            if (u < 0) break;
             const bool up = u < n_up;
             const int v = up ? u : u - n_up;
             const int m_blocks = up ? g.m_up : g.m_down;
@@ -342,7 +403,7 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
                 // proxy (the TMA loads of H), the warp barrier orders them before lane 0's release
                 fence_proxy_async_global();
                 __syncwarp();
-                const bool hold = g.debug_hold && blockIdx.x == 0 && u == (int)blockIdx.x;
+                const bool hold = g.debug_hold && u == 0;
                 if (lane == 0 && !hold) red_release_add(g.done + s_idx, 1);
             }
             if (++acc == 2) {
@@ -393,7 +454,8 @@ bool map_ffn(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, bool 
 }  // namespace
 
 // Both projections of the grouped FFN in one launch.  xp [rows][H] and hb [rows][F]
-// (bf16, or E4M3 codes), y [rows][H] bf16; done: max_sched ints, zero before the launch.
+// (bf16, or E4M3 codes), y [rows][H] bf16; done: max_sched + 1 ints (the per-entry counters, then
+// the unit claim counter), zero before the launch.
 cudaError_t launch_grouped_ffn(bool fp8, const void* w_up, const void* w_down, int E, int F, int H, const void* xp,
                                void* hb, void* y, int64_t rows, const int4* sched, const int* n_sched, int* done,
                                const GemmPlan& plan, const float* su, const float* sd, float x_scale, float h_scale,
@@ -410,6 +472,7 @@ cudaError_t launch_grouped_ffn(bool fp8, const void* w_up, const void* w_down, i
     g.sched = sched;
     g.n_sched = n_sched;
     g.done = done;
+    g.claim = done + plan.max_sched;
     g.m_up = (F + FF_BM - 1) / FF_BM;
     g.m_down = (H + FF_BM - 1) / FF_BM;
     g.F = F;
@@ -429,7 +492,8 @@ cudaError_t launch_grouped_ffn(bool fp8, const void* w_up, const void* w_down, i
     const int64_t max_units = (int64_t)plan.max_sched * (g.m_up + g.m_down);
     const int grid = (int)(max_units < num_sms ? max_units : num_sms);
     auto kfn = fp8 ? grouped_ffn_kernel<true> : grouped_ffn_kernel<false>;
-    const size_t smem = plan.smem_bytes + 16 + (size_t)FF_EPI_WARPS * 16 * 32 * sizeof(uint16_t);
+    const size_t smem = plan.smem_bytes + 16 + (size_t)FF_EPI_WARPS * 16 * 32 * sizeof(uint16_t) +
+                        2 * FF_UQ * sizeof(uint64_t) + FF_UQ * sizeof(int);
     cudaError_t err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     return launch_k(kfn, dim3(grid), dim3(FF_THREADS), smem, stream, maps, g, ctx);

@@ -18,8 +18,8 @@ same counters, parities and arrival counts), in a discrete-event model:
 
 Under many random interleavings every consumer must read exactly the tag it
 expects, no producer may overwrite data that has not been consumed, and every
-role must finish.  Two planted protocol mistakes must be caught, so the check
-is not vacuous.
+role must finish.  Planted protocol mistakes must be caught, so the check is
+not vacuous.
 """
 import random
 from collections import deque
@@ -415,36 +415,69 @@ def gemm_pair(sim, units, k_stages, NS, n_epi=4):
 
 # ----------------------------------------------------------------------------- one-launch FFN (grouped_ffn.cu)
 
-def ffn_fused(sim, n_ctas, entries, m_up, m_down, k_up, k_down, NS, n_epi=4, plant=None):
-    """grouped_ffn_kernel on n_ctas CTAs: each walks units u = cta, cta + n_ctas, ... of the list
-    [up units (entry, block)] + [down units], with the per-CTA TMA ring and two accumulators of
-    the grouped GEMM.  A down unit of entry s reads H[s]; its producer first waits until the
-    global counter done[s] reaches n_epi * m_up (every epilogue warp of every up unit of s has
-    stored its rows and reported).  Shared: done[] and, per entry, how many up epilogue warps
-    have stored their rows of H."""
+def ffn_fused(sim, n_ctas, entries, m_up, m_down, k_up, k_down, NS, n_epi=4, UQ=4, plant=None):
+    """grouped_ffn_kernel on n_ctas CTAs.  The units are the list [up units (entry, block)] +
+    [down units]; each CTA's producer claims the next unit from a global counter (one atomic
+    step, the next claim taken while the current unit loads) and publishes it in a UQ-slot
+    queue in shared memory (uq_full: 1 arrival; uq_empty: the MMA thread and the n_epi epilogue
+    warps), from which the MMA thread and every epilogue warp read the same sequence; then the
+    per-CTA TMA ring and two accumulators of the grouped GEMM.  A down unit of entry s reads
+    H[s]; its producer first waits until the global counter done[s] reaches n_epi * m_up (every
+    epilogue warp of every up unit of s has stored its rows and reported).  Shared: the claim
+    counter, done[] and, per entry, how many up epilogue warps have stored their rows of H."""
     n_up, n_down = entries * m_up, entries * m_down
     units = [("up", u // m_up) for u in range(n_up)] + [("down", u // m_down) for u in range(n_down)]
+    n_units = len(units)
+    claim = [0]
     done = [0] * entries
     stored = [0] * entries
     target = n_epi * m_up if plant != "early_read" else n_epi * (m_up - 1)   # planted: one up unit short
+    uq_readers = 1 + n_epi if plant != "queue_short" else 1                 # planted: only the MMA frees a slot
 
     def cta(c):
-        mine = units[c::n_ctas]
         full, empty = [Bar(1) for _ in range(NS)], [Bar(1) for _ in range(NS)]
         tfull, tempty = [Bar(1) for _ in range(2)], [Bar(n_epi) for _ in range(2)]
+        uq_full, uq_empty = [Bar(1) for _ in range(UQ)], [Bar(uq_readers) for _ in range(UQ)]
+        uq = [None] * UQ
+        published = []                      # the units this CTA claimed, in order
         smem, fresh = [None] * NS, [False] * NS
         tmem = [None] * 2
 
+        def take(who, i, q, arrive=True):
+            u = uq[q]
+            check(u == (published[i] if i < len(published) else -1),
+                  f"CTA {c}: {who} read unit {u} from queue slot {q}, expected entry {i} of {published}")
+            if arrive:
+                uq_empty[q].arrive()
+            return u
+
         def producer():
-            st, ph = 0, 0
-            for i, (kind, s) in enumerate(mine):
+            st, ph, q, qph = 0, 0, 0, 0
+            nxt = claim[0]
+            claim[0] += 1
+            while True:
+                u = nxt if nxt < n_units else -1
+                yield (lambda q_=q, p=qph: uq_empty[q_].passed(p ^ 1))
+                uq[q] = u
+                if u >= 0:
+                    published.append(u)
+                uq_full[q].arrive()
+                q += 1
+                if q == UQ:
+                    q, qph = 0, qph ^ 1
+                if u < 0:
+                    return
+                yield (lambda: True)
+                nxt = claim[0]
+                claim[0] += 1
+                kind, s = units[u]
                 if kind == "down":
                     yield (lambda s=s: done[s] >= target)
                 ks_n = k_up if kind == "up" else k_down
                 for ks in range(ks_n):
                     yield (lambda s_=st, p=ph: empty[s_].passed(p ^ 1))
 
-                    def land(s_=st, tag=(c, i, ks), kind=kind, s=s):
+                    def land(s_=st, tag=(c, u, ks), kind=kind, s=s):
                         check(not fresh[s_], f"CTA {c}: TMA overwrote stage {s_} before the MMA consumed it")
                         if kind == "down":
                             check(stored[s] == n_epi * m_up, f"CTA {c}: read H of entry {s} with "
@@ -457,12 +490,21 @@ def ffn_fused(sim, n_ctas, entries, m_up, m_down, k_up, k_down, NS, n_epi=4, pla
                         st, ph = 0, ph ^ 1
 
         def mma():
-            st, ph, acc, aph = 0, 0, 0, 0
-            for i, (kind, s) in enumerate(mine):
+            st, ph, acc, aph, q, qph, i = 0, 0, 0, 0, 0, 0, 0
+            while True:
+                yield (lambda q_=q, p=qph: uq_full[q_].passed(p))
+                u = take("MMA", i, q)
+                i += 1
+                q += 1
+                if q == UQ:
+                    q, qph = 0, qph ^ 1
+                if u < 0:
+                    return
+                kind, s = units[u]
                 yield (lambda a=acc, p=aph: tempty[a].passed(p ^ 1))
                 for ks in range(k_up if kind == "up" else k_down):
                     yield (lambda s_=st, p=ph: full[s_].passed(p))
-                    check(smem[st] == (c, i, ks), f"CTA {c}: MMA read stage {st} holding {smem[st]}")
+                    check(smem[st] == (c, u, ks), f"CTA {c}: MMA read stage {st} holding {smem[st]}")
 
                     def mma_done(s_=st):
                         fresh[s_] = False
@@ -472,8 +514,8 @@ def ffn_fused(sim, n_ctas, entries, m_up, m_down, k_up, k_down, NS, n_epi=4, pla
                     if st == NS:
                         st, ph = 0, ph ^ 1
 
-                def acc_done(a=acc, i=i):
-                    tmem[a] = i
+                def acc_done(a=acc, u=u):
+                    tmem[a] = u
                     tfull[a].arrive()
                 sim.post(("tc", c), acc_done)
                 acc += 1
@@ -481,10 +523,19 @@ def ffn_fused(sim, n_ctas, entries, m_up, m_down, k_up, k_down, NS, n_epi=4, pla
                     acc, aph = 0, aph ^ 1
 
         def epilogue(w):
-            acc, aph = 0, 0
-            for i, (kind, s) in enumerate(mine):
+            acc, aph, q, qph, i = 0, 0, 0, 0, 0
+            while True:
+                yield (lambda q_=q, p=qph: uq_full[q_].passed(p))
+                u = take(f"epilogue warp {w}", i, q, arrive=plant != "queue_short")
+                i += 1
+                q += 1
+                if q == UQ:
+                    q, qph = 0, qph ^ 1
+                if u < 0:
+                    return
+                kind, s = units[u]
                 yield (lambda a=acc, p=aph: tfull[a].passed(p))
-                check(tmem[acc] == i, f"CTA {c}: epilogue read accumulator {acc} holding {tmem[acc]}")
+                check(tmem[acc] == u, f"CTA {c}: epilogue read accumulator {acc} holding {tmem[acc]}")
                 tempty[acc].arrive()
                 if kind == "up":
                     stored[s] += 1           # this warp's rows of H are stored (and fenced)
@@ -502,21 +553,39 @@ def ffn_fused(sim, n_ctas, entries, m_up, m_down, k_up, k_down, NS, n_epi=4, pla
     for c in range(n_ctas):
         cta(c)
 
+    def all_units_once():
+        return claim[0] >= n_units
+    return all_units_once
+
 
 @pytest.mark.parametrize("n_ctas,entries,m_up,m_down,k_up,k_down,NS",
                          [(3, 4, 3, 4, 4, 3, 3), (2, 5, 2, 3, 3, 2, 2), (4, 3, 2, 2, 2, 2, 4), (5, 2, 3, 2, 2, 3, 2)])
 def test_one_launch_ffn_protocol(n_ctas, entries, m_up, m_down, k_up, k_down, NS):
     for seed in range(25):
         sim = Sim(seed)
-        ffn_fused(sim, n_ctas, entries, m_up, m_down, k_up, k_down, NS)
-        assert sim.run() == "done"
+        claimed_all = ffn_fused(sim, n_ctas, entries, m_up, m_down, k_up, k_down, NS)
+        assert sim.run() == "done" and claimed_all()
+
+
+def test_a_unit_queue_freed_by_the_mma_alone_is_caught():
+    """Planted: the queue slots count only the MMA thread's read, so the producer may overwrite a
+    slot an epilogue warp has not read yet."""
+    caught = 0
+    for seed in range(40):
+        sim = Sim(seed)
+        ffn_fused(sim, 2, 6, 3, 3, 1, 1, 2, UQ=2, plant="queue_short")
+        try:
+            sim.run()
+        except Violation:
+            caught += 1
+    assert caught > 0
 
 
 def test_a_down_unit_waiting_for_too_few_reports_is_caught():
     caught = 0
     for seed in range(25):
         sim = Sim(seed)
-        ffn_fused(sim, 3, 4, 3, 4, 4, 3, 3, plant="early_read")
+        ffn_fused(sim, 4, 2, 3, 2, 3, 2, 2, plant="early_read")
         try:
             sim.run()
         except Violation:

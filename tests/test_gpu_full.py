@@ -189,7 +189,7 @@ def test_fp8_forward_parity_decode_shape(moe):
 @pytest.mark.parametrize("one_launch", [1, 0], ids=["one_launch_ffn", "two_launches"])
 def test_expired_wait_is_reported_and_the_context_stays_usable(moe, one_launch):
     """Two launches: block 0's producer withholds its first load, so the MMA's wait expires.
-    One launch: block 0's first up unit withholds its report, so the down units of its entry
+    One launch: the first up unit of the list withholds its report, so the down units of its entry
     wait on the counter in vain.  Either way the status is MOE_ETIMEOUT and the next call is
     right."""
     moe.debug_set(8, one_launch)
@@ -209,7 +209,7 @@ def _expired_wait_case(moe):
     ws = moe.alloc_workspace(dims)
     y = torch.empty(w.T * w.K, w.H, dtype=torch.bfloat16, device="cuda")
     moe.debug_set(1, 20_000_000)   # 20 ms limit on every bounded wait
-    moe.debug_set(2, 1)            # block 0 withholds its first load (or its first report)
+    moe.debug_set(2, 1)            # block 0 withholds its first load (or unit 0 its report)
     try:
         moe.expert_ffn(dims, d["x"], dev(offsets), dev(perm_src), d["wu"], d["wd"], None, y, ws)
         assert moe.check_device_error_status() == moe.MOE_ETIMEOUT
