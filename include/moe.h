@@ -334,10 +334,11 @@ moe_status moe_set_stage_events(void* const* events, int32_t n);
  * (the default) on single CTAs; what = 4: largest batch (tokens) that the
  * router computes in one launch of 8-CTA clusters split over the experts (0:
  * never; value < 0 restores the default of 256); what = 5: router of the
- * larger batches: 0 (the default) by batch size (one launch of clusters split
- * over the hidden dimension from 3072 tokens when E <= 128, else the tiled
- * logits kernel and the top-K kernel), 1 always the two kernels, 2 always the
- * hidden-split clusters when E <= 128; other values MOE_EINVAL; what = 6:
+ * larger batches: 0 (the default) by batch size (the tensor-core router --
+ * int8 slices, then exact integer products on the tensor cores -- when E <= 128,
+ * else the tiled logits kernel and the top-K kernel), 1 always the two
+ * kernels, 2 always the hidden-split clusters when E <= 128, 3 always the
+ * tensor-core router when E <= 128; other values MOE_EINVAL; what = 6:
  * value 0 launches every kernel without programmatic stream serialization
  * (each kernel then starts only after its predecessor has finished), 1 (the
  * default) lets each kernel start while its predecessor finishes and wait

@@ -675,7 +675,7 @@ moe_status moe_debug_set(int32_t what, int64_t value) {
         return MOE_OK;
     }
     if (what == 5) {
-        if (value < 0 || value > 2) return MOE_EINVAL;
+        if (value < 0 || value > 3) return MOE_EINVAL;
         set_router_split((int)value);
         return MOE_OK;
     }

@@ -17,9 +17,14 @@ struct RouterPlan {
     int S;
     int nchunks;
     int num_sms;
+    int tc;               // 1: the tensor-core router (route_tc.cu), its scratch in the P region
     size_t p_bytes, xn_bytes, wn_bytes;
 };
 RouterPlan router_plan(int64_t T, int H, int E, int num_sms);
+size_t route_tc_scratch_bytes(int64_t T, int H, int E);
+cudaError_t launch_route_tc(const uint16_t* x, const uint16_t* wr, const float* bias, int64_t T, int H, int E,
+                            int K, int32_t* idx, float* w, void* scratch, int num_sms, const DevCtx& ctx,
+                            cudaStream_t stream, void (*between)(cudaStream_t));
 cudaError_t launch_route(const uint16_t* x, const uint16_t* wr, const float* bias, int64_t T, int H, int E,
                          int K, int32_t* idx, float* w, double* P, double* xn2, double* wn2,
                          const RouterPlan& plan, const DevCtx& ctx, cudaStream_t stream,

@@ -32,6 +32,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "route_select.cuh"
 
 namespace moe {
 
@@ -181,290 +182,8 @@ struct RouterTopkArgs {
     float* w;             // [T][K]
 };
 
-constexpr int TK_MAXJ = 8;        // experts per lane (E <= 256)
 constexpr int TK_WARPS = 8;       // tokens per block
 constexpr int TK_CAP = TK_WARPS * 256;
-
-// warp arg-max of (value, -index)
-__device__ __forceinline__ void warp_argmax(double& v, int& e) {
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-        const double ov = __shfl_xor_sync(0xffffffffu, v, off);
-        const int oe = __shfl_xor_sync(0xffffffffu, e, off);
-        if (ov > v || (ov == v && oe < e)) {
-            v = ov;
-            e = oe;
-        }
-    }
-}
-
-__device__ __forceinline__ void warp_argmax_i64(long long& v, int& e) {
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-        const long long ov = __shfl_xor_sync(0xffffffffu, v, off);
-        const int oe = __shfl_xor_sync(0xffffffffu, e, off);
-        if (ov > v || (ov == v && oe < e)) {
-            v = ov;
-            e = oe;
-        }
-    }
-}
-
-// Exact fixed-point logit (units of 2^-40) of expert e for token row xr:
-// every bf16 product (exact in fp32) scaled by 2^40 and rounded to the
-// nearest integer, summed exactly; one warp, 16-byte loads issued eight
-// fragments per lane at a time so that their latencies overlap.
-__device__ long long exact_logit(const uint16_t* xr, const uint16_t* wrow, int H, const float* bias, int e,
-                                 int lane) {
-    constexpr int B = 8;
-    const uint4* xv = reinterpret_cast<const uint4*>(xr);
-    const uint4* wv = reinterpret_cast<const uint4*>(wrow);
-    const int nv = H / 8;
-    long long acc = 0;
-    for (int v0 = lane; v0 < nv; v0 += 32 * B) {
-        uint4 a[B], b[B];
-#pragma unroll
-        for (int i = 0; i < B; ++i) {
-            const int v = v0 + 32 * i;
-            a[i] = b[i] = make_uint4(0, 0, 0, 0);
-            if (v < nv) {
-                a[i] = xv[v];
-                b[i] = wv[v];
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < B; ++i) {
-            const uint32_t aa[4] = {a[i].x, a[i].y, a[i].z, a[i].w};
-            const uint32_t bb[4] = {b[i].x, b[i].y, b[i].z, b[i].w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float p0 = __fmul_rn(__uint_as_float(aa[j] << 16), __uint_as_float(bb[j] << 16));
-                const float p1 =
-                    __fmul_rn(__uint_as_float(aa[j] & 0xFFFF0000u), __uint_as_float(bb[j] & 0xFFFF0000u));
-                acc += __float2ll_rn(__fmul_rn(p0, 0x1p40f));
-                acc += __float2ll_rn(__fmul_rn(p1, 0x1p40f));
-            }
-        }
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (bias) acc += __float2ll_rn(__fmul_rn(bias[e], 0x1p40f));
-    return acc;
-}
-
-constexpr int TK_MAXK = 16;       // K <= 16
-
-// Relative bound of an approximate logit l~ (in units of ||x|| ||w_e||, which
-// bounds sum_h |x_h w_eh| by Cauchy-Schwarz) for a summation whose fp32 part
-// rounds at most n32 times along any product's path (g_n32, u = 2^-24) and
-// whose fp64 part adds at most d64 times (d64 2^-52 >= g_d64 at u = 2^-53);
-// 2^-40 is slack for the roundings of the bound's own arithmetic.
-__host__ __device__ inline double router_k_rel(int n32, int d64) {
-    const double g = (double)n32 * 0x1p-24;
-    return g / (1.0 - g) + (double)d64 * 0x1p-52 + 0x1p-40;
-}
-
-// Order-preserving integer key of a double (unsigned order = numeric order;
-// -0 is mapped with +0 by adding 0.0 first).
-__device__ __forceinline__ unsigned long long order_key(double v) {
-    const unsigned long long u = (unsigned long long)__double_as_longlong(v + 0.0);
-    return (u >> 63) ? ~u : (u | 0x8000000000000000ull);
-}
-__device__ __forceinline__ double key_value(unsigned long long k) {
-    return __longlong_as_double((long long)((k >> 63) ? (k & 0x7fffffffffffffffull) : ~k));
-}
-
-// warp arg-max of (key, -index)
-__device__ __forceinline__ void warp_argmax_key(unsigned long long& k, int& e) {
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-        const unsigned long long ok = __shfl_xor_sync(0xffffffffu, k, off);
-        const int oe = __shfl_xor_sync(0xffffffffu, e, off);
-        if (ok > k || (ok == k && oe < e)) {
-            k = ok;
-            e = oe;
-        }
-    }
-}
-
-// Per-block constants of the bound: the largest ||w_e|| (from the fp32 squared
-// norms Q, inflated by 1 + (H+64) 2^-23 to an upper bound) and the largest
-// |b_e|.  One warp; every lane returns both.
-__device__ __forceinline__ void bound_constants(const double* Q, const float* bias, int H, int E, int lane,
-                                                double& wnmax, double& bmax) {
-    double q = 0.0, b = 0.0;
-    for (int e = lane; e < E; e += 32) {
-        q = fmax(q, Q[e]);
-        if (bias) b = fmax(b, fabs((double)bias[e]));
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-        q = fmax(q, __shfl_xor_sync(0xffffffffu, q, off));
-        b = fmax(b, __shfl_xor_sync(0xffffffffu, b, off));
-    }
-    wnmax = sqrt(q * (1.0 + (double)(H + 64) * 0x1p-23));
-    bmax = b;
-}
-
-// Ranks one token's approximate logits l~ (one warp, E <= 256): the K best
-// (ties to the lower index) into out_e/out_l (shared memory of this token,
-// written by lane 0), and whether every gap among the K+1 best exceeds
-// 2 eps*.  When it does not, the token's candidates (every expert whose exact
-// logit could still be in the top K) are appended to the block's list under
-// `slot`.  With k_rel bounding |l~ - l| / (||x|| ||w_e||) for the caller's
-// summation (see router_k_rel),
-//   eps* = k_rel ||x|| max_e ||w_e|| + (H+1) 2^-41 + (2 ||x|| max_e ||w_e|| + max_e |b_e| + 1) 2^-50
-// bounds every |l~_e - l_e| (the last term covers the fp64 roundings of l~ + b).
-// The ranking compares order-preserving integer keys of l~.
-__device__ __forceinline__ bool rank_certified(const double* Lrow, double xsq, const float* bias, int H, int E,
-                                               int K, double k_rel, double wnmax, double bmax, int lane, int slot,
-                                               int* out_e, double* out_l, bool& range_bad, uint8_t* c_tok,
-                                               uint16_t* c_e, int* n_cand) {
-    const int nj = (E + 31) / 32;
-    const double xnorm = sqrt(xsq * (1.0 + (double)(H + 64) * 0x1p-23));   // fp32 norm sum -> upper bound
-    const double xw = xnorm * wnmax;
-    if (xw >= 0x1p22 || bmax >= 0x1p21) range_bad = true;
-    const double eps_star = k_rel * xw + (double)(H + 1) * 0x1p-41 + (2.0 * xw + bmax + 1.0) * 0x1p-50;
-
-    // the lane's keys, sorted once by (key, -e) descending (empty slots: key 0, below every real key)
-    unsigned long long sk[TK_MAXJ];
-    int se[TK_MAXJ];
-#pragma unroll
-    for (int j = 0; j < TK_MAXJ; ++j) {
-        const int e = lane + 32 * j;
-        sk[j] = 0ull;
-        se[j] = e;
-        if (j < nj && e < E) {
-            double l = Lrow[e];
-            if (bias) l += (double)bias[e];
-            sk[j] = order_key(l);
-        }
-    }
-    auto cx = [&](int i, int j) {   // (i, j) in descending order after the exchange
-        const bool sw = sk[i] < sk[j] || (sk[i] == sk[j] && se[i] > se[j]);
-        const unsigned long long tk = sw ? sk[j] : sk[i];
-        const int te = sw ? se[j] : se[i];
-        sk[j] = sw ? sk[i] : sk[j];
-        se[j] = sw ? se[i] : se[j];
-        sk[i] = tk;
-        se[i] = te;
-    };
-    // Batcher's odd-even merge sort of 8
-    cx(0, 1); cx(2, 3); cx(4, 5); cx(6, 7);
-    cx(0, 2); cx(1, 3); cx(4, 6); cx(5, 7);
-    cx(1, 2); cx(5, 6);
-    cx(0, 4); cx(1, 5); cx(2, 6); cx(3, 7);
-    cx(2, 4); cx(3, 5);
-    cx(1, 2); cx(3, 4); cx(5, 6);
-
-    // the K+1 best by l~ (ties to the lower index): the best of the lanes' heads, popped
-    const int nsel = min(K + 1, E);
-    double prev = 0.0, lk = 0.0;
-    bool certified = true;
-    for (int k = 0; k < nsel; ++k) {
-        unsigned long long bk = sk[0];
-        int be = se[0];
-        warp_argmax_key(bk, be);
-        const double bv = key_value(bk);
-        if (k < K) {
-            if (lane == 0) {
-                out_e[k] = be;
-                out_l[k] = bv;
-            }
-            lk = bv;
-        }
-        if (k > 0 && !(prev - bv > 2.0 * eps_star)) certified = false;
-        prev = bv;
-        if ((be & 31) == lane) {
-#pragma unroll
-            for (int j = 0; j + 1 < TK_MAXJ; ++j) {
-                sk[j] = sk[j + 1];
-                se[j] = se[j + 1];
-            }
-            sk[TK_MAXJ - 1] = 0ull;
-        }
-    }
-    if (!certified) {
-        // candidates: every expert that could still be in the exact top K
-        const unsigned long long thr = order_key(lk - 2.0 * eps_star);
-#pragma unroll
-        for (int j = 0; j < TK_MAXJ; ++j) {
-            const int e = lane + 32 * j;
-            bool c = false;
-            if (j < nj && e < E) {
-                double l = Lrow[e];
-                if (bias) l += (double)bias[e];
-                c = order_key(l) >= thr;
-            }
-            const uint32_t m = __ballot_sync(0xffffffffu, c);
-            int base = 0;
-            if (lane == 0 && m) base = atomicAdd(n_cand, __popc(m));
-            base = __shfl_sync(0xffffffffu, base, 0);
-            if (c) {
-                const int i = base + __popc(m & ((1u << lane) - 1u));
-                c_tok[i] = (uint8_t)slot;
-                c_e[i] = (uint16_t)e;
-            }
-        }
-    }
-    __syncwarp();
-    return certified;
-}
-
-// Exact fixed-point logits of the block's listed candidates, one warp each;
-// token slot s of the list is token t_base + s.
-__device__ __forceinline__ void exact_candidates(int nc, const uint8_t* c_tok, const uint16_t* c_e,
-                                                 long long* c_val, int64_t t_base, const uint16_t* x,
-                                                 const uint16_t* wr, int H, const float* bias, int warp,
-                                                 int n_warps, int lane) {
-    for (int i = warp; i < nc; i += n_warps) {
-        const int e = c_e[i];
-        const long long v = exact_logit(x + (t_base + c_tok[i]) * H, wr + (int64_t)e * H, H, bias, e, lane);
-        if (lane == 0) c_val[i] = v;
-    }
-}
-
-// Finishes one token (one warp): if its order was not certified, ranks its
-// candidates by exact logit (ties to the lower index) into out_e/out_l; then
-// the renormalised softmax over the K kept logits (w_k = exp(l_k - l_0) / z,
-// z summed in order k = 0..K-1), and the K (index, weight) pairs of row t.
-__device__ __forceinline__ void finish_token(bool certified, int slot, int64_t t, int nc, uint8_t* c_tok,
-                                             const uint16_t* c_e, const long long* c_val, int K, int* out_e,
-                                             double* out_l, int lane, int32_t* idx, float* w) {
-    if (!certified) {
-        for (int k = 0; k < K; ++k) {
-            long long bv = LLONG_MIN;
-            int be = 0x7fffffff, bi = -1;
-            for (int i = lane; i < nc; i += 32) {
-                if (c_tok[i] != slot) continue;   // other tokens, or already taken (0xFF)
-                const long long v = c_val[i];
-                const int e = c_e[i];
-                if (bi < 0 || v > bv || (v == bv && e < be)) {
-                    bv = v;
-                    be = e;
-                    bi = i;
-                }
-            }
-            int src_e = be;
-            warp_argmax_i64(bv, src_e);
-            if (bi >= 0 && be == src_e) c_tok[bi] = 0xFF;   // taken (this lane held it)
-            if (lane == 0) {
-                out_e[k] = src_e;
-                out_l[k] = (double)bv * 0x1p-40;
-            }
-            __syncwarp();
-        }
-    }
-    // lane k < K holds term k
-    const double l0 = out_l[0];
-    const float ex = lane < K ? expf((float)(out_l[lane < K ? lane : 0] - l0)) : 0.0f;
-    float z = 0.0f;
-    for (int k = 0; k < K; ++k) z += __shfl_sync(0xffffffffu, ex, k);
-    if (lane < K) {
-        idx[t * K + lane] = out_e[lane];
-        w[t * K + lane] = ex / z;
-    }
-}
 
 // One warp per token ranks l~; tokens whose order the bound leaves open put
 // their candidates in a block-wide list whose exact logits all 8 warps
@@ -1103,19 +822,26 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(NTH, 1)
 
 // ----------------------------------------------------------------------------- host
 
-// Batch-size boundaries of the three router shapes, from CUDA-event timings
-// on B200 (H=2688, E=128, K=6): the expert-split clusters up to 256 tokens
-// (17 us at 64), the two-kernel router in between, the hidden-split clusters
-// from 3072 tokens (101 us at 4096 against 154).
+// Batch-size boundaries of the router shapes, from CUDA-graph timings on
+// B200 (H=2688, E=128, K=6): the expert-split clusters up to 256 tokens
+// (14 us at 64), the two-kernel router up to 2047, the tensor-core router
+// (route_tc.cu) from 2048 tokens (61 / 82 / 148 us at 2048 / 4096 / 8192,
+// against 83 / 98 / 193 for the best of the other two large-batch shapes).
 constexpr int64_t kRouterSmallMaxDefault = 256;
 constexpr int64_t kRouterSplitMin = 3072;
+constexpr int64_t kRouterTcMin = 2048;  // batches from this size take the tensor-core router (E <= 128)
 constexpr size_t kRouterSmallSmemMax = 200 * 1024;
 
 static int router_tt(int64_t T) { return T > 256 ? 64 : 16; }
 
+// Whether a batch takes the tensor-core router (route_tc.cu): by size, or always under
+// hook value 3; never for E > 128, K > 16 or a batch the expert-split clusters take.
+static bool router_tc(int64_t T, int H, int E);
+
 RouterPlan router_plan(int64_t T, int H, int E, int num_sms) {
     RouterPlan p;
     p.num_sms = num_sms;
+    p.tc = router_tc(T, H, E) ? 1 : 0;
     p.nchunks = (H + RT_HC - 1) / RT_HC;
     const int tt = router_tt(T);
     const int64_t tiles = ((T + tt - 1) / tt) * ((E + RT_TE - 1) / RT_TE);
@@ -1128,6 +854,12 @@ RouterPlan router_plan(int64_t T, int H, int E, int num_sms) {
     if (want < 1) want = 1;
     p.S = (int)want;
     p.p_bytes = (size_t)p.S * (size_t)T * (size_t)E * sizeof(double);
+    if (E <= RF_E) {
+        // room for the tensor-core router's slices whenever it could run (sizes do not depend
+        // on the test hooks that choose the path)
+        const size_t tcb = route_tc_scratch_bytes(T, H, E);
+        if (tcb > p.p_bytes) p.p_bytes = tcb;
+    }
     p.xn_bytes = (size_t)p.S * (size_t)T * sizeof(double);
     p.wn_bytes = (size_t)p.S * (size_t)E * sizeof(double);
     return p;
@@ -1137,11 +869,12 @@ RouterPlan router_plan(int64_t T, int H, int E, int num_sms) {
 // use the tiled logits kernel and router_topk_kernel.
 std::atomic<int64_t> g_router_small_max{kRouterSmallMaxDefault};
 // 0: by batch size; 1: every larger batch takes the two-kernel router; 2: every larger
-// batch with E <= 128 takes the hidden-split clusters
+// batch with E <= 128 takes the hidden-split clusters; 3: every larger batch with E <= 128
+// takes the tensor-core router
 std::atomic<int> g_router_split{0};
 
 void set_router_small_max(int64_t v) { g_router_small_max.store(v < 0 ? kRouterSmallMaxDefault : v); }
-void set_router_split(int v) { g_router_split.store(v == 1 || v == 2 ? v : 0); }
+void set_router_split(int v) { g_router_split.store(v >= 1 && v <= 3 ? v : 0); }
 
 // How many clusters of the split-cluster router fit on the device at once (a
 // cluster sits inside one GPC, so this is not the SM count over CS); cached
@@ -1231,6 +964,12 @@ static int router_small_tb(int64_t T, int H, int E, bool query) {
     return (T + 3) / 4 <= router_small_max_clusters(4, H, E) ? 4 : 8;
 }
 
+static bool router_tc(int64_t T, int H, int E) {
+    if (E > RF_E || router_small_tb(T, H, E, false) > 0) return false;
+    const int mode = g_router_split.load();
+    return mode == 3 || (mode == 0 && T >= kRouterTcMin);
+}
+
 template <int TB>
 static cudaError_t launch_router_small(const RouterSmallArgs& ra, const DevCtx& ctx, cudaStream_t stream) {
     const size_t smem = rs_smem_bytes(TB, ra.H, ra.E);
@@ -1246,6 +985,7 @@ static cudaError_t launch_router_small(const RouterSmallArgs& ra, const DevCtx& 
 int route_launches(int64_t T, int H, int E) {
     if (T == 0) return 0;
     if (router_small_tb(T, H, E, false) > 0) return 1;   // expert-split clusters
+    if (router_tc(T, H, E)) return 3;                    // slices, integer products, selection
     const int split_mode = g_router_split.load();
     if (E <= RF_E && split_mode != 1 && (split_mode == 2 || T >= kRouterSplitMin)) return 1;   // hidden-split
     return 2;   // logits, then top-K
@@ -1256,6 +996,7 @@ cudaError_t launch_route(const uint16_t* x, const uint16_t* wr, const float* bia
                          const RouterPlan& plan, const DevCtx& ctx, cudaStream_t stream,
                          void (*between)(cudaStream_t)) {
     if (T == 0) return cudaSuccess;
+    if (plan.tc) return launch_route_tc(x, wr, bias, T, H, E, K, idx, w, P, plan.num_sms, ctx, stream, between);
     const int tb = router_small_tb(T, H, E, true);
     if (tb > 0) {
         RouterSmallArgs ra{x, wr, bias, T, H, E, K, idx, w};

@@ -68,7 +68,8 @@ extern "C" moe_status moe_route_static(const moe_dims* d, const void* x, const v
     // the smallest plan (one split of the hidden dimension) must fit the array; this is
     // checked before any device call
     moe::RouterPlan plan{};
-    const auto resize = [&](int S) {
+    const auto resize = [&](int S) {   // the split-K kernels' scratch (never the tensor-core router's)
+        plan.tc = 0;
         plan.S = S;
         plan.p_bytes = (size_t)S * (size_t)d->T * (size_t)d->E * sizeof(double);
         plan.xn_bytes = (size_t)S * (size_t)d->T * sizeof(double);
@@ -83,6 +84,8 @@ extern "C" moe_status moe_route_static(const moe_dims* d, const void* x, const v
 
     // the library's usual split of the hidden dimension, reduced until it fits
     plan = moe::router_plan(d->T, d->H, d->E, sms);
+    // the tensor-core router only when its slices fit; otherwise the split-K kernels' own sizes
+    if (!plan.tc || scratch_bytes(plan) > kRouteScratchBytes) resize(plan.S);
     while (plan.S > 1 && scratch_bytes(plan) > kRouteScratchBytes) resize(plan.S - 1);
     if (scratch_bytes(plan) > kRouteScratchBytes) return MOE_EWORKSPACE;
 

@@ -159,17 +159,17 @@ def test_shared_expert_dims_and_pointers_are_checked_on_the_host(moe):
 
 
 def test_forward_launch_count_follows_the_dispatch(moe):
-    """Router: one launch up to 256 tokens (expert-split clusters) and from 3072 (hidden-split
-    clusters), two in between; permutation: one block up to 4096 assignments, else three kernels;
+    """Router: one launch up to 256 tokens (expert-split clusters), two up to 2047 (logits, top-K),
+    three from 2048 (the tensor-core router); permutation: one block up to 4096 assignments, else three kernels;
     then the row gather, the expert FFN (one launch for bf16 and E4M3 experts without a shared
     expert, else the two projections) and the combine."""
     count = lambda T, **kw: moe.forward_launches(moe.dims(T, 2688, 128, 6, 1856, **kw))
-    assert [count(T) for T in (0, 1, 64, 256, 257, 682, 683, 3071, 3072, 4096)] == [0, 5, 5, 5, 6, 6, 8, 8, 7, 7]
+    assert [count(T) for T in (0, 1, 64, 256, 257, 682, 683, 2047, 2048, 4096)] == [0, 5, 5, 5, 6, 6, 8, 8, 9, 9]
     assert count(64, fp8=True) == 5
     assert count(64, nvfp4=True) == count(64, fp8_b128=True) == count(64, Fs=1856) == 6
     try:
         moe.debug_set(8, 0)             # the two projections as two launches
-        assert count(64) == 6 and count(4096) == 8
+        assert count(64) == 6 and count(4096) == 10
         moe.debug_set(8, 1)
         moe.debug_set(4, 0)             # never the expert-split clusters
         assert count(64) == 6
@@ -177,6 +177,8 @@ def test_forward_launch_count_follows_the_dispatch(moe):
         assert count(64) == 5 and count(576) == 5
         moe.debug_set(5, 1)             # always the two kernels
         assert count(4096) == 8
+        moe.debug_set(5, 3)             # always the tensor-core router (slices, products, selection)
+        assert count(576) == 7 and count(4096) == 9
     finally:
         moe.debug_set(8, 1)
         moe.debug_set(4, -1)

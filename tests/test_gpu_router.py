@@ -1,10 +1,11 @@
 """GPU parity of every router shape against the oracle's fixed-point ranking.
 
 Small batches run as one launch of 8-CTA clusters split over the experts;
-larger ones as one launch of clusters split over the hidden dimension (E <=
-128), or as the tiled logits kernel plus the top-K kernel.  Debug hooks 4
-and 5 choose the path, so every case here runs through all three (a case
-with E > 128 sent to the split clusters takes the two-kernel router).
+larger ones as int8 slices multiplied exactly on the tensor cores (E <= 128),
+as one launch of clusters split over the hidden dimension (E <= 128), or as
+the tiled logits kernel plus the top-K kernel.  Debug hooks 4 and 5 choose
+the path, so every case here runs through all four (a case with E > 128 sent
+to the tensor cores or the split clusters takes the two-kernel router).
 Indices must be bit-exact and weights within 1e-5 (fp32 softmax over exact
 selections).
 """
@@ -20,8 +21,9 @@ from _gpu import dev, dev_bf16
 
 pytestmark = pytest.mark.gpu
 
-# path: (largest batch of the expert-split clusters, router of larger batches: 1 two kernels, 2 hidden-split clusters)
-PATHS = {"cluster": (1 << 40, 0), "split": (0, 2), "tiled": (0, 1)}
+# path: (largest batch of the expert-split clusters, router of larger batches: 1 two kernels,
+# 2 hidden-split clusters, 3 tensor cores)
+PATHS = {"cluster": (1 << 40, 0), "split": (0, 2), "tiled": (0, 1), "tensor": (0, 3)}
 
 
 @pytest.fixture(scope="module")
@@ -126,3 +128,23 @@ def test_router_reports_the_range_error(moe, path):
         assert moe.check_device_error_status() == moe.MOE_ERANGE
     finally:
         restore(moe)
+
+
+@pytest.mark.parametrize("path", sorted(PATHS))
+def test_router_wide_dynamic_range(moe, path):
+    """Rows whose values span many binades (a few values near 2^6, the rest down to 2^-20 and
+    subnormal-sized, zeros and a zero row): the tensor-core router's int8 slices drop the small
+    values' low bits, so its bound is wide and many tokens go to the exact pass; the ranking
+    must still be the oracle's."""
+    T, H, E, K = 300, 2688, 128, 6
+    rng = np.random.default_rng(5)
+    x = synth.normal_bf16(synth.key(79, synth.T_X, 0), T * H, W.SIGMA_X).reshape(T, H).copy()
+    wr = synth.normal_bf16(synth.key(79, synth.T_WR, 0), E * H, W.SIGMA_W).reshape(E, H).copy()
+    xf = oracle.bf16_to_f64(x) * np.exp2(rng.integers(-20, 1, size=(T, H)))
+    xf[:, :3] = 64.0 * np.sign(xf[:, :3] + 1e-30)
+    xf[7] = 0.0
+    xf[:, 100:110] = 0.0
+    x = oracle.round_bf16(xf)
+    wf = oracle.bf16_to_f64(wr) * np.exp2(rng.integers(-12, 1, size=(E, H)))
+    wr = oracle.round_bf16(wf)
+    route_case(moe, path, x, wr, W.zipf_bias(80, E), K)
