@@ -459,9 +459,12 @@ def roofline_entry(wl, stages, touched, peaks, peak_kind, workload):
         tc_peak, src = peaks["fp8_tflops"], peaks["fp8_source"]
         tc_sust = None
     else:
-        tc_peak = peaks["bf16_tflops"] * (2.0 if fp8 else 1.0)
-        src = f"{peak_kind} bf16 burst" + (" x 2 (fp8/bf16 nominal ratio)" if fp8 else "")
-        tc_sust = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * (2.0 if fp8 else 1.0)
+        # a contraction takes its own dtype's peak: the measured bf16 one times the nominal ratio
+        ratio = 4.0 if wl.nvfp4 else 2.0 if fp8 else 1.0
+        tc_peak = peaks["bf16_tflops"] * ratio
+        src = f"{peak_kind} bf16 burst" + (" x 4 (nvfp4/bf16 nominal ratio)" if wl.nvfp4 else
+                                           " x 2 (fp8/bf16 nominal ratio)" if fp8 else "")
+        tc_sust = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * ratio
     tflops = flops / (ms * 1e-3) / 1e12
     common = {"kernel": kernel, "ms_per_launch": ms, "algorithmic_bytes_per_launch": algo,
               "algorithmic_flops_per_launch": flops, "traffic": traffic_from_profile(kernel, workload),

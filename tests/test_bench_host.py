@@ -52,6 +52,15 @@ def test_nvfp4_bytes_count_half_byte_codes_and_padded_block_scales():
                                                  + rows * (F // 2 + ksp_f))
 
 
+def test_nvfp4_prefill_takes_the_fp4_tensor_peak():
+    """A contraction is reported against its own dtype's peak: for NVFP4 the measured bf16 burst
+    peak times the nominal fp4/bf16 ratio of 4."""
+    r = entry(6, 128, 0.2, 0.19, "prefill_nvfp4")
+    assert r["bound"] == "tensor" and r["peak"] == pytest.approx(4 * PEAKS["bf16_tflops"])
+    assert r["frac"] == pytest.approx(r["achieved"] / (4 * PEAKS["bf16_tflops"]))
+    assert "x 4" in r["peak_source"]
+
+
 def test_fp8_b128_bytes_count_padded_codes_and_block_scales():
     up = entry(9, 121, 0.2, 0.1, "decode_fp8_b128")
     rows = 64 * 6
