@@ -148,3 +148,24 @@ def test_router_wide_dynamic_range(moe, path):
     wf = oracle.bf16_to_f64(wr) * np.exp2(rng.integers(-12, 1, size=(E, H)))
     wr = oracle.round_bf16(wf)
     route_case(moe, path, x, wr, W.zipf_bias(80, E), K)
+
+
+@pytest.mark.parametrize("fill", [0x00, 0xFF])
+def test_tensor_core_router_ignores_stale_workspace(moe, fill):
+    """The tensor-core router writes every slice, scale and partial it reads: a workspace full of
+    stale bytes gives the oracle's ranking, call after call."""
+    T, H, E, K = 2100, 2688, 128, 6
+    x = synth.normal_bf16(synth.key(81, synth.T_X, 0), T * H, W.SIGMA_X).reshape(T, H)
+    wr = synth.normal_bf16(synth.key(81, synth.T_WR, 0), E * H, W.SIGMA_W).reshape(E, H)
+    bias = W.zipf_bias(81, E)
+    dims = moe.dims(T, H, E, K, 16)
+    ws = moe.alloc_workspace(dims)
+    _, ridx, rw = oracle.route(x, wr, bias, K)
+    for _ in range(2):
+        ws.fill_(fill)
+        idx = torch.empty(T, K, dtype=torch.int32, device="cuda")
+        wt = torch.empty(T, K, dtype=torch.float32, device="cuda")
+        moe.route(dims, dev_bf16(x), dev_bf16(wr), dev(bias), idx, wt, ws)   # T >= 2048: the tensor cores
+        moe.check_device_error()
+        assert np.array_equal(idx.cpu().numpy(), ridx)
+        assert np.max(np.abs(wt.cpu().numpy().astype(np.float64) - rw)) <= 1e-5

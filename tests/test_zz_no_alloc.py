@@ -105,3 +105,28 @@ def test_static_scratch_router_at_large_batches(moe, T, split):
             assert np.max(np.abs(wt - ref_w)) <= 1e-5
     finally:
         moe.debug_set(5, 0)
+
+
+def test_static_scratch_takes_the_tensor_core_router_when_its_slices_fit(moe):
+    """With the tensor-core router forced (debug hooks 4 = 0, 5 = 3), a batch whose int8 slices
+    and partials fit the 8 MiB array (T = 100) takes it from the static scratch too: indices bit
+    for bit against the workspace router under the same hooks, weights within 1e-5."""
+    import synth
+    T, H, E, K, F = 100, 2688, 128, 6, 1856
+    stream = torch.cuda.current_stream().cuda_stream
+    x = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
+    wr = torch.empty(E, H, dtype=torch.bfloat16, device="cuda")
+    synth.normal_bf16_device(synth.key(12, synth.T_X, 0), x.numel(), W.SIGMA_X, x.data_ptr(), stream)
+    synth.normal_bf16_device(synth.key(12, synth.T_WR, 0), wr.numel(), W.SIGMA_W, wr.data_ptr(), stream)
+    dims = moe.dims(T, H, E, K, F)
+    moe.debug_set(4, 0)
+    moe.debug_set(5, 3)
+    try:
+        ref_idx, ref_w = _route_with_workspace(moe, dims, x, wr, None, T, K)
+        for _ in range(2):
+            idx, wt = _route_static_abi(moe, dims, x, wr, None, T, K)
+            assert np.array_equal(idx, ref_idx)
+            assert np.max(np.abs(wt - ref_w)) <= 1e-5
+    finally:
+        moe.debug_set(4, -1)
+        moe.debug_set(5, 0)
