@@ -824,12 +824,12 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(NTH, 1)
 
 // Batch-size boundaries of the router shapes, from CUDA-graph timings on
 // B200 (H=2688, E=128, K=6): the expert-split clusters up to 256 tokens
-// (14 us at 64), the two-kernel router up to 2047, the tensor-core router
-// (route_tc.cu) from 2048 tokens (61 / 82 / 148 us at 2048 / 4096 / 8192,
-// against 83 / 98 / 193 for the best of the other two large-batch shapes).
+// (14 us at 64), the two-kernel router up to 1023, the tensor-core router
+// (route_tc.cu) from 1024 tokens (43 / 54 / 75 / 131 us at 1024 / 2048 / 4096 /
+// 8192, against 50 / 83 / 98 / 193 for the best of the other large-batch shapes).
 constexpr int64_t kRouterSmallMaxDefault = 256;
 constexpr int64_t kRouterSplitMin = 3072;
-constexpr int64_t kRouterTcMin = 2048;  // batches from this size take the tensor-core router (E <= 128)
+constexpr int64_t kRouterTcMin = 1024;  // batches from this size take the tensor-core router (E <= 128)
 constexpr size_t kRouterSmallSmemMax = 200 * 1024;
 
 static int router_tt(int64_t T) { return T > 256 ? 64 : 16; }

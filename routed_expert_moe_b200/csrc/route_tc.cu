@@ -63,9 +63,9 @@ struct RouterQuantArgs {
 };
 
 // One warp per row.  The largest biased exponent e1 of the row's values gives
-// |v| < 2^(e1 - 126), so q = 148 - e1 keeps |X| < 2^22.  A value m8 2^(e - 134)
-// (m8 its 8-bit significand, e its biased exponent, 1 for subnormals) becomes
-// X = m8 2^sh with sh = e - e1 + 14 <= 14, rounded to nearest even when sh < 0.
+// |v| < 2^(e1 - 126), so q = 148 - e1 keeps |X| = |rint(v 2^q)| < 2^22 (a value
+// m8 2^(e - 134), m8 its 8-bit significand, becomes m8 2^(e - e1 + 14), rounded
+// to nearest even).
 __global__ void __launch_bounds__(256) router_quant_kernel(RouterQuantArgs a, DevCtx ctx) {
     pdl_enter();
     const int lane = threadIdx.x & 31;
@@ -74,31 +74,32 @@ __global__ void __launch_bounds__(256) router_quant_kernel(RouterQuantArgs a, De
     for (int64_t r = (int64_t)blockIdx.x * 8 + threadIdx.x / 32; r < rows; r += (int64_t)gridDim.x * 8) {
         const uint4* src = reinterpret_cast<const uint4*>(r < a.T ? a.x + r * a.H : a.wr + (r - a.T) * a.H);
         const size_t plane = (size_t)rows * a.H;
-        // a value with exponent field eb becomes X = m8 2^(eb - e1 + 14), rounded (see above)
-        auto encode = [&](uint32_t h, int e1, long long& S, uint32_t& hb, uint32_t& mb, uint32_t& lb, int sh8) {
-            const int eb = (int)((h >> 7) & 0xFFu);
-            const int m8 = eb ? (int)(0x80u | (h & 0x7Fu)) : (int)(h & 0x7Fu);
-            const int sh = (eb ? eb : 1) - e1 + 14;
-            // m8 2^sh with 8 fractional bits, rounded to nearest even (0 when m8 2^sh < 1/2)
-            const int f8 = sh >= -8 ? m8 << (sh + 8) : 0;
-            int X = (f8 + 127 + ((f8 >> 8) & 1)) >> 8;
-            S += X;
-            if (h & 0x8000u) X = -X;
-            // X = 2^16 h + 2^8 m + l with l, m in [-128, 127]: l is X's low byte as a signed value
-            const int lo = (int)(int8_t)(X & 0xFF);
-            const int X1 = (X - lo) >> 8;
-            const int mi = (int)(int8_t)(X1 & 0xFF);
-            const int hi = (X1 - mi) >> 8;
-            hb |= (uint32_t)(hi & 0xFF) << sh8;
-            mb |= (uint32_t)(mi & 0xFF) << sh8;
-            lb |= (uint32_t)(lo & 0xFF) << sh8;
-        };
-        auto emit = [&](const uint4& f, int v, int e1, long long& S) {
+        // X = rint(v 2^q): v (bf16, exact in fp32) times 2^q in two exact power-of-two steps
+        // (q may exceed fp32's exponent range), rounded to nearest even by the conversion; a
+        // product below 2^-149 would round to X = 0 anyway
+        auto emit = [&](const uint4& f, int v, float s1, float s2, long long& S) {
             const uint32_t u[4] = {f.x, f.y, f.z, f.w};
+            int X[8];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                X[2 * j] = __float2int_rn(__fmul_rn(__fmul_rn(__uint_as_float(u[j] << 16), s1), s2));
+                X[2 * j + 1] = __float2int_rn(__fmul_rn(__fmul_rn(__uint_as_float(u[j] & 0xFFFF0000u), s1), s2));
+            }
+            int sa = 0;   // |X| < 2^22: eight of them fit an int
             uint32_t ph[2] = {0u, 0u}, pm[2] = {0u, 0u}, pl[2] = {0u, 0u};
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-                encode((u[j >> 1] >> ((j & 1) * 16)) & 0xFFFFu, e1, S, ph[j >> 2], pm[j >> 2], pl[j >> 2], (j & 3) * 8);
+            for (int j = 0; j < 8; ++j) {
+                sa += abs(X[j]);
+                // X = 2^16 h + 2^8 m + l with l, m in [-128, 127]: l is X's low byte as a signed value
+                const int lo = (int)(int8_t)(X[j] & 0xFF);
+                const int X1 = (X[j] - lo) >> 8;
+                const int mi = (int)(int8_t)(X1 & 0xFF);
+                const int hi = (X1 - mi) >> 8;
+                ph[j >> 2] |= (uint32_t)(hi & 0xFF) << ((j & 3) * 8);
+                pm[j >> 2] |= (uint32_t)(mi & 0xFF) << ((j & 3) * 8);
+                pl[j >> 2] |= (uint32_t)(lo & 0xFF) << ((j & 3) * 8);
+            }
+            S += sa;
             int8_t* d = a.sl + r * a.H + 8 * v;
             *reinterpret_cast<uint2*>(d) = make_uint2(ph[0], ph[1]);
             *reinterpret_cast<uint2*>(d + plane) = make_uint2(pm[0], pm[1]);
@@ -124,19 +125,22 @@ __global__ void __launch_bounds__(256) router_quant_kernel(RouterQuantArgs a, De
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) emax = max(emax, __shfl_xor_sync(0xffffffffu, emax, off));
         e1 = emax > 0 ? (int)emax : 1;
+        const int q = 148 - e1;                      // in [-106, 147]
+        const int qa = q > 100 ? 100 : q;
+        const float s1 = __uint_as_float((uint32_t)(127 + qa) << 23), s2 = __uint_as_float((uint32_t)(127 + q - qa) << 23);
         for (int v0 = lane; v0 < nv; v0 += 32 * RQ_B) {
             uint4 f[RQ_B];
 #pragma unroll
             for (int b = 0; b < RQ_B; ++b) f[b] = v0 + 32 * b < nv ? src[v0 + 32 * b] : make_uint4(0, 0, 0, 0);
 #pragma unroll
             for (int b = 0; b < RQ_B; ++b)
-                if (v0 + 32 * b < nv) emit(f[b], v0 + 32 * b, e1, S);
+                if (v0 + 32 * b < nv) emit(f[b], v0 + 32 * b, s1, s2, S);
         }
         if (emax == 0xFFu && lane == 0) record_error(ctx.err, MOE_ERANGE);   // an infinity or NaN
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) S += __shfl_xor_sync(0xffffffffu, S, off);
         if (lane == 0) {
-            a.q[r] = 148 - e1;
+            a.q[r] = q;
             a.S[r] = S;
         }
     }
