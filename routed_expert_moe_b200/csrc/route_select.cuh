@@ -18,21 +18,7 @@
 
 namespace moe {
 
-constexpr int TK_MAXJ = 8;        // experts per lane (E <= 256)
-
 // warp arg-max of (value, -index)
-__device__ __forceinline__ void warp_argmax(double& v, int& e) {
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-        const double ov = __shfl_xor_sync(0xffffffffu, v, off);
-        const int oe = __shfl_xor_sync(0xffffffffu, e, off);
-        if (ov > v || (ov == v && oe < e)) {
-            v = ov;
-            e = oe;
-        }
-    }
-}
-
 __device__ __forceinline__ void warp_argmax_i64(long long& v, int& e) {
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {
@@ -105,22 +91,6 @@ __device__ __forceinline__ unsigned long long order_key(double v) {
     const unsigned long long u = (unsigned long long)__double_as_longlong(v + 0.0);
     return (u >> 63) ? ~u : (u | 0x8000000000000000ull);
 }
-__device__ __forceinline__ double key_value(unsigned long long k) {
-    return __longlong_as_double((long long)((k >> 63) ? (k & 0x7fffffffffffffffull) : ~k));
-}
-
-// warp arg-max of (key, -index)
-__device__ __forceinline__ void warp_argmax_key(unsigned long long& k, int& e) {
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-        const unsigned long long ok = __shfl_xor_sync(0xffffffffu, k, off);
-        const int oe = __shfl_xor_sync(0xffffffffu, e, off);
-        if (ok > k || (ok == k && oe < e)) {
-            k = ok;
-            e = oe;
-        }
-    }
-}
 
 // Per-block constants of the bound: the largest ||w_e|| (from the fp32 squared
 // norms Q, inflated by 1 + (H+64) 2^-23 to an upper bound) and the largest
@@ -149,51 +119,65 @@ __device__ __forceinline__ void bound_constants(const double* Q, const float* bi
 // expert whose exact logit could still be in the top K) are appended to the
 // block's list under `slot`.  The ranking compares order-preserving integer
 // keys of l~ + b.
-__device__ __forceinline__ bool rank_certified_eps(const double* Lrow, double eps_star, const float* bias, int E,
-                                                   int K, int lane, int slot, int* out_e, double* out_l,
-                                                   uint8_t* c_tok, uint16_t* c_e, int* n_cand) {
-    const int nj = (E + 31) / 32;
-
-    // the lane's keys, sorted once by (key, -e) descending (empty slots: key 0, below every real key)
-    unsigned long long sk[TK_MAXJ];
-    int se[TK_MAXJ];
+template <int NJ>
+__device__ __forceinline__ bool rank_packed(const double* Lrow, double eps_star, const float* bias, int E, int K,
+                                            int lane, int slot, int* out_e, double* out_l, uint8_t* c_tok,
+                                            uint16_t* c_e, int* n_cand) {
+    auto lval = [&](int e) {
+        double l = Lrow[e];
+        if (bias) l += (double)bias[e];
+        return l;
+    };
+    // Packed keys: the order key of l~ + b with its low 8 bits replaced by 255 - e.  One 64-bit
+    // maximum then ranks by value and breaks ties toward the lower index; two values whose keys
+    // differ only in those 8 bits are within 2^-44 of each other relatively, and the bound below
+    // is widened by 2^-43 max |l~ + b| so that such a pair is never certified.  The exact values
+    // are read back for the gaps and the weights.  Empty slots: key 0, below every real key.
+    unsigned long long pk[NJ];
+    double amax = 0.0;
 #pragma unroll
-    for (int j = 0; j < TK_MAXJ; ++j) {
+    for (int j = 0; j < NJ; ++j) {
         const int e = lane + 32 * j;
-        sk[j] = 0ull;
-        se[j] = e;
-        if (j < nj && e < E) {
-            double l = Lrow[e];
-            if (bias) l += (double)bias[e];
-            sk[j] = order_key(l);
+        pk[j] = 0ull;
+        if (e < E) {
+            const double l = lval(e);
+            amax = fmax(amax, fabs(l));
+            pk[j] = (order_key(l) & ~0xFFull) | (unsigned long long)(255 - e);
         }
     }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) amax = fmax(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    const double eps = eps_star + amax * 0x1p-43;
     auto cx = [&](int i, int j) {   // (i, j) in descending order after the exchange
-        const bool sw = sk[i] < sk[j] || (sk[i] == sk[j] && se[i] > se[j]);
-        const unsigned long long tk = sw ? sk[j] : sk[i];
-        const int te = sw ? se[j] : se[i];
-        sk[j] = sw ? sk[i] : sk[j];
-        se[j] = sw ? se[i] : se[j];
-        sk[i] = tk;
-        se[i] = te;
+        const unsigned long long a = pk[i], b = pk[j];
+        pk[i] = a > b ? a : b;
+        pk[j] = a > b ? b : a;
     };
-    // Batcher's odd-even merge sort of 8
-    cx(0, 1); cx(2, 3); cx(4, 5); cx(6, 7);
-    cx(0, 2); cx(1, 3); cx(4, 6); cx(5, 7);
-    cx(1, 2); cx(5, 6);
-    cx(0, 4); cx(1, 5); cx(2, 6); cx(3, 7);
-    cx(2, 4); cx(3, 5);
-    cx(1, 2); cx(3, 4); cx(5, 6);
+    if constexpr (NJ == 4) {
+        cx(0, 1); cx(2, 3); cx(0, 2); cx(1, 3); cx(1, 2);
+    } else {
+        // Batcher's odd-even merge sort of 8
+        cx(0, 1); cx(2, 3); cx(4, 5); cx(6, 7);
+        cx(0, 2); cx(1, 3); cx(4, 6); cx(5, 7);
+        cx(1, 2); cx(5, 6);
+        cx(0, 4); cx(1, 5); cx(2, 6); cx(3, 7);
+        cx(2, 4); cx(3, 5);
+        cx(1, 2); cx(3, 4); cx(5, 6);
+    }
 
-    // the K+1 best by l~ (ties to the lower index): the best of the lanes' heads, popped
+    // the K+1 best (ties to the lower index): the best of the lanes' heads, popped
     const int nsel = min(K + 1, E);
     double prev = 0.0, lk = 0.0;
     bool certified = true;
     for (int k = 0; k < nsel; ++k) {
-        unsigned long long bk = sk[0];
-        int be = se[0];
-        warp_argmax_key(bk, be);
-        const double bv = key_value(bk);
+        unsigned long long b = pk[0];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const unsigned long long o = __shfl_xor_sync(0xffffffffu, b, off);
+            b = o > b ? o : b;
+        }
+        const int be = 255 - (int)(b & 0xFFull);
+        const double bv = lval(be);
         if (k < K) {
             if (lane == 0) {
                 out_e[k] = be;
@@ -201,29 +185,21 @@ __device__ __forceinline__ bool rank_certified_eps(const double* Lrow, double ep
             }
             lk = bv;
         }
-        if (k > 0 && !(prev - bv > 2.0 * eps_star)) certified = false;
+        if (k > 0 && !(prev - bv > 2.0 * eps)) certified = false;
         prev = bv;
-        if ((be & 31) == lane) {
+        if (pk[0] == b) {   // the lane that held it (keys are unique)
 #pragma unroll
-            for (int j = 0; j + 1 < TK_MAXJ; ++j) {
-                sk[j] = sk[j + 1];
-                se[j] = se[j + 1];
-            }
-            sk[TK_MAXJ - 1] = 0ull;
+            for (int j = 0; j + 1 < NJ; ++j) pk[j] = pk[j + 1];
+            pk[NJ - 1] = 0ull;
         }
     }
     if (!certified) {
         // candidates: every expert that could still be in the exact top K
-        const unsigned long long thr = order_key(lk - 2.0 * eps_star);
+        const unsigned long long thr = order_key(lk - 2.0 * eps);
 #pragma unroll
-        for (int j = 0; j < TK_MAXJ; ++j) {
+        for (int j = 0; j < NJ; ++j) {
             const int e = lane + 32 * j;
-            bool c = false;
-            if (j < nj && e < E) {
-                double l = Lrow[e];
-                if (bias) l += (double)bias[e];
-                c = order_key(l) >= thr;
-            }
+            const bool c = e < E && order_key(lval(e)) >= thr;
             const uint32_t m = __ballot_sync(0xffffffffu, c);
             int base = 0;
             if (lane == 0 && m) base = atomicAdd(n_cand, __popc(m));
@@ -237,6 +213,13 @@ __device__ __forceinline__ bool rank_certified_eps(const double* Lrow, double ep
     }
     __syncwarp();
     return certified;
+}
+
+__device__ __forceinline__ bool rank_certified_eps(const double* Lrow, double eps_star, const float* bias, int E,
+                                                   int K, int lane, int slot, int* out_e, double* out_l,
+                                                   uint8_t* c_tok, uint16_t* c_e, int* n_cand) {
+    return E <= 128 ? rank_packed<4>(Lrow, eps_star, bias, E, K, lane, slot, out_e, out_l, c_tok, c_e, n_cand)
+                    : rank_packed<8>(Lrow, eps_star, bias, E, K, lane, slot, out_e, out_l, c_tok, c_e, n_cand);
 }
 
 // rank_certified_eps with the bound of the fp32-chain logits: k_rel bounds
