@@ -206,13 +206,24 @@ constexpr int FG_KR = 256;                    // K values per stage (128 code by
 constexpr int FG_A_CODES = FG_BM * 128;       // 16 KB
 constexpr int FG_A_SC = FG_BM * 16;           // 2 KB
 constexpr int FG_ATOM = 512;                  // scales of one K block of 64 for 128 rows
-constexpr int FG_TMEM_COLS = 512;
-constexpr int FG_ACC_COLS = 224;              // two accumulators of up to 224 token columns
-constexpr int FG_SFA_COL = 2 * FG_ACC_COLS;   // A scales: 4 K blocks x 4 columns
-constexpr int FG_SFB_COL = FG_SFA_COL + 16;   // B scales: 4 K blocks x 8 columns (two atoms)
-constexpr int FG_BN_MAX = FG_ACC_COLS;        // token rows per schedule entry
+// TMEM layout: two accumulators of ACC token columns, then the A scales (4 K blocks x 4 columns)
+// and the B scales (4 K blocks x 8 columns, two atoms).  Tiles of up to 224 token rows take all
+// 512 columns and one CTA per SM; tiles of up to 64 rows (decode) take 256 columns and two CTAs
+// per SM: the tensor pipe then interleaves two CTAs' chains of scale copies and small MMAs,
+// which one CTA leaves waiting on each other (the up projection at decode: 139 -> 86 us).
+template <bool SMALL>
+struct Fp4Tmem {
+    static constexpr int COLS = SMALL ? 256 : 512;
+    static constexpr int ACC = SMALL ? 64 : 224;
+    static constexpr int SFA = 2 * ACC;
+    static constexpr int SFB = SFA + 16;
+    static constexpr int CTAS = SMALL ? 2 : 1;        // CTAs per SM
+    static constexpr int RING = SMALL ? 100 * 1024 : 216 * 1024;
+    static_assert(SFB + 32 <= COLS, "TMEM columns");
+};
+constexpr int FG_BN_MAX = Fp4Tmem<false>::ACC;          // token rows per schedule entry
+constexpr int FG_BN_SMALL = Fp4Tmem<true>::ACC;         // at most this many: two CTAs per SM
 static_assert(FG_BN_MAX == kFp4MaxTileRows, "NVFP4 tile rows");
-static_assert(FG_SFB_COL + 32 <= FG_TMEM_COLS, "TMEM columns");
 
 struct Fp4Args {
     const int4* sched;
@@ -222,7 +233,7 @@ struct Fp4Args {
     int Kdim;
     int k_stages;            // ceil(K / 256)
     int ns;                  // ring depth
-    int bn;                  // max rows per schedule entry (<= FG_BN_MAX)
+    int bn;                  // max rows per schedule entry (<= the layout's ACC)
     int stage_bytes;
     const float* w_tscale;   // [E]
     float in_tscale;         // x (up) or H (down) tensor scale
@@ -282,9 +293,10 @@ __device__ __forceinline__ void mma_fp4(uint32_t d_tmem, uint64_t a, uint64_t b,
         ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb));
 }
 
-template <bool UP>
-__global__ void __launch_bounds__(FG_THREADS, 1)
+template <bool UP, bool SMALL>
+__global__ void __launch_bounds__(FG_THREADS, Fp4Tmem<SMALL>::CTAS)
     grouped_gemm_fp4_kernel(const __grid_constant__ Fp4Maps maps, Fp4Args g, DevCtx ctx) {
+    using TM = Fp4Tmem<SMALL>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
@@ -317,7 +329,7 @@ __global__ void __launch_bounds__(FG_THREADS, 1)
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 1) tmem_alloc(smem_u32(tmem_holder), FG_TMEM_COLS);
+    if (warp == 1) tmem_alloc(smem_u32(tmem_holder), TM::COLS);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -456,7 +468,7 @@ __global__ void __launch_bounds__(FG_THREADS, 1)
             int acc = 0;
             uint32_t acc_phase = 0;
             bool ok = true, issued = false;
-            const uint32_t sfa = tmem_base + FG_SFA_COL, sfb = tmem_base + FG_SFB_COL;
+            const uint32_t sfa = tmem_base + TM::SFA, sfb = tmem_base + TM::SFB;
             for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
                 const int4 sc = g.sched[u / g.m_blocks];
                 const int n_mma = max(16, (sc.z + 15) & ~15);
@@ -466,7 +478,7 @@ __global__ void __launch_bounds__(FG_THREADS, 1)
                     break;
                 }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * FG_ACC_COLS);
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * TM::ACC);
                 for (int ks = 0; ks < g.k_stages; ++ks) {
                     if (!mbar_wait(smem_u32(&sfready[stage]), phase, ctx, abort_flag)) {
                         ok = false;
@@ -524,7 +536,7 @@ __global__ void __launch_bounds__(FG_THREADS, 1)
             tc_fence_after();
             const int f16 = mb * FG_BM + q * 32 + th * 16;   // first feature of this lane's block
             const float scale = __fmul_rn(g.w_tscale[sc.x], g.in_tscale);
-            const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * FG_ACC_COLS);
+            const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * TM::ACC);
             const int nchunks = (sc.z + 15) / 16;
             for (int c = 0; c < nchunks; ++c) {
                 uint32_t v[16];
@@ -593,7 +605,7 @@ __global__ void __launch_bounds__(FG_THREADS, 1)
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, FG_TMEM_COLS);
+        tmem_dealloc(tmem_base, TM::COLS);
     }
 }
 
@@ -632,10 +644,11 @@ static bool make_map_u8(CUtensorMap* m, const void* base, int64_t rows, int64_t 
 static int ksp_of(int K) { return (K / 16 + 15) / 16 * 16; }
 
 // Ring depth of the NVFP4 kernel for entries of up to bn token rows: as many stages as fit in
-// 216 KB of shared memory, at most 8; then the barriers and the epilogue's 8 KB turn-around tiles.
-static int fp4_stages(int bn, size_t* smem) {
+// the layout's ring budget (216 KB, or 100 KB with two CTAs per SM), at most 8; then the
+// barriers and the epilogue's 8 KB turn-around tiles.
+static int fp4_stages(int bn, bool small, size_t* smem) {
     const Fp4Stage L(bn);
-    int ns = (216 * 1024) / L.bytes;
+    int ns = (small ? Fp4Tmem<true>::RING : Fp4Tmem<false>::RING) / L.bytes;
     if (ns > 8) ns = 8;
     if (ns < 2) ns = 2;
     *smem = 1024 + (size_t)ns * L.bytes + (size_t)(3 * ns + 5) * 8 + 32 + 4 * 16 * 32 * sizeof(float);
@@ -644,10 +657,10 @@ static int fp4_stages(int bn, size_t* smem) {
 
 size_t nvfp4_scale_row_bytes(int K) { return (size_t)ksp_of(K); }
 
-template <bool UP>
+template <bool UP, bool SMALL>
 static cudaError_t launch_fp4(const Fp4Maps& maps, const Fp4Args& g, int grid, size_t smem, cudaStream_t stream,
                               const DevCtx& ctx) {
-    auto kfn = grouped_gemm_fp4_kernel<UP>;
+    auto kfn = grouped_gemm_fp4_kernel<UP, SMALL>;
     cudaError_t err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     return launch_k(kfn, dim3(grid), dim3(FG_THREADS), smem, stream, maps, g, ctx);
@@ -678,9 +691,10 @@ cudaError_t launch_grouped_gemm_fp4(bool up, const uint8_t* w_codes, const uint8
         !make_map_u8(&maps.bs16, a_scales, rows, ksp, ksp, 16, 16, false))
         return cudaErrorInvalidValue;
     if (bn > FG_BN_MAX) return cudaErrorInvalidValue;
+    const bool small = bn <= FG_BN_SMALL;
     size_t smem = 0;
     Fp4Args g;
-    g.ns = fp4_stages(bn, &smem);
+    g.ns = fp4_stages(bn, small, &smem);
     g.stage_bytes = Fp4Stage(bn).bytes;
     g.sched = sched;
     g.n_sched = n_sched;
@@ -696,9 +710,13 @@ cudaError_t launch_grouped_gemm_fp4(bool up, const uint8_t* w_codes, const uint8
     g.out_scale = out_scale;
     g.debug_withhold = debug_withhold;
     const int64_t max_units = (int64_t)max_sched * g.m_blocks;
-    const int grid = (int)(max_units < num_sms ? max_units : num_sms);
-    return up ? launch_fp4<true>(maps, g, grid, smem, stream, ctx)
-              : launch_fp4<false>(maps, g, grid, smem, stream, ctx);
+    const int64_t slots = (int64_t)num_sms * (small ? Fp4Tmem<true>::CTAS : Fp4Tmem<false>::CTAS);
+    const int grid = (int)(max_units < slots ? max_units : slots);
+    if (small)
+        return up ? launch_fp4<true, true>(maps, g, grid, smem, stream, ctx)
+                  : launch_fp4<false, true>(maps, g, grid, smem, stream, ctx);
+    return up ? launch_fp4<true, false>(maps, g, grid, smem, stream, ctx)
+              : launch_fp4<false, false>(maps, g, grid, smem, stream, ctx);
 }
 
 cudaError_t launch_quantize_nvfp4(int64_t n_tensors, int64_t rows, int K, const uint16_t* src, uint8_t* codes,
