@@ -49,9 +49,20 @@ constexpr int FF_THREADS = 192;
 constexpr int FF_BM = 128;
 constexpr int FF_ROW_BYTES = 128;
 constexpr int FF_A_BYTES = FF_BM * FF_ROW_BYTES;
-constexpr int FF_TMEM_COLS = 512;
 constexpr int FF_EPI_WARPS = 4;
 constexpr int FF_UQ = 4;   // unit queue slots (producer -> MMA and epilogue warps)
+
+// TMEM layout: two accumulators of ACC token columns.  Tiles of up to 256 rows take all 512
+// columns and one CTA per SM with a ring of up to 220 KB; tiles of up to 128 rows (decode) take
+// 256 columns, a ring of up to 100 KB and two CTAs per SM, whose two in-order streams of TMA
+// stages keep more bytes landing than one deeper ring (decode FFN 354 -> 350 us).
+template <bool SMALL>
+struct FfnTmem {
+    static constexpr int COLS = SMALL ? 256 : 512;
+    static constexpr int ACC = SMALL ? 128 : 256;
+    static constexpr int CTAS = SMALL ? 2 : 1;
+    static constexpr int RING = SMALL ? 100 * 1024 : 220 * 1024;
+};
 
 struct FfnArgs {
     int* claim;             // unit counter (zero at launch; right after done[]): producers claim units
@@ -108,9 +119,10 @@ __device__ __forceinline__ bool wait_count(const int* p, int target, const DevCt
     }
 }
 
-template <bool FP8>
-__global__ void __launch_bounds__(FF_THREADS, 1)
+template <bool FP8, bool SMALL>
+__global__ void __launch_bounds__(FF_THREADS, FfnTmem<SMALL>::CTAS)
     grouped_ffn_kernel(const __grid_constant__ FfnMaps maps, FfnArgs g, DevCtx ctx) {
+    using TM = FfnTmem<SMALL>;
     constexpr int KEL = FF_ROW_BYTES / (FP8 ? 1 : 2);   // elements of K per stage
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -152,7 +164,7 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 1) tmem_alloc(smem_u32(tmem_holder), FF_TMEM_COLS);
+    if (warp == 1) tmem_alloc(smem_u32(tmem_holder), TM::COLS);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -275,7 +287,7 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
                     break;
                 }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * 256);
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * TM::ACC);
                 for (int ks = 0; ks < k_stages; ++ks) {
                     if (!mbar_wait(smem_u32(&full[stage]), phase, ctx, abort_flag)) {
                         ok = false;
@@ -342,7 +354,7 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
             const int f16 = mb * FF_BM + q * 32 + th * 16;   // first of this lane's 16 features
             float scale = 1.0f;
             if constexpr (FP8) scale = up ? __fmul_rn(g.su[sc.x], g.x_scale) : __fmul_rn(g.sd[sc.x], g.h_scale);
-            const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * 256);
+            const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * TM::ACC);
             const int nchunks = (sc.z + 15) / 16;
             for (int c = 0; c < nchunks; ++c) {
                 uint32_t vv[16];
@@ -417,7 +429,7 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, FF_TMEM_COLS);
+        tmem_dealloc(tmem_base, TM::COLS);
     }
 }
 
@@ -480,7 +492,14 @@ cudaError_t launch_grouped_ffn(bool fp8, const void* w_up, const void* w_down, i
     const int es = fp8 ? 1 : 2;
     g.k_up = (int)(((int64_t)H * es + FF_ROW_BYTES - 1) / FF_ROW_BYTES);
     g.k_down = (int)(((int64_t)F * es + FF_ROW_BYTES - 1) / FF_ROW_BYTES);
-    g.n_stages = plan.n_stages;
+    if (plan.bn > FfnTmem<false>::ACC) return cudaErrorInvalidValue;
+    const bool small = plan.bn <= FfnTmem<true>::ACC;
+    // ring depth for this launch's layout: as many stages as fit in its budget, 2 to 8
+    const int stage_bytes = FF_A_BYTES + plan.bn * FF_ROW_BYTES;
+    int ns = (small ? FfnTmem<true>::RING : FfnTmem<false>::RING) / stage_bytes;
+    if (ns > 8) ns = 8;
+    if (ns < 2) ns = 2;
+    g.n_stages = ns;
     g.b_stage_bytes = plan.bn * FF_ROW_BYTES;
     g.hb = hb;
     g.y = y;
@@ -490,10 +509,15 @@ cudaError_t launch_grouped_ffn(bool fp8, const void* w_up, const void* w_down, i
     g.h_scale = h_scale;
     g.debug_hold = debug_hold;
     const int64_t max_units = (int64_t)plan.max_sched * (g.m_up + g.m_down);
-    const int grid = (int)(max_units < num_sms ? max_units : num_sms);
-    auto kfn = fp8 ? grouped_ffn_kernel<true> : grouped_ffn_kernel<false>;
-    const size_t smem = plan.smem_bytes + 16 + (size_t)FF_EPI_WARPS * 16 * 32 * sizeof(uint16_t) +
-                        2 * FF_UQ * sizeof(uint64_t) + FF_UQ * sizeof(int);
+    const int64_t slots = (int64_t)num_sms * (small ? FfnTmem<true>::CTAS : FfnTmem<false>::CTAS);
+    const int grid = (int)(max_units < slots ? max_units : slots);
+    auto kfn = small ? (fp8 ? grouped_ffn_kernel<true, true> : grouped_ffn_kernel<false, true>)
+                     : (fp8 ? grouped_ffn_kernel<true, false> : grouped_ffn_kernel<false, false>);
+    // ring, its barriers (full, empty, two tfull, two tempty, drain), the abort flag and TMEM
+    // holder, the epilogue's turn-around tiles and the unit queue
+    const size_t smem = 1024 + (size_t)ns * stage_bytes + (size_t)(2 * ns + 5) * 8 + 16 + 16 +
+                        (size_t)FF_EPI_WARPS * 16 * 32 * sizeof(uint16_t) + 2 * FF_UQ * sizeof(uint64_t) +
+                        FF_UQ * sizeof(int);
     cudaError_t err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     return launch_k(kfn, dim3(grid), dim3(FF_THREADS), smem, stream, maps, g, ctx);
