@@ -283,16 +283,20 @@ __global__ void __launch_bounds__(TK_WARPS * 32, 2) router_topk_kernel(RouterTop
 // one launch.  CTA r of the cluster owns experts [r*ceil(E/8), ...), whose
 // router rows are one contiguous block of W_r: two bulk copies bring that
 // block and the group's x rows into shared memory.  A warp handles experts
-// e and e+8 of the slice; each lane takes pairs of 16-byte fragments, which
-// give, per token, a chain of 16 fp32 FMAs from zero, added into an fp64
-// total; the warp then sums its lanes' totals in fp64.  The logits and the
-// squared weight norms go to the leader CTA's shared memory (distributed
-// shared memory); after the cluster barrier the leader's warps run the same
-// certified selection as router_topk_kernel, one token each.
+// e and e+8 of the slice over one half of H (16 warps: 8 expert pairs x 2
+// halves); each lane takes pairs of 16-byte fragments, which give, per token,
+// a chain of 16 fp32 FMAs from zero, added into an fp64 total; the warp sums
+// its lanes' totals in fp64 and the two halves are added in fp64.  The logits
+// and the squared weight norms go to the leader CTA's shared memory
+// (distributed shared memory); after the cluster barrier the leader's warps
+// run the same certified selection as router_topk_kernel, one token each.
 
 constexpr int RS_CLUSTER = 8;
-constexpr int RS_THREADS = 256;
+constexpr int RS_THREADS = 512;
 constexpr int RS_WARPS = RS_THREADS / 32;
+constexpr int RS_PAIRW = 8;                      // warps per half of H (expert pairs in flight)
+constexpr int RS_SPLIT = RS_WARPS / RS_PAIRW;    // halves of H
+static_assert(RS_SPLIT == 2, "the fp64 depth of the bound counts one add of the halves");
 
 struct RouterSmallArgs {
     const uint16_t* x;
@@ -308,12 +312,13 @@ __host__ __device__ constexpr int rs_epc(int E) { return (E + RS_CLUSTER - 1) / 
 __host__ __device__ constexpr size_t rs_align(size_t v) { return (v + 15) & ~size_t(15); }
 
 // dynamic shared memory of one CTA: xs [TB][H] bf16 | ws [epc][H] bf16 | Ls [TB][E] f64 |
-// Qs [E] f64 | Xs [TB] f64 | xred [TB][8] f32 | c_val [TB*E] i64 | c_e [TB*E] u16 |
-// c_tok [TB*E] u8 | n_cand, abort flag | mbarrier
+// Qs [E] f64 | Xs [TB] f64 | xred [TB][RS_WARPS] f32 | Ph [2][epc][TB] f64 | Qh [2][epc] f32 |
+// c_val [TB*E] i64 | c_e [TB*E] u16 | c_tok [TB*E] u8 | n_cand, abort flag | mbarrier
 __host__ __device__ inline size_t rs_smem_bytes(int TB, int H, int E) {
     size_t o = rs_align((size_t)TB * H * 2) + rs_align((size_t)rs_epc(E) * H * 2);
     o += rs_align((size_t)TB * E * 8) + rs_align((size_t)E * 8) + rs_align((size_t)TB * 8);
     o += rs_align((size_t)TB * RS_WARPS * 4);
+    o += rs_align((size_t)RS_SPLIT * rs_epc(E) * TB * 8) + rs_align((size_t)RS_SPLIT * rs_epc(E) * 4);
     o += rs_align((size_t)TB * E * 8) + rs_align((size_t)TB * E * 2) + rs_align((size_t)TB * E) + 16 + 16;
     return o;
 }
@@ -348,6 +353,10 @@ __global__ void __cluster_dims__(RS_CLUSTER, 1, 1) __launch_bounds__(RS_THREADS)
     p += rs_align((size_t)TB * 8);
     float* xred = reinterpret_cast<float*>(p);
     p += rs_align((size_t)TB * RS_WARPS * 4);
+    double* Ph = reinterpret_cast<double*>(p);   // [half][local expert][token] partial logits
+    p += rs_align((size_t)RS_SPLIT * epc * TB * 8);
+    float* Qh = reinterpret_cast<float*>(p);     // [half][local expert] partial squared norms
+    p += rs_align((size_t)RS_SPLIT * epc * 4);
     long long* c_val = reinterpret_cast<long long*>(p);
     p += rs_align((size_t)TB * E * 8);
     uint16_t* c_e = reinterpret_cast<uint16_t*>(p);
@@ -408,8 +417,12 @@ __global__ void __cluster_dims__(RS_CLUSTER, 1, 1) __launch_bounds__(RS_THREADS)
     // 2. this CTA's experts: warp w takes local experts w + 16m and w + 16m + 8
     double* Ls_lead = cluster.map_shared_rank(Ls, 0);
     double* Qs_lead = cluster.map_shared_rank(Qs, 0);
-    for (int l0 = warp; l0 < n_e; l0 += 2 * RS_WARPS) {
-        const int l1 = l0 + RS_WARPS;
+    // warp (pair, half): local experts pair + 16m and pair + 16m + 8, fragments [vs, ve) of H
+    const int pair = warp % RS_PAIRW, half = warp / RS_PAIRW;
+    const int hv_half = (HV + RS_SPLIT - 1) / RS_SPLIT;
+    const int vs = half * hv_half, ve = min(HV, vs + hv_half);
+    for (int l0 = pair; l0 < n_e; l0 += 2 * RS_PAIRW) {
+        const int l1 = l0 + RS_PAIRW;
         const bool has1 = l1 < n_e;
         const uint16_t* w0 = ws + (size_t)l0 * H;
         const uint16_t* w1 = ws + (size_t)(has1 ? l1 : l0) * H;
@@ -417,9 +430,9 @@ __global__ void __cluster_dims__(RS_CLUSTER, 1, 1) __launch_bounds__(RS_THREADS)
 #pragma unroll
         for (int t = 0; t < TB; ++t) acc0[t] = acc1[t] = 0.0;
         float q0 = 0.0f, q1 = 0.0f;
-        for (int v0 = lane; v0 < HV; v0 += 64) {
+        for (int v0 = vs + lane; v0 < ve; v0 += 64) {
             const int v1 = v0 + 32;
-            const bool ok1 = v1 < HV;
+            const bool ok1 = v1 < ve;
             const uint4 z4 = make_uint4(0, 0, 0, 0);
             float a0[16], a1[16];
             {
@@ -475,19 +488,26 @@ __global__ void __cluster_dims__(RS_CLUSTER, 1, 1) __launch_bounds__(RS_THREADS)
             q1 = __fadd_rn(q1, __shfl_xor_sync(0xffffffffu, q1, off));
         }
         if (lane < TB) {
-            // lane t writes token t's two logits (registers indexed at compile time)
+            // lane t parks token t's two partial logits (registers indexed at compile time)
 #pragma unroll
             for (int t = 0; t < TB; ++t)
                 if (t == lane) {
-                    Ls_lead[t * E + e_lo + l0] = acc0[t];
-                    if (has1) Ls_lead[t * E + e_lo + l1] = acc1[t];
+                    Ph[((size_t)half * epc + l0) * TB + t] = acc0[t];
+                    if (has1) Ph[((size_t)half * epc + l1) * TB + t] = acc1[t];
                 }
         }
         if (lane == 0) {
-            Qs_lead[e_lo + l0] = (double)q0;
-            if (has1) Qs_lead[e_lo + l1] = (double)q1;
+            Qh[half * epc + l0] = q0;
+            if (has1) Qh[half * epc + l1] = q1;
         }
     }
+    __syncthreads();
+    // the two halves of each (expert, token) logit, added in fp64, go to the leader
+    for (int i = tid; i < n_e * TB; i += RS_THREADS) {
+        const int l = i / TB, t = i % TB;
+        Ls_lead[t * E + e_lo + l] = Ph[(size_t)l * TB + t] + Ph[((size_t)epc + l) * TB + t];
+    }
+    for (int l = tid; l < n_e; l += RS_THREADS) Qs_lead[e_lo + l] = (double)__fadd_rn(Qh[l], Qh[epc + l]);
     // every CTA's stores to the leader become visible to it here
     cluster.sync();
     if (!leader) return;
@@ -505,8 +525,9 @@ __global__ void __cluster_dims__(RS_CLUSTER, 1, 1) __launch_bounds__(RS_THREADS)
         }
     }
     __syncthreads();
-    // fp32 chains of 16 terms; fp64: the lane's chain sums, then 5 warp levels
-    const double k_rel = router_k_rel(16, (HV + 63) / 64 + 6);
+    // fp32 chains of 16 terms; fp64: the lane's chain sums over its half of H, 5 warp levels,
+    // the add of the two halves (and one spare)
+    const double k_rel = router_k_rel(16, ((HV + RS_SPLIT - 1) / RS_SPLIT + 63) / 64 + 7);
     const bool active = warp < n_tok;
     bool certified = true;
     bool range_bad = false;
