@@ -151,8 +151,13 @@ bool fused_ffn(const moe_dims* d) {
 
 GemmPlan ffn_plan(const moe_dims* d) {
     GemmPlan gp = gemm_plan(d->T, d->K, d->E);
+    // The one-launch FFN takes sparse batches (experts average under 128 rows) in tiles of at
+    // most 128 rows, which run two CTAs per SM: the skewed T=576 batch's FFN 292 -> 283 us
+    // against 224-row tiles (hot experts split into more tiles; their weights re-read from L2).
+    const bool sparse = d->T * d->K < (int64_t)kFfnSparseRows * d->E;
     const int cap = d->expert_dtype == MOE_FP8_B128 ? kB128MaxTileRows
                     : d->expert_dtype == MOE_NVFP4    ? kFp4MaxTileRows
+                    : fused_ffn(d) && sparse          ? kFfnSparseRows
                                                       : 0;
     if (cap > 0 && gp.bn > cap) {
         const int64_t rows = d->T * d->K;

@@ -64,6 +64,8 @@ struct FfnTmem {
     static constexpr int RING = SMALL ? 100 * 1024 : 220 * 1024;
 };
 
+static_assert(FfnTmem<true>::ACC == kFfnSparseRows, "sparse batches' tiles fit the two-CTA layout");
+
 struct FfnArgs {
     int* claim;             // unit counter (zero at launch; right after done[]): producers claim units
     const int4* sched;      // {e, row0, nrows, 0}

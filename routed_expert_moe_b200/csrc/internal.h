@@ -99,6 +99,10 @@ constexpr int kB128MaxTileRows = 128;
 // accumulators of this many columns leave room for the scale factors.
 constexpr int kFp4MaxTileRows = 224;
 
+// Token rows per schedule entry of the one-launch FFN on sparse batches (fewer than this many
+// rows per expert on average): the tile height of its two-CTA-per-SM layout.
+constexpr int kFfnSparseRows = 128;
+
 // Sizes the plans must keep: a plan is passed by value and by reference
 // between files, so a field added in one place shows up as a size change here.
 static_assert(sizeof(RouterPlan) == 40, "RouterPlan layout changed: update every user");
