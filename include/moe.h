@@ -49,7 +49,7 @@ extern "C" {
 typedef enum {
     MOE_OK = 0,
     MOE_EINVAL = 1,        /* invalid argument: null pointer, bad size, misalignment */
-    MOE_EUNSUPPORTED = 2,  /* valid request this build does not support (e.g. not sm_100) */
+    MOE_EUNSUPPORTED = 2,  /* a valid request the library does not support (e.g. not sm_100) */
     MOE_ECUDA = 3,         /* a CUDA runtime call or a launch failed */
     MOE_ETIMEOUT = 4,      /* a bounded wait inside a kernel expired (device error word) */
     MOE_EWORKSPACE = 5,    /* workspace smaller than moe_workspace_size() */
