@@ -75,19 +75,111 @@ def dist_env():
 # --------------------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons, sampled while the timed region runs."""
+    """Clocks and throttle reasons, sampled while the timed region runs.
+
+    Through NVML every 1-2 ms when the bindings load (a decode timed region of 20 steps lasts
+    under 10 ms), in a child process so that the timed loop's thread does not starve it, else
+    through `nvidia-smi -lms 100`.  Samples are stamped with the host's monotonic clock (the
+    same in both processes); `window(t0, t1)` keeps those taken between the timed region's
+    start and end (the bench records both around its synchronised loop), so the line's clocks
+    are those under load.
+    """
+
+    # the child: one line per sample, "t, sm, max, power, reasons, hw_slowdown, hw_thermal,
+    # sw_thermal, sw_power_cap" (the nvidia-smi field order after the time stamp)
+    NVML_CHILD = r"""
+import sys, time, pynvml as nv
+nv.nvmlInit()
+u = sys.argv[1]
+h = nv.nvmlDeviceGetHandleByUUID(u) if u else nv.nvmlDeviceGetHandleByIndex(0)
+bits = [nv.nvmlClocksEventReasonHwSlowdown, nv.nvmlClocksEventReasonHwThermalSlowdown,
+        nv.nvmlClocksEventReasonSwThermalSlowdown, nv.nvmlClocksEventReasonSwPowerCap]
+mx = str(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+print("ready", flush=True)
+n = 0
+pw = "0.0"
+while True:
+    # two queries per sample (the SM clock and the reasons); the power draw every 16th
+    t = time.perf_counter()
+    sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+    r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+    if n % 16 == 0:
+        pw = f"{nv.nvmlDeviceGetPowerUsage(h) / 1000.0:.1f}"
+    n += 1
+    f = ["Active" if r & b else "Not Active" for b in bits]
+    print(", ".join([f"{t:.6f}", str(sm), mx, pw, hex(r)] + f), flush=True)
+    time.sleep(0.001)
+"""
 
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_uuid: str | None):
+    NVML_PERIOD_S = 0.002
+
+    def __init__(self, gpu_uuid: str | None, nvml=None):
         self.uuid = gpu_uuid
         self.proc = None
-        self.lines = []
+        self.lines = []      # (host time, csv line in the nvidia-smi field order)
         self.thread = None
+        self.nvml = nvml
+        self.handle = None
+        self.stop_flag = threading.Event()
+        self.win = None
+        self.stamped = False
+        self.source = "nvidia-smi -lms 100"
+
+    def _nvml_open(self):
+        try:
+            nv = self.nvml
+            if nv is None:
+                import pynvml as nv
+            nv.nvmlInit()
+            h = nv.nvmlDeviceGetHandleByUUID(self.uuid) if self.uuid else nv.nvmlDeviceGetHandleByIndex(0)
+            self.nvml, self.handle = nv, h
+            self.source = "nvml, every 2 ms"
+            return True
+        except Exception:
+            self.nvml = self.handle = None
+            return False
+
+    def _nvml_loop(self):
+        nv, h = self.nvml, self.handle
+        bits = [("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+                ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+                ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+                ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap")]
+        while not self.stop_flag.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+                pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                flags = ["Active" if r & getattr(nv, name) else "Not Active" for _, name in bits]
+                self.lines.append((time.perf_counter(), ", ".join([str(sm), str(mx), f"{pw:.1f}", hex(r)] + flags)))
+            except Exception:
+                return
+            time.sleep(self.NVML_PERIOD_S)
 
     def start(self):
+        if self.nvml is not None and self._nvml_open():   # an injected NVML (tests): a thread
+            self.thread = threading.Thread(target=self._nvml_loop, daemon=True)
+            self.thread.start()
+            return
+        try:
+            self.proc = subprocess.Popen([sys.executable, "-c", self.NVML_CHILD, self.uuid or ""],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            if self.proc.stdout.readline().strip() == "ready":
+                self.source = "nvml child process, ~1 ms apart"
+                self.stamped = True
+                self.thread = threading.Thread(target=self._read, daemon=True)
+                self.thread.start()
+                return
+            self.proc.kill()
+            self.proc.wait(timeout=5)
+        except (OSError, subprocess.TimeoutExpired):
+            pass
+        self.proc = None
         cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
         if self.uuid:
             cmd[1:1] = ["-i", self.uuid]
@@ -101,9 +193,30 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            line = line.strip()
+            if self.stamped:
+                t, _, rest = line.partition(",")
+                try:
+                    self.lines.append((float(t), rest.strip()))
+                except ValueError:
+                    pass
+            else:
+                self.lines.append((time.perf_counter(), line))
+
+    def window(self, t0: float, t1: float):
+        """Keep the summary to samples taken between t0 and t1 (host perf_counter seconds)."""
+        self.win = (t0, t1)
 
     def stop(self):
+        if self.handle is not None:
+            self.stop_flag.set()
+            if self.thread:
+                self.thread.join(timeout=2)
+            try:
+                self.nvml.nvmlShutdown()
+            except Exception:
+                pass
+            return self.summary()
         if not self.proc:
             return None
         self.proc.terminate()
@@ -118,7 +231,16 @@ class ClockSampler:
     def summary(self):
         sm, mx, reasons = [], 0.0, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        lines = self.lines
+        if self.win is not None:
+            inside = [x for x in lines if self.win[0] <= x[0] <= self.win[1]]
+            if inside:
+                lines = inside
+            elif lines:
+                # a region shorter than the sampling period: the sample nearest its middle
+                mid = 0.5 * (self.win[0] + self.win[1])
+                lines = [min(lines, key=lambda x: abs(x[0] - mid))]
+        for _, ln in lines:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 8:
                 continue
@@ -131,9 +253,9 @@ class ClockSampler:
                 if v.lower().startswith("active"):
                     reasons.add(n)
         if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "sampler": self.source}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "sampler": self.source}
 
 
 # --------------------------------------------------------------------------- native arm
@@ -315,11 +437,13 @@ def timed_loop(layer, steps, warmup, barrier):
     barrier()
     torch.cuda.synchronize()
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    timed_loop.window = (time.perf_counter(), None)
     start.record()
     for i in range(steps):
         layer.step(i)
     stop.record()
     torch.cuda.synchronize()
+    timed_loop.window = (timed_loop.window[0], time.perf_counter())
     barrier()
     return start.elapsed_time(stop)
 
@@ -741,6 +865,7 @@ def run_native(args):
     sampler.start()
     time.sleep(0.3)
     ms = timed_loop(layer, args.steps, args.warmup, barrier)
+    sampler.window(*timed_loop.window)
     clocks = sampler.stop()
 
     ms = reduce_max(ms, dist if ws > 1 else None, device)
@@ -885,10 +1010,15 @@ def run_ep(args):
     barrier = lambda: dist.barrier()
     wl = W.WORKLOADS[WORKLOADS[args.workload]]
     layer = EpLayer(wl, device)
-    sampler = ClockSampler(None)
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+    except Exception:
+        uuid = None
+    sampler = ClockSampler(uuid)
     sampler.start()
     time.sleep(0.3)
     ms = timed_loop(layer, args.steps, args.warmup, barrier)
+    sampler.window(*timed_loop.window)
     clocks = sampler.stop()
     ms = reduce_max(ms, dist, device)
     # end to end: this rank's batch from pinned host memory, its output back, every step

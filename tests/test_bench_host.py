@@ -118,3 +118,51 @@ def test_one_launch_ffn_counts_both_projections():
     assert r["algorithmic_bytes_per_launch"] == 2 * 121 * F * H * 2 + rows * (H + F) * 2 + rows * (F + H) * 2
     assert r["algorithmic_flops_per_launch"] == 2 * 2.0 * rows * F * H
     assert bench.stage_view({"up_gemm": 1.0, "down_gemm": 2.0}, False) == {"up_gemm": 1.0, "down_gemm": 2.0}
+
+
+def _line(sm, reasons_active):
+    flags = ["Active" if r else "Not Active" for r in reasons_active]
+    return ", ".join([str(sm), "1965", "700.0", "0x0"] + flags)
+
+
+def test_clock_summary_keeps_the_timed_window():
+    """Only samples taken between the timed region's start and end count: idle samples before
+    the loop (a low clock) must not pull the median down, nor their reasons leak in."""
+    s = bench.ClockSampler(None)
+    s.lines = [(0.0, _line(345, [0, 0, 0, 0])), (1.0, _line(1965, [0, 0, 0, 1])),
+               (2.0, _line(1950, [0, 0, 0, 0])), (3.0, _line(900, [1, 0, 0, 0]))]
+    s.window(0.5, 2.5)
+    c = s.summary()
+    assert c["samples"] == 2 and c["sm_mhz"] == pytest.approx(1957.5) and c["reasons"] == ["sw_power_cap"]
+    s.window(2.9, 2.95)      # shorter than the sampling period: the sample nearest its middle
+    c = s.summary()
+    assert c["samples"] == 1 and c["sm_mhz"] == 900 and c["reasons"] == ["hw_slowdown"]
+
+
+def test_clock_sampler_reads_nvml_every_few_milliseconds():
+    import time
+
+    class FakeNvml:
+        NVML_CLOCK_SM = 1
+        nvmlClocksEventReasonHwSlowdown = 0x8
+        nvmlClocksEventReasonHwThermalSlowdown = 0x40
+        nvmlClocksEventReasonSwThermalSlowdown = 0x20
+        nvmlClocksEventReasonSwPowerCap = 0x4
+
+        def nvmlInit(self): pass
+        def nvmlShutdown(self): pass
+        def nvmlDeviceGetHandleByUUID(self, u): return u
+        def nvmlDeviceGetHandleByIndex(self, i): return i
+        def nvmlDeviceGetClockInfo(self, h, c): return 1965
+        def nvmlDeviceGetMaxClockInfo(self, h, c): return 1965
+        def nvmlDeviceGetPowerUsage(self, h): return 950000
+        def nvmlDeviceGetCurrentClocksEventReasons(self, h): return 0x4
+
+    s = bench.ClockSampler("GPU-0", nvml=FakeNvml())
+    s.start()
+    t0 = time.perf_counter()
+    time.sleep(0.05)
+    s.window(t0, time.perf_counter())
+    c = s.stop()
+    assert c["sampler"].startswith("nvml") and c["samples"] >= 5
+    assert c["sm_mhz"] == 1965 and c["reasons"] == ["sw_power_cap"]
