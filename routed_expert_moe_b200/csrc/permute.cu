@@ -105,7 +105,11 @@ struct PermuteArgs {
     int K;
 };
 
-__global__ void __launch_bounds__(PM_THREADS) permute_kernel(PermuteArgs a, DevCtx ctx) {
+// NT threads (a power of two, 256..1024): the fewest warps that hold the assignments, so that
+// the per-warp count table and its column scans stay short for small batches.
+template <int NT>
+__global__ void __launch_bounds__(NT) permute_kernel(PermuteArgs a, DevCtx ctx) {
+    constexpr int NW = NT / 32;
     pdl_enter();
     extern __shared__ int sm[];
     const int E = a.E;
@@ -113,14 +117,14 @@ __global__ void __launch_bounds__(PM_THREADS) permute_kernel(PermuteArgs a, DevC
     int* base = hist + E;         // [E] next free row of each expert
     int* tot = base + E;          // [E] chunk totals
     int* offs = tot + E;          // [E+1]
-    int* wtab = offs + E + 1;     // [32][E] per-warp counts of the chunk
+    int* wtab = offs + E + 1;     // [NW][E] per-warp counts of the chunk
     const int tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
     const uint32_t lt_mask = (1u << lane) - 1u;
 
-    for (int e = tid; e < E; e += PM_THREADS) hist[e] = 0;
+    for (int e = tid; e < E; e += NT) hist[e] = 0;
     __syncthreads();
     int bad = 0;
-    for (int64_t i = tid; i < a.n; i += PM_THREADS) {
+    for (int64_t i = tid; i < a.n; i += NT) {
         const int e = a.idx[i];
         if (e < 0 || e >= E) {
             bad = 1;
@@ -131,10 +135,10 @@ __global__ void __launch_bounds__(PM_THREADS) permute_kernel(PermuteArgs a, DevC
     if (__syncthreads_or(bad)) {
         if (tid == 0) record_error(ctx.err, MOE_EINDEX);
     }
-    for (int e = tid; e < E; e += PM_THREADS) offs[e] = hist[e];
+    for (int e = tid; e < E; e += NT) offs[e] = hist[e];
     __syncthreads();
     const int total = block_exclusive_scan256(offs, E);
-    for (int e = tid; e < E; e += PM_THREADS) {
+    for (int e = tid; e < E; e += NT) {
         base[e] = offs[e];
         a.offsets[e] = offs[e];
         a.counts[e] = hist[e];
@@ -145,19 +149,19 @@ __global__ void __launch_bounds__(PM_THREADS) permute_kernel(PermuteArgs a, DevC
     }
     __syncthreads();
 
-    for (int64_t c0 = 0; c0 < a.n; c0 += PM_THREADS) {
+    for (int64_t c0 = 0; c0 < a.n; c0 += NT) {
         const int64_t i = c0 + tid;
         int e = i < a.n ? a.idx[i] : -1;
         if (e >= E) e = -1;
-        for (int q = tid; q < 32 * E; q += PM_THREADS) wtab[q] = 0;
+        for (int q = tid; q < NW * E; q += NT) wtab[q] = 0;
         __syncthreads();
         const uint32_t peers = __match_any_sync(0xffffffffu, e);
         const int rank_w = __popc(peers & lt_mask);
         if (e >= 0 && rank_w == 0) wtab[warp * E + e] = __popc(peers);
         __syncthreads();
-        for (int ex = tid; ex < E; ex += PM_THREADS) {
+        for (int ex = tid; ex < E; ex += NT) {
             int run = 0;
-            for (int w = 0; w < 32; ++w) {
+            for (int w = 0; w < NW; ++w) {
                 const int v = wtab[w * E + ex];
                 wtab[w * E + ex] = run;
                 run += v;
@@ -171,7 +175,7 @@ __global__ void __launch_bounds__(PM_THREADS) permute_kernel(PermuteArgs a, DevC
             a.inv_row[i] = r;
         }
         __syncthreads();
-        for (int ex = tid; ex < E; ex += PM_THREADS) base[ex] += tot[ex];
+        for (int ex = tid; ex < E; ex += NT) base[ex] += tot[ex];
         __syncthreads();
     }
     if (a.sched) build_schedule(offs, E, a.bn, hist, a.sched, a.n_sched, a.ns, (int)(a.n / a.K), (int)a.n);
@@ -371,7 +375,9 @@ cudaError_t launch_permute(const int32_t* idx, int64_t n, int K, int E, int32_t*
                            int* scratch, const DevCtx& ctx, cudaStream_t stream) {
     if (n <= kPermuteOneBlockMax) {
         PermuteArgs a{idx, n, E, counts, offsets, perm_src, inv_row, sched, n_sched, bn, ns, K};
-        return launch_k(permute_kernel, dim3(1), dim3(PM_THREADS), permute_smem_bytes(E), stream, a, ctx);
+        if (n <= 256) return launch_k(permute_kernel<256>, dim3(1), dim3(256), permute_smem_bytes(E), stream, a, ctx);
+        if (n <= 512) return launch_k(permute_kernel<512>, dim3(1), dim3(512), permute_smem_bytes(E), stream, a, ctx);
+        return launch_k(permute_kernel<1024>, dim3(1), dim3(1024), permute_smem_bytes(E), stream, a, ctx);
     }
     if (!scratch) return cudaErrorInvalidValue;
     const int G = (int)((n + PM_THREADS - 1) / PM_THREADS);
