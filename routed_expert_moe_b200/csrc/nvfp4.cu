@@ -209,8 +209,8 @@ constexpr int FG_ATOM = 512;                  // scales of one K block of 64 for
 // TMEM layout: two accumulators of ACC token columns, then the A scales (4 K blocks x 4 columns)
 // and the B scales (4 K blocks x 8 columns, two atoms).  Tiles of up to 224 token rows take all
 // 512 columns and one CTA per SM; tiles of up to 64 rows (decode) take 256 columns and two CTAs
-// per SM: the tensor pipe then interleaves two CTAs' chains of scale copies and small MMAs,
-// which one CTA leaves waiting on each other (the up projection at decode: 139 -> 86 us).
+// per SM, so that one CTA's stage hand-offs (TMA, the scale warps' transposition, barrier waits)
+// overlap the other's scale copies and MMAs (the up projection at decode: 139 -> 86 us).
 template <bool SMALL>
 struct Fp4Tmem {
     static constexpr int COLS = SMALL ? 256 : 512;
