@@ -636,15 +636,24 @@ def _fused_entry(wl, stages, touched, peaks, peak_kind, workload):
     rows = T * K
     es = 1 if wl.fp8 else 2
     ms = stages["expert_ffn"]
-    algo = 2 * touched * F * H * es + rows * H * es + rows * F * es + rows * F * es + rows * H * 2
+    if wl.nvfp4:
+        # packed codes (half a byte per value) + one E4M3 block scale per 16 values (rows padded
+        # to 16 bytes): both banks, x's codes in, H's codes out and back in, bf16 Y out
+        ksp = lambda k: (k // 16 + 15) // 16 * 16
+        algo = (touched * F * (H / 2 + ksp(H)) + touched * H * (F / 2 + ksp(F)) + rows * (H / 2 + ksp(H))
+                + 2 * rows * (F / 2 + ksp(F)) + rows * H * 2)
+    else:
+        algo = 2 * touched * F * H * es + rows * H * es + rows * F * es + rows * F * es + rows * H * 2
     flops = 2 * 2.0 * rows * F * H
     gbs = algo / (ms * 1e-3) / 1e9
     hbm_peak = peaks["hbm_gbs"]
     if wl.fp8 and peaks.get("fp8_tflops"):
         tc_peak, src = peaks["fp8_tflops"], peaks["fp8_source"]
     else:
-        tc_peak = peaks["bf16_tflops"] * (2.0 if wl.fp8 else 1.0)
-        src = f"{peak_kind} bf16 burst" + (" x 2 (fp8/bf16 nominal ratio)" if wl.fp8 else "")
+        ratio = 4.0 if wl.nvfp4 else 2.0 if wl.fp8 else 1.0
+        tc_peak = peaks["bf16_tflops"] * ratio
+        src = f"{peak_kind} bf16 burst" + (" x 4 (nvfp4/bf16 nominal ratio)" if wl.nvfp4 else
+                                           " x 2 (fp8/bf16 nominal ratio)" if wl.fp8 else "")
     tflops = flops / (ms * 1e-3) / 1e12
     common = {"kernel": "expert_ffn (up and down projections, one launch)", "ms_per_launch": ms,
               "algorithmic_bytes_per_launch": algo, "algorithmic_flops_per_launch": flops,

@@ -143,10 +143,10 @@ struct ForwardWs {
 // NVFP4 at 224: its accumulators share TMEM with the scale factors),
 // plus the shared expert's entries (ns chunks of T rows, cut into tiles of at
 // most bn).
-// Whether the expert FFN runs as one launch (bf16 or E4M3 experts without a shared expert).
+// Whether the expert FFN runs as one launch (bf16, E4M3 or NVFP4 experts without a shared expert).
 bool fused_ffn(const moe_dims* d) {
     return g_fused_ffn.load() && n_shared(d) == 0 &&
-           (d->expert_dtype == MOE_BF16 || d->expert_dtype == MOE_FP8_E4M3);
+           (d->expert_dtype == MOE_BF16 || d->expert_dtype == MOE_FP8_E4M3 || d->expert_dtype == MOE_NVFP4);
 }
 
 GemmPlan ffn_plan(const moe_dims* d) {
@@ -259,12 +259,25 @@ moe_status run_ffn(const moe_dims* d, const DeviceInfo* dev, const DevCtx& ctx, 
     }
     if (d->expert_dtype == MOE_NVFP4) {
         const int withhold4 = g_debug_withhold.load();
+        const bool fused4 = fused_ffn(d);
         if (marks) stage_mark(3, st);
+        // the NVFP4 codes and block scales of the permuted rows; they also zero the one-launch
+        // FFN's per-entry counters and its claim counter
         cudaError_t e4 = launch_gather_nvfp4(static_cast<const uint16_t*>(x), perm_src, rows, d->K, d->T, d->H,
                                              sc->x_scale, static_cast<uint8_t*>(fw.xp), fw.xp_block, dev->num_sms,
-                                             ctx, st);
+                                             ctx, st, fused4 ? fw.done : nullptr, fused4 ? gp.max_sched + 1 : 0);
         if (e4 != cudaSuccess) return cuda_status(e4);
         if (marks) stage_mark(4, st);
+        if (fused4) {
+            e4 = launch_grouped_ffn_fp4(static_cast<const uint8_t*>(w_up), sc->w_up_block, sc->w_up_scale,
+                                        static_cast<const uint8_t*>(w_down), sc->w_down_block, sc->w_down_scale,
+                                        d->E, d->F, d->H, static_cast<const uint8_t*>(fw.xp), fw.xp_block,
+                                        sc->x_scale, sc->h_scale, static_cast<uint8_t*>(fw.hb), fw.hb_block, y_perm,
+                                        rows, fw.sched, fw.n_sched, gp.bn, gp.max_sched, fw.done, dev->num_sms,
+                                        withhold4, ctx, st);
+            if (marks) stage_mark(5, st);
+            return cuda_status(e4);
+        }
         e4 = launch_grouped_gemm_fp4(true, static_cast<const uint8_t*>(w_up), sc->w_up_block, sc->w_up_scale, d->E,
                                      d->F, d->H, static_cast<const uint8_t*>(fw.xp), fw.xp_block, sc->x_scale,
                                      sc->h_scale, rows, fw.sched, fw.n_sched, gp.bn, gp.max_sched, fw.hb,
@@ -392,7 +405,8 @@ moe_status moe_forward_launches(const moe_dims* d, int32_t* launches) {
     int n = route_launches(d->T, d->H, d->E);
     n += permute_scratch_ints(d->T * d->K, d->E) == 0 ? 1 : 3;   // one block, or histogram + scan + scatter
     // row gather, up and down projections (one launch or two), combine
-    n += 1 + (fused_ffn(d) && !(g_gemm_pair.load() && gemm_plan(d->T, d->K, d->E).bn > 64) ? 1 : 2) + 1;
+    const bool pair = d->expert_dtype != MOE_NVFP4 && g_gemm_pair.load() && gemm_plan(d->T, d->K, d->E).bn > 64;
+    n += 1 + (fused_ffn(d) && !pair ? 1 : 2) + 1;
     *launches = n;
     return MOE_OK;
 }

@@ -122,6 +122,38 @@ __device__ __forceinline__ void pdl_enter() {
     asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
+// Cross-CTA counters (the one-launch FFNs' per-entry reports): acquire loads, release adds, the
+// async-proxy fence that orders generic stores before later TMA reads, and a bounded wait.
+__device__ __forceinline__ int ld_acquire(const int* p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void red_release_add(int* p, int v) {
+    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Bounded wait until *p >= target (acquire).  Gives up on the time limit or the block's abort flag.
+__device__ __forceinline__ bool wait_count(const int* p, int target, const DevCtx& ctx, volatile int* abort) {
+    if (ld_acquire(p) >= target) return true;
+    const uint64_t t0 = globaltimer();
+    while (true) {
+        __nanosleep(64);
+        if (ld_acquire(p) >= target) return true;
+        if (*abort) return false;
+        if (globaltimer() - t0 > ctx.timeout_ns) {
+            record_error(ctx.err, MOE_ETIMEOUT);
+            *abort = 1;
+            return false;
+        }
+    }
+}
+
 // Untiled bulk copy from global memory into this CTA's shared memory,
 // completing on `bar` (no multicast).  dst, src and bytes: multiples of 16.
 __device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {

@@ -71,7 +71,13 @@ cudaError_t launch_quantize_nvfp4(int64_t n_tensors, int64_t rows, int K, const 
                                   uint8_t* bscale, float* tscale, int num_sms, cudaStream_t stream);
 cudaError_t launch_gather_nvfp4(const uint16_t* x, const int32_t* perm_src, int64_t rows, int K, int64_t T, int H,
                                 float s_t, uint8_t* codes, uint8_t* bscale, int num_sms, const DevCtx& ctx,
-                                cudaStream_t stream);
+                                cudaStream_t stream, int* zero = nullptr, int64_t n_zero = 0);
+cudaError_t launch_grouped_ffn_fp4(const uint8_t* wu_codes, const uint8_t* wu_scales, const float* wu_tscale,
+                                   const uint8_t* wd_codes, const uint8_t* wd_scales, const float* wd_tscale, int E,
+                                   int F, int H, const uint8_t* x_codes, const uint8_t* x_scales, float x_tscale,
+                                   float h_tscale, uint8_t* hb, uint8_t* hb_block, void* y, int64_t rows,
+                                   const int4* sched, const int* n_sched, int bn, int max_sched, int* done,
+                                   int num_sms, int debug_hold, const DevCtx& ctx, cudaStream_t stream);
 size_t nvfp4_scale_row_bytes(int K);
 cudaError_t launch_grouped_gemm_b128(bool up, const uint8_t* W, const float* w_scale, int E, int Nout, int Kdim,
                                      const uint8_t* act, int64_t rows, const int4* sched, const int* n_sched, int bn,

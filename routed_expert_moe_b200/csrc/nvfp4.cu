@@ -144,8 +144,11 @@ __global__ void __launch_bounds__(256) nvfp4_gather_kernel(const uint16_t* __res
                                                            const int32_t* __restrict__ perm_src, int64_t rows,
                                                            int K, int64_t T, int H, float s_t,
                                                            uint8_t* __restrict__ codes, uint8_t* __restrict__ bscale,
-                                                           DevCtx ctx) {
+                                                           int* zero, int64_t n_zero, DevCtx ctx) {
     pdl_enter();
+    // counters of the kernel that follows (the one-launch NVFP4 FFN), zero before it starts
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_zero; i += (int64_t)gridDim.x * blockDim.x)
+        zero[i] = 0;
     const int lane = threadIdx.x % 32;
     const int nb = H / 16, ksp = (nb + 15) / 16 * 16;
     const int64_t warps = (int64_t)gridDim.x * (blockDim.x / 32);
@@ -609,6 +612,452 @@ __global__ void __launch_bounds__(FG_THREADS, Fp4Tmem<SMALL>::CTAS)
     }
 }
 
+// ----------------------------------------------------------------------------- one-launch FFN
+
+// Both NVFP4 projections in one persistent launch, as the bf16 one-launch FFN (grouped_ffn.cu)
+// does it: every up unit (schedule entry x 128-row block of F), then every down unit (entry x
+// block of H), claimed in that order from a global counter by each CTA's producer and passed to
+// the MMA thread, the scale warps and the epilogue warps through a small queue in shared
+// memory.  An up unit's epilogue warps store their rows of H (codes and block scales), fence
+// them for the async proxy and each add 1 to done[entry] with release semantics; the producer
+// of a down unit waits (bounded) until done[entry] reaches 4 x (blocks of F) before it loads
+// the entry's H.  Units are claimed in list order and processed in claim order, so every up
+// unit a down unit waits for belongs to a running CTA that needs nothing else to finish it.
+constexpr int FF4_UQ = 4;   // unit queue slots
+
+struct Fp4FfnArgs {
+    int* claim;              // unit counter (zero at launch; right after done[])
+    int* done;               // [max_sched] up epilogue warps finished per entry (zero at launch)
+    const int4* sched;
+    const int* n_sched;
+    int m_up, m_down;        // 128-row blocks of F and of H
+    int F, H;
+    int k_up, k_down;        // 256-value K stages of H and of F
+    int ns;                  // ring depth
+    int bn;                  // max rows per schedule entry (<= the layout's ACC)
+    const float* wu_tscale;  // [E]
+    const float* wd_tscale;  // [E]
+    float x_tscale, h_tscale;
+    uint8_t* hb;             // H codes [rows][F/2]
+    uint8_t* hb_block;       // H block scales [rows][ksp(F)]
+    void* y;                 // bf16 [rows][H]
+    int debug_hold;          // 1: the list's first up unit never reports its rows (a wait must expire)
+};
+
+struct Fp4FfnMaps {
+    Fp4Maps up, down;
+};
+
+struct Fp4Unit {
+    bool up;
+    int s, mb;               // schedule entry, 128-row block of the projection's outputs
+    int Nout, Kdim, k_stages;
+};
+
+__device__ __forceinline__ Fp4Unit fp4_unit(const Fp4FfnArgs& g, int u, int n_up) {
+    Fp4Unit r;
+    r.up = u < n_up;
+    const int v = r.up ? u : u - n_up;
+    const int m = r.up ? g.m_up : g.m_down;
+    r.s = v / m;
+    r.mb = v % m;
+    r.Nout = r.up ? g.F : g.H;
+    r.Kdim = r.up ? g.H : g.F;
+    r.k_stages = r.up ? g.k_up : g.k_down;
+    return r;
+}
+
+template <bool SMALL>
+__global__ void __launch_bounds__(FG_THREADS, Fp4Tmem<SMALL>::CTAS)
+    grouped_ffn_fp4_kernel(const __grid_constant__ Fp4FfnMaps maps, Fp4FfnArgs g, DevCtx ctx) {
+    using TM = Fp4Tmem<SMALL>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    const int NS = g.ns;
+    const Fp4Stage L(g.bn);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)NS * L.bytes);
+    uint64_t* full = bars;
+    uint64_t* sfready = full + NS;
+    uint64_t* empty = sfready + NS;
+    uint64_t* tfull = empty + NS;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* drain = tempty + 2;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(drain + 1);
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1) + 1;
+    float* tbuf = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(tmem_holder + 1) + 15) &
+                                           ~static_cast<uintptr_t>(15));   // 4 x (16 x 32) fp32
+    // the unit queue: the units this block claimed, in claim order
+    uint64_t* uq_full = reinterpret_cast<uint64_t*>(tbuf + 4 * 16 * 32);
+    uint64_t* uq_empty = uq_full + FF4_UQ;
+    volatile int* uq = reinterpret_cast<volatile int*>(uq_empty + FF4_UQ);
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(smem_u32(&full[s]), 1);
+            mbar_init(smem_u32(&sfready[s]), 128);
+            mbar_init(smem_u32(&empty[s]), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(smem_u32(&tfull[a]), 1);
+            mbar_init(smem_u32(&tempty[a]), 128);
+        }
+        mbar_init(smem_u32(drain), 1);
+        for (int q = 0; q < FF4_UQ; ++q) {
+            mbar_init(smem_u32(&uq_full[q]), 1);
+            mbar_init(smem_u32(&uq_empty[q]), 1 + 4 + 4);   // the MMA thread, 4 epilogue and 4 scale warps
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) tmem_alloc(smem_u32(tmem_holder), TM::COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+    pdl_enter();
+
+    const int n_sched = *g.n_sched;
+    const int n_up = n_sched * g.m_up;
+    const int n_units = n_up + n_sched * g.m_down;
+    const int up_target = 4 * g.m_up;   // reports of one entry's up units
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- producer
+        if (lane == 0) {
+            const uint64_t pol_w = l2_policy_evict_first();
+            const uint64_t pol_x = l2_policy_evict_last();
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            int qs = 0;
+            uint32_t qph = 0;
+            int claim = atomicAdd(g.claim, 1);
+            while (ok) {
+                const int u = claim < n_units ? claim : -1;
+                if (!mbar_wait(smem_u32(&uq_empty[qs]), qph ^ 1u, ctx, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                uq[qs] = u;
+                mbar_arrive(smem_u32(&uq_full[qs]));
+                if (++qs == FF4_UQ) {
+                    qs = 0;
+                    qph ^= 1u;
+                }
+                if (u < 0) break;
+                claim = atomicAdd(g.claim, 1);   // the next unit, claimed while this one loads
+                const Fp4Unit un = fp4_unit(g, u, n_up);
+                const Fp4Maps& mp = un.up ? maps.up : maps.down;
+                const int4 sc = g.sched[un.s];
+                const bool a_full = un.Nout - un.mb * FG_BM > 64;
+                const int n16 = (sc.z + 15) / 16;
+                const int n128 = n16 / 8, n64 = (n16 % 8) / 4, r16 = n16 % 4;
+                const int arows = a_full ? 128 : 64;
+                const uint32_t bytes = (uint32_t)(arows * (128 + 16) + n16 * 16 * (128 + 16));
+                const int a_y = sc.x * un.Nout + un.mb * FG_BM;
+                if (!un.up) {
+                    // the rows of H this unit reads are written by the up units of its entry
+                    if (!wait_count(g.done + un.s, up_target, ctx, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    fence_proxy_async_global();
+                }
+                for (int ks = 0; ks < un.k_stages; ++ks) {
+                    if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, ctx, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t fb = smem_u32(&full[stage]);
+                    mbar_arrive_expect_tx(fb, bytes);
+                    const uint32_t st = smem_u32(smem + (size_t)stage * L.bytes);
+                    const uint32_t b_c = st + L.b_codes, a_s = st + L.a_sc, b_s = st + L.b_sc;
+                    tma_load_2d(st, a_full ? &mp.a128 : &mp.a64, fb, ks * 128, a_y, pol_w);
+                    tma_load_2d(a_s, a_full ? &mp.as128 : &mp.as64, fb, ks * 16, a_y, pol_w);
+                    int row = 0;
+                    for (int j = 0; j < n128; ++j, row += 128) {
+                        tma_load_2d(b_c + row * 128, &mp.b128, fb, ks * 128, sc.y + row, pol_x);
+                        tma_load_2d(b_s + row * 16, &mp.bs128, fb, ks * 16, sc.y + row, pol_x);
+                    }
+                    for (int j = 0; j < n64; ++j, row += 64) {
+                        tma_load_2d(b_c + row * 128, &mp.b64, fb, ks * 128, sc.y + row, pol_x);
+                        tma_load_2d(b_s + row * 16, &mp.bs64, fb, ks * 16, sc.y + row, pol_x);
+                    }
+                    for (int j = 0; j < r16; ++j, row += 16) {
+                        tma_load_2d(b_c + row * 128, &mp.b16, fb, ks * 128, sc.y + row, pol_x);
+                        tma_load_2d(b_s + row * 16, &mp.bs16, fb, ks * 16, sc.y + row, pol_x);
+                    }
+                    if (++stage == NS) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                // let loads already in flight land before the block exits
+                const uint64_t t0 = globaltimer();
+                while (globaltimer() - t0 < 200000ull) __nanosleep(1000);
+            }
+        }
+    } else if (warp >= 6) {
+        // ---------------------------------------------------------------- scale warps
+        // Thread i moves weight row i's 16 scales (four per K block) and token rows i and
+        // i + 128 into the stage's atoms; rows past the tile's rows get zero scales.
+        const int i = threadIdx.x - 192;
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        int qs = 0;
+        uint32_t qph = 0;
+        // Every lane waits on the barrier itself (it then sees the TMA's bytes) and the warp
+        // votes, so that a lane that gave up alone cannot split its warp's control flow.
+        auto wait_all = [&](uint32_t bar, uint32_t parity) {
+            return __all_sync(0xffffffffu, mbar_wait(bar, parity, ctx, abort_flag)) != 0;
+        };
+        while (ok) {
+            if (!wait_all(smem_u32(&uq_full[qs]), qph)) break;
+            const int u = uq[qs];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&uq_empty[qs]));
+            if (++qs == FF4_UQ) {
+                qs = 0;
+                qph ^= 1u;
+            }
+            if (u < 0) break;
+            const Fp4Unit un = fp4_unit(g, u, n_up);
+            const int4 sc = g.sched[un.s];
+            const int arows = un.Nout - un.mb * FG_BM > 64 ? 128 : 64;
+            const int nrows = (sc.z + 15) / 16 * 16;
+            const int nbk = un.Kdim / 16;   // scale blocks along K; the rest of a padded scale row is masked
+            for (int ks = 0; ks < un.k_stages; ++ks) {
+                if (!wait_all(smem_u32(&full[stage]), phase)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t* st = smem + (size_t)stage * L.bytes;
+                const int valid = min(16, max(0, nbk - ks * 16));
+                uint4 km;
+                km.x = valid >= 4 ? 0xFFFFFFFFu : (valid <= 0 ? 0u : (0xFFFFFFFFu >> (8 * (4 - valid))));
+                km.y = valid >= 8 ? 0xFFFFFFFFu : (valid <= 4 ? 0u : (0xFFFFFFFFu >> (8 * (8 - valid))));
+                km.z = valid >= 12 ? 0xFFFFFFFFu : (valid <= 8 ? 0u : (0xFFFFFFFFu >> (8 * (12 - valid))));
+                km.w = valid >= 16 ? 0xFFFFFFFFu : (valid <= 12 ? 0u : (0xFFFFFFFFu >> (8 * (16 - valid))));
+                {
+                    uint4 v = i < arows ? *reinterpret_cast<const uint4*>(st + L.a_sc + 16 * i)
+                                        : make_uint4(0u, 0u, 0u, 0u);
+                    v.x &= km.x;
+                    v.y &= km.y;
+                    v.z &= km.z;
+                    v.w &= km.w;
+                    uint8_t* at = st + L.a_atoms + 16 * (i % 32) + 4 * (i / 32);
+                    *reinterpret_cast<uint32_t*>(at) = v.x;
+                    *reinterpret_cast<uint32_t*>(at + FG_ATOM) = v.y;
+                    *reinterpret_cast<uint32_t*>(at + 2 * FG_ATOM) = v.z;
+                    *reinterpret_cast<uint32_t*>(at + 3 * FG_ATOM) = v.w;
+                }
+                for (int n = i; n < L.nbat * 128; n += 128) {
+                    uint4 v = n < nrows ? *reinterpret_cast<const uint4*>(st + L.b_sc + 16 * n)
+                                        : make_uint4(0u, 0u, 0u, 0u);
+                    v.x &= km.x;
+                    v.y &= km.y;
+                    v.z &= km.z;
+                    v.w &= km.w;
+                    uint8_t* at = st + L.b_atoms + (n / 128) * FG_ATOM + 16 * (n % 32) + 4 * ((n / 32) % 4);
+                    const int kstep = L.nbat * FG_ATOM;
+                    *reinterpret_cast<uint32_t*>(at) = v.x;
+                    *reinterpret_cast<uint32_t*>(at + kstep) = v.y;
+                    *reinterpret_cast<uint32_t*>(at + 2 * kstep) = v.z;
+                    *reinterpret_cast<uint32_t*>(at + 3 * kstep) = v.w;
+                }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                mbar_arrive(smem_u32(&sfready[stage]));
+                if (++stage == NS) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true, issued = false;
+            int qs = 0;
+            uint32_t qph = 0;
+            const uint32_t sfa = tmem_base + TM::SFA, sfb = tmem_base + TM::SFB;
+            while (ok) {
+                if (!mbar_wait(smem_u32(&uq_full[qs]), qph, ctx, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                const int u = uq[qs];
+                mbar_arrive(smem_u32(&uq_empty[qs]));
+                if (++qs == FF4_UQ) {
+                    qs = 0;
+                    qph ^= 1u;
+                }
+                if (u < 0) break;
+                const Fp4Unit un = fp4_unit(g, u, n_up);
+                const int4 sc = g.sched[un.s];
+                const int n_mma = max(16, (sc.z + 15) & ~15);
+                const uint32_t idesc = fp4_idesc(FG_BM, n_mma);
+                if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1u, ctx, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * TM::ACC);
+                for (int ks = 0; ks < un.k_stages; ++ks) {
+                    if (!mbar_wait(smem_u32(&sfready[stage]), phase, ctx, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t st = smem_u32(smem + (size_t)stage * L.bytes);
+                    const int left = un.Kdim - ks * FG_KR;
+                    const int nk = left >= FG_KR ? 4 : (left + 63) / 64;
+                    for (int kk = 0; kk < nk; ++kk) {
+                        tmem_cp_atom(sfa + 4 * kk, atom_desc(st + L.a_atoms + kk * FG_ATOM));
+                        for (int j = 0; j < L.nbat; ++j)
+                            tmem_cp_atom(sfb + 8 * kk + 4 * j, atom_desc(st + L.b_atoms + (kk * L.nbat + j) * FG_ATOM));
+                    }
+                    for (int kk = 0; kk < nk; ++kk)
+                        mma_fp4(d_tmem, sw128_desc(st + kk * 32), sw128_desc(st + L.b_codes + kk * 32), idesc,
+                                sfa + 4 * kk, sfb + 8 * kk, (ks | kk) != 0 ? 1u : 0u);
+                    issued = true;
+                    mma_commit(smem_u32(&empty[stage]));
+                    if (++stage == NS) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                mma_commit(smem_u32(&tfull[acc]));
+                if (++acc == 2) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
+            }
+            if (!ok && issued) {
+                mma_commit(smem_u32(drain));
+                mbar_wait_drain(smem_u32(drain), 0, ctx.timeout_ns);
+            }
+        }
+    } else {
+        // ---------------------------------------------------------------- epilogue (warps 2..5)
+        // As in grouped_gemm_fp4_kernel: a warp reads 32 features x 16 token columns from TMEM
+        // and turns the tile around in shared memory, so that a lane holds one 16-feature block
+        // of one token.  Up units quantise H to NVFP4 and report their rows; down units store Y.
+        const int q = warp & 3;
+        float* tb = tbuf + (warp - 2) * (16 * 32);
+        const int tj = lane & 15, th = lane >> 4;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        int qs = 0;
+        uint32_t qph = 0;
+        const int fsp = (g.F / 16 + 15) / 16 * 16;   // padded block-scale row of the H tensor
+        const float r6 = __frcp_rn(6.0f), rts = __frcp_rn(g.h_tscale);   // quotients via nv_div
+        while (true) {
+            if (!mbar_wait_warp(smem_u32(&uq_full[qs]), qph, ctx, abort_flag)) break;
+            const int u = uq[qs];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&uq_empty[qs]));
+            if (++qs == FF4_UQ) {
+                qs = 0;
+                qph ^= 1u;
+            }
+            if (u < 0) break;
+            const Fp4Unit un = fp4_unit(g, u, n_up);
+            const int4 sc = g.sched[un.s];
+            if (!mbar_wait_warp(smem_u32(&tfull[acc]), acc_phase, ctx, abort_flag)) break;
+            tc_fence_after();
+            const int f16 = un.mb * FG_BM + q * 32 + th * 16;   // first feature of this lane's block
+            const float scale = un.up ? __fmul_rn(g.wu_tscale[sc.x], g.x_tscale)
+                                      : __fmul_rn(g.wd_tscale[sc.x], g.h_tscale);
+            const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * TM::ACC);
+            const int nchunks = (sc.z + 15) / 16;
+            for (int c = 0; c < nchunks; ++c) {
+                uint32_t v[16];
+                tmem_ld16(t_row + (uint32_t)(c * 16), v);
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    float z = __fmul_rn(__uint_as_float(v[j]), scale);
+                    if (un.up) z = z > 0.0f ? __fmul_rn(z, z) : 0.0f;   // H = relu(z)^2
+                    tb[j * 32 + (((lane >> 2) ^ (j & 7)) << 2) + (lane & 3)] = z;
+                }
+                __syncwarp();
+                float a[16];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float4 t4 = *reinterpret_cast<const float4*>(tb + tj * 32 + (((4 * th + k) ^ (tj & 7)) << 2));
+                    a[4 * k] = t4.x;
+                    a[4 * k + 1] = t4.y;
+                    a[4 * k + 2] = t4.z;
+                    a[4 * k + 3] = t4.w;
+                }
+                __syncwarp();
+                const int r = c * 16 + tj;
+                if (r < sc.z && f16 < un.Nout) {
+                    const int64_t row = sc.y + r;
+                    if (un.up) {
+                        // one block of 16 features, quantised with the static tensor scale s_h
+                        float amax = 0.0f;
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) amax = fmaxf(amax, a[i]);
+                        const uint32_t scode = e4m3_code(nv_div(nv_div(amax, 6.0f, r6), g.h_tscale, rts));
+                        const float e = __fmul_rn(e4m3_value(scode), g.h_tscale);
+                        uint32_t packed[2] = {0u, 0u};
+                        if (e != 0.0f) {
+                            const float y = __frcp_rn(e);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i)
+                                packed[i / 4] |= e2m1_pack(nv_div(a[2 * i], e, y), nv_div(a[2 * i + 1], e, y))
+                                                 << (8 * (i % 4));
+                        }
+                        *reinterpret_cast<uint2*>(g.hb + row * (g.F / 2) + f16 / 2) = make_uint2(packed[0], packed[1]);
+                        g.hb_block[row * fsp + f16 / 16] = (uint8_t)scode;
+                    } else {
+                        uint32_t w8[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const __nv_bfloat162 p2 = __floats2bfloat162_rn(a[2 * i], a[2 * i + 1]);
+                            w8[i] = *reinterpret_cast<const uint32_t*>(&p2);
+                        }
+                        uint4* d4 = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.y) + row * g.H + f16);
+                        d4[0] = make_uint4(w8[0], w8[1], w8[2], w8[3]);
+                        d4[1] = make_uint4(w8[4], w8[5], w8[6], w8[7]);
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(smem_u32(&tempty[acc]));
+            if (un.up) {
+                // this warp's rows of H are complete: every lane orders its stores for the async
+                // proxy (the TMA loads of H), the warp barrier orders them before lane 0's release
+                fence_proxy_async_global();
+                __syncwarp();
+                const bool hold = g.debug_hold && u == 0;
+                if (lane == 0 && !hold) red_release_add(g.done + un.s, 1);
+            }
+            if (++acc == 2) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, TM::COLS);
+    }
+}
+
 // ----------------------------------------------------------------------------- host
 
 typedef CUresult (*EncodeTiledFn4)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -643,6 +1092,24 @@ static bool make_map_u8(CUtensorMap* m, const void* base, int64_t rows, int64_t 
 
 static int ksp_of(int K) { return (K / 16 + 15) / 16 * 16; }
 
+// The maps of one projection: weight codes [E*Nout][K/2] and block scales [E*Nout][KSP(K)],
+// activation codes [rows][K/2] and block scales [rows][KSP(K)].
+static bool make_fp4_maps(Fp4Maps* m, const uint8_t* w_codes, const uint8_t* w_scales, int E, int Nout, int Kdim,
+                          const uint8_t* a_codes, const uint8_t* a_scales, int64_t rows) {
+    const int ksp = ksp_of(Kdim);
+    const int64_t wrows = (int64_t)E * Nout;
+    return make_map_u8(&m->a128, w_codes, wrows, Kdim / 2, Kdim / 2, 128, 128, true) &&
+           make_map_u8(&m->a64, w_codes, wrows, Kdim / 2, Kdim / 2, 128, 64, true) &&
+           make_map_u8(&m->as128, w_scales, wrows, ksp, ksp, 16, 128, false) &&
+           make_map_u8(&m->as64, w_scales, wrows, ksp, ksp, 16, 64, false) &&
+           make_map_u8(&m->b128, a_codes, rows, Kdim / 2, Kdim / 2, 128, 128, true) &&
+           make_map_u8(&m->b64, a_codes, rows, Kdim / 2, Kdim / 2, 128, 64, true) &&
+           make_map_u8(&m->b16, a_codes, rows, Kdim / 2, Kdim / 2, 128, 16, true) &&
+           make_map_u8(&m->bs128, a_scales, rows, ksp, ksp, 16, 128, false) &&
+           make_map_u8(&m->bs64, a_scales, rows, ksp, ksp, 16, 64, false) &&
+           make_map_u8(&m->bs16, a_scales, rows, ksp, ksp, 16, 16, false);
+}
+
 // Ring depth of the NVFP4 kernel for entries of up to bn token rows: as many stages as fit in
 // the layout's ring budget (216 KB, or 100 KB with two CTAs per SM), at most 8; then the
 // barriers and the epilogue's 8 KB turn-around tiles.
@@ -676,19 +1143,8 @@ cudaError_t launch_grouped_gemm_fp4(bool up, const uint8_t* w_codes, const uint8
                                     const int* n_sched, int bn, int max_sched, void* out, uint8_t* out_scale,
                                     int num_sms, int debug_withhold, const DevCtx& ctx, cudaStream_t stream) {
     if (rows == 0) return cudaSuccess;
-    const int ksp = ksp_of(Kdim);
-    const int64_t wrows = (int64_t)E * Nout;
     Fp4Maps maps;
-    if (!make_map_u8(&maps.a128, w_codes, wrows, Kdim / 2, Kdim / 2, 128, 128, true) ||
-        !make_map_u8(&maps.a64, w_codes, wrows, Kdim / 2, Kdim / 2, 128, 64, true) ||
-        !make_map_u8(&maps.as128, w_scales, wrows, ksp, ksp, 16, 128, false) ||
-        !make_map_u8(&maps.as64, w_scales, wrows, ksp, ksp, 16, 64, false) ||
-        !make_map_u8(&maps.b128, a_codes, rows, Kdim / 2, Kdim / 2, 128, 128, true) ||
-        !make_map_u8(&maps.b64, a_codes, rows, Kdim / 2, Kdim / 2, 128, 64, true) ||
-        !make_map_u8(&maps.b16, a_codes, rows, Kdim / 2, Kdim / 2, 128, 16, true) ||
-        !make_map_u8(&maps.bs128, a_scales, rows, ksp, ksp, 16, 128, false) ||
-        !make_map_u8(&maps.bs64, a_scales, rows, ksp, ksp, 16, 64, false) ||
-        !make_map_u8(&maps.bs16, a_scales, rows, ksp, ksp, 16, 16, false))
+    if (!make_fp4_maps(&maps, w_codes, w_scales, E, Nout, Kdim, a_codes, a_scales, rows))
         return cudaErrorInvalidValue;
     if (bn > FG_BN_MAX) return cudaErrorInvalidValue;
     const bool small = bn <= FG_BN_SMALL;
@@ -719,6 +1175,54 @@ cudaError_t launch_grouped_gemm_fp4(bool up, const uint8_t* w_codes, const uint8
               : launch_fp4<false, false>(maps, g, grid, smem, stream, ctx);
 }
 
+// Both NVFP4 projections in one launch.  done: max_sched + 1 ints (the per-entry counters, then
+// the unit claim counter), zero before the launch.  The H codes and block scales go to hb and
+// hb_block; Y (bf16 [rows][H]) to y.
+cudaError_t launch_grouped_ffn_fp4(const uint8_t* wu_codes, const uint8_t* wu_scales, const float* wu_tscale,
+                                   const uint8_t* wd_codes, const uint8_t* wd_scales, const float* wd_tscale, int E,
+                                   int F, int H, const uint8_t* x_codes, const uint8_t* x_scales, float x_tscale,
+                                   float h_tscale, uint8_t* hb, uint8_t* hb_block, void* y, int64_t rows,
+                                   const int4* sched, const int* n_sched, int bn, int max_sched, int* done,
+                                   int num_sms, int debug_hold, const DevCtx& ctx, cudaStream_t stream) {
+    if (rows == 0) return cudaSuccess;
+    Fp4FfnMaps maps;
+    if (!make_fp4_maps(&maps.up, wu_codes, wu_scales, E, F, H, x_codes, x_scales, rows) ||
+        !make_fp4_maps(&maps.down, wd_codes, wd_scales, E, H, F, hb, hb_block, rows))
+        return cudaErrorInvalidValue;
+    if (bn > FG_BN_MAX) return cudaErrorInvalidValue;
+    const bool small = bn <= FG_BN_SMALL;
+    size_t smem = 0;
+    Fp4FfnArgs g;
+    g.ns = fp4_stages(bn, small, &smem);
+    smem += 16 + 2 * FF4_UQ * sizeof(uint64_t) + FF4_UQ * sizeof(int);   // the unit queue (after the tiles)
+    g.bn = bn;
+    g.done = done;
+    g.claim = done + max_sched;
+    g.sched = sched;
+    g.n_sched = n_sched;
+    g.m_up = (F + FG_BM - 1) / FG_BM;
+    g.m_down = (H + FG_BM - 1) / FG_BM;
+    g.F = F;
+    g.H = H;
+    g.k_up = (H + FG_KR - 1) / FG_KR;
+    g.k_down = (F + FG_KR - 1) / FG_KR;
+    g.wu_tscale = wu_tscale;
+    g.wd_tscale = wd_tscale;
+    g.x_tscale = x_tscale;
+    g.h_tscale = h_tscale;
+    g.hb = hb;
+    g.hb_block = hb_block;
+    g.y = y;
+    g.debug_hold = debug_hold;
+    const int64_t max_units = (int64_t)max_sched * (g.m_up + g.m_down);
+    const int64_t slots = (int64_t)num_sms * (small ? Fp4Tmem<true>::CTAS : Fp4Tmem<false>::CTAS);
+    const int grid = (int)(max_units < slots ? max_units : slots);
+    auto kfn = small ? grouped_ffn_fp4_kernel<true> : grouped_ffn_fp4_kernel<false>;
+    cudaError_t err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    return launch_k(kfn, dim3(grid), dim3(FG_THREADS), smem, stream, maps, g, ctx);
+}
+
 cudaError_t launch_quantize_nvfp4(int64_t n_tensors, int64_t rows, int K, const uint16_t* src, uint8_t* codes,
                                   uint8_t* bscale, float* tscale, int num_sms, cudaStream_t stream) {
     if (n_tensors == 0 || rows == 0) return cudaSuccess;
@@ -746,13 +1250,13 @@ cudaError_t launch_quantize_nvfp4(int64_t n_tensors, int64_t rows, int K, const 
 
 cudaError_t launch_gather_nvfp4(const uint16_t* x, const int32_t* perm_src, int64_t rows, int K, int64_t T, int H,
                                 float s_t, uint8_t* codes, uint8_t* bscale, int num_sms, const DevCtx& ctx,
-                                cudaStream_t stream) {
+                                cudaStream_t stream, int* zero, int64_t n_zero) {
     if (rows == 0) return cudaSuccess;
     int64_t blocks = (rows + 7) / 8;
     const int64_t cap = (int64_t)num_sms * 8;
     if (blocks > cap) blocks = cap;
     return launch_k(nvfp4_gather_kernel, dim3((unsigned)blocks), dim3(256), 0, stream, x, perm_src, rows, K, T, H, s_t,
-                    codes, bscale, ctx);
+                    codes, bscale, zero, n_zero, ctx);
 }
 
 }  // namespace moe

@@ -166,3 +166,18 @@ def test_clock_sampler_reads_nvml_every_few_milliseconds():
     c = s.stop()
     assert c["sampler"].startswith("nvml") and c["samples"] >= 5
     assert c["sm_mhz"] == 1965 and c["reasons"] == ["sw_power_cap"]
+
+
+def test_one_launch_nvfp4_ffn_counts_both_banks_codes_and_scales():
+    """The one-launch NVFP4 FFN moves both banks (half a byte per value plus padded block scales),
+    x's codes in, H's codes out and back in, and bf16 Y out; its flops go against the fp4 peak."""
+    st = {"expert_ffn": 0.2, "combine": 0.01}
+    r = bench.roofline_entry(W.WORKLOADS[5], st, 121, PEAKS, "measured", "decode_nvfp4")
+    rows = 64 * 6
+    ksp_h, ksp_f = 176, 128
+    assert r["bound"] == "hbm" and r["kernel"].startswith("expert_ffn")
+    assert r["algorithmic_bytes_per_launch"] == (121 * F * (H // 2 + ksp_h) + 121 * H * (F // 2 + ksp_f)
+                                                 + rows * (H // 2 + ksp_h) + 2 * rows * (F // 2 + ksp_f)
+                                                 + rows * H * 2)
+    p = bench.roofline_entry(W.WORKLOADS[6], st, 128, PEAKS, "measured", "prefill_nvfp4")
+    assert p["bound"] == "tensor" and p["peak"] == pytest.approx(4 * PEAKS["bf16_tflops"])

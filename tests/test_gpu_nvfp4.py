@@ -129,7 +129,19 @@ def test_nvfp4_forward_parity_prefill_shape(moe):
     assert nvfp4_case(moe, w, inputs(w), tokens=np.arange(3, 4096, 611)) <= NVFP4_TOL
 
 
-def test_nvfp4_expired_wait_is_reported(moe):
+@pytest.mark.parametrize("one_launch", [1, 0], ids=["one_launch_ffn", "two_launches"])
+def test_nvfp4_expired_wait_is_reported(moe, one_launch):
+    """One launch: the list's first up unit withholds its report, so the down units of its entry
+    wait in vain.  Two launches: block 0's producer withholds its first load.  Either way the
+    status is MOE_ETIMEOUT and the next call is right."""
+    moe.debug_set(8, one_launch)
+    try:
+        _nvfp4_expired_wait_case(moe)
+    finally:
+        moe.debug_set(8, 1)
+
+
+def _nvfp4_expired_wait_case(moe):
     w = W.WORKLOADS[0]
     h = inputs(w)
     cu, bu, tu = gpu_bank(moe, h["wu"])
@@ -150,3 +162,34 @@ def test_nvfp4_expired_wait_is_reported(moe):
         moe.debug_set(1, 0)
     moe.expert_ffn(dims, dev_bf16(h["x"]), dev(offsets), dev(perm_src), cu, cd, sc, y, ws)
     moe.check_device_error()
+
+
+@pytest.mark.parametrize("w", [W.WORKLOADS[0], W.Workload("nvfp4_ragged_T37", 37, 512, 16, 4, 192, seed=26),
+                               W.Workload("nvfp4_tail_F224_T300", 300, 256, 8, 3, 224, seed=27),
+                               W.Workload("nvfp4_decode_T64", 64, 2688, 128, 6, 1856, seed=28),
+                               W.Workload("nvfp4_prefill_T4096", 4096, 2688, 128, 6, 1856, seed=29)],
+                         ids=lambda w: w.name)
+def test_nvfp4_one_launch_ffn_equals_two_launches_bitwise(moe, w):
+    """Both projections in one launch run the same units (same tiles, same accumulation order,
+    the same quantisation of H), so the layer output is the same bit for bit as with two
+    launches, at both TMEM layouts (tiles of up to 64 rows on two CTAs per SM, and up to 224)."""
+    h = inputs(w)
+    cu, bu, tu = gpu_bank(moe, h["wu"])
+    cd, bd, td = gpu_bank(moe, h["wd"])
+    tx, th = oracle.calibrate_nvfp4(h["x"][:64], h["wr"], h["bias"], h["wu"], w.K)
+    dims = moe.dims(w.T, w.H, w.E, w.K, w.F, nvfp4=True)
+    ws = moe.alloc_workspace(dims)
+    sc = moe.nvfp4_scales(tu, td, float(tx), float(th), bu, bd)
+    x, wr = dev_bf16(h["x"]), dev_bf16(h["wr"])
+    bias = None if h["bias"] is None else dev(h["bias"])
+    outs = []
+    for one in (1, 0):
+        moe.debug_set(8, one)
+        try:
+            out = torch.empty(w.T, w.H, dtype=torch.bfloat16, device="cuda")
+            moe.forward(dims, x, wr, bias, cu, cd, out, ws, scales=sc)
+            moe.check_device_error()
+            outs.append(out)
+        finally:
+            moe.debug_set(8, 1)
+    assert torch.equal(outs[0], outs[1])
