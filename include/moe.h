@@ -328,7 +328,7 @@ moe_status moe_set_stage_events(void* const* events, int32_t n);
  * what = 1: limit of every bounded wait in nanoseconds (value <= 0 restores
  * the default of 4 s); what = 2: the grouped-GEMM producer of block 0
  * withholds its first load (value 1) so the consumer's wait must expire --
- * in the one-launch FFN, the list's first up unit withholds its report so
+ * in the one-launch FFNs, the list's first up unit withholds its report so
  * that the down units of its entry wait in vain; 0 turns it off; what = 3: value 1 runs the grouped GEMMs of batches with
  * tiles of more than 64 tokens on CTA pairs (cta_group::2, M = 256), value 0
  * (the default) on single CTAs; what = 4: largest batch (tokens) that the
@@ -345,10 +345,10 @@ moe_status moe_set_stage_events(void* const* events, int32_t n);
  * on the device for it; what = 7: value 1 reads the shared expert's down
  * weight through the fallback map (the plain [H][Fs] matrix, chunk j from
  * column j*F) instead of the chunked 3-D view, 0 (the default) restores the
- * view; what = 8: value 1 (the default) runs both expert projections of bf16
- * and E4M3 layers without a shared expert in one launch (the down units of a
- * schedule entry start once that entry's up units have reported), 0 as two
- * launches.  Other `what`: MOE_EINVAL. */
+ * view; what = 8: value 1 (the default) runs both expert projections of bf16,
+ * E4M3 and NVFP4 layers without a shared expert in one launch (the down units
+ * of a schedule entry start once that entry's up units have reported), 0 as
+ * two launches.  Other `what`: MOE_EINVAL. */
 moe_status moe_debug_set(int32_t what, int64_t value);
 
 #ifdef __cplusplus
