@@ -634,9 +634,16 @@ def _fused_entry(wl, stages, touched, peaks, peak_kind, workload):
     the down projection together, over the launch's duration."""
     H, F, T, K = wl.H, wl.F, wl.T, wl.K
     rows = T * K
-    es = 1 if wl.fp8 else 2
+    fp8 = wl.fp8 or wl.fp8_b128
+    es = 1 if fp8 else 2
     ms = stages["expert_ffn"]
-    if wl.nvfp4:
+    if wl.fp8_b128:
+        # codes padded to whole blocks of 128 along K + one fp32 scale per block, both banks;
+        # x's codes in, H's codes out and back in, bf16 Y out
+        kp = lambda k: (k + 127) // 128 * 128
+        algo = (touched * F * (kp(H) + kp(H) // 128 * 4) + touched * H * (kp(F) + kp(F) // 128 * 4)
+                + rows * H + 2 * rows * F + rows * H * 2)
+    elif wl.nvfp4:
         # packed codes (half a byte per value) + one E4M3 block scale per 16 values (rows padded
         # to 16 bytes): both banks, x's codes in, H's codes out and back in, bf16 Y out
         ksp = lambda k: (k // 16 + 15) // 16 * 16
@@ -647,13 +654,13 @@ def _fused_entry(wl, stages, touched, peaks, peak_kind, workload):
     flops = 2 * 2.0 * rows * F * H
     gbs = algo / (ms * 1e-3) / 1e9
     hbm_peak = peaks["hbm_gbs"]
-    if wl.fp8 and peaks.get("fp8_tflops"):
+    if fp8 and peaks.get("fp8_tflops"):
         tc_peak, src = peaks["fp8_tflops"], peaks["fp8_source"]
     else:
-        ratio = 4.0 if wl.nvfp4 else 2.0 if wl.fp8 else 1.0
+        ratio = 4.0 if wl.nvfp4 else 2.0 if fp8 else 1.0
         tc_peak = peaks["bf16_tflops"] * ratio
         src = f"{peak_kind} bf16 burst" + (" x 4 (nvfp4/bf16 nominal ratio)" if wl.nvfp4 else
-                                           " x 2 (fp8/bf16 nominal ratio)" if wl.fp8 else "")
+                                           " x 2 (fp8/bf16 nominal ratio)" if fp8 else "")
     tflops = flops / (ms * 1e-3) / 1e12
     common = {"kernel": "expert_ffn (up and down projections, one launch)", "ms_per_launch": ms,
               "algorithmic_bytes_per_launch": algo, "algorithmic_flops_per_launch": flops,

@@ -143,10 +143,11 @@ struct ForwardWs {
 // NVFP4 at 224: its accumulators share TMEM with the scale factors),
 // plus the shared expert's entries (ns chunks of T rows, cut into tiles of at
 // most bn).
-// Whether the expert FFN runs as one launch (bf16, E4M3 or NVFP4 experts without a shared expert).
+// Whether the expert FFN runs as one launch (any expert format, without a shared expert).
 bool fused_ffn(const moe_dims* d) {
     return g_fused_ffn.load() && n_shared(d) == 0 &&
-           (d->expert_dtype == MOE_BF16 || d->expert_dtype == MOE_FP8_E4M3 || d->expert_dtype == MOE_NVFP4);
+           (d->expert_dtype == MOE_BF16 || d->expert_dtype == MOE_FP8_E4M3 || d->expert_dtype == MOE_NVFP4 ||
+            d->expert_dtype == MOE_FP8_B128);
 }
 
 GemmPlan ffn_plan(const moe_dims* d) {
@@ -242,11 +243,23 @@ moe_status run_ffn(const moe_dims* d, const DeviceInfo* dev, const DevCtx& ctx, 
     const int ns = n_shared(d);
     if (d->expert_dtype == MOE_FP8_B128) {
         const int withhold_b = g_debug_withhold.load();
+        const bool fusedb = fused_ffn(d);
         if (marks) stage_mark(3, st);
+        // E4M3 codes of the permuted rows; they also zero the one-launch FFN's counters
         cudaError_t eb = launch_gather(static_cast<const uint16_t*>(x), perm_src, rows, rows, d->K, d->T, d->H,
-                                       fw.xp, true, sc->x_scale, dev->num_sms, ctx, st);
+                                       fw.xp, true, sc->x_scale, dev->num_sms, ctx, st,
+                                       fusedb ? fw.done : nullptr, fusedb ? gp.max_sched + 1 : 0);
         if (eb != cudaSuccess) return cuda_status(eb);
         if (marks) stage_mark(4, st);
+        if (fusedb) {
+            eb = launch_grouped_ffn_b128(static_cast<const uint8_t*>(w_up), sc->w_up_scale,
+                                         static_cast<const uint8_t*>(w_down), sc->w_down_scale, d->E, d->F, d->H,
+                                         static_cast<const uint8_t*>(fw.xp), static_cast<uint8_t*>(fw.hb), y_perm,
+                                         rows, fw.sched, fw.n_sched, gp.bn, gp.max_sched, fw.done, sc->x_scale,
+                                         sc->h_scale, dev->num_sms, withhold_b, ctx, st);
+            if (marks) stage_mark(5, st);
+            return cuda_status(eb);
+        }
         eb = launch_grouped_gemm_b128(true, static_cast<const uint8_t*>(w_up), sc->w_up_scale, d->E, d->F, d->H,
                                       static_cast<const uint8_t*>(fw.xp), rows, fw.sched, fw.n_sched, gp.bn,
                                       gp.max_sched, fw.hb, sc->x_scale, sc->h_scale, dev->num_sms, withhold_b, ctx, st);
@@ -405,7 +418,8 @@ moe_status moe_forward_launches(const moe_dims* d, int32_t* launches) {
     int n = route_launches(d->T, d->H, d->E);
     n += permute_scratch_ints(d->T * d->K, d->E) == 0 ? 1 : 3;   // one block, or histogram + scan + scatter
     // row gather, up and down projections (one launch or two), combine
-    const bool pair = d->expert_dtype != MOE_NVFP4 && g_gemm_pair.load() && gemm_plan(d->T, d->K, d->E).bn > 64;
+    const bool pair = (d->expert_dtype == MOE_BF16 || d->expert_dtype == MOE_FP8_E4M3) && g_gemm_pair.load() &&
+                      gemm_plan(d->T, d->K, d->E).bn > 64;
     n += 1 + (fused_ffn(d) && !pair ? 1 : 2) + 1;
     *launches = n;
     return MOE_OK;

@@ -266,6 +266,327 @@ __global__ void __launch_bounds__(GB_THREADS, 1)
     }
 }
 
+// ----------------------------------------------------------------------------- one-launch FFN
+
+// Both FP8_B128 projections in one persistent launch, as the bf16 one-launch FFN
+// (grouped_ffn.cu) does it: every up unit (schedule entry x 128-row block of F), then every
+// down unit (entry x block of H), claimed in that order from a global counter by each CTA's
+// producer and passed to the MMA thread and the epilogue warps through a small queue in shared
+// memory.  An up unit's epilogue warps store their features of H, fence them for the async
+// proxy and each add 1 to done[entry] with release semantics; the producer of a down unit
+// waits (bounded) until done[entry] reaches 4 x (blocks of F) before it loads the entry's H.
+// Tiles of up to 64 rows (TMEM: 4 partial slots of 64 columns) run two CTAs per SM with a
+// 100 KB ring each; tiles of up to 128 rows one CTA per SM with up to 200 KB.
+constexpr int FB_UQ = 4;   // unit queue slots
+
+template <int BN>
+struct B128Layout {
+    static constexpr int CTAS = BN <= 64 ? 2 : 1;
+    static constexpr int RING = BN <= 64 ? 100 * 1024 : 200 * 1024;
+};
+
+struct B128FfnArgs {
+    int* claim;              // unit counter (zero at launch; right after done[])
+    int* done;               // [max_sched] up epilogue warps finished per entry (zero at launch)
+    const int4* sched;
+    const int* n_sched;
+    int m_up, m_down;        // 128-row blocks of F and of H
+    int F, H;
+    int k_up, k_down;        // scale blocks (K stages) of H and of F
+    int n_stages;
+    int b_stage_bytes;
+    const float* su;         // [E][F][k_up]
+    const float* sd;         // [E][H][k_down]
+    float x_scale, h_scale;
+    uint8_t* hb;             // H codes [rows][F]
+    void* y;                 // bf16 [rows][H]
+    int debug_hold;          // 1: the list's first up unit never reports its rows (a wait must expire)
+};
+
+struct B128FfnMaps {
+    B128Maps up, down;
+};
+
+template <int BN>
+__global__ void __launch_bounds__(GB_THREADS, B128Layout<BN>::CTAS)
+    grouped_ffn_b128_kernel(const __grid_constant__ B128FfnMaps maps, B128FfnArgs g, DevCtx ctx) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    const int NS = g.n_stages;
+    uint8_t* smA = smem;
+    uint8_t* smB = smA + (size_t)NS * GB_A_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smB + (size_t)NS * g.b_stage_bytes);
+    uint64_t* full = bars;
+    uint64_t* empty = bars + NS;
+    uint64_t* pfull = bars + 2 * NS;
+    uint64_t* pempty = pfull + GB_NP;
+    uint64_t* drain = pempty + GB_NP;
+    uint64_t* uq_full = drain + 1;
+    uint64_t* uq_empty = uq_full + FB_UQ;
+    volatile int* uq = reinterpret_cast<volatile int*>(uq_empty + FB_UQ);
+    volatile int* abort_flag = uq + FB_UQ;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(const_cast<int*>(abort_flag + 1));
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(smem_u32(&full[s]), 1);
+            mbar_init(smem_u32(&empty[s]), 1);
+        }
+        for (int p = 0; p < GB_NP; ++p) {
+            mbar_init(smem_u32(&pfull[p]), 1);
+            mbar_init(smem_u32(&pempty[p]), 128);
+        }
+        mbar_init(smem_u32(drain), 1);
+        for (int q = 0; q < FB_UQ; ++q) {
+            mbar_init(smem_u32(&uq_full[q]), 1);
+            mbar_init(smem_u32(&uq_empty[q]), 1 + 4);   // the MMA thread and the 4 epilogue warps
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) tmem_alloc(smem_u32(tmem_holder), GB_NP * BN);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+    pdl_enter();
+
+    const int n_sched = *g.n_sched;
+    const int n_up = n_sched * g.m_up;
+    const int n_units = n_up + n_sched * g.m_down;
+    const int up_target = 4 * g.m_up;   // reports of one entry's up units
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- producer
+        if (lane == 0) {
+            const uint64_t pol_w = l2_policy_evict_first();
+            const uint64_t pol_x = l2_policy_evict_last();
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            int qs = 0;
+            uint32_t qph = 0;
+            int claim = atomicAdd(g.claim, 1);
+            while (ok) {
+                const int u = claim < n_units ? claim : -1;
+                if (!mbar_wait(smem_u32(&uq_empty[qs]), qph ^ 1u, ctx, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                uq[qs] = u;
+                mbar_arrive(smem_u32(&uq_full[qs]));
+                if (++qs == FB_UQ) {
+                    qs = 0;
+                    qph ^= 1u;
+                }
+                if (u < 0) break;
+                claim = atomicAdd(g.claim, 1);   // the next unit, claimed while this one loads
+                const bool up = u < n_up;
+                const int v = up ? u : u - n_up;
+                const int m_blocks = up ? g.m_up : g.m_down;
+                const int s_idx = v / m_blocks, mb = v % m_blocks;
+                const int4 sc = g.sched[s_idx];
+                const int Nout = up ? g.F : g.H;
+                const int k_stages = up ? g.k_up : g.k_down;
+                const B128Maps& mp = up ? maps.up : maps.down;
+                const bool a_full = Nout - mb * GB_BM > 64;
+                const int n16 = (sc.z + 15) / 16;
+                const int n64 = n16 / 4, r16 = n16 % 4;
+                const uint32_t bytes = (uint32_t)((a_full ? 128 : 64) * GB_ROW + n16 * 16 * GB_ROW);
+                const int a_y = sc.x * Nout + mb * GB_BM;
+                if (!up) {
+                    // the rows of H this unit reads are written by the up units of its entry
+                    if (!wait_count(g.done + s_idx, up_target, ctx, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    fence_proxy_async_global();
+                }
+                for (int ks = 0; ks < k_stages; ++ks) {
+                    if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, ctx, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t fb = smem_u32(&full[stage]);
+                    mbar_arrive_expect_tx(fb, bytes);
+                    const int kx = ks * GB_ROW;
+                    const uint32_t a_dst = smem_u32(smA + (size_t)stage * GB_A_BYTES);
+                    const uint32_t b_dst = smem_u32(smB + (size_t)stage * g.b_stage_bytes);
+                    tma_load_2d(a_dst, a_full ? &mp.a128 : &mp.a64, fb, kx, a_y, pol_w);
+                    int row = 0;
+                    for (int j = 0; j < n64; ++j, row += 64)
+                        tma_load_2d(b_dst + row * GB_ROW, &mp.b64, fb, kx, sc.y + row, pol_x);
+                    for (int j = 0; j < r16; ++j, row += 16)
+                        tma_load_2d(b_dst + row * GB_ROW, &mp.b16, fb, kx, sc.y + row, pol_x);
+                    if (++stage == NS) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                const uint64_t t0 = globaltimer();
+                while (globaltimer() - t0 < 200000ull) __nanosleep(1000);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA
+        if (lane == 0) {
+            int stage = 0, ps = 0;
+            uint32_t phase = 0, pph = 0;
+            bool ok = true, issued = false;
+            int qs = 0;
+            uint32_t qph = 0;
+            while (ok) {
+                if (!mbar_wait(smem_u32(&uq_full[qs]), qph, ctx, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                const int u = uq[qs];
+                mbar_arrive(smem_u32(&uq_empty[qs]));
+                if (++qs == FB_UQ) {
+                    qs = 0;
+                    qph ^= 1u;
+                }
+                if (u < 0) break;
+                const bool up = u < n_up;
+                const int v = up ? u : u - n_up;
+                const int4 sc = g.sched[v / (up ? g.m_up : g.m_down)];
+                const int k_stages = up ? g.k_up : g.k_down;
+                const int n_mma = max(16, (sc.z + 15) & ~15);
+                const uint32_t idesc = make_idesc(0u, GB_BM, n_mma);
+                for (int ks = 0; ks < k_stages; ++ks) {
+                    if (!mbar_wait(smem_u32(&full[stage]), phase, ctx, abort_flag) ||
+                        !mbar_wait(smem_u32(&pempty[ps]), pph ^ 1u, ctx, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t d_tmem = tmem_base + (uint32_t)(ps * BN);
+                    const uint32_t a_base = smem_u32(smA + (size_t)stage * GB_A_BYTES);
+                    const uint32_t b_base = smem_u32(smB + (size_t)stage * g.b_stage_bytes);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)   // 4 x K = 32: the block's sum, the slot overwritten first
+                        mma_ss<true>(d_tmem, sw128_desc(a_base + kk * 32), sw128_desc(b_base + kk * 32), idesc,
+                                     kk != 0 ? 1u : 0u);
+                    issued = true;
+                    mma_commit(smem_u32(&empty[stage]));
+                    mma_commit(smem_u32(&pfull[ps]));
+                    if (++stage == NS) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                    if (++ps == GB_NP) {
+                        ps = 0;
+                        pph ^= 1u;
+                    }
+                }
+            }
+            if (!ok && issued) {
+                mma_commit(smem_u32(drain));
+                mbar_wait_drain(smem_u32(drain), 0, ctx.timeout_ns);
+            }
+        }
+    } else {
+        // ---------------------------------------------------------------- block sums and epilogue
+        const int q = warp & 3;   // TMEM lane quadrant of this warp
+        int ps = 0;
+        uint32_t pph = 0;
+        bool ok = true;
+        int qs = 0;
+        uint32_t qph = 0;
+        const float inv_h = __frcp_rn(g.h_scale);
+        while (ok) {
+            if (!mbar_wait_warp(smem_u32(&uq_full[qs]), qph, ctx, abort_flag)) break;
+            const int u = uq[qs];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&uq_empty[qs]));
+            if (++qs == FB_UQ) {
+                qs = 0;
+                qph ^= 1u;
+            }
+            if (u < 0) break;
+            const bool up = u < n_up;
+            const int v = up ? u : u - n_up;
+            const int m_blocks = up ? g.m_up : g.m_down;
+            const int s_idx = v / m_blocks, mb = v % m_blocks;
+            const int4 sc = g.sched[s_idx];
+            const int Nout = up ? g.F : g.H;
+            const int k_stages = up ? g.k_up : g.k_down;
+            const int f = mb * GB_BM + q * 32 + lane;
+            const bool fvalid = f < Nout;
+            const int nch = (sc.z + 15) / 16;   // warp-uniform, <= BN / 16
+            const float* wrow = (up ? g.su : g.sd) + ((int64_t)sc.x * Nout + (fvalid ? f : 0)) * k_stages;
+            const float in_scale = up ? g.x_scale : g.h_scale;
+            float acc[BN];
+#pragma unroll
+            for (int i = 0; i < BN; ++i) acc[i] = 0.0f;
+            for (int ks = 0; ks < k_stages; ++ks) {
+                if (!mbar_wait_warp(smem_u32(&pfull[ps]), pph, ctx, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const float sw = wrow[ks];
+                const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(ps * BN);
+#pragma unroll
+                for (int c = 0; c < BN / 16; ++c) {
+                    if (c < nch) {
+                        uint32_t vv[16];
+                        tmem_ld16(t_row + (uint32_t)(c * 16), vv);
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) acc[c * 16 + j] = __fmaf_rn(sw, __uint_as_float(vv[j]), acc[c * 16 + j]);
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(smem_u32(&pempty[ps]));
+                if (++ps == GB_NP) {
+                    ps = 0;
+                    pph ^= 1u;
+                }
+            }
+            if (!ok) break;
+            if (fvalid) {
+#pragma unroll
+                for (int c = 0; c < BN / 16; ++c) {
+                    if (c >= nch) break;
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int r = c * 16 + j;
+                        if (r < sc.z) {
+                            const float z = __fmul_rn(acc[r], in_scale);
+                            if (up) {
+                                const float a = z > 0.0f ? __fmul_rn(z, z) : 0.0f;
+                                g.hb[(int64_t)(sc.y + r) * g.F + f] =
+                                    (uint8_t)__nv_cvt_float_to_fp8(__fmul_rn(a, inv_h), __NV_SATFINITE, __NV_E4M3);
+                            } else {
+                                static_cast<__nv_bfloat16*>(g.y)[(int64_t)(sc.y + r) * g.H + f] = __float2bfloat16_rn(z);
+                            }
+                        }
+                    }
+                }
+            }
+            if (up) {
+                // this warp's features of H are complete: every lane orders its stores for the async
+                // proxy (the TMA loads of H), the warp barrier orders them before lane 0's release
+                fence_proxy_async_global();
+                __syncwarp();
+                const bool hold = g.debug_hold && u == 0;
+                if (lane == 0 && !hold) red_release_add(g.done + s_idx, 1);
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, GB_NP * BN);
+    }
+}
+
 // One warp per (row, block of 128): scale amax / 448 (1 for a zero block),
 // codes e4m3(fl32(w / scale)) nearest-even and saturating, zero past K.
 __global__ void quantize_fp8_b128_kernel(const uint16_t* __restrict__ src, int64_t rows, int K, int Kp,
@@ -373,6 +694,64 @@ cudaError_t launch_grouped_gemm_b128(bool up, const uint8_t* W, const float* w_s
     const int grid = (int)(max_units < num_sms ? max_units : num_sms);
     auto kfn = bn > 64 ? (up ? grouped_gemm_b128_kernel<true, 128> : grouped_gemm_b128_kernel<false, 128>)
                        : (up ? grouped_gemm_b128_kernel<true, 64> : grouped_gemm_b128_kernel<false, 64>);
+    cudaError_t err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    return launch_k(kfn, dim3(grid), dim3(GB_THREADS), smem, stream, maps, g, ctx);
+}
+
+// Both FP8_B128 projections in one launch.  W_up codes [E*F][Kp(H)] with scales su
+// [E][F][Kp(H)/128], W_down codes [E*H][Kp(F)] with sd [E][H][Kp(F)/128]; xp: E4M3 codes of the
+// permuted rows [rows][H]; hb: H's E4M3 codes [rows][F]; y: bf16 [rows][H].  done: max_sched + 1
+// ints (the per-entry counters, then the unit claim counter), zero before the launch.
+cudaError_t launch_grouped_ffn_b128(const uint8_t* w_up, const float* su, const uint8_t* w_down, const float* sd,
+                                    int E, int F, int H, const uint8_t* xp, uint8_t* hb, void* y, int64_t rows,
+                                    const int4* sched, const int* n_sched, int bn, int max_sched, int* done,
+                                    float x_scale, float h_scale, int num_sms, int debug_hold, const DevCtx& ctx,
+                                    cudaStream_t stream) {
+    if (rows == 0) return cudaSuccess;
+    if (bn < 16 || bn > kB128MaxTileRows || bn % 16 != 0) return cudaErrorInvalidValue;
+    const int Kh = b128_kp(H), Kf = b128_kp(F);
+    B128FfnMaps maps;
+    if (!make_map_u8_b128(&maps.up.a128, w_up, (int64_t)E * F, Kh, 128) ||
+        !make_map_u8_b128(&maps.up.a64, w_up, (int64_t)E * F, Kh, 64) ||
+        !make_map_u8_b128(&maps.up.b64, xp, rows, H, 64) || !make_map_u8_b128(&maps.up.b16, xp, rows, H, 16) ||
+        !make_map_u8_b128(&maps.down.a128, w_down, (int64_t)E * H, Kf, 128) ||
+        !make_map_u8_b128(&maps.down.a64, w_down, (int64_t)E * H, Kf, 64) ||
+        !make_map_u8_b128(&maps.down.b64, hb, rows, F, 64) || !make_map_u8_b128(&maps.down.b16, hb, rows, F, 16))
+        return cudaErrorInvalidValue;
+    const bool small = bn <= 64;
+    B128FfnArgs g;
+    g.done = done;
+    g.claim = done + max_sched;
+    g.sched = sched;
+    g.n_sched = n_sched;
+    g.m_up = (F + GB_BM - 1) / GB_BM;
+    g.m_down = (H + GB_BM - 1) / GB_BM;
+    g.F = F;
+    g.H = H;
+    g.k_up = Kh / GB_ROW;
+    g.k_down = Kf / GB_ROW;
+    g.b_stage_bytes = bn * GB_ROW;
+    const int stage = GB_A_BYTES + g.b_stage_bytes;
+    int ns = (small ? B128Layout<64>::RING : B128Layout<128>::RING) / stage;
+    if (ns > 8) ns = 8;
+    if (ns < 2) ns = 2;
+    g.n_stages = ns;
+    g.su = su;
+    g.sd = sd;
+    g.x_scale = x_scale;
+    g.h_scale = h_scale;
+    g.hb = hb;
+    g.y = y;
+    g.debug_hold = debug_hold;
+    // ring, barriers (full, empty, 4 pfull, 4 pempty, drain, the queue's full and empty), the
+    // queue, the abort flag and the TMEM holder
+    const size_t smem = 1024 + (size_t)ns * stage + (size_t)(2 * ns + 2 * GB_NP + 1 + 2 * FB_UQ) * 8 +
+                        FB_UQ * sizeof(int) + 8 + 16;
+    const int64_t max_units = (int64_t)max_sched * (g.m_up + g.m_down);
+    const int64_t slots = (int64_t)num_sms * (small ? B128Layout<64>::CTAS : B128Layout<128>::CTAS);
+    const int grid = (int)(max_units < slots ? max_units : slots);
+    auto kfn = small ? grouped_ffn_b128_kernel<64> : grouped_ffn_b128_kernel<128>;
     cudaError_t err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     return launch_k(kfn, dim3(grid), dim3(GB_THREADS), smem, stream, maps, g, ctx);

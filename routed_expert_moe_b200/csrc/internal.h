@@ -83,6 +83,11 @@ cudaError_t launch_grouped_gemm_b128(bool up, const uint8_t* W, const float* w_s
                                      const uint8_t* act, int64_t rows, const int4* sched, const int* n_sched, int bn,
                                      int max_sched, void* out, float in_scale, float out_scale, int num_sms,
                                      int debug_withhold, const DevCtx& ctx, cudaStream_t stream);
+cudaError_t launch_grouped_ffn_b128(const uint8_t* w_up, const float* su, const uint8_t* w_down, const float* sd,
+                                    int E, int F, int H, const uint8_t* xp, uint8_t* hb, void* y, int64_t rows,
+                                    const int4* sched, const int* n_sched, int bn, int max_sched, int* done,
+                                    float x_scale, float h_scale, int num_sms, int debug_hold, const DevCtx& ctx,
+                                    cudaStream_t stream);
 cudaError_t launch_quantize_fp8_b128(int64_t rows, int K, const uint16_t* src, uint8_t* codes, float* scales,
                                      int num_sms, cudaStream_t stream);
 cudaError_t launch_combine(const uint16_t* yp, const int32_t* inv_row, const float* w, const uint16_t* residual,

@@ -181,3 +181,14 @@ def test_one_launch_nvfp4_ffn_counts_both_banks_codes_and_scales():
                                                  + rows * H * 2)
     p = bench.roofline_entry(W.WORKLOADS[6], st, 128, PEAKS, "measured", "prefill_nvfp4")
     assert p["bound"] == "tensor" and p["peak"] == pytest.approx(4 * PEAKS["bf16_tflops"])
+
+
+def test_one_launch_fp8_b128_ffn_counts_padded_codes_and_block_scales():
+    st = {"expert_ffn": 0.2}
+    r = bench.roofline_entry(W.WORKLOADS[9], st, 121, PEAKS, "measured", "decode_fp8_b128")
+    rows = 64 * 6
+    assert r["bound"] == "hbm"
+    assert r["algorithmic_bytes_per_launch"] == (121 * F * (2688 + 21 * 4) + 121 * H * (1920 + 15 * 4)
+                                                 + rows * H + 2 * rows * F + rows * H * 2)
+    p = bench.roofline_entry(W.WORKLOADS[10], st, 128, PEAKS, "measured", "prefill_fp8_b128")
+    assert p["bound"] == "tensor" and p["peak"] == 2 * PEAKS["bf16_tflops"]

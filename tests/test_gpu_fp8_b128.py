@@ -79,7 +79,19 @@ def test_b128_forward_parity_decode_shape(moe):
     assert b128_case(moe, w, inputs(w), tokens=np.arange(0, 64, 7)) <= FP8_TOL
 
 
-def test_b128_expired_wait_is_reported(moe):
+@pytest.mark.parametrize("one_launch", [1, 0], ids=["one_launch_ffn", "two_launches"])
+def test_b128_expired_wait_is_reported(moe, one_launch):
+    """One launch: the list's first up unit withholds its report, so the down units of its entry
+    wait in vain.  Two launches: block 0's producer withholds its first load.  Either way the
+    status is MOE_ETIMEOUT and the next call is right."""
+    moe.debug_set(8, one_launch)
+    try:
+        _b128_expired_wait_case(moe)
+    finally:
+        moe.debug_set(8, 1)
+
+
+def _b128_expired_wait_case(moe):
     w = W.WORKLOADS[0]
     h = inputs(w)
     cu, su = gpu_bank(moe, h["wu"])
@@ -143,3 +155,35 @@ def test_b128_forward_parity_prefill_shape(moe):
     r = oracle.moe_layer_fp8_b128(x, wr, None, bu, bd, sx, sh, w.K, w.H, w.F, tokens=tok, slot=slot)
     assert np.array_equal(r["idx"], ridx[tok])
     assert rel_err(host_f64(out)[tok], r["out"]) <= FP8_TOL
+
+
+@pytest.mark.parametrize("w", [W.WORKLOADS[0], W.Workload("b128_ragged_T37_F192", 37, 512, 16, 4, 192, seed=51),
+                               W.Workload("b128_tails_H272_F208", 21, 272, 8, 3, 208, seed=52),
+                               W.Workload("b128_hot_T300", 300, 256, 4, 2, 128, seed=53),
+                               W.Workload("b128_decode_T64", 64, 2688, 128, 6, 1856, seed=54),
+                               W.Workload("b128_T700", 700, 512, 16, 4, 320, seed=55)],
+                         ids=lambda w: w.name)
+def test_b128_one_launch_ffn_equals_two_launches_bitwise(moe, w):
+    """Both projections in one launch run the same units (same tiles, same block sums in the
+    same order), so the output is the same bit for bit as with two launches, for tiles of up to
+    64 rows (two CTAs per SM) and up to 128."""
+    h = inputs(w)
+    cu, su = gpu_bank(moe, h["wu"])
+    cd, sd = gpu_bank(moe, h["wd"])
+    sx, sh = oracle.calibrate_fp8(h["x"][:64], h["wr"], h["bias"], h["wu"], w.K)
+    dims = moe.dims(w.T, w.H, w.E, w.K, w.F, fp8_b128=True)
+    ws = moe.alloc_workspace(dims)
+    sc = moe.fp8_scales(su, sd, float(sx), float(sh))
+    x, wr = dev_bf16(h["x"]), dev_bf16(h["wr"])
+    bias = None if h["bias"] is None else dev(h["bias"])
+    outs = []
+    for one in (1, 0):
+        moe.debug_set(8, one)
+        try:
+            out = torch.empty(w.T, w.H, dtype=torch.bfloat16, device="cuda")
+            moe.forward(dims, x, wr, bias, cu, cd, out, ws, scales=sc)
+            moe.check_device_error()
+            outs.append(out)
+        finally:
+            moe.debug_set(8, 1)
+    assert torch.equal(outs[0], outs[1])
