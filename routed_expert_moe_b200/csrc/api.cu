@@ -156,7 +156,7 @@ GemmPlan ffn_plan(const moe_dims* d) {
     // most 128 rows, which run two CTAs per SM: the skewed T=576 batch's FFN 292 -> 283 us
     // against 224-row tiles (hot experts split into more tiles; their weights re-read from L2).
     const bool sparse = d->T * d->K < (int64_t)kFfnSparseRows * d->E;
-    const int cap = d->expert_dtype == MOE_FP8_B128 ? kB128MaxTileRows
+    const int cap = d->expert_dtype == MOE_FP8_B128 ? (fused_ffn(d) ? kB128OneLaunchTileRows : kB128MaxTileRows)
                     : d->expert_dtype == MOE_NVFP4    ? kFp4MaxTileRows
                     : fused_ffn(d) && sparse          ? kFfnSparseRows
                                                       : 0;

@@ -275,15 +275,12 @@ __global__ void __launch_bounds__(GB_THREADS, 1)
 // memory.  An up unit's epilogue warps store their features of H, fence them for the async
 // proxy and each add 1 to done[entry] with release semantics; the producer of a down unit
 // waits (bounded) until done[entry] reaches 4 x (blocks of F) before it loads the entry's H.
-// Tiles of up to 64 rows (TMEM: 4 partial slots of 64 columns) run two CTAs per SM with a
-// 100 KB ring each; tiles of up to 128 rows one CTA per SM with up to 200 KB.
+// Tiles of up to 64 rows (TMEM: 4 partial slots of 64 columns, 256 in all) run two CTAs per SM
+// with a 100 KB ring each.
 constexpr int FB_UQ = 4;   // unit queue slots
-
-template <int BN>
-struct B128Layout {
-    static constexpr int CTAS = BN <= 64 ? 2 : 1;
-    static constexpr int RING = BN <= 64 ? 100 * 1024 : 200 * 1024;
-};
+constexpr int FB_BN = 64;  // token rows per schedule entry at most
+constexpr int FB_RING = 100 * 1024;
+static_assert(FB_BN == kB128OneLaunchTileRows, "one-launch FP8_B128 tile rows");
 
 struct B128FfnArgs {
     int* claim;              // unit counter (zero at launch; right after done[])
@@ -308,7 +305,7 @@ struct B128FfnMaps {
 };
 
 template <int BN>
-__global__ void __launch_bounds__(GB_THREADS, B128Layout<BN>::CTAS)
+__global__ void __launch_bounds__(GB_THREADS, 2)
     grouped_ffn_b128_kernel(const __grid_constant__ B128FfnMaps maps, B128FfnArgs g, DevCtx ctx) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -709,7 +706,7 @@ cudaError_t launch_grouped_ffn_b128(const uint8_t* w_up, const float* su, const 
                                     float x_scale, float h_scale, int num_sms, int debug_hold, const DevCtx& ctx,
                                     cudaStream_t stream) {
     if (rows == 0) return cudaSuccess;
-    if (bn < 16 || bn > kB128MaxTileRows || bn % 16 != 0) return cudaErrorInvalidValue;
+    if (bn < 16 || bn > FB_BN || bn % 16 != 0) return cudaErrorInvalidValue;
     const int Kh = b128_kp(H), Kf = b128_kp(F);
     B128FfnMaps maps;
     if (!make_map_u8_b128(&maps.up.a128, w_up, (int64_t)E * F, Kh, 128) ||
@@ -719,7 +716,6 @@ cudaError_t launch_grouped_ffn_b128(const uint8_t* w_up, const float* su, const 
         !make_map_u8_b128(&maps.down.a64, w_down, (int64_t)E * H, Kf, 64) ||
         !make_map_u8_b128(&maps.down.b64, hb, rows, F, 64) || !make_map_u8_b128(&maps.down.b16, hb, rows, F, 16))
         return cudaErrorInvalidValue;
-    const bool small = bn <= 64;
     B128FfnArgs g;
     g.done = done;
     g.claim = done + max_sched;
@@ -733,7 +729,7 @@ cudaError_t launch_grouped_ffn_b128(const uint8_t* w_up, const float* su, const 
     g.k_down = Kf / GB_ROW;
     g.b_stage_bytes = bn * GB_ROW;
     const int stage = GB_A_BYTES + g.b_stage_bytes;
-    int ns = (small ? B128Layout<64>::RING : B128Layout<128>::RING) / stage;
+    int ns = FB_RING / stage;
     if (ns > 8) ns = 8;
     if (ns < 2) ns = 2;
     g.n_stages = ns;
@@ -749,9 +745,9 @@ cudaError_t launch_grouped_ffn_b128(const uint8_t* w_up, const float* su, const 
     const size_t smem = 1024 + (size_t)ns * stage + (size_t)(2 * ns + 2 * GB_NP + 1 + 2 * FB_UQ) * 8 +
                         FB_UQ * sizeof(int) + 8 + 16;
     const int64_t max_units = (int64_t)max_sched * (g.m_up + g.m_down);
-    const int64_t slots = (int64_t)num_sms * (small ? B128Layout<64>::CTAS : B128Layout<128>::CTAS);
+    const int64_t slots = (int64_t)num_sms * 2;   // two CTAs per SM
     const int grid = (int)(max_units < slots ? max_units : slots);
-    auto kfn = small ? grouped_ffn_b128_kernel<64> : grouped_ffn_b128_kernel<128>;
+    auto kfn = grouped_ffn_b128_kernel<FB_BN>;
     cudaError_t err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     return launch_k(kfn, dim3(grid), dim3(GB_THREADS), smem, stream, maps, g, ctx);

@@ -106,6 +106,11 @@ cudaError_t launch_ep_regroup(const int64_t* recv_counts, int W, int E_loc, int6
 // keeps one running fp32 sum per row in registers.
 constexpr int kB128MaxTileRows = 128;
 
+// Token rows per schedule entry of the one-launch FP8_B128 FFN: tiles of 64 rows run two CTAs per
+// SM, which outweighs reading an expert's weights for three tiles instead of two at prefill
+// (FP8_B128 prefill layer 993 -> 767 us).
+constexpr int kB128OneLaunchTileRows = 64;
+
 // Token rows per schedule entry of the NVFP4 grouped GEMM: its two TMEM
 // accumulators of this many columns leave room for the scale factors.
 constexpr int kFp4MaxTileRows = 224;

@@ -164,9 +164,10 @@ def test_b128_forward_parity_prefill_shape(moe):
                                W.Workload("b128_T700", 700, 512, 16, 4, 320, seed=55)],
                          ids=lambda w: w.name)
 def test_b128_one_launch_ffn_equals_two_launches_bitwise(moe, w):
-    """Both projections in one launch run the same units (same tiles, same block sums in the
-    same order), so the output is the same bit for bit as with two launches, for tiles of up to
-    64 rows (two CTAs per SM) and up to 128."""
+    """Both projections in one launch run the same block sums in the same order for every
+    (token, feature), so the output is the same bit for bit as with two launches, although the
+    one launch cuts experts into tiles of at most 64 rows and the two launches into up to 128
+    (T = 700 here, 175 rows per expert)."""
     h = inputs(w)
     cu, su = gpu_bank(moe, h["wu"])
     cd, sd = gpu_bank(moe, h["wd"])
