@@ -143,11 +143,13 @@ struct ForwardWs {
 // NVFP4 at 224: its accumulators share TMEM with the scale factors),
 // plus the shared expert's entries (ns chunks of T rows, cut into tiles of at
 // most bn).
-// Whether the expert FFN runs as one launch (any expert format, without a shared expert).
+// Whether the expert FFN runs as one launch (every expert format; a shared expert, which only
+// bf16 layers take, adds its chunks as entries of the same unit list).
 bool fused_ffn(const moe_dims* d) {
-    return g_fused_ffn.load() && n_shared(d) == 0 &&
-           (d->expert_dtype == MOE_BF16 || d->expert_dtype == MOE_FP8_E4M3 || d->expert_dtype == MOE_NVFP4 ||
-            d->expert_dtype == MOE_FP8_B128);
+    if (!g_fused_ffn.load()) return false;
+    if (n_shared(d) > 0) return d->expert_dtype == MOE_BF16;
+    return d->expert_dtype == MOE_BF16 || d->expert_dtype == MOE_FP8_E4M3 || d->expert_dtype == MOE_NVFP4 ||
+           d->expert_dtype == MOE_FP8_B128;
 }
 
 GemmPlan ffn_plan(const moe_dims* d) {
@@ -318,7 +320,8 @@ moe_status run_ffn(const moe_dims* d, const DeviceInfo* dev, const DevCtx& ctx, 
         if (marks) stage_mark(4, st);
         e = launch_grouped_ffn(fp8, w_up, w_down, d->E, d->F, d->H, fw.xp, fw.hb, y_perm, rows, fw.sched, fw.n_sched,
                                fw.done, gp, fp8 ? sc->w_up_scale : nullptr, fp8 ? sc->w_down_scale : nullptr,
-                               fp8 ? sc->x_scale : 1.0f, fp8 ? sc->h_scale : 1.0f, dev->num_sms, withhold, ctx, st);
+                               fp8 ? sc->x_scale : 1.0f, fp8 ? sc->h_scale : 1.0f, dev->num_sms, withhold, ctx, st,
+                               w_up_s, w_down_s, ns);
         if (marks) stage_mark(5, st);
         return cuda_status(e);
     }

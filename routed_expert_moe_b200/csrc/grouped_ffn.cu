@@ -83,6 +83,8 @@ struct FfnArgs {
     const float* sd;
     float x_scale, h_scale;
     int debug_hold;         // 1: the list's first up unit never reports its rows (a wait must expire)
+    int e_shared;           // entries with e >= e_shared are chunk e - e_shared of the shared expert (bf16)
+    int shared_cols;        // shared down weight through the 2-D fallback: chunk j from column j * F
 };
 
 struct FfnMaps {
@@ -90,6 +92,8 @@ struct FfnMaps {
     CUtensorMap ub128, ub64, ub16;    // X_perm [rows][H]
     CUtensorMap da128, da64;          // W_down [E * H][F]
     CUtensorMap db128, db64, db16;    // H [rows][F]
+    CUtensorMap us128, us64;          // shared expert's up weight [n * F][H]
+    CUtensorMap ds128, ds64;          // shared expert's down weight [H][n * F] as {F, H, n} (or {n F, H, 1})
 };
 
 template <bool FP8, bool SMALL>
@@ -189,7 +193,23 @@ __global__ void __launch_bounds__(FF_THREADS, FfnTmem<SMALL>::CTAS)
                 const CUtensorMap* b128 = up ? &maps.ub128 : &maps.db128;
                 const CUtensorMap* b64 = up ? &maps.ub64 : &maps.db64;
                 const CUtensorMap* b16 = up ? &maps.ub16 : &maps.db16;
-                const int ay = sc.x * Nout + mb * FF_BM;
+                int ay = sc.x * Nout + mb * FF_BM;
+                // a chunk j of the shared expert: its up weight's rows j * F + ..., or its down
+                // weight's columns j * F + ... (a 3-D load: (kx, row, j) or (j * F + kx, row, 0))
+                const bool shd = sc.x >= g.e_shared;
+                int sx0 = 0, sz = 0;
+                if (shd) {
+                    const int j = sc.x - g.e_shared;
+                    if (up) {
+                        amap = a_full ? &maps.us128 : &maps.us64;
+                        ay = j * Nout + mb * FF_BM;
+                    } else {
+                        amap = a_full ? &maps.ds128 : &maps.ds64;
+                        ay = mb * FF_BM;
+                        sx0 = g.shared_cols ? j * g.shared_cols : 0;
+                        sz = g.shared_cols ? 0 : j;
+                    }
+                }
                 if (!up) {
                     // the rows of H this unit reads are written by the up units of its entry
                     if (!wait_count(g.done + s_idx, up_target, ctx, abort_flag)) {
@@ -208,7 +228,10 @@ __global__ void __launch_bounds__(FF_THREADS, FfnTmem<SMALL>::CTAS)
                     const int kx = ks * KEL;
                     const uint32_t a_dst = smem_u32(smA + (size_t)stage * FF_A_BYTES);
                     const uint32_t b_dst = smem_u32(smB + (size_t)stage * g.b_stage_bytes);
-                    tma_load_2d(a_dst, amap, fb, kx, ay, pol_w);
+                    if (shd && !up)
+                        tma_load_3d(a_dst, amap, fb, sx0 + kx, ay, sz, pol_w);
+                    else
+                        tma_load_2d(a_dst, amap, fb, kx, ay, pol_w);
                     int row = 0;
                     for (int j = 0; j < n128; ++j, row += 128)
                         tma_load_2d(b_dst + row * FF_ROW_BYTES, b128, fb, kx, sc.y + row, pol_x);
@@ -444,7 +467,8 @@ bool map_ffn(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, bool 
 cudaError_t launch_grouped_ffn(bool fp8, const void* w_up, const void* w_down, int E, int F, int H, const void* xp,
                                void* hb, void* y, int64_t rows, const int4* sched, const int* n_sched, int* done,
                                const GemmPlan& plan, const float* su, const float* sd, float x_scale, float h_scale,
-                               int num_sms, int debug_hold, const DevCtx& ctx, cudaStream_t stream) {
+                               int num_sms, int debug_hold, const DevCtx& ctx, cudaStream_t stream,
+                               const void* w_up_s, const void* w_down_s, int n_shared) {
     if (rows == 0) return cudaSuccess;
     FfnMaps maps;
     if (!map_ffn(&maps.ua128, w_up, (int64_t)E * F, H, fp8, 128) || !map_ffn(&maps.ua64, w_up, (int64_t)E * F, H, fp8, 64) ||
@@ -453,7 +477,30 @@ cudaError_t launch_grouped_ffn(bool fp8, const void* w_up, const void* w_down, i
         !map_ffn(&maps.da64, w_down, (int64_t)E * H, F, fp8, 64) || !map_ffn(&maps.db128, hb, rows, F, fp8, 128) ||
         !map_ffn(&maps.db64, hb, rows, F, fp8, 64) || !map_ffn(&maps.db16, hb, rows, F, fp8, 16))
         return cudaErrorInvalidValue;
+    // the shared expert (bf16 only): n_shared chunks of width F, schedule entries E .. E + n_shared - 1
+    int shared_cols = 0;
+    maps.us128 = maps.ua128;   // read only by units of shared-expert entries
+    maps.us64 = maps.ua64;
+    maps.ds128 = maps.ds64 = maps.da128;
+    if (n_shared > 0) {
+        if (fp8 || !w_up_s || !w_down_s) return cudaErrorInvalidValue;
+        if (!map_ffn(&maps.us128, w_up_s, (int64_t)n_shared * F, H, false, 128) ||
+            !map_ffn(&maps.us64, w_up_s, (int64_t)n_shared * F, H, false, 64))
+            return cudaErrorInvalidValue;
+        bool ok = !shared_map_2d() && make_map_chunks(&maps.ds128, w_down_s, H, F, n_shared, 128) &&
+                  make_map_chunks(&maps.ds64, w_down_s, H, F, n_shared, 64);
+        if (!ok) {
+            // the plain [H][n * F] matrix as {n * F, H, 1}, chunk j from column j * F (a K tail meets
+            // activation columns that read as zero)
+            shared_cols = F;
+            ok = make_map_chunks(&maps.ds128, w_down_s, H, (int64_t)n_shared * F, 1, 128) &&
+                 make_map_chunks(&maps.ds64, w_down_s, H, (int64_t)n_shared * F, 1, 64);
+        }
+        if (!ok) return cudaErrorInvalidValue;
+    }
     FfnArgs g;
+    g.e_shared = n_shared > 0 ? E : 0x7fffffff;
+    g.shared_cols = shared_cols;
     g.sched = sched;
     g.n_sched = n_sched;
     g.done = done;

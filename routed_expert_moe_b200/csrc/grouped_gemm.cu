@@ -344,8 +344,8 @@ static bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t col
 // 3-D bf16 map with dims {d0, d1, d2} (d0 contiguous) and byte strides s1,
 // s2 of dims 1 and 2; box = 128 bytes x box_rows x 1, 128-byte swizzle,
 // out-of-range elements read as zero.
-static bool make_map3(CUtensorMap* m, const void* base, int64_t d0, int64_t d1, int64_t d2, int64_t s1,
-                      int64_t s2, int box_rows) {
+bool make_map3(CUtensorMap* m, const void* base, int64_t d0, int64_t d1, int64_t d2, int64_t s1,
+               int64_t s2, int box_rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[3] = {(cuuint64_t)d0, (cuuint64_t)d1, (cuuint64_t)d2};
@@ -360,8 +360,8 @@ static bool make_map3(CUtensorMap* m, const void* base, int64_t d0, int64_t d1, 
 
 // The column chunks of a row-major bf16 [rows][n * chunk] matrix as {chunk,
 // rows, n}: a box never reads into the next chunk.
-static bool make_map_chunks(CUtensorMap* m, const void* base, int64_t rows, int64_t chunk, int64_t n,
-                            int box_rows) {
+bool make_map_chunks(CUtensorMap* m, const void* base, int64_t rows, int64_t chunk, int64_t n,
+                     int box_rows) {
     return make_map3(m, base, chunk, rows, n, n * chunk * 2, chunk * 2, box_rows);
 }
 

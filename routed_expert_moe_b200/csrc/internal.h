@@ -5,6 +5,7 @@
 // file, so a change to a layout or a signature is seen by all of them.
 #pragma once
 
+#include <cuda.h>
 #include <cstddef>
 #include <cstdint>
 #include <cuda_runtime.h>
@@ -54,10 +55,17 @@ cudaError_t launch_grouped_gemm(bool fp8, bool up, const void* W, int E, int Nou
                                 void* out, const float* w_scale, float in_scale, float out_scale, int num_sms,
                                 int debug_withhold, const DevCtx& ctx, cudaStream_t stream, const void* Ws,
                                 int n_shared);
+// 3-D bf16 maps with a 128-byte swizzle, box {64, box_rows, 1}: {d0, d1, d2} with byte strides s1,
+// s2; make_map_chunks views a row-major [rows][n * chunk] matrix as {chunk, rows, n}, so that a
+// box never reads into the next chunk.
+bool make_map3(CUtensorMap* m, const void* base, int64_t d0, int64_t d1, int64_t d2, int64_t s1, int64_t s2,
+               int box_rows);
+bool make_map_chunks(CUtensorMap* m, const void* base, int64_t rows, int64_t chunk, int64_t n, int box_rows);
 cudaError_t launch_grouped_ffn(bool fp8, const void* w_up, const void* w_down, int E, int F, int H, const void* xp,
                                void* hb, void* y, int64_t rows, const int4* sched, const int* n_sched, int* done,
                                const GemmPlan& plan, const float* su, const float* sd, float x_scale, float h_scale,
-                               int num_sms, int debug_hold, const DevCtx& ctx, cudaStream_t stream);
+                               int num_sms, int debug_hold, const DevCtx& ctx, cudaStream_t stream,
+                               const void* w_up_s = nullptr, const void* w_down_s = nullptr, int n_shared = 0);
 cudaError_t launch_grouped_gemm_pair(bool fp8, bool up, const void* W, int E, int Nout, int Kdim, const void* act,
                                      int64_t rows, const int4* sched, const int* n_sched, int bn, int max_sched,
                                      void* out, const float* w_scale, float in_scale, float out_scale,

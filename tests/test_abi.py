@@ -161,15 +161,15 @@ def test_shared_expert_dims_and_pointers_are_checked_on_the_host(moe):
 def test_forward_launch_count_follows_the_dispatch(moe):
     """Router: one launch up to 256 tokens (expert-split clusters), two up to 1023 (logits, top-K),
     three from 1024 (the tensor-core router); permutation: one block up to 4096 assignments, else three kernels;
-    then the row gather, the expert FFN (one launch without a shared expert, else the two
-    projections) and the combine."""
+    then the row gather, the expert FFN (both projections in one launch; two with the test hook
+    off) and the combine."""
     count = lambda T, **kw: moe.forward_launches(moe.dims(T, 2688, 128, 6, 1856, **kw))
     assert [count(T) for T in (0, 1, 64, 256, 257, 682, 683, 1023, 1024, 4096)] == [0, 5, 5, 5, 6, 6, 8, 8, 9, 9]
-    assert count(64, fp8=True) == count(64, nvfp4=True) == count(64, fp8_b128=True) == 5
-    assert count(64, Fs=1856) == 6
+    assert count(64, fp8=True) == count(64, nvfp4=True) == count(64, fp8_b128=True) == count(64, Fs=1856) == 5
     try:
         moe.debug_set(8, 0)             # the two projections as two launches
         assert count(64) == 6 and count(4096) == 10 and count(64, nvfp4=True) == count(64, fp8_b128=True) == 6
+        assert count(64, Fs=1856) == 6
         moe.debug_set(8, 1)
         moe.debug_set(4, 0)             # never the expert-split clusters
         assert count(64) == 6

@@ -132,3 +132,30 @@ def test_shared_full_size_sampled_outputs(moe, cfg):
     r = oracle.moe_layer_bf16(x, wr, None, W.host_w_up(w, experts=used), W.host_w_down(w, experts=used), w.K,
                               tokens=tok, slot=slot, shared=(W.host_w_up_shared(w), W.host_w_down_shared(w)))
     assert rel_err(host_f64(out)[tok], r["out"]) <= BF16_TOL
+
+
+@pytest.mark.parametrize("w", [SMALL[2], SMALL[4], SMALL[6],
+                               with_shared(W.Workload("T300_E32_K6", 300, 512, 32, 6, 192, seed=17), 384)],
+                         ids=lambda w: w.name)
+def test_shared_one_launch_ffn_equals_two_launches_bitwise(moe, w):
+    """The shared expert's chunks are entries of the one-launch FFN's unit list: the layer output
+    is the same bit for bit as with the two projections in two launches (T = 300: several tiles
+    per chunk)."""
+    h = inputs(w)
+    wu_d, wd_d = dev_bf16(h["wu"]), dev_bf16(h["wd"])
+    su_d, sd_d = dev_bf16(W.host_w_up_shared(w)), dev_bf16(W.host_w_down_shared(w))
+    dims = moe.dims(w.T, w.H, w.E, w.K, w.F, Fs=w.shared)
+    ws = moe.alloc_workspace(dims)
+    x, wr = dev_bf16(h["x"]), dev_bf16(h["wr"])
+    bias = None if h["bias"] is None else dev(h["bias"])
+    outs = []
+    for one in (1, 0):
+        moe.debug_set(8, one)
+        try:
+            out = torch.empty(w.T, w.H, dtype=torch.bfloat16, device="cuda")
+            moe.forward(dims, x, wr, bias, wu_d, wd_d, out, ws, shared=(su_d, sd_d))
+            moe.check_device_error()
+            outs.append(out)
+        finally:
+            moe.debug_set(8, 1)
+    assert torch.equal(outs[0], outs[1])
