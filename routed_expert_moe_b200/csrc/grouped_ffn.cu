@@ -96,7 +96,9 @@ struct FfnMaps {
     CUtensorMap ds128, ds64;          // shared expert's down weight [H][n * F] as {F, H, n} (or {n F, H, 1})
 };
 
-template <bool FP8, bool SMALL>
+// SHD: the schedule may name chunks of the shared expert (a separate instantiation, so that the
+// routed-only kernel's producer keeps its per-stage path: the prefill FFN is bound by its ingest).
+template <bool FP8, bool SMALL, bool SHD>
 __global__ void __launch_bounds__(FF_THREADS, FfnTmem<SMALL>::CTAS)
     grouped_ffn_kernel(const __grid_constant__ FfnMaps maps, FfnArgs g, DevCtx ctx) {
     using TM = FfnTmem<SMALL>;
@@ -196,7 +198,7 @@ __global__ void __launch_bounds__(FF_THREADS, FfnTmem<SMALL>::CTAS)
                 int ay = sc.x * Nout + mb * FF_BM;
                 // a chunk j of the shared expert: its up weight's rows j * F + ..., or its down
                 // weight's columns j * F + ... (a 3-D load: (kx, row, j) or (j * F + kx, row, 0))
-                const bool shd = sc.x >= g.e_shared;
+                const bool shd = SHD && sc.x >= g.e_shared;
                 int sx0 = 0, sz = 0;
                 if (shd) {
                     const int j = sc.x - g.e_shared;
@@ -228,7 +230,7 @@ __global__ void __launch_bounds__(FF_THREADS, FfnTmem<SMALL>::CTAS)
                     const int kx = ks * KEL;
                     const uint32_t a_dst = smem_u32(smA + (size_t)stage * FF_A_BYTES);
                     const uint32_t b_dst = smem_u32(smB + (size_t)stage * g.b_stage_bytes);
-                    if (shd && !up)
+                    if (SHD && shd && !up)
                         tma_load_3d(a_dst, amap, fb, sx0 + kx, ay, sz, pol_w);
                     else
                         tma_load_2d(a_dst, amap, fb, kx, ay, pol_w);
@@ -531,8 +533,10 @@ cudaError_t launch_grouped_ffn(bool fp8, const void* w_up, const void* w_down, i
     const int64_t max_units = (int64_t)plan.max_sched * (g.m_up + g.m_down);
     const int64_t slots = (int64_t)num_sms * (small ? FfnTmem<true>::CTAS : FfnTmem<false>::CTAS);
     const int grid = (int)(max_units < slots ? max_units : slots);
-    auto kfn = small ? (fp8 ? grouped_ffn_kernel<true, true> : grouped_ffn_kernel<false, true>)
-                     : (fp8 ? grouped_ffn_kernel<true, false> : grouped_ffn_kernel<false, false>);
+    const bool shd = n_shared > 0;   // bf16 only
+    auto kfn = shd ? (small ? grouped_ffn_kernel<false, true, true> : grouped_ffn_kernel<false, false, true>)
+               : small ? (fp8 ? grouped_ffn_kernel<true, true, false> : grouped_ffn_kernel<false, true, false>)
+                       : (fp8 ? grouped_ffn_kernel<true, false, false> : grouped_ffn_kernel<false, false, false>);
     // ring, its barriers (full, empty, two tfull, two tempty, drain), the abort flag and TMEM
     // holder, the epilogue's turn-around tiles and the unit queue
     const size_t smem = 1024 + (size_t)ns * stage_bytes + (size_t)(2 * ns + 5) * 8 + 16 + 16 +
