@@ -59,6 +59,48 @@ struct B128Args {
     int debug_withhold;
 };
 
+// The epilogue warps' part of one K stage: add s_w[f, block] times the stage's partial (its first
+// nch 16-column chunks at t_row) to the running fp32 sums of this lane's weight row.
+template <int BN>
+__device__ __forceinline__ void b128_add_block(float (&acc)[BN], uint32_t t_row, int nch, float sw) {
+#pragma unroll
+    for (int c = 0; c < BN / 16; ++c) {
+        if (c < nch) {
+            uint32_t v[16];
+            tmem_ld16(t_row + (uint32_t)(c * 16), v);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) acc[c * 16 + j] = __fmaf_rn(sw, __uint_as_float(v[j]), acc[c * 16 + j]);
+        }
+    }
+}
+
+// After a unit's last block: this lane's feature f for the tile's token rows r < nrows (row0 + r):
+// times the activation scale, then ReLU^2 and the E4M3 code of H / s_h (up, into h [.][ld]) or
+// the bf16 Y (down, into y [.][ld]).
+template <int BN>
+__device__ __forceinline__ void b128_store_unit(const float (&acc)[BN], int nch, int nrows, int64_t row0, int f,
+                                                bool up, float in_scale, float inv_h, uint8_t* h,
+                                                __nv_bfloat16* y, int64_t ld) {
+#pragma unroll
+    for (int c = 0; c < BN / 16; ++c) {
+        if (c >= nch) break;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const int r = c * 16 + j;
+            if (r < nrows) {
+                const float z = __fmul_rn(acc[r], in_scale);
+                const int64_t o = (row0 + r) * ld + f;
+                if (up) {
+                    const float a = z > 0.0f ? __fmul_rn(z, z) : 0.0f;
+                    h[o] = (uint8_t)__nv_cvt_float_to_fp8(__fmul_rn(a, inv_h), __NV_SATFINITE, __NV_E4M3);
+                } else {
+                    y[o] = __float2bfloat16_rn(z);
+                }
+            }
+        }
+    }
+}
+
 template <bool UP, int BN>
 __global__ void __launch_bounds__(GB_THREADS, 1)
     grouped_gemm_b128_kernel(const __grid_constant__ B128Maps maps, B128Args g, DevCtx ctx) {
@@ -215,17 +257,8 @@ __global__ void __launch_bounds__(GB_THREADS, 1)
                     break;
                 }
                 tc_fence_after();
-                const float sw = wrow[ks];
                 const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(ps * BN);
-#pragma unroll
-                for (int c = 0; c < BN / 16; ++c) {
-                    if (c < nch) {
-                        uint32_t v[16];
-                        tmem_ld16(t_row + (uint32_t)(c * 16), v);
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) acc[c * 16 + j] = __fmaf_rn(sw, __uint_as_float(v[j]), acc[c * 16 + j]);
-                    }
-                }
+                b128_add_block<BN>(acc, t_row, nch, wrow[ks]);
                 tc_fence_before();
                 mbar_arrive(smem_u32(&pempty[ps]));
                 if (++ps == GB_NP) {
@@ -234,27 +267,9 @@ __global__ void __launch_bounds__(GB_THREADS, 1)
                 }
             }
             if (!ok) break;
-            if (fvalid) {
-#pragma unroll
-                for (int c = 0; c < BN / 16; ++c) {
-                    if (c >= nch) break;
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int r = c * 16 + j;
-                        if (r < sc.z) {
-                            const float z = __fmul_rn(acc[r], g.in_scale);
-                            const int64_t o = (int64_t)(sc.y + r) * g.out_ld + f;
-                            if constexpr (UP) {
-                                const float a = z > 0.0f ? __fmul_rn(z, z) : 0.0f;
-                                static_cast<uint8_t*>(g.out)[o] =
-                                    (uint8_t)__nv_cvt_float_to_fp8(__fmul_rn(a, inv_out), __NV_SATFINITE, __NV_E4M3);
-                            } else {
-                                static_cast<__nv_bfloat16*>(g.out)[o] = __float2bfloat16_rn(z);
-                            }
-                        }
-                    }
-                }
-            }
+            if (fvalid)
+                b128_store_unit<BN>(acc, nch, sc.z, sc.y, f, UP, g.in_scale, inv_out, static_cast<uint8_t*>(g.out),
+                                    static_cast<__nv_bfloat16*>(g.out), g.out_ld);
         }
     }
 
@@ -526,17 +541,8 @@ __global__ void __launch_bounds__(GB_THREADS, 2)
                     break;
                 }
                 tc_fence_after();
-                const float sw = wrow[ks];
                 const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(ps * BN);
-#pragma unroll
-                for (int c = 0; c < BN / 16; ++c) {
-                    if (c < nch) {
-                        uint32_t vv[16];
-                        tmem_ld16(t_row + (uint32_t)(c * 16), vv);
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) acc[c * 16 + j] = __fmaf_rn(sw, __uint_as_float(vv[j]), acc[c * 16 + j]);
-                    }
-                }
+                b128_add_block<BN>(acc, t_row, nch, wrow[ks]);
                 tc_fence_before();
                 mbar_arrive(smem_u32(&pempty[ps]));
                 if (++ps == GB_NP) {
@@ -545,26 +551,9 @@ __global__ void __launch_bounds__(GB_THREADS, 2)
                 }
             }
             if (!ok) break;
-            if (fvalid) {
-#pragma unroll
-                for (int c = 0; c < BN / 16; ++c) {
-                    if (c >= nch) break;
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int r = c * 16 + j;
-                        if (r < sc.z) {
-                            const float z = __fmul_rn(acc[r], in_scale);
-                            if (up) {
-                                const float a = z > 0.0f ? __fmul_rn(z, z) : 0.0f;
-                                g.hb[(int64_t)(sc.y + r) * g.F + f] =
-                                    (uint8_t)__nv_cvt_float_to_fp8(__fmul_rn(a, inv_h), __NV_SATFINITE, __NV_E4M3);
-                            } else {
-                                static_cast<__nv_bfloat16*>(g.y)[(int64_t)(sc.y + r) * g.H + f] = __float2bfloat16_rn(z);
-                            }
-                        }
-                    }
-                }
-            }
+            if (fvalid)
+                b128_store_unit<BN>(acc, nch, sc.z, sc.y, f, up, in_scale, inv_h, g.hb, static_cast<__nv_bfloat16*>(g.y),
+                                    up ? g.F : g.H);
             if (up) {
                 // this warp's features of H are complete: every lane orders its stores for the async
                 // proxy (the TMA loads of H), the warp barrier orders them before lane 0's release

@@ -296,6 +296,120 @@ __device__ __forceinline__ void mma_fp4(uint32_t d_tmem, uint64_t a, uint64_t b,
         ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb));
 }
 
+// One stage's scale atoms, by thread i of the 128 scale threads: weight row i's 16 scales (four
+// per K block of 64) and token rows i and i + 128, written where tcgen05.cp expects them; rows
+// past the tile's rows (arows weight rows, nrows token rows) get zero scales, and scales of blocks
+// past K (nbk blocks in all) read as zero whatever the padding bytes hold (the H tensor's padding
+// is never written), so that 0 codes times them stay 0.
+__device__ __forceinline__ void fp4_stage_atoms(uint8_t* st, const Fp4Stage& L, int i, int arows, int nrows,
+                                                int nbk, int ks) {
+    const int valid = min(16, max(0, nbk - ks * 16));
+    uint4 km;
+    km.x = valid >= 4 ? 0xFFFFFFFFu : (valid <= 0 ? 0u : (0xFFFFFFFFu >> (8 * (4 - valid))));
+    km.y = valid >= 8 ? 0xFFFFFFFFu : (valid <= 4 ? 0u : (0xFFFFFFFFu >> (8 * (8 - valid))));
+    km.z = valid >= 12 ? 0xFFFFFFFFu : (valid <= 8 ? 0u : (0xFFFFFFFFu >> (8 * (12 - valid))));
+    km.w = valid >= 16 ? 0xFFFFFFFFu : (valid <= 12 ? 0u : (0xFFFFFFFFu >> (8 * (16 - valid))));
+    {
+        uint4 v = i < arows ? *reinterpret_cast<const uint4*>(st + L.a_sc + 16 * i) : make_uint4(0u, 0u, 0u, 0u);
+        v.x &= km.x;
+        v.y &= km.y;
+        v.z &= km.z;
+        v.w &= km.w;
+        uint8_t* at = st + L.a_atoms + 16 * (i % 32) + 4 * (i / 32);
+        *reinterpret_cast<uint32_t*>(at) = v.x;
+        *reinterpret_cast<uint32_t*>(at + FG_ATOM) = v.y;
+        *reinterpret_cast<uint32_t*>(at + 2 * FG_ATOM) = v.z;
+        *reinterpret_cast<uint32_t*>(at + 3 * FG_ATOM) = v.w;
+    }
+    for (int n = i; n < L.nbat * 128; n += 128) {
+        uint4 v = n < nrows ? *reinterpret_cast<const uint4*>(st + L.b_sc + 16 * n) : make_uint4(0u, 0u, 0u, 0u);
+        v.x &= km.x;
+        v.y &= km.y;
+        v.z &= km.z;
+        v.w &= km.w;
+        uint8_t* at = st + L.b_atoms + (n / 128) * FG_ATOM + 16 * (n % 32) + 4 * ((n / 32) % 4);
+        const int kstep = L.nbat * FG_ATOM;
+        *reinterpret_cast<uint32_t*>(at) = v.x;
+        *reinterpret_cast<uint32_t*>(at + kstep) = v.y;
+        *reinterpret_cast<uint32_t*>(at + 2 * kstep) = v.z;
+        *reinterpret_cast<uint32_t*>(at + 3 * kstep) = v.w;
+    }
+}
+
+// One stage's scale copies and block-scaled MMAs (nk of K = 64) into d_tmem: the A atoms to
+// columns sfa + 4 kk, the B atoms to sfb + 8 kk (+ 4 for a second atom); the first MMA of a
+// unit (ks == 0) overwrites the accumulator.
+__device__ __forceinline__ void fp4_stage_mma(uint32_t st, const Fp4Stage& L, int nk, uint32_t sfa, uint32_t sfb,
+                                              uint32_t d_tmem, uint32_t idesc, int ks) {
+    for (int kk = 0; kk < nk; ++kk) {
+        tmem_cp_atom(sfa + 4 * kk, atom_desc(st + L.a_atoms + kk * FG_ATOM));
+        for (int j = 0; j < L.nbat; ++j)
+            tmem_cp_atom(sfb + 8 * kk + 4 * j, atom_desc(st + L.b_atoms + (kk * L.nbat + j) * FG_ATOM));
+    }
+    for (int kk = 0; kk < nk; ++kk)
+        mma_fp4(d_tmem, sw128_desc(st + kk * 32), sw128_desc(st + L.b_codes + kk * 32), idesc, sfa + 4 * kk,
+                sfb + 8 * kk, (ks | kk) != 0 ? 1u : 0u);
+}
+
+// One chunk of a unit's epilogue: the 16 token columns at t_col of this warp's 32 TMEM lanes
+// (features), times `scale`, squared after the ReLU for the up projection, turned around in
+// the warp's shared tile tb so that lane (tj + 16 th) holds features f16 .. f16 + 15 of token
+// row tj; then, if `store`, the up projection quantises them as one NVFP4 block of H (static
+// tensor scale s_h: E4M3 block scale code, E2M1 codes) and the down projection stores bf16 Y.
+__device__ __forceinline__ void fp4_epilogue_chunk(uint32_t t_col, float* tb, int lane, bool up, float scale,
+                                                   bool store, int64_t row, int f16, int n_out, uint8_t* hc,
+                                                   uint8_t* hs, int fsp, __nv_bfloat16* y, float s_h, float r6,
+                                                   float rts) {
+    const int tj = lane & 15, th = lane >> 4;
+    uint32_t v[16];
+    tmem_ld16(t_col, v);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        float z = __fmul_rn(__uint_as_float(v[j]), scale);
+        if (up) z = z > 0.0f ? __fmul_rn(z, z) : 0.0f;   // H = relu(z)^2
+        tb[j * 32 + (((lane >> 2) ^ (j & 7)) << 2) + (lane & 3)] = z;
+    }
+    __syncwarp();
+    float a[16];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const float4 t4 = *reinterpret_cast<const float4*>(tb + tj * 32 + (((4 * th + k) ^ (tj & 7)) << 2));
+        a[4 * k] = t4.x;
+        a[4 * k + 1] = t4.y;
+        a[4 * k + 2] = t4.z;
+        a[4 * k + 3] = t4.w;
+    }
+    __syncwarp();
+    if (!store) return;
+    if (up) {
+        // one block of 16 features, quantised with the static tensor scale s_h
+        float amax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) amax = fmaxf(amax, a[i]);
+        const uint32_t scode = e4m3_code(nv_div(nv_div(amax, 6.0f, r6), s_h, rts));
+        const float e = __fmul_rn(e4m3_value(scode), s_h);
+        uint32_t packed[2] = {0u, 0u};
+        if (e != 0.0f) {
+            const float yv = __frcp_rn(e);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                packed[i / 4] |= e2m1_pack(nv_div(a[2 * i], e, yv), nv_div(a[2 * i + 1], e, yv)) << (8 * (i % 4));
+        }
+        *reinterpret_cast<uint2*>(hc + row * (n_out / 2) + f16 / 2) = make_uint2(packed[0], packed[1]);
+        hs[row * fsp + f16 / 16] = (uint8_t)scode;
+    } else {
+        uint32_t w8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const __nv_bfloat162 p2 = __floats2bfloat162_rn(a[2 * i], a[2 * i + 1]);
+            w8[i] = *reinterpret_cast<const uint32_t*>(&p2);
+        }
+        uint4* d4 = reinterpret_cast<uint4*>(y + row * n_out + f16);
+        d4[0] = make_uint4(w8[0], w8[1], w8[2], w8[3]);
+        d4[1] = make_uint4(w8[4], w8[5], w8[6], w8[7]);
+    }
+}
+
 template <bool UP, bool SMALL>
 __global__ void __launch_bounds__(FG_THREADS, Fp4Tmem<SMALL>::CTAS)
     grouped_gemm_fp4_kernel(const __grid_constant__ Fp4Maps maps, Fp4Args g, DevCtx ctx) {
@@ -419,41 +533,7 @@ __global__ void __launch_bounds__(FG_THREADS, Fp4Tmem<SMALL>::CTAS)
                     break;
                 }
                 uint8_t* st = smem + (size_t)stage * L.bytes;
-                // scales of blocks past K read as zero whatever the padding bytes hold (the H
-                // tensor's padding is never written), so that 0 codes times them stay 0
-                const int valid = min(16, max(0, nbk - ks * 16));
-                uint4 km;
-                km.x = valid >= 4 ? 0xFFFFFFFFu : (valid <= 0 ? 0u : (0xFFFFFFFFu >> (8 * (4 - valid))));
-                km.y = valid >= 8 ? 0xFFFFFFFFu : (valid <= 4 ? 0u : (0xFFFFFFFFu >> (8 * (8 - valid))));
-                km.z = valid >= 12 ? 0xFFFFFFFFu : (valid <= 8 ? 0u : (0xFFFFFFFFu >> (8 * (12 - valid))));
-                km.w = valid >= 16 ? 0xFFFFFFFFu : (valid <= 12 ? 0u : (0xFFFFFFFFu >> (8 * (16 - valid))));
-                {
-                    uint4 v = i < arows ? *reinterpret_cast<const uint4*>(st + L.a_sc + 16 * i)
-                                        : make_uint4(0u, 0u, 0u, 0u);
-                    v.x &= km.x;
-                    v.y &= km.y;
-                    v.z &= km.z;
-                    v.w &= km.w;
-                    uint8_t* at = st + L.a_atoms + 16 * (i % 32) + 4 * (i / 32);
-                    *reinterpret_cast<uint32_t*>(at) = v.x;
-                    *reinterpret_cast<uint32_t*>(at + FG_ATOM) = v.y;
-                    *reinterpret_cast<uint32_t*>(at + 2 * FG_ATOM) = v.z;
-                    *reinterpret_cast<uint32_t*>(at + 3 * FG_ATOM) = v.w;
-                }
-                for (int n = i; n < L.nbat * 128; n += 128) {
-                    uint4 v = n < nrows ? *reinterpret_cast<const uint4*>(st + L.b_sc + 16 * n)
-                                        : make_uint4(0u, 0u, 0u, 0u);
-                    v.x &= km.x;
-                    v.y &= km.y;
-                    v.z &= km.z;
-                    v.w &= km.w;
-                    uint8_t* at = st + L.b_atoms + (n / 128) * FG_ATOM + 16 * (n % 32) + 4 * ((n / 32) % 4);
-                    const int kstep = L.nbat * FG_ATOM;
-                    *reinterpret_cast<uint32_t*>(at) = v.x;
-                    *reinterpret_cast<uint32_t*>(at + kstep) = v.y;
-                    *reinterpret_cast<uint32_t*>(at + 2 * kstep) = v.z;
-                    *reinterpret_cast<uint32_t*>(at + 3 * kstep) = v.w;
-                }
+                fp4_stage_atoms(st, L, i, arows, nrows, nbk, ks);
                 // the atoms become visible to the tensor cores' copies
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 mbar_arrive(smem_u32(&sfready[stage]));
@@ -491,14 +571,7 @@ __global__ void __launch_bounds__(FG_THREADS, Fp4Tmem<SMALL>::CTAS)
                     const uint32_t st = smem_u32(smem + (size_t)stage * L.bytes);
                     const int left = g.Kdim - ks * FG_KR;                 // K values of this stage
                     const int nk = left >= FG_KR ? 4 : (left + 63) / 64;   // MMAs of K = 64
-                    for (int kk = 0; kk < nk; ++kk) {
-                        tmem_cp_atom(sfa + 4 * kk, atom_desc(st + L.a_atoms + kk * FG_ATOM));
-                        for (int j = 0; j < L.nbat; ++j)
-                            tmem_cp_atom(sfb + 8 * kk + 4 * j, atom_desc(st + L.b_atoms + (kk * L.nbat + j) * FG_ATOM));
-                    }
-                    for (int kk = 0; kk < nk; ++kk)
-                        mma_fp4(d_tmem, sw128_desc(st + kk * 32), sw128_desc(st + L.b_codes + kk * 32), idesc,
-                                sfa + 4 * kk, sfb + 8 * kk, (ks | kk) != 0 ? 1u : 0u);
+                    fp4_stage_mma(st, L, nk, sfa, sfb, d_tmem, idesc, ks);
                     issued = true;
                     mma_commit(smem_u32(&empty[stage]));
                     if (++stage == NS) {
@@ -542,58 +615,10 @@ __global__ void __launch_bounds__(FG_THREADS, Fp4Tmem<SMALL>::CTAS)
             const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * TM::ACC);
             const int nchunks = (sc.z + 15) / 16;
             for (int c = 0; c < nchunks; ++c) {
-                uint32_t v[16];
-                tmem_ld16(t_row + (uint32_t)(c * 16), v);
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    float z = __fmul_rn(__uint_as_float(v[j]), scale);
-                    if constexpr (UP) z = z > 0.0f ? __fmul_rn(z, z) : 0.0f;   // H = relu(z)^2
-                    tb[j * 32 + (((lane >> 2) ^ (j & 7)) << 2) + (lane & 3)] = z;
-                }
-                __syncwarp();
-                float a[16];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const float4 t4 = *reinterpret_cast<const float4*>(tb + tj * 32 + (((4 * th + k) ^ (tj & 7)) << 2));
-                    a[4 * k] = t4.x;
-                    a[4 * k + 1] = t4.y;
-                    a[4 * k + 2] = t4.z;
-                    a[4 * k + 3] = t4.w;
-                }
-                __syncwarp();
                 const int r = c * 16 + tj;
-                if (r < sc.z && f16 < g.Nout) {
-                    const int64_t row = sc.y + r;
-                    if constexpr (UP) {
-                        // one block of 16 features, quantised with the static tensor scale s_h
-                        float amax = 0.0f;
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) amax = fmaxf(amax, a[i]);
-                        const uint32_t scode = e4m3_code(nv_div(nv_div(amax, 6.0f, r6), g.out_tscale, rts));
-                        const float e = __fmul_rn(e4m3_value(scode), g.out_tscale);
-                        uint32_t packed[2] = {0u, 0u};
-                        if (e != 0.0f) {
-                            const float y = __frcp_rn(e);
-#pragma unroll
-                            for (int i = 0; i < 8; ++i)
-                                packed[i / 4] |= e2m1_pack(nv_div(a[2 * i], e, y), nv_div(a[2 * i + 1], e, y))
-                                                 << (8 * (i % 4));
-                        }
-                        *reinterpret_cast<uint2*>(static_cast<uint8_t*>(g.out) + row * (g.Nout / 2) + f16 / 2) =
-                            make_uint2(packed[0], packed[1]);
-                        g.out_scale[row * fsp + f16 / 16] = (uint8_t)scode;
-                    } else {
-                        uint32_t w8[8];
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const __nv_bfloat162 p2 = __floats2bfloat162_rn(a[2 * i], a[2 * i + 1]);
-                            w8[i] = *reinterpret_cast<const uint32_t*>(&p2);
-                        }
-                        uint4* d4 = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) + row * g.Nout + f16);
-                        d4[0] = make_uint4(w8[0], w8[1], w8[2], w8[3]);
-                        d4[1] = make_uint4(w8[4], w8[5], w8[6], w8[7]);
-                    }
-                }
+                fp4_epilogue_chunk(t_row + (uint32_t)(c * 16), tb, lane, UP, scale, r < sc.z && f16 < g.Nout,
+                                   sc.y + r, f16, g.Nout, static_cast<uint8_t*>(g.out), g.out_scale, fsp,
+                                   static_cast<__nv_bfloat16*>(g.out), g.out_tscale, r6, rts);
             }
             tc_fence_before();
             mbar_arrive(smem_u32(&tempty[acc]));
@@ -837,39 +862,7 @@ __global__ void __launch_bounds__(FG_THREADS, Fp4Tmem<SMALL>::CTAS)
                     break;
                 }
                 uint8_t* st = smem + (size_t)stage * L.bytes;
-                const int valid = min(16, max(0, nbk - ks * 16));
-                uint4 km;
-                km.x = valid >= 4 ? 0xFFFFFFFFu : (valid <= 0 ? 0u : (0xFFFFFFFFu >> (8 * (4 - valid))));
-                km.y = valid >= 8 ? 0xFFFFFFFFu : (valid <= 4 ? 0u : (0xFFFFFFFFu >> (8 * (8 - valid))));
-                km.z = valid >= 12 ? 0xFFFFFFFFu : (valid <= 8 ? 0u : (0xFFFFFFFFu >> (8 * (12 - valid))));
-                km.w = valid >= 16 ? 0xFFFFFFFFu : (valid <= 12 ? 0u : (0xFFFFFFFFu >> (8 * (16 - valid))));
-                {
-                    uint4 v = i < arows ? *reinterpret_cast<const uint4*>(st + L.a_sc + 16 * i)
-                                        : make_uint4(0u, 0u, 0u, 0u);
-                    v.x &= km.x;
-                    v.y &= km.y;
-                    v.z &= km.z;
-                    v.w &= km.w;
-                    uint8_t* at = st + L.a_atoms + 16 * (i % 32) + 4 * (i / 32);
-                    *reinterpret_cast<uint32_t*>(at) = v.x;
-                    *reinterpret_cast<uint32_t*>(at + FG_ATOM) = v.y;
-                    *reinterpret_cast<uint32_t*>(at + 2 * FG_ATOM) = v.z;
-                    *reinterpret_cast<uint32_t*>(at + 3 * FG_ATOM) = v.w;
-                }
-                for (int n = i; n < L.nbat * 128; n += 128) {
-                    uint4 v = n < nrows ? *reinterpret_cast<const uint4*>(st + L.b_sc + 16 * n)
-                                        : make_uint4(0u, 0u, 0u, 0u);
-                    v.x &= km.x;
-                    v.y &= km.y;
-                    v.z &= km.z;
-                    v.w &= km.w;
-                    uint8_t* at = st + L.b_atoms + (n / 128) * FG_ATOM + 16 * (n % 32) + 4 * ((n / 32) % 4);
-                    const int kstep = L.nbat * FG_ATOM;
-                    *reinterpret_cast<uint32_t*>(at) = v.x;
-                    *reinterpret_cast<uint32_t*>(at + kstep) = v.y;
-                    *reinterpret_cast<uint32_t*>(at + 2 * kstep) = v.z;
-                    *reinterpret_cast<uint32_t*>(at + 3 * kstep) = v.w;
-                }
+                fp4_stage_atoms(st, L, i, arows, nrows, nbk, ks);
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 mbar_arrive(smem_u32(&sfready[stage]));
                 if (++stage == NS) {
@@ -920,14 +913,7 @@ __global__ void __launch_bounds__(FG_THREADS, Fp4Tmem<SMALL>::CTAS)
                     const uint32_t st = smem_u32(smem + (size_t)stage * L.bytes);
                     const int left = un.Kdim - ks * FG_KR;
                     const int nk = left >= FG_KR ? 4 : (left + 63) / 64;
-                    for (int kk = 0; kk < nk; ++kk) {
-                        tmem_cp_atom(sfa + 4 * kk, atom_desc(st + L.a_atoms + kk * FG_ATOM));
-                        for (int j = 0; j < L.nbat; ++j)
-                            tmem_cp_atom(sfb + 8 * kk + 4 * j, atom_desc(st + L.b_atoms + (kk * L.nbat + j) * FG_ATOM));
-                    }
-                    for (int kk = 0; kk < nk; ++kk)
-                        mma_fp4(d_tmem, sw128_desc(st + kk * 32), sw128_desc(st + L.b_codes + kk * 32), idesc,
-                                sfa + 4 * kk, sfb + 8 * kk, (ks | kk) != 0 ? 1u : 0u);
+                    fp4_stage_mma(st, L, nk, sfa, sfb, d_tmem, idesc, ks);
                     issued = true;
                     mma_commit(smem_u32(&empty[stage]));
                     if (++stage == NS) {
@@ -981,57 +967,10 @@ __global__ void __launch_bounds__(FG_THREADS, Fp4Tmem<SMALL>::CTAS)
             const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * TM::ACC);
             const int nchunks = (sc.z + 15) / 16;
             for (int c = 0; c < nchunks; ++c) {
-                uint32_t v[16];
-                tmem_ld16(t_row + (uint32_t)(c * 16), v);
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    float z = __fmul_rn(__uint_as_float(v[j]), scale);
-                    if (un.up) z = z > 0.0f ? __fmul_rn(z, z) : 0.0f;   // H = relu(z)^2
-                    tb[j * 32 + (((lane >> 2) ^ (j & 7)) << 2) + (lane & 3)] = z;
-                }
-                __syncwarp();
-                float a[16];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const float4 t4 = *reinterpret_cast<const float4*>(tb + tj * 32 + (((4 * th + k) ^ (tj & 7)) << 2));
-                    a[4 * k] = t4.x;
-                    a[4 * k + 1] = t4.y;
-                    a[4 * k + 2] = t4.z;
-                    a[4 * k + 3] = t4.w;
-                }
-                __syncwarp();
                 const int r = c * 16 + tj;
-                if (r < sc.z && f16 < un.Nout) {
-                    const int64_t row = sc.y + r;
-                    if (un.up) {
-                        // one block of 16 features, quantised with the static tensor scale s_h
-                        float amax = 0.0f;
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) amax = fmaxf(amax, a[i]);
-                        const uint32_t scode = e4m3_code(nv_div(nv_div(amax, 6.0f, r6), g.h_tscale, rts));
-                        const float e = __fmul_rn(e4m3_value(scode), g.h_tscale);
-                        uint32_t packed[2] = {0u, 0u};
-                        if (e != 0.0f) {
-                            const float y = __frcp_rn(e);
-#pragma unroll
-                            for (int i = 0; i < 8; ++i)
-                                packed[i / 4] |= e2m1_pack(nv_div(a[2 * i], e, y), nv_div(a[2 * i + 1], e, y))
-                                                 << (8 * (i % 4));
-                        }
-                        *reinterpret_cast<uint2*>(g.hb + row * (g.F / 2) + f16 / 2) = make_uint2(packed[0], packed[1]);
-                        g.hb_block[row * fsp + f16 / 16] = (uint8_t)scode;
-                    } else {
-                        uint32_t w8[8];
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const __nv_bfloat162 p2 = __floats2bfloat162_rn(a[2 * i], a[2 * i + 1]);
-                            w8[i] = *reinterpret_cast<const uint32_t*>(&p2);
-                        }
-                        uint4* d4 = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.y) + row * g.H + f16);
-                        d4[0] = make_uint4(w8[0], w8[1], w8[2], w8[3]);
-                        d4[1] = make_uint4(w8[4], w8[5], w8[6], w8[7]);
-                    }
-                }
+                fp4_epilogue_chunk(t_row + (uint32_t)(c * 16), tb, lane, un.up, scale, r < sc.z && f16 < un.Nout,
+                                   sc.y + r, f16, un.Nout, g.hb, g.hb_block, fsp, static_cast<__nv_bfloat16*>(g.y),
+                                   g.h_tscale, r6, rts);
             }
             tc_fence_before();
             mbar_arrive(smem_u32(&tempty[acc]));
