@@ -415,8 +415,13 @@ def gemm_pair(sim, units, k_stages, NS, n_epi=4):
 
 # ----------------------------------------------------------------------------- one-launch FFN (grouped_ffn.cu)
 
-def ffn_fused(sim, n_ctas, entries, m_up, m_down, k_up, k_down, NS, n_epi=4, UQ=4, plant=None):
-    """grouped_ffn_kernel on n_ctas CTAs.  The units are the list [up units (entry, block)] +
+def ffn_fused(sim, n_ctas, entries, m_up, m_down, k_up, k_down, NS, n_epi=4, UQ=4, plant=None, form="bf16",
+              n_sc=4, NP=4):
+    """The one-launch FFNs on n_ctas CTAs (form "bf16": grouped_ffn_kernel; "fp4":
+    grouped_ffn_fp4_kernel, whose stages also pass through the n_sc scale warps -- full, then
+    sfready, then the MMA -- and whose scale warps read the unit queue too; "b128":
+    grouped_ffn_b128_kernel, whose MMA writes one of NP TMEM partial slots per stage, read by
+    every epilogue warp per stage instead of one accumulator per unit).  The units are the list [up units (entry, block)] +
     [down units]; each CTA's producer claims the next unit from a global counter (one atomic
     step, the next claim taken while the current unit loads) and publishes it in a UQ-slot
     queue in shared memory (uq_full: 1 arrival; uq_empty: the MMA thread and the n_epi epilogue
@@ -433,10 +438,15 @@ def ffn_fused(sim, n_ctas, entries, m_up, m_down, k_up, k_down, NS, n_epi=4, UQ=
     stored = [0] * entries
     target = n_epi * m_up if plant != "early_read" else n_epi * (m_up - 1)   # planted: one up unit short
     uq_readers = 1 + n_epi if plant != "queue_short" else 1                 # planted: only the MMA frees a slot
+    if form == "fp4" and plant not in ("queue_short", "queue_no_scale"):
+        uq_readers += n_sc
 
     def cta(c):
         full, empty = [Bar(1) for _ in range(NS)], [Bar(1) for _ in range(NS)]
         tfull, tempty = [Bar(1) for _ in range(2)], [Bar(n_epi) for _ in range(2)]
+        sfready, atoms = [Bar(n_sc) for _ in range(NS)], [[None] * n_sc for _ in range(NS)]
+        pfull, pempty = [Bar(1) for _ in range(NP)], [Bar(n_epi) for _ in range(NP)]
+        part, preaders = [None] * NP, [n_epi] * NP
         uq_full, uq_empty = [Bar(1) for _ in range(UQ)], [Bar(uq_readers) for _ in range(UQ)]
         uq = [None] * UQ
         published = []                      # the units this CTA claimed, in order
@@ -490,7 +500,7 @@ def ffn_fused(sim, n_ctas, entries, m_up, m_down, k_up, k_down, NS, n_epi=4, UQ=
                         st, ph = 0, ph ^ 1
 
         def mma():
-            st, ph, acc, aph, q, qph, i = 0, 0, 0, 0, 0, 0, 0
+            st, ph, acc, aph, q, qph, i, ps, pph = 0, 0, 0, 0, 0, 0, 0, 0, 0
             while True:
                 yield (lambda q_=q, p=qph: uq_full[q_].passed(p))
                 u = take("MMA", i, q)
@@ -501,18 +511,39 @@ def ffn_fused(sim, n_ctas, entries, m_up, m_down, k_up, k_down, NS, n_epi=4, UQ=
                 if u < 0:
                     return
                 kind, s = units[u]
-                yield (lambda a=acc, p=aph: tempty[a].passed(p ^ 1))
+                if form != "b128":
+                    yield (lambda a=acc, p=aph: tempty[a].passed(p ^ 1))
                 for ks in range(k_up if kind == "up" else k_down):
-                    yield (lambda s_=st, p=ph: full[s_].passed(p))
+                    if form == "fp4":
+                        yield (lambda s_=st, p=ph: sfready[s_].passed(p))
+                        check(all(t == (c, u, ks) for t in atoms[st]), f"CTA {c}: MMA copied atoms {atoms[st]}")
+                    else:
+                        yield (lambda s_=st, p=ph: full[s_].passed(p))
                     check(smem[st] == (c, u, ks), f"CTA {c}: MMA read stage {st} holding {smem[st]}")
+                    if form == "b128":
+                        yield (lambda q_=ps, p=pph: pempty[q_].passed(p ^ 1))
+                        check(preaders[ps] == n_epi, f"CTA {c}: MMA wrote partial slot {ps} while it was read")
+                        preaders[ps] = 0
 
-                    def mma_done(s_=st):
-                        fresh[s_] = False
-                        empty[s_].arrive()
-                    sim.post(("tc", c), mma_done)
+                        def part_done(s_=st, q_=ps, tag=(u, ks)):
+                            fresh[s_] = False
+                            part[q_] = tag
+                            empty[s_].arrive()
+                            pfull[q_].arrive()
+                        sim.post(("tc", c), part_done)
+                        ps += 1
+                        if ps == NP:
+                            ps, pph = 0, pph ^ 1
+                    else:
+                        def mma_done(s_=st):
+                            fresh[s_] = False
+                            empty[s_].arrive()
+                        sim.post(("tc", c), mma_done)
                     st += 1
                     if st == NS:
                         st, ph = 0, ph ^ 1
+                if form == "b128":
+                    continue
 
                 def acc_done(a=acc, u=u):
                     tmem[a] = u
@@ -522,8 +553,29 @@ def ffn_fused(sim, n_ctas, entries, m_up, m_down, k_up, k_down, NS, n_epi=4, UQ=
                 if acc == 2:
                     acc, aph = 0, aph ^ 1
 
+        def scale_warp(j):
+            st, ph, q, qph, i = 0, 0, 0, 0, 0
+            while True:
+                yield (lambda q_=q, p=qph: uq_full[q_].passed(p))
+                u = take(f"scale warp {j}", i, q)
+                i += 1
+                q += 1
+                if q == UQ:
+                    q, qph = 0, qph ^ 1
+                if u < 0:
+                    return
+                kind, s = units[u]
+                for ks in range(k_up if kind == "up" else k_down):
+                    yield (lambda s_=st, p=ph: full[s_].passed(p))
+                    check(smem[st] == (c, u, ks), f"CTA {c}: scale warp {j} read stage {st} holding {smem[st]}")
+                    atoms[st][j] = (c, u, ks)
+                    sfready[st].arrive()
+                    st += 1
+                    if st == NS:
+                        st, ph = 0, ph ^ 1
+
         def epilogue(w):
-            acc, aph, q, qph, i = 0, 0, 0, 0, 0
+            acc, aph, q, qph, i, ps, pph = 0, 0, 0, 0, 0, 0, 0
             while True:
                 yield (lambda q_=q, p=qph: uq_full[q_].passed(p))
                 u = take(f"epilogue warp {w}", i, q, arrive=plant != "queue_short")
@@ -534,9 +586,19 @@ def ffn_fused(sim, n_ctas, entries, m_up, m_down, k_up, k_down, NS, n_epi=4, UQ=
                 if u < 0:
                     return
                 kind, s = units[u]
-                yield (lambda a=acc, p=aph: tfull[a].passed(p))
-                check(tmem[acc] == u, f"CTA {c}: epilogue read accumulator {acc} holding {tmem[acc]}")
-                tempty[acc].arrive()
+                if form == "b128":
+                    for ks in range(k_up if kind == "up" else k_down):
+                        yield (lambda q_=ps, p=pph: pfull[q_].passed(p))
+                        check(part[ps] == (u, ks), f"CTA {c}: epilogue read partial slot {ps} holding {part[ps]}")
+                        preaders[ps] += 1
+                        pempty[ps].arrive()
+                        ps += 1
+                        if ps == NP:
+                            ps, pph = 0, pph ^ 1
+                else:
+                    yield (lambda a=acc, p=aph: tfull[a].passed(p))
+                    check(tmem[acc] == u, f"CTA {c}: epilogue read accumulator {acc} holding {tmem[acc]}")
+                    tempty[acc].arrive()
                 if kind == "up":
                     stored[s] += 1           # this warp's rows of H are stored (and fenced)
                     yield (lambda: True)
@@ -549,6 +611,9 @@ def ffn_fused(sim, n_ctas, entries, m_up, m_down, k_up, k_down, NS, n_epi=4, UQ=
         sim.role(f"mma{c}", mma())
         for w in range(n_epi):
             sim.role(f"epilogue{c}.{w}", epilogue(w))
+        if form == "fp4":
+            for j in range(n_sc):
+                sim.role(f"scale{c}.{j}", scale_warp(j))
 
     for c in range(n_ctas):
         cta(c)
@@ -565,6 +630,32 @@ def test_one_launch_ffn_protocol(n_ctas, entries, m_up, m_down, k_up, k_down, NS
         sim = Sim(seed)
         claimed_all = ffn_fused(sim, n_ctas, entries, m_up, m_down, k_up, k_down, NS)
         assert sim.run() == "done" and claimed_all()
+
+
+@pytest.mark.parametrize("form", ["fp4", "b128"])
+@pytest.mark.parametrize("n_ctas,entries,m_up,m_down,k_up,k_down,NS",
+                         [(3, 4, 3, 4, 4, 3, 3), (2, 5, 2, 3, 3, 2, 2), (4, 3, 2, 2, 2, 2, 4)])
+def test_one_launch_ffn_protocol_nvfp4_and_b128(form, n_ctas, entries, m_up, m_down, k_up, k_down, NS):
+    """The NVFP4 one-launch kernel (the scale warps read the unit queue and hand each stage on)
+    and the FP8_B128 one (per-stage partial slots instead of per-unit accumulators)."""
+    for seed in range(20):
+        sim = Sim(seed)
+        claimed_all = ffn_fused(sim, n_ctas, entries, m_up, m_down, k_up, k_down, NS, form=form)
+        assert sim.run() == "done" and claimed_all()
+
+
+def test_a_unit_queue_not_waiting_for_the_scale_warps_is_caught():
+    """Planted: the NVFP4 queue slots count only the MMA thread and the epilogue warps, so the
+    producer may overwrite a slot a scale warp has not read yet."""
+    caught = 0
+    for seed in range(40):
+        sim = Sim(seed)
+        ffn_fused(sim, 2, 6, 3, 3, 1, 1, 2, UQ=2, plant="queue_no_scale", form="fp4")
+        try:
+            sim.run()
+        except Violation:
+            caught += 1
+    assert caught > 0
 
 
 def test_a_unit_queue_freed_by_the_mma_alone_is_caught():
