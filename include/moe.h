@@ -198,7 +198,7 @@ moe_status moe_combine(const moe_dims* d, const void* y_perm, const int32_t* inv
  * intermediates in the workspace.  topk_idx / topk_w ([T][K]) may be NULL;
  * when given they receive the routing.  out may alias residual.  With
  * d->Fs > 0 the shared expert (w_up_shared [Fs][H], w_down_shared [H][Fs],
- * bf16) runs in the same grouped GEMM launches as the routed experts and its
+ * bf16) runs in the same expert FFN launch as the routed experts and its
  * output joins the combine with weight 1; both pointers NULL when Fs = 0. */
 moe_status moe_forward(const moe_dims* d, const void* x, const void* w_router, const float* bias,
                        const void* w_up, const void* w_down, const void* w_up_shared,
@@ -345,10 +345,10 @@ moe_status moe_set_stage_events(void* const* events, int32_t n);
  * on the device for it; what = 7: value 1 reads the shared expert's down
  * weight through the fallback map (the plain [H][Fs] matrix, chunk j from
  * column j*F) instead of the chunked 3-D view, 0 (the default) restores the
- * view; what = 8: value 1 (the default) runs both expert projections of bf16,
- * E4M3 and NVFP4 layers without a shared expert in one launch (the down units
- * of a schedule entry start once that entry's up units have reported), 0 as
- * two launches.  Other `what`: MOE_EINVAL. */
+ * view; what = 8: value 1 (the default) runs both expert projections in one
+ * launch, for every expert format and with a shared expert (the down units of
+ * a schedule entry start once that entry's up units have reported), 0 as two
+ * launches.  Other `what`: MOE_EINVAL. */
 moe_status moe_debug_set(int32_t what, int64_t value);
 
 #ifdef __cplusplus
