@@ -633,7 +633,7 @@ def _fused_entry(wl, stages, touched, peaks, peak_kind, workload):
     """Roofline of the one-launch expert FFN (both projections): the bytes and flops of the up and
     the down projection together, over the launch's duration."""
     H, F, T, K = wl.H, wl.F, wl.T, wl.K
-    rows = T * K
+    rows = T * (K + wl.shared // F)    # a shared expert's Fs/F chunks add T rows each (touched counts them)
     fp8 = wl.fp8 or wl.fp8_b128
     es = 1 if fp8 else 2
     ms = stages["expert_ffn"]

@@ -192,3 +192,13 @@ def test_one_launch_fp8_b128_ffn_counts_padded_codes_and_block_scales():
                                                  + rows * H + 2 * rows * F + rows * H * 2)
     p = bench.roofline_entry(W.WORKLOADS[10], st, 128, PEAKS, "measured", "prefill_fp8_b128")
     assert p["bound"] == "tensor" and p["peak"] == 2 * PEAKS["bf16_tflops"]
+
+
+def test_one_launch_ffn_with_a_shared_expert_counts_its_chunks():
+    """With a shared expert of Fs = F the one-launch FFN also streams that expert's weights (one
+    more 'touched' expert) and T more rows through both projections."""
+    st = {"expert_ffn": 0.4}
+    base = bench.roofline_entry(W.WORKLOADS[1], st, 121, PEAKS, "measured", "decode")
+    sh = bench.roofline_entry(W.WORKLOADS[7], st, 121, PEAKS, "measured", "decode_shared")
+    assert sh["algorithmic_bytes_per_launch"] - base["algorithmic_bytes_per_launch"] == 2 * F * H * 2 + 64 * (H + F) * 2 * 2
+    assert sh["algorithmic_flops_per_launch"] == 4.0 * 64 * 7 * F * H
