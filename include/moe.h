@@ -348,7 +348,11 @@ moe_status moe_set_stage_events(void* const* events, int32_t n);
  * view; what = 8: value 1 (the default) runs both expert projections in one
  * launch, for every expert format and with a shared expert (the down units of
  * a schedule entry start once that entry's up units have reported), 0 as two
- * launches.  Other `what`: MOE_EINVAL. */
+ * launches; what = 9: bytes of the up bank's start (its first experts'
+ * weights, which the FFN's first units read) that the small-batch router
+ * prefetches into L2 from the clusters the device fits beside the batch's
+ * (value 0: none; value < 0 restores the default of 48 MiB; clamped to the
+ * bank's size); the prefetch changes no result.  Other `what`: MOE_EINVAL. */
 moe_status moe_debug_set(int32_t what, int64_t value);
 
 #ifdef __cplusplus

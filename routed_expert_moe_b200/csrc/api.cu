@@ -1,6 +1,7 @@
 // C ABI (include/moe.h): argument validation, workspace layout, per-device
 // setup and the launch sequence of each entry point.  All computation is in
 // the kernels of route.cu, permute.cu, grouped_gemm.cu and combine.cu.
+#include <algorithm>
 #include <atomic>
 #include <cstdint>
 #include <cstring>
@@ -24,6 +25,12 @@ std::atomic<int> g_gemm_pair{0};
 std::atomic<int> g_fused_ffn{1};   // 1: both bf16/E4M3 projections in one launch (grouped_ffn.cu)
 std::atomic<int> g_pdl{1};
 std::atomic<int> g_shared_2d{0};   // 1: the shared down weight through its 2-D fallback map
+// Bytes of the up weight bank (its first experts: the FFN's first units) that the decode
+// router's spare clusters prefetch into L2 while routing.  On B200 at T=64 (bf16): the FFN
+// 347 -> 340 us and the router 20.3 -> 20.8 us at 48 MB; 64 MB and 96 MB slow the router's
+// own loads more (22.0, 22.6 us) than they save.
+constexpr int64_t kL2WarmDefault = (int64_t)48 << 20;
+std::atomic<int64_t> g_l2_warm{kL2WarmDefault};
 void* g_stage_events[MOE_STAGE_EVENTS] = {};
 std::atomic<int> g_stage_events_on{0};
 
@@ -138,11 +145,6 @@ struct ForwardWs {
     void* y_perm;
 };
 
-// Plan of the expert FFN: one tile schedule for every expert dtype (FP8_B128
-// caps a tile at 128 token rows: its epilogue keeps a tile's sums in registers;
-// NVFP4 at 224: its accumulators share TMEM with the scale factors),
-// plus the shared expert's entries (ns chunks of T rows, cut into tiles of at
-// most bn).
 // Whether the expert FFN runs as one launch (every expert format; a shared expert, which only
 // bf16 layers take, adds its chunks as entries of the same unit list).
 bool fused_ffn(const moe_dims* d) {
@@ -152,6 +154,11 @@ bool fused_ffn(const moe_dims* d) {
            d->expert_dtype == MOE_FP8_B128;
 }
 
+// Plan of the expert FFN: one tile schedule for every expert dtype (FP8_B128
+// caps a tile at 128 token rows: its epilogue keeps a tile's sums in registers;
+// NVFP4 at 224: its accumulators share TMEM with the scale factors),
+// plus the shared expert's entries (ns chunks of T rows, cut into tiles of at
+// most bn).
 GemmPlan ffn_plan(const moe_dims* d) {
     GemmPlan gp = gemm_plan(d->T, d->K, d->E);
     // The one-launch FFN takes sparse batches (experts average under 128 rows) in tiles of at
@@ -531,9 +538,13 @@ moe_status moe_forward(const moe_dims* d, const void* x, const void* w_router, c
     Carve cr;
     RouteWs rw = carve_route(cr, sbase, d, rp);
     stage_mark(0, st);
+    // the up bank's leading bytes (expert 0 first, in every format's layout), bounded by its size
+    const int64_t up_bytes = (int64_t)d->E * d->F * d->H / (d->expert_dtype == MOE_NVFP4 ? 2 : 1) *
+                             (d->expert_dtype == MOE_BF16 ? 2 : 1);
+    const int64_t warm = std::min(g_l2_warm.load(), up_bytes);
     cudaError_t e = launch_route(static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(w_router), bias, d->T,
                                  d->H, d->E, d->K, idx, w, rw.P, rw.xn2, rw.wn2, rp, ctx, st,
-                                 g_stage_events_on.load() ? mark_stage1 : nullptr);
+                                 g_stage_events_on.load() ? mark_stage1 : nullptr, w_up, warm);
     if (e != cudaSuccess) return cuda_status(e);
 
     const GemmPlan gp = ffn_plan(d);
@@ -708,6 +719,10 @@ moe_status moe_debug_set(int32_t what, int64_t value) {
     }
     if (what == 8) {
         g_fused_ffn.store(value ? 1 : 0);
+        return MOE_OK;
+    }
+    if (what == 9) {
+        g_l2_warm.store(value < 0 ? kL2WarmDefault : value);
         return MOE_OK;
     }
     if (what == 5) {

@@ -29,7 +29,8 @@ cudaError_t launch_route_tc(const uint16_t* x, const uint16_t* wr, const float* 
 cudaError_t launch_route(const uint16_t* x, const uint16_t* wr, const float* bias, int64_t T, int H, int E,
                          int K, int32_t* idx, float* w, double* P, double* xn2, double* wn2,
                          const RouterPlan& plan, const DevCtx& ctx, cudaStream_t stream,
-                         void (*between)(cudaStream_t) = nullptr);
+                         void (*between)(cudaStream_t) = nullptr, const void* warm = nullptr,
+                         int64_t warm_bytes = 0);
 cudaError_t launch_permute(const int32_t* idx, int64_t n, int K, int E, int32_t* counts, int32_t* offsets,
                            int32_t* perm_src, int32_t* inv_row, int4* sched, int* n_sched, int bn, int ns,
                            int* scratch, const DevCtx& ctx, cudaStream_t stream);

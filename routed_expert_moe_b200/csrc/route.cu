@@ -306,7 +306,11 @@ struct RouterSmallArgs {
     int H, E, K;
     int32_t* idx;
     float* w;
+    const uint8_t* warm;    // bytes the next kernels read first (null: none): prefetched into L2
+    int64_t warm_bytes;     // a multiple of 16 (0 when warm is null)
 };
+
+constexpr int64_t RS_WARM_PIECE = 32 * 1024;   // bytes of one L2 prefetch
 
 __host__ __device__ constexpr int rs_epc(int E) { return (E + RS_CLUSTER - 1) / RS_CLUSTER; }
 __host__ __device__ constexpr size_t rs_align(size_t v) { return (v + 15) & ~size_t(15); }
@@ -336,6 +340,23 @@ template <int TB>
 __global__ void __cluster_dims__(RS_CLUSTER, 1, 1) __launch_bounds__(RS_THREADS)
     router_small_kernel(RouterSmallArgs a, DevCtx ctx) {
     pdl_enter();
+    // Clusters past the batch's groups only warm L2: they prefetch the bytes the expert FFN
+    // reads first (its first experts' up weights) while the router and the permutation run,
+    // when the memory system is otherwise idle.  They run on SMs the router leaves free, so
+    // that no routing warp waits on the prefetches' issue; pieces of 32 KB, strided over their
+    // lanes.
+    const int64_t n_groups = (a.T + TB - 1) / TB;
+    if ((int64_t)(blockIdx.x / RS_CLUSTER) >= n_groups) {
+        const int64_t first = n_groups * RS_CLUSTER * 32;
+        const int64_t pieces = (a.warm_bytes + RS_WARM_PIECE - 1) / RS_WARM_PIECE;
+        const int64_t stride = ((int64_t)gridDim.x - n_groups * RS_CLUSTER) * 32;
+        for (int64_t q = (int64_t)blockIdx.x * 32 + threadIdx.x % 32 - first; threadIdx.x < 32 && q < pieces;
+             q += stride) {
+            const int64_t off = q * RS_WARM_PIECE;
+            bulk_prefetch_l2(a.warm + off, (uint32_t)min(RS_WARM_PIECE, a.warm_bytes - off));
+        }
+        return;
+    }
     namespace cg = cooperative_groups;
     extern __shared__ __align__(16) unsigned char rs_smem[];
     const int H = a.H, E = a.E;
@@ -998,7 +1019,10 @@ static cudaError_t launch_router_small(const RouterSmallArgs& ra, const DevCtx& 
     cudaError_t err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     const unsigned groups = (unsigned)((ra.T + TB - 1) / TB);
-    return launch_k(kfn, dim3(groups * RS_CLUSTER), dim3(RS_THREADS), smem, stream, ra, ctx);
+    // clusters that only warm L2: those the device still fits beside the batch's groups
+    const int fit = ra.warm ? router_small_max_clusters(TB, ra.H, ra.E) : 0;
+    const unsigned warm = fit > (int)groups ? (unsigned)fit - groups : 0;
+    return launch_k(kfn, dim3((groups + warm) * RS_CLUSTER), dim3(RS_THREADS), smem, stream, ra, ctx);
 }
 
 // Kernel launches launch_route makes for these sizes under the current hooks:
@@ -1015,12 +1039,14 @@ int route_launches(int64_t T, int H, int E) {
 cudaError_t launch_route(const uint16_t* x, const uint16_t* wr, const float* bias, int64_t T, int H,
                          int E, int K, int32_t* idx, float* w, double* P, double* xn2, double* wn2,
                          const RouterPlan& plan, const DevCtx& ctx, cudaStream_t stream,
-                         void (*between)(cudaStream_t)) {
+                         void (*between)(cudaStream_t), const void* warm, int64_t warm_bytes) {
     if (T == 0) return cudaSuccess;
     if (plan.tc) return launch_route_tc(x, wr, bias, T, H, E, K, idx, w, P, plan.num_sms, ctx, stream, between);
     const int tb = router_small_tb(T, H, E, true);
     if (tb > 0) {
-        RouterSmallArgs ra{x, wr, bias, T, H, E, K, idx, w};
+        RouterSmallArgs ra{x, wr, bias, T, H, E, K, idx, w, static_cast<const uint8_t*>(warm),
+                           warm ? (warm_bytes & ~(int64_t)15) : 0};
+        if (ra.warm_bytes <= 0) ra.warm = nullptr;
         const cudaError_t err = tb == 4 ? launch_router_small<4>(ra, ctx, stream)
                                         : launch_router_small<8>(ra, ctx, stream);
         if (err == cudaSuccess && between) between(stream);   // one launch: nothing between

@@ -86,6 +86,8 @@ def test_null_and_missing_arguments(moe):
     assert lib.moe_rmsnorm(4, 2690, 1e-5, None, None, None) == moe.MOE_EINVAL
     assert lib.moe_quantize_fp8(-1, 4, None, None, None, None) == moe.MOE_EINVAL
     assert lib.moe_debug_set(99, 0) == moe.MOE_EINVAL
+    assert lib.moe_debug_set(9, 0) == moe.MOE_OK       # router L2 prefetch off
+    assert lib.moe_debug_set(9, -1) == moe.MOE_OK      # its default
     assert lib.moe_gather_rows(-1, 4, 256, 1, None, None, None, None) == moe.MOE_EINVAL
     assert lib.moe_gather_rows(4, 4, 260, 1, None, None, None, None) == moe.MOE_EINVAL   # H % 8
     assert lib.moe_gather_rows(4, 4, 256, 0, None, None, None, None) == moe.MOE_EINVAL   # K < 1

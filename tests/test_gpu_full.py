@@ -293,6 +293,31 @@ def test_one_launch_ffn_equals_two_launches_bitwise(moe, w, fp8, with_residual):
     assert torch.equal(outs[0], outs[1])
 
 
+@pytest.mark.parametrize("w", [W.WORKLOADS[0], W.WORKLOADS[1]], ids=lambda w: w.name)
+def test_router_l2_prefetch_changes_no_result(moe, w):
+    """The decode router's L2 prefetch of the up bank's leading bytes is a hint: off, a ragged
+    size (48 bytes, one 32 KB piece and 16 bytes), the default and a size past the bank's end
+    (clamped to it) give the same routing and layer output bit for bit."""
+    h = inputs(w)
+    d = device_inputs(h)
+    dims = moe.dims(w.T, w.H, w.E, w.K, w.F)
+    ws = moe.alloc_workspace(dims)
+    runs = []
+    for warm in (0, 48, 32 * 1024 + 16, -1, 1 << 40):
+        moe.debug_set(9, warm)
+        try:
+            out = torch.empty(w.T, w.H, dtype=torch.bfloat16, device="cuda")
+            idx = torch.empty(w.T, w.K, dtype=torch.int32, device="cuda")
+            wt = torch.empty(w.T, w.K, dtype=torch.float32, device="cuda")
+            moe.forward(dims, d["x"], d["wr"], d["bias"], d["wu"], d["wd"], out, ws, topk_idx=idx, topk_w=wt)
+            moe.check_device_error()
+            runs.append((out, idx, wt))
+        finally:
+            moe.debug_set(9, -1)
+    for out, idx, wt in runs[1:]:
+        assert torch.equal(out, runs[0][0]) and torch.equal(idx, runs[0][1]) and torch.equal(wt, runs[0][2])
+
+
 @pytest.mark.parametrize("fill", [0x00, 0x7F, 0xFF], ids=["zeros", "0x7F", "0xFF"])
 def test_one_launch_ffn_ignores_stale_workspace(moe, fill):
     """The one-launch FFN's per-entry counters live in the workspace and are zeroed by the row
