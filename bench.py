@@ -670,11 +670,13 @@ def _fused_entry(wl, stages, touched, peaks, peak_kind, workload):
     if workload in TENSOR_BOUND:
         return dict(bound="tensor", achieved=tflops, peak=tc_peak, unit="TFLOP/s", frac=tflops / tc_peak,
                     peak_source=src, **common)
-    # the small-batch router's spare clusters (15 clusters of 8 fit a 148-SM B200; the batch
-    # takes ceil(T/8)) prefetch the up bank's first bytes into L2 before this launch: achieved
-    # counts every algorithmic byte, so frac can pass the copy peak by up to warm / algo
+    # the small-batch router (T <= 256: clusters of 4 tokens when they all fit at once, else of
+    # 8; 15 clusters of 8 CTAs fit a 148-SM B200) fills the clusters left over with L2 prefetches
+    # of the up bank's first bytes before this launch: achieved counts every algorithmic byte, so
+    # frac can pass the copy peak by up to warm / algo
     bank = wl.E * F * H // 2 if wl.nvfp4 else wl.E * F * H * es
-    warm = min(L2_WARM_BYTES, bank) if (T + 7) // 8 < 15 else 0
+    tb = 4 if (T + 3) // 4 <= 15 else 8
+    warm = min(L2_WARM_BYTES, bank) if T <= 256 and (T + tb - 1) // tb < 15 else 0
     return dict(bound="hbm", achieved=gbs, peak=hbm_peak, unit="GB/s", frac=gbs / hbm_peak,
                 peak_source=f"{peak_kind} hbm copy", l2_warm_bytes_before_launch=warm, **common)
 

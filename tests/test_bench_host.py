@@ -217,3 +217,5 @@ def test_hbm_roofline_names_the_routers_l2_prefetch():
     assert s["l2_warm_bytes_before_launch"] == 0                 # 72 clusters of 8 tokens: none spare
     t = bench.roofline_entry(W.WORKLOADS[0], st, 8, PEAKS, "measured", "tiny")
     assert t["l2_warm_bytes_before_launch"] == 8 * 128 * 256 * 2  # the whole bf16 bank
+    e = bench.roofline_entry(W.Workload("t60", 60, 2688, 128, 6, 1856, seed=1), st, 121, PEAKS, "measured", "decode")
+    assert e["l2_warm_bytes_before_launch"] == 0                 # 15 clusters of 4 tokens fill the device
