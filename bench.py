@@ -38,7 +38,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 WORKLOADS = {"tiny": 0, "decode": 1, "prefill": 2, "skewed": 3, "chain": 4, "decode_nvfp4": 5,
              "prefill_nvfp4": 6, "decode_shared": 7, "prefill_shared": 8, "decode_fp8_b128": 9,
              "prefill_fp8_b128": 10}
-L2_WARM_BYTES = 48 << 20   # the library's default L2 prefetch of the up bank at small batches
+L2_WARM_BYTES = 48 << 20   # the library's default L2 prefetch of a bf16 up bank at small batches
 TENSOR_BOUND = ("prefill", "chain", "prefill_nvfp4", "prefill_shared",
                 "prefill_fp8_b128")   # reported against the tensor peak
 
@@ -674,9 +674,9 @@ def _fused_entry(wl, stages, touched, peaks, peak_kind, workload):
     # 8; 15 clusters of 8 CTAs fit a 148-SM B200) fills the clusters left over with L2 prefetches
     # of the up bank's first bytes before this launch: achieved counts every algorithmic byte, so
     # frac can pass the copy peak by up to warm / algo
-    bank = wl.E * F * H // 2 if wl.nvfp4 else wl.E * F * H * es
     tb = 4 if (T + 3) // 4 <= 15 else 8
-    warm = min(L2_WARM_BYTES, bank) if T <= 256 and (T + tb - 1) // tb < 15 else 0
+    bf16 = not (fp8 or wl.nvfp4)   # the library prefetches only bf16 banks
+    warm = min(L2_WARM_BYTES, wl.E * F * H * 2) if bf16 and T <= 256 and (T + tb - 1) // tb < 15 else 0
     return dict(bound="hbm", achieved=gbs, peak=hbm_peak, unit="GB/s", frac=gbs / hbm_peak,
                 peak_source=f"{peak_kind} hbm copy", l2_warm_bytes_before_launch=warm, **common)
 

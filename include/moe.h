@@ -348,11 +348,14 @@ moe_status moe_set_stage_events(void* const* events, int32_t n);
  * view; what = 8: value 1 (the default) runs both expert projections in one
  * launch, for every expert format and with a shared expert (the down units of
  * a schedule entry start once that entry's up units have reported), 0 as two
- * launches; what = 9: bytes of the up bank's start (its first experts'
+ * launches; what = 9: bytes of a bf16 up bank's start (its first experts'
  * weights, which the FFN's first units read) that the small-batch router
  * prefetches into L2 from the clusters the device fits beside the batch's
  * (value 0: none; value < 0 restores the default of 48 MiB; clamped to the
- * bank's size); the prefetch changes no result.  Other `what`: MOE_EINVAL. */
+ * bank's size; other expert dtypes: none); the prefetch changes no result.
+ * The prefetching clusters come last in the router's grid: where kernels of
+ * other streams hold the SMs, they can wait for SMs and so delay the
+ * router's completion (value 0 avoids that).  Other `what`: MOE_EINVAL. */
 moe_status moe_debug_set(int32_t what, int64_t value);
 
 #ifdef __cplusplus

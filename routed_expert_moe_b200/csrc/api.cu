@@ -25,10 +25,12 @@ std::atomic<int> g_gemm_pair{0};
 std::atomic<int> g_fused_ffn{1};   // 1: both bf16/E4M3 projections in one launch (grouped_ffn.cu)
 std::atomic<int> g_pdl{1};
 std::atomic<int> g_shared_2d{0};   // 1: the shared down weight through its 2-D fallback map
-// Bytes of the up weight bank (its first experts: the FFN's first units) that the decode
-// router's spare clusters prefetch into L2 while routing.  On B200 at T=64 (bf16): the FFN
-// 347 -> 340 us and the router 20.3 -> 20.8 us at 48 MB; 64 MB and 96 MB slow the router's
-// own loads more (22.0, 22.6 us) than they save.
+// Bytes of the bf16 up weight bank (its first experts: the FFN's first units) that the decode
+// router's spare clusters prefetch into L2 while routing.  On B200 at T=64: the FFN 347 ->
+// 340 us and the router 20.3 -> 20.8 us at 48 MB; 64 MB and 96 MB slow the router's own loads
+// more (22.0, 22.6 us) than they save.  The NVFP4 and FP8_B128 FFNs, not bound by DRAM at
+// decode, gain nothing (NVFP4 layer 172.9 us either way; FP8_B128 219.0 -> 225.6 us), so
+// their banks are not prefetched.
 constexpr int64_t kL2WarmDefault = (int64_t)48 << 20;
 std::atomic<int64_t> g_l2_warm{kL2WarmDefault};
 void* g_stage_events[MOE_STAGE_EVENTS] = {};
@@ -538,10 +540,9 @@ moe_status moe_forward(const moe_dims* d, const void* x, const void* w_router, c
     Carve cr;
     RouteWs rw = carve_route(cr, sbase, d, rp);
     stage_mark(0, st);
-    // the up bank's leading bytes (expert 0 first, in every format's layout), bounded by its size
-    const int64_t up_bytes = (int64_t)d->E * d->F * d->H / (d->expert_dtype == MOE_NVFP4 ? 2 : 1) *
-                             (d->expert_dtype == MOE_BF16 ? 2 : 1);
-    const int64_t warm = std::min(g_l2_warm.load(), up_bytes);
+    // the bf16 up bank's leading bytes (expert 0 first), bounded by its size
+    const int64_t warm =
+        d->expert_dtype == MOE_BF16 ? std::min(g_l2_warm.load(), (int64_t)d->E * d->F * d->H * 2) : 0;
     cudaError_t e = launch_route(static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(w_router), bias, d->T,
                                  d->H, d->E, d->K, idx, w, rw.P, rw.xn2, rw.wn2, rp, ctx, st,
                                  g_stage_events_on.load() ? mark_stage1 : nullptr, w_up, warm);

@@ -205,14 +205,16 @@ def test_one_launch_ffn_with_a_shared_expert_counts_its_chunks():
 
 
 def test_hbm_roofline_names_the_routers_l2_prefetch():
-    """At decode the router's spare clusters prefetch the up bank's first 48 MiB into L2 before
-    the FFN launch (the whole bank when it is smaller); a batch whose router clusters fill the
-    device prefetches nothing."""
+    """At decode the router's spare clusters prefetch a bf16 up bank's first 48 MiB into L2
+    before the FFN launch (the whole bank when it is smaller); NVFP4 and FP8_B128 banks are not
+    prefetched, nor is anything for a batch whose router clusters fill the device."""
     st = {"expert_ffn": 0.35}
     r = bench.roofline_entry(W.WORKLOADS[1], st, 121, PEAKS, "measured", "decode")
     assert r["l2_warm_bytes_before_launch"] == 48 << 20
     f = bench.roofline_entry(W.WORKLOADS[5], st, 121, PEAKS, "measured", "decode_nvfp4")
-    assert f["l2_warm_bytes_before_launch"] == 48 << 20          # 128 x 1856 x 1344 bytes > 48 MiB
+    assert f["l2_warm_bytes_before_launch"] == 0                 # NVFP4 bank: not prefetched
+    b = bench.roofline_entry(W.WORKLOADS[9], st, 121, PEAKS, "measured", "decode_fp8_b128")
+    assert b["l2_warm_bytes_before_launch"] == 0
     s = bench.roofline_entry(W.WORKLOADS[3], st, 128, PEAKS, "measured", "skewed")
     assert s["l2_warm_bytes_before_launch"] == 0                 # 72 clusters of 8 tokens: none spare
     t = bench.roofline_entry(W.WORKLOADS[0], st, 8, PEAKS, "measured", "tiny")
