@@ -339,12 +339,12 @@ __device__ __forceinline__ void bf16x8(const uint4& v, float (&f)[8]) {
 template <int TB>
 __global__ void __cluster_dims__(RS_CLUSTER, 1, 1) __launch_bounds__(RS_THREADS)
     router_small_kernel(RouterSmallArgs a, DevCtx ctx) {
-    pdl_enter();
     // Clusters past the batch's groups only warm L2: they prefetch the bytes the expert FFN
     // reads first (its first experts' up weights) while the router and the permutation run,
     // when the memory system is otherwise idle.  They run on SMs the router leaves free, so
     // that no routing warp waits on the prefetches' issue; pieces of 32 KB, strided over their
-    // lanes.
+    // lanes.  They start before the wait on the preceding kernel (the weight banks are not
+    // written by it, and a prefetch changes no data), so the copies overlap its tail too.
     const int64_t n_groups = (a.T + TB - 1) / TB;
     if ((int64_t)(blockIdx.x / RS_CLUSTER) >= n_groups) {
         const int64_t first = n_groups * RS_CLUSTER * 32;
@@ -357,6 +357,7 @@ __global__ void __cluster_dims__(RS_CLUSTER, 1, 1) __launch_bounds__(RS_THREADS)
         }
         return;
     }
+    pdl_enter();
     namespace cg = cooperative_groups;
     extern __shared__ __align__(16) unsigned char rs_smem[];
     const int H = a.H, E = a.E;
